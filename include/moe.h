@@ -1,0 +1,181 @@
+/*
+ * moe.h - C ABI of libmoe.so: the MoE expert-parallel token shuffle on one B200 (sm_100a).
+ *
+ * The path has four stream-ordered calls, each a set of hand-written CUDA kernels:
+ *
+ *   moe_route       fused fp32 softmax + top-k router with a per-expert histogram
+ *   moe_dispatch    per-expert counts, offsets and stable positions, then the packed
+ *                   expert-major (= rank-major) send buffer, bf16 or FP8 e4m3 + fp32 block scales,
+ *                   with optional capacity dropping in token order
+ *   moe_expert_ffn  grouped SwiGLU expert FFN on the packed rows (tcgen05 / TMEM / TMA)
+ *   moe_combine     weighted gather back into token order, fp32 accumulate in fixed slot order
+ *
+ * Expert-parallel ranks are emulated as partitions of one HBM pool: rank r owns experts
+ * [r*E/R, (r+1)*E/R), so the expert-major send buffer is rank-major too and rank r's slice is
+ * rows rank_offsets[r] .. rank_offsets[r+1].
+ *
+ * Conventions for every call:
+ *  - Ownership: every pointer is caller-owned memory.  Unless stated otherwise it is DEVICE memory
+ *    of the current CUDA device.  The library allocates nothing and frees nothing; scratch memory is
+ *    the caller's workspace (sizes from the *_workspace_size queries).  This follows the
+ *    group/handle split with caller-registered allocation of the NCCL EP page ("NCCL EP架构解析",
+ *    sections 1 and 3.1).
+ *  - Layout: row-major, contiguous.  Pointers to arrays read or written with 16-byte vectors
+ *    (x, send, expert_out, y, weights) must be 16-byte aligned.
+ *  - Synchrony: every call only enqueues work on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and returns.  No call synchronises with the host; the number of kept rows stays on the
+ *    device (expert_offsets[E]).
+ *  - Errors: the return value reports host-side argument validation (checked before anything is
+ *    launched) and launch failures.  Errors found on the device (an expert id out of range, a
+ *    pipeline wait that ran out) are recorded in a status word at the start of the workspace and
+ *    reported by moe_sync_status.  Error names follow the NCCL EP page's error table (section 5.1:
+ *    INVALID_TOPK for an out-of-range routing index, CUDA_ERROR for a failed launch).
+ *  - Workspaces must be zero-filled once after allocation (cudaMemset); the calls keep them in a
+ *    reusable state afterwards.  Calls that share one workspace must not overlap on the GPU.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* == cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer, k > E, E % R != 0 ... */
+  MOE_ERR_INVALID_TOPK = 2, /* a routing index outside [0, E) (found on the device)               */
+  MOE_ERR_UNSUPPORTED = 3,  /* valid but not implemented here (e.g. H % 64 != 0)                  */
+  MOE_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed                               */
+  MOE_ERR_WORKSPACE = 5,    /* workspace too small or not 256-byte aligned                        */
+  MOE_ERR_TIMEOUT = 6       /* a bounded device-side wait ran out; the kernel stopped early       */
+} moe_status_t;
+
+typedef enum {
+  MOE_PAYLOAD_BF16 = 0,         /* send rows are the token's bf16 bytes                             */
+  MOE_PAYLOAD_FP8_E4M3_B128 = 1 /* send rows are e4m3 codes + one fp32 scale per 128 elements       */
+} moe_payload_t;
+
+/* Version of this interface (incremented on any incompatible change). */
+int moe_abi_version(void);
+
+/* Static, NUL-terminated description of a status code. */
+const char* moe_status_string(moe_status_t status);
+
+/*
+ * Per-expert capacity C = ceil(cf * T * k / E), computed in double; cf <= 0 returns 0 (no limit).
+ * Mean expert load is T*k/E ("大模型MoE稀疏激活原理与硬件适配实战", section 2.3: (B*S*K)/E with
+ * the example 32*2048*2/128 = 1024).  Host function; returns -1 for T < 0, k < 1 or E < 1.
+ */
+int moe_capacity(double cf, int T, int k, int E);
+
+/*
+ * Router: per token, the k largest fp32 logits (ties -> lower expert id; NaN ranks below -inf),
+ * in descending order, and their routing weights; the selection and the weights are fp32 ("大模型
+ * MoE稀疏激活原理与硬件适配实战", section 3.2, fine ranking; section 5.3, scenario 3: router in FP32;
+ * section 4.1: one token's experts are distinct).
+ *   logits        fp32 [T, E]       router logits (any bias already added)
+ *   renormalize   1: weights = softmax over the k selected logits (they sum to 1)
+ *                 0: weights = the selected entries of the softmax over all E logits
+ *   topk_idx      int32 [T, k]      out: expert ids, best first
+ *   topk_w        fp32  [T, k]      out: routing weights, same order
+ *   expert_routed int32 [E] or NULL out: number of tokens routed to each expert (overwritten)
+ * Limits: 1 <= k <= E <= 1024, k <= 32, T >= 0 (T == 0 launches nothing but clears expert_routed).
+ * Non-finite logits: the weights are the softmax's limits (NaN counts as -inf; +inf entries share
+ * the mass; an all -inf denominator shares it equally).
+ */
+moe_status_t moe_route(const float* logits, int T, int E, int k, int renormalize,
+                       int32_t* topk_idx, float* topk_w, int32_t* expert_routed,
+                       moe_stream_t stream);
+
+/* Bytes of scratch moe_dispatch needs for T tokens, E experts, k slots per token. */
+size_t moe_dispatch_workspace_size(int T, int E, int k);
+
+/*
+ * Dispatch: pack every kept (token, slot) into one contiguous expert-major send buffer (the
+ * ThunderEP page, section 2.1, redundancy 1: all tokens bound for one destination in one buffer;
+ * NCCL EP page, section 2.2: packed [sum T x H] high-throughput layout; section 2.1: expert-major
+ * layout, FP8 payload with a scale tensor).
+ *
+ * Within an expert, rows are in ascending token order.  With capacity C > 0, a slot whose position
+ * among its expert's slots (in token order) is >= C is dropped: slot_row = -1, no row is written.
+ *   x              bf16 [T, H]              token activations
+ *   topk_idx       int32 [T, k]             expert ids (each in [0, E))
+ *   capacity       0 = keep every slot, else C (see moe_capacity)
+ *   payload        MOE_PAYLOAD_BF16 or MOE_PAYLOAD_FP8_E4M3_B128 (needs H % 128 == 0)
+ *   send           [T*k, H] bf16 or e4m3    out: rows 0 .. expert_offsets[E]-1 are written
+ *   send_scales    fp32 [T*k, H/128]        out (FP8 only, else may be NULL): per-block scales,
+ *                                           scale = amax/448 (1 if amax == 0), code =
+ *                                           e4m3_rn_satfinite(x / scale), fp32 IEEE division
+ *   expert_counts  int32 [E]                out: kept rows per expert
+ *   expert_offsets int32 [E+1]              out: exclusive scan of expert_counts
+ *   rank_offsets   int32 [R+1]              out: rank_offsets[r] = expert_offsets[r*E/R]
+ *   slot_row       int32 [T, k]             out: packed row of each slot, -1 if dropped
+ *   row_token      int32 [T*k]              out: token of each packed row (first S entries)
+ *   ws, ws_bytes   device scratch >= moe_dispatch_workspace_size(T, E, k), 256-byte aligned,
+ *                  zero-filled once after allocation
+ * Limits: T*k < 2^31, 1 <= k <= E <= 1024, R >= 1, E % R == 0, H % 8 == 0, H >= 8.
+ * An expert id outside [0, E) is not written anywhere: its slot gets slot_row = -1 and the status
+ * word records MOE_ERR_INVALID_TOPK (reported by moe_sync_status).
+ */
+moe_status_t moe_dispatch(const void* x, int T, int H, const int32_t* topk_idx, int k, int E,
+                          int R, int capacity, moe_payload_t payload, void* send,
+                          float* send_scales, int32_t* expert_counts, int32_t* expert_offsets,
+                          int32_t* rank_offsets, int32_t* slot_row, int32_t* row_token, void* ws,
+                          size_t ws_bytes, moe_stream_t stream);
+
+/* Bytes of scratch moe_expert_ffn needs (status word, the bf16 intermediate h [max_rows, F] and,
+ * for the FP8 payload, the dequantised bf16 input rows [max_rows, H]). */
+size_t moe_ffn_workspace_size(int max_rows, int E, int H, int F, moe_payload_t payload);
+
+/*
+ * Grouped SwiGLU expert FFN on the packed rows ("细粒度专家并行方案对比：MegaMoE与传统方案",
+ * section 核心差异分析 1: two linear layers and SwiGLU per expert; "DWDP: 在NVL72上的高性能分布式权重
+ * 数据并行", run_moe: fused w3_w1 first projection with SwiGLU, then w2).  For expert e and every
+ * packed row x in [expert_offsets[e], expert_offsets[e+1]):
+ *     h = bf16( silu(x . W_gate[e]^T) * (x . W_up[e]^T) ),  silu(g) = g * sigmoid(g)
+ *     expert_out = bf16( h . W_down[e]^T )
+ * with bf16 operands on the tensor cores and fp32 accumulation.  For the FP8 payload the input
+ * row is first dequantised: x = bf16(fp32(q) * scale).
+ *   send           [max_rows, H] bf16 or e4m3 (rows past expert_offsets[E] are ignored)
+ *   send_scales    fp32 [max_rows, H/128] (FP8 only, else NULL)
+ *   expert_offsets int32 [E+1] device array (read on the device; no host sync)
+ *   w_gate, w_up   bf16 [E, F, H], one contiguous block per expert
+ *   w_down         bf16 [E, H, F]
+ *   expert_out     bf16 [max_rows, H]       out: rows 0 .. expert_offsets[E]-1
+ *   ws, ws_bytes   device scratch >= moe_ffn_workspace_size(...), 256-byte aligned, zero-filled once
+ * Limits: H % 64 == 0, F % 64 == 0 (else MOE_ERR_UNSUPPORTED), E <= 1024,
+ * expert_offsets[E] <= max_rows (rows beyond max_rows are not computed).
+ */
+moe_status_t moe_expert_ffn(const void* send, const float* send_scales, moe_payload_t payload,
+                            const int32_t* expert_offsets, int max_rows, int E, int H, int F,
+                            const void* w_gate, const void* w_up, const void* w_down,
+                            void* expert_out, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Combine: y[t] = bf16( sum_{j=0..k-1, slot_row[t,j] >= 0} topk_w[t,j] * expert_out[slot_row[t,j]] )
+ * accumulated in fp32 in slot order j = 0, 1, ... with each product and sum rounded to fp32
+ * separately (the NCCL EP page, section 2.1: the combine loops over the top-k slots and adds each
+ * expert output times the token's routing weight).  A token whose slots were all dropped gives 0.
+ *   expert_out bf16 [max_rows, H]; slot_row int32 [T, k]; topk_w fp32 [T, k]; y bf16 [T, H] (out)
+ * Rows outside [0, max_rows) are treated as dropped.  Limits: H % 8 == 0.
+ */
+moe_status_t moe_combine(const void* expert_out, int max_rows, const int32_t* slot_row,
+                         const float* topk_w, int T, int k, int H, void* y, moe_stream_t stream);
+
+/*
+ * Synchronise `stream`, read the device status word at the start of a dispatch or FFN workspace,
+ * clear it, and report it: MOE_OK, MOE_ERR_INVALID_TOPK or MOE_ERR_TIMEOUT (MOE_ERR_CUDA if the
+ * stream itself failed).
+ */
+moe_status_t moe_sync_status(void* ws, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

@@ -1,0 +1,284 @@
+"""Plain CPU oracle of the MoE expert-parallel token shuffle: route -> dispatch -> SwiGLU FFN -> combine.
+
+TEST INFRASTRUCTURE ONLY.  Nothing under ``oracle/`` is part of the product path: only ``tests/``,
+``__graft_entry__.smoke()`` and the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py``
+may import it.  It shares no code with the CUDA library and never takes inputs from it.
+
+Sources (web pages on expert-parallel MoE communication):
+
+* "大模型MoE稀疏激活原理与硬件适配实战" (MoE sparse activation and hardware fit), section 3.2
+  (fine ranking: sort the router logits, take the top experts), section 4.1 (the heat map's diagonal
+  is zero: one token's experts are distinct), section 5.3 scenario 3 (the router runs in FP32),
+  section 2.3 (mean expert load (B*S*K)/E, per-expert capacity).
+* The ThunderEP page, section 2.1, redundancy 1 (pack every token bound for one destination into
+  one contiguous buffer on the sender) and section 2.2 (each rank keeps only its own slice of the
+  routing table).
+* "NCCL EP架构解析" (NCCL EP architecture), section 2.1 (expert-major layout for the expert compute;
+  FP8 payload with a scale tensor; the combine weights expert outputs by the token's routing
+  weights, looping over the top-k slots), section 2.2 (high-throughput layout: one packed
+  [sum T x H] buffer), section 5.1 (INVALID_TOPK when a routing index is out of range).
+* "细粒度专家并行方案对比：MegaMoE与传统方案" (MegaMoE vs non-fused expert parallelism), section
+  "核心差异分析 1" (two linear layers with a SwiGLU activation per expert), and
+  "DWDP: 在NVL72上的高性能分布式权重数据并行", the ``NvFp4WeightView`` / ``run_moe`` passage
+  (fused ``w3_w1`` first projection with SwiGLU, ``w2`` second projection, finalize = weighted
+  scatter back to token order).
+
+Readings where the pages are silent (each is listed with its reason in the design notes):
+selection is on fp32 logits, ties to the lower expert id, slots ordered by descending logit; NaN
+ranks below -inf; weights are the softmax over the selected k (``renormalize``) or the full-E
+softmax; h = silu(x W_gate^T) * (x W_up^T) rounded to bf16, y = h W_down^T rounded to bf16; rows of
+one expert are in ascending token order and overflow past the capacity is dropped in token order;
+capacity C = ceil(cf * T * k / E); FP8 scale = amax / 448 per 128-element block (1 when amax = 0),
+q = e4m3 round-to-nearest-even, saturating, of x / scale in fp32.
+
+Precision: fp64 for the router weights and the FFN, as the pages fix neither.  The FP8 scale and
+quotient are taken in fp32 (IEEE division), because they decide the quantised codes and the GPU
+takes that decision in fp32.  The combine accumulates in fp32 in the fixed slot order, because the
+pages' combine loop is written in float.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+from .numerics import bf16_bits, bf16_from_bits, bf16_round, e4m3_decode, e4m3_encode_satfinite
+
+__all__ = ["capacity", "route", "dispatch_plan", "dispatch_payload", "expert_ffn", "combine",
+           "pipeline", "QBLOCK"]
+
+QBLOCK = 128   # elements per FP8 scale block
+E4M3_MAX_F32 = np.float32(448.0)
+
+
+def capacity(cf: float, T: int, k: int, E: int) -> int:
+    """Per-expert capacity ceil(cf * T * k / E); 0 means no limit (cf == 0).
+
+    Mean load per expert is T*k/E (MoE sparse activation page, section 2.3: (B*S*K)/E, printed
+    example 32*2048*2/128 = 1024)."""
+    if cf <= 0:
+        return 0
+    return int(math.ceil(cf * (T * k) / E))
+
+
+def _as_f32(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+
+
+def route(logits, k: int, renormalize: bool = True):
+    """Top-k selection and routing weights per token.
+
+    For each token the experts are sorted by (logit descending, expert id ascending), NaN after
+    every number (including -inf); the first k are the token's experts, in that order.  Weights are
+    the softmax of the selected logits (``renormalize``) or their full softmax over all E experts,
+    computed in fp64 and stored as fp32.  Limits of the softmax define the non-finite cases: NaN
+    counts as -inf; if any +inf is present the +inf entries share the mass equally; if every entry
+    of the denominator is -inf the mass is shared equally among them.
+
+    Returns ``(topk_idx int32 [T,k], topk_w fp32 [T,k], expert_routed int32 [E])``.
+    """
+    l = _as_f32(logits)
+    T, E = l.shape
+    if not 1 <= k <= E:
+        raise ValueError("need 1 <= k <= E")
+    nan = np.isnan(l)
+    neg = np.where(nan, 0.0, -l.astype(np.float64))
+    ids = np.broadcast_to(np.arange(E), (T, E))
+    order = np.lexsort((ids, neg, nan), axis=-1)        # primary: NaN last; then logit desc; then id
+    idx = order[:, :k].astype(np.int32)
+
+    lv = np.where(nan, -np.inf, l.astype(np.float64))    # NaN counts as -inf in the weights
+    sel = np.take_along_axis(lv, idx.astype(np.int64), axis=1)
+    den_src = sel if renormalize else lv
+    w = np.empty((T, k), dtype=np.float64)
+    for t in range(T):
+        s, d = sel[t], den_src[t]
+        n_pinf = np.count_nonzero(d == np.inf)
+        if n_pinf:
+            w[t] = np.where(s == np.inf, 1.0 / n_pinf, 0.0)
+        elif np.all(d == -np.inf):
+            w[t] = 1.0 / d.size
+        else:
+            m = np.max(d)
+            w[t] = np.exp(s - m) / np.sum(np.exp(d - m))
+    routed = np.bincount(idx.ravel(), minlength=E).astype(np.int32)
+    return idx, w.astype(np.float32), routed
+
+
+def dispatch_plan(topk_idx, E: int, R: int, cap: int = 0):
+    """Positions of every routed slot in the packed expert-major send buffer.
+
+    Walking the slots in token order, a slot's position inside its expert is the number of earlier
+    slots routed to the same expert.  A slot is kept when there is no capacity (``cap == 0``) or its
+    position is below ``cap``; kept slots of expert e occupy rows
+    ``expert_offsets[e] .. expert_offsets[e+1]`` in ascending token order, experts in ascending id.
+    Rank r owns experts [r*E/R, (r+1)*E/R), so the buffer is also rank-major and
+    ``rank_offsets[r] = expert_offsets[r*E/R]``.
+
+    Returns a dict with int32 arrays ``expert_routed`` [E], ``expert_counts`` (kept) [E],
+    ``expert_offsets`` [E+1], ``rank_offsets`` [R+1], ``slot_row`` [T,k] (-1 = dropped),
+    ``row_token`` [S] and the kept total ``S``.
+    """
+    idx = np.asarray(topk_idx, dtype=np.int64)
+    T, k = idx.shape
+    if E % R:
+        raise ValueError("E must be a multiple of R")
+    if idx.size and (idx.min() < 0 or idx.max() >= E):
+        raise ValueError("routing index out of range")
+    pos = np.empty((T, k), dtype=np.int64)
+    running = [0] * E
+    for t in range(T):
+        for j in range(k):
+            e = int(idx[t, j])
+            pos[t, j] = running[e]
+            running[e] += 1
+    routed = np.array(running, dtype=np.int64)
+    kept = np.minimum(routed, cap) if cap > 0 else routed
+    offsets = np.zeros(E + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(kept)
+    S = int(offsets[E])
+    slot_row = np.full((T, k), -1, dtype=np.int64)
+    row_token = np.empty(S, dtype=np.int64)
+    for t in range(T):
+        for j in range(k):
+            e = int(idx[t, j])
+            if cap == 0 or pos[t, j] < cap:
+                row = int(offsets[e] + pos[t, j])
+                slot_row[t, j] = row
+                row_token[row] = t
+    per_rank = E // R
+    rank_offsets = offsets[::per_rank][: R + 1]
+    return {
+        "expert_routed": routed.astype(np.int32),
+        "expert_counts": kept.astype(np.int32),
+        "expert_offsets": offsets.astype(np.int32),
+        "rank_offsets": rank_offsets.astype(np.int32),
+        "slot_row": slot_row.astype(np.int32),
+        "row_token": row_token.astype(np.int32),
+        "S": S,
+    }
+
+
+def quantize_row_fp8(x_row_f32: np.ndarray):
+    """One token row -> (e4m3 codes [H], fp32 scales [H/128]).
+
+    Per 128-element block: amax = max |x| (exact in fp32); scale = amax / 448 in fp32 (1 when
+    amax = 0); code = e4m3 round-to-nearest-even, saturating, of the fp32 quotient x / scale."""
+    x = x_row_f32.astype(np.float32).reshape(-1, QBLOCK)
+    amax = np.max(np.abs(x), axis=1)
+    scale = np.where(amax == 0, np.float32(1.0), amax / np.float32(E4M3_MAX_F32)).astype(np.float32)
+    q = (x / scale[:, None]).astype(np.float32)            # fp32 IEEE division
+    return e4m3_encode_satfinite(q).reshape(-1), scale
+
+
+
+def dispatch_payload(x_bf16_bits, plan, fp8: bool = False):
+    """Packed send buffer: ``send[row] = payload(x[row_token[row]])`` for every kept row.
+
+    bf16 payload: the token's bytes.  FP8 payload: per-block e4m3 codes plus one fp32 scale per
+    128-element block.  Returns ``(send, send_scales or None)`` with S rows."""
+    xb = np.asarray(x_bf16_bits, dtype=np.uint16)
+    T, H = xb.shape
+    rt = plan["row_token"]
+    S = plan["S"]
+    if not fp8:
+        return xb[rt].copy(), None
+    if H % QBLOCK:
+        raise ValueError("FP8 payload needs H % 128 == 0")
+    xf = bf16_from_bits(xb)
+    codes = np.empty((T, H), dtype=np.uint8)
+    scales = np.empty((T, H // QBLOCK), dtype=np.float32)
+    for t in range(T):
+        codes[t], scales[t] = quantize_row_fp8(xf[t])
+    return codes[rt].copy(), scales[rt].copy()
+
+
+def dequantize_fp8_rows(codes, scales) -> np.ndarray:
+    """bf16 values (as float64) of the FFN input rows of an FP8 payload: bf16(fp32(q) * scale)."""
+    q = e4m3_decode(codes).astype(np.float32)
+    s = np.repeat(np.asarray(scales, dtype=np.float32), QBLOCK, axis=1)
+    prod = (q * s).astype(np.float32)                       # one fp32 product per element
+    return bf16_round(prod)
+
+
+def expert_ffn(send_rows_f64: np.ndarray, expert_offsets, w_gate_bits, w_up_bits, w_down_bits,
+               rows=None):
+    """Grouped SwiGLU FFN on the packed rows, expert by expert.
+
+    For expert e and each of its rows x: g = x W_gate[e]^T, u = x W_up[e]^T (fp64 accumulate),
+    h = bf16(g * sigmoid(g) * u), y = bf16(h W_down[e]^T) (fp64 accumulate).
+
+    ``send_rows_f64`` holds the FFN input values (bf16 values as float64) of every packed row.
+    ``rows`` optionally restricts the computation to those packed row indices (the other output
+    rows are left as NaN).  Returns (h, y) as bf16 bit patterns; h has F columns, y has H.
+    """
+    off = np.asarray(expert_offsets, dtype=np.int64)
+    E = off.size - 1
+    S = int(off[E])
+    H = w_gate_bits.shape[2]
+    F = w_gate_bits.shape[1]
+    want = np.arange(S) if rows is None else np.asarray(rows, dtype=np.int64)
+    h_out = np.full((S, F), 0x7FC0, dtype=np.uint16)
+    y_out = np.full((S, H), 0x7FC0, dtype=np.uint16)
+    for e in range(E):
+        lo, hi = off[e], off[e + 1]
+        r = want[(want >= lo) & (want < hi)]
+        if r.size == 0:
+            continue
+        x = np.asarray(send_rows_f64[r], dtype=np.float64)
+        wg = bf16_from_bits(w_gate_bits[e]).astype(np.float64)
+        wu = bf16_from_bits(w_up_bits[e]).astype(np.float64)
+        g = x @ wg.T
+        u = x @ wu.T
+        del wg, wu
+        h = bf16_round(g / (1.0 + np.exp(-g)) * u)
+        wd = bf16_from_bits(w_down_bits[e]).astype(np.float64)
+        y = h @ wd.T
+        h_out[r] = bf16_bits(h)
+        y_out[r] = bf16_bits(y)
+    return h_out, y_out
+
+
+def combine(expert_out_bits, slot_row, topk_w, T: int, H: int):
+    """y[t] = bf16( sum over j in 0..k-1 with slot_row[t,j] >= 0 of w[t,j] * expert_out[row] ).
+
+    The sum is taken in fp32 in slot order j = 0, 1, ..., starting from 0, with each product and
+    each addition rounded to fp32 separately.  A token whose slots were all dropped gives 0.
+    Returns bf16 bit patterns [T,H]."""
+    eo = bf16_from_bits(np.asarray(expert_out_bits, dtype=np.uint16))
+    sr = np.asarray(slot_row, dtype=np.int64)
+    w = _as_f32(topk_w)
+    k = sr.shape[1]
+    acc = np.zeros((T, H), dtype=np.float32)
+    for j in range(k):
+        rows = sr[:, j]
+        valid = rows >= 0
+        prod = (w[valid, j][:, None] * eo[rows[valid]]).astype(np.float32)
+        acc[valid] = (acc[valid] + prod).astype(np.float32)
+    return bf16_bits(acc)
+
+
+def ffn_inputs(send, send_scales, fp8: bool) -> np.ndarray:
+    """FFN input values (float64) of the packed rows: the bf16 rows, or the dequantised FP8 rows."""
+    if fp8:
+        return dequantize_fp8_rows(send, send_scales)
+    return bf16_from_bits(send).astype(np.float64)
+
+
+def pipeline(logits, x_bf16_bits, w_gate_bits, w_up_bits, w_down_bits, k: int, R: int,
+             cf: float = 0.0, fp8: bool = False, renormalize: bool = True, ffn_rows=None):
+    """The whole path on the CPU.  Returns every intermediate as a dict."""
+    T, E = np.asarray(logits).shape
+    H = np.asarray(x_bf16_bits).shape[1]
+    idx, w, routed = route(logits, k, renormalize)
+    cap = capacity(cf, T, k, E)
+    plan = dispatch_plan(idx, E, R, cap)
+    send, scales = dispatch_payload(x_bf16_bits, plan, fp8)
+    xin = ffn_inputs(send, scales, fp8)
+    h, y_e = expert_ffn(xin, plan["expert_offsets"], w_gate_bits, w_up_bits, w_down_bits, ffn_rows)
+    out = dict(plan)
+    out.update(topk_idx=idx, topk_w=w, routed=routed, cap=cap, send=send, send_scales=scales,
+               h=h, expert_out=y_e)
+    if ffn_rows is None:
+        out["y"] = combine(y_e, plan["slot_row"], w, T, H)
+    return out
