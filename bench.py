@@ -1,0 +1,384 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE token shuffle (route -> dispatch -> grouped SwiGLU FFN -> combine) on B200.
+
+One step = one pass of the whole path over one batch of synthetic tokens (all four C-ABI calls on
+one stream), inputs and weights already resident in HBM.  Prints one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode] [--impl ours|reference]
+
+Multi-GPU (torchrun): every rank runs an independent replica of the workload (its own batch of T
+tokens, emulated expert-parallel ranks inside each GPU), no data-path collective; the step time is
+the max over ranks and ``value`` counts the tokens of all ranks ("weak" scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import moe_inputs as mi  # noqa: E402
+
+METRIC = "dispatch+FFN+combine tokens/s and shuffle HBM GB/s (% of roofline) on 1 B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = mi.l2_flush_bytes()
+
+
+# ---------------------------------------------------------------------------------------------
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while the benchmark runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        sm, mx, reasons, power = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                c = [x.strip() for x in line.split(",")]
+                if len(c) < 9:
+                    continue
+                try:
+                    sm.append(float(c[1]))
+                    mx = float(c[2])
+                    power.append(float(c[3]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, c[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+# ---------------------------------------------------------------------------------------------
+def algorithmic(w, S: int, active_experts: int):
+    """Algorithmic bytes / flops per step of each stage (what the stage must move or compute)."""
+    fp8 = w.payload == "fp8"
+    b = 1 if fp8 else 2
+    route = w.T * w.E * 4 + w.T * w.k * 8 + w.E * 4
+    dispatch = (w.T * w.H * 2 + S * w.H * b + (S * (w.H // 128) * 4 if fp8 else 0)
+                + w.T * w.k * 4 * 3 + S * 4 + (w.E * 2 + 1 + w.R + 1) * 4)
+    weights = active_experts * 3 * w.H * w.F * 2
+    acts = S * w.H * 2 + 2 * S * w.F * 2 + S * w.H * 2   # A read, h write+read, out write
+    if fp8:
+        acts += S * w.H + S * (w.H // 128) * 4 + S * w.H * 2  # dequant: read codes+scales, write
+    ffn_bytes = weights + acts
+    ffn_flops = 6 * S * w.H * w.F
+    combine = S * w.H * 2 + w.T * w.k * 8 + w.T * w.H * 2
+    return dict(route=route, dispatch=dispatch, ffn_bytes=ffn_bytes, ffn_weight_bytes=weights,
+                ffn_flops=ffn_flops, combine=combine)
+
+
+def cpu_baseline_run(w, d_cpu, budget_s: float = 12.0, n_tokens: int | None = None):
+    """Oracle pipeline on a bounded token sample (the first n tokens).  Returns (tokens/s, info)."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    from oracle import moe
+
+    def bits(t):
+        return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    wg, wu, wd = bits(d_cpu["w_gate"]), bits(d_cpu["w_up"]), bits(d_cpu["w_down"])
+    logits, x = d_cpu["logits"].numpy(), bits(d_cpu["x"])
+    cap = moe.capacity(w.capacity_factor, w.T, w.k, w.E)
+
+    def run(n):
+        idx, wt, _ = moe.route(logits[:n], w.k)
+        plan = moe.dispatch_plan(idx, w.E, w.R, cap)
+        send, sc = moe.dispatch_payload(x[:n], plan, w.payload == "fp8")
+        xin = moe.ffn_inputs(send, sc, w.payload == "fp8")
+        _, y_e = moe.expert_ffn(xin, plan["expert_offsets"], wg, wu, wd)
+        moe.combine(y_e, plan["slot_row"], wt, n, w.H)
+
+    if n_tokens is None:
+        n, spent, t = 1, 0.0, 0.0
+        while True:
+            t0 = time.perf_counter()
+            run(n)
+            t = time.perf_counter() - t0
+            spent += t
+            if t > budget_s / 4 or n >= w.T or spent > budget_s:
+                break
+            n = min(w.T, n * 2)
+    else:
+        n = min(n_tokens, w.T)
+        t0 = time.perf_counter()
+        run(n)
+        t = time.perf_counter() - t0
+    threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    return n / t, {"cores": threads, "tokens": n, "seconds": t}
+
+
+# ---------------------------------------------------------------------------------------------
+def run_reference(args, w, rank: int):
+    """The oracle, as it stands, timed on the host cores on bounded token samples of the workload."""
+    if rank != 0:
+        return
+    d = mi.make_inputs(w, seed=0, device="cpu")
+    budget = 150.0
+    # size each step so that warm-up + timed steps stay within a few minutes
+    _, info = cpu_baseline_run(w, d, n_tokens=1)
+    per_token = max(info["seconds"], 1e-3)
+    n = max(1, min(w.T, int(budget / max(args.steps + args.warmup, 1) / per_token)))
+    for _ in range(args.warmup):
+        cpu_baseline_run(w, d, n_tokens=n)
+    total, toks = 0.0, 0
+    for _ in range(args.steps):
+        _, inf = cpu_baseline_run(w, d, n_tokens=n)
+        total += inf["seconds"]
+        toks += inf["tokens"]
+    value = toks / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, args),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": info["cores"],
+                         "kind": "oracle",
+                         "sample": f"first {n} tokens of the workload per step (route, dispatch, "
+                                   f"SwiGLU FFN on their rows, combine)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w, args):
+    import math
+    cap = math.ceil(w.capacity_factor * w.T * w.k / w.E) if w.capacity_factor else 0
+    return {"workload": w.name, "T": w.T, "H": w.H, "E": w.E, "k": w.k, "R": w.R, "F": w.F,
+            "payload": w.payload, "capacity": cap, "bias": w.bias,
+            "parallelism": f"replicas x{args.gpus} (ranks emulated inside each GPU)",
+            "l2": "flushed (256 MB write) before every timed step"}
+
+
+# ---------------------------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="decode", choices=sorted(mi.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = mi.get(args.workload)
+
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return
+
+    import datetime
+    import torch.distributed as dist
+    from combine_moe_route_10_b200 import MoeShuffle
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    d = mi.make_inputs(w, seed=rank, device=str(dev))
+    cap_rows = (__import__("math").ceil(w.capacity_factor * w.T * w.k / w.E)
+                if w.capacity_factor else 0)
+    m = MoeShuffle(w.T, w.H, w.E, w.k, w.R, w.F, payload=w.payload, capacity=cap_rows, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        m.route(d["logits"])
+        m.dispatch(d["x"])
+        m.expert_ffn(d["w_gate"], d["w_up"], d["w_down"])
+        m.combine()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    st = m.status()
+    if st != 0:
+        raise SystemExit(f"device status {st} after warm-up")
+    S = int(m.expert_offsets[w.E].item())
+    active = int((m.expert_counts > 0).sum().item())
+
+    n_ev = 5
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(1)
+        e = evs[i]
+        e[0].record(stream)
+        m.route(d["logits"])
+        e[1].record(stream)
+        m.dispatch(d["x"])
+        e[2].record(stream)
+        m.expert_ffn(d["w_gate"], d["w_up"], d["w_down"])
+        e[3].record(stream)
+        m.combine()
+        e[4].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    stage_ms = [[e[j].elapsed_time(e[j + 1]) for j in range(n_ev - 1)] for e in evs]
+    total_ms = sum(sum(s) for s in stage_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    mean_stage = [sum(s[j] for s in stage_ms) / args.steps for j in range(n_ev - 1)]
+
+    # end to end through the public API: pinned host inputs in, result back to pinned host memory
+    logits_h = d["logits"].cpu().pin_memory()
+    x_h = d["x"].cpu().pin_memory()
+    y_h = torch.empty(m.y.shape, dtype=m.y.dtype).pin_memory()
+    logits_d, x_d = torch.empty_like(d["logits"]), torch.empty_like(d["x"])
+    e2e_steps = max(3, min(args.steps, 50))
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(e2e_steps)]
+    for i in range(e2e_steps + 2):
+        flush.fill_(1)
+        if i >= 2:
+            e2e_ev[i - 2][0].record(stream)
+        logits_d.copy_(logits_h, non_blocking=True)
+        x_d.copy_(x_h, non_blocking=True)
+        m.forward(logits_d, x_d, d["w_gate"], d["w_up"], d["w_down"])
+        y_h.copy_(m.y, non_blocking=True)
+        if i >= 2:
+            e2e_ev[i - 2][1].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    st = m.status()
+    if st != 0:
+        raise SystemExit(f"device status {st} after timing")
+
+    pk, pk_src = peaks()
+    alg = algorithmic(w, S, active)
+    ms = total_ms / args.steps
+    value = world * w.T * args.steps / (total_ms * 1e-3)
+    t_route, t_disp, t_ffn, t_comb = mean_stage
+    hbm = pk["hbm_gbs"]
+    ffn_t_hbm = alg["ffn_bytes"] / (hbm * 1e9)
+    ffn_t_tc = alg["ffn_flops"] / (pk["bf16_tflops_sustained"] * 1e12)
+    if ffn_t_hbm >= ffn_t_tc:
+        ach = alg["ffn_bytes"] / (t_ffn * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm}
+    else:
+        ach = alg["ffn_flops"] / (t_ffn * 1e-3) / 1e12
+        p = pk["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "achieved": ach, "peak": p, "unit": "TFLOP/s", "frac": ach / p}
+    roof.update({
+        "kernel": "grouped_gemm_kernel x2 (GEMM-1 gate/up + SwiGLU, GEMM-2 down) = moe_expert_ffn",
+        "traffic": None, "peak_source": pk_src,
+        "algorithmic_bytes": alg["ffn_bytes"], "algorithmic_flops": alg["ffn_flops"],
+        "frac_of_max_time_bound": max(ffn_t_hbm, ffn_t_tc) / (t_ffn * 1e-3)})
+
+    def gbs(b, t):
+        return b / (t * 1e-3) / 1e9
+
+    shuffle = {
+        "route": {"ms": t_route, "GB/s": gbs(alg["route"], t_route)},
+        "dispatch": {"ms": t_disp, "GB/s": gbs(alg["dispatch"], t_disp),
+                     "frac": gbs(alg["dispatch"], t_disp) / hbm},
+        "ffn": {"ms": t_ffn, "TFLOP/s": alg["ffn_flops"] / (t_ffn * 1e-3) / 1e12,
+                "GB/s": gbs(alg["ffn_bytes"], t_ffn)},
+        "combine": {"ms": t_comb, "GB/s": gbs(alg["combine"], t_comb),
+                    "frac": gbs(alg["combine"], t_comb) / hbm},
+    }
+    launches_per_step = 1 + 3 + (3 if w.payload == "fp8" else 2) + 1
+    h2d = d["logits"].numel() * 4 + d["x"].numel() * 2
+    d2h = m.y.numel() * 2
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8+bf16" if w.payload == "fp8" else "bf16",
+        "data": "synthetic (seeded; random-init expert weights N(0,0.02))",
+        "config": config_of(w, args),
+        "roofline": roof,
+        "stages": shuffle,
+        "kept_rows": S, "active_experts": active,
+        "e2e": {"value": world * w.T * e2e_steps / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        d_cpu = {k: v.cpu() for k, v in d.items()}
+        v, info = cpu_baseline_run(w, d_cpu)
+        line["cpu_baseline"] = {
+            "value": v, "unit": "tokens/s", "cores": info["cores"], "kind": "oracle",
+            "sample": f"first {info['tokens']} tokens of the workload (route, dispatch, SwiGLU FFN "
+                      f"on their rows, combine), {info['seconds']:.1f} s"}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,142 @@
+"""ctypes binding of libmoe.so (include/moe.h).  Argument marshalling only: every step of the path
+runs in the library's CUDA kernels; there is no CPU fallback and loading fails loudly when the
+library is missing."""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_INVALID_TOPK = 2
+MOE_ERR_UNSUPPORTED = 3
+MOE_ERR_CUDA = 4
+MOE_ERR_WORKSPACE = 5
+MOE_ERR_TIMEOUT = 6
+MOE_PAYLOAD_BF16 = 0
+MOE_PAYLOAD_FP8_E4M3_B128 = 1
+
+EXPORTS = ["moe_abi_version", "moe_status_string", "moe_capacity", "moe_route",
+           "moe_dispatch_workspace_size", "moe_dispatch", "moe_ffn_workspace_size",
+           "moe_expert_ffn", "moe_combine", "moe_sync_status"]
+
+_lib = None
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, call: str):
+        self.status = status
+        super().__init__(f"{call}: {status_string(status)}")
+
+
+def load() -> ctypes.CDLL:
+    """Load libmoe.so (built by ``python -m combine_moe_route_10_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libmoe.so not found at {LIB_PATH}; build it with "
+                          "`python -m combine_moe_route_10_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, Z, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_double
+    sig = {
+        "moe_abi_version": (I, []),
+        "moe_status_string": (ctypes.c_char_p, [I]),
+        "moe_capacity": (I, [D, I, I, I]),
+        "moe_route": (I, [P, I, I, I, I, P, P, P, P]),
+        "moe_dispatch_workspace_size": (Z, [I, I, I]),
+        "moe_dispatch": (I, [P, I, I, P, I, I, I, I, I, P, P, P, P, P, P, P, P, Z, P]),
+        "moe_ffn_workspace_size": (Z, [I, I, I, I, I]),
+        "moe_expert_ffn": (I, [P, P, I, P, I, I, I, I, P, P, P, P, P, Z, P]),
+        "moe_combine": (I, [P, I, P, P, I, I, I, P, P]),
+        "moe_sync_status": (I, [P, P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().moe_status_string(int(status)).decode()
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(st: int, call: str, raise_on_error: bool):
+    if raise_on_error and st != MOE_OK:
+        raise MoeError(st, call)
+    return st
+
+
+def moe_abi_version() -> int:
+    return load().moe_abi_version()
+
+
+def moe_capacity(cf: float, T: int, k: int, E: int) -> int:
+    return load().moe_capacity(float(cf), T, k, E)
+
+
+def moe_route(logits, T, E, k, renormalize, topk_idx, topk_w, expert_routed=None, stream=None,
+              raise_on_error=True):
+    st = load().moe_route(_ptr(logits), T, E, k, int(renormalize), _ptr(topk_idx), _ptr(topk_w),
+                          _ptr(expert_routed), _stream(stream))
+    return _check(st, "moe_route", raise_on_error)
+
+
+def moe_dispatch_workspace_size(T, E, k) -> int:
+    return load().moe_dispatch_workspace_size(T, E, k)
+
+
+def moe_dispatch(x, T, H, topk_idx, k, E, R, capacity, payload, send, send_scales, expert_counts,
+                 expert_offsets, rank_offsets, slot_row, row_token, ws, ws_bytes, stream=None,
+                 raise_on_error=True):
+    st = load().moe_dispatch(_ptr(x), T, H, _ptr(topk_idx), k, E, R, capacity, payload, _ptr(send),
+                             _ptr(send_scales), _ptr(expert_counts), _ptr(expert_offsets),
+                             _ptr(rank_offsets), _ptr(slot_row), _ptr(row_token), _ptr(ws),
+                             ws_bytes, _stream(stream))
+    return _check(st, "moe_dispatch", raise_on_error)
+
+
+def moe_ffn_workspace_size(max_rows, E, H, F, payload) -> int:
+    return load().moe_ffn_workspace_size(max_rows, E, H, F, payload)
+
+
+def moe_expert_ffn(send, send_scales, payload, expert_offsets, max_rows, E, H, F, w_gate, w_up,
+                   w_down, expert_out, ws, ws_bytes, stream=None, raise_on_error=True):
+    st = load().moe_expert_ffn(_ptr(send), _ptr(send_scales), payload, _ptr(expert_offsets),
+                               max_rows, E, H, F, _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+                               _ptr(expert_out), _ptr(ws), ws_bytes, _stream(stream))
+    return _check(st, "moe_expert_ffn", raise_on_error)
+
+
+def moe_combine(expert_out, max_rows, slot_row, topk_w, T, k, H, y, stream=None,
+                raise_on_error=True):
+    st = load().moe_combine(_ptr(expert_out), max_rows, _ptr(slot_row), _ptr(topk_w), T, k, H,
+                            _ptr(y), _stream(stream))
+    return _check(st, "moe_combine", raise_on_error)
+
+
+def moe_sync_status(ws, stream=None) -> int:
+    return load().moe_sync_status(_ptr(ws), _stream(stream))

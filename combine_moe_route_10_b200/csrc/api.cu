@@ -1,0 +1,175 @@
+// C ABI of libmoe (include/moe.h): argument validation, workspace checks and launches.
+// Every check here runs on the host before anything is enqueued; device-side findings go to the
+// workspace status word and are reported by moe_sync_status.
+#include <math.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+#include "common.cuh"
+#include "launch.h"
+
+namespace moe {
+
+int num_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+}  // namespace moe
+
+namespace {
+
+constexpr int kMaxE = 1024;
+constexpr int kMaxK = 32;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+moe_status_t from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return MOE_OK;
+  cudaGetLastError();  // clear a sticky launch error so the next call starts clean
+  return MOE_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_abi_version(void) { return 1; }
+
+const char* moe_status_string(moe_status_t st) {
+  switch (st) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: invalid argument";
+    case MOE_ERR_INVALID_TOPK: return "MOE_ERR_INVALID_TOPK: routing index out of range";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: shape not supported";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: CUDA launch or runtime error";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace too small or misaligned";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT: a bounded device wait ran out";
+  }
+  return "unknown moe_status_t";
+}
+
+int moe_capacity(double cf, int T, int k, int E) {
+  if (T < 0 || k < 1 || E < 1) return -1;
+  if (!(cf > 0.0)) return 0;
+  const double c = ceil(cf * (static_cast<double>(T) * k) / E);
+  if (c > 2147483647.0) return 2147483647;
+  return static_cast<int>(c);
+}
+
+moe_status_t moe_route(const float* logits, int T, int E, int k, int renormalize,
+                       int32_t* topk_idx, float* topk_w, int32_t* expert_routed,
+                       moe_stream_t stream) {
+  if (T < 0 || E < 1 || E > kMaxE || k < 1 || k > E || k > kMaxK) return MOE_ERR_INVALID_ARG;
+  if (static_cast<long long>(T) * E > INT32_MAX) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (logits == nullptr || topk_idx == nullptr || topk_w == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(logits, 4) || !aligned(topk_idx, 4) || !aligned(topk_w, 4) ||
+      !aligned(expert_routed, 4))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_route(logits, T, E, k, renormalize ? 1 : 0, topk_idx, topk_w,
+                                     expert_routed, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_dispatch_workspace_size(int T, int E, int k) {
+  (void)k;
+  if (T < 0 || E < 1) return 0;
+  return moe::dispatch_workspace_bytes(T, E);
+}
+
+moe_status_t moe_dispatch(const void* x, int T, int H, const int32_t* topk_idx, int k, int E,
+                          int R, int capacity, moe_payload_t payload, void* send,
+                          float* send_scales, int32_t* expert_counts, int32_t* expert_offsets,
+                          int32_t* rank_offsets, int32_t* slot_row, int32_t* row_token, void* ws,
+                          size_t ws_bytes, moe_stream_t stream) {
+  if (T < 0 || E < 1 || E > kMaxE || k < 1 || k > E || k > kMaxK || R < 1 || E % R != 0 ||
+      capacity < 0 || H < 8)
+    return MOE_ERR_INVALID_ARG;
+  if (static_cast<long long>(T) * k >= INT32_MAX) return MOE_ERR_INVALID_ARG;
+  if (payload != MOE_PAYLOAD_BF16 && payload != MOE_PAYLOAD_FP8_E4M3_B128)
+    return MOE_ERR_INVALID_ARG;
+  if (H % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  const bool fp8 = payload == MOE_PAYLOAD_FP8_E4M3_B128;
+  if (fp8 && H % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (expert_counts == nullptr || expert_offsets == nullptr || rank_offsets == nullptr ||
+      ws == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (x == nullptr || topk_idx == nullptr || send == nullptr || slot_row == nullptr ||
+                row_token == nullptr || (fp8 && send_scales == nullptr)))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(send, 16) || !aligned(send_scales, 4) || !aligned(topk_idx, 4))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(ws, 256) || ws_bytes < moe::dispatch_workspace_bytes(T, E)) return MOE_ERR_WORKSPACE;
+  return from_cuda(moe::launch_dispatch(x, T, H, topk_idx, k, E, R, capacity, fp8 ? 1 : 0, send,
+                                        send_scales, expert_counts, expert_offsets, rank_offsets,
+                                        slot_row, row_token, ws,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_ffn_workspace_size(int max_rows, int E, int H, int F, moe_payload_t payload) {
+  (void)E;
+  if (max_rows < 0 || H < 1 || F < 1) return 0;
+  return moe::ffn_workspace_bytes(max_rows, H, F, payload == MOE_PAYLOAD_FP8_E4M3_B128);
+}
+
+moe_status_t moe_expert_ffn(const void* send, const float* send_scales, moe_payload_t payload,
+                            const int32_t* expert_offsets, int max_rows, int E, int H, int F,
+                            const void* w_gate, const void* w_up, const void* w_down,
+                            void* expert_out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (max_rows < 0 || E < 1 || E > kMaxE || H < 1 || F < 1) return MOE_ERR_INVALID_ARG;
+  if (payload != MOE_PAYLOAD_BF16 && payload != MOE_PAYLOAD_FP8_E4M3_B128)
+    return MOE_ERR_INVALID_ARG;
+  const bool fp8 = payload == MOE_PAYLOAD_FP8_E4M3_B128;
+  if (H % 64 != 0 || F % 64 != 0 || (fp8 && H % 128 != 0)) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(E) * F > INT32_MAX || static_cast<long long>(E) * H > INT32_MAX)
+    return MOE_ERR_UNSUPPORTED;
+  if (expert_offsets == nullptr || w_gate == nullptr || w_up == nullptr || w_down == nullptr ||
+      ws == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (max_rows > 0 && (send == nullptr || expert_out == nullptr || (fp8 && send_scales == nullptr)))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(send, 16) || !aligned(w_gate, 16) || !aligned(w_up, 16) || !aligned(w_down, 16) ||
+      !aligned(expert_out, 16) || !aligned(expert_offsets, 4) || !aligned(send_scales, 4))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(ws, 256) || ws_bytes < moe::ffn_workspace_bytes(max_rows, H, F, fp8 ? 1 : 0))
+    return MOE_ERR_WORKSPACE;
+  return from_cuda(moe::launch_expert_ffn(send, send_scales, fp8 ? 1 : 0, expert_offsets, max_rows,
+                                          E, H, F, w_gate, w_up, w_down, expert_out, ws,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_combine(const void* expert_out, int max_rows, const int32_t* slot_row,
+                         const float* topk_w, int T, int k, int H, void* y, moe_stream_t stream) {
+  if (T < 0 || k < 1 || k > kMaxK || H < 8 || max_rows < 0) return MOE_ERR_INVALID_ARG;
+  if (H % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (T > 0 && (slot_row == nullptr || topk_w == nullptr || y == nullptr ||
+                (max_rows > 0 && expert_out == nullptr)))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(expert_out, 16) || !aligned(y, 16) || !aligned(slot_row, 4) || !aligned(topk_w, 4))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_combine(expert_out, max_rows, slot_row, topk_w, T, k, H, y,
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_sync_status(void* ws, moe_stream_t stream) {
+  if (ws == nullptr || !aligned(ws, 4)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return from_cuda(cudaErrorUnknown);
+  int word = 0;
+  if (cudaMemcpy(&word, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return from_cuda(cudaErrorUnknown);
+  if (word != 0 && cudaMemset(ws, 0, sizeof(int)) != cudaSuccess) return from_cuda(cudaErrorUnknown);
+  if (word & moe::kStatusInvalidTopk) return MOE_ERR_INVALID_TOPK;
+  if (word & moe::kStatusTimeout) return MOE_ERR_TIMEOUT;
+  return MOE_OK;
+}
+
+}  // extern "C"

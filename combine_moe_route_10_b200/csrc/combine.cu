@@ -1,0 +1,122 @@
+// Combine: weighted gather of each token's expert outputs back into token order.
+//
+// The NCCL EP page's low-latency combine (section 2.1) loops over the token's top-k slots and adds
+// each expert output times the token's routing weight.  Here: one warp per token, 16-byte gathers
+// of the k packed rows, fp32 accumulation in the fixed slot order j = 0, 1, ... with every product
+// and every sum rounded separately (no fused multiply-add, so the result does not depend on
+// contraction choices), one bf16 rounding at the end.  Dropped slots (row -1) contribute nothing.
+#include "common.cuh"
+#include "launch.h"
+
+namespace moe {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxSlotsInFlight = 8;  // rows whose vectors are loaded together per step
+
+__device__ __forceinline__ void accumulate(float acc[8], float w, uint4 v) {
+  const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    acc[2 * i] = __fadd_rn(acc[2 * i], __fmul_rn(w, bf16_lo(words[i])));
+    acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], __fmul_rn(w, bf16_hi(words[i])));
+  }
+}
+
+template <int UNROLL>
+__global__ void __launch_bounds__(kThreads)
+    combine_kernel(const uint4* __restrict__ expert_out, int max_rows,
+                   const int32_t* __restrict__ slot_row, const float* __restrict__ topk_w, int T,
+                   int k, int nvec, uint4* __restrict__ y) {
+  const int lane = threadIdx.x & 31;
+  const int nwarps = gridDim.x * kWarps;
+  for (int t = blockIdx.x * kWarps + (threadIdx.x >> 5); t < T; t += nwarps) {
+    int my_row = -1;
+    float my_w = 0.0f;
+    if (lane < k) {
+      my_row = __ldg(slot_row + static_cast<size_t>(t) * k + lane);
+      my_w = __ldg(topk_w + static_cast<size_t>(t) * k + lane);
+      if (my_row >= max_rows) my_row = -1;
+    }
+    const unsigned live = __ballot_sync(0xFFFFFFFFu, my_row >= 0);
+    uint4* dst = y + static_cast<size_t>(t) * nvec;
+    for (int v0 = 0; v0 < nvec; v0 += 32 * UNROLL) {
+      float acc[UNROLL][8];
+#pragma unroll
+      for (int u = 0; u < UNROLL; ++u)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[u][i] = 0.0f;
+      // slots in ascending j, kMaxSlotsInFlight rows loaded before they are accumulated
+      for (unsigned m = live; m != 0;) {
+        int rows[kMaxSlotsInFlight];
+        float ws[kMaxSlotsInFlight];
+        int n = 0;
+#pragma unroll
+        for (int q = 0; q < kMaxSlotsInFlight; ++q) {
+          rows[q] = -1;
+          ws[q] = 0.0f;
+          if (m != 0) {
+            const int j = __ffs(m) - 1;
+            m &= m - 1;
+            rows[q] = j;
+            n = q + 1;
+          }
+        }
+        uint4 vals[kMaxSlotsInFlight][UNROLL];
+#pragma unroll
+        for (int q = 0; q < kMaxSlotsInFlight; ++q) {
+          if (q < n) {
+            const int j = rows[q];
+            const int row = __shfl_sync(0xFFFFFFFFu, my_row, j);
+            ws[q] = __shfl_sync(0xFFFFFFFFu, my_w, j);
+            const uint4* src = expert_out + static_cast<size_t>(row) * nvec;
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) {
+              const int v = v0 + u * 32 + lane;
+              if (v < nvec) vals[q][u] = ld_nc_v4(src + v);
+            }
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < kMaxSlotsInFlight; ++q) {
+          if (q < n) {
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) {
+              const int v = v0 + u * 32 + lane;
+              if (v < nvec) accumulate(acc[u], ws[q], vals[q][u]);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < UNROLL; ++u) {
+        const int v = v0 + u * 32 + lane;
+        if (v < nvec) {
+          uint4 o;
+          o.x = pack_bf16x2(acc[u][0], acc[u][1]);
+          o.y = pack_bf16x2(acc[u][2], acc[u][3]);
+          o.z = pack_bf16x2(acc[u][4], acc[u][5]);
+          o.w = pack_bf16x2(acc[u][6], acc[u][7]);
+          st_v4(dst + v, o);
+        }
+      }
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const void* expert_out, int max_rows, const int32_t* slot_row,
+                           const float* topk_w, int T, int k, int H, void* y, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  int blocks = (T + kWarps - 1) / kWarps;
+  const int cap = num_sms() * 8;
+  if (blocks > cap) blocks = cap;
+  combine_kernel<2><<<blocks, kThreads, 0, s>>>(static_cast<const uint4*>(expert_out), max_rows,
+                                                slot_row, topk_w, T, k, H / 8,
+                                                static_cast<uint4*>(y));
+  return cudaGetLastError();
+}
+
+}  // namespace moe

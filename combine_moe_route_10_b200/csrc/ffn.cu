@@ -1,0 +1,586 @@
+// Grouped SwiGLU expert FFN on the packed send buffer: tcgen05 tensor cores, TMEM accumulators,
+// TMA-fed shared-memory pipeline.
+//
+// Per expert e and each of its packed rows x (expert-major layout of the NCCL EP page, section
+// 2.1; two linear layers with SwiGLU per expert as in "细粒度专家并行方案对比：MegaMoE与传统方案",
+// section 核心差异分析 1; fused w3_w1 projection with the SwiGLU epilogue, then w2, as in the
+// run_moe passage of "DWDP: 在NVL72上的高性能分布式权重数据并行"):
+//     h = bf16( silu(x W_gate[e]^T) * (x W_up[e]^T) ),   expert_out = bf16( h W_down[e]^T ).
+//
+// Two launches of one persistent kernel template (one CTA per SM, 192 threads):
+//   warp 0      TMA producer: A tile (128 rows x 64 k) + B tile (256 rows x 64 k) per stage,
+//               128-byte swizzle, 4-stage mbarrier ring;
+//   warp 1      TMEM allocator and MMA issuer: one thread issues tcgen05.mma (M=128, N=256,
+//               K=16, bf16 -> fp32) into one of two 256-column TMEM accumulators, and
+//               tcgen05.commit frees smem stages / publishes finished accumulators;
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (one TMEM lane quarter per warp), then
+//               SwiGLU (GEMM-1: gate columns 0..127 and up columns 128..255 of one accumulator)
+//               or a plain bf16 cast (GEMM-2), masked row/column stores.
+// The tile schedule (expert, row block, column block) is derived on the device from
+// expert_offsets, so nothing is synchronised with the host.  Row blocks of an expert are the
+// fastest-varying index, so CTAs running together share weight column blocks through L2.
+// Every mbarrier wait is bounded; on a timeout the CTA records MOE status bit kStatusTimeout,
+// drains its own outstanding TMA loads and MMAs, frees TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128;          // rows per tile (UMMA M, one TMEM lane per row)
+constexpr int BK = 64;           // k per stage: 64 bf16 = one 128-byte swizzle atom row
+constexpr int UMMA_K = 16;       // k per tcgen05.mma for kind::f16
+constexpr int kStages = 4;
+constexpr int kAccCols = 256;    // fp32 TMEM columns per accumulator
+constexpr int kTmemCols = 512;   // two accumulators
+constexpr int kThreads = 192;
+constexpr int kATileBytes = BM * BK * 2;   // 16 KB
+constexpr int kBTileBytes = 256 * BK * 2;  // 32 KB
+constexpr int kStageBytes = kATileBytes + kBTileBytes;
+
+enum Mode { kSwiGLU = 0, kPlain = 1 };
+
+struct GemmArgs {
+  const int32_t* expert_offsets;  // [E+1], device
+  int E;
+  int max_rows;
+  int N;       // output columns (F for SwiGLU, H for the plain GEMM)
+  int K;       // reduction length (H, resp. F)
+  int n_tile;  // output columns per tile (128 for SwiGLU; 256 or 128 for plain)
+  int b_rows_per_expert;  // rows of one expert in the B tensor map(s)
+  __nv_bfloat16* out;     // [max_rows, N]
+  int* status;
+};
+
+// ---- PTX wrappers ------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm, uint32_t bar,
+                                            int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major bf16 tile stored with the 128-byte swizzle:
+// rows of 128 bytes, 8-row groups 1024 bytes apart (stride byte offset), descriptor version 1,
+// layout type 2 (SWIZZLE_128B).  The leading byte offset is unused for swizzled K-major tiles.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(1) << 16;                // leading byte offset (16 B, unused)
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;        // stride byte offset
+  d |= static_cast<uint64_t>(1) << 46;                // descriptor version
+  d |= static_cast<uint64_t>(2) << 61;                // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator, bf16 A and B, both K-major.
+__host__ __device__ constexpr uint32_t make_idesc(int M, int N) {
+  return (1u << 4)                                    // D format: f32
+         | (1u << 7)                                  // A format: bf16
+         | (1u << 10)                                 // B format: bf16
+         | (static_cast<uint32_t>(N >> 3) << 17)      // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);     // M / 16
+}
+
+struct Smem {
+  uint8_t* tiles;         // kStages x (A | B), 1024-byte aligned
+  uint64_t* full;         // [kStages]
+  uint64_t* empty;        // [kStages]
+  uint64_t* acc_full;     // [2]
+  uint64_t* acc_empty;    // [2]
+  uint64_t* drain;        // [1]
+  uint32_t* tmem_base;
+  int* abort_flag;
+  int* off;               // [E+1] row offsets (clamped to max_rows)
+  int* tstart;            // [E+1] first tile of each expert; tstart[E] = total tiles
+  int* mtiles;            // [E]
+};
+
+__device__ __forceinline__ Smem carve(uint8_t* raw, int E) {
+  Smem s;
+  const uint32_t a = smem_addr(raw);
+  uint8_t* p = raw + ((1024u - (a & 1023u)) & 1023u);
+  s.tiles = p;
+  p += kStages * kStageBytes;
+  s.full = reinterpret_cast<uint64_t*>(p);
+  s.empty = s.full + kStages;
+  s.acc_full = s.empty + kStages;
+  s.acc_empty = s.acc_full + 2;
+  s.drain = s.acc_empty + 2;
+  s.tmem_base = reinterpret_cast<uint32_t*>(s.drain + 1);
+  s.abort_flag = reinterpret_cast<int*>(s.tmem_base + 1);
+  s.off = s.abort_flag + 2;
+  s.tstart = s.off + (E + 1);
+  s.mtiles = s.tstart + (E + 1);
+  return s;
+}
+
+size_t gemm_smem_bytes(int E) {
+  return 1024 + static_cast<size_t>(kStages) * kStageBytes + 8 * (2 * kStages + 5) + 16 +
+         sizeof(int) * (3 * static_cast<size_t>(E) + 2);
+}
+
+// Bounded wait on an mbarrier phase.  Returns false if the CTA is aborting or the limit ran out.
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                           int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      record_status(status, kStatusTimeout);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void decode_tile(const Smem& s, int E, int tile, int& e, int& m_blk,
+                                            int& n_blk) {
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {  // largest expert whose first tile is <= tile (it owns the tile)
+    const int mid = (lo + hi + 1) >> 1;
+    if (s.tstart[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
+  e = lo;
+  const int local = tile - s.tstart[lo];
+  const int mt = s.mtiles[lo];
+  n_blk = local / mt;
+  m_blk = local - n_blk * mt;
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  return g / (1.0f + expf(-g)) * u;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
+                        const __grid_constant__ CUtensorMap tm_b0,
+                        const __grid_constant__ CUtensorMap tm_b1, const GemmArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  const int E = args.E;
+  Smem s = carve(smem_raw, E);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = (args.N + args.n_tile - 1) / args.n_tile;
+  const int num_kb = (args.K + BK - 1) / BK;
+  volatile int* abort_flag = s.abort_flag;
+
+  // ---- set-up: barriers, TMEM, schedule --------------------------------------------------------
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int i = 0; i < kStages; ++i) {
+        mbar_init(smem_addr(&s.full[i]), 1);
+        mbar_init(smem_addr(&s.empty[i]), 1);
+      }
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(smem_addr(&s.acc_full[i]), 1);
+        mbar_init(smem_addr(&s.acc_empty[i]), 4);  // one arrival per epilogue warp
+      }
+      mbar_init(smem_addr(s.drain), 1);
+      *s.abort_flag = 0;
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_a)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_b0)) : "memory");
+      if (MODE == kSwiGLU)
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_b1)) : "memory");
+    }
+  } else if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(s.tmem_base)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  } else if (warp == 2) {
+    // schedule: per-expert row offsets, row-block counts and the first tile of each expert
+    int carry = 0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int e = e0 + lane;
+      int lo = 0, hi = 0;
+      if (e < E) {
+        lo = min(__ldg(args.expert_offsets + e), args.max_rows);
+        hi = min(__ldg(args.expert_offsets + e + 1), args.max_rows);
+      }
+      const int rows = max(hi - lo, 0);
+      const int mt = (rows + BM - 1) / BM;
+      const int tiles = mt * n_tiles;
+      int incl = tiles;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (e < E) {
+        s.off[e] = lo;
+        s.mtiles[e] = mt;
+        s.tstart[e] = carry + incl - tiles;
+      }
+      carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    }
+    if (lane == 0) {
+      s.tstart[E] = carry;
+      s.off[E] = min(__ldg(args.expert_offsets + E), args.max_rows);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s.tmem_base;
+  const int total_tiles = s.tstart[E];
+  const uint32_t tiles_base = smem_addr(s.tiles);
+
+  if (warp == 0) {
+    // ---- TMA producer ----------------------------------------------------------------------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_parity = 0;  // per stage: issued at least once / last parity
+      const uint32_t tx = MODE == kSwiGLU ? kStageBytes
+                                          : kATileBytes + args.n_tile * BK * 2;
+      for (int tile = blockIdx.x; tile < total_tiles && !*abort_flag; tile += gridDim.x) {
+        int e, m_blk, n_blk;
+        decode_tile(s, E, tile, e, m_blk, n_blk);
+        const int row_a = s.off[e] + m_blk * BM;
+        const int row_b = e * args.b_rows_per_expert + n_blk * args.n_tile;
+        bool ok = true;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!wait_phase(smem_addr(&s.empty[stage]), phase ^ 1u, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t a_dst = tiles_base + stage * kStageBytes;
+          const uint32_t b_dst = a_dst + kATileBytes;
+          const uint32_t fb = smem_addr(&s.full[stage]);
+          mbar_arrive_expect_tx(fb, tx);
+          tma_load_2d(a_dst, &tm_a, fb, kb * BK, row_a);
+          tma_load_2d(b_dst, &tm_b0, fb, kb * BK, row_b);
+          if (MODE == kSwiGLU) tma_load_2d(b_dst + kBTileBytes / 2, &tm_b1, fb, kb * BK, row_b);
+          issued_mask |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+      }
+      if (*abort_flag) {
+        // let this CTA's own bulk copies land before the CTA (and its smem) goes away
+        volatile int no_abort = 0;
+        for (int st = 0; st < kStages; ++st)
+          if (issued_mask & (1u << st))
+            wait_phase(smem_addr(&s.full[st]), (issued_parity >> st) & 1u, &no_abort,
+                       args.status);
+      }
+    }
+  } else if (warp == 1) {
+    // ---- MMA issuer --------------------------------------------------------------------------------
+    if (lane == 0) {
+      const uint32_t idesc = make_idesc(BM, MODE == kSwiGLU ? 256 : args.n_tile);
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool issued_any = false;
+      for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_parity = (it >> 1) & 1;
+        if (!wait_phase(smem_addr(&s.acc_empty[acc]), acc_parity ^ 1u, abort_flag, args.status))
+          break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * kAccCols;
+        bool ok = true;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!wait_phase(smem_addr(&s.full[stage]), phase, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = tiles_base + stage * kStageBytes;
+          const uint32_t b_addr = a_addr + kATileBytes;
+#pragma unroll
+          for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+            tc_mma(d_tmem, sw128_desc(a_addr + kk * UMMA_K * 2), sw128_desc(b_addr + kk * UMMA_K * 2),
+                   idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          issued_any = true;
+          tc_commit(smem_addr(&s.empty[stage]));  // stage reusable once these MMAs finish
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(smem_addr(&s.acc_full[acc]));  // accumulator complete
+      }
+      if (issued_any) {
+        // all MMAs of this CTA retire before TMEM is released
+        tc_commit(smem_addr(s.drain));
+        volatile int no_abort = 0;
+        wait_phase(smem_addr(s.drain), 0, &no_abort, args.status);
+      }
+    }
+  } else {
+    // ---- epilogue: TMEM -> registers -> global ---------------------------------------------------
+    const int quarter = warp & 3;                    // TMEM lanes 32*quarter .. 32*quarter+31
+    const int r_local = quarter * 32 + lane;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
+      int e, m_blk, n_blk;
+      decode_tile(s, E, tile, e, m_blk, n_blk);
+      const int acc = it & 1;
+      const uint32_t acc_parity = (it >> 1) & 1;
+      // one lane waits and the warp follows its verdict, so the .sync.aligned TMEM loads below
+      // are always executed by the whole warp or by none of it
+      bool ok = true;
+      if (lane == 0) ok = wait_phase(smem_addr(&s.acc_full[acc]), acc_parity, abort_flag, args.status);
+      if (!__shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0)) break;
+      tc_fence_after();
+      const int row = s.off[e] + m_blk * BM + r_local;
+      const bool row_ok = row < s.off[e + 1];
+      const uint32_t t_row = tmem_base + acc * kAccCols + (static_cast<uint32_t>(quarter * 32) << 16);
+      __nv_bfloat16* out_row = args.out + static_cast<size_t>(row) * args.N;
+      if (MODE == kSwiGLU) {
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 32) {
+          uint32_t g[32], u[32];
+          tmem_ld32(t_row + c, g);
+          tmem_ld32(t_row + 128 + c, u);
+          tmem_wait_ld();
+          const int col = n_blk * 128 + c;
+          if (row_ok && col < args.N) {
+            uint32_t packed[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float h0 = silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i]));
+              const float h1 = silu_mul(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1]));
+              packed[i] = pack_bf16x2(h0, h1);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(out_row + col);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < args.n_tile; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(t_row + c, v);
+          tmem_wait_ld();
+          const int col = n_blk * args.n_tile + c;
+          if (row_ok && col < args.N) {
+            uint32_t packed[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              packed[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+            uint4* dst = reinterpret_cast<uint4*>(out_row + col);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_addr(&s.acc_empty[acc]));
+    }
+  }
+
+  // ---- teardown ------------------------------------------------------------------------------------
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// FP8 payload -> bf16 FFN input rows: x = bf16(fp32(code) * scale), rows [0, expert_offsets[E]).
+__global__ void __launch_bounds__(256)
+    dequant_fp8_kernel(const uint8_t* __restrict__ q, const float* __restrict__ scales,
+                       const int32_t* __restrict__ total_rows, int max_rows, int H,
+                       uint4* __restrict__ out) {
+  const int S = min(__ldg(total_rows), max_rows);
+  const int per_row = H / 16;  // 16 codes per thread step
+  const long long n = static_cast<long long>(S) * per_row;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long row = i / per_row;
+    const int c16 = static_cast<int>(i - row * per_row);
+    const uint4 codes = ld_nc_v4(q + i * 16);
+    const float sc = __ldg(scales + row * (H / 128) + (c16 * 16) / 128);
+    const uint32_t w[4] = {codes.x, codes.y, codes.z, codes.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>(w[j] >> (16 * h));
+        const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);  // exact
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+        o[2 * j + h] = pack_bf16x2(__fmul_rn(f.x, sc), __fmul_rn(f.y, sc));
+      }
+    }
+    out[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
+    out[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
+// ---- host side -----------------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor [rows, cols] (cols contiguous) read in boxes of box_rows x 64 with the
+// 128-byte swizzle; out-of-range elements read as zero.
+bool make_tmap(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int MODE>
+cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                        const GemmArgs& args, cudaStream_t s) {
+  const size_t smem = gemm_smem_bytes(args.E);
+  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  grouped_gemm_kernel<MODE><<<num_sms(), kThreads, smem, s>>>(a, b0, b1, args);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t ffn_workspace_bytes(int max_rows, int H, int F, int fp8) {
+  const size_t h_bytes = (static_cast<size_t>(max_rows) * F * 2 + 255) / 256 * 256;
+  const size_t x_bytes = fp8 ? (static_cast<size_t>(max_rows) * H * 2 + 255) / 256 * 256 : 0;
+  return 256 + h_bytes + x_bytes;
+}
+
+cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp8,
+                              const int32_t* expert_offsets, int max_rows, int E, int H, int F,
+                              const void* w_gate, const void* w_up, const void* w_down,
+                              void* expert_out, void* ws, cudaStream_t s) {
+  if (max_rows == 0) return cudaSuccess;
+  char* base = static_cast<char*>(ws);
+  int* status = reinterpret_cast<int*>(base);
+  __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(base + 256);
+  const void* a_src = send;
+  if (fp8) {
+    uint4* xdq = reinterpret_cast<uint4*>(
+        base + 256 + (static_cast<size_t>(max_rows) * F * 2 + 255) / 256 * 256);
+    const long long work = static_cast<long long>(max_rows) * (H / 16);
+    long long blocks = (work + 255) / 256;
+    const long long cap = static_cast<long long>(num_sms()) * 8;
+    if (blocks > cap) blocks = cap;
+    dequant_fp8_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(
+        static_cast<const uint8_t*>(send), send_scales, expert_offsets + E, max_rows, H, xdq);
+    a_src = xdq;
+  }
+  CUtensorMap tm_x, tm_g, tm_u, tm_h, tm_d;
+  const int n_tile2 = 256;
+  if (!make_tmap(&tm_x, a_src, max_rows, H, BM) ||
+      !make_tmap(&tm_g, w_gate, static_cast<uint64_t>(E) * F, H, 128) ||
+      !make_tmap(&tm_u, w_up, static_cast<uint64_t>(E) * F, H, 128) ||
+      !make_tmap(&tm_h, h, max_rows, F, BM) ||
+      !make_tmap(&tm_d, w_down, static_cast<uint64_t>(E) * H, F, n_tile2))
+    return cudaErrorInvalidValue;
+
+  GemmArgs g1{expert_offsets, E, max_rows, F, H, 128, F, h, status};
+  cudaError_t err = launch_gemm<kSwiGLU>(tm_x, tm_g, tm_u, g1, s);
+  if (err != cudaSuccess) return err;
+  GemmArgs g2{expert_offsets, E, max_rows, H, F, n_tile2, H,
+              static_cast<__nv_bfloat16*>(expert_out), status};
+  return launch_gemm<kPlain>(tm_h, tm_d, tm_d, g2, s);
+}
+
+}  // namespace moe

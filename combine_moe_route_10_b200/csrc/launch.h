@@ -1,0 +1,39 @@
+// Internal launchers of libmoe (host side).  The public C ABI is include/moe.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+int num_sms();  // SM count of the current device (cached per device)
+
+cudaError_t launch_route(const float* logits, int T, int E, int k, int renorm, int32_t* topk_idx,
+                         float* topk_w, int32_t* routed, cudaStream_t s);
+
+// Dispatch workspace layout (bytes from the 256-byte-aligned base):
+//   [0, 4)    status word (kStatus* bits)
+//   [4, 8)    arrival counter of the count/scan kernel (returns to 0 after every call)
+//   [256, ..) per-chunk expert histogram, then per-chunk base positions [n_chunks][E] int32
+constexpr int kDispatchChunk = 256;  // tokens per counting / ranking chunk
+size_t dispatch_workspace_bytes(int T, int E);
+
+cudaError_t launch_dispatch(const void* x, int T, int H, const int32_t* topk_idx, int k, int E,
+                            int R, int capacity, int fp8, void* send, float* send_scales,
+                            int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_offsets,
+                            int32_t* slot_row, int32_t* row_token, void* ws, cudaStream_t s);
+
+cudaError_t launch_combine(const void* expert_out, int max_rows, const int32_t* slot_row,
+                           const float* topk_w, int T, int k, int H, void* y, cudaStream_t s);
+
+// FFN workspace layout: [0,4) status, [256, ..) h [max_rows, F] bf16, then for the FP8 payload the
+// dequantised rows [max_rows, H] bf16.
+size_t ffn_workspace_bytes(int max_rows, int H, int F, int fp8);
+
+cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp8,
+                              const int32_t* expert_offsets, int max_rows, int E, int H, int F,
+                              const void* w_gate, const void* w_up, const void* w_down,
+                              void* expert_out, void* ws, cudaStream_t s);
+
+}  // namespace moe

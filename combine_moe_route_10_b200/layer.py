@@ -1,0 +1,101 @@
+"""Device buffers for one MoE layer shape and the four C-ABI calls in order on one stream.
+
+Memory comes from torch (the caller-owned allocation of the C ABI); all arithmetic runs in
+libmoe.so.  Nothing here synchronises with the host except ``status()``.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib
+
+
+class MoeShuffle:
+    """Route -> dispatch -> grouped SwiGLU FFN -> combine for T tokens of width H over E experts.
+
+    ``payload`` is "bf16" or "fp8" (e4m3 codes + one fp32 scale per 128 elements); ``capacity``
+    is the per-expert row limit (0 = keep every slot, see ``moe_capacity``); rank r of R owns
+    experts [r*E/R, (r+1)*E/R).
+    """
+
+    def __init__(self, T: int, H: int, E: int, k: int, R: int, F: int, payload: str = "bf16",
+                 capacity: int = 0, renormalize: bool = True, device="cuda"):
+        _lib.load()
+        self.T, self.H, self.E, self.k, self.R, self.F = T, H, E, k, R, F
+        self.capacity = int(capacity)
+        self.renormalize = bool(renormalize)
+        self.fp8 = payload == "fp8"
+        if payload not in ("bf16", "fp8"):
+            raise ValueError("payload must be 'bf16' or 'fp8'")
+        self.payload = _lib.MOE_PAYLOAD_FP8_E4M3_B128 if self.fp8 else _lib.MOE_PAYLOAD_BF16
+        dev = torch.device(device)
+        i32 = dict(dtype=torch.int32, device=dev)
+        S = T * k
+        self.max_rows = S
+        self.topk_idx = torch.empty((T, k), **i32)
+        self.topk_w = torch.empty((T, k), dtype=torch.float32, device=dev)
+        self.expert_routed = torch.empty(E, **i32)
+        if self.fp8:
+            self.send = torch.empty((S, H), dtype=torch.uint8, device=dev)
+            self.send_scales = torch.empty((S, H // 128), dtype=torch.float32, device=dev)
+        else:
+            self.send = torch.empty((S, H), dtype=torch.bfloat16, device=dev)
+            self.send_scales = None
+        self.expert_counts = torch.empty(E, **i32)
+        self.expert_offsets = torch.empty(E + 1, **i32)
+        self.rank_offsets = torch.empty(R + 1, **i32)
+        self.slot_row = torch.empty((T, k), **i32)
+        self.row_token = torch.empty(max(S, 1), **i32)
+        self.expert_out = torch.empty((S, H), dtype=torch.bfloat16, device=dev)
+        self.y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        self.ws_dispatch_bytes = _lib.moe_dispatch_workspace_size(T, E, k)
+        self.ws_dispatch = torch.zeros(self.ws_dispatch_bytes, dtype=torch.uint8, device=dev)
+        self.ws_ffn_bytes = _lib.moe_ffn_workspace_size(S, E, H, F, self.payload)
+        self.ws_ffn = torch.zeros(self.ws_ffn_bytes, dtype=torch.uint8, device=dev)
+
+    # -- views into the FFN workspace ----------------------------------------------------------
+    @property
+    def h(self) -> torch.Tensor:
+        """The bf16 SwiGLU intermediate [max_rows, F] (inside the FFN workspace)."""
+        n = self.max_rows * self.F * 2
+        return self.ws_ffn[256:256 + n].view(torch.bfloat16).view(self.max_rows, self.F)
+
+    # -- the four stages ----------------------------------------------------------------------
+    def route(self, logits: torch.Tensor, stream=None):
+        _lib.moe_route(logits, self.T, self.E, self.k, self.renormalize, self.topk_idx,
+                       self.topk_w, self.expert_routed, stream)
+
+    def dispatch(self, x: torch.Tensor, topk_idx: torch.Tensor | None = None, stream=None):
+        idx = self.topk_idx if topk_idx is None else topk_idx
+        _lib.moe_dispatch(x, self.T, self.H, idx, self.k, self.E, self.R, self.capacity,
+                          self.payload, self.send, self.send_scales, self.expert_counts,
+                          self.expert_offsets, self.rank_offsets, self.slot_row, self.row_token,
+                          self.ws_dispatch, self.ws_dispatch_bytes, stream)
+
+    def expert_ffn(self, w_gate, w_up, w_down, send=None, send_scales=None, expert_offsets=None,
+                   stream=None):
+        _lib.moe_expert_ffn(self.send if send is None else send,
+                            self.send_scales if send_scales is None else send_scales,
+                            self.payload,
+                            self.expert_offsets if expert_offsets is None else expert_offsets,
+                            self.max_rows, self.E, self.H, self.F, w_gate, w_up, w_down,
+                            self.expert_out, self.ws_ffn, self.ws_ffn_bytes, stream)
+
+    def combine(self, expert_out=None, slot_row=None, topk_w=None, stream=None):
+        _lib.moe_combine(self.expert_out if expert_out is None else expert_out, self.max_rows,
+                         self.slot_row if slot_row is None else slot_row,
+                         self.topk_w if topk_w is None else topk_w, self.T, self.k, self.H,
+                         self.y, stream)
+
+    def forward(self, logits, x, w_gate, w_up, w_down, stream=None) -> torch.Tensor:
+        self.route(logits, stream)
+        self.dispatch(x, stream=stream)
+        self.expert_ffn(w_gate, w_up, w_down, stream=stream)
+        self.combine(stream=stream)
+        return self.y
+
+    def status(self, stream=None) -> int:
+        """Synchronise and return (then clear) the device status of the dispatch and FFN stages."""
+        a = _lib.moe_sync_status(self.ws_dispatch, stream)
+        b = _lib.moe_sync_status(self.ws_ffn, stream)
+        return a if a != _lib.MOE_OK else b

@@ -1,0 +1,128 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every function that
+include/moe.h declares, and rejects invalid arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import combine_moe_route_10_b200 as pkg
+from combine_moe_route_10_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from combine_moe_route_10_b200 import build
+    build.build()
+    return pkg.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_four_calls():
+    names = declared_functions()
+    for n in ["moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(_lib.EXPORTS) == names
+
+
+def test_abi_version_and_status_strings(lib):
+    assert pkg.moe_abi_version() == 1
+    for code in range(7):
+        assert pkg.status_string(code).startswith("MOE_")
+    assert "unknown" in pkg.status_string(99)
+
+
+def test_capacity_helper(lib):
+    assert pkg.moe_capacity(1.0, 65536, 2, 128) == 1024     # printed example
+    assert pkg.moe_capacity(1.25, 16384, 2, 128) == 320
+    assert pkg.moe_capacity(1.0, 10, 1, 3) == 4
+    assert pkg.moe_capacity(0.0, 10, 1, 3) == 0
+    assert pkg.moe_capacity(1.0, -1, 1, 3) == -1
+
+
+FAKE = 1 << 20   # never dereferenced: every call below fails validation first
+
+
+def test_route_rejects_bad_arguments(lib):
+    bad = [dict(T=-1, E=8, k=2), dict(T=4, E=0, k=1), dict(T=4, E=8, k=9), dict(T=4, E=8, k=0),
+           dict(T=4, E=2048, k=2), dict(T=4, E=64, k=33)]
+    for a in bad:
+        st = lib.moe_route(FAKE, a["T"], a["E"], a["k"], 1, FAKE, FAKE, None, None)
+        assert st == pkg.MOE_ERR_INVALID_ARG, a
+    assert lib.moe_route(None, 4, 8, 2, 1, FAKE, FAKE, None, None) == pkg.MOE_ERR_INVALID_ARG
+    assert lib.moe_route(FAKE + 2, 4, 8, 2, 1, FAKE, FAKE, None, None) == pkg.MOE_ERR_INVALID_ARG
+
+
+def dispatch(lib, **kw):
+    a = dict(x=FAKE, T=16, H=256, idx=FAKE, k=2, E=8, R=4, cap=0, payload=0, send=FAKE,
+             scales=FAKE, counts=FAKE, offsets=FAKE, rank_offsets=FAKE, slot_row=FAKE,
+             row_token=FAKE, ws=FAKE, ws_bytes=1 << 20)
+    a.update(kw)
+    return lib.moe_dispatch(a["x"], a["T"], a["H"], a["idx"], a["k"], a["E"], a["R"], a["cap"],
+                            a["payload"], a["send"], a["scales"], a["counts"], a["offsets"],
+                            a["rank_offsets"], a["slot_row"], a["row_token"], a["ws"],
+                            a["ws_bytes"], None)
+
+
+def test_dispatch_rejects_bad_arguments(lib):
+    E = pkg.MOE_ERR_INVALID_ARG
+    assert dispatch(lib, R=3) == E                       # E % R != 0
+    assert dispatch(lib, k=9) == E                       # k > E
+    assert dispatch(lib, cap=-1) == E
+    assert dispatch(lib, payload=7) == E
+    assert dispatch(lib, x=FAKE + 8) == E                # x not 16-byte aligned
+    assert dispatch(lib, send=None) == E
+    assert dispatch(lib, payload=1, scales=None) == E    # FP8 needs the scale output
+    assert dispatch(lib, H=100) == pkg.MOE_ERR_UNSUPPORTED
+    assert dispatch(lib, payload=1, H=320) == pkg.MOE_ERR_UNSUPPORTED
+    assert dispatch(lib, ws_bytes=16) == pkg.MOE_ERR_WORKSPACE
+    assert dispatch(lib, ws=FAKE + 64) == pkg.MOE_ERR_WORKSPACE
+
+
+def test_workspace_sizes(lib):
+    s1 = pkg.moe_dispatch_workspace_size(16384, 128, 2)
+    assert s1 >= 256 + 64 * 128 * 4 and s1 % 256 == 0
+    f = pkg.moe_ffn_workspace_size(32768, 256, 7168, 2048, pkg.MOE_PAYLOAD_FP8_E4M3_B128)
+    assert f >= 256 + 32768 * 2048 * 2 + 32768 * 7168 * 2
+    assert pkg.moe_ffn_workspace_size(100, 8, 256, 512, pkg.MOE_PAYLOAD_BF16) >= 256 + 100 * 512 * 2
+
+
+def test_ffn_and_combine_reject_bad_arguments(lib):
+    ffn = lambda **kw: lib.moe_expert_ffn(
+        kw.get("send", FAKE), kw.get("scales", None), kw.get("payload", 0), FAKE,
+        kw.get("rows", 64), kw.get("E", 8), kw.get("H", 256), kw.get("F", 512), FAKE, FAKE, FAKE,
+        FAKE, kw.get("ws", FAKE), kw.get("ws_bytes", 1 << 30), None)
+    assert ffn(H=200) == pkg.MOE_ERR_UNSUPPORTED
+    assert ffn(F=96) == pkg.MOE_ERR_UNSUPPORTED
+    assert ffn(payload=1) == pkg.MOE_ERR_INVALID_ARG       # FP8 without scales
+    assert ffn(E=0) == pkg.MOE_ERR_INVALID_ARG
+    assert ffn(ws_bytes=100) == pkg.MOE_ERR_WORKSPACE
+    assert ffn(send=FAKE + 4) == pkg.MOE_ERR_INVALID_ARG
+    comb = lambda **kw: lib.moe_combine(FAKE, 64, FAKE, FAKE, kw.get("T", 4), kw.get("k", 2),
+                                        kw.get("H", 256), kw.get("y", FAKE), None)
+    assert comb(k=0) == pkg.MOE_ERR_INVALID_ARG
+    assert comb(H=12) == pkg.MOE_ERR_UNSUPPORTED
+    assert comb(y=FAKE + 2) == pkg.MOE_ERR_INVALID_ARG
+    assert lib.moe_sync_status(None, None) == pkg.MOE_ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "libmoe.so"))
+    with pytest.raises(ImportError):
+        _lib.load()

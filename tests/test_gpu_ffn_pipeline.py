@@ -1,0 +1,160 @@
+"""GPU parity of the grouped SwiGLU FFN and of the whole path against the CPU oracle (C ABI).
+
+The FFN runs bf16 operands on the tensor cores with fp32 accumulation; the oracle accumulates in
+fp64.  Both round h and the output to bf16.  Parity bar (per output tensor): max |gpu - ref| /
+max |ref| <= 1e-2.  Small workloads are compared on every row; the full-size workloads on sampled
+rows (the first and last row of sampled experts plus random rows), run in the same launch
+configuration as the benchmark."""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs as mi
+from _helpers import bits16, bytes8, np_, rel_max_err, to_dev_bf16_from_bits
+from oracle import moe
+
+pytestmark = pytest.mark.gpu
+
+RTOL = 1e-2
+SMALL = ["tiny", "decode-small", "train-small", "finegrained-small", "skewed-small"]
+FULL = ["decode", "train", "finegrained", "skewed"]
+
+
+def shuffle_for(w):
+    from combine_moe_route_10_b200 import MoeShuffle
+    cap = moe.capacity(w.capacity_factor, w.T, w.k, w.E)
+    return MoeShuffle(w.T, w.H, w.E, w.k, w.R, w.F, payload=w.payload, capacity=cap), cap
+
+
+def oracle_plan(w, d):
+    idx, wt, _ = moe.route(np_(d["logits"]), w.k)
+    cap = moe.capacity(w.capacity_factor, w.T, w.k, w.E)
+    plan = moe.dispatch_plan(idx, w.E, w.R, cap)
+    send, scales = moe.dispatch_payload(bits16(d["x"]), plan, w.payload == "fp8")
+    return idx, wt, plan, send, scales
+
+
+def run_gpu_ffn_on_oracle_rows(m, w, plan, send, scales, d):
+    """GPU FFN with the oracle's packed rows and offsets as inputs."""
+    S = plan["S"]
+    if w.payload == "fp8":
+        send_dev = torch.zeros((m.max_rows, w.H), dtype=torch.uint8, device="cuda")
+        send_dev[:S] = torch.from_numpy(send).cuda()
+        sc_dev = torch.zeros((m.max_rows, w.H // 128), dtype=torch.float32, device="cuda")
+        sc_dev[:S] = torch.from_numpy(scales).cuda()
+    else:
+        send_dev = torch.zeros((m.max_rows, w.H), dtype=torch.bfloat16, device="cuda")
+        send_dev[:S] = to_dev_bf16_from_bits(send, "cuda")
+        sc_dev = None
+    off = torch.from_numpy(plan["expert_offsets"]).cuda()
+    m.expert_ffn(d["w_gate"], d["w_up"], d["w_down"], send=send_dev, send_scales=sc_dev,
+                 expert_offsets=off)
+    assert m.status() == 0
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_ffn_parity_all_rows(cuda, name):
+    w = mi.get(name)
+    d = mi.make_inputs(w, seed=0, device="cuda")
+    _, _, plan, send, scales = oracle_plan(w, d)
+    m, _ = shuffle_for(w)
+    run_gpu_ffn_on_oracle_rows(m, w, plan, send, scales, d)
+    xin = moe.ffn_inputs(send, scales, w.payload == "fp8")
+    h_ref, y_ref = moe.expert_ffn(xin, plan["expert_offsets"], bits16(d["w_gate"]),
+                                  bits16(d["w_up"]), bits16(d["w_down"]))
+    S = plan["S"]
+    assert rel_max_err(bits16(m.h)[:S], h_ref) <= RTOL
+    assert rel_max_err(bits16(m.expert_out)[:S], y_ref) <= RTOL
+
+
+def sample_rows(plan, n_experts, n_random, seed):
+    off = plan["expert_offsets"]
+    E = off.size - 1
+    nonempty = [e for e in range(E) if off[e + 1] > off[e]]
+    g = np.random.default_rng(seed)
+    big = sorted(nonempty, key=lambda e: off[e] - off[e + 1])[:2]      # the largest experts
+    pick = set(big) | set(g.choice(nonempty, size=min(n_experts, len(nonempty)), replace=False))
+    rows = {}
+    for e in sorted(pick):
+        lo, hi = int(off[e]), int(off[e + 1])
+        r = {lo, hi - 1} | set(g.integers(lo, hi, size=n_random).tolist())
+        rows[e] = np.array(sorted(r))
+    return rows
+
+
+def oracle_rows(w, d, xin, rows_by_expert):
+    """Oracle FFN output for selected rows, expert by expert (weights copied per expert)."""
+    out = {}
+    for e, r in rows_by_expert.items():
+        wg, wu, wd = (bits16(d[n][e:e + 1]) for n in ("w_gate", "w_up", "w_down"))
+        h, y = moe.expert_ffn(xin[r], np.array([0, r.size]), wg, wu, wd)
+        out[e] = (h, y)
+    return out
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_ffn_parity_full_size_sampled(cuda, name):
+    w = mi.get(name)
+    d = mi.make_inputs(w, seed=0, device="cuda")
+    _, _, plan, send, scales = oracle_plan(w, d)
+    m, _ = shuffle_for(w)
+    run_gpu_ffn_on_oracle_rows(m, w, plan, send, scales, d)
+    rows = sample_rows(plan, n_experts=4, n_random=6, seed=1)
+    all_rows = np.concatenate(list(rows.values()))
+    xin = moe.ffn_inputs(send[all_rows], None if scales is None else scales[all_rows],
+                         w.payload == "fp8")
+    xin_full = np.zeros((plan["S"], w.H))
+    xin_full[all_rows] = xin
+    ref = oracle_rows(w, d, xin_full, rows)
+    h_gpu, y_gpu = bits16(m.h), bits16(m.expert_out)
+    for e, r in rows.items():
+        h_ref, y_ref = ref[e]
+        assert rel_max_err(h_gpu[r], h_ref) <= RTOL, e
+        assert rel_max_err(y_gpu[r], y_ref) <= RTOL, e
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_pipeline_end_to_end(cuda, name):
+    w = mi.get(name)
+    d = mi.make_inputs(w, seed=2, device="cuda")
+    m, cap = shuffle_for(w)
+    y = m.forward(d["logits"], d["x"], d["w_gate"], d["w_up"], d["w_down"])
+    assert m.status() == 0
+    o = moe.pipeline(np_(d["logits"]), bits16(d["x"]), bits16(d["w_gate"]), bits16(d["w_up"]),
+                     bits16(d["w_down"]), w.k, w.R, w.capacity_factor, w.payload == "fp8")
+    assert np.array_equal(np_(m.topk_idx), o["topk_idx"])
+    assert np.array_equal(np_(m.slot_row), o["slot_row"])
+    assert np.array_equal(np_(m.expert_offsets), o["expert_offsets"])
+    assert rel_max_err(bits16(m.expert_out)[:o["S"]], o["expert_out"]) <= RTOL
+    assert rel_max_err(bits16(y), o["y"]) <= RTOL
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_pipeline_full_size_sampled_tokens(cuda, name):
+    """The benchmark's launch configuration at full size; oracle on a token sample."""
+    w = mi.get(name)
+    d = mi.make_inputs(w, seed=0, device="cuda")
+    m, cap = shuffle_for(w)
+    y = m.forward(d["logits"], d["x"], d["w_gate"], d["w_up"], d["w_down"])
+    assert m.status() == 0
+    idx, wt, plan, send, scales = oracle_plan(w, d)
+    assert np.array_equal(np_(m.slot_row), plan["slot_row"])
+    g = np.random.default_rng(4)
+    toks = np.unique(np.concatenate([[0, w.T - 1], g.integers(0, w.T, size=6)]))
+    sr = plan["slot_row"][toks]
+    rows = sr[sr >= 0]
+    by_e = {}
+    off = plan["expert_offsets"]
+    for r in rows:
+        e = int(np.searchsorted(off, r, side="right") - 1)
+        by_e.setdefault(e, []).append(int(r))
+    by_e = {e: np.array(sorted(v)) for e, v in by_e.items()}
+    xin_full = np.zeros((plan["S"], w.H))
+    xin_full[rows] = moe.ffn_inputs(send[rows], None if scales is None else scales[rows],
+                                    w.payload == "fp8")
+    ref = oracle_rows(w, d, xin_full, by_e)
+    y_e = np.full((plan["S"], w.H), 0x7FC0, dtype=np.uint16)
+    for e, r in by_e.items():
+        y_e[r] = ref[e][1]
+    y_ref = moe.combine(y_e, sr, wt[toks], toks.size, w.H)
+    assert rel_max_err(bits16(y)[toks], y_ref) <= RTOL
