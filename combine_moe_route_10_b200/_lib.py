@@ -22,7 +22,8 @@ MOE_PAYLOAD_BF16 = 0
 MOE_PAYLOAD_FP8_E4M3_B128 = 1
 
 EXPORTS = ["moe_abi_version", "moe_status_string", "moe_capacity", "moe_route",
-           "moe_dispatch_workspace_size", "moe_dispatch", "moe_ffn_workspace_size",
+           "moe_dispatch_workspace_size", "moe_dispatch", "moe_dispatch_noalloc",
+           "moe_ffn_workspace_size",
            "moe_expert_ffn", "moe_combine", "moe_sync_status"]
 
 _lib = None
@@ -51,6 +52,7 @@ def load() -> ctypes.CDLL:
         "moe_route": (I, [P, I, I, I, I, P, P, P, P]),
         "moe_dispatch_workspace_size": (Z, [I, I, I]),
         "moe_dispatch": (I, [P, I, I, P, I, I, I, I, I, P, P, P, P, P, P, P, P, Z, P]),
+        "moe_dispatch_noalloc": (I, [P, I, I, P, I, I, I, I, I, P, P, P, P, P, P, P, P, P]),
         "moe_ffn_workspace_size": (Z, [I, I, I, I, I]),
         "moe_expert_ffn": (I, [P, P, I, P, I, I, I, I, P, P, P, P, P, Z, P]),
         "moe_combine": (I, [P, I, P, P, I, I, I, P, P]),
@@ -117,6 +119,18 @@ def moe_dispatch(x, T, H, topk_idx, k, E, R, capacity, payload, send, send_scale
                              _ptr(rank_offsets), _ptr(slot_row), _ptr(row_token), _ptr(ws),
                              ws_bytes, _stream(stream))
     return _check(st, "moe_dispatch", raise_on_error)
+
+
+def moe_dispatch_noalloc(x, T, H, topk_idx, k, E, R, capacity, payload, send, send_scales,
+                         expert_counts, expert_offsets, rank_offsets, slot_row, row_token,
+                         status=None, stream=None, raise_on_error=True):
+    """moe_dispatch without a workspace: for callers that cannot allocate device memory (the
+    library keeps a 1 MiB static device array for the scratch; see include/moe.h)."""
+    st = load().moe_dispatch_noalloc(_ptr(x), T, H, _ptr(topk_idx), k, E, R, capacity, payload,
+                                     _ptr(send), _ptr(send_scales), _ptr(expert_counts),
+                                     _ptr(expert_offsets), _ptr(rank_offsets), _ptr(slot_row),
+                                     _ptr(row_token), _ptr(status), _stream(stream))
+    return _check(st, "moe_dispatch_noalloc", raise_on_error)
 
 
 def moe_ffn_workspace_size(max_rows, E, H, F, payload) -> int:

@@ -338,4 +338,37 @@ cudaError_t launch_dispatch(const void* x, int T, int H, const int32_t* topk_idx
   return cudaGetLastError();
 }
 
+cudaError_t launch_dispatch_parts(const void* x, int T, int H, const int32_t* topk_idx, int k,
+                                  int E, int R, int capacity, int fp8, void* send,
+                                  float* send_scales, int32_t* expert_counts,
+                                  int32_t* expert_offsets, int32_t* rank_offsets,
+                                  int32_t* slot_row, int32_t* row_token, int* status,
+                                  unsigned* arrivals, int32_t* chunk_tab, cudaStream_t s) {
+  if (T == 0) {
+    cudaError_t e1 = cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * E, s);
+    if (e1 != cudaSuccess) return e1;
+    e1 = cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (E + 1), s);
+    if (e1 != cudaSuccess) return e1;
+    return cudaMemsetAsync(rank_offsets, 0, sizeof(int32_t) * (R + 1), s);
+  }
+  const int n_chunks = (T + kDispatchChunk - 1) / kDispatchChunk;
+  const int scan_n = E > 4 * kThreads ? E : 4 * kThreads;
+  count_scan_kernel<<<n_chunks, kThreads, sizeof(int) * scan_n, s>>>(
+      topk_idx, T, k, E, R, capacity, status, arrivals, chunk_tab, expert_counts, expert_offsets,
+      rank_offsets);
+  const size_t rank_smem = sizeof(int) * kWarps * E;
+  rank_kernel<<<n_chunks, kThreads, rank_smem, s>>>(topk_idx, T, k, E, capacity, chunk_tab,
+                                                    expert_offsets, slot_row, row_token);
+  const int grid = permute_grid(T);
+  if (fp8) {
+    permute_fp8_kernel<2><<<grid, kThreads, 0, s>>>(static_cast<const uint4*>(x), T, H, k,
+                                                    slot_row, static_cast<uint8_t*>(send),
+                                                    send_scales);
+  } else {
+    permute_bf16_kernel<8><<<grid, kThreads, 0, s>>>(static_cast<const uint4*>(x), T, H / 8, k,
+                                                     slot_row, static_cast<uint4*>(send));
+  }
+  return cudaGetLastError();
+}
+
 }  // namespace moe

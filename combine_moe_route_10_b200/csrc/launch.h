@@ -24,6 +24,15 @@ cudaError_t launch_dispatch(const void* x, int T, int H, const int32_t* topk_idx
                             int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_offsets,
                             int32_t* slot_row, int32_t* row_token, void* ws, cudaStream_t s);
 
+// The same three kernels with the scratch pieces given separately (status word, arrival counter,
+// chunk table); the arrival counter must be zero on entry.
+cudaError_t launch_dispatch_parts(const void* x, int T, int H, const int32_t* topk_idx, int k,
+                                  int E, int R, int capacity, int fp8, void* send,
+                                  float* send_scales, int32_t* expert_counts,
+                                  int32_t* expert_offsets, int32_t* rank_offsets,
+                                  int32_t* slot_row, int32_t* row_token, int* status,
+                                  unsigned* arrivals, int32_t* chunk_tab, cudaStream_t s);
+
 cudaError_t launch_combine(const void* expert_out, int max_rows, const int32_t* slot_row,
                            const float* topk_w, int T, int k, int H, void* y, cudaStream_t s);
 

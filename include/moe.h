@@ -128,6 +128,35 @@ moe_status_t moe_dispatch(const void* x, int T, int H, const int32_t* topk_idx, 
                           int32_t* rank_offsets, int32_t* slot_row, int32_t* row_token, void* ws,
                           size_t ws_bytes, moe_stream_t stream);
 
+/*
+ * moe_dispatch_noalloc: moe_dispatch for callers that cannot allocate.  The pages have no
+ * counterpart; this is a convenience of this library.
+ *
+ * Some callers cannot hand the library a workspace: programs that route every device allocation
+ * through their own pool and forbid others, plug-ins inside such programs, and latency-critical
+ * code that must not call cudaMalloc (it can synchronise the whole device).  This entry point takes
+ * the same inputs and outputs as moe_dispatch, without ws / ws_bytes, and calls no cudaMalloc,
+ * cudaFree or allocating library routine.  Its scratch is a static device array of
+ * MOE_DISPATCH_NOALLOC_SCRATCH_BYTES (1 MiB) inside the library, which every GPU that loads the
+ * library holds until the process exits.
+ *   status  optional (may be NULL) device int32 owned by the caller, zeroed by the caller: device
+ *           findings are OR-ed into it (1 = expert id out of range); moe_sync_status(status, s)
+ *           reads and clears it like a workspace status word.
+ * Limits: those of moe_dispatch, plus 256 + ceil(T/256) * E * 4 <= 1 MiB (e.g. T <= 65280 tokens at
+ * E = 1024, T <= 522240 at E = 128); larger shapes return MOE_ERR_WORKSPACE without launching.
+ * The first call on each device looks up the array's device address (cudaGetSymbolAddress with
+ * that device current); make that first call before any stream capture.  All calls share the one
+ * array: calls that overlap on the GPU (different streams, or the same array from several host
+ * threads without ordering) race and give wrong results; order them on one stream.
+ */
+#define MOE_DISPATCH_NOALLOC_SCRATCH_BYTES (1u << 20)
+moe_status_t moe_dispatch_noalloc(const void* x, int T, int H, const int32_t* topk_idx, int k,
+                                  int E, int R, int capacity, moe_payload_t payload, void* send,
+                                  float* send_scales, int32_t* expert_counts,
+                                  int32_t* expert_offsets, int32_t* rank_offsets,
+                                  int32_t* slot_row, int32_t* row_token, int32_t* status,
+                                  moe_stream_t stream);
+
 /* Bytes of scratch moe_expert_ffn needs (status word, the bf16 intermediate h [max_rows, F] and,
  * for the FP8 payload, the dequantised bf16 input rows [max_rows, H]). */
 size_t moe_ffn_workspace_size(int max_rows, int E, int H, int F, moe_payload_t payload);
