@@ -13,7 +13,6 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kMaxSlotsInFlight = 8;  // rows whose vectors are loaded together per step
 
 __device__ __forceinline__ void accumulate(float acc[8], float w, uint4 v) {
   const uint32_t words[4] = {v.x, v.y, v.z, v.w};
@@ -24,13 +23,17 @@ __device__ __forceinline__ void accumulate(float acc[8], float w, uint4 v) {
   }
 }
 
-template <int UNROLL>
+// KS rows are gathered together per step (loads issued before any accumulation); UNROLL vectors
+// per lane per row.
+template <int KS, int UNROLL>
 __global__ void __launch_bounds__(kThreads)
     combine_kernel(const uint4* __restrict__ expert_out, int max_rows,
                    const int32_t* __restrict__ slot_row, const float* __restrict__ topk_w, int T,
                    int k, int nvec, uint4* __restrict__ y) {
   const int lane = threadIdx.x & 31;
   const int nwarps = gridDim.x * kWarps;
+  griddep_wait();
+  griddep_launch_dependents();
   for (int t = blockIdx.x * kWarps + (threadIdx.x >> 5); t < T; t += nwarps) {
     int my_row = -1;
     float my_w = 0.0f;
@@ -47,13 +50,13 @@ __global__ void __launch_bounds__(kThreads)
       for (int u = 0; u < UNROLL; ++u)
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[u][i] = 0.0f;
-      // slots in ascending j, kMaxSlotsInFlight rows loaded before they are accumulated
+      // slots in ascending j, KS rows loaded before they are accumulated
       for (unsigned m = live; m != 0;) {
-        int rows[kMaxSlotsInFlight];
-        float ws[kMaxSlotsInFlight];
+        int rows[KS];
+        float ws[KS];
         int n = 0;
 #pragma unroll
-        for (int q = 0; q < kMaxSlotsInFlight; ++q) {
+        for (int q = 0; q < KS; ++q) {
           rows[q] = -1;
           ws[q] = 0.0f;
           if (m != 0) {
@@ -63,9 +66,9 @@ __global__ void __launch_bounds__(kThreads)
             n = q + 1;
           }
         }
-        uint4 vals[kMaxSlotsInFlight][UNROLL];
+        uint4 vals[KS][UNROLL];
 #pragma unroll
-        for (int q = 0; q < kMaxSlotsInFlight; ++q) {
+        for (int q = 0; q < KS; ++q) {
           if (q < n) {
             const int j = rows[q];
             const int row = __shfl_sync(0xFFFFFFFFu, my_row, j);
@@ -79,7 +82,7 @@ __global__ void __launch_bounds__(kThreads)
           }
         }
 #pragma unroll
-        for (int q = 0; q < kMaxSlotsInFlight; ++q) {
+        for (int q = 0; q < KS; ++q) {
           if (q < n) {
 #pragma unroll
             for (int u = 0; u < UNROLL; ++u) {
@@ -113,9 +116,14 @@ cudaError_t launch_combine(const void* expert_out, int max_rows, const int32_t* 
   int blocks = (T + kWarps - 1) / kWarps;
   const int cap = num_sms() * 8;
   if (blocks > cap) blocks = cap;
-  combine_kernel<2><<<blocks, kThreads, 0, s>>>(static_cast<const uint4*>(expert_out), max_rows,
-                                                slot_row, topk_w, T, k, H / 8,
-                                                static_cast<uint4*>(y));
+  const uint4* eo = static_cast<const uint4*>(expert_out);
+  uint4* yo = static_cast<uint4*>(y);
+  // rows gathered together sized to k: enough loads in flight, few registers (high occupancy)
+  void (*kern)(const uint4*, int, const int32_t*, const float*, int, int, int, uint4*) =
+      k <= 2 ? combine_kernel<2, 4> : (k <= 4 ? combine_kernel<4, 2> : combine_kernel<8, 1>);
+  const cudaError_t err = launch_pdl(kern, dim3(blocks), dim3(kThreads), 0, s, eo, max_rows,
+                                     slot_row, topk_w, T, k, H / 8, yo);
+  if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 

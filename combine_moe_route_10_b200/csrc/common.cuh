@@ -27,6 +27,17 @@ __device__ __forceinline__ void record_status(int* status, int bit) {
   if (status != nullptr) atomicOr(status, bit);
 }
 
+// Programmatic dependent launch: every kernel of the path is launched with programmatic stream
+// serialisation, so its launch and pre-wait prologue overlap the previous kernel's tail.  Each
+// kernel calls griddep_wait() before its first global-memory access (read or write), which returns
+// once the previous grid has completed and its memory is visible: stream-order semantics are kept.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
   uint4 v;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"

@@ -92,7 +92,7 @@ extern "C" moe_status_t moe_dispatch_noalloc(const void* x, int T, int H, const 
   const cudaError_t err = moe::launch_dispatch_parts(
       x, T, H, topk_idx, k, E, R, capacity, fp8 ? 1 : 0, send, send_scales, expert_counts,
       expert_offsets, rank_offsets, slot_row, row_token, reinterpret_cast<int*>(status), arrivals,
-      chunk_tab, s);
+      chunk_tab, /*pdl_first=*/false, s);  // the memset above precedes it: ordinary launch
   if (err != cudaSuccess) {
     cudaGetLastError();
     return MOE_ERR_CUDA;

@@ -42,6 +42,15 @@ constexpr int kATileBytes = BM * BK * 2;   // 16 KB
 constexpr int kBTileBytes = 256 * BK * 2;  // 32 KB
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
 
+// Experts with at least this many 128-row blocks are "hot" (their weight blocks are reused from L2
+// by several row blocks, so their tiles are tensor-bound); their tiles are interleaved evenly with
+// the other experts' tiles, which stream weights from HBM, so both kinds run at the same time.
+// 0 disables the interleave (plain expert order).
+#ifndef MOE_FFN_HOT_MTILES
+#define MOE_FFN_HOT_MTILES 2
+#endif
+constexpr int kGemm2NTile = 256;  // output columns per GEMM-2 tile (128 measured slower)
+
 enum Mode { kSwiGLU = 0, kPlain = 1 };
 
 struct GemmArgs {
@@ -158,8 +167,10 @@ struct Smem {
   uint32_t* tmem_base;
   int* abort_flag;
   int* off;               // [E+1] row offsets (clamped to max_rows)
-  int* tstart;            // [E+1] first tile of each expert; tstart[E] = total tiles
+  int* tstart;            // [E+1] first tile of each non-hot expert among non-hot tiles
+  int* hstart;            // [E+1] first tile of each hot expert among hot tiles
   int* mtiles;            // [E]
+  int* totals;            // [2]: non-hot tiles, hot tiles
 };
 
 __device__ __forceinline__ Smem carve(uint8_t* raw, int E) {
@@ -177,13 +188,15 @@ __device__ __forceinline__ Smem carve(uint8_t* raw, int E) {
   s.abort_flag = reinterpret_cast<int*>(s.tmem_base + 1);
   s.off = s.abort_flag + 2;
   s.tstart = s.off + (E + 1);
-  s.mtiles = s.tstart + (E + 1);
+  s.hstart = s.tstart + (E + 1);
+  s.mtiles = s.hstart + (E + 1);
+  s.totals = s.mtiles + E;
   return s;
 }
 
 size_t gemm_smem_bytes(int E) {
   return 1024 + static_cast<size_t>(kStages) * kStageBytes + 8 * (2 * kStages + 5) + 16 +
-         sizeof(int) * (3 * static_cast<size_t>(E) + 2);
+         sizeof(int) * (4 * static_cast<size_t>(E) + 5);
 }
 
 // Bounded wait on an mbarrier phase.  Returns false if the CTA is aborting or the limit ran out.
@@ -202,16 +215,41 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volati
   }
 }
 
+__device__ __forceinline__ int owner_of(const int* start, int E, int idx) {
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {  // largest expert whose first tile is <= idx (it owns the tile)
+    const int mid = (lo + hi + 1) >> 1;
+    if (start[mid] <= idx) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Tile -> (expert, row block, column block).  Row blocks are the fastest index inside an expert.
+// With hot experts present, tile t is hot iff floor((t+1)*Hn/N) > floor(t*Hn/N) (an even spread of
+// the Hn hot tiles over all N tiles), and indexes its own list.
 __device__ __forceinline__ void decode_tile(const Smem& s, int E, int tile, int& e, int& m_blk,
                                             int& n_blk) {
-  int lo = 0, hi = E - 1;
-  while (lo < hi) {  // largest expert whose first tile is <= tile (it owns the tile)
-    const int mid = (lo + hi + 1) >> 1;
-    if (s.tstart[mid] <= tile) lo = mid; else hi = mid - 1;
+  const int n_cold = s.totals[0], n_hot = s.totals[1];
+  const int* start = s.tstart;
+  int idx = tile;
+  if (n_hot > 0) {
+    if (n_cold == 0) {
+      start = s.hstart;
+    } else {
+      const long long N = static_cast<long long>(n_cold) + n_hot;
+      const long long h0 = static_cast<long long>(tile) * n_hot / N;
+      const long long h1 = static_cast<long long>(tile + 1) * n_hot / N;
+      if (h1 > h0) {
+        start = s.hstart;
+        idx = static_cast<int>(h0);
+      } else {
+        idx = tile - static_cast<int>(h0);
+      }
+    }
   }
-  e = lo;
-  const int local = tile - s.tstart[lo];
-  const int mt = s.mtiles[lo];
+  e = owner_of(start, E, idx);
+  const int local = idx - start[e];
+  const int mt = s.mtiles[e];
   n_blk = local / mt;
   m_blk = local - n_blk * mt;
 }
@@ -260,8 +298,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   } else if (warp == 2) {
-    // schedule: per-expert row offsets, row-block counts and the first tile of each expert
-    int carry = 0;
+    griddep_wait();
+    // schedule: per-expert row offsets, row-block counts, and the first tile of each expert in
+    // its list (non-hot or hot)
+    int carry_c = 0, carry_h = 0;
     for (int e0 = 0; e0 < E; e0 += 32) {
       const int e = e0 + lane;
       int lo = 0, hi = 0;
@@ -271,30 +311,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const int rows = max(hi - lo, 0);
       const int mt = (rows + BM - 1) / BM;
-      const int tiles = mt * n_tiles;
-      int incl = tiles;
+      const bool hot = MOE_FFN_HOT_MTILES > 0 && mt >= MOE_FFN_HOT_MTILES;
+      const int tiles_c = hot ? 0 : mt * n_tiles;
+      const int tiles_h = hot ? mt * n_tiles : 0;
+      int inc_c = tiles_c, inc_h = tiles_h;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-        if (lane >= o) incl += y;
+        const int yc = __shfl_up_sync(0xFFFFFFFFu, inc_c, o);
+        const int yh = __shfl_up_sync(0xFFFFFFFFu, inc_h, o);
+        if (lane >= o) {
+          inc_c += yc;
+          inc_h += yh;
+        }
       }
       if (e < E) {
         s.off[e] = lo;
         s.mtiles[e] = mt;
-        s.tstart[e] = carry + incl - tiles;
+        s.tstart[e] = carry_c + inc_c - tiles_c;
+        s.hstart[e] = carry_h + inc_h - tiles_h;
       }
-      carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+      carry_c += __shfl_sync(0xFFFFFFFFu, inc_c, 31);
+      carry_h += __shfl_sync(0xFFFFFFFFu, inc_h, 31);
     }
     if (lane == 0) {
-      s.tstart[E] = carry;
+      s.tstart[E] = carry_c;
+      s.hstart[E] = carry_h;
+      s.totals[0] = carry_c;
+      s.totals[1] = carry_h;
       s.off[E] = min(__ldg(args.expert_offsets + E), args.max_rows);
     }
   }
+  griddep_wait();  // every thread: the previous grid's outputs are visible from here on
+  griddep_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s.tmem_base;
-  const int total_tiles = s.tstart[E];
+  const int total_tiles = s.totals[0] + s.totals[1];
   const uint32_t tiles_base = smem_addr(s.tiles);
 
   if (warp == 0) {
@@ -470,6 +523,8 @@ __global__ void __launch_bounds__(256)
     dequant_fp8_kernel(const uint8_t* __restrict__ q, const float* __restrict__ scales,
                        const int32_t* __restrict__ total_rows, int max_rows, int H,
                        uint4* __restrict__ out) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int S = min(__ldg(total_rows), max_rows);
   const int per_row = H / 16;  // 16 codes per thread step
   const long long n = static_cast<long long>(S) * per_row;
@@ -534,7 +589,9 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUten
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  grouped_gemm_kernel<MODE><<<num_sms(), kThreads, smem, s>>>(a, b0, b1, args);
+  err = launch_pdl(grouped_gemm_kernel<MODE>, dim3(num_sms()), dim3(kThreads), smem, s, a, b0, b1,
+                   args);
+  if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 
@@ -562,12 +619,14 @@ cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp
     long long blocks = (work + 255) / 256;
     const long long cap = static_cast<long long>(num_sms()) * 8;
     if (blocks > cap) blocks = cap;
-    dequant_fp8_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(
-        static_cast<const uint8_t*>(send), send_scales, expert_offsets + E, max_rows, H, xdq);
+    const cudaError_t e0 = launch_pdl(dequant_fp8_kernel, dim3(static_cast<int>(blocks)), dim3(256),
+                                      0, s, static_cast<const uint8_t*>(send), send_scales,
+                                      expert_offsets + E, max_rows, H, xdq);
+    if (e0 != cudaSuccess) return e0;
     a_src = xdq;
   }
   CUtensorMap tm_x, tm_g, tm_u, tm_h, tm_d;
-  const int n_tile2 = 256;
+  const int n_tile2 = kGemm2NTile;
   if (!make_tmap(&tm_x, a_src, max_rows, H, BM) ||
       !make_tmap(&tm_g, w_gate, static_cast<uint64_t>(E) * F, H, 128) ||
       !make_tmap(&tm_u, w_up, static_cast<uint64_t>(E) * F, H, 128) ||

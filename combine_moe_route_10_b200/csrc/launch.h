@@ -5,9 +5,41 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
+#ifndef MOE_USE_PDL
+#define MOE_USE_PDL 1
+#endif
+
 namespace moe {
 
 int num_sms();  // SM count of the current device (cached per device)
+
+// Launch with programmatic stream serialisation (see griddep_wait in common.cuh).  pdl = false
+// gives an ordinary launch; it is used when the previous operation on the stream is not a kernel
+// (a memset), so that ordering never depends on how programmatic serialisation treats it.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl_if(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = (pdl && MOE_USE_PDL) ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args&&... args) {
+  return launch_pdl_if(true, kernel, grid, block, smem, s, std::forward<Args>(args)...);
+}
+  // SM count of the current device (cached per device)
 
 cudaError_t launch_route(const float* logits, int T, int E, int k, int renorm, int32_t* topk_idx,
                          float* topk_w, int32_t* routed, cudaStream_t s);
@@ -16,7 +48,8 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int renorm, i
 //   [0, 4)    status word (kStatus* bits)
 //   [4, 8)    arrival counter of the count/scan kernel (returns to 0 after every call)
 //   [256, ..) per-chunk expert histogram, then per-chunk base positions [n_chunks][E] int32
-constexpr int kDispatchChunk = 256;  // tokens per counting / ranking chunk
+constexpr int kDispatchChunk = 256;  // tokens per counting chunk
+constexpr int kDispatchTileMax = 16; // max tokens per rank+permute CTA (divides kDispatchChunk)
 size_t dispatch_workspace_bytes(int T, int E);
 
 cudaError_t launch_dispatch(const void* x, int T, int H, const int32_t* topk_idx, int k, int E,
@@ -31,7 +64,8 @@ cudaError_t launch_dispatch_parts(const void* x, int T, int H, const int32_t* to
                                   float* send_scales, int32_t* expert_counts,
                                   int32_t* expert_offsets, int32_t* rank_offsets,
                                   int32_t* slot_row, int32_t* row_token, int* status,
-                                  unsigned* arrivals, int32_t* chunk_tab, cudaStream_t s);
+                                  unsigned* arrivals, int32_t* chunk_tab, bool pdl_first,
+                                  cudaStream_t s);
 
 cudaError_t launch_combine(const void* expert_out, int max_rows, const int32_t* slot_row,
                            const float* topk_w, int T, int k, int H, void* y, cudaStream_t s);

@@ -38,6 +38,8 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
                                                     int32_t* __restrict__ routed) {
   extern __shared__ int s_hist[];
   for (int i = threadIdx.x; i < E; i += blockDim.x) s_hist[i] = 0;
+  griddep_wait();
+  griddep_launch_dependents();
   __syncthreads();
 
   const int lane = threadIdx.x & 31;
@@ -145,10 +147,12 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int renorm, i
   const int max_blocks = num_sms() * 8;
   if (blocks > max_blocks) blocks = max_blocks;
   const size_t smem = sizeof(int) * E;
-#define MOE_ROUTE_CASE(VPL)                                                                    \
-  route_kernel<VPL><<<blocks, kThreads, smem, s>>>(logits, T, E, k, renorm, topk_idx, topk_w, \
-                                                   routed);                                   \
+  const bool pdl = routed == nullptr;  // after the histogram memset: ordinary launch
+#define MOE_ROUTE_CASE(VPL)                                                                 \
+  err = launch_pdl_if(pdl, route_kernel<VPL>, dim3(blocks), dim3(kThreads), smem, s, logits, T, \
+                      E, k, renorm, topk_idx, topk_w, routed);                                 \
   break;
+  cudaError_t err = cudaSuccess;
   switch ((E + 31) / 32) {
     case 1: MOE_ROUTE_CASE(1)
     case 2: MOE_ROUTE_CASE(2)
@@ -160,6 +164,7 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int renorm, i
     case 16: MOE_ROUTE_CASE(16)
     default: MOE_ROUTE_CASE(32)
   }
+  if (err != cudaSuccess) return err;
 #undef MOE_ROUTE_CASE
   return cudaGetLastError();
 }
