@@ -80,9 +80,8 @@ moe_status_t moe_route(const float* logits, int T, int E, int k, int renormalize
 }
 
 size_t moe_dispatch_workspace_size(int T, int E, int k) {
-  (void)k;
-  if (T < 0 || E < 1) return 0;
-  return moe::dispatch_workspace_bytes(T, E);
+  if (T < 0 || E < 1 || k < 1) return 0;
+  return moe::dispatch_workspace_bytes(T, E, k);
 }
 
 moe_status_t moe_dispatch(const void* x, int T, int H, const int32_t* topk_idx, int k, int E,
@@ -107,7 +106,7 @@ moe_status_t moe_dispatch(const void* x, int T, int H, const int32_t* topk_idx, 
     return MOE_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(send, 16) || !aligned(send_scales, 4) || !aligned(topk_idx, 4))
     return MOE_ERR_INVALID_ARG;
-  if (!aligned(ws, 256) || ws_bytes < moe::dispatch_workspace_bytes(T, E)) return MOE_ERR_WORKSPACE;
+  if (!aligned(ws, 256) || ws_bytes < moe::dispatch_workspace_bytes(T, E, k)) return MOE_ERR_WORKSPACE;
   return from_cuda(moe::launch_dispatch(x, T, H, topk_idx, k, E, R, capacity, fp8 ? 1 : 0, send,
                                         send_scales, expert_counts, expert_offsets, rank_offsets,
                                         slot_row, row_token, ws,

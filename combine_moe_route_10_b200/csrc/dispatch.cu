@@ -7,16 +7,18 @@
 // expert range, so the buffer is rank-major too and a rank's slice is given by rank_offsets (the
 // ThunderEP page's section 2.2: each rank keeps only its own slice of the routing table).
 //
-// Two kernels, no host synchronisation, no order-dependent atomics in any result:
-//   1. count_scan: one CTA per 256-token chunk builds the chunk's expert histogram; the last CTA to
-//      arrive turns the [chunk][expert] table into per-chunk base positions and writes the kept
-//      counts (capacity applied), the expert offsets and the rank offsets.
-//   2. rank_permute: one CTA per 16 tokens gives each of its slots its position inside its expert,
-//      in token order (recount of the chunk's earlier slots, then warp-synchronous __match_any
-//      ranking), writes slot_row and row_token (slots at positions >= capacity are dropped: -1),
-//      then one warp per token reads the row once with 16-byte loads and writes it to each of its
-//      kept rows (bf16), or quantises it per 128-element block to e4m3 with an fp32 scale and
-//      writes codes and scales to each kept row (FP8).
+// Two kernels, no host synchronisation, no order-dependent atomics in any result.  Slots are cut
+// into chunks of C tokens (about 2048 slots per chunk).
+//   1. count: one CTA per chunk writes the chunk's expert histogram hist[chunk][E].
+//   2. rank_permute: one CTA per `tile` tokens.  Before waiting for the count kernel (inputs only):
+//      L2 prefetch of its token rows, the per-expert count of the chunk's slots before its first
+//      token, and the warp-synchronous (__match_any) ranking of its own slots, giving each slot its
+//      position relative to the chunk start.  After the wait: from hist, every CTA derives its
+//      chunk's base position per expert and the expert totals, applies the capacity, scans the kept
+//      counts into expert offsets (CTA 0 also writes counts / offsets / rank offsets), turns
+//      positions into rows (position >= capacity: dropped, -1), writes slot_row / row_token, and
+//      copies the rows (bf16) or quantises them per 128-element block to e4m3 with an fp32 scale
+//      (FP8), one warp (or a segment of a row per warp) per token.
 #include <cuda_fp8.h>
 
 #include "common.cuh"
@@ -27,6 +29,11 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+
+// Add 1 to hist[e] for a valid expert id (shared-memory atomics: counts are order-independent).
+__device__ __forceinline__ void hist_add(int* hist, int e, bool ok) {
+  if (ok) atomicAdd(&hist[e], 1);
+}
 
 // Exclusive scan of n <= 4*kThreads ints in shared memory; returns the total.  All threads call.
 __device__ int block_exclusive_scan(int* data, int n, int* warp_tot) {
@@ -69,61 +76,6 @@ __device__ int block_exclusive_scan(int* data, int n, int* warp_tot) {
   return total;
 }
 
-__global__ void __launch_bounds__(kThreads)
-    count_scan_kernel(const int32_t* __restrict__ topk_idx, int T, int k, int E, int R, int cap,
-                      int* status, unsigned* arrivals, int32_t* chunk_tab,
-                      int32_t* __restrict__ expert_counts, int32_t* __restrict__ expert_offsets,
-                      int32_t* __restrict__ rank_offsets) {
-  extern __shared__ int s_hist[];  // E (+ padding to 4*kThreads for the scan)
-  __shared__ int s_warp_tot[kWarps + 1];
-  __shared__ bool s_last;
-  const int tid = threadIdx.x;
-  const int c = blockIdx.x;
-  for (int e = tid; e < E; e += kThreads) s_hist[e] = 0;
-  griddep_wait();
-  __syncthreads();
-  const long long s0 = static_cast<long long>(c) * kDispatchChunk * k;
-  const long long s1 = static_cast<long long>(min(T, (c + 1) * kDispatchChunk)) * k;
-  bool bad = false;
-  for (long long s = s0 + tid; s < s1; s += kThreads) {
-    const int e = __ldg(topk_idx + s);
-    if (static_cast<unsigned>(e) < static_cast<unsigned>(E))
-      atomicAdd(&s_hist[e], 1);
-    else
-      bad = true;
-  }
-  if (__syncthreads_or(bad) && tid == 0) record_status(status, kStatusInvalidTopk);
-  for (int e = tid; e < E; e += kThreads) chunk_tab[static_cast<size_t>(c) * E + e] = s_hist[e];
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(arrivals, 1u) == gridDim.x - 1);
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-
-  // Last CTA: per-chunk base positions (exclusive over chunks, in place) and expert totals.
-  const int n_chunks = gridDim.x;
-  for (int e = tid; e < E; e += kThreads) {
-    int run = 0;
-    for (int cc = 0; cc < n_chunks; ++cc) {
-      int32_t* p = chunk_tab + static_cast<size_t>(cc) * E + e;
-      const int v = __ldcg(p);
-      *p = run;
-      run += v;
-    }
-    const int kept = cap > 0 ? min(run, cap) : run;
-    expert_counts[e] = kept;
-    s_hist[e] = kept;
-  }
-  __syncthreads();
-  const int total = block_exclusive_scan(s_hist, E, s_warp_tot);
-  for (int e = tid; e < E; e += kThreads) expert_offsets[e] = s_hist[e];
-  if (tid == 0) expert_offsets[E] = total;
-  const int per_rank = E / R;
-  for (int r = tid; r <= R; r += kThreads) rank_offsets[r] = (r == R) ? total : s_hist[r * per_rank];
-  if (tid == 0) *arrivals = 0u;  // every CTA has arrived: ready for the next call
-}
-
 // bf16 payload of one token: the warp reads the row once (UNROLL 16-byte vectors in flight per
 // lane) and writes it to each kept row.
 template <int UNROLL>
@@ -144,7 +96,7 @@ __device__ __forceinline__ void copy_token_bf16(const uint4* __restrict__ src, i
 #pragma unroll
       for (int u = 0; u < UNROLL; ++u) {
         const int v = v0 + u * 32 + lane;
-        if (v < vend) st_v4(dst + v, buf[u]);
+        if (v < vend) st_cs_v4(dst + v, buf[u]);  // streaming: evict-first in L2
       }
     }
   }
@@ -213,39 +165,61 @@ __device__ __forceinline__ void quant_token_fp8(const uint4* __restrict__ src, i
   }
 }
 
-// Rank + permute, one CTA per `tile` tokens (a power of two <= 16 that divides the 256-token chunk).  A slot's position inside its expert is
-// chunk_base[chunk][e] (slots of expert e in earlier chunks) + the slots of e earlier in this chunk:
-// the CTA recounts the chunk's slots before its first token, then ranks its own slots in token order
-// (warp-synchronous __match_any), writes slot_row / row_token, and copies or quantises its tokens
-// (one warp per token, or 8/tile warps per token, each taking a segment of the row).  Slots at
-// positions >= capacity are dropped (-1).  Before waiting for count_scan the CTA asks L2 to
-// prefetch its token rows: x was produced before count_scan started, and this kernel is launched
-// only after every count_scan CTA has exited (count_scan never triggers its dependents early).
+__global__ void __launch_bounds__(kThreads)
+    count_kernel(const int32_t* __restrict__ topk_idx, int T, int k, int E, int chunk_tokens,
+                 int* status, int32_t* __restrict__ hist) {
+  extern __shared__ int s_hist[];
+  const int tid = threadIdx.x;
+  const int c = blockIdx.x;
+  for (int e = tid; e < E; e += kThreads) s_hist[e] = 0;
+  griddep_wait();
+  // rank_permute may start now: its pre-wait phase reads only the dispatch inputs, which are
+  // complete once every CTA of this grid has passed the wait above
+  griddep_launch_dependents();
+  __syncthreads();
+  const long long s0 = static_cast<long long>(c) * chunk_tokens * k;
+  const long long s1 = static_cast<long long>(min(T, (c + 1) * chunk_tokens)) * k;
+  bool bad = false;
+  for (long long s = s0 + tid; s < s1; s += kThreads) {
+    const int e = __ldg(topk_idx + s);
+    const bool ok = static_cast<unsigned>(e) < static_cast<unsigned>(E);
+    hist_add(s_hist, e, ok);
+    bad |= !ok;
+  }
+  if (__syncthreads_or(bad) && tid == 0) record_status(status, kStatusInvalidTopk);
+  for (int e = tid; e < E; e += kThreads) hist[static_cast<size_t>(c) * E + e] = s_hist[e];
+}
+
 template <bool FP8, int UNROLL>
 __global__ void __launch_bounds__(kThreads)
-    rank_permute_kernel(const int32_t* __restrict__ topk_idx, int T, int k, int E, int cap,
-                        const int32_t* __restrict__ chunk_base,
-                        const int32_t* __restrict__ expert_offsets, int32_t* __restrict__ slot_row,
+    rank_permute_kernel(const int32_t* __restrict__ topk_idx, int T, int k, int E, int R, int cap,
+                        int chunk_tokens, int n_chunks, const int32_t* __restrict__ hist,
+                        int32_t* __restrict__ expert_counts, int32_t* __restrict__ expert_offsets,
+                        int32_t* __restrict__ rank_offsets, int32_t* __restrict__ slot_row,
                         int32_t* __restrict__ row_token, const uint4* __restrict__ x, int H,
                         int tile, void* __restrict__ send, float* __restrict__ send_scales) {
   extern __shared__ int s_mem[];
-  int* cnt = s_mem;           // [E] running position per expert
-  int* s_rows = s_mem + E;    // [tile * k] rows of this CTA's slots
+  int* cnt = s_mem;               // [E] relative positions, then chunk base + relative count
+  int* s_off = cnt + E;           // [max(E, 4*kThreads)] kept counts, scanned into offsets
+  int* s_rel = s_off + max(E, 4 * kThreads);  // [tile*k] relative position (or -1) per slot
+  int* s_exp = s_rel + tile * k;  // [tile*k] expert per slot
+  __shared__ int s_warp_tot[kWarps + 1];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t0 = blockIdx.x * tile;
   const int t1 = min(T, t0 + tile);
-  const int c = t0 / kDispatchChunk;
+  const int c = t0 / chunk_tokens;
+
+  // ---- before the wait: inputs only ---------------------------------------------------------------
   if (tid < t1 - t0) {
     const char* row = reinterpret_cast<const char*>(x) + static_cast<size_t>(t0 + tid) * H * 2;
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(row), "r"(H * 2) : "memory");
   }
-  griddep_wait();
-  for (int e = tid; e < E; e += kThreads) cnt[e] = __ldg(chunk_base + static_cast<size_t>(c) * E + e);
+  for (int e = tid; e < E; e += kThreads) cnt[e] = 0;
   __syncthreads();
   const long long p1 = static_cast<long long>(t0) * k;
-  for (long long s = static_cast<long long>(c) * kDispatchChunk * k + tid; s < p1; s += kThreads) {
+  for (long long s = static_cast<long long>(c) * chunk_tokens * k + tid; s < p1; s += kThreads) {
     const int e = __ldg(topk_idx + s);
-    if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) atomicAdd(&cnt[e], 1);
+    hist_add(cnt, e, static_cast<unsigned>(e) < static_cast<unsigned>(E));
   }
   __syncthreads();
   if (warp == 0) {
@@ -258,23 +232,60 @@ __global__ void __launch_bounds__(kThreads)
       const bool ok = valid && static_cast<unsigned>(e) < static_cast<unsigned>(E);
       const int key = ok ? e : E + lane;  // unique key for lanes without a slot
       const unsigned peers = __match_any_sync(0xFFFFFFFFu, key);
-      int pos = 0;
-      if (ok) pos = cnt[e] + __popc(peers & lt_mask);
+      int rel = -1;
+      if (ok) rel = cnt[e] + __popc(peers & lt_mask);
       __syncwarp();
       if (ok && lane == __ffs(peers) - 1) cnt[e] += __popc(peers);
       __syncwarp();
       if (valid) {
-        int row = -1;
-        if (ok && (cap == 0 || pos < cap)) {
-          row = __ldg(expert_offsets + e) + pos;
-          row_token[row] = static_cast<int32_t>(s / k);
-        }
-        slot_row[s] = row;
-        s_rows[s - p1] = row;
+        s_rel[s - p1] = rel;
+        s_exp[s - p1] = ok ? e : -1;
       }
     }
   }
+
+  // ---- after the wait: the histogram is complete ---------------------------------------------------
+  griddep_wait();
+  griddep_launch_dependents();
   __syncthreads();
+  for (int e = tid; e < E; e += kThreads) {
+    int before = 0, total = 0;
+#pragma unroll 8
+    for (int cc = 0; cc < n_chunks; ++cc) {
+      const int v = __ldcg(hist + static_cast<size_t>(cc) * E + e);
+      total += v;
+      before += cc < c ? v : 0;
+    }
+    cnt[e] = before;                                // positions of expert e before this chunk
+    s_off[e] = cap > 0 ? min(total, cap) : total;   // kept rows of expert e
+  }
+  __syncthreads();
+  if (blockIdx.x == 0)
+    for (int e = tid; e < E; e += kThreads) expert_counts[e] = s_off[e];
+  const int total_kept = block_exclusive_scan(s_off, E, s_warp_tot);
+  if (blockIdx.x == 0) {
+    for (int e = tid; e < E; e += kThreads) expert_offsets[e] = s_off[e];
+    if (tid == 0) expert_offsets[E] = total_kept;
+    const int per_rank = E / R;
+    for (int r = tid; r <= R; r += kThreads)
+      rank_offsets[r] = (r == R) ? total_kept : s_off[r * per_rank];
+  }
+  const int n_slots = (t1 - t0) * k;
+  for (int i = tid; i < n_slots; i += kThreads) {
+    const int e = s_exp[i];
+    int row = -1;
+    if (e >= 0) {
+      const int pos = cnt[e] + s_rel[i];
+      if (cap == 0 || pos < cap) {
+        row = s_off[e] + pos;
+        row_token[row] = t0 + i / k;
+      }
+    }
+    slot_row[p1 + i] = row;
+    s_rel[i] = row;
+  }
+  __syncthreads();
+
   // warps per token: 1 when tile >= 8, else 8/tile warps split the row into segments
   const int wpt = tile >= kWarps ? 1 : kWarps / tile;
   const int seg = warp % wpt;
@@ -282,7 +293,7 @@ __global__ void __launch_bounds__(kThreads)
   const int per = ((units + wpt - 1) / wpt + (FP8 ? 1 : 31)) / (FP8 ? 2 : 32) * (FP8 ? 2 : 32);
   const int ubeg = min(units, seg * per), uend = min(units, ubeg + per);
   for (int t = t0 + warp / wpt; t < t1; t += kWarps / wpt) {
-    const int my_row = lane < k ? s_rows[(t - t0) * k + lane] : -1;
+    const int my_row = lane < k ? s_rel[(t - t0) * k + lane] : -1;
     if (FP8)
       quant_token_fp8<UNROLL>(x + static_cast<size_t>(t) * (H / 8), H, ubeg, uend, my_row,
                               static_cast<uint8_t*>(send), send_scales);
@@ -294,8 +305,14 @@ __global__ void __launch_bounds__(kThreads)
 
 }  // namespace
 
-size_t dispatch_workspace_bytes(int T, int E) {
-  const size_t n_chunks = (static_cast<size_t>(T) + kDispatchChunk - 1) / kDispatchChunk;
+int dispatch_chunk_tokens(int k) {
+  const int c = 16 * (128 / k);
+  return c < 16 ? 16 : c;
+}
+
+size_t dispatch_workspace_bytes(int T, int E, int k) {
+  const size_t ct = static_cast<size_t>(dispatch_chunk_tokens(k));
+  const size_t n_chunks = (static_cast<size_t>(T) + ct - 1) / ct;
   const size_t tab = (n_chunks > 0 ? n_chunks : 1) * static_cast<size_t>(E) * sizeof(int32_t);
   return 256 + (tab + 255) / 256 * 256;
 }
@@ -307,8 +324,8 @@ cudaError_t launch_dispatch(const void* x, int T, int H, const int32_t* topk_idx
   char* base = static_cast<char*>(ws);
   return launch_dispatch_parts(x, T, H, topk_idx, k, E, R, capacity, fp8, send, send_scales,
                                expert_counts, expert_offsets, rank_offsets, slot_row, row_token,
-                               reinterpret_cast<int*>(base), reinterpret_cast<unsigned*>(base + 4),
-                               reinterpret_cast<int32_t*>(base + 256), true, s);
+                               reinterpret_cast<int*>(base), reinterpret_cast<int32_t*>(base + 256),
+                               s);
 }
 
 cudaError_t launch_dispatch_parts(const void* x, int T, int H, const int32_t* topk_idx, int k,
@@ -316,8 +333,7 @@ cudaError_t launch_dispatch_parts(const void* x, int T, int H, const int32_t* to
                                   float* send_scales, int32_t* expert_counts,
                                   int32_t* expert_offsets, int32_t* rank_offsets,
                                   int32_t* slot_row, int32_t* row_token, int* status,
-                                  unsigned* arrivals, int32_t* chunk_tab, bool pdl_first,
-                                  cudaStream_t s) {
+                                  int32_t* hist, cudaStream_t s) {
   if (T == 0) {
     // nothing routed: zero counts and offsets
     cudaError_t e1 = cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * E, s);
@@ -326,26 +342,23 @@ cudaError_t launch_dispatch_parts(const void* x, int T, int H, const int32_t* to
     if (e1 != cudaSuccess) return e1;
     return cudaMemsetAsync(rank_offsets, 0, sizeof(int32_t) * (R + 1), s);
   }
-  const int n_chunks = (T + kDispatchChunk - 1) / kDispatchChunk;
-  const int scan_n = E > 4 * kThreads ? E : 4 * kThreads;
-  cudaError_t err = launch_pdl_if(pdl_first, count_scan_kernel, dim3(n_chunks), dim3(kThreads),
-                               sizeof(int) * scan_n, s, topk_idx, T, k, E, R, capacity, status,
-                               arrivals, chunk_tab, expert_counts, expert_offsets, rank_offsets);
+  const int chunk_tokens = dispatch_chunk_tokens(k);
+  const int n_chunks = (T + chunk_tokens - 1) / chunk_tokens;
+  cudaError_t err = launch_pdl(count_kernel, dim3(n_chunks), dim3(kThreads), sizeof(int) * E, s,
+                               topk_idx, T, k, E, chunk_tokens, status, hist);
   if (err != cudaSuccess) return err;
   // tokens per rank+permute CTA: about four CTAs per SM, at most 16
   int tile = 1;
   while (tile < kDispatchTileMax && (T + 2 * tile - 1) / (2 * tile) >= 4 * num_sms()) tile *= 2;
   const int tiles = (T + tile - 1) / tile;
-  const size_t smem = sizeof(int) * (E + tile * k);
+  const int scan_n = E > 4 * kThreads ? E : 4 * kThreads;
+  const size_t smem = sizeof(int) * (E + scan_n + 2 * tile * k);
   const uint4* xv = static_cast<const uint4*>(x);
-  if (fp8)
-    err = launch_pdl(rank_permute_kernel<true, 2>, dim3(tiles), dim3(kThreads), smem, s, topk_idx,
-                     T, k, E, capacity, chunk_tab, expert_offsets, slot_row, row_token, xv, H, tile,
-                     send, send_scales);
-  else
-    err = launch_pdl(rank_permute_kernel<false, 8>, dim3(tiles), dim3(kThreads), smem, s,
-                     topk_idx, T, k, E, capacity, chunk_tab, expert_offsets, slot_row, row_token, xv,
-                     H, tile, send, send_scales);
+  auto kern = fp8 ? rank_permute_kernel<true, 2> : rank_permute_kernel<false, 8>;
+  err = launch_pdl(kern, dim3(tiles), dim3(kThreads), smem, s, topk_idx, T, k, E, R, capacity,
+                   chunk_tokens, n_chunks, static_cast<const int32_t*>(hist), expert_counts,
+                   expert_offsets, rank_offsets, slot_row, row_token, xv, H, tile, send,
+                   send_scales);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }

@@ -6,7 +6,7 @@
 // plug-ins embedded in such programs, and latency-critical paths where cudaMalloc (which can
 // synchronise the device) is not acceptable.  This entry point needs only the inputs and outputs.
 //
-// The scratch (status word, arrival counter, per-chunk expert table) lives in g_dispatch_scratch,
+// The scratch (the per-chunk expert histogram) lives in g_dispatch_scratch,
 // a file-scope __device__ array of kNoallocScratchBytes.  Every GPU that loads the library keeps it
 // until the process exits.  Host code must not pass the array's name to a kernel (on the host it is
 // only a stand-in symbol); the device address is looked up once per device with
@@ -73,7 +73,7 @@ extern "C" moe_status_t moe_dispatch_noalloc(const void* x, int T, int H, const 
       !aligned(topk_idx, 4) || !aligned(status, 4))
     return MOE_ERR_INVALID_ARG;
   // the static scratch has a fixed size: reject shapes whose chunk table does not fit
-  if (moe::dispatch_workspace_bytes(T, E) > kNoallocScratchBytes) return MOE_ERR_WORKSPACE;
+  if (moe::dispatch_workspace_bytes(T, E, k) > kNoallocScratchBytes) return MOE_ERR_WORKSPACE;
 
   unsigned char* scratch = nullptr;
   if (scratch_for_current_device(&scratch) != cudaSuccess) {
@@ -81,18 +81,13 @@ extern "C" moe_status_t moe_dispatch_noalloc(const void* x, int T, int H, const 
     return MOE_ERR_CUDA;
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // The array keeps the previous call's contents.  The arrival counter must start at zero; the
-  // chunk table is fully written before it is read; the status word is the caller's.
-  unsigned* arrivals = reinterpret_cast<unsigned*>(scratch + 4);
-  if (cudaMemsetAsync(arrivals, 0, sizeof(unsigned), s) != cudaSuccess) {
-    cudaGetLastError();
-    return MOE_ERR_CUDA;
-  }
-  int32_t* chunk_tab = reinterpret_cast<int32_t*>(scratch + 256);
+  // The array keeps the previous call's contents.  Nothing in it has to start at zero: the
+  // histogram table is fully written by the count kernel before it is read, and the status word
+  // is the caller's.
+  int32_t* hist = reinterpret_cast<int32_t*>(scratch + 256);
   const cudaError_t err = moe::launch_dispatch_parts(
       x, T, H, topk_idx, k, E, R, capacity, fp8 ? 1 : 0, send, send_scales, expert_counts,
-      expert_offsets, rank_offsets, slot_row, row_token, reinterpret_cast<int*>(status), arrivals,
-      chunk_tab, /*pdl_first=*/false, s);  // the memset above precedes it: ordinary launch
+      expert_offsets, rank_offsets, slot_row, row_token, reinterpret_cast<int*>(status), hist, s);
   if (err != cudaSuccess) {
     cudaGetLastError();
     return MOE_ERR_CUDA;

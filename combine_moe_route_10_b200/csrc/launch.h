@@ -46,26 +46,23 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int renorm, i
 
 // Dispatch workspace layout (bytes from the 256-byte-aligned base):
 //   [0, 4)    status word (kStatus* bits)
-//   [4, 8)    arrival counter of the count/scan kernel (returns to 0 after every call)
-//   [256, ..) per-chunk expert histogram, then per-chunk base positions [n_chunks][E] int32
-constexpr int kDispatchChunk = 256;  // tokens per counting chunk
-constexpr int kDispatchTileMax = 16; // max tokens per rank+permute CTA (divides kDispatchChunk)
-size_t dispatch_workspace_bytes(int T, int E);
+//   [256, ..) per-chunk expert histogram [n_chunks][E] int32, chunks of dispatch_chunk_tokens(k)
+constexpr int kDispatchTileMax = 16;  // max tokens per rank+permute CTA (divides every chunk)
+int dispatch_chunk_tokens(int k);     // 16 * floor(128 / k), at least 16: ~2048 slots per chunk
+size_t dispatch_workspace_bytes(int T, int E, int k);
 
 cudaError_t launch_dispatch(const void* x, int T, int H, const int32_t* topk_idx, int k, int E,
                             int R, int capacity, int fp8, void* send, float* send_scales,
                             int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_offsets,
                             int32_t* slot_row, int32_t* row_token, void* ws, cudaStream_t s);
 
-// The same three kernels with the scratch pieces given separately (status word, arrival counter,
-// chunk table); the arrival counter must be zero on entry.
+// The same two kernels with the scratch pieces given separately (status word, histogram table).
 cudaError_t launch_dispatch_parts(const void* x, int T, int H, const int32_t* topk_idx, int k,
                                   int E, int R, int capacity, int fp8, void* send,
                                   float* send_scales, int32_t* expert_counts,
                                   int32_t* expert_offsets, int32_t* rank_offsets,
                                   int32_t* slot_row, int32_t* row_token, int* status,
-                                  unsigned* arrivals, int32_t* chunk_tab, bool pdl_first,
-                                  cudaStream_t s);
+                                  int32_t* hist, cudaStream_t s);
 
 cudaError_t launch_combine(const void* expert_out, int max_rows, const int32_t* slot_row,
                            const float* topk_w, int T, int k, int H, void* y, cudaStream_t s);

@@ -92,7 +92,8 @@ moe_status_t moe_route(const float* logits, int T, int E, int k, int renormalize
                        int32_t* topk_idx, float* topk_w, int32_t* expert_routed,
                        moe_stream_t stream);
 
-/* Bytes of scratch moe_dispatch needs for T tokens, E experts, k slots per token. */
+/* Bytes of scratch moe_dispatch needs for T tokens, E experts, k slots per token: a status word and
+ * one expert histogram per chunk of 16 * floor(128 / k) tokens. */
 size_t moe_dispatch_workspace_size(int T, int E, int k);
 
 /*
@@ -142,8 +143,9 @@ moe_status_t moe_dispatch(const void* x, int T, int H, const int32_t* topk_idx, 
  *   status  optional (may be NULL) device int32 owned by the caller, zeroed by the caller: device
  *           findings are OR-ed into it (1 = expert id out of range); moe_sync_status(status, s)
  *           reads and clears it like a workspace status word.
- * Limits: those of moe_dispatch, plus 256 + ceil(T/256) * E * 4 <= 1 MiB (e.g. T <= 65280 tokens at
- * E = 1024, T <= 522240 at E = 128); larger shapes return MOE_ERR_WORKSPACE without launching.
+ * Limits: those of moe_dispatch, plus 256 + ceil(T / C) * E * 4 <= 1 MiB, where C = 16 * floor(128 / k)
+ * tokens (at least 16) is the counting chunk (e.g. T <= 261120 at E = 1024, k = 2; T <= 65280 at
+ * E = 1024, k = 8); larger shapes return MOE_ERR_WORKSPACE without launching.
  * The first call on each device looks up the array's device address (cudaGetSymbolAddress with
  * that device current); make that first call before any stream capture.  All calls share the one
  * array: calls that overlap on the GPU (different streams, or the same array from several host

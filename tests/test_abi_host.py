@@ -95,8 +95,10 @@ def test_dispatch_rejects_bad_arguments(lib):
 
 
 def test_workspace_sizes(lib):
-    s1 = pkg.moe_dispatch_workspace_size(16384, 128, 2)
-    assert s1 >= 256 + 64 * 128 * 4 and s1 % 256 == 0
+    s1 = pkg.moe_dispatch_workspace_size(16384, 128, 2)     # 16 chunks of 1024 tokens
+    assert s1 >= 256 + 16 * 128 * 4 and s1 % 256 == 0
+    s8 = pkg.moe_dispatch_workspace_size(4096, 256, 8)      # 16 chunks of 256 tokens
+    assert s8 >= 256 + 16 * 256 * 4 and s8 % 256 == 0
     f = pkg.moe_ffn_workspace_size(32768, 256, 7168, 2048, pkg.MOE_PAYLOAD_FP8_E4M3_B128)
     assert f >= 256 + 32768 * 2048 * 2 + 32768 * 7168 * 2
     assert pkg.moe_ffn_workspace_size(100, 8, 256, 512, pkg.MOE_PAYLOAD_BF16) >= 256 + 100 * 512 * 2

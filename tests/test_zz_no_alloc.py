@@ -90,8 +90,8 @@ def test_noalloc_reports_bad_expert_ids_through_status(cuda):
 def test_noalloc_rejects_shapes_beyond_the_static_scratch():
     lib = pkg.load()
     fake = 1 << 20          # never dereferenced: the call returns before launching anything
-    # 256 + ceil(T/256) * E * 4 > 1 MiB
-    st = lib.moe_dispatch_noalloc(fake, 70000, 256, fake, 2, 1024, 8, 0, 0, fake, None, fake, fake,
+    # 256 + ceil(T / C) * E * 4 > 1 MiB with C = 16 * floor(128 / k) = 256 tokens for k = 8
+    st = lib.moe_dispatch_noalloc(fake, 70000, 256, fake, 8, 1024, 8, 0, 0, fake, None, fake, fake,
                                   fake, fake, fake, None, None)
     assert st == pkg.MOE_ERR_WORKSPACE
     st = lib.moe_dispatch_noalloc(fake, 64, 256, fake, 2, 8, 3, 0, 0, fake, None, fake, fake,
