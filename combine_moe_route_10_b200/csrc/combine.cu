@@ -25,16 +25,20 @@ __device__ __forceinline__ void accumulate(float acc[8], float w, uint4 v) {
 
 // KS rows are gathered together per step (loads issued before any accumulation); UNROLL vectors
 // per lane per row.
-template <int KS, int UNROLL>
+template <int KS, int UNROLL, bool SPLIT>
 __global__ void __launch_bounds__(kThreads)
     combine_kernel(const uint4* __restrict__ expert_out, int max_rows,
                    const int32_t* __restrict__ slot_row, const float* __restrict__ topk_w, int T,
-                   int k, int nvec, uint4* __restrict__ y) {
+                   int k, int nvec, int wpt, uint4* __restrict__ y) {
   const int lane = threadIdx.x & 31;
+  const int gwarp = blockIdx.x * kWarps + (threadIdx.x >> 5);
   const int nwarps = gridDim.x * kWarps;
+  // wpt warps per token (wpt divides nvec), each takes nseg consecutive vectors of the row
+  const int nseg = SPLIT ? nvec / wpt : nvec;
+  const int vofs = SPLIT ? (gwarp % wpt) * nseg : 0;
   griddep_wait();
   griddep_launch_dependents();
-  for (int t = blockIdx.x * kWarps + (threadIdx.x >> 5); t < T; t += nwarps) {
+  for (int t = SPLIT ? gwarp / wpt : gwarp; t < T; t += SPLIT ? nwarps / wpt : nwarps) {
     int my_row = -1;
     float my_w = 0.0f;
     if (lane < k) {
@@ -43,8 +47,8 @@ __global__ void __launch_bounds__(kThreads)
       if (my_row >= max_rows) my_row = -1;
     }
     const unsigned live = __ballot_sync(0xFFFFFFFFu, my_row >= 0);
-    uint4* dst = y + static_cast<size_t>(t) * nvec;
-    for (int v0 = 0; v0 < nvec; v0 += 32 * UNROLL) {
+    uint4* dst = y + static_cast<size_t>(t) * nvec + vofs;
+    for (int v0 = 0; v0 < nseg; v0 += 32 * UNROLL) {
       float acc[UNROLL][8];
 #pragma unroll
       for (int u = 0; u < UNROLL; ++u)
@@ -73,11 +77,11 @@ __global__ void __launch_bounds__(kThreads)
             const int j = rows[q];
             const int row = __shfl_sync(0xFFFFFFFFu, my_row, j);
             ws[q] = __shfl_sync(0xFFFFFFFFu, my_w, j);
-            const uint4* src = expert_out + static_cast<size_t>(row) * nvec;
+            const uint4* src = expert_out + static_cast<size_t>(row) * nvec + vofs;
 #pragma unroll
             for (int u = 0; u < UNROLL; ++u) {
               const int v = v0 + u * 32 + lane;
-              if (v < nvec) vals[q][u] = ld_nc_v4(src + v);
+              if (v < nseg) vals[q][u] = ld_nc_v4(src + v);
             }
           }
         }
@@ -87,7 +91,7 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
             for (int u = 0; u < UNROLL; ++u) {
               const int v = v0 + u * 32 + lane;
-              if (v < nvec) accumulate(acc[u], ws[q], vals[q][u]);
+              if (v < nseg) accumulate(acc[u], ws[q], vals[q][u]);
             }
           }
         }
@@ -95,7 +99,7 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
       for (int u = 0; u < UNROLL; ++u) {
         const int v = v0 + u * 32 + lane;
-        if (v < nvec) {
+        if (v < nseg) {
           uint4 o;
           o.x = pack_bf16x2(acc[u][0], acc[u][1]);
           o.y = pack_bf16x2(acc[u][2], acc[u][3]);
@@ -113,16 +117,29 @@ __global__ void __launch_bounds__(kThreads)
 cudaError_t launch_combine(const void* expert_out, int max_rows, const int32_t* slot_row,
                            const float* topk_w, int T, int k, int H, void* y, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
-  int blocks = (T + kWarps - 1) / kWarps;
+  // warps per token: split rows so that about 64 warps per SM have work (small T)
+  const int nvec = H / 8;
+  int wpt = 1;
+  while (wpt < 8 && static_cast<long long>(T) * wpt < 64LL * num_sms() && nvec % (2 * wpt) == 0 &&
+         nvec / (2 * wpt) >= 32)
+    wpt *= 2;
+  const long long warps = static_cast<long long>(T) * wpt;
+  int blocks = static_cast<int>((warps + kWarps - 1) / kWarps);
   const int cap = num_sms() * 8;
-  if (blocks > cap) blocks = cap;
+  if (blocks > cap) blocks = cap;  // grid-stride; cap is a multiple of 8, so of wpt
   const uint4* eo = static_cast<const uint4*>(expert_out);
   uint4* yo = static_cast<uint4*>(y);
   // rows gathered together sized to k: enough loads in flight, few registers (high occupancy)
-  void (*kern)(const uint4*, int, const int32_t*, const float*, int, int, int, uint4*) =
-      k <= 2 ? combine_kernel<2, 4> : (k <= 4 ? combine_kernel<4, 2> : combine_kernel<8, 1>);
+  using Kern = void (*)(const uint4*, int, const int32_t*, const float*, int, int, int, int, uint4*);
+  Kern kern;
+  if (wpt > 1)
+    kern = k <= 2 ? combine_kernel<2, 4, true>
+                  : (k <= 4 ? combine_kernel<4, 2, true> : combine_kernel<8, 1, true>);
+  else
+    kern = k <= 2 ? combine_kernel<2, 4, false>
+                  : (k <= 4 ? combine_kernel<4, 2, false> : combine_kernel<8, 1, false>);
   const cudaError_t err = launch_pdl(kern, dim3(blocks), dim3(kThreads), 0, s, eo, max_rows,
-                                     slot_row, topk_w, T, k, H / 8, yo);
+                                     slot_row, topk_w, T, k, nvec, wpt, yo);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
