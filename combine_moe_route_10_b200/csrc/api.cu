@@ -114,9 +114,8 @@ moe_status_t moe_dispatch(const void* x, int T, int H, const int32_t* topk_idx, 
 }
 
 size_t moe_ffn_workspace_size(int max_rows, int E, int H, int F, moe_payload_t payload) {
-  (void)E;
-  if (max_rows < 0 || H < 1 || F < 1) return 0;
-  return moe::ffn_workspace_bytes(max_rows, H, F, payload == MOE_PAYLOAD_FP8_E4M3_B128);
+  if (max_rows < 0 || E < 1 || H < 1 || F < 1) return 0;
+  return moe::ffn_workspace_bytes(max_rows, H, F, payload == MOE_PAYLOAD_FP8_E4M3_B128, E);
 }
 
 moe_status_t moe_expert_ffn(const void* send, const float* send_scales, moe_payload_t payload,
@@ -138,7 +137,7 @@ moe_status_t moe_expert_ffn(const void* send, const float* send_scales, moe_payl
   if (!aligned(send, 16) || !aligned(w_gate, 16) || !aligned(w_up, 16) || !aligned(w_down, 16) ||
       !aligned(expert_out, 16) || !aligned(expert_offsets, 4) || !aligned(send_scales, 4))
     return MOE_ERR_INVALID_ARG;
-  if (!aligned(ws, 256) || ws_bytes < moe::ffn_workspace_bytes(max_rows, H, F, fp8 ? 1 : 0))
+  if (!aligned(ws, 256) || ws_bytes < moe::ffn_workspace_bytes(max_rows, H, F, fp8 ? 1 : 0, E))
     return MOE_ERR_WORKSPACE;
   return from_cuda(moe::launch_expert_ffn(send, send_scales, fp8 ? 1 : 0, expert_offsets, max_rows,
                                           E, H, F, w_gate, w_up, w_down, expert_out, ws,

@@ -7,7 +7,8 @@
 // run_moe passage of "DWDP: 在NVL72上的高性能分布式权重数据并行"):
 //     h = bf16( silu(x W_gate[e]^T) * (x W_up[e]^T) ),   expert_out = bf16( h W_down[e]^T ).
 //
-// Two launches of one persistent kernel template (one CTA per SM, 192 threads):
+// One persistent launch (one CTA per SM, 192 threads) runs the GEMM-1 tiles and then the GEMM-2
+// tiles (the latter wait on per-row-block completion counters of the former):
 //   warp 0      TMA producer: A tile (128 rows x 64 k) + B tile (256 rows x 64 k) per stage,
 //               128-byte swizzle, 4-stage mbarrier ring;
 //   warp 1      TMEM allocator and MMA issuer: one thread issues tcgen05.mma (M=128, N=256,
@@ -51,19 +52,6 @@ constexpr int kStageBytes = kATileBytes + kBTileBytes;
 #endif
 constexpr int kGemm2NTile = 256;  // output columns per GEMM-2 tile (128 measured slower)
 
-enum Mode { kSwiGLU = 0, kPlain = 1 };
-
-struct GemmArgs {
-  const int32_t* expert_offsets;  // [E+1], device
-  int E;
-  int max_rows;
-  int N;       // output columns (F for SwiGLU, H for the plain GEMM)
-  int K;       // reduction length (H, resp. F)
-  int n_tile;  // output columns per tile (128 for SwiGLU; 256 or 128 for plain)
-  int b_rows_per_expert;  // rows of one expert in the B tensor map(s)
-  __nv_bfloat16* out;     // [max_rows, N]
-  int* status;
-};
 
 // ---- PTX wrappers ------------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
@@ -157,48 +145,6 @@ __host__ __device__ constexpr uint32_t make_idesc(int M, int N) {
          | (static_cast<uint32_t>(M >> 4) << 24);     // M / 16
 }
 
-struct Smem {
-  uint8_t* tiles;         // kStages x (A | B), 1024-byte aligned
-  uint64_t* full;         // [kStages]
-  uint64_t* empty;        // [kStages]
-  uint64_t* acc_full;     // [2]
-  uint64_t* acc_empty;    // [2]
-  uint64_t* drain;        // [1]
-  uint32_t* tmem_base;
-  int* abort_flag;
-  int* off;               // [E+1] row offsets (clamped to max_rows)
-  int* tstart;            // [E+1] first tile of each non-hot expert among non-hot tiles
-  int* hstart;            // [E+1] first tile of each hot expert among hot tiles
-  int* mtiles;            // [E]
-  int* totals;            // [2]: non-hot tiles, hot tiles
-};
-
-__device__ __forceinline__ Smem carve(uint8_t* raw, int E) {
-  Smem s;
-  const uint32_t a = smem_addr(raw);
-  uint8_t* p = raw + ((1024u - (a & 1023u)) & 1023u);
-  s.tiles = p;
-  p += kStages * kStageBytes;
-  s.full = reinterpret_cast<uint64_t*>(p);
-  s.empty = s.full + kStages;
-  s.acc_full = s.empty + kStages;
-  s.acc_empty = s.acc_full + 2;
-  s.drain = s.acc_empty + 2;
-  s.tmem_base = reinterpret_cast<uint32_t*>(s.drain + 1);
-  s.abort_flag = reinterpret_cast<int*>(s.tmem_base + 1);
-  s.off = s.abort_flag + 2;
-  s.tstart = s.off + (E + 1);
-  s.hstart = s.tstart + (E + 1);
-  s.mtiles = s.hstart + (E + 1);
-  s.totals = s.mtiles + E;
-  return s;
-}
-
-size_t gemm_smem_bytes(int E) {
-  return 1024 + static_cast<size_t>(kStages) * kStageBytes + 8 * (2 * kStages + 5) + 16 +
-         sizeof(int) * (4 * static_cast<size_t>(E) + 5);
-}
-
 // Bounded wait on an mbarrier phase.  Returns false if the CTA is aborting or the limit ran out.
 __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                            int* status) {
@@ -224,54 +170,158 @@ __device__ __forceinline__ int owner_of(const int* start, int E, int idx) {
   return lo;
 }
 
-// Tile -> (expert, row block, column block).  Row blocks are the fastest index inside an expert.
-// With hot experts present, tile t is hot iff floor((t+1)*Hn/N) > floor(t*Hn/N) (an even spread of
-// the Hn hot tiles over all N tiles), and indexes its own list.
-__device__ __forceinline__ void decode_tile(const Smem& s, int E, int tile, int& e, int& m_blk,
-                                            int& n_blk) {
-  const int n_cold = s.totals[0], n_hot = s.totals[1];
-  const int* start = s.tstart;
-  int idx = tile;
-  if (n_hot > 0) {
-    if (n_cold == 0) {
-      start = s.hstart;
-    } else {
-      const long long N = static_cast<long long>(n_cold) + n_hot;
-      const long long h0 = static_cast<long long>(tile) * n_hot / N;
-      const long long h1 = static_cast<long long>(tile + 1) * n_hot / N;
-      if (h1 > h0) {
-        start = s.hstart;
-        idx = static_cast<int>(h0);
-      } else {
-        idx = tile - static_cast<int>(h0);
-      }
-    }
-  }
-  e = owner_of(start, E, idx);
-  const int local = idx - start[e];
-  const int mt = s.mtiles[e];
-  n_blk = local / mt;
-  m_blk = local - n_blk * mt;
-}
-
 __device__ __forceinline__ float silu_mul(float g, float u) {
   return g / (1.0f + expf(-g)) * u;
 }
 
-template <int MODE>
+// ---- fused FFN: GEMM-1 (gate|up + SwiGLU) and GEMM-2 (down) tiles in one persistent launch -------
+//
+// Tiles are numbered [all GEMM-1 tiles][all GEMM-2 tiles]; each CTA takes tiles blockIdx.x,
+// blockIdx.x + gridDim.x, ... in increasing order.  A GEMM-2 tile (expert e, row block m) reads the
+// rows of h that the GEMM-1 tiles of (e, m) write, so its producer first waits (bounded) until the
+// completion counter of (e, m) reaches 4 * n1 (four epilogue warps per GEMM-1 tile, n1 column
+// blocks).  GEMM-1 tiles never wait, and every CTA finishes its GEMM-1 tiles before it reaches its
+// GEMM-2 tiles, so with all CTAs resident (one per SM) the waits always end; they are bounded
+// anyway.  Writers: st.global of h, fence.proxy.async (generic -> async proxy), release increment.
+// Readers: acquire load of the counter, fence.proxy.async, then the TMA loads of h.
+struct FfnArgs {
+  const int32_t* expert_offsets;  // [E+1], device
+  int E, max_rows, H, F;
+  __nv_bfloat16* h;               // [max_rows, F] workspace
+  __nv_bfloat16* out;             // [max_rows, H]
+  int* status;
+  int* done;                      // [sum of row blocks] GEMM-1 completion counters, zero on entry
+};
+
+struct FSmem {
+  uint8_t* tiles;
+  uint64_t *full, *empty, *acc_full, *acc_empty, *drain;
+  uint32_t* tmem_base;
+  int* abort_flag;
+  int* off;      // [E+1] row offsets (clamped to max_rows)
+  int* mt;       // [E]   row blocks per expert
+  int* ms_all;   // [E+1] first global row block of each expert
+  int* ms_cold;  // [E+1] first row block of each non-hot expert among non-hot row blocks
+  int* ms_hot;   // [E+1] same among hot row blocks
+  int* totals;   // [2] non-hot, hot row blocks
+};
+
+__device__ __forceinline__ FSmem fcarve(uint8_t* raw, int E) {
+  FSmem s;
+  const uint32_t a = smem_addr(raw);
+  uint8_t* p = raw + ((1024u - (a & 1023u)) & 1023u);
+  s.tiles = p;
+  p += kStages * kStageBytes;
+  s.full = reinterpret_cast<uint64_t*>(p);
+  s.empty = s.full + kStages;
+  s.acc_full = s.empty + kStages;
+  s.acc_empty = s.acc_full + 2;
+  s.drain = s.acc_empty + 2;
+  s.tmem_base = reinterpret_cast<uint32_t*>(s.drain + 1);
+  s.abort_flag = reinterpret_cast<int*>(s.tmem_base + 1);
+  s.off = s.abort_flag + 2;
+  s.mt = s.off + (E + 1);
+  s.ms_all = s.mt + E;
+  s.ms_cold = s.ms_all + (E + 1);
+  s.ms_hot = s.ms_cold + (E + 1);
+  s.totals = s.ms_hot + (E + 1);
+  return s;
+}
+
+size_t fused_smem_bytes(int E) {
+  return 1024 + static_cast<size_t>(kStages) * kStageBytes + 8 * (2 * kStages + 5) + 16 +
+         sizeof(int) * (5 * static_cast<size_t>(E) + 8);
+}
+
+struct FTile {
+  int phase;  // 1: GEMM-1 (SwiGLU), 2: GEMM-2 (down)
+  int e, m_blk, n_blk, mg;
+};
+
+// Tile -> phase, expert, row block, column block (row blocks fastest inside an expert); hot and
+// non-hot experts' tiles are spread evenly over each phase as in the two-launch kernel.
+__device__ __forceinline__ FTile fdecode(const FSmem& s, int E, int n1, int n2, int tile) {
+  FTile t;
+  const int MC = s.totals[0], MH = s.totals[1];
+  const int N1 = (MC + MH) * n1;
+  int nt, idx;
+  if (tile < N1) {
+    t.phase = 1;
+    nt = n1;
+    idx = tile;
+  } else {
+    t.phase = 2;
+    nt = n2;
+    idx = tile - N1;
+  }
+  const int* ms = s.ms_cold;
+  if (MH > 0) {
+    if (MC == 0) {
+      ms = s.ms_hot;
+    } else {
+      const long long Nt = static_cast<long long>(MC + MH) * nt;
+      const long long hn = static_cast<long long>(MH) * nt;
+      const long long h0 = static_cast<long long>(idx) * hn / Nt;
+      const long long h1 = static_cast<long long>(idx + 1) * hn / Nt;
+      if (h1 > h0) {
+        ms = s.ms_hot;
+        idx = static_cast<int>(h0);
+      } else {
+        idx -= static_cast<int>(h0);
+      }
+    }
+  }
+  t.e = owner_of(ms, E, idx / nt);
+  const int local = idx - nt * ms[t.e];
+  const int mt = s.mt[t.e];
+  t.n_blk = local / mt;
+  t.m_blk = local - t.n_blk * mt;
+  t.mg = s.ms_all[t.e] + t.m_blk;
+  return t;
+}
+
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_add(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Bounded wait until *p >= target (acquire).  False if the CTA aborts or the limit runs out.
+__device__ __forceinline__ bool wait_counter(const int* p, int target, volatile int* abort_flag,
+                                             int* status) {
+  if (ld_acquire(p) >= target) return true;
+  const unsigned long long t0 = global_timer_ns();
+  while (true) {
+    __nanosleep(64);
+    if (ld_acquire(p) >= target) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      record_status(status, kStatusTimeout);
+      return false;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
-                        const __grid_constant__ CUtensorMap tm_b0,
-                        const __grid_constant__ CUtensorMap tm_b1, const GemmArgs args) {
+    fused_ffn_kernel(const __grid_constant__ CUtensorMap tm_x,
+                     const __grid_constant__ CUtensorMap tm_g,
+                     const __grid_constant__ CUtensorMap tm_u,
+                     const __grid_constant__ CUtensorMap tm_h,
+                     const __grid_constant__ CUtensorMap tm_d, const FfnArgs args) {
   extern __shared__ uint8_t smem_raw[];
   const int E = args.E;
-  Smem s = carve(smem_raw, E);
+  FSmem s = fcarve(smem_raw, E);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_tiles = (args.N + args.n_tile - 1) / args.n_tile;
-  const int num_kb = (args.K + BK - 1) / BK;
+  const int n1 = (args.F + 127) / 128;       // GEMM-1 column blocks (128 h columns each)
+  const int n2 = (args.H + 255) / 256;       // GEMM-2 column blocks (256 output columns each)
+  const int kb1 = (args.H + BK - 1) / BK, kb2 = (args.F + BK - 1) / BK;
   volatile int* abort_flag = s.abort_flag;
 
-  // ---- set-up: barriers, TMEM, schedule --------------------------------------------------------
   if (warp == 0) {
     if (lane == 0) {
       for (int i = 0; i < kStages; ++i) {
@@ -280,16 +330,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int i = 0; i < 2; ++i) {
         mbar_init(smem_addr(&s.acc_full[i]), 1);
-        mbar_init(smem_addr(&s.acc_empty[i]), 4);  // one arrival per epilogue warp
+        mbar_init(smem_addr(&s.acc_empty[i]), 4);
       }
       mbar_init(smem_addr(s.drain), 1);
       *s.abort_flag = 0;
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_a)) : "memory");
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_b0)) : "memory");
-      if (MODE == kSwiGLU)
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_b1)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_x)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_g)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_u)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_h)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_d)) : "memory");
     }
   } else if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -299,9 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   } else if (warp == 2) {
     griddep_wait();
-    // schedule: per-expert row offsets, row-block counts, and the first tile of each expert in
-    // its list (non-hot or hot)
-    int carry_c = 0, carry_h = 0;
+    int carry_a = 0, carry_c = 0, carry_h = 0;
     for (int e0 = 0; e0 < E; e0 += 32) {
       const int e = e0 + lane;
       int lo = 0, hi = 0;
@@ -309,45 +358,48 @@ __global__ void __launch_bounds__(kThreads, 1)
         lo = min(__ldg(args.expert_offsets + e), args.max_rows);
         hi = min(__ldg(args.expert_offsets + e + 1), args.max_rows);
       }
-      const int rows = max(hi - lo, 0);
-      const int mt = (rows + BM - 1) / BM;
+      const int mt = (max(hi - lo, 0) + BM - 1) / BM;
       const bool hot = MOE_FFN_HOT_MTILES > 0 && mt >= MOE_FFN_HOT_MTILES;
-      const int tiles_c = hot ? 0 : mt * n_tiles;
-      const int tiles_h = hot ? mt * n_tiles : 0;
-      int inc_c = tiles_c, inc_h = tiles_h;
+      const int mc = hot ? 0 : mt, mh = hot ? mt : 0;
+      int ia = mt, ic = mc, ih = mh;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const int yc = __shfl_up_sync(0xFFFFFFFFu, inc_c, o);
-        const int yh = __shfl_up_sync(0xFFFFFFFFu, inc_h, o);
+        const int ya = __shfl_up_sync(0xFFFFFFFFu, ia, o);
+        const int yc = __shfl_up_sync(0xFFFFFFFFu, ic, o);
+        const int yh = __shfl_up_sync(0xFFFFFFFFu, ih, o);
         if (lane >= o) {
-          inc_c += yc;
-          inc_h += yh;
+          ia += ya;
+          ic += yc;
+          ih += yh;
         }
       }
       if (e < E) {
         s.off[e] = lo;
-        s.mtiles[e] = mt;
-        s.tstart[e] = carry_c + inc_c - tiles_c;
-        s.hstart[e] = carry_h + inc_h - tiles_h;
+        s.mt[e] = mt;
+        s.ms_all[e] = carry_a + ia - mt;
+        s.ms_cold[e] = carry_c + ic - mc;
+        s.ms_hot[e] = carry_h + ih - mh;
       }
-      carry_c += __shfl_sync(0xFFFFFFFFu, inc_c, 31);
-      carry_h += __shfl_sync(0xFFFFFFFFu, inc_h, 31);
+      carry_a += __shfl_sync(0xFFFFFFFFu, ia, 31);
+      carry_c += __shfl_sync(0xFFFFFFFFu, ic, 31);
+      carry_h += __shfl_sync(0xFFFFFFFFu, ih, 31);
     }
     if (lane == 0) {
-      s.tstart[E] = carry_c;
-      s.hstart[E] = carry_h;
+      s.ms_all[E] = carry_a;
+      s.ms_cold[E] = carry_c;
+      s.ms_hot[E] = carry_h;
       s.totals[0] = carry_c;
       s.totals[1] = carry_h;
       s.off[E] = min(__ldg(args.expert_offsets + E), args.max_rows);
     }
   }
-  griddep_wait();  // every thread: the previous grid's outputs are visible from here on
+  griddep_wait();
   griddep_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s.tmem_base;
-  const int total_tiles = s.totals[0] + s.totals[1];
+  const int total_tiles = (s.totals[0] + s.totals[1]) * (n1 + n2);
   const uint32_t tiles_base = smem_addr(s.tiles);
 
   if (warp == 0) {
@@ -355,16 +407,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t issued_mask = 0, issued_parity = 0;  // per stage: issued at least once / last parity
-      const uint32_t tx = MODE == kSwiGLU ? kStageBytes
-                                          : kATileBytes + args.n_tile * BK * 2;
+      uint32_t issued_mask = 0, issued_parity = 0;
       for (int tile = blockIdx.x; tile < total_tiles && !*abort_flag; tile += gridDim.x) {
-        int e, m_blk, n_blk;
-        decode_tile(s, E, tile, e, m_blk, n_blk);
-        const int row_a = s.off[e] + m_blk * BM;
-        const int row_b = e * args.b_rows_per_expert + n_blk * args.n_tile;
+        const FTile t = fdecode(s, E, n1, n2, tile);
+        const int row_a = s.off[t.e] + t.m_blk * BM;
+        int nkb;
+        const CUtensorMap *ma, *mb;
+        int row_b;
+        if (t.phase == 1) {
+          nkb = kb1;
+          ma = &tm_x;
+          mb = &tm_g;
+          row_b = t.e * args.F + t.n_blk * 128;
+        } else {
+          // the rows of h this tile reads are complete once all GEMM-1 tiles of (e, m) are
+          if (!wait_counter(args.done + t.mg, 4 * n1, abort_flag, args.status)) break;
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+          nkb = kb2;
+          ma = &tm_h;
+          mb = &tm_d;
+          row_b = t.e * args.H + t.n_blk * 256;
+        }
         bool ok = true;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = 0; kb < nkb; ++kb) {
           if (!wait_phase(smem_addr(&s.empty[stage]), phase ^ 1u, abort_flag, args.status)) {
             ok = false;
             break;
@@ -372,10 +437,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t a_dst = tiles_base + stage * kStageBytes;
           const uint32_t b_dst = a_dst + kATileBytes;
           const uint32_t fb = smem_addr(&s.full[stage]);
-          mbar_arrive_expect_tx(fb, tx);
-          tma_load_2d(a_dst, &tm_a, fb, kb * BK, row_a);
-          tma_load_2d(b_dst, &tm_b0, fb, kb * BK, row_b);
-          if (MODE == kSwiGLU) tma_load_2d(b_dst + kBTileBytes / 2, &tm_b1, fb, kb * BK, row_b);
+          mbar_arrive_expect_tx(fb, kStageBytes);
+          tma_load_2d(a_dst, ma, fb, kb * BK, row_a);
+          tma_load_2d(b_dst, mb, fb, kb * BK, row_b);
+          if (t.phase == 1) tma_load_2d(b_dst + kBTileBytes / 2, &tm_u, fb, kb * BK, row_b);
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == kStages) {
@@ -386,7 +451,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
       }
       if (*abort_flag) {
-        // let this CTA's own bulk copies land before the CTA (and its smem) goes away
         volatile int no_abort = 0;
         for (int st = 0; st < kStages; ++st)
           if (issued_mask & (1u << st))
@@ -395,14 +459,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    // ---- MMA issuer --------------------------------------------------------------------------------
+    // ---- MMA issuer (M=128, N=256 for both phases) -------------------------------------------------
     if (lane == 0) {
-      const uint32_t idesc = make_idesc(BM, MODE == kSwiGLU ? 256 : args.n_tile);
+      const uint32_t idesc = make_idesc(BM, 256);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
       bool issued_any = false;
       for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
+        const int nkb = tile < (s.totals[0] + s.totals[1]) * n1 ? kb1 : kb2;
         const int acc = it & 1;
         const uint32_t acc_parity = (it >> 1) & 1;
         if (!wait_phase(smem_addr(&s.acc_empty[acc]), acc_parity ^ 1u, abort_flag, args.status))
@@ -410,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kAccCols;
         bool ok = true;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = 0; kb < nkb; ++kb) {
           if (!wait_phase(smem_addr(&s.full[stage]), phase, abort_flag, args.status)) {
             ok = false;
             break;
@@ -419,56 +484,51 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t a_addr = tiles_base + stage * kStageBytes;
           const uint32_t b_addr = a_addr + kATileBytes;
 #pragma unroll
-          for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-            tc_mma(d_tmem, sw128_desc(a_addr + kk * UMMA_K * 2), sw128_desc(b_addr + kk * UMMA_K * 2),
-                   idesc, (kb | kk) != 0 ? 1u : 0u);
-          }
+          for (int kk = 0; kk < BK / UMMA_K; ++kk)
+            tc_mma(d_tmem, sw128_desc(a_addr + kk * UMMA_K * 2),
+                   sw128_desc(b_addr + kk * UMMA_K * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
           issued_any = true;
-          tc_commit(smem_addr(&s.empty[stage]));  // stage reusable once these MMAs finish
+          tc_commit(smem_addr(&s.empty[stage]));
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit(smem_addr(&s.acc_full[acc]));  // accumulator complete
+        tc_commit(smem_addr(&s.acc_full[acc]));
       }
       if (issued_any) {
-        // all MMAs of this CTA retire before TMEM is released
         tc_commit(smem_addr(s.drain));
         volatile int no_abort = 0;
         wait_phase(smem_addr(s.drain), 0, &no_abort, args.status);
       }
     }
   } else {
-    // ---- epilogue: TMEM -> registers -> global ---------------------------------------------------
-    const int quarter = warp & 3;                    // TMEM lanes 32*quarter .. 32*quarter+31
+    // ---- epilogue ----------------------------------------------------------------------------------
+    const int quarter = warp & 3;
     const int r_local = quarter * 32 + lane;
     int it = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
-      int e, m_blk, n_blk;
-      decode_tile(s, E, tile, e, m_blk, n_blk);
+      const FTile t = fdecode(s, E, n1, n2, tile);
       const int acc = it & 1;
       const uint32_t acc_parity = (it >> 1) & 1;
-      // one lane waits and the warp follows its verdict, so the .sync.aligned TMEM loads below
-      // are always executed by the whole warp or by none of it
       bool ok = true;
       if (lane == 0) ok = wait_phase(smem_addr(&s.acc_full[acc]), acc_parity, abort_flag, args.status);
       if (!__shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0)) break;
       tc_fence_after();
-      const int row = s.off[e] + m_blk * BM + r_local;
-      const bool row_ok = row < s.off[e + 1];
+      const int row = s.off[t.e] + t.m_blk * BM + r_local;
+      const bool row_ok = row < s.off[t.e + 1];
       const uint32_t t_row = tmem_base + acc * kAccCols + (static_cast<uint32_t>(quarter * 32) << 16);
-      __nv_bfloat16* out_row = args.out + static_cast<size_t>(row) * args.N;
-      if (MODE == kSwiGLU) {
+      if (t.phase == 1) {
+        __nv_bfloat16* out_row = args.h + static_cast<size_t>(row) * args.F;
 #pragma unroll 1
         for (int c = 0; c < 128; c += 32) {
           uint32_t g[32], u[32];
           tmem_ld32(t_row + c, g);
           tmem_ld32(t_row + 128 + c, u);
           tmem_wait_ld();
-          const int col = n_blk * 128 + c;
-          if (row_ok && col < args.N) {
+          const int col = t.n_blk * 128 + c;
+          if (row_ok && col < args.F) {
             uint32_t packed[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -482,14 +542,20 @@ __global__ void __launch_bounds__(kThreads, 1)
               dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
           }
         }
+        // publish: this warp's rows of h for (e, m, n) are written
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) red_release_add(args.done + t.mg, 1);
       } else {
+        __nv_bfloat16* out_row = args.out + static_cast<size_t>(row) * args.H;
 #pragma unroll 1
-        for (int c = 0; c < args.n_tile; c += 32) {
+        for (int c = 0; c < 256; c += 32) {
           uint32_t v[32];
           tmem_ld32(t_row + c, v);
           tmem_wait_ld();
-          const int col = n_blk * args.n_tile + c;
-          if (row_ok && col < args.N) {
+          const int col = t.n_blk * 256 + c;
+          if (row_ok && col < args.H) {
             uint32_t packed[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
@@ -507,7 +573,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  // ---- teardown ------------------------------------------------------------------------------------
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -581,26 +646,19 @@ bool make_tmap(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t cols, u
   return r == CUDA_SUCCESS;
 }
 
-template <int MODE>
-cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                        const GemmArgs& args, cudaStream_t s) {
-  const size_t smem = gemm_smem_bytes(args.E);
-  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-  if (err != cudaSuccess) return err;
-  err = launch_pdl(grouped_gemm_kernel<MODE>, dim3(num_sms()), dim3(kThreads), smem, s, a, b0, b1,
-                   args);
-  if (err != cudaSuccess) return err;
-  return cudaGetLastError();
-}
-
 }  // namespace
 
-size_t ffn_workspace_bytes(int max_rows, int H, int F, int fp8) {
-  const size_t h_bytes = (static_cast<size_t>(max_rows) * F * 2 + 255) / 256 * 256;
-  const size_t x_bytes = fp8 ? (static_cast<size_t>(max_rows) * H * 2 + 255) / 256 * 256 : 0;
-  return 256 + h_bytes + x_bytes;
+// Workspace: [0,4) status | [256, ..) h bf16 [max_rows, F] | (FP8) dequantised rows bf16
+// [max_rows, H] | GEMM-1 completion counters int32 [max_rows/128 + E + 1].
+static size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+static size_t ffn_counter_count(int max_rows, int E) {
+  return static_cast<size_t>(max_rows) / BM + static_cast<size_t>(E) + 1;
+}
+
+size_t ffn_workspace_bytes(int max_rows, int H, int F, int fp8, int E) {
+  const size_t h_bytes = round256(static_cast<size_t>(max_rows) * F * 2);
+  const size_t x_bytes = fp8 ? round256(static_cast<size_t>(max_rows) * H * 2) : 0;
+  return 256 + h_bytes + x_bytes + round256(ffn_counter_count(max_rows, E) * sizeof(int));
 }
 
 cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp8,
@@ -611,35 +669,48 @@ cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp
   char* base = static_cast<char*>(ws);
   int* status = reinterpret_cast<int*>(base);
   __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(base + 256);
+  size_t off = 256 + round256(static_cast<size_t>(max_rows) * F * 2);
+  uint4* xdq = nullptr;
+  if (fp8) {
+    xdq = reinterpret_cast<uint4*>(base + off);
+    off += round256(static_cast<size_t>(max_rows) * H * 2);
+  }
+  int* done = reinterpret_cast<int*>(base + off);
+  // GEMM-1 completion counters start at zero; the next launch follows a memset, so it is an
+  // ordinary (not programmatic) launch
+  cudaError_t err = cudaMemsetAsync(done, 0, ffn_counter_count(max_rows, E) * sizeof(int), s);
+  if (err != cudaSuccess) return err;
+  bool pdl_next = false;
   const void* a_src = send;
   if (fp8) {
-    uint4* xdq = reinterpret_cast<uint4*>(
-        base + 256 + (static_cast<size_t>(max_rows) * F * 2 + 255) / 256 * 256);
     const long long work = static_cast<long long>(max_rows) * (H / 16);
     long long blocks = (work + 255) / 256;
     const long long cap = static_cast<long long>(num_sms()) * 8;
     if (blocks > cap) blocks = cap;
-    const cudaError_t e0 = launch_pdl(dequant_fp8_kernel, dim3(static_cast<int>(blocks)), dim3(256),
-                                      0, s, static_cast<const uint8_t*>(send), send_scales,
-                                      expert_offsets + E, max_rows, H, xdq);
-    if (e0 != cudaSuccess) return e0;
+    err = launch_pdl_if(pdl_next, dequant_fp8_kernel, dim3(static_cast<int>(blocks)), dim3(256), 0,
+                        s, static_cast<const uint8_t*>(send), send_scales, expert_offsets + E,
+                        max_rows, H, xdq);
+    if (err != cudaSuccess) return err;
     a_src = xdq;
+    pdl_next = true;
   }
   CUtensorMap tm_x, tm_g, tm_u, tm_h, tm_d;
-  const int n_tile2 = kGemm2NTile;
   if (!make_tmap(&tm_x, a_src, max_rows, H, BM) ||
       !make_tmap(&tm_g, w_gate, static_cast<uint64_t>(E) * F, H, 128) ||
       !make_tmap(&tm_u, w_up, static_cast<uint64_t>(E) * F, H, 128) ||
       !make_tmap(&tm_h, h, max_rows, F, BM) ||
-      !make_tmap(&tm_d, w_down, static_cast<uint64_t>(E) * H, F, n_tile2))
+      !make_tmap(&tm_d, w_down, static_cast<uint64_t>(E) * H, F, kGemm2NTile))
     return cudaErrorInvalidValue;
-
-  GemmArgs g1{expert_offsets, E, max_rows, F, H, 128, F, h, status};
-  cudaError_t err = launch_gemm<kSwiGLU>(tm_x, tm_g, tm_u, g1, s);
+  FfnArgs fa{expert_offsets, E, max_rows, H, F, h, static_cast<__nv_bfloat16*>(expert_out), status,
+             done};
+  const size_t smem = fused_smem_bytes(E);
+  err = cudaFuncSetAttribute(fused_ffn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  GemmArgs g2{expert_offsets, E, max_rows, H, F, n_tile2, H,
-              static_cast<__nv_bfloat16*>(expert_out), status};
-  return launch_gemm<kPlain>(tm_h, tm_d, tm_d, g2, s);
+  err = launch_pdl_if(pdl_next, fused_ffn_kernel, dim3(num_sms()), dim3(kThreads), smem, s, tm_x,
+                      tm_g, tm_u, tm_h, tm_d, fa);
+  if (err != cudaSuccess) return err;
+  return cudaGetLastError();
 }
 
 }  // namespace moe

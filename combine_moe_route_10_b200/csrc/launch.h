@@ -68,8 +68,8 @@ cudaError_t launch_combine(const void* expert_out, int max_rows, const int32_t* 
                            const float* topk_w, int T, int k, int H, void* y, cudaStream_t s);
 
 // FFN workspace layout: [0,4) status, [256, ..) h [max_rows, F] bf16, then for the FP8 payload the
-// dequantised rows [max_rows, H] bf16.
-size_t ffn_workspace_bytes(int max_rows, int H, int F, int fp8);
+// dequantised rows [max_rows, H] bf16, then the GEMM-1 completion counters.
+size_t ffn_workspace_bytes(int max_rows, int H, int F, int fp8, int E);
 
 cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp8,
                               const int32_t* expert_offsets, int max_rows, int E, int H, int F,
