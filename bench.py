@@ -99,6 +99,26 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------------------------
+def max_over_ranks(local_ms: float, device) -> float:
+    """The slowest rank's time (all ranks call this together; a single process returns its own)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(local_ms)
+    t = torch.tensor([float(local_ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(local_ms: float, tokens_per_rank: int, steps: int, device) -> dict:
+    """Whole-job throughput of independent replicas: every rank's tokens over the slowest rank's
+    time (weak scaling)."""
+    import torch.distributed as dist
+    world = dist.get_world_size() if dist.is_available() and dist.is_initialized() else 1
+    ms = max_over_ranks(local_ms, device)
+    return {"value": world * tokens_per_rank * steps / (ms * 1e-3), "ms_per_step": ms / steps,
+            "total_ms": ms, "n_ranks": world}
+
+
 def algorithmic(w, S: int, active_experts: int):
     """Algorithmic bytes / flops per step of each stage (what the stage must move or compute)."""
     fp8 = w.payload == "fp8"
@@ -279,11 +299,8 @@ def main():
     if world > 1:
         dist.barrier()
     stage_ms = [[e[j].elapsed_time(e[j + 1]) for j in range(n_ev - 1)] for e in evs]
-    total_ms = sum(sum(s) for s in stage_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    agg = aggregate(sum(sum(s) for s in stage_ms), w.T, args.steps, dev)
+    total_ms = agg["total_ms"]
     mean_stage = [sum(s[j] for s in stage_ms) / args.steps for j in range(n_ev - 1)]
 
     # end to end through the public API: pinned host inputs in, result back to pinned host memory
@@ -306,19 +323,15 @@ def main():
             e2e_ev[i - 2][1].record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e = aggregate(sum(a.elapsed_time(b) for a, b in e2e_ev), w.T, e2e_steps, dev)
     st = m.status()
     if st != 0:
         raise SystemExit(f"device status {st} after timing")
 
     pk, pk_src = peaks()
     alg = algorithmic(w, S, active)
-    ms = total_ms / args.steps
-    value = world * w.T * args.steps / (total_ms * 1e-3)
+    ms = agg["ms_per_step"]
+    value = agg["value"]
     t_route, t_disp, t_ffn, t_comb = mean_stage
     hbm = pk["hbm_gbs"]
     ffn_t_hbm = alg["ffn_bytes"] / (hbm * 1e9)
@@ -361,7 +374,7 @@ def main():
         "roofline": roof,
         "stages": shuffle,
         "kept_rows": S, "active_experts": active,
-        "e2e": {"value": world * w.T * e2e_steps / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": e2e["value"], "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
