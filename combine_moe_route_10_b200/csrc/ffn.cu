@@ -190,7 +190,8 @@ struct FfnArgs {
   __nv_bfloat16* h;               // [max_rows, F] workspace
   __nv_bfloat16* out;             // [max_rows, H]
   int* status;
-  int* done;                      // [sum of row blocks] GEMM-1 completion counters, zero on entry
+  int* done;                      // [row blocks] GEMM-1 completion counters, zero on entry
+  int* used;                      // [row blocks] GEMM-2 tiles that passed the wait, zero on entry
 };
 
 struct FSmem {
@@ -423,6 +424,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           // the rows of h this tile reads are complete once all GEMM-1 tiles of (e, m) are
           if (!wait_counter(args.done + t.mg, 4 * n1, abort_flag, args.status)) break;
           asm volatile("fence.proxy.async.global;" ::: "memory");
+          // the last of the n2 GEMM-2 tiles of (e, m) to get here returns both counters to zero,
+          // so the workspace is ready for the next call without a memset
+          if (atomicAdd(args.used + t.mg, 1) == n2 - 1) {
+            atomicExch(args.done + t.mg, 0);
+            atomicExch(args.used + t.mg, 0);
+          }
           nkb = kb2;
           ma = &tm_h;
           mb = &tm_d;
@@ -649,7 +656,8 @@ bool make_tmap(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t cols, u
 }  // namespace
 
 // Workspace: [0,4) status | [256, ..) h bf16 [max_rows, F] | (FP8) dequantised rows bf16
-// [max_rows, H] | GEMM-1 completion counters int32 [max_rows/128 + E + 1].
+// [max_rows, H] | GEMM-1 completion counters and GEMM-2 arrival counters, int32
+// [2][max_rows/128 + E + 1].
 static size_t round256(size_t b) { return (b + 255) / 256 * 256; }
 static size_t ffn_counter_count(int max_rows, int E) {
   return static_cast<size_t>(max_rows) / BM + static_cast<size_t>(E) + 1;
@@ -658,7 +666,7 @@ static size_t ffn_counter_count(int max_rows, int E) {
 size_t ffn_workspace_bytes(int max_rows, int H, int F, int fp8, int E) {
   const size_t h_bytes = round256(static_cast<size_t>(max_rows) * F * 2);
   const size_t x_bytes = fp8 ? round256(static_cast<size_t>(max_rows) * H * 2) : 0;
-  return 256 + h_bytes + x_bytes + round256(ffn_counter_count(max_rows, E) * sizeof(int));
+  return 256 + h_bytes + x_bytes + round256(2 * ffn_counter_count(max_rows, E) * sizeof(int));
 }
 
 cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp8,
@@ -676,11 +684,10 @@ cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp
     off += round256(static_cast<size_t>(max_rows) * H * 2);
   }
   int* done = reinterpret_cast<int*>(base + off);
-  // GEMM-1 completion counters start at zero; the next launch follows a memset, so it is an
-  // ordinary (not programmatic) launch
-  cudaError_t err = cudaMemsetAsync(done, 0, ffn_counter_count(max_rows, E) * sizeof(int), s);
-  if (err != cudaSuccess) return err;
-  bool pdl_next = false;
+  int* used = done + ffn_counter_count(max_rows, E);
+  // both counter arrays are zero on entry (zero-filled workspace, reset by the previous call)
+  cudaError_t err = cudaSuccess;
+  bool pdl_next = true;
   const void* a_src = send;
   if (fp8) {
     const long long work = static_cast<long long>(max_rows) * (H / 16);
@@ -702,7 +709,7 @@ cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp
       !make_tmap(&tm_d, w_down, static_cast<uint64_t>(E) * H, F, kGemm2NTile))
     return cudaErrorInvalidValue;
   FfnArgs fa{expert_offsets, E, max_rows, H, F, h, static_cast<__nv_bfloat16*>(expert_out), status,
-             done};
+             done, used};
   const size_t smem = fused_smem_bytes(E);
   err = cudaFuncSetAttribute(fused_ffn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));

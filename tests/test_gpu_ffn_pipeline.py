@@ -158,3 +158,19 @@ def test_pipeline_full_size_sampled_tokens(cuda, name):
         y_e[r] = ref[e][1]
     y_ref = moe.combine(y_e, sr, wt[toks], toks.size, w.H)
     assert rel_max_err(bits16(y)[toks], y_ref) <= RTOL
+
+
+def test_ffn_workspace_reused_across_calls_with_different_routing(cuda):
+    """One FFN workspace, consecutive calls whose expert offsets differ: the GEMM-1 completion
+    counters inside the workspace return to zero after every call."""
+    w = mi.get("train-small")
+    m, _ = shuffle_for(w)
+    for seed in (0, 1, 2):
+        d = mi.make_inputs(w, seed=seed, device="cuda")
+        y = m.forward(d["logits"], d["x"], d["w_gate"], d["w_up"], d["w_down"])
+        assert m.status() == 0
+        o = moe.pipeline(np_(d["logits"]), bits16(d["x"]), bits16(d["w_gate"]), bits16(d["w_up"]),
+                         bits16(d["w_down"]), w.k, w.R)
+        assert np.array_equal(np_(m.expert_offsets), o["expert_offsets"])
+        assert rel_max_err(bits16(m.expert_out)[:o["S"]], o["expert_out"]) <= RTOL
+        assert rel_max_err(bits16(y), o["y"]) <= RTOL
