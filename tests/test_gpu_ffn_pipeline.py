@@ -174,3 +174,28 @@ def test_ffn_workspace_reused_across_calls_with_different_routing(cuda):
         assert np.array_equal(np_(m.expert_offsets), o["expert_offsets"])
         assert rel_max_err(bits16(m.expert_out)[:o["S"]], o["expert_out"]) <= RTOL
         assert rel_max_err(bits16(y), o["y"]) <= RTOL
+
+
+@pytest.mark.parametrize("rows", [
+    [150, 200, 256, 129, 180, 222, 140, 255],          # every expert: two 128-row blocks
+    [150, 200, 256, 40, 300, 129, 0, 180],             # mostly two blocks, plus 1-, 3- and 0-block
+    [130, 0, 0, 0, 0, 0, 0, 0],                        # a single two-block expert
+])
+def test_ffn_two_block_experts(cuda, rows):
+    """Experts with 129..256 rows run as 256-row tiles (two MMAs sharing one weight tile) when
+    they are the majority; other experts keep 128-row tiles in the same launch."""
+    from combine_moe_route_10_b200 import MoeShuffle
+    E, H, F = len(rows), 256, 320
+    off = np.concatenate([[0], np.cumsum(rows)]).astype(np.int32)
+    S = int(off[-1])
+    g = torch.Generator(device="cuda").manual_seed(sum(rows))
+    x = mi.randn_bf16((S, H), g)
+    wg, wu = mi.randn_bf16((E, F, H), g, 0.05), mi.randn_bf16((E, F, H), g, 0.05)
+    wd = mi.randn_bf16((E, H, F), g, 0.05)
+    m = MoeShuffle(S, H, E, 1, 1, F)                   # max_rows = S
+    m.expert_ffn(wg, wu, wd, send=x, expert_offsets=torch.from_numpy(off).cuda())
+    assert m.status() == 0
+    h_ref, y_ref = moe.expert_ffn(moe.ffn_inputs(bits16(x), None, False), off, bits16(wg),
+                                  bits16(wu), bits16(wd))
+    assert rel_max_err(bits16(m.h)[:S], h_ref) <= RTOL
+    assert rel_max_err(bits16(m.expert_out)[:S], y_ref) <= RTOL
