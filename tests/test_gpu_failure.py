@@ -1,0 +1,53 @@
+"""Failure detection on the GPU without a fault: a bounded device wait is made to run out.
+
+The fused FFN's GEMM-2 tiles wait (bounded, about one second) on per-row-block completion counters
+in the workspace.  Setting those counters to a value that the GEMM-1 epilogues can never raise to
+the target is a flag that nothing sets: the waits run out, the kernel records MOE_ERR_TIMEOUT in the
+workspace status word, drains its own copies and MMAs, frees TMEM and returns.  The context stays
+usable: after re-zeroing the workspace the same call gives correct results again."""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs as mi
+from _helpers import bits16, np_, rel_max_err
+from oracle import moe
+
+pytestmark = pytest.mark.gpu
+
+
+def counter_slice(m, w):
+    """int32 view of the GEMM-1 completion counters inside the FFN workspace."""
+    def r256(b):
+        return (b + 255) // 256 * 256
+    off = 256 + r256(m.max_rows * w.F * 2)
+    if w.payload == "fp8":
+        off += r256(m.max_rows * w.H * 2)
+    n = m.max_rows // 128 + w.E + 1
+    return m.ws_ffn[off:off + 4 * n].view(torch.int32)
+
+
+def test_ffn_wait_timeout_is_reported_and_recoverable(cuda):
+    import combine_moe_route_10_b200 as pkg
+    from combine_moe_route_10_b200 import MoeShuffle
+    w = mi.get("train-small")
+    d = mi.make_inputs(w, seed=5, device="cuda")
+    m = MoeShuffle(w.T, w.H, w.E, w.k, w.R, w.F)
+    m.forward(d["logits"], d["x"], d["w_gate"], d["w_up"], d["w_down"])
+    assert m.status() == pkg.MOE_OK
+    y_ok = m.y.clone()
+
+    counter_slice(m, w).fill_(-(1 << 30))          # no GEMM-1 epilogue can reach the target now
+    torch.cuda.synchronize()
+    m.expert_ffn(d["w_gate"], d["w_up"], d["w_down"])
+    st = pkg.moe_sync_status(m.ws_ffn)
+    assert st == pkg.MOE_ERR_TIMEOUT
+    assert torch.cuda.is_available() and torch.ones(4, device="cuda").sum().item() == 4.0
+
+    m.ws_ffn.zero_()                               # documented recovery: zero-fill the workspace
+    m.forward(d["logits"], d["x"], d["w_gate"], d["w_up"], d["w_down"])
+    assert m.status() == pkg.MOE_OK
+    assert torch.equal(m.y, y_ok)
+    o = moe.pipeline(np_(d["logits"]), bits16(d["x"]), bits16(d["w_gate"]), bits16(d["w_up"]),
+                     bits16(d["w_down"]), w.k, w.R)
+    assert rel_max_err(bits16(m.y), o["y"]) <= 1e-2
