@@ -55,7 +55,7 @@ def load() -> ctypes.CDLL:
         "moe_dispatch_noalloc": (I, [P, I, I, P, I, I, I, I, I, P, P, P, P, P, P, P, P, P]),
         "moe_ffn_workspace_size": (Z, [I, I, I, I, I]),
         "moe_expert_ffn": (I, [P, P, I, P, I, I, I, I, P, P, P, P, P, Z, P]),
-        "moe_combine": (I, [P, I, P, P, I, I, I, P, P]),
+        "moe_combine": (I, [P, I, P, P, I, I, I, P, P, P]),
         "moe_sync_status": (I, [P, P]),
     }
     for name, (res, args) in sig.items():
@@ -145,10 +145,10 @@ def moe_expert_ffn(send, send_scales, payload, expert_offsets, max_rows, E, H, F
     return _check(st, "moe_expert_ffn", raise_on_error)
 
 
-def moe_combine(expert_out, max_rows, slot_row, topk_w, T, k, H, y, stream=None,
+def moe_combine(expert_out, max_rows, slot_row, topk_w, T, k, H, y, status=None, stream=None,
                 raise_on_error=True):
     st = load().moe_combine(_ptr(expert_out), max_rows, _ptr(slot_row), _ptr(topk_w), T, k, H,
-                            _ptr(y), _stream(stream))
+                            _ptr(y), _ptr(status), _stream(stream))
     return _check(st, "moe_combine", raise_on_error)
 
 

@@ -145,15 +145,18 @@ moe_status_t moe_expert_ffn(const void* send, const float* send_scales, moe_payl
 }
 
 moe_status_t moe_combine(const void* expert_out, int max_rows, const int32_t* slot_row,
-                         const float* topk_w, int T, int k, int H, void* y, moe_stream_t stream) {
+                         const float* topk_w, int T, int k, int H, void* y, int32_t* status,
+                         moe_stream_t stream) {
   if (T < 0 || k < 1 || k > kMaxK || H < 8 || max_rows < 0) return MOE_ERR_INVALID_ARG;
   if (H % 8 != 0) return MOE_ERR_UNSUPPORTED;
   if (T > 0 && (slot_row == nullptr || topk_w == nullptr || y == nullptr ||
                 (max_rows > 0 && expert_out == nullptr)))
     return MOE_ERR_INVALID_ARG;
-  if (!aligned(expert_out, 16) || !aligned(y, 16) || !aligned(slot_row, 4) || !aligned(topk_w, 4))
+  if (!aligned(expert_out, 16) || !aligned(y, 16) || !aligned(slot_row, 4) ||
+      !aligned(topk_w, 4) || !aligned(status, 4))
     return MOE_ERR_INVALID_ARG;
   return from_cuda(moe::launch_combine(expert_out, max_rows, slot_row, topk_w, T, k, H, y,
+                                       reinterpret_cast<int*>(status),
                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 

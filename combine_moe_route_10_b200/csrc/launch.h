@@ -65,7 +65,8 @@ cudaError_t launch_dispatch_parts(const void* x, int T, int H, const int32_t* to
                                   int32_t* hist, cudaStream_t s);
 
 cudaError_t launch_combine(const void* expert_out, int max_rows, const int32_t* slot_row,
-                           const float* topk_w, int T, int k, int H, void* y, cudaStream_t s);
+                           const float* topk_w, int T, int k, int H, void* y, int* status,
+                           cudaStream_t s);
 
 // FFN workspace layout: [0,4) status, [256, ..) h [max_rows, F] bf16, then for the FP8 payload the
 // dequantised rows [max_rows, H] bf16, then the GEMM-1 completion counters.

@@ -82,10 +82,11 @@ class MoeShuffle:
                             self.expert_out, self.ws_ffn, self.ws_ffn_bytes, stream)
 
     def combine(self, expert_out=None, slot_row=None, topk_w=None, stream=None):
+        # the combine reports a wait that ran out into the FFN workspace's status word
         _lib.moe_combine(self.expert_out if expert_out is None else expert_out, self.max_rows,
                          self.slot_row if slot_row is None else slot_row,
                          self.topk_w if topk_w is None else topk_w, self.T, self.k, self.H,
-                         self.y, stream)
+                         self.y, self.ws_ffn, stream)
 
     def forward(self, logits, x, w_gate, w_up, w_down, stream=None) -> torch.Tensor:
         self.route(logits, stream)

@@ -195,14 +195,18 @@ moe_status_t moe_expert_ffn(const void* send, const float* send_scales, moe_payl
  * separately (the NCCL EP page, section 2.1: the combine loops over the top-k slots and adds each
  * expert output times the token's routing weight).  A token whose slots were all dropped gives 0.
  *   expert_out bf16 [max_rows, H]; slot_row int32 [T, k]; topk_w fp32 [T, k]; y bf16 [T, H] (out)
+ *   status     optional (may be NULL) device int32 status word (e.g. the first word of a dispatch
+ *              or FFN workspace) for device-side findings, reported by moe_sync_status(status,
+ *              stream); the current combine kernel has no device-side waits and never sets it
  * Rows outside [0, max_rows) are treated as dropped.  Limits: H % 8 == 0.
  */
 moe_status_t moe_combine(const void* expert_out, int max_rows, const int32_t* slot_row,
-                         const float* topk_w, int T, int k, int H, void* y, moe_stream_t stream);
+                         const float* topk_w, int T, int k, int H, void* y, int32_t* status,
+                         moe_stream_t stream);
 
 /*
- * Synchronise `stream`, read the device status word at the start of a dispatch or FFN workspace,
- * clear it, and report it: MOE_OK, MOE_ERR_INVALID_TOPK or MOE_ERR_TIMEOUT (MOE_ERR_CUDA if the
+ * Synchronise `stream`, read the device status word at the start of a dispatch or FFN workspace
+ * (or any status word given to moe_combine / moe_dispatch_noalloc), clear it, and report it: MOE_OK, MOE_ERR_INVALID_TOPK or MOE_ERR_TIMEOUT (MOE_ERR_CUDA if the
  * stream itself failed).
  */
 moe_status_t moe_sync_status(void* ws, moe_stream_t stream);

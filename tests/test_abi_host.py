@@ -116,10 +116,12 @@ def test_ffn_and_combine_reject_bad_arguments(lib):
     assert ffn(ws_bytes=100) == pkg.MOE_ERR_WORKSPACE
     assert ffn(send=FAKE + 4) == pkg.MOE_ERR_INVALID_ARG
     comb = lambda **kw: lib.moe_combine(FAKE, 64, FAKE, FAKE, kw.get("T", 4), kw.get("k", 2),
-                                        kw.get("H", 256), kw.get("y", FAKE), None)
+                                        kw.get("H", 256), kw.get("y", FAKE), kw.get("st", None),
+                                        None)
     assert comb(k=0) == pkg.MOE_ERR_INVALID_ARG
     assert comb(H=12) == pkg.MOE_ERR_UNSUPPORTED
     assert comb(y=FAKE + 2) == pkg.MOE_ERR_INVALID_ARG
+    assert comb(st=FAKE + 2) == pkg.MOE_ERR_INVALID_ARG
     assert lib.moe_sync_status(None, None) == pkg.MOE_ERR_INVALID_ARG
 
 
