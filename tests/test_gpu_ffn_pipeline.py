@@ -199,3 +199,31 @@ def test_ffn_two_block_experts(cuda, rows):
                                   bits16(wu), bits16(wd))
     assert rel_max_err(bits16(m.h)[:S], h_ref) <= RTOL
     assert rel_max_err(bits16(m.expert_out)[:S], y_ref) <= RTOL
+
+
+@pytest.mark.parametrize("T,H,E,k,R,F,payload,cf", [
+    (0, 128, 4, 2, 2, 128, "bf16", 0.0),      # empty batch
+    (1, 128, 1, 1, 1, 128, "bf16", 0.0),      # one token, one expert: a dense SwiGLU MLP
+    (3, 64, 2, 2, 1, 64, "bf16", 0.0),        # 6 rows in all, one k-block, F below the tile
+    (5, 256, 4, 1, 2, 192, "fp8", 0.0),       # FP8 payload, tiny T
+    (64, 320, 16, 4, 4, 64, "bf16", 1.0),     # H not a multiple of 256, drops at capacity 16
+    (200, 192, 8, 8, 8, 128, "bf16", 0.0),    # k = E
+])
+def test_pipeline_edge_shapes(cuda, T, H, E, k, R, F, payload, cf):
+    from combine_moe_route_10_b200 import MoeShuffle
+    w = mi.Workload("edge", T, H, E, k, R, F, payload=payload, capacity_factor=cf)
+    d = mi.make_inputs(w, seed=9, device="cuda")
+    cap = moe.capacity(cf, T, k, E)
+    m = MoeShuffle(T, H, E, k, R, F, payload=payload, capacity=cap)
+    y = m.forward(d["logits"], d["x"], d["w_gate"], d["w_up"], d["w_down"])
+    assert m.status() == 0
+    o = moe.pipeline(np_(d["logits"]), bits16(d["x"]), bits16(d["w_gate"]), bits16(d["w_up"]),
+                     bits16(d["w_down"]), k, R, cf, payload == "fp8")
+    assert np.array_equal(np_(m.expert_offsets), o["expert_offsets"])
+    assert np.array_equal(np_(m.slot_row), o["slot_row"])
+    if T == 0:
+        assert y.numel() == 0
+        return
+    if o["S"]:
+        assert rel_max_err(bits16(m.expert_out)[:o["S"]], o["expert_out"]) <= RTOL
+    assert rel_max_err(bits16(y), o["y"]) <= RTOL
