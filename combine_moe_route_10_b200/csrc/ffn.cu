@@ -20,8 +20,9 @@
 // The tile schedule (expert, row block, column block) is derived on the device from
 // expert_offsets, so nothing is synchronised with the host.  Row blocks of an expert are the
 // fastest-varying index, so CTAs running together share weight column blocks through L2.
-// Every mbarrier wait is bounded; on a timeout the CTA records MOE status bit kStatusTimeout,
-// drains its own outstanding TMA loads and MMAs, frees TMEM and returns.
+// Every mbarrier and counter wait is bounded; on a timeout the CTA records MOE status bit
+// kStatusTimeout, drains its own outstanding TMA loads and MMAs, frees TMEM and returns.
+// For the FP8 payload a separate pass (dequant_fp8_kernel) first writes the bf16 input rows.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_fp8.h>
