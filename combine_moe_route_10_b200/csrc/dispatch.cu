@@ -8,18 +8,22 @@
 // ThunderEP page's section 2.2: each rank keeps only its own slice of the routing table).
 //
 // Two kernels, no host synchronisation, no order-dependent atomics in any result.  Slots are cut
-// into chunks of C tokens (about 2048 slots per chunk).
+// into chunks of C tokens (C * k <= 2048 slots).
 //   1. count: one CTA per chunk writes the chunk's expert histogram hist[chunk][E].
-//   2. rank_permute: one CTA per `tile` tokens.  Before waiting for the count kernel (inputs only):
-//      L2 prefetch of its token rows, the per-expert count of the chunk's slots before its first
-//      token, and the warp-synchronous (__match_any) ranking of its own slots, giving each slot its
-//      position relative to the chunk start.  After the wait: from hist, every CTA derives its
-//      chunk's base position per expert and the expert totals, applies the capacity, scans the kept
-//      counts into expert offsets (CTA 0 also writes counts / offsets / rank offsets), turns
-//      positions into rows (position >= capacity: dropped, -1), writes slot_row / row_token, and
-//      copies the rows (bf16) or quantises them per 128-element block to e4m3 with an fp32 scale
-//      (FP8), one warp (or a segment of a row per warp) per token.
+//   2. rank_permute: CTA b of G owns the tokens [T*b/G, T*(b+1)/G) (any length; a range may cross
+//      chunk boundaries).  Before waiting for the count kernel (inputs only): L2 prefetch of the
+//      rows its warps copy first, the per-expert count of the slots between the start of its first
+//      token's chunk and its first token, and the warp-synchronous (__match_any) ranking of its
+//      own slots in slot order, which continues that count.  After the wait: from hist, the slots
+//      of every expert in the chunks before, the expert totals, the capacity and the scanned
+//      expert offsets (CTA 0 also writes counts / offsets / rank offsets); then each slot's row
+//      (position >= capacity: dropped, -1), slot_row / row_token, and the copy of the rows (bf16)
+//      or their per-128-element e4m3 quantisation with an fp32 scale (FP8).  The CTA's token x
+//      copy-unit space is split evenly over its warps, and each warp keeps an L2 prefetch one
+//      token ahead of its copy.
 #include <cuda_fp8.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "launch.h"
@@ -29,6 +33,18 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+// Tokens per chunk are 16 * floor(128 / k), so a chunk holds at most kChunkSlotsMax slots.
+constexpr int kChunkSlotsMax = 2048;
+constexpr int kPerThread = kChunkSlotsMax / kThreads;
+// Launch shape of rank_permute (measured on B200): one wave of kCtasPerSm CTAs per SM while that
+// leaves at most kPersistMax tokens per CTA, else CTAs of kTokensPerCta tokens (many short CTAs
+// pace the L2 prefetch of large inputs better than long-lived ones); never fewer CTAs than
+// min(T, kCtasPerSm * SMs).
+constexpr int kCtasPerSm = 3;
+constexpr int kPersistMaxBf16 = 12, kPersistMaxFp8 = 1;
+constexpr int kTokensPerCta = 8;
+constexpr int kPrefetchDepth = 1;  // tokens of a warp's share prefetched ahead of its copy
+constexpr int kUnrollBf16 = 8, kUnrollFp8 = 2;  // 16-byte loads in flight per lane per step
 
 // Add 1 to hist[e] for a valid expert id (shared-memory atomics: counts are order-independent).
 __device__ __forceinline__ void hist_add(int* hist, int e, bool ok) {
@@ -179,17 +195,80 @@ __global__ void __launch_bounds__(kThreads)
   __syncthreads();
   const long long s0 = static_cast<long long>(c) * chunk_tokens * k;
   const long long s1 = static_cast<long long>(min(T, (c + 1) * chunk_tokens)) * k;
+  // a chunk holds at most kChunkSlotsMax slots: every load is issued before the first atomic
+  int ev[kPerThread];
+#pragma unroll
+  for (int i = 0; i < kPerThread; ++i) {
+    const long long s = s0 + tid + i * kThreads;
+    ev[i] = s < s1 ? __ldg(topk_idx + s) : 0;
+  }
   bool bad = false;
-  for (long long s = s0 + tid; s < s1; s += kThreads) {
-    const int e = __ldg(topk_idx + s);
-    const bool ok = static_cast<unsigned>(e) < static_cast<unsigned>(E);
-    hist_add(s_hist, e, ok);
-    bad |= !ok;
+#pragma unroll
+  for (int i = 0; i < kPerThread; ++i) {
+    if (s0 + tid + i * kThreads < s1) {
+      const bool ok = static_cast<unsigned>(ev[i]) < static_cast<unsigned>(E);
+      hist_add(s_hist, ev[i], ok);
+      bad |= !ok;
+    }
   }
   if (__syncthreads_or(bad) && tid == 0) record_status(status, kStatusInvalidTopk);
   for (int e = tid; e < E; e += kThreads) hist[static_cast<size_t>(c) * E + e] = s_hist[e];
 }
 
+// Warp 0 ranks slots [q0, q1) in slot order: s_rel[i] = running count of the slot's expert before
+// it (cnt[e] on entry counts the earlier slots), s_exp[i] = its expert or -1; cnt is advanced.
+__device__ __forceinline__ void rank_slots(const int32_t* __restrict__ topk_idx, long long q0,
+                                           long long q1, int E, int* cnt, int* s_rel,
+                                           int* s_exp) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  int e_next = q0 + lane < q1 ? __ldg(topk_idx + q0 + lane) : -1;
+  for (long long base = q0; base < q1; base += 32) {
+    const long long s = base + lane;
+    const bool valid = s < q1;
+    const int e = e_next;
+    e_next = s + 32 < q1 ? __ldg(topk_idx + s + 32) : -1;  // next round's load in flight
+    const bool ok = valid && static_cast<unsigned>(e) < static_cast<unsigned>(E);
+    const int key = ok ? e : E + lane;  // unique key for lanes without a slot
+    const unsigned peers = __match_any_sync(0xFFFFFFFFu, key);
+    int rel = -1;
+    if (ok) rel = cnt[e] + __popc(peers & lt_mask);
+    __syncwarp();
+    if (ok && lane == __ffs(peers) - 1) cnt[e] += __popc(peers);
+    __syncwarp();
+    if (valid) {
+      s_rel[s - q0] = rel;
+      s_exp[s - q0] = ok ? e : -1;
+    }
+  }
+}
+
+// The contiguous share [ubeg, uend) of n_units copy units taken by `warp`, in multiples of gran.
+__device__ __forceinline__ void warp_share(int n_units, int gran, int warp, int& ubeg, int& uend) {
+  const int per = ((n_units + kWarps - 1) / kWarps + gran - 1) / gran * gran;
+  ubeg = min(n_units, warp * per);
+  uend = min(n_units, ubeg + per);
+}
+
+// L2 prefetch of the part of token (ub / upr + j) that lies in the unit range [ub, ue) of the batch
+// starting at token tb (nothing when that part is empty).
+template <int kUnitElems>
+__device__ __forceinline__ void prefetch_share_token(const uint4* x, int tb, int H, int upr, int ub,
+                                                     int ue, int j) {
+  if (ub >= ue) return;
+  const int tt = ub / upr + j;
+  const int a = max(ub, tt * upr), b = min(ue, (tt + 1) * upr);
+  if (a >= b) return;
+  const char* p = reinterpret_cast<const char*>(x) +
+                  (static_cast<size_t>(tb + tt) * H + static_cast<size_t>(a - tt * upr) * kUnitElems) * 2;
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"((b - a) * kUnitElems * 2)
+               : "memory");
+}
+
+// Rank + permute.  CTA b of G owns the tokens [T*b/G, T*(b+1)/G), at most ceil(T/G) of them (the
+// launcher sizes the per-slot shared arrays for that).  A copy unit is a 16-byte vector (bf16) or a
+// 128-element block (FP8); the CTA's token x unit space is split evenly over the warps, so a warp
+// may finish one token and start the next.
 template <bool FP8, int UNROLL>
 __global__ void __launch_bounds__(kThreads)
     rank_permute_kernel(const int32_t* __restrict__ topk_idx, int T, int k, int E, int R, int cap,
@@ -197,52 +276,49 @@ __global__ void __launch_bounds__(kThreads)
                         int32_t* __restrict__ expert_counts, int32_t* __restrict__ expert_offsets,
                         int32_t* __restrict__ rank_offsets, int32_t* __restrict__ slot_row,
                         int32_t* __restrict__ row_token, const uint4* __restrict__ x, int H,
-                        int tile, void* __restrict__ send, float* __restrict__ send_scales) {
+                        void* __restrict__ send, float* __restrict__ send_scales, int max_slots) {
   extern __shared__ int s_mem[];
-  int* cnt = s_mem;               // [E] relative positions, then chunk base + relative count
-  int* s_off = cnt + E;           // [max(E, 4*kThreads)] kept counts, scanned into offsets
-  int* s_rel = s_off + max(E, 4 * kThreads);  // [tile*k] relative position (or -1) per slot
-  int* s_exp = s_rel + tile * k;  // [tile*k] expert per slot
+  int* cnt = s_mem;                            // [E] slots of expert e from the chunk start on
+  int* s_base = cnt + E;                       // [E] slots of expert e in earlier chunks
+  int* s_off = s_base + E;                     // [max(E, 4*kThreads)] kept counts -> offsets
+  int* s_rel = s_off + max(E, 4 * kThreads);   // [ceil(T/G)*k] relative position, then row
+  int* s_exp = s_rel + max_slots;              // [ceil(T/G)*k] expert per slot (or -1)
   __shared__ int s_warp_tot[kWarps + 1];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int t0 = blockIdx.x * tile;
-  const int t1 = min(T, t0 + tile);
+  const int t0 = static_cast<int>(static_cast<long long>(T) * blockIdx.x / gridDim.x);
+  const int t1 = static_cast<int>(static_cast<long long>(T) * (blockIdx.x + 1) / gridDim.x);
   const int c = t0 / chunk_tokens;
+  constexpr int kUnitElems = FP8 ? 128 : 8;
+  constexpr int kGran = FP8 ? 2 : 32;  // units one warp step covers per lane group
+  const int upr = H / kUnitElems;      // copy units per row
 
   // ---- before the wait: inputs only ---------------------------------------------------------------
-  if (tid < t1 - t0) {
-    const char* row = reinterpret_cast<const char*>(x) + static_cast<size_t>(t0 + tid) * H * 2;
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(row), "r"(H * 2) : "memory");
+  {
+    // L2 prefetch of the first kPrefetchDepth tokens of each warp's share
+    int ub, ue;
+    warp_share((t1 - t0) * upr, kGran, warp, ub, ue);
+    if (lane < kPrefetchDepth) prefetch_share_token<kUnitElems>(x, t0, H, upr, ub, ue, lane);
   }
   for (int e = tid; e < E; e += kThreads) cnt[e] = 0;
   __syncthreads();
-  const long long p1 = static_cast<long long>(t0) * k;
-  for (long long s = static_cast<long long>(c) * chunk_tokens * k + tid; s < p1; s += kThreads) {
-    const int e = __ldg(topk_idx + s);
-    hist_add(cnt, e, static_cast<unsigned>(e) < static_cast<unsigned>(E));
+  {
+    // slots of the chunk before t0 (at most kChunkSlotsMax): loads first, then the atomics
+    const long long pc0 = static_cast<long long>(c) * chunk_tokens * k;
+    const long long p1 = static_cast<long long>(t0) * k;
+    int ev[kPerThread];
+#pragma unroll
+    for (int i = 0; i < kPerThread; ++i) {
+      const long long s = pc0 + tid + i * kThreads;
+      ev[i] = s < p1 ? __ldg(topk_idx + s) : -1;
+    }
+#pragma unroll
+    for (int i = 0; i < kPerThread; ++i)
+      hist_add(cnt, ev[i], static_cast<unsigned>(ev[i]) < static_cast<unsigned>(E));
   }
   __syncthreads();
-  if (warp == 0) {
-    const unsigned lt_mask = (1u << lane) - 1u;
-    const long long q1 = static_cast<long long>(t1) * k;
-    for (long long base = p1; base < q1; base += 32) {
-      const long long s = base + lane;
-      const bool valid = s < q1;
-      const int e = valid ? __ldg(topk_idx + s) : -1;
-      const bool ok = valid && static_cast<unsigned>(e) < static_cast<unsigned>(E);
-      const int key = ok ? e : E + lane;  // unique key for lanes without a slot
-      const unsigned peers = __match_any_sync(0xFFFFFFFFu, key);
-      int rel = -1;
-      if (ok) rel = cnt[e] + __popc(peers & lt_mask);
-      __syncwarp();
-      if (ok && lane == __ffs(peers) - 1) cnt[e] += __popc(peers);
-      __syncwarp();
-      if (valid) {
-        s_rel[s - p1] = rel;
-        s_exp[s - p1] = ok ? e : -1;
-      }
-    }
-  }
+  if (warp == 0)
+    rank_slots(topk_idx, static_cast<long long>(t0) * k, static_cast<long long>(t1) * k, E, cnt,
+               s_rel, s_exp);
 
   // ---- after the wait: the histogram is complete ---------------------------------------------------
   griddep_wait();
@@ -256,7 +332,7 @@ __global__ void __launch_bounds__(kThreads)
       total += v;
       before += cc < c ? v : 0;
     }
-    cnt[e] = before;                                // positions of expert e before this chunk
+    s_base[e] = before;
     s_off[e] = cap > 0 ? min(total, cap) : total;   // kept rows of expert e
   }
   __syncthreads();
@@ -270,36 +346,39 @@ __global__ void __launch_bounds__(kThreads)
     for (int r = tid; r <= R; r += kThreads)
       rank_offsets[r] = (r == R) ? total_kept : s_off[r * per_rank];
   }
+
+  const long long q0 = static_cast<long long>(t0) * k;
   const int n_slots = (t1 - t0) * k;
   for (int i = tid; i < n_slots; i += kThreads) {
     const int e = s_exp[i];
     int row = -1;
     if (e >= 0) {
-      const int pos = cnt[e] + s_rel[i];
+      const int pos = s_base[e] + s_rel[i];
       if (cap == 0 || pos < cap) {
         row = s_off[e] + pos;
         row_token[row] = t0 + i / k;
       }
     }
-    slot_row[p1 + i] = row;
+    slot_row[q0 + i] = row;
     s_rel[i] = row;
   }
   __syncthreads();
-
-  // warps per token: 1 when tile >= 8, else 8/tile warps split the row into segments
-  const int wpt = tile >= kWarps ? 1 : kWarps / tile;
-  const int seg = warp % wpt;
-  const int units = FP8 ? H / 128 : H / 8;                 // 128-element blocks or 16-B vectors
-  const int per = ((units + wpt - 1) / wpt + (FP8 ? 1 : 31)) / (FP8 ? 2 : 32) * (FP8 ? 2 : 32);
-  const int ubeg = min(units, seg * per), uend = min(units, ubeg + per);
-  for (int t = t0 + warp / wpt; t < t1; t += kWarps / wpt) {
-    const int my_row = lane < k ? s_rel[(t - t0) * k + lane] : -1;
+  int ub, ue;
+  warp_share((t1 - t0) * upr, kGran, warp, ub, ue);
+  for (int u = ub; u < ue;) {
+    const int tt = u / upr, a = u - tt * upr, b = min(upr, a + (ue - u));
+    const int t = t0 + tt;
+    // keep the prefetch kPrefetchDepth tokens of the share ahead of the copy
+    if (lane == 0)
+      prefetch_share_token<kUnitElems>(x, t0, H, upr, ub, ue, tt - ub / upr + kPrefetchDepth);
+    const int my_row = lane < k ? s_rel[tt * k + lane] : -1;
     if (FP8)
-      quant_token_fp8<UNROLL>(x + static_cast<size_t>(t) * (H / 8), H, ubeg, uend, my_row,
+      quant_token_fp8<UNROLL>(x + static_cast<size_t>(t) * (H / 8), H, a, b, my_row,
                               static_cast<uint8_t*>(send), send_scales);
     else
-      copy_token_bf16<UNROLL>(x + static_cast<size_t>(t) * (H / 8), H / 8, ubeg, uend, my_row,
+      copy_token_bf16<UNROLL>(x + static_cast<size_t>(t) * (H / 8), H / 8, a, b, my_row,
                               static_cast<uint4*>(send));
+    u += b - a;
   }
 }
 
@@ -347,18 +426,20 @@ cudaError_t launch_dispatch_parts(const void* x, int T, int H, const int32_t* to
   cudaError_t err = launch_pdl(count_kernel, dim3(n_chunks), dim3(kThreads), sizeof(int) * E, s,
                                topk_idx, T, k, E, chunk_tokens, status, hist);
   if (err != cudaSuccess) return err;
-  // tokens per rank+permute CTA: about four CTAs per SM, at most 16
-  int tile = 1;
-  while (tile < kDispatchTileMax && (T + 2 * tile - 1) / (2 * tile) >= 4 * num_sms()) tile *= 2;
-  const int tiles = (T + tile - 1) / tile;
+  const long long resident = static_cast<long long>(kCtasPerSm) * num_sms();
+  long long grid_ll = T < resident ? T : resident;
+  if (T > grid_ll * (fp8 ? kPersistMaxFp8 : kPersistMaxBf16))
+    grid_ll = std::max(grid_ll, (static_cast<long long>(T) + kTokensPerCta - 1) / kTokensPerCta);
+  const int grid = static_cast<int>(grid_ll);
+  const int max_slots = static_cast<int>((T + grid_ll - 1) / grid_ll) * k;  // <= 12 * 32
   const int scan_n = E > 4 * kThreads ? E : 4 * kThreads;
-  const size_t smem = sizeof(int) * (E + scan_n + 2 * tile * k);
+  const size_t smem = sizeof(int) * (2 * E + scan_n + 2 * static_cast<size_t>(max_slots));
   const uint4* xv = static_cast<const uint4*>(x);
-  auto kern = fp8 ? rank_permute_kernel<true, 2> : rank_permute_kernel<false, 8>;
-  err = launch_pdl(kern, dim3(tiles), dim3(kThreads), smem, s, topk_idx, T, k, E, R, capacity,
+  auto kern = fp8 ? rank_permute_kernel<true, kUnrollFp8> : rank_permute_kernel<false, kUnrollBf16>;
+  err = launch_pdl(kern, dim3(grid), dim3(kThreads), smem, s, topk_idx, T, k, E, R, capacity,
                    chunk_tokens, n_chunks, static_cast<const int32_t*>(hist), expert_counts,
-                   expert_offsets, rank_offsets, slot_row, row_token, xv, H, tile, send,
-                   send_scales);
+                   expert_offsets, rank_offsets, slot_row, row_token, xv, H, send, send_scales,
+                   max_slots);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }

@@ -52,6 +52,9 @@ constexpr int kStageBytes = kATileBytes + kBTileBytes;
 #define MOE_FFN_HOT_MTILES 2
 #endif
 constexpr int kGemm2NTile = 256;  // output columns per GEMM-2 tile (128 measured slower)
+#ifndef MOE_FFN_SMALL_BOX
+#define MOE_FFN_SMALL_BOX 1
+#endif
 
 
 // ---- PTX wrappers ------------------------------------------------------------------------------
@@ -269,11 +272,24 @@ __device__ __forceinline__ bool wait_counter(const int* p, int target, volatile 
   }
 }
 
+// Tensor maps of the A operand (input rows, h) with row boxes of 16, 32 and 64: a row block with
+// few rows loads only the rows it has (the stale rows above them in shared memory feed only
+// accumulator rows the epilogue does not store).
+struct SmallBoxMaps {
+  CUtensorMap m[3];
+};
+__host__ __device__ constexpr int small_box_rows(int i) { return 16 << i; }
+__device__ __forceinline__ int small_box_index(int rows) {
+  return rows <= 16 ? 0 : (rows <= 32 ? 1 : (rows <= 64 ? 2 : 3));
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     fused_ffn_kernel(const __grid_constant__ CUtensorMap tm_x,
+                     const __grid_constant__ SmallBoxMaps tm_xs,
                      const __grid_constant__ CUtensorMap tm_g,
                      const __grid_constant__ CUtensorMap tm_u,
                      const __grid_constant__ CUtensorMap tm_h,
+                     const __grid_constant__ SmallBoxMaps tm_hs,
                      const __grid_constant__ CUtensorMap tm_d, const FfnArgs args) {
   extern __shared__ uint8_t smem_raw[];
   const int E = args.E;
@@ -303,6 +319,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_u)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_h)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_d)) : "memory");
+      for (int i = 0; i < 3; ++i) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_xs.m[i]))
+                     : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_hs.m[i]))
+                     : "memory");
+      }
     }
   } else if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -373,12 +395,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int tile = blockIdx.x; tile < total_tiles && !*abort_flag; tile += gridDim.x) {
         const FTile t = fdecode(s, E, n1, n2, tile);
         const int row_a = s.off[t.e] + t.m_blk * BM;
+        // rows of this block: the A box shrinks to 16 / 32 / 64 rows when that covers them
+        const int bi = MOE_FFN_SMALL_BOX
+                           ? small_box_index(min(BM, s.off[t.e + 1] - row_a))
+                           : 3;
+        const uint32_t stage_tx = (bi < 3 ? small_box_rows(bi) * BK * 2 : kATileBytes) + kBTileBytes;
         int nkb;
         const CUtensorMap *ma, *mb;
         int row_b;
         if (t.phase == 1) {
           nkb = kb1;
-          ma = &tm_x;
+          ma = bi < 3 ? &tm_xs.m[bi] : &tm_x;
           mb = &tm_g;
           row_b = t.e * args.F + t.n_blk * 128;
         } else {
@@ -392,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             atomicExch(args.used + t.mg, 0);
           }
           nkb = kb2;
-          ma = &tm_h;
+          ma = bi < 3 ? &tm_hs.m[bi] : &tm_h;
           mb = &tm_d;
           row_b = t.e * args.H + t.n_blk * 256;
         }
@@ -405,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t a_dst = tiles_base + stage * kStageBytes;
           const uint32_t b_dst = a_dst + kATileBytes;
           const uint32_t fb = smem_addr(&s.full[stage]);
-          mbar_arrive_expect_tx(fb, kStageBytes);
+          mbar_arrive_expect_tx(fb, stage_tx);
           tma_load_2d(a_dst, ma, fb, kb * BK, row_a);
           tma_load_2d(b_dst, mb, fb, kb * BK, row_b);
           if (t.phase == 1) tma_load_2d(b_dst + kBTileBytes / 2, &tm_u, fb, kb * BK, row_b);
@@ -663,6 +690,11 @@ cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp
     pdl_next = true;
   }
   CUtensorMap tm_x, tm_g, tm_u, tm_h, tm_d;
+  SmallBoxMaps tm_xs, tm_hs;
+  for (int i = 0; i < 3; ++i)
+    if (!make_tmap(&tm_xs.m[i], a_src, max_rows, H, small_box_rows(i)) ||
+        !make_tmap(&tm_hs.m[i], h, max_rows, F, small_box_rows(i)))
+      return cudaErrorInvalidValue;
   if (!make_tmap(&tm_x, a_src, max_rows, H, BM) ||
       !make_tmap(&tm_g, w_gate, static_cast<uint64_t>(E) * F, H, 128) ||
       !make_tmap(&tm_u, w_up, static_cast<uint64_t>(E) * F, H, 128) ||
@@ -676,7 +708,7 @@ cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp
                              static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   err = launch_pdl_if(pdl_next, fused_ffn_kernel, dim3(num_sms()), dim3(kThreads), smem, s, tm_x,
-                      tm_g, tm_u, tm_h, tm_d, fa);
+                      tm_xs, tm_g, tm_u, tm_h, tm_hs, tm_d, fa);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }

@@ -47,7 +47,6 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int renorm, i
 // Dispatch workspace layout (bytes from the 256-byte-aligned base):
 //   [0, 4)    status word (kStatus* bits)
 //   [256, ..) per-chunk expert histogram [n_chunks][E] int32, chunks of dispatch_chunk_tokens(k)
-constexpr int kDispatchTileMax = 16;  // max tokens per rank+permute CTA (divides every chunk)
 int dispatch_chunk_tokens(int k);     // 16 * floor(128 / k), at least 16: ~2048 slots per chunk
 size_t dispatch_workspace_bytes(int T, int E, int k);
 

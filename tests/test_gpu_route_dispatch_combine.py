@@ -131,7 +131,7 @@ def test_dispatch_parity(cuda, name):
 
 
 @pytest.mark.parametrize("case", ["one_expert", "cap1", "k_eq_E", "T1", "empty_experts",
-                                  "ragged_T", "fp8_subnormal"])
+                                  "ragged_T", "fp8_subnormal", "many_slots", "many_slots_fp8"])
 def test_dispatch_edge_cases(cuda, case):
     g = np.random.default_rng(7)
     T, H, E, k, R, cap, fp8 = 300, 256, 8, 2, 4, 0, False
@@ -155,6 +155,12 @@ def test_dispatch_edge_cases(cuda, case):
         idx = np.argsort(-(g.random((T, E)) + (np.arange(E) < 4) * 0.5), 1)[:, :k].astype(np.int32)
     elif case == "fp8_subnormal":
         fp8, H = True, 384
+        idx = np.argsort(-g.random((T, E)), 1)[:, :k].astype(np.int32)
+    elif case in ("many_slots", "many_slots_fp8"):
+        # 1.9M slots, k = 32: thousands of rank/permute CTAs, each 256 slots spread over 64 experts
+        T, E, k, R = 60000, 64, 32, 8
+        fp8 = case == "many_slots_fp8"
+        H, cap = (128, 25000) if fp8 else (64, 0)
         idx = np.argsort(-g.random((T, E)), 1)[:, :k].astype(np.int32)
     xf = g.normal(size=(T, H)).astype(np.float32)
     if case == "fp8_subnormal":
