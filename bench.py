@@ -31,6 +31,11 @@ import moe_inputs as mi  # noqa: E402
 METRIC = "dispatch+FFN+combine tokens/s and shuffle HBM GB/s (% of roofline) on 1 B200"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = mi.l2_flush_bytes()
+# DRAM read + write bytes per call of the FFN stage (fused_ffn_kernel, plus dequant_fp8_kernel for
+# the FP8 payload) at full size: ncu dram__bytes_read.sum + dram__bytes_write.sum, one capture of
+# `bench.py --workload <w> --steps 3 --warmup 3` on B200, kernels as built from this tree.  To be
+# reset to None whenever either kernel changes.
+FFN_TRAFFIC = {"decode": 2.839e9, "train": 3.668e9, "finegrained": 14.86e9, "skewed": 13.89e9}
 
 
 # ---------------------------------------------------------------------------------------------
@@ -219,7 +224,10 @@ def config_of(w, args):
     return {"workload": w.name, "T": w.T, "H": w.H, "E": w.E, "k": w.k, "R": w.R, "F": w.F,
             "payload": w.payload, "capacity": cap, "bias": w.bias,
             "parallelism": f"replicas x{args.gpus} (ranks emulated inside each GPU)",
-            "l2": "flushed (256 MB write) before every timed step"}
+            "l2": ("flushed before every timed step: 256 MB written" +
+                   (", then another 256 MB buffer read (its clean lines evict the written ones, so "
+                    "no flush data is written back inside the timed region)"
+                    if args.flush == "write-read" else ""))}
 
 
 # ---------------------------------------------------------------------------------------------
@@ -231,6 +239,7 @@ def main():
     ap.add_argument("--workload", default="decode", choices=sorted(mi.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--flush", default="write-read", choices=["write", "write-read"])
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -258,7 +267,14 @@ def main():
                 if w.capacity_factor else 0)
     m = MoeShuffle(w.T, w.H, w.E, w.k, w.R, w.F, payload=w.payload, capacity=cap_rows, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    flush_rd = (torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+                if args.flush == "write-read" else None)
     stream = torch.cuda.current_stream(dev)
+
+    def flush_l2():
+        flush.fill_(1)
+        if flush_rd is not None:
+            flush_rd.sum()  # evicts the dirty lines of the write, leaving clean ones
 
     def step():
         m.route(d["logits"])
@@ -269,7 +285,7 @@ def main():
     sampler = ClockSampler(local)
     sampler.start()
     for _ in range(args.warmup):
-        flush.fill_(1)
+        flush_l2()
         step()
     torch.cuda.synchronize()
     st = m.status()
@@ -291,11 +307,11 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     for i in range(args.steps):
-        flush.fill_(1)
+        flush_l2()
         step_ev[i][0].record(stream)
         step()
         step_ev[i][1].record(stream)
-        flush.fill_(1)
+        flush_l2()
         e = evs[i]
         e[0].record(stream)
         m.route(d["logits"])
@@ -382,8 +398,9 @@ def main():
         p = pk["bf16_tflops_sustained"]
         roof = {"bound": "tensor", "achieved": ach, "peak": p, "unit": "TFLOP/s", "frac": ach / p}
     roof.update({
-        "kernel": "grouped_gemm_kernel x2 (GEMM-1 gate/up + SwiGLU, GEMM-2 down) = moe_expert_ffn",
-        "traffic": None, "peak_source": pk_src,
+        "kernel": ("fused_ffn_kernel (one persistent launch: GEMM-1 gate|up + SwiGLU, GEMM-2 down)"
+                   + (" + dequant_fp8_kernel" if w.payload == "fp8" else "") + " = moe_expert_ffn"),
+        "traffic": FFN_TRAFFIC.get(w.name), "peak_source": pk_src,
         "algorithmic_bytes": alg["ffn_bytes"], "algorithmic_flops": alg["ffn_flops"],
         "frac_of_max_time_bound": max(ffn_t_hbm, ffn_t_tc) / (t_ffn * 1e-3)})
 
