@@ -240,6 +240,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--flush", default="write-read", choices=["write", "write-read"])
+    ap.add_argument("--e2e-eager", action="store_true",
+                    help="end-to-end loop calls forward eagerly instead of replaying CUDA graphs")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -341,6 +343,10 @@ def main():
     y_stage = [torch.empty_like(m.y) for _ in range(2)]
     up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     e2e_steps = max(3, min(args.steps, 50))
+    # each buffer slot's step (forward + copy of y) is one captured CUDA graph (--e2e-eager: not)
+    graphs = (None if args.e2e_eager else
+              [m.capture(logits_d[b], x_d[b], d["w_gate"], d["w_up"], d["w_down"], out=y_stage[b])
+               for b in range(2)])
 
     def e2e_loop(n):
         ev = lambda: torch.cuda.Event()  # noqa: E731
@@ -360,10 +366,15 @@ def main():
                 x_d[b].copy_(x_h, non_blocking=True)
                 h2d[b].record(up)
             stream.wait_event(h2d[b])
-            m.forward(logits_d[b], x_d[b], d["w_gate"], d["w_up"], d["w_down"])
-            if i >= 2:
-                stream.wait_event(d2h[b])          # step i-2's download finished reading y_stage[b]
-            y_stage[b].copy_(m.y)
+            if graphs is not None:
+                if i >= 2:
+                    stream.wait_event(d2h[b])      # step i-2's download finished reading y_stage[b]
+                graphs[b].replay()
+            else:
+                m.forward(logits_d[b], x_d[b], d["w_gate"], d["w_up"], d["w_down"])
+                if i >= 2:
+                    stream.wait_event(d2h[b])      # step i-2's download finished reading y_stage[b]
+                y_stage[b].copy_(m.y)
             fwd[b].record(stream)
             with torch.cuda.stream(down):
                 down.wait_event(fwd[b])
@@ -433,7 +444,9 @@ def main():
                        "ms_per_step come from the metric steps' boundary events only",
         "kept_rows": S, "active_experts": active,
         "e2e": {"value": e2e["value"], "unit": "tokens/s",
-                "method": "uploads/downloads on two copy streams, double-buffered, overlapping "
+                "method": ("each step one replay of a captured CUDA graph (forward + copy of y); "
+                           if not args.e2e_eager else "eager forward per step; ") +
+                          "uploads/downloads on two copy streams, double-buffered, overlapping "
                           "the neighbouring steps' compute; L2 not flushed inside this loop (each "
                           f"step streams {alg['ffn_weight_bytes'] / 1e9:.2f} GB of weights)",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

@@ -95,6 +95,23 @@ class MoeShuffle:
         self.combine(stream=stream)
         return self.y
 
+    def capture(self, logits, x, w_gate, w_up, w_down, out=None) -> torch.cuda.CUDAGraph:
+        """Record ``forward`` on these exact tensors (and, if given, ``out.copy_(y)``) as a CUDA graph.
+
+        ``replay()`` of the returned graph reruns the whole step with one launch from the host: new
+        inputs are written into the same ``logits`` / ``x`` tensors before each replay.  The step
+        allocates nothing and never synchronises, and the FFN's counters return to zero inside
+        every call, so a replay needs no reset.  One eager call runs first, outside the capture.
+        """
+        self.forward(logits, x, w_gate, w_up, w_down)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.forward(logits, x, w_gate, w_up, w_down)
+            if out is not None:
+                out.copy_(self.y)
+        return g
+
     def status(self, stream=None) -> int:
         """Synchronise and return (then clear) the device status of the dispatch and FFN stages."""
         a = _lib.moe_sync_status(self.ws_dispatch, stream)
