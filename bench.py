@@ -35,7 +35,7 @@ L2_FLUSH_BYTES = mi.l2_flush_bytes()
 # the FP8 payload) at full size: ncu dram__bytes_read.sum + dram__bytes_write.sum, one capture of
 # `bench.py --workload <w> --steps 3 --warmup 3` on B200, kernels as built from this tree.  To be
 # reset to None whenever either kernel changes.
-FFN_TRAFFIC = {"decode": 2.839e9, "train": 3.668e9, "finegrained": 14.86e9, "skewed": 13.89e9}
+FFN_TRAFFIC = {}
 
 
 # ---------------------------------------------------------------------------------------------

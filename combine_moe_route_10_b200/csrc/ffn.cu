@@ -8,9 +8,12 @@
 //     h = bf16( silu(x W_gate[e]^T) * (x W_up[e]^T) ),   expert_out = bf16( h W_down[e]^T ).
 //
 // One persistent launch (one CTA per SM, 192 threads) runs the GEMM-1 tiles and then the GEMM-2
-// tiles (the latter wait on per-row-block completion counters of the former):
-//   warp 0      TMA producer: A tile (128 rows x 64 k) + B tile (256 rows x 64 k) per stage,
-//               128-byte swizzle, 4-stage mbarrier ring;
+// tiles (the latter wait on per-row-block completion counters of the former); each CTA claims its
+// next tile at run time from a global counter:
+//   warp 0      TMA producer: claims tiles, passes their ids to the other roles through a small
+//               shared-memory queue, and loads an A tile (128 rows x 64 k; 16/32/64 rows for a
+//               small row block) + B tile (256 rows x 64 k) per stage, 128-byte swizzle, 4-stage
+//               mbarrier ring;
 //   warp 1      TMEM allocator and MMA issuer: one thread issues tcgen05.mma (M=128, N=256,
 //               K=16, bf16 -> fp32) into one of two 256-column TMEM accumulators, and
 //               tcgen05.commit frees smem stages / publishes finished accumulators;
@@ -52,6 +55,13 @@ constexpr int kStageBytes = kATileBytes + kBTileBytes;
 #define MOE_FFN_HOT_MTILES 2
 #endif
 constexpr int kGemm2NTile = 256;  // output columns per GEMM-2 tile (128 measured slower)
+// Tiles are claimed at run time from a global counter (1) or taken statically blockIdx.x + i*grid
+// (0).  The producer claims; a kTileQ-deep shared-memory queue passes the ids to the MMA thread and
+// the epilogue warps.
+#ifndef MOE_FFN_DYNAMIC
+#define MOE_FFN_DYNAMIC 1
+#endif
+constexpr int kTileQ = 4;
 #ifndef MOE_FFN_SMALL_BOX
 #define MOE_FFN_SMALL_BOX 1
 #endif
@@ -140,13 +150,13 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
 
 // ---- fused FFN: GEMM-1 (gate|up + SwiGLU) and GEMM-2 (down) tiles in one persistent launch -------
 //
-// Tiles are numbered [all GEMM-1 tiles][all GEMM-2 tiles]; each CTA takes tiles blockIdx.x,
-// blockIdx.x + gridDim.x, ... in increasing order.  A GEMM-2 tile (expert e, row block m) reads the
-// rows of h that the GEMM-1 tiles of (e, m) write, so its producer first waits (bounded) until the
-// completion counter of (e, m) reaches 4 * n1 (four epilogue warps per GEMM-1 tile, n1 column
-// blocks).  GEMM-1 tiles never wait, and every CTA finishes its GEMM-1 tiles before it reaches its
-// GEMM-2 tiles, so with all CTAs resident (one per SM) the waits always end; they are bounded
-// anyway.  Writers: st.global of h, fence.proxy.async (generic -> async proxy), release increment.
+// Tiles are numbered [all GEMM-1 tiles][all GEMM-2 tiles]; CTAs claim them in increasing order
+// (atomic counter; with MOE_FFN_DYNAMIC 0, statically blockIdx.x, blockIdx.x + gridDim.x, ...).
+// A GEMM-2 tile (expert e, row block m) reads the rows of h that the GEMM-1 tiles of (e, m) write,
+// so its producer first waits (bounded) until the completion counter of (e, m) reaches 4 * n1 (four
+// epilogue warps per GEMM-1 tile, n1 column blocks).  GEMM-1 tiles never wait, and every GEMM-1
+// tile is claimed before any GEMM-2 tile, by a CTA that finishes it without waiting, so with all
+// CTAs resident (one per SM) the waits always end; they are bounded anyway.  Writers: st.global of h, fence.proxy.async (generic -> async proxy), release increment.
 // Readers: acquire load of the counter, fence.proxy.async, then the TMA loads of h.
 struct FfnArgs {
   const int32_t* expert_offsets;  // [E+1], device
@@ -156,11 +166,13 @@ struct FfnArgs {
   int* status;
   int* done;                      // [row blocks] GEMM-1 completion counters, zero on entry
   int* used;                      // [row blocks] GEMM-2 tiles that passed the wait, zero on entry
+  int* sched;                     // [2] next tile to claim, CTAs that finished; zero on entry
 };
 
 struct FSmem {
   uint8_t* tiles;
-  uint64_t *full, *empty, *acc_full, *acc_empty, *drain;
+  uint64_t *full, *empty, *acc_full, *acc_empty, *drain, *q_full, *q_empty;
+  int* tile_q;   // [kTileQ] claimed tile ids (-1: no more tiles)
   uint32_t* tmem_base;
   int* abort_flag;
   int* off;      // [E+1] row offsets (clamped to max_rows)
@@ -182,9 +194,12 @@ __device__ __forceinline__ FSmem fcarve(uint8_t* raw, int E) {
   s.acc_full = s.empty + kStages;
   s.acc_empty = s.acc_full + 2;
   s.drain = s.acc_empty + 2;
-  s.tmem_base = reinterpret_cast<uint32_t*>(s.drain + 1);
+  s.q_full = s.drain + 1;
+  s.q_empty = s.q_full + kTileQ;
+  s.tmem_base = reinterpret_cast<uint32_t*>(s.q_empty + kTileQ);
   s.abort_flag = reinterpret_cast<int*>(s.tmem_base + 1);
-  s.off = s.abort_flag + 2;
+  s.tile_q = s.abort_flag + 2;
+  s.off = s.tile_q + kTileQ;
   s.mt = s.off + (E + 1);
   s.ms_all = s.mt + E;
   s.ms_cold = s.ms_all + (E + 1);
@@ -194,8 +209,8 @@ __device__ __forceinline__ FSmem fcarve(uint8_t* raw, int E) {
 }
 
 size_t fused_smem_bytes(int E) {
-  return 1024 + static_cast<size_t>(kStages) * kStageBytes + 8 * (2 * kStages + 5) + 16 +
-         sizeof(int) * (5 * static_cast<size_t>(E) + 8);
+  return 1024 + static_cast<size_t>(kStages) * kStageBytes + 8 * (2 * kStages + 5 + 2 * kTileQ) +
+         16 + sizeof(int) * (5 * static_cast<size_t>(E) + 8 + kTileQ);
 }
 
 struct FTile {
@@ -311,6 +326,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(smem_addr(&s.acc_empty[i]), 4);
       }
       mbar_init(smem_addr(s.drain), 1);
+      for (int i = 0; i < kTileQ; ++i) {
+        mbar_init(smem_addr(&s.q_full[i]), 1);
+        mbar_init(smem_addr(&s.q_empty[i]), 5);  // the MMA thread and the four epilogue warps
+      }
       *s.abort_flag = 0;
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -392,7 +411,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_parity = 0;
-      for (int tile = blockIdx.x; tile < total_tiles && !*abort_flag; tile += gridDim.x) {
+      int qi = 0;
+      uint32_t qph = 0;
+      for (int next = blockIdx.x; !*abort_flag; next += gridDim.x) {
+        int tile = MOE_FFN_DYNAMIC ? atomicAdd(args.sched, 1) : next;
+        if (tile >= total_tiles) tile = -1;
+        // hand the id to the MMA thread and the epilogue warps
+        if (!wait_phase(smem_addr(&s.q_empty[qi]), qph ^ 1u, abort_flag, args.status)) break;
+        s.tile_q[qi] = tile;
+        mbar_arrive(smem_addr(&s.q_full[qi]));
+        if (++qi == kTileQ) {
+          qi = 0;
+          qph ^= 1u;
+        }
+        if (tile < 0) break;
         const FTile t = fdecode(s, E, n1, n2, tile);
         const int row_a = s.off[t.e] + t.m_blk * BM;
         // rows of this block: the A box shrinks to 16 / 32 / 64 rows when that covers them
@@ -461,7 +493,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       int it = 0;
       bool issued_any = false;
-      for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
+      int qi = 0;
+      uint32_t qph = 0;
+      for (;; ++it) {
+        if (!wait_phase(smem_addr(&s.q_full[qi]), qph, abort_flag, args.status)) break;
+        const int tile = s.tile_q[qi];
+        mbar_arrive(smem_addr(&s.q_empty[qi]));
+        if (++qi == kTileQ) {
+          qi = 0;
+          qph ^= 1u;
+        }
+        if (tile < 0) break;
         const int nkb = tile < (s.totals[0] + s.totals[1]) * n1 ? kb1 : kb2;
         const int acc = it & 1;
         const uint32_t acc_parity = (it >> 1) & 1;
@@ -503,7 +545,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;
     const int r_local = quarter * 32 + lane;
     int it = 0;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
+    int qi = 0;
+    uint32_t qph = 0;
+    for (;; ++it) {
+      int tile = -1;
+      bool okq = true;
+      if (lane == 0) {
+        okq = wait_phase(smem_addr(&s.q_full[qi]), qph, abort_flag, args.status);
+        if (okq) {
+          tile = s.tile_q[qi];
+          mbar_arrive(smem_addr(&s.q_empty[qi]));
+        }
+      }
+      if (++qi == kTileQ) {
+        qi = 0;
+        qph ^= 1u;
+      }
+      okq = __shfl_sync(0xFFFFFFFFu, okq ? 1 : 0, 0) != 0;
+      tile = __shfl_sync(0xFFFFFFFFu, tile, 0);
+      if (!okq || tile < 0) break;
       const FTile t = fdecode(s, E, n1, n2, tile);
       const int acc = it & 1;
       const uint32_t acc_parity = (it >> 1) & 1;
@@ -570,6 +630,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) {
+    // every claim of this CTA is done: the last CTA to get here returns the counters to zero
+    __threadfence();
+    if (atomicAdd(args.sched + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+      atomicExch(args.sched, 0);
+      atomicExch(args.sched + 1, 0);
+    }
+  }
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
@@ -645,7 +713,7 @@ bool make_tmap(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t cols, u
 
 // Workspace: [0,4) status | [256, ..) h bf16 [max_rows, F] | (FP8) dequantised rows bf16
 // [max_rows, H] | GEMM-1 completion counters and GEMM-2 arrival counters, int32
-// [2][max_rows/128 + E + 1].
+// [2][max_rows/128 + E + 1] | tile-claim counter and finished-CTA counter, int32 [2].
 static size_t round256(size_t b) { return (b + 255) / 256 * 256; }
 static size_t ffn_counter_count(int max_rows, int E) {
   return static_cast<size_t>(max_rows) / BM + static_cast<size_t>(E) + 1;
@@ -654,7 +722,7 @@ static size_t ffn_counter_count(int max_rows, int E) {
 size_t ffn_workspace_bytes(int max_rows, int H, int F, int fp8, int E) {
   const size_t h_bytes = round256(static_cast<size_t>(max_rows) * F * 2);
   const size_t x_bytes = fp8 ? round256(static_cast<size_t>(max_rows) * H * 2) : 0;
-  return 256 + h_bytes + x_bytes + round256(2 * ffn_counter_count(max_rows, E) * sizeof(int));
+  return 256 + h_bytes + x_bytes + round256((2 * ffn_counter_count(max_rows, E) + 2) * sizeof(int));
 }
 
 cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp8,
@@ -673,7 +741,8 @@ cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp
   }
   int* done = reinterpret_cast<int*>(base + off);
   int* used = done + ffn_counter_count(max_rows, E);
-  // both counter arrays are zero on entry (zero-filled workspace, reset by the previous call)
+  int* sched = used + ffn_counter_count(max_rows, E);
+  // all counters are zero on entry (zero-filled workspace, reset by the previous call)
   cudaError_t err = cudaSuccess;
   bool pdl_next = true;
   const void* a_src = send;
@@ -702,7 +771,7 @@ cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp
       !make_tmap(&tm_d, w_down, static_cast<uint64_t>(E) * H, F, kGemm2NTile))
     return cudaErrorInvalidValue;
   FfnArgs fa{expert_offsets, E, max_rows, H, F, h, static_cast<__nv_bfloat16*>(expert_out), status,
-             done, used};
+             done, used, sched};
   const size_t smem = fused_smem_bytes(E);
   err = cudaFuncSetAttribute(fused_ffn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));

@@ -181,8 +181,9 @@ size_t moe_ffn_workspace_size(int max_rows, int E, int H, int F, moe_payload_t p
  *   ws, ws_bytes   device scratch >= moe_ffn_workspace_size(...), 256-byte aligned, zero-filled once
  * Limits: H % 64 == 0, F % 64 == 0 (else MOE_ERR_UNSUPPORTED), E <= 1024,
  * expert_offsets[E] <= max_rows (rows beyond max_rows are not computed).
- * The workspace also holds per-row-block completion counters that every successful call leaves at
- * zero; after a call that reported MOE_ERR_TIMEOUT, zero-fill the workspace again before reuse.
+ * The workspace also holds per-row-block completion counters and the tile-claim counters of the
+ * kernel's run-time tile scheduler, which every successful call leaves at zero; after a call that
+ * reported MOE_ERR_TIMEOUT, zero-fill the workspace again before reuse.
  */
 moe_status_t moe_expert_ffn(const void* send, const float* send_scales, moe_payload_t payload,
                             const int32_t* expert_offsets, int max_rows, int E, int H, int F,
