@@ -55,16 +55,9 @@ constexpr int kStageBytes = kATileBytes + kBTileBytes;
 #define MOE_FFN_HOT_MTILES 2
 #endif
 constexpr int kGemm2NTile = 256;  // output columns per GEMM-2 tile (128 measured slower)
-// Tiles are claimed at run time from a global counter (1) or taken statically blockIdx.x + i*grid
-// (0).  The producer claims; a kTileQ-deep shared-memory queue passes the ids to the MMA thread and
-// the epilogue warps.
-#ifndef MOE_FFN_DYNAMIC
-#define MOE_FFN_DYNAMIC 1
-#endif
+// Tiles are claimed at run time from a global counter by the producer; a kTileQ-deep shared-memory
+// queue passes the ids to the MMA thread and the epilogue warps.
 constexpr int kTileQ = 4;
-#ifndef MOE_FFN_SMALL_BOX
-#define MOE_FFN_SMALL_BOX 1
-#endif
 
 
 // ---- PTX wrappers ------------------------------------------------------------------------------
@@ -151,7 +144,7 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
 // ---- fused FFN: GEMM-1 (gate|up + SwiGLU) and GEMM-2 (down) tiles in one persistent launch -------
 //
 // Tiles are numbered [all GEMM-1 tiles][all GEMM-2 tiles]; CTAs claim them in increasing order
-// (atomic counter; with MOE_FFN_DYNAMIC 0, statically blockIdx.x, blockIdx.x + gridDim.x, ...).
+// from an atomic counter.
 // A GEMM-2 tile (expert e, row block m) reads the rows of h that the GEMM-1 tiles of (e, m) write,
 // so its producer first waits (bounded) until the completion counter of (e, m) reaches 4 * n1 (four
 // epilogue warps per GEMM-1 tile, n1 column blocks).  GEMM-1 tiles never wait, and every GEMM-1
@@ -413,8 +406,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t issued_mask = 0, issued_parity = 0;
       int qi = 0;
       uint32_t qph = 0;
-      for (int next = blockIdx.x; !*abort_flag; next += gridDim.x) {
-        int tile = MOE_FFN_DYNAMIC ? atomicAdd(args.sched, 1) : next;
+      while (!*abort_flag) {
+        int tile = atomicAdd(args.sched, 1);
         if (tile >= total_tiles) tile = -1;
         // hand the id to the MMA thread and the epilogue warps
         if (!wait_phase(smem_addr(&s.q_empty[qi]), qph ^ 1u, abort_flag, args.status)) break;
@@ -428,9 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const FTile t = fdecode(s, E, n1, n2, tile);
         const int row_a = s.off[t.e] + t.m_blk * BM;
         // rows of this block: the A box shrinks to 16 / 32 / 64 rows when that covers them
-        const int bi = MOE_FFN_SMALL_BOX
-                           ? small_box_index(min(BM, s.off[t.e + 1] - row_a))
-                           : 3;
+        const int bi = small_box_index(min(BM, s.off[t.e + 1] - row_a));
         const uint32_t stage_tx = (bi < 3 ? small_box_rows(bi) * BK * 2 : kATileBytes) + kBTileBytes;
         int nkb;
         const CUtensorMap *ma, *mb;
