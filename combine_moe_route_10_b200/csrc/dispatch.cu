@@ -250,8 +250,8 @@ __device__ __forceinline__ void warp_share(int n_units, int gran, int warp, int&
   uend = min(n_units, ubeg + per);
 }
 
-// L2 prefetch of the part of token (ub / upr + j) that lies in the unit range [ub, ue) of the batch
-// starting at token tb (nothing when that part is empty).
+// L2 prefetch of the part of token (ub / upr + j) that lies in the unit range [ub, ue) of the token
+// range starting at token tb (nothing when that part is empty).
 template <int kUnitElems>
 __device__ __forceinline__ void prefetch_share_token(const uint4* x, int tb, int H, int upr, int ub,
                                                      int ue, int j) {
