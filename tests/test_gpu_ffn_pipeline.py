@@ -2,9 +2,9 @@
 
 The FFN runs bf16 operands on the tensor cores with fp32 accumulation; the oracle accumulates in
 fp64.  Both round h and the output to bf16.  Parity bar (per output tensor): max |gpu - ref| /
-max |ref| <= 1e-2.  Small workloads are compared on every row; the full-size workloads on sampled
-rows (the first and last row of sampled experts plus random rows), run in the same launch
-configuration as the benchmark."""
+max |ref| <= 1e-2.  Small workloads are compared on every row; the full-size workloads on every
+row too (train, skewed, finegrained FFN; decode's whole path), and on sampled rows (the first and
+last row of sampled experts plus random rows), in the same launch configuration as the benchmark."""
 import numpy as np
 import pytest
 import torch
@@ -113,6 +113,29 @@ def test_ffn_parity_full_size_sampled(cuda, name):
         assert rel_max_err(y_gpu[r], y_ref) <= RTOL, e
 
 
+@pytest.mark.parametrize("name", ["train", "skewed", "finegrained"])
+def test_ffn_parity_full_size_all_rows(cuda, name):
+    """Full size, every packed row, in the benchmark's launch configuration: train (tensor-bound;
+    experts of 300-2300 rows: full 128-row blocks and ragged last blocks), skewed (capacity-capped
+    experts of 2-3 blocks) and finegrained (FP8 payload; 256 experts from 1 row to 32 blocks).
+    The oracle runs expert by expert with that expert's weights only."""
+    w = mi.get(name)
+    d = mi.make_inputs(w, seed=0, device="cuda")
+    _, _, plan, send, scales = oracle_plan(w, d)
+    m, _ = shuffle_for(w)
+    run_gpu_ffn_on_oracle_rows(m, w, plan, send, scales, d)
+    xin = moe.ffn_inputs(send, scales, w.payload == "fp8")
+    off = plan["expert_offsets"]
+    rows = {e: np.arange(off[e], off[e + 1]) for e in range(w.E) if off[e + 1] > off[e]}
+    ref = oracle_rows(w, d, xin, rows)
+    S = plan["S"]
+    h_ref = np.concatenate([ref[e][0] for e in sorted(ref)])
+    y_ref = np.concatenate([ref[e][1] for e in sorted(ref)])
+    assert h_ref.shape[0] == S
+    assert rel_max_err(bits16(m.h)[:S], h_ref) <= RTOL
+    assert rel_max_err(bits16(m.expert_out)[:S], y_ref) <= RTOL
+
+
 @pytest.mark.parametrize("name", SMALL)
 def test_pipeline_end_to_end(cuda, name):
     w = mi.get(name)
@@ -127,6 +150,28 @@ def test_pipeline_end_to_end(cuda, name):
     assert np.array_equal(np_(m.expert_offsets), o["expert_offsets"])
     assert rel_max_err(bits16(m.expert_out)[:o["S"]], o["expert_out"]) <= RTOL
     assert rel_max_err(bits16(y), o["y"]) <= RTOL
+
+
+def test_pipeline_decode_full_size_every_token(cuda):
+    """The benchmark's default workload at full size (T=128, H=4096, E=8, F=14336, the bench's seed)
+    in the bench's launch configuration: every token and every packed row against the oracle."""
+    w = mi.get("decode")
+    d = mi.make_inputs(w, seed=0, device="cuda")
+    m, _ = shuffle_for(w)
+    y = m.forward(d["logits"], d["x"], d["w_gate"], d["w_up"], d["w_down"])
+    assert m.status() == 0
+    o = moe.pipeline(np_(d["logits"]), bits16(d["x"]), bits16(d["w_gate"]), bits16(d["w_up"]),
+                     bits16(d["w_down"]), w.k, w.R, w.capacity_factor, w.payload == "fp8")
+    assert np.array_equal(np_(m.topk_idx), o["topk_idx"])
+    assert np.array_equal(np_(m.slot_row), o["slot_row"])
+    assert np.array_equal(np_(m.expert_offsets), o["expert_offsets"])
+    assert np.array_equal(bits16(m.send)[:o["S"]], o["send"])
+    assert rel_max_err(bits16(m.h)[:o["S"]], o["h"]) <= RTOL
+    assert rel_max_err(bits16(m.expert_out)[:o["S"]], o["expert_out"]) <= RTOL
+    assert rel_max_err(bits16(y), o["y"]) <= RTOL
+    # the combine is exact given its inputs: the oracle's combine of the GPU's expert outputs
+    assert np.array_equal(bits16(y), moe.combine(bits16(m.expert_out), np_(m.slot_row),
+                                                 np_(m.topk_w), w.T, w.H))
 
 
 @pytest.mark.parametrize("name", FULL)
