@@ -343,8 +343,10 @@ def main():
     y_stage = [torch.empty_like(m.y) for _ in range(2)]
     up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     e2e_steps = max(3, min(args.steps, 50))
-    # each buffer slot's step (forward + copy of y) is one captured CUDA graph (--e2e-eager: not)
-    graphs = (None if args.e2e_eager else
+    # each buffer slot's step (forward + copy of y) is one captured CUDA graph (--e2e-eager: not;
+    # with several ranks the loop stays eager, as no graph is recorded next to a communicator)
+    use_graphs = not args.e2e_eager and world == 1
+    graphs = (None if not use_graphs else
               [m.capture(logits_d[b], x_d[b], d["w_gate"], d["w_up"], d["w_down"], out=y_stage[b])
                for b in range(2)])
 
@@ -445,7 +447,7 @@ def main():
         "kept_rows": S, "active_experts": active,
         "e2e": {"value": e2e["value"], "unit": "tokens/s",
                 "method": ("each step one replay of a captured CUDA graph (forward + copy of y); "
-                           if not args.e2e_eager else "eager forward per step; ") +
+                           if use_graphs else "eager forward per step; ") +
                           "uploads/downloads on two copy streams, double-buffered, overlapping "
                           "the neighbouring steps' compute; L2 not flushed inside this loop (each "
                           f"step streams {alg['ffn_weight_bytes'] / 1e9:.2f} GB of weights)",

@@ -106,7 +106,9 @@ class MoeShuffle:
         self.forward(logits, x, w_gate, w_up, w_down)
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
+        # thread-local capture: other threads of the process (a communicator's watchdog, say) may
+        # keep making CUDA calls while this thread records
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
             self.forward(logits, x, w_gate, w_up, w_down)
             if out is not None:
                 out.copy_(self.y)
