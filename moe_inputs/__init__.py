@@ -76,7 +76,12 @@ _SMALL = [
     Workload("finegrained-small", 300, 1024, 256, 8, 32, 256, payload="fp8", bias="zipf1.2"),
     Workload("skewed-small", 2048, 512, 128, 2, 16, 320, capacity_factor=1.25, bias="hot0+3"),
 ]
-WORKLOADS: Dict[str, Workload] = {w.name: w for w in _FULL + _SMALL}
+# Profiler-sized: the train shapes (H=4096, F=14336) with two experts and k=1, so the expert FFN is
+# tensor-bound like train's (about 1000 rows per expert) while all buffers fit in about 1 GB.
+_PROFILE = [
+    Workload("train-e2", 2048, 4096, 2, 1, 2, 14336),
+]
+WORKLOADS: Dict[str, Workload] = {w.name: w for w in _FULL + _SMALL + _PROFILE}
 
 
 def get(name: str) -> Workload:
