@@ -273,6 +273,8 @@ def test_ffn_two_block_experts(cuda, rows):
     (5, 256, 4, 1, 2, 192, "fp8", 0.0),       # FP8 payload, tiny T
     (64, 320, 16, 4, 4, 64, "bf16", 1.0),     # H not a multiple of 256, drops at capacity 16
     (200, 192, 8, 8, 8, 128, "bf16", 0.0),    # k = E
+    (64, 128, 1024, 32, 32, 64, "bf16", 0.0),  # E and k at their limits: ~2 rows per expert
+    (64, 128, 1024, 32, 32, 64, "fp8", 1.0),   # the same with the FP8 payload and capacity 2
 ])
 def test_pipeline_edge_shapes(cuda, T, H, E, k, R, F, payload, cf):
     from combine_moe_route_10_b200 import MoeShuffle
