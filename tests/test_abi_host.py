@@ -1,6 +1,5 @@
 """Host-side checks of the C ABI (no GPU needed): the library loads, exports every function that
 include/moe.h declares, and rejects invalid arguments before launching anything."""
-import ctypes
 import os
 import re
 

@@ -1,9 +1,7 @@
 """The multi-GPU path of bench.py (independent replicas, max over ranks) on CPU with gloo ranks."""
-import os
 import socket
 
 import pytest
-import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 

@@ -5,7 +5,6 @@ in the workspace.  Setting those counters to a value that the GEMM-1 epilogues c
 the target is a flag that nothing sets: the waits run out, the kernel records MOE_ERR_TIMEOUT in the
 workspace status word, drains its own copies and MMAs, frees TMEM and returns.  The context stays
 usable: after re-zeroing the workspace the same call gives correct results again."""
-import numpy as np
 import pytest
 import torch
 

@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import moe_inputs as mi
-from _helpers import bits16, bytes8, np_, rel_max_err, to_dev_bf16_from_bits
+from _helpers import bits16, np_, rel_max_err, to_dev_bf16_from_bits
 from oracle import moe
 
 pytestmark = pytest.mark.gpu

@@ -1,6 +1,5 @@
 """Pins of the oracle's bf16 and e4m3 rounding against the formats' definitions and torch's casts."""
 import numpy as np
-import pytest
 import torch
 
 from oracle.numerics import (bf16_bits, bf16_from_bits, bf16_round, e4m3_decode,

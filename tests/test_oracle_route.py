@@ -1,7 +1,6 @@
 """Pins of the oracle router: brute-force sort, tie rule, distinct ids, softmax identities."""
 import itertools
 import math
-import os
 
 import numpy as np
 import pytest
