@@ -159,8 +159,9 @@ moe_status_t moe_dispatch_noalloc(const void* x, int T, int H, const int32_t* to
                                   int32_t* slot_row, int32_t* row_token, int32_t* status,
                                   moe_stream_t stream);
 
-/* Bytes of scratch moe_expert_ffn needs (status word, the bf16 intermediate h [max_rows, F] and,
- * for the FP8 payload, the dequantised bf16 input rows [max_rows, H]). */
+/* Bytes of scratch moe_expert_ffn needs: a status word, the bf16 intermediate h [max_rows, F], for
+ * the FP8 payload the dequantised bf16 input rows [max_rows, H], and the int32 counters of the
+ * tile pipeline (two per 128-row block plus two for the run-time tile scheduler). */
 size_t moe_ffn_workspace_size(int max_rows, int E, int H, int F, moe_payload_t payload);
 
 /*
