@@ -13,6 +13,9 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+// Three CTAs (24 warps) per SM: the k <= 2 variants otherwise take 84 registers, which the
+// per-warp register granularity turns into two CTAs per SM (measured: train combine 26.6 -> 24.5 us).
+constexpr int kMinCtasPerSm = 3;
 
 __device__ __forceinline__ void accumulate(float acc[8], float w, uint4 v) {
   const uint32_t words[4] = {v.x, v.y, v.z, v.w};
@@ -26,7 +29,7 @@ __device__ __forceinline__ void accumulate(float acc[8], float w, uint4 v) {
 // KS rows are gathered together per step (loads issued before any accumulation); UNROLL vectors
 // per lane per row.
 template <int KS, int UNROLL, bool SPLIT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, kMinCtasPerSm)
     combine_kernel(const uint4* __restrict__ expert_out, int max_rows,
                    const int32_t* __restrict__ slot_row, const float* __restrict__ topk_w, int T,
                    int k, int nvec, int wpt, uint4* __restrict__ y) {
