@@ -10,6 +10,24 @@ import torch
 from . import _lib
 
 
+def expect(t, shape, dtype, name: str, device=None) -> None:
+    """Raise unless ``t`` is a contiguous tensor of this shape and dtype (on ``device`` if given).
+
+    The kernels trust these shapes (a short ``x`` would be read past its end), so every tensor a
+    caller hands to ``MoeShuffle`` is checked here, on the host, before anything is launched.
+    """
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous (row-major)")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name}: on {t.device}, expected {device}")
+
+
 class MoeShuffle:
     """Route -> dispatch -> grouped SwiGLU FFN -> combine for T tokens of width H over E experts.
 
@@ -29,6 +47,9 @@ class MoeShuffle:
             raise ValueError("payload must be 'bf16' or 'fp8'")
         self.payload = _lib.MOE_PAYLOAD_FP8_E4M3_B128 if self.fp8 else _lib.MOE_PAYLOAD_BF16
         dev = torch.device(device)
+        if dev.type == "cuda" and dev.index is None:
+            dev = torch.device("cuda", torch.cuda.current_device())
+        self.device = dev
         i32 = dict(dtype=torch.int32, device=dev)
         S = T * k
         self.max_rows = S
@@ -62,11 +83,14 @@ class MoeShuffle:
 
     # -- the four stages ----------------------------------------------------------------------
     def route(self, logits: torch.Tensor, stream=None):
+        expect(logits, (self.T, self.E), torch.float32, "logits", self.device)
         _lib.moe_route(logits, self.T, self.E, self.k, self.renormalize, self.topk_idx,
                        self.topk_w, self.expert_routed, stream)
 
     def dispatch(self, x: torch.Tensor, topk_idx: torch.Tensor | None = None, stream=None):
         idx = self.topk_idx if topk_idx is None else topk_idx
+        expect(x, (self.T, self.H), torch.bfloat16, "x", self.device)
+        expect(idx, (self.T, self.k), torch.int32, "topk_idx", self.device)
         _lib.moe_dispatch(x, self.T, self.H, idx, self.k, self.E, self.R, self.capacity,
                           self.payload, self.send, self.send_scales, self.expert_counts,
                           self.expert_offsets, self.rank_offsets, self.slot_row, self.row_token,
@@ -74,6 +98,17 @@ class MoeShuffle:
 
     def expert_ffn(self, w_gate, w_up, w_down, send=None, send_scales=None, expert_offsets=None,
                    stream=None):
+        bf16 = torch.bfloat16
+        expect(w_gate, (self.E, self.F, self.H), bf16, "w_gate", self.device)
+        expect(w_up, (self.E, self.F, self.H), bf16, "w_up", self.device)
+        expect(w_down, (self.E, self.H, self.F), bf16, "w_down", self.device)
+        if send is not None:
+            expect(send, (self.max_rows, self.H), self.send.dtype, "send", self.device)
+        if send_scales is not None:
+            expect(send_scales, (self.max_rows, self.H // 128), torch.float32, "send_scales",
+                   self.device)
+        if expert_offsets is not None:
+            expect(expert_offsets, (self.E + 1,), torch.int32, "expert_offsets", self.device)
         _lib.moe_expert_ffn(self.send if send is None else send,
                             self.send_scales if send_scales is None else send_scales,
                             self.payload,
@@ -82,6 +117,12 @@ class MoeShuffle:
                             self.expert_out, self.ws_ffn, self.ws_ffn_bytes, stream)
 
     def combine(self, expert_out=None, slot_row=None, topk_w=None, stream=None):
+        if expert_out is not None:
+            expect(expert_out, (self.max_rows, self.H), torch.bfloat16, "expert_out", self.device)
+        if slot_row is not None:
+            expect(slot_row, (self.T, self.k), torch.int32, "slot_row", self.device)
+        if topk_w is not None:
+            expect(topk_w, (self.T, self.k), torch.float32, "topk_w", self.device)
         # the combine reports a wait that ran out into the FFN workspace's status word
         _lib.moe_combine(self.expert_out if expert_out is None else expert_out, self.max_rows,
                          self.slot_row if slot_row is None else slot_row,
