@@ -25,6 +25,32 @@ def declared_functions():
     return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", src)))
 
 
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    """A C11 program that takes the address of every declared function compiles against moe.h with
+    warnings as errors and links against libmoe.so: the boundary is usable from plain C."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    names = declared_functions()
+    body = "\n".join(f"  fns[{i}] = (void (*)(void))&{n};" for i, n in enumerate(names))
+    src = tmp_path / "use_moe.c"
+    src.write_text(
+        '#include "moe.h"\n#include <stdio.h>\n'
+        f"int main(void) {{\n  void (*fns[{len(names)}])(void);\n{body}\n"
+        '  printf("%d %d\\n", moe_abi_version(), moe_capacity(1.25, 16384, 2, 128));\n'
+        "  return fns[0] == 0;\n}\n")
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    exe = tmp_path / "use_moe"
+    subprocess.run([cc, "-std=c11", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                    "-L", libdir, "-l:" + os.path.basename(_lib.LIB_PATH), "-Wl,-rpath," + libdir],
+                   check=True, capture_output=True, text=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    assert out == [str(pkg.moe_abi_version()), "320"]
+
+
 def test_header_declares_the_four_calls():
     names = declared_functions()
     for n in ["moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine"]:
