@@ -9,10 +9,11 @@
 // The scratch (the per-chunk expert histogram) lives in g_dispatch_scratch,
 // a file-scope __device__ array of kNoallocScratchBytes.  Every GPU that loads the library keeps it
 // until the process exits.  Host code must not pass the array's name to a kernel (on the host it is
-// only a stand-in symbol); the device address is looked up once per device with
-// cudaGetSymbolAddress while that device is current, during the first call on that device.
-#include <mutex>
-
+// only a stand-in symbol): every call looks up the array's device address in the context that is
+// current at that moment (cudaGetSymbolAddress, a host-side lookup that allocates nothing), so the
+// address is never one left over from another context of the same device (a driver-API context of
+// the caller's, or the primary context before a cudaDeviceReset).  The first call in a context may
+// load the library's module there, which is why it should come before any stream capture.
 #include "../../include/moe.h"
 #include "common.cuh"
 #include "launch.h"
@@ -20,27 +21,15 @@
 namespace {
 
 constexpr size_t kNoallocScratchBytes = MOE_DISPATCH_NOALLOC_SCRATCH_BYTES;
-constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_dispatch_scratch[kNoallocScratchBytes];
 
-unsigned char* g_scratch_ptr[kMaxDevices] = {nullptr};
-std::mutex g_scratch_mu;
-
-// Device address of g_dispatch_scratch on the current device (looked up once per device).
-cudaError_t scratch_for_current_device(unsigned char** out) {
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
+// Device address of g_dispatch_scratch in the current context (looked up on every call).
+cudaError_t scratch_for_current_context(unsigned char** out) {
+  void* p = nullptr;
+  const cudaError_t err = cudaGetSymbolAddress(&p, g_dispatch_scratch);
   if (err != cudaSuccess) return err;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    err = cudaGetSymbolAddress(&p, g_dispatch_scratch);
-    if (err != cudaSuccess) return err;
-    g_scratch_ptr[dev] = static_cast<unsigned char*>(p);
-  }
-  *out = g_scratch_ptr[dev];
+  *out = static_cast<unsigned char*>(p);
   return cudaSuccess;
 }
 
@@ -76,7 +65,7 @@ extern "C" moe_status_t moe_dispatch_noalloc(const void* x, int T, int H, const 
   if (moe::dispatch_workspace_bytes(T, E, k) > kNoallocScratchBytes) return MOE_ERR_WORKSPACE;
 
   unsigned char* scratch = nullptr;
-  if (scratch_for_current_device(&scratch) != cudaSuccess) {
+  if (scratch_for_current_context(&scratch) != cudaSuccess) {
     cudaGetLastError();
     return MOE_ERR_CUDA;
   }

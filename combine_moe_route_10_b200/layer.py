@@ -123,11 +123,11 @@ class MoeShuffle:
             expect(slot_row, (self.T, self.k), torch.int32, "slot_row", self.device)
         if topk_w is not None:
             expect(topk_w, (self.T, self.k), torch.float32, "topk_w", self.device)
-        # the combine reports a wait that ran out into the FFN workspace's status word
+        # the combine has no device-side waits and no device-side findings: no status word
         _lib.moe_combine(self.expert_out if expert_out is None else expert_out, self.max_rows,
                          self.slot_row if slot_row is None else slot_row,
                          self.topk_w if topk_w is None else topk_w, self.T, self.k, self.H,
-                         self.y, self.ws_ffn, stream)
+                         self.y, None, stream)
 
     def forward(self, logits, x, w_gate, w_up, w_down, stream=None) -> torch.Tensor:
         self.route(logits, stream)

@@ -93,7 +93,9 @@ moe_status_t moe_route(const float* logits, int T, int E, int k, int renormalize
                        moe_stream_t stream);
 
 /* Bytes of scratch moe_dispatch needs for T tokens, E experts, k slots per token: a status word and
- * one expert histogram per chunk of 16 * floor(128 / k) tokens. */
+ * one expert histogram per chunk of 16 * floor(128 / k) tokens.  The caller allocates it (the NCCL
+ * EP page, sections 1 and 3.1: the caller registers the memory a group or handle works in); returns
+ * 0 for T < 0, E < 1 or k < 1. */
 size_t moe_dispatch_workspace_size(int T, int E, int k);
 
 /*
@@ -146,8 +148,9 @@ moe_status_t moe_dispatch(const void* x, int T, int H, const int32_t* topk_idx, 
  * Limits: those of moe_dispatch, plus 256 + ceil(T / C) * E * 4 <= 1 MiB, where C = 16 * floor(128 / k)
  * tokens (at least 16) is the counting chunk (e.g. T <= 261120 at E = 1024, k = 2; T <= 65280 at
  * E = 1024, k = 8); larger shapes return MOE_ERR_WORKSPACE without launching.
- * The first call on each device looks up the array's device address (cudaGetSymbolAddress with
- * that device current); make that first call before any stream capture.  All calls share the one
+ * Every call looks up the array's device address in the current context (cudaGetSymbolAddress, no
+ * allocation); the first call in a context may load the library's module there, so make that first
+ * call before any stream capture.  All calls share the one
  * array: calls that overlap on the GPU (different streams, or the same array from several host
  * threads without ordering) race and give wrong results; order them on one stream.
  */
@@ -161,7 +164,9 @@ moe_status_t moe_dispatch_noalloc(const void* x, int T, int H, const int32_t* to
 
 /* Bytes of scratch moe_expert_ffn needs: a status word, the bf16 intermediate h [max_rows, F], for
  * the FP8 payload the dequantised bf16 input rows [max_rows, H], and the int32 counters of the
- * tile pipeline (two per 128-row block plus two for the run-time tile scheduler). */
+ * tile pipeline (two per 128-row block plus two for the run-time tile scheduler).  Caller-allocated
+ * as for moe_dispatch_workspace_size (NCCL EP page, sections 1 and 3.1); `payload` is needed
+ * because only the FP8 payload has the dequantised rows.  Returns 0 for invalid sizes. */
 size_t moe_ffn_workspace_size(int max_rows, int E, int H, int F, moe_payload_t payload);
 
 /*
@@ -208,8 +213,11 @@ moe_status_t moe_combine(const void* expert_out, int max_rows, const int32_t* sl
 
 /*
  * Synchronise `stream`, read the device status word at the start of a dispatch or FFN workspace
- * (or any status word given to moe_combine / moe_dispatch_noalloc), clear it, and report it: MOE_OK, MOE_ERR_INVALID_TOPK or MOE_ERR_TIMEOUT (MOE_ERR_CUDA if the
- * stream itself failed).
+ * (or any status word given to moe_combine / moe_dispatch_noalloc), clear it, and report it:
+ * MOE_OK, MOE_ERR_INVALID_TOPK or MOE_ERR_TIMEOUT (MOE_ERR_CUDA if the stream itself failed).
+ * This is how device-side findings reach the host as the error codes of the NCCL EP page's table
+ * ("NCCL EP架构解析", section 5.1: INVALID_TOPK for a routing index out of range, CUDA_ERROR for a
+ * failed kernel).  It is the only call of the library that waits for the GPU.
  */
 moe_status_t moe_sync_status(void* ws, moe_stream_t stream);
 

@@ -31,5 +31,39 @@ def rel_max_err(got_bits, ref_bits) -> float:
     return float(np.max(np.abs(g - r)) / denom)
 
 
+# Element-wise parity bar for bf16 outputs of the FFN and the whole path: an element fails when
+# |got - ref| > RTOL * |ref| + ATOL_REL * max|ref|.  RTOL covers one bf16 rounding step (2^-8 of the
+# value) with margin; the absolute term, scaled to the tensor's magnitude, covers elements near zero
+# where rows of fp32-accumulated sums cancel (their error is set by the size of the summands, not by
+# the element's own value).
+RTOL = 1e-2
+ATOL_REL = 1e-3
+
+
+def parity_report(got_bits, ref_bits) -> dict:
+    """max |got - ref| / max |ref|, the Frobenius relative error, and the count of elements outside
+    the element-wise bar (NaN on either side counts as outside)."""
+    g, r = bf16_values(got_bits), bf16_values(ref_bits)
+    assert g.shape == r.shape, (g.shape, r.shape)
+    if g.size == 0:
+        return {"rel_max": 0.0, "frob": 0.0, "n_bad": 0, "n": 0}
+    d = np.abs(g - r)
+    scale = float(np.max(np.abs(r)))
+    bound = RTOL * np.abs(r) + ATOL_REL * scale
+    bad = ~(d <= bound)                      # NaN compares false: counted as bad
+    nr = float(np.linalg.norm(r))
+    return {"rel_max": float(np.max(d) / scale) if scale > 0 else float(np.max(d)),
+            "frob": float(np.linalg.norm(np.nan_to_num(g - r, nan=np.inf)) / nr) if nr > 0 else 0.0,
+            "n_bad": int(np.count_nonzero(bad)), "n": int(g.size)}
+
+
+def assert_close_bf16(got_bits, ref_bits, what: str = "") -> dict:
+    """The parity bar for a bf16 output tensor: max-relative error <= RTOL and no element outside
+    the element-wise bar."""
+    rep = parity_report(got_bits, ref_bits)
+    assert rep["rel_max"] <= RTOL and rep["n_bad"] == 0, f"{what}: {rep}"
+    return rep
+
+
 def to_dev_bf16_from_bits(bits: np.ndarray, device) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)

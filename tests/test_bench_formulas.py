@@ -32,9 +32,10 @@ def test_finegrained_fp8_bytes():
     # 469.8 MB of bf16 expert outputs read, 58.7 MB written
     assert close(a["combine"], 528.5 * MB, 0.005)
     assert close(a["ffn_weight_bytes"], 22.5 * GB, 0.005)
-    # the FFN stage also moves the dequantisation pass: codes + scales read, bf16 rows written
-    acts = S * w.H * 2 + 2 * S * w.F * 2 + S * w.H * 2 + S * w.H + S * (w.H // 128) * 4 + S * w.H * 2
-    assert a["ffn_bytes"] == a["ffn_weight_bytes"] + acts
+    # the FFN's method bytes: the codes and scales as dispatched, read once, and bf16 outputs
+    # written once; the bf16 intermediate and the dequantised rows are the implementation's own
+    assert a["ffn_bytes"] == a["ffn_weight_bytes"] + S * w.H + S * (w.H // 128) * 4 + S * w.H * 2
+    assert a["ffn_impl_overhead"] == 2 * S * w.F * 2 + 4 * S * w.H
 
 
 def test_decode_and_skewed_ffn_figures():
@@ -53,7 +54,8 @@ def test_decode_and_skewed_ffn_figures():
 
 def test_recorded_traffic_is_near_the_algorithmic_bytes():
     """The DRAM traffic recorded from ncu captures lies between 0.95x and 1.3x the algorithmic FFN
-    bytes of the same workload (active experts and kept rows from the oracle's routing)."""
+    bytes plus the implementation's own overhead, for the same workload (active experts and kept
+    rows from the oracle's routing)."""
     import numpy as np
     from oracle import moe
     assert set(bench.FFN_TRAFFIC) <= set(mi.WORKLOADS)
@@ -63,5 +65,6 @@ def test_recorded_traffic_is_near_the_algorithmic_bytes():
         idx, _, _ = moe.route(d["logits"].numpy(), w.k)
         plan = moe.dispatch_plan(idx, w.E, w.R, moe.capacity(w.capacity_factor, w.T, w.k, w.E))
         active = int((np.diff(plan["expert_offsets"]) > 0).sum())
-        alg = bench.algorithmic(w, plan["S"], active)["ffn_bytes"]
+        a = bench.algorithmic(w, plan["S"], active)
+        alg = a["ffn_bytes"] + a["ffn_impl_overhead"]
         assert 0.95 * alg <= t <= 1.3 * alg, (name, t / alg)

@@ -3,9 +3,10 @@
 Programs that route every device allocation through their own pool (and plug-ins inside them), or
 latency-critical code that must not call cudaMalloc, cannot hand moe_dispatch a workspace.  The
 no-alloc entry point keeps its scratch in a static device array inside the library.  These tests
-call it through the C ABI and compare every output with moe_dispatch's on the same inputs
-(bit-exact, the bar of all dispatch tests), on consecutive calls whose shapes differ, so that
-anything the shared array keeps from the previous call would show up.  This file is collected last.
+call it through the C ABI and compare every output with moe_dispatch's on the same inputs and with
+the oracle's plan and payload (bit-exact, the bar of all dispatch tests), on consecutive calls whose
+shapes differ, so that anything the shared array keeps from the previous call, or an address lookup
+that went stale between calls, would show up.  This file is collected last.
 """
 import numpy as np
 import pytest
@@ -56,6 +57,20 @@ def run_both(w, seed):
     assert torch.equal(got["send"][:S].view(torch.uint8), ref["send"][:S].view(torch.uint8))
     if ref["scales"] is not None:
         assert torch.equal(got["scales"][:S].view(torch.int32), ref["scales"][:S].view(torch.int32))
+    # and directly against the oracle's plan and payload, so that a fault shared by both entry
+    # points would not go unnoticed
+    plan = moe.dispatch_plan(idx_np, w.E, w.R, cap)
+    assert S == plan["S"]
+    for key, pk in (("counts", "expert_counts"), ("offsets", "expert_offsets"),
+                    ("rank_offsets", "rank_offsets"), ("slot_row", "slot_row")):
+        assert np.array_equal(got[key].cpu().numpy(), plan[pk]), key
+    assert np.array_equal(got["row_token"][:S].cpu().numpy(), plan["row_token"])
+    x_bits = d["x"].cpu().view(torch.int16).numpy().view(np.uint16)
+    send_ref, sc_ref = moe.dispatch_payload(x_bits, plan, w.payload == "fp8")
+    assert np.array_equal(got["send"][:S].cpu().view(torch.uint8).numpy(),
+                          np.ascontiguousarray(send_ref).view(np.uint8).reshape(S, -1))
+    if sc_ref is not None:
+        assert np.array_equal(got["scales"][:S].cpu().numpy().view(np.uint32), sc_ref.view(np.uint32))
     return S
 
 
