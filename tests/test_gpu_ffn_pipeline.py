@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import moe_inputs as mi
-from _helpers import bits16, np_, assert_close_bf16, to_dev_bf16_from_bits
+from _helpers import assert_close_bf16, bits16, combine_magnitude, np_, to_dev_bf16_from_bits
 from oracle import moe
 
 pytestmark = pytest.mark.gpu
@@ -117,7 +117,8 @@ def test_pipeline_full_size_every_row_and_token(cuda, name):
     # the combine is exact given its inputs: every token
     assert np.array_equal(y_bits, moe.combine(eo, np_(m.slot_row), np_(m.topk_w), w.T, w.H))
     # the whole path on every token, against the oracle's expert outputs and routing weights
-    assert_close_bf16(y_bits, moe.combine(y_ref, plan["slot_row"], wt, w.T, w.H), "y")
+    assert_close_bf16(y_bits, moe.combine(y_ref, plan["slot_row"], wt, w.T, w.H), "y",
+                      combine_magnitude(y_ref, plan["slot_row"], wt))
 
 
 @pytest.mark.parametrize("name", ["finegrained", "skewed"])
@@ -153,7 +154,8 @@ def test_pipeline_end_to_end(cuda, name):
     assert np.array_equal(np_(m.slot_row), o["slot_row"])
     assert np.array_equal(np_(m.expert_offsets), o["expert_offsets"])
     assert_close_bf16(bits16(m.expert_out)[:o["S"]], o["expert_out"])
-    assert_close_bf16(bits16(y), o["y"])
+    assert_close_bf16(bits16(y), o["y"], "y",
+                      combine_magnitude(o["expert_out"], o["slot_row"], o["topk_w"]))
 
 
 def test_pipeline_decode_full_size_every_token(cuda):
@@ -172,7 +174,8 @@ def test_pipeline_decode_full_size_every_token(cuda):
     assert np.array_equal(bits16(m.send)[:o["S"]], o["send"])
     assert_close_bf16(bits16(m.h)[:o["S"]], o["h"])
     assert_close_bf16(bits16(m.expert_out)[:o["S"]], o["expert_out"])
-    assert_close_bf16(bits16(y), o["y"])
+    assert_close_bf16(bits16(y), o["y"], "y",
+                      combine_magnitude(o["expert_out"], o["slot_row"], o["topk_w"]))
     # the combine is exact given its inputs: the oracle's combine of the GPU's expert outputs
     assert np.array_equal(bits16(y), moe.combine(bits16(m.expert_out), np_(m.slot_row),
                                                  np_(m.topk_w), w.T, w.H))
@@ -191,7 +194,8 @@ def test_ffn_workspace_reused_across_calls_with_different_routing(cuda):
                          bits16(d["w_down"]), w.k, w.R)
         assert np.array_equal(np_(m.expert_offsets), o["expert_offsets"])
         assert_close_bf16(bits16(m.expert_out)[:o["S"]], o["expert_out"])
-        assert_close_bf16(bits16(y), o["y"])
+        assert_close_bf16(bits16(y), o["y"], "y",
+                      combine_magnitude(o["expert_out"], o["slot_row"], o["topk_w"]))
 
 
 @pytest.mark.parametrize("rows", [
@@ -247,4 +251,5 @@ def test_pipeline_edge_shapes(cuda, T, H, E, k, R, F, payload, cf):
         return
     if o["S"]:
         assert_close_bf16(bits16(m.expert_out)[:o["S"]], o["expert_out"])
-    assert_close_bf16(bits16(y), o["y"])
+    assert_close_bf16(bits16(y), o["y"], "y",
+                      combine_magnitude(o["expert_out"], o["slot_row"], o["topk_w"]))

@@ -1,7 +1,7 @@
 """The element-wise parity bar used by the GPU tests flags what it should, on the CPU."""
 import numpy as np
 
-from _helpers import assert_close_bf16, parity_report
+from _helpers import assert_close_bf16, bf16_values, parity_report
 from oracle.numerics import bf16_bits
 
 
@@ -30,3 +30,20 @@ def test_nan_counts_as_outside_the_bar():
     got = ref.copy()
     got[1, 1] = 0x7FC0
     assert parity_report(got, ref)["n_bad"] == 1
+
+
+def test_combine_output_is_judged_against_the_size_of_its_summands():
+    # y = 0.5 * a + 0.5 * b with a ~ -b: y is near zero, and a one-ulp difference in a (as two
+    # fp32-accumulated FFNs may round differently) moves y by half an ulp of a
+    from _helpers import combine_magnitude
+    a = np.array([[1.5, 2.0]]), np.array([[-1.49, 1.0]])
+    eo = bf16_bits(np.concatenate(a))
+    sr = np.array([[0, 1]])
+    w = np.array([[0.5, 0.5]], dtype=np.float32)
+    ref = bf16_bits(0.5 * bf16_values(eo[0]) + 0.5 * bf16_values(eo[1]))[None, :]
+    eo2 = eo.copy()
+    eo2[0, 0] += 1                                   # one ulp of 1.5 = 2^-7
+    got = bf16_bits(0.5 * bf16_values(eo2[0]) + 0.5 * bf16_values(eo2[1]))[None, :]
+    assert parity_report(got, ref)["n_bad"] == 1     # judged against |y| ~ 0.004 alone: fails
+    rep = parity_report(got, ref, combine_magnitude(eo, sr, w))
+    assert rep["n_bad"] == 0                          # against 0.5*1.5 + 0.5*1.49: passes
