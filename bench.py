@@ -4,7 +4,12 @@
 One step = one pass of the whole path over one batch of synthetic tokens (all four C-ABI calls on
 one stream), inputs and weights already resident in HBM.  Prints one JSON line on rank 0.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload skewed] [--also train,finegrained]
+                    [--impl ours|reference]
+
+The headline workload (default ``skewed``: T=16384, H=7168, E=128, top-2, capacity 320, the largest
+configuration that fits one GPU) gives ``value``; the ``--also`` workloads are timed the same way
+in the same run and reported under ``workloads``.
 
 Multi-GPU (torchrun): every rank runs an independent replica of the workload (its own batch of T
 tokens, emulated expert-parallel ranks inside each GPU), no data-path collective; the step time is
@@ -30,12 +35,15 @@ import moe_inputs as mi  # noqa: E402
 
 METRIC = "dispatch+FFN+combine tokens/s and shuffle HBM GB/s (% of roofline) on 1 B200"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Nominal B200 figures, for the secondary fractions: HBM3e about 8 TB/s, dense bf16 2.25 PFLOP/s.
+NOMINAL = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 L2_FLUSH_BYTES = mi.l2_flush_bytes()
 # DRAM read + write bytes per call of the FFN stage (fused_ffn_kernel, plus dequant_fp8_kernel for
-# the FP8 payload) at full size: ncu dram__bytes_read.sum + dram__bytes_write.sum, one capture of
-# `bench.py --workload <w> --steps 3 --warmup 3` on B200, kernels as built from this tree.  To be
-# reset to None whenever either kernel changes.
-FFN_TRAFFIC = {"decode": 2.839e9, "train": 3.673e9, "finegrained": 14.73e9, "skewed": 12.07e9}
+# the FP8 payload): ncu dram__bytes_read.sum + dram__bytes_write.sum of the kernels as built from
+# this tree.  An entry is None (or absent) once either kernel has changed since its counters were
+# taken.  New counters come from small captures (one kernel, a few launches, a few GB on the
+# device), scaled to a full call by the units processed, never from a capture of a full-size run.
+FFN_TRAFFIC: dict = {}
 
 
 # ---------------------------------------------------------------------------------------------
@@ -125,21 +133,27 @@ def aggregate(local_ms: float, tokens_per_rank: int, steps: int, device) -> dict
 
 
 def algorithmic(w, S: int, active_experts: int):
-    """Algorithmic bytes / flops per step of each stage (what the stage must move or compute)."""
+    """Algorithmic bytes / flops per step of each stage: what the method must move or compute.
+
+    The FFN's algorithmic bytes are the active experts' weights, its input rows read once (bf16, or
+    for the FP8 payload the e4m3 codes and fp32 scales as dispatched) and its output rows written
+    once.  Traffic that this implementation adds on top (the bf16 intermediate h written and read
+    back between the two GEMMs; for FP8, the dequantisation pass's bf16 rows, written once and read
+    by the GEMM instead of the codes) is ``ffn_impl_overhead`` and is not counted as achieved work.
+    """
     fp8 = w.payload == "fp8"
     b = 1 if fp8 else 2
+    scales = S * (w.H // 128) * 4 if fp8 else 0
     route = w.T * w.E * 4 + w.T * w.k * 8 + w.E * 4
-    dispatch = (w.T * w.H * 2 + S * w.H * b + (S * (w.H // 128) * 4 if fp8 else 0)
+    dispatch = (w.T * w.H * 2 + S * w.H * b + scales
                 + w.T * w.k * 4 * 3 + S * 4 + (w.E * 2 + 1 + w.R + 1) * 4)
     weights = active_experts * 3 * w.H * w.F * 2
-    acts = S * w.H * 2 + 2 * S * w.F * 2 + S * w.H * 2   # A read, h write+read, out write
-    if fp8:
-        acts += S * w.H + S * (w.H // 128) * 4 + S * w.H * 2  # dequant: read codes+scales, write
-    ffn_bytes = weights + acts
+    ffn_bytes = weights + S * w.H * b + scales + S * w.H * 2
+    overhead = 2 * S * w.F * 2 + (4 * S * w.H if fp8 else 0)
     ffn_flops = 6 * S * w.H * w.F
     combine = S * w.H * 2 + w.T * w.k * 8 + w.T * w.H * 2
     return dict(route=route, dispatch=dispatch, ffn_bytes=ffn_bytes, ffn_weight_bytes=weights,
-                ffn_flops=ffn_flops, combine=combine)
+                ffn_impl_overhead=overhead, ffn_flops=ffn_flops, combine=combine)
 
 
 def cpu_baseline_run(w, d_cpu, budget_s: float = 12.0, n_tokens: int | None = None):
@@ -188,7 +202,12 @@ def run_reference(args, w, rank: int):
     """The oracle, as it stands, timed on the host cores on bounded token samples of the workload."""
     if rank != 0:
         return
-    d = mi.make_inputs(w, seed=0, device="cpu")
+    # the same inputs as the GPU arm's rank 0 (drawn by the same generator on the GPU when there is
+    # one), copied to host memory; the oracle then runs on the host cores only
+    gen_dev = "cuda" if torch.cuda.is_available() else "cpu"
+    d = {k: v.cpu() for k, v in mi.make_inputs(w, seed=0, device=gen_dev).items()}
+    if gen_dev == "cuda":
+        torch.cuda.empty_cache()
     budget = 150.0
     # size each step so that warm-up + timed steps stay within a few minutes
     _, info = cpu_baseline_run(w, d, n_tokens=1)
@@ -236,7 +255,10 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="decode", choices=sorted(mi.WORKLOADS))
+    ap.add_argument("--workload", default="skewed", choices=sorted(mi.WORKLOADS))
+    ap.add_argument("--also", default="train,finegrained",
+                    help="comma-separated workloads timed after the headline one, reported under "
+                         "'workloads' in the same line ('' for none)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--flush", default="write-read", choices=["write", "write-read"])
@@ -256,17 +278,68 @@ def main():
 
     import datetime
     import torch.distributed as dist
-    from combine_moe_route_10_b200 import MoeShuffle
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
+    also = [n for n in args.also.split(",") if n and n != w.name]
+    for n in also:
+        if n not in mi.WORKLOADS:
+            raise SystemExit(f"unknown workload {n}")
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    head = measure(w, args, dev, world, rank, e2e=True)
+    extra = {n: measure(mi.get(n), args, dev, world, rank, e2e=False) for n in also}
+    clocks = sampler.stop()
+
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8+bf16" if w.payload == "fp8" else "bf16",
+        "data": "synthetic (seeded; random-init expert weights N(0,0.02))",
+        "config": config_of(w, args),
+        "roofline": head["roofline"],
+        "stages": head["stages"],
+        "stages_note": "per-stage CUDA events on breakdown steps interleaved with the metric steps "
+                       "(each event ends the programmatic launch overlap around it); value and "
+                       "ms_per_step come from the metric steps' boundary events only; frac = of "
+                       "the measured HBM copy rate, frac_nominal = of 8 TB/s",
+        "kept_rows": head["kept_rows"], "active_experts": head["active_experts"],
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"],
+        "clocks": clocks,
+        "workloads": {n: {k: v for k, v in r.items() if k != "e2e"} for n, r in extra.items()},
+        "workloads_note": "the other large workloads, each timed the same way in the same run "
+                          "(own warm-up, L2 flush, metric and breakdown steps); gpu_launches counts "
+                          "the headline workload's timed region only",
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        d_cpu = {k: v.cpu() for k, v in mi.make_inputs(w, seed=rank, device=str(dev)).items()}
+        v, info = cpu_baseline_run(w, d_cpu)
+        line["cpu_baseline"] = {
+            "value": v, "unit": "tokens/s", "cores": info["cores"], "kind": "oracle",
+            "sample": f"first {info['tokens']} tokens of the workload (route, dispatch, SwiGLU FFN "
+                      f"on their rows, combine), {info['seconds']:.1f} s"}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def measure(w, args, dev, world: int, rank: int, e2e: bool) -> dict:
+    """Time K steps of workload ``w`` on this GPU (plus, with ``e2e``, the end-to-end loop through
+    the public API) and return its throughput, stage breakdown and FFN roofline."""
+    import math
+    import torch.distributed as dist
+    from combine_moe_route_10_b200 import MoeShuffle
 
     d = mi.make_inputs(w, seed=rank, device=str(dev))
-    cap_rows = (__import__("math").ceil(w.capacity_factor * w.T * w.k / w.E)
-                if w.capacity_factor else 0)
+    cap_rows = math.ceil(w.capacity_factor * w.T * w.k / w.E) if w.capacity_factor else 0
     m = MoeShuffle(w.T, w.H, w.E, w.k, w.R, w.F, payload=w.payload, capacity=cap_rows, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
     flush_rd = (torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
@@ -284,15 +357,13 @@ def main():
         m.expert_ffn(d["w_gate"], d["w_up"], d["w_down"])
         m.combine()
 
-    sampler = ClockSampler(local)
-    sampler.start()
     for _ in range(args.warmup):
         flush_l2()
         step()
     torch.cuda.synchronize()
     st = m.status()
     if st != 0:
-        raise SystemExit(f"device status {st} after warm-up")
+        raise SystemExit(f"{w.name}: device status {st} after warm-up")
     S = int(m.expert_offsets[w.E].item())
     active = int((m.expert_counts > 0).sum().item())
 
@@ -331,10 +402,65 @@ def main():
     stage_ms = [[e[j].elapsed_time(e[j + 1]) for j in range(n_ev - 1)] for e in evs]
     mean_stage = [sum(s[j] for s in stage_ms) / args.steps for j in range(n_ev - 1)]
 
-    # end to end through the public API, as a serving loop runs it: every step uploads its logits and
-    # tokens from pinned host memory and downloads its result to pinned host memory; uploads and
-    # downloads run on their own streams, double-buffered, so they overlap the neighbouring steps'
-    # compute (timed from the first upload to the last download)
+    e2e_out = None
+    if e2e:
+        e2e_out = e2e_run(w, m, d, args, dev, world, stream)
+    st = m.status()
+    if st != 0:
+        raise SystemExit(f"{w.name}: device status {st} after timing")
+
+    pk, pk_src = peaks()
+    alg = algorithmic(w, S, active)
+    t_route, t_disp, t_ffn, t_comb = mean_stage
+    hbm = pk["hbm_gbs"]
+    ffn_t_hbm = alg["ffn_bytes"] / (hbm * 1e9)
+    ffn_t_tc = alg["ffn_flops"] / (pk["bf16_tflops_sustained"] * 1e12)
+    if ffn_t_hbm >= ffn_t_tc:
+        ach = alg["ffn_bytes"] / (t_ffn * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                "frac_nominal": ach / NOMINAL["hbm_gbs"]}
+    else:
+        ach = alg["ffn_flops"] / (t_ffn * 1e-3) / 1e12
+        p = pk["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "achieved": ach, "peak": p, "unit": "TFLOP/s", "frac": ach / p,
+                "frac_burst": ach / pk["bf16_tflops"], "frac_nominal": ach / NOMINAL["bf16_tflops"]}
+    roof.update({
+        "kernel": ("fused_ffn_kernel (one persistent launch: GEMM-1 gate|up + SwiGLU, GEMM-2 down)"
+                   + (" + dequant_fp8_kernel" if w.payload == "fp8" else "") + " = moe_expert_ffn"),
+        "traffic": FFN_TRAFFIC.get(w.name), "peak_source": pk_src,
+        "algorithmic_bytes": alg["ffn_bytes"], "algorithmic_flops": alg["ffn_flops"],
+        "impl_overhead_bytes": alg["ffn_impl_overhead"],
+        "frac_of_max_time_bound": max(ffn_t_hbm, ffn_t_tc) / (t_ffn * 1e-3)})
+
+    def gbs(b, t):
+        return b / (t * 1e-3) / 1e9
+
+    def shuffle_stage(b, t):
+        return {"ms": t, "GB/s": gbs(b, t), "frac": gbs(b, t) / hbm,
+                "frac_nominal": gbs(b, t) / NOMINAL["hbm_gbs"]}
+
+    stages = {
+        "route": {"ms": t_route, "GB/s": gbs(alg["route"], t_route)},
+        "dispatch": shuffle_stage(alg["dispatch"], t_disp),
+        "ffn": {"ms": t_ffn, "TFLOP/s": alg["ffn_flops"] / (t_ffn * 1e-3) / 1e12,
+                "GB/s": gbs(alg["ffn_bytes"], t_ffn)},
+        "combine": shuffle_stage(alg["combine"], t_comb),
+    }
+    launches_per_step = 5 + (1 if w.payload == "fp8" else 0)   # route, count, rank_permute, FFN, combine
+    out = {"value": agg["value"], "ms_per_step": agg["ms_per_step"], "config": config_of(w, args),
+           "roofline": roof, "stages": stages, "kept_rows": S, "active_experts": active,
+           "gpu_launches": 2 * launches_per_step * args.steps,  # metric + breakdown steps
+           "e2e": e2e_out}
+    del m, d, flush, flush_rd
+    torch.cuda.empty_cache()
+    return out
+
+
+def e2e_run(w, m, d, args, dev, world: int, stream) -> dict:
+    """End to end through the public API, as a serving loop runs it: every step uploads its logits
+    and tokens from pinned host memory and downloads its result to pinned host memory; uploads and
+    downloads run on their own streams, double-buffered, so they overlap the neighbouring steps'
+    compute (timed from the first upload to the last download)."""
     logits_h = d["logits"].cpu().pin_memory()
     x_h = d["x"].cpu().pin_memory()
     y_h = [torch.empty(m.y.shape, dtype=m.y.dtype).pin_memory() for _ in range(2)]
@@ -389,84 +515,17 @@ def main():
         return t0.elapsed_time(t1)
 
     e2e_loop(3)  # warm-up
-    e2e = aggregate(e2e_loop(e2e_steps), w.T, e2e_steps, dev)
-    clocks = sampler.stop()
-    st = m.status()
-    if st != 0:
-        raise SystemExit(f"device status {st} after timing")
-
-    pk, pk_src = peaks()
-    alg = algorithmic(w, S, active)
-    ms = agg["ms_per_step"]
-    value = agg["value"]
-    t_route, t_disp, t_ffn, t_comb = mean_stage
-    hbm = pk["hbm_gbs"]
-    ffn_t_hbm = alg["ffn_bytes"] / (hbm * 1e9)
-    ffn_t_tc = alg["ffn_flops"] / (pk["bf16_tflops_sustained"] * 1e12)
-    if ffn_t_hbm >= ffn_t_tc:
-        ach = alg["ffn_bytes"] / (t_ffn * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm}
-    else:
-        ach = alg["ffn_flops"] / (t_ffn * 1e-3) / 1e12
-        p = pk["bf16_tflops_sustained"]
-        roof = {"bound": "tensor", "achieved": ach, "peak": p, "unit": "TFLOP/s", "frac": ach / p}
-    roof.update({
-        "kernel": ("fused_ffn_kernel (one persistent launch: GEMM-1 gate|up + SwiGLU, GEMM-2 down)"
-                   + (" + dequant_fp8_kernel" if w.payload == "fp8" else "") + " = moe_expert_ffn"),
-        "traffic": FFN_TRAFFIC.get(w.name), "peak_source": pk_src,
-        "algorithmic_bytes": alg["ffn_bytes"], "algorithmic_flops": alg["ffn_flops"],
-        "frac_of_max_time_bound": max(ffn_t_hbm, ffn_t_tc) / (t_ffn * 1e-3)})
-
-    def gbs(b, t):
-        return b / (t * 1e-3) / 1e9
-
-    shuffle = {
-        "route": {"ms": t_route, "GB/s": gbs(alg["route"], t_route)},
-        "dispatch": {"ms": t_disp, "GB/s": gbs(alg["dispatch"], t_disp),
-                     "frac": gbs(alg["dispatch"], t_disp) / hbm},
-        "ffn": {"ms": t_ffn, "TFLOP/s": alg["ffn_flops"] / (t_ffn * 1e-3) / 1e12,
-                "GB/s": gbs(alg["ffn_bytes"], t_ffn)},
-        "combine": {"ms": t_comb, "GB/s": gbs(alg["combine"], t_comb),
-                    "frac": gbs(alg["combine"], t_comb) / hbm},
-    }
-    launches_per_step = 5 + (1 if w.payload == "fp8" else 0)   # route, count, rank_permute, FFN, combine
-    h2d = d["logits"].numel() * 4 + d["x"].numel() * 2
-    d2h = m.y.numel() * 2
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "fp8+bf16" if w.payload == "fp8" else "bf16",
-        "data": "synthetic (seeded; random-init expert weights N(0,0.02))",
-        "config": config_of(w, args),
-        "roofline": roof,
-        "stages": shuffle,
-        "stages_note": "per-stage CUDA events on breakdown steps interleaved with the metric steps "
-                       "(each event ends the programmatic launch overlap around it); value and "
-                       "ms_per_step come from the metric steps' boundary events only",
-        "kept_rows": S, "active_experts": active,
-        "e2e": {"value": e2e["value"], "unit": "tokens/s",
-                "method": ("each step one replay of a captured CUDA graph (forward + copy of y); "
-                           if use_graphs else "eager forward per step; ") +
-                          "uploads/downloads on two copy streams, double-buffered, overlapping "
-                          "the neighbouring steps' compute; L2 not flushed inside this loop (each "
-                          f"step streams {alg['ffn_weight_bytes'] / 1e9:.2f} GB of weights)",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 2 * launches_per_step * args.steps,  # metric + breakdown steps
-        "clocks": clocks,
-    }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        d_cpu = {k: v.cpu() for k, v in d.items()}
-        v, info = cpu_baseline_run(w, d_cpu)
-        line["cpu_baseline"] = {
-            "value": v, "unit": "tokens/s", "cores": info["cores"], "kind": "oracle",
-            "sample": f"first {info['tokens']} tokens of the workload (route, dispatch, SwiGLU FFN "
-                      f"on their rows, combine), {info['seconds']:.1f} s"}
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+    agg = aggregate(e2e_loop(e2e_steps), w.T, e2e_steps, dev)
+    weights_gb = 3 * w.E * w.H * w.F * 2 / 1e9
+    del graphs
+    return {"value": agg["value"], "unit": "tokens/s",
+            "method": ("each step one replay of a captured CUDA graph (forward + copy of y); "
+                       if use_graphs else "eager forward per step; ") +
+                      "uploads/downloads on two copy streams, double-buffered, overlapping "
+                      "the neighbouring steps' compute; L2 not flushed inside this loop (each "
+                      f"step streams up to {weights_gb:.2f} GB of weights)",
+            "h2d_bytes_per_step": d["logits"].numel() * 4 + d["x"].numel() * 2,
+            "d2h_bytes_per_step": m.y.numel() * 2}
 
 
 if __name__ == "__main__":

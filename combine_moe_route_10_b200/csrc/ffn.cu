@@ -1,5 +1,5 @@
 // Grouped SwiGLU expert FFN on the packed send buffer: tcgen05 tensor cores, TMEM accumulators,
-// TMA-fed shared-memory pipeline.
+// TMA-fed shared-memory pipelines.
 //
 // Per expert e and each of its packed rows x (expert-major layout of the NCCL EP page, section
 // 2.1; two linear layers with SwiGLU per expert as in "细粒度专家并行方案对比：MegaMoE与传统方案",
@@ -7,24 +7,31 @@
 // run_moe passage of "DWDP: 在NVL72上的高性能分布式权重数据并行"):
 //     h = bf16( silu(x W_gate[e]^T) * (x W_up[e]^T) ),   expert_out = bf16( h W_down[e]^T ).
 //
-// One persistent launch (one CTA per SM, 192 threads) runs the GEMM-1 tiles and then the GEMM-2
-// tiles (the latter wait on per-row-block completion counters of the former); each CTA claims its
-// next tile at run time from a global counter:
-//   warp 0      TMA producer: claims tiles, passes their ids to the other roles through a small
-//               shared-memory queue, and loads an A tile (128 rows x 64 k; 16/32/64 rows for a
-//               small row block) + B tile (256 rows x 64 k) per stage, 128-byte swizzle, 4-stage
-//               mbarrier ring;
-//   warp 1      TMEM allocator and MMA issuer: one thread issues tcgen05.mma (M=128, N=256,
-//               K=16, bf16 -> fp32) into one of two 256-column TMEM accumulators, and
-//               tcgen05.commit frees smem stages / publishes finished accumulators;
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (one TMEM lane quarter per warp), then
-//               SwiGLU (GEMM-1: gate columns 0..127 and up columns 128..255 of one accumulator)
-//               or a plain bf16 cast (GEMM-2), masked row/column stores.
-// The tile schedule (expert, row block, column block) is derived on the device from
-// expert_offsets, so nothing is synchronised with the host.  Row blocks of an expert are the
-// fastest-varying index, so CTAs running together share weight column blocks through L2.
-// Every mbarrier and counter wait is bounded; on a timeout the CTA records MOE status bit
-// kStatusTimeout, drains its own outstanding TMA loads and MMAs, frees TMEM and returns.
+// Two persistent kernels split the experts by size, each running all GEMM-1 tiles of its experts
+// and then all their GEMM-2 tiles (a GEMM-2 tile waits on per-row-block completion counters of
+// the GEMM-1 tiles), with tiles claimed at run time from a global counter:
+//
+// * ffn_pair_kernel: experts with two or more 128-row blocks.  A 2-CTA cluster computes a tile of
+//   (expert, pair of row blocks, column block) as one 256 x 256 product with
+//   tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16): CTA v holds its row block of A and rows
+//   [128v, 128v + 128) of the 256 weight rows of B, so each SM stages half of the weight tile per
+//   k-step, a stage is 32 KB and six are in flight; CTA v's TMEM receives its 128 rows x 256
+//   columns.  GEMM-1 puts the gate rows in CTA 0's half of B and the up rows in CTA 1's.  CTA 1's
+//   TMA loads complete their bytes on CTA 0's barriers, CTA 0's single MMA thread issues for both
+//   and its commits arrive on both CTAs' barriers (multicast commit, not multicast loads).
+// * ffn_single_kernel: experts with one row block (mostly a handful of rows, so a tile is bound
+//   by streaming the expert's weights, not by the MMA).  One CTA per tile: tcgen05.mma.cta_group::1
+//   (M = 128, N = 256), 48 KB stages (the A box shrinks to the rows present), four in flight.
+//
+// Roles (192 threads): warp 0 = TMA producer (CTA 0 of a pair also claims tiles and passes the ids
+// to both CTAs through shared-memory queues); warp 1 = TMEM allocation and the MMA thread;
+// warps 2..5 = epilogue of the CTA's 128 rows: tcgen05.ld of the accumulator, then SwiGLU (GEMM-1:
+// gate columns 0..127 and up columns 128..255 of one accumulator) or a bf16 cast (GEMM-2), masked
+// row / column stores.  Two 256-column accumulators let the epilogue of one tile overlap the MMAs
+// of the next.  Every mbarrier and counter wait is bounded; on a timeout a CTA records
+// kStatusTimeout (and stops its peer), drains what it issued, and both CTAs of a pair meet at the
+// final cluster barrier before TMEM is freed.  No TMA multicast anywhere.  The tile schedules are
+// derived on the device from expert_offsets, so nothing is synchronised with the host.
 // For the FP8 payload a separate pass (dequant_fp8_kernel) first writes the bf16 input rows.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -36,29 +43,24 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 128;          // rows per tile (UMMA M, one TMEM lane per row)
+constexpr int BM = 128;          // rows per CTA tile (one TMEM lane per row)
 constexpr int BK = 64;           // k per stage: 64 bf16 = one 128-byte swizzle atom row
 constexpr int UMMA_K = 16;       // k per tcgen05.mma for kind::f16
-constexpr int kStages = 4;
 constexpr int kAccCols = 256;    // fp32 TMEM columns per accumulator
 constexpr int kTmemCols = 512;   // two accumulators
 constexpr int kThreads = 192;
-constexpr int kATileBytes = BM * BK * 2;   // 16 KB
-constexpr int kBTileBytes = 256 * BK * 2;  // 32 KB
-constexpr int kStageBytes = kATileBytes + kBTileBytes;
-
-// Experts with at least this many 128-row blocks are "hot" (their weight blocks are reused from L2
-// by several row blocks, so their tiles are tensor-bound); their tiles are interleaved evenly with
-// the other experts' tiles, which stream weights from HBM, so both kinds run at the same time.
-// 0 disables the interleave (plain expert order).
-#ifndef MOE_FFN_HOT_MTILES
-#define MOE_FFN_HOT_MTILES 2
-#endif
-constexpr int kGemm2NTile = 256;  // output columns per GEMM-2 tile (128 measured slower)
-// Tiles are claimed at run time from a global counter by the producer; a kTileQ-deep shared-memory
-// queue passes the ids to the MMA thread and the epilogue warps.
+constexpr int kATileBytes = BM * BK * 2;   // 16 KB: 128 rows of A
+constexpr int kBHalfBytes = 128 * BK * 2;  // 16 KB: 128 weight rows
+// Experts with at least this many row blocks run in the pair kernel, the others in the single one.
+constexpr int kPairMinBlocks = 2;
+// Pair kernel: six 32-KB stages (A rows + half of B); single kernel: four 48-KB stages (A + B).
+constexpr int kStagesPair = 6;
+constexpr int kStagesSingle = 4;
 constexpr int kTileQ = 4;
-
+// Consumers of a pair kernel's queue slot, all arriving on CTA 0's q_empty: CTA 0's MMA thread and
+// four epilogue warps, CTA 1's producer and four epilogue warps.
+constexpr int kPairQueueConsumers = 10;
+constexpr int kSingleQueueConsumers = 5;  // the MMA thread and four epilogue warps
 
 // ---- PTX wrappers ------------------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm, uint32_t bar,
@@ -69,25 +71,21 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm,
       "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(bar)
       : "memory");
 }
+// CTA 1's copy into its own shared memory, completing its bytes on CTA 0's barrier `bar_cta0`
+// (a shared::cluster address); a plain (not multicast) load.
+__device__ __forceinline__ void tma_load_2d_to_leader(uint32_t dst, const CUtensorMap* tm,
+                                                      uint32_t bar_cta0, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(bar_cta0)
+      : "memory");
+}
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
 }
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
@@ -104,6 +102,118 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+// cta_group::1 (single kernel)
+__device__ __forceinline__ void tc_commit1(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tc_mma1(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                        uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// cta_group::2 (pair kernel)
+// Arrive once on the mbarrier at this shared-memory offset in BOTH CTAs of the pair when the MMAs
+// issued so far have completed.
+__device__ __forceinline__ void tc_commit2_both(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar),
+      "h"(static_cast<uint16_t>(3))
+      : "memory");
+}
+// Arrive on this CTA's own mbarrier when the MMAs issued so far have completed.
+__device__ __forceinline__ void tc_commit2_local(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma2(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                        uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// ---- cluster helpers ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Shared::cluster address of the same shared-memory offset in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t peer_addr(uint32_t local, uint32_t rank) {
+  uint32_t out;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(local), "r"(rank));
+  return out;
+}
+__device__ __forceinline__ void st_cluster_s32(uint32_t cluster_addr, int v) {
+  asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+// Arrive on an mbarrier of the other CTA, releasing this thread's prior writes at cluster scope.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cl(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+
+// Abort state of a CTA: its own flag and, in the pair kernel, the peer's flag, so that a timeout
+// in either CTA ends the waits of both.
+struct Abort {
+  volatile int* local;
+  uint32_t peer;  // shared::cluster address of the peer's flag (pair kernel only)
+  bool has_peer;
+  int* status;
+  __device__ __forceinline__ void raise_timeout() const {
+    *local = 1;
+    if (has_peer) st_cluster_s32(peer, 1);
+    record_status(status, kStatusTimeout);
+  }
+};
+
+// Bounded wait on an mbarrier phase (arrivals may come from either CTA of a pair).  False if this
+// CTA is aborting or the limit ran out (which raises the abort).
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Abort& ab) {
+  if (mbar_try_wait_cl(bar, parity)) return true;
+  const unsigned long long t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait_cl(bar, parity)) return true;
+    if (*ab.local) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      ab.raise_timeout();
+      return false;
+    }
+  }
+}
+// The same wait that ignores the abort flag (used to drain a CTA's own copies and MMAs).
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait_cl(bar, parity)) return;
+  const unsigned long long t0 = global_timer_ns();
+  while (!mbar_try_wait_cl(bar, parity) && global_timer_ns() - t0 <= kWaitLimitNs) {
+  }
 }
 
 // Shared-memory matrix descriptor of a K-major bf16 tile stored with the 128-byte swizzle:
@@ -130,7 +240,7 @@ __host__ __device__ constexpr uint32_t make_idesc(int M, int N) {
 
 __device__ __forceinline__ int owner_of(const int* start, int E, int idx) {
   int lo = 0, hi = E - 1;
-  while (lo < hi) {  // largest expert whose first tile is <= idx (it owns the tile)
+  while (lo < hi) {  // largest expert whose first unit is <= idx (it owns the tile)
     const int mid = (lo + hi + 1) >> 1;
     if (start[mid] <= idx) lo = mid; else hi = mid - 1;
   }
@@ -139,118 +249,6 @@ __device__ __forceinline__ int owner_of(const int* start, int E, int idx) {
 
 __device__ __forceinline__ float silu_mul(float g, float u) {
   return g / (1.0f + expf(-g)) * u;
-}
-
-// ---- fused FFN: GEMM-1 (gate|up + SwiGLU) and GEMM-2 (down) tiles in one persistent launch -------
-//
-// Tiles are numbered [all GEMM-1 tiles][all GEMM-2 tiles]; CTAs claim them in increasing order
-// from an atomic counter.
-// A GEMM-2 tile (expert e, row block m) reads the rows of h that the GEMM-1 tiles of (e, m) write,
-// so its producer first waits (bounded) until the completion counter of (e, m) reaches 4 * n1 (four
-// epilogue warps per GEMM-1 tile, n1 column blocks).  GEMM-1 tiles never wait, and every GEMM-1
-// tile is claimed before any GEMM-2 tile, by a CTA that finishes it without waiting, so with all
-// CTAs resident (one per SM) the waits always end; they are bounded anyway.  Writers: st.global of h, fence.proxy.async (generic -> async proxy), release increment.
-// Readers: acquire load of the counter, fence.proxy.async, then the TMA loads of h.
-struct FfnArgs {
-  const int32_t* expert_offsets;  // [E+1], device
-  int E, max_rows, H, F;
-  __nv_bfloat16* h;               // [max_rows, F] workspace
-  __nv_bfloat16* out;             // [max_rows, H]
-  int* status;
-  int* done;                      // [row blocks] GEMM-1 completion counters, zero on entry
-  int* used;                      // [row blocks] GEMM-2 tiles that passed the wait, zero on entry
-  int* sched;                     // [2] next tile to claim, CTAs that finished; zero on entry
-};
-
-struct FSmem {
-  uint8_t* tiles;
-  uint64_t *full, *empty, *acc_full, *acc_empty, *drain, *q_full, *q_empty;
-  int* tile_q;   // [kTileQ] claimed tile ids (-1: no more tiles)
-  uint32_t* tmem_base;
-  int* abort_flag;
-  int* off;      // [E+1] row offsets (clamped to max_rows)
-  int* mt;       // [E]   row blocks per expert
-  int* ms_all;   // [E+1] first global row block of each expert
-  int* ms_cold;  // [E+1] first row block of each non-hot expert among non-hot row blocks
-  int* ms_hot;   // [E+1] same among hot row blocks
-  int* totals;   // [2] non-hot, hot row blocks
-};
-
-__device__ __forceinline__ FSmem fcarve(uint8_t* raw, int E) {
-  FSmem s;
-  const uint32_t a = smem_addr(raw);
-  uint8_t* p = raw + ((1024u - (a & 1023u)) & 1023u);
-  s.tiles = p;
-  p += kStages * kStageBytes;
-  s.full = reinterpret_cast<uint64_t*>(p);
-  s.empty = s.full + kStages;
-  s.acc_full = s.empty + kStages;
-  s.acc_empty = s.acc_full + 2;
-  s.drain = s.acc_empty + 2;
-  s.q_full = s.drain + 1;
-  s.q_empty = s.q_full + kTileQ;
-  s.tmem_base = reinterpret_cast<uint32_t*>(s.q_empty + kTileQ);
-  s.abort_flag = reinterpret_cast<int*>(s.tmem_base + 1);
-  s.tile_q = s.abort_flag + 2;
-  s.off = s.tile_q + kTileQ;
-  s.mt = s.off + (E + 1);
-  s.ms_all = s.mt + E;
-  s.ms_cold = s.ms_all + (E + 1);
-  s.ms_hot = s.ms_cold + (E + 1);
-  s.totals = s.ms_hot + (E + 1);
-  return s;
-}
-
-size_t fused_smem_bytes(int E) {
-  return 1024 + static_cast<size_t>(kStages) * kStageBytes + 8 * (2 * kStages + 5 + 2 * kTileQ) +
-         16 + sizeof(int) * (5 * static_cast<size_t>(E) + 8 + kTileQ);
-}
-
-struct FTile {
-  int phase;  // 1: GEMM-1 (SwiGLU), 2: GEMM-2 (down)
-  int e, m_blk, n_blk, mg;
-};
-
-// Tile -> phase, expert, row block, column block (row blocks fastest inside an expert); hot and
-// non-hot experts' tiles are spread evenly over each phase as in the two-launch kernel.
-__device__ __forceinline__ FTile fdecode(const FSmem& s, int E, int n1, int n2, int tile) {
-  FTile t;
-  const int MC = s.totals[0], MH = s.totals[1];
-  const int N1 = (MC + MH) * n1;
-  int nt, idx;
-  if (tile < N1) {
-    t.phase = 1;
-    nt = n1;
-    idx = tile;
-  } else {
-    t.phase = 2;
-    nt = n2;
-    idx = tile - N1;
-  }
-  const int* ms = s.ms_cold;
-  if (MH > 0) {
-    if (MC == 0) {
-      ms = s.ms_hot;
-    } else {
-      const long long Nt = static_cast<long long>(MC + MH) * nt;
-      const long long hn = static_cast<long long>(MH) * nt;
-      const long long h0 = static_cast<long long>(idx) * hn / Nt;
-      const long long h1 = static_cast<long long>(idx + 1) * hn / Nt;
-      if (h1 > h0) {
-        ms = s.ms_hot;
-        idx = static_cast<int>(h0);
-      } else {
-        idx -= static_cast<int>(h0);
-      }
-    }
-  }
-  t.e = owner_of(ms, E, idx / nt);
-  const int local = idx - nt * ms[t.e];
-  const int mt = s.mt[t.e];
-  t.n_blk = local / mt;
-  t.m_blk = local - t.n_blk * mt;
-  t.mg = s.ms_all[t.e] + t.m_blk;
-  return t;
 }
 
 __device__ __forceinline__ int ld_acquire(const int* p) {
@@ -264,17 +262,15 @@ __device__ __forceinline__ void red_release_add(int* p, int v) {
 }
 
 // Bounded wait until *p >= target (acquire).  False if the CTA aborts or the limit runs out.
-__device__ __forceinline__ bool wait_counter(const int* p, int target, volatile int* abort_flag,
-                                             int* status) {
+__device__ __forceinline__ bool wait_counter(const int* p, int target, const Abort& ab) {
   if (ld_acquire(p) >= target) return true;
   const unsigned long long t0 = global_timer_ns();
   while (true) {
     __nanosleep(64);
     if (ld_acquire(p) >= target) return true;
-    if (*abort_flag) return false;
+    if (*ab.local) return false;
     if (global_timer_ns() - t0 > kWaitLimitNs) {
-      *abort_flag = 1;
-      record_status(status, kStatusTimeout);
+      ab.raise_timeout();
       return false;
     }
   }
@@ -290,53 +286,576 @@ __host__ __device__ constexpr int small_box_rows(int i) { return 16 << i; }
 __device__ __forceinline__ int small_box_index(int rows) {
   return rows <= 16 ? 0 : (rows <= 32 ? 1 : (rows <= 64 ? 2 : 3));
 }
+// Bytes of the A box that covers `rows` rows (0 when there are none).
+__device__ __forceinline__ uint32_t a_box_bytes(int rows) {
+  if (rows <= 0) return 0u;
+  const int bi = small_box_index(rows);
+  return bi < 3 ? static_cast<uint32_t>(small_box_rows(bi) * BK * 2) : kATileBytes;
+}
 
+// ---- tile schedule -------------------------------------------------------------------------------
+//
+// The tiles of a kernel are numbered [all GEMM-1 tiles][all GEMM-2 tiles] over the experts of its
+// class; inside a phase expert by expert, column block by column block, with the units (row
+// blocks, or pairs of row blocks) fastest, so tiles running together share a weight column block
+// through L2.  A GEMM-2 tile reads the rows of h that the GEMM-1 tiles of its row block write, so
+// its producer first waits (bounded) until the block's completion counter reaches 4 * n1 (four
+// epilogue warps per GEMM-1 tile, n1 column blocks).  GEMM-1 tiles never wait, and every GEMM-1
+// tile is claimed before any GEMM-2 tile, by a CTA that finishes it without waiting, so the waits
+// of running CTAs always end; they are bounded anyway.  Writers: st.global of h, fence.proxy.async
+// (generic -> async proxy), release increment.  Readers: acquire load of the counter,
+// fence.proxy.async, then the TMA loads of h.
+struct FfnArgs {
+  const int32_t* expert_offsets;  // [E+1], device
+  int E, max_rows, H, F;
+  __nv_bfloat16* h;               // [max_rows, F] workspace
+  __nv_bfloat16* out;             // [max_rows, H]
+  int* status;
+  int* done;                      // [row blocks] GEMM-1 completion counters, zero on entry
+  int* used;                      // [row blocks] GEMM-2 tiles that passed the wait, zero on entry
+  int* sched;                     // [2] this kernel's next tile to claim, CTAs that finished
+};
+
+struct Tables {
+  int* off;     // [E+1] row offsets (clamped to max_rows)
+  int* mt;      // [E]   row blocks per expert
+  int* units;   // [E]   units of this kernel's class per expert (0 for the other class)
+  int* ms_rb;   // [E+1] first global row block of each expert (over all experts)
+  int* ms_u;    // [E+1] first unit of each expert among this kernel's units
+};
+__host__ __device__ constexpr int table_ints(int E) { return 5 * E + 3; }
+
+__device__ __forceinline__ Tables carve_tables(int* p, int E) {
+  Tables t;
+  t.off = p;
+  t.mt = t.off + (E + 1);
+  t.units = t.mt + E;
+  t.ms_rb = t.units + E;
+  t.ms_u = t.ms_rb + (E + 1);
+  return t;
+}
+
+// One warp builds the tables from expert_offsets (warp scans).  PAIRS: the units are pairs of row
+// blocks of the experts with >= kPairMinBlocks blocks; otherwise the row blocks of the others.
+template <bool PAIRS>
+__device__ __forceinline__ void build_tables(const Tables& tb, const FfnArgs& args, int lane) {
+  const int E = args.E;
+  int carry_r = 0, carry_u = 0;
+  for (int e0 = 0; e0 < E; e0 += 32) {
+    const int e = e0 + lane;
+    int lo = 0, hi = 0;
+    if (e < E) {
+      lo = min(__ldg(args.expert_offsets + e), args.max_rows);
+      hi = min(__ldg(args.expert_offsets + e + 1), args.max_rows);
+    }
+    const int mt = (max(hi - lo, 0) + BM - 1) / BM;
+    const bool paired = mt >= kPairMinBlocks;
+    const int u = PAIRS ? (paired ? (mt + 1) / 2 : 0) : (paired ? 0 : mt);
+    int ir = mt, iu = u;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int yr = __shfl_up_sync(0xFFFFFFFFu, ir, o);
+      const int yu = __shfl_up_sync(0xFFFFFFFFu, iu, o);
+      if (lane >= o) {
+        ir += yr;
+        iu += yu;
+      }
+    }
+    if (e < E) {
+      tb.off[e] = lo;
+      tb.mt[e] = mt;
+      tb.units[e] = u;
+      tb.ms_rb[e] = carry_r + ir - mt;
+      tb.ms_u[e] = carry_u + iu - u;
+    }
+    carry_r += __shfl_sync(0xFFFFFFFFu, ir, 31);
+    carry_u += __shfl_sync(0xFFFFFFFFu, iu, 31);
+  }
+  if (lane == 0) {
+    tb.ms_rb[E] = carry_r;
+    tb.ms_u[E] = carry_u;
+    tb.off[E] = min(__ldg(args.expert_offsets + E), args.max_rows);
+  }
+}
+
+struct FTile {
+  int phase;  // 1: GEMM-1 (SwiGLU), 2: GEMM-2 (down)
+  int e, unit, n_blk;
+};
+
+__device__ __forceinline__ FTile fdecode(const Tables& tb, int E, int n1, int n2, int tile) {
+  FTile t;
+  const int U = tb.ms_u[E];
+  int nt, idx;
+  if (tile < U * n1) {
+    t.phase = 1;
+    nt = n1;
+    idx = tile;
+  } else {
+    t.phase = 2;
+    nt = n2;
+    idx = tile - U * n1;
+  }
+  t.e = owner_of(tb.ms_u, E, idx / nt);
+  const int local = idx - nt * tb.ms_u[t.e];
+  const int u = tb.units[t.e];
+  t.n_blk = local / u;
+  t.unit = local - t.n_blk * u;
+  return t;
+}
+
+// GEMM-2 producer side of row block m_blk of expert e: wait for its rows of h, then the last of the
+// n2 GEMM-2 tiles of the block to get here returns both counters to zero, so the workspace is
+// ready for the next call without a memset.
+__device__ __forceinline__ bool gemm2_acquire(const FfnArgs& args, const Tables& tb, int e,
+                                              int m_blk, int n1, int n2, const Abort& ab) {
+  const int rb = tb.ms_rb[e] + m_blk;
+  if (!wait_counter(args.done + rb, 4 * n1, ab)) return false;
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  if (atomicAdd(args.used + rb, 1) == n2 - 1) {
+    atomicExch(args.done + rb, 0);
+    atomicExch(args.used + rb, 0);
+  }
+  return true;
+}
+
+// Epilogue of one accumulator for this warp's 32 rows (r_local) of row block m_blk of expert e.
+__device__ __forceinline__ void epilogue_tile(const FfnArgs& args, const Tables& tb, int phase,
+                                              int e, int m_blk, int n_blk, uint32_t t_row,
+                                              int r_local, int lane) {
+  const int row = tb.off[e] + m_blk * BM + r_local;
+  const bool row_ok = row < tb.off[e + 1];
+  if (phase == 1) {
+    __nv_bfloat16* out_row = args.h + static_cast<size_t>(row) * args.F;
+#pragma unroll 1
+    for (int c = 0; c < 128; c += 32) {
+      uint32_t g[32], u[32];
+      tmem_ld32(t_row + c, g);
+      tmem_ld32(t_row + 128 + c, u);
+      tmem_wait_ld();
+      const int col = n_blk * 128 + c;
+      if (row_ok && col < args.F) {
+        uint32_t packed[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float h0 = silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i]));
+          const float h1 = silu_mul(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1]));
+          packed[i] = pack_bf16x2(h0, h1);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(out_row + col);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+      }
+    }
+    if (m_blk < tb.mt[e]) {
+      // publish: this warp's rows of h for (e, block, n) are written
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) red_release_add(args.done + tb.ms_rb[e] + m_blk, 1);
+    }
+  } else {
+    __nv_bfloat16* out_row = args.out + static_cast<size_t>(row) * args.H;
+#pragma unroll 1
+    for (int c = 0; c < 256; c += 32) {
+      uint32_t v[32];
+      tmem_ld32(t_row + c, v);
+      tmem_wait_ld();
+      const int col = n_blk * 256 + c;
+      if (row_ok && col < args.H) {
+        uint32_t packed[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          packed[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+        uint4* dst = reinterpret_cast<uint4*>(out_row + col);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+      }
+    }
+  }
+}
+
+// Shared-memory layout common to both kernels: the stage ring, the mbarriers, the tile queue and
+// the tables.
+struct Ring {
+  uint8_t* tiles;
+  uint64_t *full, *empty, *acc_full, *acc_empty, *drain, *q_full, *q_empty;
+  int* tile_q;  // [kTileQ] claimed tile ids (-1: no more tiles)
+  uint32_t* tmem_base;
+  int* abort_flag;
+  Tables tb;
+};
+
+__device__ __forceinline__ Ring carve(uint8_t* raw, int E, int stages, int stage_bytes) {
+  Ring s;
+  const uint32_t a = smem_addr(raw);
+  uint8_t* p = raw + ((1024u - (a & 1023u)) & 1023u);
+  s.tiles = p;
+  p += static_cast<size_t>(stages) * stage_bytes;
+  s.full = reinterpret_cast<uint64_t*>(p);
+  s.empty = s.full + stages;
+  s.acc_full = s.empty + stages;
+  s.acc_empty = s.acc_full + 2;
+  s.drain = s.acc_empty + 2;
+  s.q_full = s.drain + 1;
+  s.q_empty = s.q_full + kTileQ;
+  s.tmem_base = reinterpret_cast<uint32_t*>(s.q_empty + kTileQ);
+  s.abort_flag = reinterpret_cast<int*>(s.tmem_base + 1);
+  s.tile_q = s.abort_flag + 2;
+  s.tb = carve_tables(s.tile_q + kTileQ, E);
+  return s;
+}
+
+size_t ring_smem_bytes(int E, int stages, int stage_bytes) {
+  return 1024 + static_cast<size_t>(stages) * stage_bytes +
+         8 * (2 * static_cast<size_t>(stages) + 5 + 2 * kTileQ) + 16 +
+         sizeof(int) * (static_cast<size_t>(table_ints(E)) + 2 + kTileQ);
+}
+
+__device__ __forceinline__ void init_ring(const Ring& s, int stages, int acc_empty_count,
+                                          int q_consumers) {
+  for (int i = 0; i < stages; ++i) {
+    mbar_init(smem_addr(&s.full[i]), 1);
+    mbar_init(smem_addr(&s.empty[i]), 1);
+  }
+  for (int i = 0; i < 2; ++i) {
+    mbar_init(smem_addr(&s.acc_full[i]), 1);
+    mbar_init(smem_addr(&s.acc_empty[i]), acc_empty_count);
+  }
+  mbar_init(smem_addr(s.drain), 1);
+  for (int i = 0; i < kTileQ; ++i) {
+    mbar_init(smem_addr(&s.q_full[i]), 1);
+    mbar_init(smem_addr(&s.q_empty[i]), q_consumers);
+  }
+  *s.abort_flag = 0;
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Next tile id from this CTA's queue (bounded).  remote_empty: the slot's q_empty is CTA 0's.
+__device__ __forceinline__ bool take_tile(const Ring& s, int& qi, uint32_t& qph, bool remote_empty,
+                                          const Abort& ab, int& tile) {
+  if (!wait_bar(smem_addr(&s.q_full[qi]), qph, ab)) return false;
+  tile = s.tile_q[qi];
+  const uint32_t qe = smem_addr(&s.q_empty[qi]);
+  if (remote_empty)
+    mbar_arrive_cluster(peer_addr(qe, 0));
+  else
+    mbar_arrive(qe);
+  if (++qi == kTileQ) {
+    qi = 0;
+    qph ^= 1u;
+  }
+  return true;
+}
+
+// The epilogue warps' queue step: lane 0 takes the tile, every lane advances its slot index.
+__device__ __forceinline__ bool warp_take_tile(const Ring& s, int& qi, uint32_t& qph,
+                                               bool remote_empty, const Abort& ab, int lane,
+                                               int& tile) {
+  bool okq = true;
+  tile = -1;
+  if (lane == 0) {
+    okq = take_tile(s, qi, qph, remote_empty, ab, tile);
+  } else if (++qi == kTileQ) {
+    qi = 0;
+    qph ^= 1u;
+  }
+  okq = __shfl_sync(0xFFFFFFFFu, okq ? 1 : 0, 0) != 0;
+  tile = __shfl_sync(0xFFFFFFFFu, tile, 0);
+  return okq;
+}
+
+__device__ __forceinline__ void prefetch_maps(const CUtensorMap* a, const CUtensorMap* b,
+                                              const CUtensorMap* c, const CUtensorMap* d,
+                                              const CUtensorMap* e, const SmallBoxMaps& xs,
+                                              const SmallBoxMaps& hs) {
+  const CUtensorMap* all[5] = {a, b, c, d, e};
+  for (int i = 0; i < 5; ++i)
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(all[i])) : "memory");
+  for (int i = 0; i < 3; ++i) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xs.m[i])) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&hs.m[i])) : "memory");
+  }
+}
+
+// Every claim of this CTA is done: the last CTA of the grid to get here returns this kernel's
+// claim counters to zero.
+__device__ __forceinline__ void release_schedule(int* sched) {
+  __threadfence();
+  if (atomicAdd(sched + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+    atomicExch(sched, 0);
+    atomicExch(sched + 1, 0);
+  }
+}
+
+// ================================================================================================
+// Pair kernel: experts with >= kPairMinBlocks row blocks; 2-CTA clusters, cta_group::2.
+// ================================================================================================
 __global__ void __launch_bounds__(kThreads, 1)
-    fused_ffn_kernel(const __grid_constant__ CUtensorMap tm_x,
-                     const __grid_constant__ SmallBoxMaps tm_xs,
-                     const __grid_constant__ CUtensorMap tm_g,
-                     const __grid_constant__ CUtensorMap tm_u,
-                     const __grid_constant__ CUtensorMap tm_h,
-                     const __grid_constant__ SmallBoxMaps tm_hs,
-                     const __grid_constant__ CUtensorMap tm_d, const FfnArgs args) {
+    ffn_pair_kernel(const __grid_constant__ CUtensorMap tm_x,
+                    const __grid_constant__ SmallBoxMaps tm_xs,
+                    const __grid_constant__ CUtensorMap tm_g,
+                    const __grid_constant__ CUtensorMap tm_u,
+                    const __grid_constant__ CUtensorMap tm_h,
+                    const __grid_constant__ SmallBoxMaps tm_hs,
+                    const __grid_constant__ CUtensorMap tm_d128, const FfnArgs args) {
+  constexpr int kStages = kStagesPair;
+  constexpr int kStageBytes = kATileBytes + kBHalfBytes;
   extern __shared__ uint8_t smem_raw[];
   const int E = args.E;
-  FSmem s = fcarve(smem_raw, E);
+  const Ring s = carve(smem_raw, E, kStages, kStageBytes);
+  const Tables& tb = s.tb;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n1 = (args.F + 127) / 128;       // GEMM-1 column blocks (128 h columns each)
-  const int n2 = (args.H + 255) / 256;       // GEMM-2 column blocks (256 output columns each)
+  const uint32_t rank = cluster_rank();  // CTA 0 claims the tiles and issues the MMAs
+  const int n1 = (args.F + 127) / 128;   // GEMM-1 column blocks (128 h columns each)
+  const int n2 = (args.H + 255) / 256;   // GEMM-2 column blocks (256 output columns each)
   const int kb1 = (args.H + BK - 1) / BK, kb2 = (args.F + BK - 1) / BK;
-  volatile int* abort_flag = s.abort_flag;
+  const Abort ab{s.abort_flag, peer_addr(smem_addr(s.abort_flag), rank ^ 1u), true, args.status};
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int i = 0; i < kStages; ++i) {
-        mbar_init(smem_addr(&s.full[i]), 1);
-        mbar_init(smem_addr(&s.empty[i]), 1);
+      init_ring(s, kStages, 8, kPairQueueConsumers);  // acc_empty: four epilogue warps per CTA
+      prefetch_maps(&tm_x, &tm_g, &tm_u, &tm_h, &tm_d128, tm_xs, tm_hs);
+    }
+  } else if (warp == 1) {
+    // the same warp of both CTAs allocates, as cta_group::2 requires
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(s.tmem_base)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  } else if (warp == 2) {
+    griddep_wait();
+    build_tables<true>(tb, args, lane);
+  }
+  griddep_wait();
+  griddep_launch_dependents();
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers are initialised before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem_base = *s.tmem_base;
+  const int U = tb.ms_u[E];
+  const int total_tiles = U * (n1 + n2);
+  const uint32_t tiles_base = smem_addr(s.tiles);
+  volatile int* abort_flag = s.abort_flag;
+
+  if (warp == 0) {
+    // ---- TMA producer of this CTA's A rows and B half ------------------------------------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_parity = 0;
+      int qi = 0;
+      uint32_t qph = 0;
+      while (!*abort_flag) {
+        int tile;
+        if (rank == 0) {
+          tile = atomicAdd(args.sched, 1);
+          if (tile >= total_tiles) tile = -1;
+          // hand the id to the consumers of both CTAs
+          if (!wait_bar(smem_addr(&s.q_empty[qi]), qph ^ 1u, ab)) break;
+          s.tile_q[qi] = tile;
+          st_cluster_s32(peer_addr(smem_addr(&s.tile_q[qi]), 1), tile);
+          mbar_arrive(smem_addr(&s.q_full[qi]));
+          mbar_arrive_cluster(peer_addr(smem_addr(&s.q_full[qi]), 1));
+          if (++qi == kTileQ) {
+            qi = 0;
+            qph ^= 1u;
+          }
+        } else {
+          if (!take_tile(s, qi, qph, true, ab, tile)) break;
+        }
+        if (tile < 0) break;
+        const FTile t = fdecode(tb, E, n1, n2, tile);
+        const int m_blk = 2 * t.unit + static_cast<int>(rank);  // this CTA's row block
+        const int row_a = tb.off[t.e] + m_blk * BM;
+        const int rows = m_blk < tb.mt[t.e] ? min(BM, tb.off[t.e + 1] - row_a) : 0;
+        const int bi = small_box_index(rows);
+        // CTA 0's barrier counts both CTAs' bytes of each stage
+        const int row_a1 = tb.off[t.e] + (2 * t.unit + 1) * BM;
+        const int rows1 = 2 * t.unit + 1 < tb.mt[t.e] ? min(BM, tb.off[t.e + 1] - row_a1) : 0;
+        const int row_a0 = tb.off[t.e] + 2 * t.unit * BM;
+        const int rows0 = min(BM, tb.off[t.e + 1] - row_a0);
+        const uint32_t stage_tx = a_box_bytes(rows0) + a_box_bytes(rows1) + 2 * kBHalfBytes;
+        int nkb;
+        const CUtensorMap *ma, *mb;
+        int row_b;
+        if (t.phase == 1) {
+          nkb = kb1;
+          ma = bi < 3 ? &tm_xs.m[bi] : &tm_x;
+          mb = rank == 0 ? &tm_g : &tm_u;  // gate rows -> accumulator columns 0..127, up -> 128..
+          row_b = t.e * args.F + t.n_blk * 128;
+        } else {
+          if (rows > 0 && !gemm2_acquire(args, tb, t.e, m_blk, n1, n2, ab)) break;
+          nkb = kb2;
+          ma = bi < 3 ? &tm_hs.m[bi] : &tm_h;
+          mb = &tm_d128;
+          row_b = t.e * args.H + t.n_blk * 256 + static_cast<int>(rank) * 128;
+        }
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!wait_bar(smem_addr(&s.empty[stage]), phase ^ 1u, ab)) {
+            ok = false;
+            break;
+          }
+          const uint32_t a_dst = tiles_base + stage * kStageBytes;
+          const uint32_t b_dst = a_dst + kATileBytes;
+          const uint32_t fb = smem_addr(&s.full[stage]);
+          if (rank == 0) {
+            mbar_arrive_expect_tx(fb, stage_tx);
+            if (rows > 0) tma_load_2d(a_dst, ma, fb, kb * BK, row_a);
+            tma_load_2d(b_dst, mb, fb, kb * BK, row_b);
+          } else {
+            const uint32_t fb0 = peer_addr(fb, 0);
+            if (rows > 0) tma_load_2d_to_leader(a_dst, ma, fb0, kb * BK, row_a);
+            tma_load_2d_to_leader(b_dst, mb, fb0, kb * BK, row_b);
+          }
+          issued_mask |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
       }
-      for (int i = 0; i < 2; ++i) {
-        mbar_init(smem_addr(&s.acc_full[i]), 1);
-        mbar_init(smem_addr(&s.acc_empty[i]), 4);
+      if (*abort_flag) {
+        if (rank == 0) {
+          // CTA 0's barriers count both CTAs' bytes: wait for the latest phase of each stage
+          for (int st = 0; st < kStages; ++st)
+            if (issued_mask & (1u << st)) drain_wait(smem_addr(&s.full[st]), (issued_parity >> st) & 1u);
+        } else if (issued_mask != 0) {
+          // CTA 1's copies complete on CTA 0's barriers: give them time to land (a copy takes
+          // microseconds) before this CTA may leave
+          const unsigned long long t0 = global_timer_ns();
+          while (global_timer_ns() - t0 < 100000ull) __nanosleep(1000);
+        }
       }
-      mbar_init(smem_addr(s.drain), 1);
-      for (int i = 0; i < kTileQ; ++i) {
-        mbar_init(smem_addr(&s.q_full[i]), 1);
-        mbar_init(smem_addr(&s.q_empty[i]), 5);  // the MMA thread and the four epilogue warps
+    }
+  } else if (warp == 1) {
+    // ---- MMA issuer (CTA 0): M = 256 over the pair, N = 256 ------------------------------------
+    if (rank == 0 && lane == 0) {
+      const uint32_t idesc = make_idesc(2 * BM, 256);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool issued_any = false;
+      int qi = 0;
+      uint32_t qph = 0;
+      for (int it = 0;; ++it) {
+        int tile;
+        if (!take_tile(s, qi, qph, false, ab, tile)) break;
+        if (tile < 0) break;
+        const int nkb = tile < U * n1 ? kb1 : kb2;
+        const int acc = it & 1;
+        const uint32_t acc_parity = (it >> 1) & 1;
+        if (!wait_bar(smem_addr(&s.acc_empty[acc]), acc_parity ^ 1u, ab)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * kAccCols;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!wait_bar(smem_addr(&s.full[stage]), phase, ab)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = tiles_base + stage * kStageBytes;
+          const uint32_t b_addr = a_addr + kATileBytes;
+#pragma unroll
+          for (int kk = 0; kk < BK / UMMA_K; ++kk)
+            tc_mma2(d_tmem, sw128_desc(a_addr + kk * UMMA_K * 2),
+                    sw128_desc(b_addr + kk * UMMA_K * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
+          issued_any = true;
+          tc_commit2_both(smem_addr(&s.empty[stage]));
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit2_both(smem_addr(&s.acc_full[acc]));
       }
-      *s.abort_flag = 0;
-      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_x)) : "memory");
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_g)) : "memory");
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_u)) : "memory");
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_h)) : "memory");
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_d)) : "memory");
-      for (int i = 0; i < 3; ++i) {
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_xs.m[i]))
-                     : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_hs.m[i]))
-                     : "memory");
+      if (issued_any) {
+        tc_commit2_local(smem_addr(s.drain));
+        drain_wait(smem_addr(s.drain), 0);
       }
+    }
+  } else {
+    // ---- epilogue of this CTA's 128 rows ---------------------------------------------------------
+    const int quarter = warp & 3;
+    const int r_local = quarter * 32 + lane;
+    const uint32_t acc_empty0 = smem_addr(&s.acc_empty[0]);
+    int qi = 0;
+    uint32_t qph = 0;
+    for (int it = 0;; ++it) {
+      int tile;
+      if (!warp_take_tile(s, qi, qph, rank != 0, ab, lane, tile) || tile < 0) break;
+      const FTile t = fdecode(tb, E, n1, n2, tile);
+      const int acc = it & 1;
+      const uint32_t acc_parity = (it >> 1) & 1;
+      bool ok = true;
+      if (lane == 0) ok = wait_bar(smem_addr(&s.acc_full[acc]), acc_parity, ab);
+      if (!__shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0)) break;
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + acc * kAccCols + (static_cast<uint32_t>(quarter * 32) << 16);
+      epilogue_tile(args, tb, t.phase, t.e, 2 * t.unit + static_cast<int>(rank), t.n_blk, t_row,
+                    r_local, lane);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        const uint32_t ae = acc_empty0 + acc * 8;
+        if (rank == 0)
+          mbar_arrive(ae);
+        else
+          mbar_arrive_cluster(peer_addr(ae, 0));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0) release_schedule(args.sched);
+  // neither CTA leaves (or frees TMEM) while the other may still touch its shared memory or TMEM
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// ================================================================================================
+// Single kernel: experts with one row block; one CTA per tile, cta_group::1.
+// ================================================================================================
+__global__ void __launch_bounds__(kThreads, 1)
+    ffn_single_kernel(const __grid_constant__ CUtensorMap tm_x,
+                      const __grid_constant__ SmallBoxMaps tm_xs,
+                      const __grid_constant__ CUtensorMap tm_g,
+                      const __grid_constant__ CUtensorMap tm_u,
+                      const __grid_constant__ CUtensorMap tm_h,
+                      const __grid_constant__ SmallBoxMaps tm_hs,
+                      const __grid_constant__ CUtensorMap tm_d256, const FfnArgs args) {
+  constexpr int kStages = kStagesSingle;
+  constexpr int kBTileBytes = 2 * kBHalfBytes;  // all 256 weight rows
+  constexpr int kStageBytes = kATileBytes + kBTileBytes;
+  extern __shared__ uint8_t smem_raw[];
+  const int E = args.E;
+  const Ring s = carve(smem_raw, E, kStages, kStageBytes);
+  const Tables& tb = s.tb;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n1 = (args.F + 127) / 128;
+  const int n2 = (args.H + 255) / 256;
+  const int kb1 = (args.H + BK - 1) / BK, kb2 = (args.F + BK - 1) / BK;
+  const Abort ab{s.abort_flag, 0u, false, args.status};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      init_ring(s, kStages, 4, kSingleQueueConsumers);
+      prefetch_maps(&tm_x, &tm_g, &tm_u, &tm_h, &tm_d256, tm_xs, tm_hs);
     }
   } else if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -346,48 +865,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   } else if (warp == 2) {
     griddep_wait();
-    int carry_a = 0, carry_c = 0, carry_h = 0;
-    for (int e0 = 0; e0 < E; e0 += 32) {
-      const int e = e0 + lane;
-      int lo = 0, hi = 0;
-      if (e < E) {
-        lo = min(__ldg(args.expert_offsets + e), args.max_rows);
-        hi = min(__ldg(args.expert_offsets + e + 1), args.max_rows);
-      }
-      const int mt = (max(hi - lo, 0) + BM - 1) / BM;
-      const bool hot = MOE_FFN_HOT_MTILES > 0 && mt >= MOE_FFN_HOT_MTILES;
-      const int mc = hot ? 0 : mt, mh = hot ? mt : 0;
-      int ia = mt, ic = mc, ih = mh;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int ya = __shfl_up_sync(0xFFFFFFFFu, ia, o);
-        const int yc = __shfl_up_sync(0xFFFFFFFFu, ic, o);
-        const int yh = __shfl_up_sync(0xFFFFFFFFu, ih, o);
-        if (lane >= o) {
-          ia += ya;
-          ic += yc;
-          ih += yh;
-        }
-      }
-      if (e < E) {
-        s.off[e] = lo;
-        s.mt[e] = mt;
-        s.ms_all[e] = carry_a + ia - mt;
-        s.ms_cold[e] = carry_c + ic - mc;
-        s.ms_hot[e] = carry_h + ih - mh;
-      }
-      carry_a += __shfl_sync(0xFFFFFFFFu, ia, 31);
-      carry_c += __shfl_sync(0xFFFFFFFFu, ic, 31);
-      carry_h += __shfl_sync(0xFFFFFFFFu, ih, 31);
-    }
-    if (lane == 0) {
-      s.ms_all[E] = carry_a;
-      s.ms_cold[E] = carry_c;
-      s.ms_hot[E] = carry_h;
-      s.totals[0] = carry_c;
-      s.totals[1] = carry_h;
-      s.off[E] = min(__ldg(args.expert_offsets + E), args.max_rows);
-    }
+    build_tables<false>(tb, args, lane);
   }
   griddep_wait();
   griddep_launch_dependents();
@@ -395,8 +873,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s.tmem_base;
-  const int total_tiles = (s.totals[0] + s.totals[1]) * (n1 + n2);
+  const int U = tb.ms_u[E];
+  const int total_tiles = U * (n1 + n2);
   const uint32_t tiles_base = smem_addr(s.tiles);
+  volatile int* abort_flag = s.abort_flag;
 
   if (warp == 0) {
     // ---- TMA producer ----------------------------------------------------------------------------
@@ -410,7 +890,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int tile = atomicAdd(args.sched, 1);
         if (tile >= total_tiles) tile = -1;
         // hand the id to the MMA thread and the epilogue warps
-        if (!wait_phase(smem_addr(&s.q_empty[qi]), qph ^ 1u, abort_flag, args.status)) break;
+        if (!wait_bar(smem_addr(&s.q_empty[qi]), qph ^ 1u, ab)) break;
         s.tile_q[qi] = tile;
         mbar_arrive(smem_addr(&s.q_full[qi]));
         if (++qi == kTileQ) {
@@ -418,37 +898,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           qph ^= 1u;
         }
         if (tile < 0) break;
-        const FTile t = fdecode(s, E, n1, n2, tile);
-        const int row_a = s.off[t.e] + t.m_blk * BM;
-        // rows of this block: the A box shrinks to 16 / 32 / 64 rows when that covers them
-        const int bi = small_box_index(min(BM, s.off[t.e + 1] - row_a));
-        const uint32_t stage_tx = (bi < 3 ? small_box_rows(bi) * BK * 2 : kATileBytes) + kBTileBytes;
+        const FTile t = fdecode(tb, E, n1, n2, tile);
+        const int m_blk = t.unit;
+        const int row_a = tb.off[t.e] + m_blk * BM;
+        const int rows = min(BM, tb.off[t.e + 1] - row_a);
+        const int bi = small_box_index(rows);
+        const uint32_t stage_tx = a_box_bytes(rows) + kBTileBytes;
         int nkb;
-        const CUtensorMap *ma, *mb;
+        const CUtensorMap* ma;
         int row_b;
         if (t.phase == 1) {
           nkb = kb1;
           ma = bi < 3 ? &tm_xs.m[bi] : &tm_x;
-          mb = &tm_g;
           row_b = t.e * args.F + t.n_blk * 128;
         } else {
-          // the rows of h this tile reads are complete once all GEMM-1 tiles of (e, m) are
-          if (!wait_counter(args.done + t.mg, 4 * n1, abort_flag, args.status)) break;
-          asm volatile("fence.proxy.async.global;" ::: "memory");
-          // the last of the n2 GEMM-2 tiles of (e, m) to get here returns both counters to zero,
-          // so the workspace is ready for the next call without a memset
-          if (atomicAdd(args.used + t.mg, 1) == n2 - 1) {
-            atomicExch(args.done + t.mg, 0);
-            atomicExch(args.used + t.mg, 0);
-          }
+          if (!gemm2_acquire(args, tb, t.e, m_blk, n1, n2, ab)) break;
           nkb = kb2;
           ma = bi < 3 ? &tm_hs.m[bi] : &tm_h;
-          mb = &tm_d;
           row_b = t.e * args.H + t.n_blk * 256;
         }
         bool ok = true;
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!wait_phase(smem_addr(&s.empty[stage]), phase ^ 1u, abort_flag, args.status)) {
+          if (!wait_bar(smem_addr(&s.empty[stage]), phase ^ 1u, ab)) {
             ok = false;
             break;
           }
@@ -457,8 +928,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t fb = smem_addr(&s.full[stage]);
           mbar_arrive_expect_tx(fb, stage_tx);
           tma_load_2d(a_dst, ma, fb, kb * BK, row_a);
-          tma_load_2d(b_dst, mb, fb, kb * BK, row_b);
-          if (t.phase == 1) tma_load_2d(b_dst + kBTileBytes / 2, &tm_u, fb, kb * BK, row_b);
+          if (t.phase == 1) {
+            // gate rows -> B rows 0..127 (accumulator columns 0..127), up rows -> 128..255
+            tma_load_2d(b_dst, &tm_g, fb, kb * BK, row_b);
+            tma_load_2d(b_dst + kBHalfBytes, &tm_u, fb, kb * BK, row_b);
+          } else {
+            tma_load_2d(b_dst, &tm_d256, fb, kb * BK, row_b);
+          }
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == kStages) {
@@ -469,42 +945,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
       }
       if (*abort_flag) {
-        volatile int no_abort = 0;
         for (int st = 0; st < kStages; ++st)
-          if (issued_mask & (1u << st))
-            wait_phase(smem_addr(&s.full[st]), (issued_parity >> st) & 1u, &no_abort,
-                       args.status);
+          if (issued_mask & (1u << st)) drain_wait(smem_addr(&s.full[st]), (issued_parity >> st) & 1u);
       }
     }
   } else if (warp == 1) {
-    // ---- MMA issuer (M=128, N=256 for both phases) -------------------------------------------------
+    // ---- MMA issuer (M = 128, N = 256) ---------------------------------------------------------
     if (lane == 0) {
       const uint32_t idesc = make_idesc(BM, 256);
       int stage = 0;
       uint32_t phase = 0;
-      int it = 0;
       bool issued_any = false;
       int qi = 0;
       uint32_t qph = 0;
-      for (;; ++it) {
-        if (!wait_phase(smem_addr(&s.q_full[qi]), qph, abort_flag, args.status)) break;
-        const int tile = s.tile_q[qi];
-        mbar_arrive(smem_addr(&s.q_empty[qi]));
-        if (++qi == kTileQ) {
-          qi = 0;
-          qph ^= 1u;
-        }
+      for (int it = 0;; ++it) {
+        int tile;
+        if (!take_tile(s, qi, qph, false, ab, tile)) break;
         if (tile < 0) break;
-        const int nkb = tile < (s.totals[0] + s.totals[1]) * n1 ? kb1 : kb2;
+        const int nkb = tile < U * n1 ? kb1 : kb2;
         const int acc = it & 1;
         const uint32_t acc_parity = (it >> 1) & 1;
-        if (!wait_phase(smem_addr(&s.acc_empty[acc]), acc_parity ^ 1u, abort_flag, args.status))
-          break;
+        if (!wait_bar(smem_addr(&s.acc_empty[acc]), acc_parity ^ 1u, ab)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kAccCols;
         bool ok = true;
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!wait_phase(smem_addr(&s.full[stage]), phase, abort_flag, args.status)) {
+          if (!wait_bar(smem_addr(&s.full[stage]), phase, ab)) {
             ok = false;
             break;
           }
@@ -513,106 +979,41 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t b_addr = a_addr + kATileBytes;
 #pragma unroll
           for (int kk = 0; kk < BK / UMMA_K; ++kk)
-            tc_mma(d_tmem, sw128_desc(a_addr + kk * UMMA_K * 2),
-                   sw128_desc(b_addr + kk * UMMA_K * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
+            tc_mma1(d_tmem, sw128_desc(a_addr + kk * UMMA_K * 2),
+                    sw128_desc(b_addr + kk * UMMA_K * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
           issued_any = true;
-          tc_commit(smem_addr(&s.empty[stage]));
+          tc_commit1(smem_addr(&s.empty[stage]));
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit(smem_addr(&s.acc_full[acc]));
+        tc_commit1(smem_addr(&s.acc_full[acc]));
       }
       if (issued_any) {
-        tc_commit(smem_addr(s.drain));
-        volatile int no_abort = 0;
-        wait_phase(smem_addr(s.drain), 0, &no_abort, args.status);
+        tc_commit1(smem_addr(s.drain));
+        drain_wait(smem_addr(s.drain), 0);
       }
     }
   } else {
-    // ---- epilogue ----------------------------------------------------------------------------------
+    // ---- epilogue --------------------------------------------------------------------------------
     const int quarter = warp & 3;
     const int r_local = quarter * 32 + lane;
-    int it = 0;
     int qi = 0;
     uint32_t qph = 0;
-    for (;; ++it) {
-      int tile = -1;
-      bool okq = true;
-      if (lane == 0) {
-        okq = wait_phase(smem_addr(&s.q_full[qi]), qph, abort_flag, args.status);
-        if (okq) {
-          tile = s.tile_q[qi];
-          mbar_arrive(smem_addr(&s.q_empty[qi]));
-        }
-      }
-      if (++qi == kTileQ) {
-        qi = 0;
-        qph ^= 1u;
-      }
-      okq = __shfl_sync(0xFFFFFFFFu, okq ? 1 : 0, 0) != 0;
-      tile = __shfl_sync(0xFFFFFFFFu, tile, 0);
-      if (!okq || tile < 0) break;
-      const FTile t = fdecode(s, E, n1, n2, tile);
+    for (int it = 0;; ++it) {
+      int tile;
+      if (!warp_take_tile(s, qi, qph, false, ab, lane, tile) || tile < 0) break;
+      const FTile t = fdecode(tb, E, n1, n2, tile);
       const int acc = it & 1;
       const uint32_t acc_parity = (it >> 1) & 1;
       bool ok = true;
-      if (lane == 0) ok = wait_phase(smem_addr(&s.acc_full[acc]), acc_parity, abort_flag, args.status);
+      if (lane == 0) ok = wait_bar(smem_addr(&s.acc_full[acc]), acc_parity, ab);
       if (!__shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0)) break;
       tc_fence_after();
-      const int row = s.off[t.e] + t.m_blk * BM + r_local;
-      const bool row_ok = row < s.off[t.e + 1];
       const uint32_t t_row = tmem_base + acc * kAccCols + (static_cast<uint32_t>(quarter * 32) << 16);
-      if (t.phase == 1) {
-        __nv_bfloat16* out_row = args.h + static_cast<size_t>(row) * args.F;
-#pragma unroll 1
-        for (int c = 0; c < 128; c += 32) {
-          uint32_t g[32], u[32];
-          tmem_ld32(t_row + c, g);
-          tmem_ld32(t_row + 128 + c, u);
-          tmem_wait_ld();
-          const int col = t.n_blk * 128 + c;
-          if (row_ok && col < args.F) {
-            uint32_t packed[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float h0 = silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i]));
-              const float h1 = silu_mul(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1]));
-              packed[i] = pack_bf16x2(h0, h1);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(out_row + col);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
-          }
-        }
-        // publish: this warp's rows of h for (e, m, n) are written
-        asm volatile("fence.proxy.async.global;" ::: "memory");
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) red_release_add(args.done + t.mg, 1);
-      } else {
-        __nv_bfloat16* out_row = args.out + static_cast<size_t>(row) * args.H;
-#pragma unroll 1
-        for (int c = 0; c < 256; c += 32) {
-          uint32_t v[32];
-          tmem_ld32(t_row + c, v);
-          tmem_wait_ld();
-          const int col = t.n_blk * 256 + c;
-          if (row_ok && col < args.H) {
-            uint32_t packed[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              packed[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-            uint4* dst = reinterpret_cast<uint4*>(out_row + col);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
-          }
-        }
-      }
+      epilogue_tile(args, tb, t.phase, t.e, t.unit, t.n_blk, t_row, r_local, lane);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_addr(&s.acc_empty[acc]));
@@ -621,14 +1022,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (threadIdx.x == 0) {
-    // every claim of this CTA is done: the last CTA to get here returns the counters to zero
-    __threadfence();
-    if (atomicAdd(args.sched + 1, 1) == static_cast<int>(gridDim.x) - 1) {
-      atomicExch(args.sched, 0);
-      atomicExch(args.sched + 1, 0);
-    }
-  }
+  if (threadIdx.x == 0) release_schedule(args.sched);
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
@@ -702,9 +1096,39 @@ bool make_tmap(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t cols, u
 
 }  // namespace
 
+// Persistent grid of the pair kernel: as many 2-CTA clusters as can be resident at once (one CTA
+// per SM), looked up once per device and shared-memory size.
+static cudaError_t pair_grid(const cudaLaunchConfig_t& cfg_in, int* grid) {
+  struct Entry {
+    int dev;
+    size_t smem;
+    int grid;
+  };
+  static Entry cache[16];
+  static int n_cache = 0;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  for (int i = 0; i < n_cache; ++i)
+    if (cache[i].dev == dev && cache[i].smem == cfg_in.dynamicSmemBytes) {
+      *grid = cache[i].grid;
+      return cudaSuccess;
+    }
+  cudaLaunchConfig_t cfg = cfg_in;
+  cfg.gridDim = dim3(2 * (num_sms() / 2));
+  int clusters = 0;
+  err = cudaOccupancyMaxActiveClusters(&clusters, ffn_pair_kernel, &cfg);
+  if (err != cudaSuccess) return err;
+  if (clusters < 1) return cudaErrorInvalidConfiguration;
+  *grid = 2 * (clusters < num_sms() / 2 ? clusters : num_sms() / 2);
+  if (n_cache < 16) cache[n_cache++] = Entry{dev, cfg_in.dynamicSmemBytes, *grid};
+  return cudaSuccess;
+}
+
 // Workspace: [0,4) status | [256, ..) h bf16 [max_rows, F] | (FP8) dequantised rows bf16
 // [max_rows, H] | GEMM-1 completion counters and GEMM-2 arrival counters, int32
-// [2][max_rows/128 + E + 1] | tile-claim counter and finished-CTA counter, int32 [2].
+// [2][max_rows/128 + E + 1] | the claim and finished-CTA counters of the pair and of the single
+// kernel, int32 [4].
 static size_t round256(size_t b) { return (b + 255) / 256 * 256; }
 static size_t ffn_counter_count(int max_rows, int E) {
   return static_cast<size_t>(max_rows) / BM + static_cast<size_t>(E) + 1;
@@ -713,7 +1137,7 @@ static size_t ffn_counter_count(int max_rows, int E) {
 size_t ffn_workspace_bytes(int max_rows, int H, int F, int fp8, int E) {
   const size_t h_bytes = round256(static_cast<size_t>(max_rows) * F * 2);
   const size_t x_bytes = fp8 ? round256(static_cast<size_t>(max_rows) * H * 2) : 0;
-  return 256 + h_bytes + x_bytes + round256((2 * ffn_counter_count(max_rows, E) + 2) * sizeof(int));
+  return 256 + h_bytes + x_bytes + round256((2 * ffn_counter_count(max_rows, E) + 4) * sizeof(int));
 }
 
 cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp8,
@@ -732,24 +1156,22 @@ cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp
   }
   int* done = reinterpret_cast<int*>(base + off);
   int* used = done + ffn_counter_count(max_rows, E);
-  int* sched = used + ffn_counter_count(max_rows, E);
+  int* sched = used + ffn_counter_count(max_rows, E);  // [0..1] pair kernel, [2..3] single kernel
   // all counters are zero on entry (zero-filled workspace, reset by the previous call)
   cudaError_t err = cudaSuccess;
-  bool pdl_next = true;
   const void* a_src = send;
   if (fp8) {
     const long long work = static_cast<long long>(max_rows) * (H / 16);
     long long blocks = (work + 255) / 256;
     const long long cap = static_cast<long long>(num_sms()) * 8;
     if (blocks > cap) blocks = cap;
-    err = launch_pdl_if(pdl_next, dequant_fp8_kernel, dim3(static_cast<int>(blocks)), dim3(256), 0,
-                        s, static_cast<const uint8_t*>(send), send_scales, expert_offsets + E,
-                        max_rows, H, xdq);
+    err = launch_pdl(dequant_fp8_kernel, dim3(static_cast<int>(blocks)), dim3(256), 0, s,
+                     static_cast<const uint8_t*>(send), send_scales, expert_offsets + E, max_rows,
+                     H, xdq);
     if (err != cudaSuccess) return err;
     a_src = xdq;
-    pdl_next = true;
   }
-  CUtensorMap tm_x, tm_g, tm_u, tm_h, tm_d;
+  CUtensorMap tm_x, tm_g, tm_u, tm_h, tm_d128, tm_d256;
   SmallBoxMaps tm_xs, tm_hs;
   for (int i = 0; i < 3; ++i)
     if (!make_tmap(&tm_xs.m[i], a_src, max_rows, H, small_box_rows(i)) ||
@@ -759,17 +1181,52 @@ cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp
       !make_tmap(&tm_g, w_gate, static_cast<uint64_t>(E) * F, H, 128) ||
       !make_tmap(&tm_u, w_up, static_cast<uint64_t>(E) * F, H, 128) ||
       !make_tmap(&tm_h, h, max_rows, F, BM) ||
-      !make_tmap(&tm_d, w_down, static_cast<uint64_t>(E) * H, F, kGemm2NTile))
+      !make_tmap(&tm_d128, w_down, static_cast<uint64_t>(E) * H, F, 128) ||
+      !make_tmap(&tm_d256, w_down, static_cast<uint64_t>(E) * H, F, 256))
     return cudaErrorInvalidValue;
-  FfnArgs fa{expert_offsets, E, max_rows, H, F, h, static_cast<__nv_bfloat16*>(expert_out), status,
-             done, used, sched};
-  const size_t smem = fused_smem_bytes(E);
-  err = cudaFuncSetAttribute(fused_ffn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-  if (err != cudaSuccess) return err;
-  err = launch_pdl_if(pdl_next, fused_ffn_kernel, dim3(num_sms()), dim3(kThreads), smem, s, tm_x,
-                      tm_xs, tm_g, tm_u, tm_h, tm_hs, tm_d, fa);
-  if (err != cudaSuccess) return err;
+
+  // 1. experts with >= 2 row blocks: 2-CTA clusters
+  {
+    const FfnArgs fa{expert_offsets, E, max_rows, H, F, h, static_cast<__nv_bfloat16*>(expert_out),
+                     status, done, used, sched};
+    const size_t smem = ring_smem_bytes(E, kStagesPair, kATileBytes + kBHalfBytes);
+    err = cudaFuncSetAttribute(ffn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int grid = 0;
+    err = pair_grid(cfg, &grid);
+    if (err != cudaSuccess) return err;
+    cfg.gridDim = dim3(grid);
+    cfg.numAttrs = MOE_USE_PDL ? 2 : 1;
+    err = cudaLaunchKernelEx(&cfg, ffn_pair_kernel, tm_x, tm_xs, tm_g, tm_u, tm_h, tm_hs, tm_d128,
+                             fa);
+    if (err != cudaSuccess) return err;
+  }
+  // 2. experts with one row block: one CTA per tile
+  {
+    const FfnArgs fa{expert_offsets, E, max_rows, H, F, h, static_cast<__nv_bfloat16*>(expert_out),
+                     status, done, used, sched + 2};
+    const size_t smem = ring_smem_bytes(E, kStagesSingle, kATileBytes + 2 * kBHalfBytes);
+    err = cudaFuncSetAttribute(ffn_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    err = launch_pdl(ffn_single_kernel, dim3(num_sms()), dim3(kThreads), smem, s, tm_x, tm_xs, tm_g,
+                     tm_u, tm_h, tm_hs, tm_d256, fa);
+    if (err != cudaSuccess) return err;
+  }
   return cudaGetLastError();
 }
 

@@ -164,7 +164,7 @@ moe_status_t moe_dispatch_noalloc(const void* x, int T, int H, const int32_t* to
 
 /* Bytes of scratch moe_expert_ffn needs: a status word, the bf16 intermediate h [max_rows, F], for
  * the FP8 payload the dequantised bf16 input rows [max_rows, H], and the int32 counters of the
- * tile pipeline (two per 128-row block plus two for the run-time tile scheduler).  Caller-allocated
+ * tile pipeline (two per 128-row block plus two for each of the two run-time tile schedulers).  Caller-allocated
  * as for moe_dispatch_workspace_size (NCCL EP page, sections 1 and 3.1); `payload` is needed
  * because only the FP8 payload has the dequantised rows.  Returns 0 for invalid sizes. */
 size_t moe_ffn_workspace_size(int max_rows, int E, int H, int F, moe_payload_t payload);
@@ -177,7 +177,9 @@ size_t moe_ffn_workspace_size(int max_rows, int E, int H, int F, moe_payload_t p
  *     h = bf16( silu(x . W_gate[e]^T) * (x . W_up[e]^T) ),  silu(g) = g * sigmoid(g)
  *     expert_out = bf16( h . W_down[e]^T )
  * with bf16 operands on the tensor cores and fp32 accumulation.  For the FP8 payload the input
- * row is first dequantised: x = bf16(fp32(q) * scale).
+ * row is first dequantised: x = bf16(fp32(q) * scale).  Experts with two or more 128-row blocks
+ * run as 256-row tiles on pairs of SMs (2-CTA clusters), the others as 128-row tiles on one SM;
+ * every output element is computed by one tile in a fixed k order, so results are reproducible.
  *   send           [max_rows, H] bf16 or e4m3 (rows past expert_offsets[E] are ignored)
  *   send_scales    fp32 [max_rows, H/128] (FP8 only, else NULL)
  *   expert_offsets int32 [E+1] device array (read on the device; no host sync)

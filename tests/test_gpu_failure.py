@@ -9,7 +9,7 @@ import pytest
 import torch
 
 import moe_inputs as mi
-from _helpers import assert_close_bf16, bits16, combine_magnitude, np_
+from _helpers import assert_ffn_and_combine, bits16, np_
 from oracle import moe
 
 pytestmark = pytest.mark.gpu
@@ -49,5 +49,6 @@ def test_ffn_wait_timeout_is_reported_and_recoverable(cuda):
     assert torch.equal(m.y, y_ok)
     o = moe.pipeline(np_(d["logits"]), bits16(d["x"]), bits16(d["w_gate"]), bits16(d["w_up"]),
                      bits16(d["w_down"]), w.k, w.R)
-    assert_close_bf16(bits16(m.y), o["y"], "y",
-                      combine_magnitude(o["expert_out"], o["slot_row"], o["topk_w"]))
+    assert_ffn_and_combine(bits16(m.h)[:o["S"]], bits16(m.expert_out)[:o["S"]], bits16(m.y), o["h"],
+                           o["expert_out"], o["y"], o["expert_offsets"], d["w_down"],
+                           o["slot_row"], o["topk_w"], "after recovery")

@@ -1,8 +1,10 @@
 """GPU parity of the grouped SwiGLU FFN and of the whole path against the CPU oracle (C ABI).
 
 The FFN runs bf16 operands on the tensor cores with fp32 accumulation; the oracle accumulates in
-fp64.  Both round h and the output to bf16.  Parity bar per bf16 output tensor (assert_close_bf16):
-max |gpu - ref| / max |ref| <= 1e-2, and no element with |gpu - ref| > 1e-2 |ref| + 1e-3 max |ref|.
+fp64.  Both round h and the output to bf16.  Parity bar per bf16 output tensor: max |gpu - ref| /
+max |ref| <= 1e-2, and no element outside 1e-2 |ref| + 1e-3 max |ref|, plus for expert_out the
+row allowance of four one-ulp flips of h, and for y the expert_out allowance carried through the
+combine weights with the size of the summands as magnitude (assert_ffn_and_combine).
 Every workload is compared on every packed row and every token: the small ones through the whole
 path, the full-size ones in the benchmark's launch configuration."""
 import numpy as np
@@ -10,7 +12,7 @@ import pytest
 import torch
 
 import moe_inputs as mi
-from _helpers import assert_close_bf16, bits16, combine_magnitude, np_, to_dev_bf16_from_bits
+from _helpers import assert_ffn_and_combine, bits16, np_, to_dev_bf16_from_bits
 from oracle import moe
 
 pytestmark = pytest.mark.gpu
@@ -61,8 +63,8 @@ def test_ffn_parity_all_rows(cuda, name):
     h_ref, y_ref = moe.expert_ffn(xin, plan["expert_offsets"], bits16(d["w_gate"]),
                                   bits16(d["w_up"]), bits16(d["w_down"]))
     S = plan["S"]
-    assert_close_bf16(bits16(m.h)[:S], h_ref)
-    assert_close_bf16(bits16(m.expert_out)[:S], y_ref)
+    assert_ffn_and_combine(bits16(m.h)[:S], bits16(m.expert_out)[:S], None, h_ref, y_ref, None,
+                           plan["expert_offsets"], d["w_down"], None, None, name)
 
 
 def oracle_rows(w, d, xin, rows_by_expert):
@@ -109,16 +111,15 @@ def test_pipeline_full_size_every_row_and_token(cuda, name):
     y_ref = np.concatenate([ref[e][1] for e in sorted(ref)])
     del ref, xin
     assert h_ref.shape[0] == S
-    assert_close_bf16(bits16(m.h)[:S], h_ref, "h")
-    del h_ref
     eo = bits16(m.expert_out)[:S]
-    assert_close_bf16(eo, y_ref, "expert_out")
     y_bits = bits16(y)
     # the combine is exact given its inputs: every token
     assert np.array_equal(y_bits, moe.combine(eo, np_(m.slot_row), np_(m.topk_w), w.T, w.H))
-    # the whole path on every token, against the oracle's expert outputs and routing weights
-    assert_close_bf16(y_bits, moe.combine(y_ref, plan["slot_row"], wt, w.T, w.H), "y",
-                      combine_magnitude(y_ref, plan["slot_row"], wt))
+    # h and expert_out on every packed row, y on every token, against the oracle's expert outputs
+    # and routing weights
+    assert_ffn_and_combine(bits16(m.h)[:S], eo, y_bits, h_ref, y_ref,
+                           moe.combine(y_ref, plan["slot_row"], wt, w.T, w.H), off, d["w_down"],
+                           plan["slot_row"], wt, name)
 
 
 @pytest.mark.parametrize("name", ["finegrained", "skewed"])
@@ -153,9 +154,9 @@ def test_pipeline_end_to_end(cuda, name):
     assert np.array_equal(np_(m.topk_idx), o["topk_idx"])
     assert np.array_equal(np_(m.slot_row), o["slot_row"])
     assert np.array_equal(np_(m.expert_offsets), o["expert_offsets"])
-    assert_close_bf16(bits16(m.expert_out)[:o["S"]], o["expert_out"])
-    assert_close_bf16(bits16(y), o["y"], "y",
-                      combine_magnitude(o["expert_out"], o["slot_row"], o["topk_w"]))
+    assert_ffn_and_combine(bits16(m.h)[:o["S"]], bits16(m.expert_out)[:o["S"]], bits16(y), o["h"],
+                           o["expert_out"], o["y"], o["expert_offsets"], d["w_down"],
+                           o["slot_row"], o["topk_w"], name)
 
 
 def test_pipeline_decode_full_size_every_token(cuda):
@@ -172,10 +173,9 @@ def test_pipeline_decode_full_size_every_token(cuda):
     assert np.array_equal(np_(m.slot_row), o["slot_row"])
     assert np.array_equal(np_(m.expert_offsets), o["expert_offsets"])
     assert np.array_equal(bits16(m.send)[:o["S"]], o["send"])
-    assert_close_bf16(bits16(m.h)[:o["S"]], o["h"])
-    assert_close_bf16(bits16(m.expert_out)[:o["S"]], o["expert_out"])
-    assert_close_bf16(bits16(y), o["y"], "y",
-                      combine_magnitude(o["expert_out"], o["slot_row"], o["topk_w"]))
+    assert_ffn_and_combine(bits16(m.h)[:o["S"]], bits16(m.expert_out)[:o["S"]], bits16(y), o["h"],
+                           o["expert_out"], o["y"], o["expert_offsets"], d["w_down"],
+                           o["slot_row"], o["topk_w"], "decode")
     # the combine is exact given its inputs: the oracle's combine of the GPU's expert outputs
     assert np.array_equal(bits16(y), moe.combine(bits16(m.expert_out), np_(m.slot_row),
                                                  np_(m.topk_w), w.T, w.H))
@@ -193,9 +193,9 @@ def test_ffn_workspace_reused_across_calls_with_different_routing(cuda):
         o = moe.pipeline(np_(d["logits"]), bits16(d["x"]), bits16(d["w_gate"]), bits16(d["w_up"]),
                          bits16(d["w_down"]), w.k, w.R)
         assert np.array_equal(np_(m.expert_offsets), o["expert_offsets"])
-        assert_close_bf16(bits16(m.expert_out)[:o["S"]], o["expert_out"])
-        assert_close_bf16(bits16(y), o["y"], "y",
-                      combine_magnitude(o["expert_out"], o["slot_row"], o["topk_w"]))
+        assert_ffn_and_combine(bits16(m.h)[:o["S"]], bits16(m.expert_out)[:o["S"]], bits16(y),
+                               o["h"], o["expert_out"], o["y"], o["expert_offsets"], d["w_down"],
+                               o["slot_row"], o["topk_w"], f"seed {seed}")
 
 
 @pytest.mark.parametrize("rows", [
@@ -220,8 +220,8 @@ def test_ffn_two_block_experts(cuda, rows):
     assert m.status() == 0
     h_ref, y_ref = moe.expert_ffn(moe.ffn_inputs(bits16(x), None, False), off, bits16(wg),
                                   bits16(wu), bits16(wd))
-    assert_close_bf16(bits16(m.h)[:S], h_ref)
-    assert_close_bf16(bits16(m.expert_out)[:S], y_ref)
+    assert_ffn_and_combine(bits16(m.h)[:S], bits16(m.expert_out)[:S], None, h_ref, y_ref, None, off,
+                           wd, None, None, str(rows))
 
 
 @pytest.mark.parametrize("T,H,E,k,R,F,payload,cf", [
@@ -249,7 +249,6 @@ def test_pipeline_edge_shapes(cuda, T, H, E, k, R, F, payload, cf):
     if T == 0:
         assert y.numel() == 0
         return
-    if o["S"]:
-        assert_close_bf16(bits16(m.expert_out)[:o["S"]], o["expert_out"])
-    assert_close_bf16(bits16(y), o["y"], "y",
-                      combine_magnitude(o["expert_out"], o["slot_row"], o["topk_w"]))
+    assert_ffn_and_combine(bits16(m.h)[:o["S"]], bits16(m.expert_out)[:o["S"]], bits16(y), o["h"],
+                           o["expert_out"], o["y"], o["expert_offsets"], d["w_down"],
+                           o["slot_row"], o["topk_w"], "edge")

@@ -47,3 +47,25 @@ def test_combine_output_is_judged_against_the_size_of_its_summands():
     assert parity_report(got, ref)["n_bad"] == 1     # judged against |y| ~ 0.004 alone: fails
     rep = parity_report(got, ref, combine_magnitude(eo, sr, w))
     assert rep["n_bad"] == 0                          # against 0.5*1.5 + 0.5*1.49: passes
+
+
+def test_row_allowance_of_expert_out_covers_one_flipped_h_and_nothing_like_a_wrong_row():
+    import torch
+    from _helpers import ffn_row_atol
+    g = np.random.default_rng(4)
+    S, F, H = 6, 64, 32
+    h = g.normal(size=(S, F))
+    wd = g.normal(0, 0.05, size=(1, H, F))
+    hb = bf16_bits(h)
+    eo_ref = bf16_bits(bf16_values(hb) @ bf16_values(bf16_bits(wd[0])).T)
+    atol = ffn_row_atol(hb, np.array([0, S]), torch.from_numpy(bf16_values(bf16_bits(wd))))
+    # the largest h of row 2 rounded one ulp the other way
+    h2 = hb.copy()
+    f = int(np.argmax(np.abs(bf16_values(hb[2]))))
+    h2[2, f] += 1
+    eo_flip = bf16_bits(bf16_values(h2) @ bf16_values(bf16_bits(wd[0])).T)
+    assert parity_report(eo_flip, eo_ref, row_atol=atol)["n_bad"] == 0
+    # another row's output in row 2: far outside
+    eo_bad = eo_ref.copy()
+    eo_bad[2] = eo_ref[3]
+    assert parity_report(eo_bad, eo_ref, row_atol=atol)["n_bad"] > H // 2
