@@ -11,7 +11,7 @@
 // and then all their GEMM-2 tiles (a GEMM-2 tile waits on per-row-block completion counters of
 // the GEMM-1 tiles), with tiles claimed at run time from a global counter:
 //
-// * ffn_pair_kernel: experts with two or more 128-row blocks.  A 2-CTA cluster computes a tile of
+// * ffn_pair_kernel: experts with more than 64 rows.  A 2-CTA cluster computes a tile of
 //   (expert, pair of row blocks, column block) as one 256 x 256 product with
 //   tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16): CTA v holds its row block of A and rows
 //   [128v, 128v + 128) of the 256 weight rows of B, so each SM stages half of the weight tile per
@@ -19,9 +19,9 @@
 //   columns.  GEMM-1 puts the gate rows in CTA 0's half of B and the up rows in CTA 1's.  CTA 1's
 //   TMA loads complete their bytes on CTA 0's barriers, CTA 0's single MMA thread issues for both
 //   and its commits arrive on both CTAs' barriers (multicast commit, not multicast loads).
-// * ffn_single_kernel: experts with one row block (mostly a handful of rows, so a tile is bound
-//   by streaming the expert's weights, not by the MMA).  One CTA per tile: tcgen05.mma.cta_group::1
-//   (M = 128, N = 256), 48 KB stages (the A box shrinks to the rows present), four in flight.
+// * ffn_single_kernel: experts with at most 64 rows (a tile is bound by streaming the expert's
+//   weights, not by the MMA).  One CTA per tile: tcgen05.mma.cta_group::1 (M = 128, N = 256),
+//   40 KB stages (an A box of 16, 32 or 64 rows + the whole weight tile), five in flight.
 //
 // Roles (192 threads): warp 0 = TMA producer (CTA 0 of a pair also claims tiles and passes the ids
 // to both CTAs through shared-memory queues); warp 1 = TMEM allocation and the MMA thread;
@@ -51,11 +51,13 @@ constexpr int kTmemCols = 512;   // two accumulators
 constexpr int kThreads = 192;
 constexpr int kATileBytes = BM * BK * 2;   // 16 KB: 128 rows of A
 constexpr int kBHalfBytes = 128 * BK * 2;  // 16 KB: 128 weight rows
-// Experts with at least this many row blocks run in the pair kernel, the others in the single one.
-constexpr int kPairMinBlocks = 2;
-// Pair kernel: six 32-KB stages (A rows + half of B); single kernel: four 48-KB stages (A + B).
+// Experts with at most this many rows run in the single-block kernel, the others in the pair kernel.
+constexpr int kSingleMaxRows = 64;
+// Pair kernel: six 32-KB stages (A rows + half of B).  Single kernel: five 40-KB stages (an A box of
+// at most 64 rows + all 256 rows of B).
 constexpr int kStagesPair = 6;
-constexpr int kStagesSingle = 4;
+constexpr int kStagesSingle = 5;
+constexpr int kASingleBytes = kSingleMaxRows * BK * 2;  // 8 KB
 constexpr int kTileQ = 4;
 // Consumers of a pair kernel's queue slot, all arriving on CTA 0's q_empty: CTA 0's MMA thread and
 // four epilogue warps, CTA 1's producer and four epilogue warps.
@@ -322,8 +324,9 @@ struct Tables {
   int* units;   // [E]   units of this kernel's class per expert (0 for the other class)
   int* ms_rb;   // [E+1] first global row block of each expert (over all experts)
   int* ms_u;    // [E+1] first unit of each expert among this kernel's units
+  int* stats;   // [2]   experts of the single-block kernel, pairs of row blocks of the others
 };
-__host__ __device__ constexpr int table_ints(int E) { return 5 * E + 3; }
+__host__ __device__ constexpr int table_ints(int E) { return 5 * E + 5; }
 
 __device__ __forceinline__ Tables carve_tables(int* p, int E) {
   Tables t;
@@ -332,25 +335,30 @@ __device__ __forceinline__ Tables carve_tables(int* p, int E) {
   t.units = t.mt + E;
   t.ms_rb = t.units + E;
   t.ms_u = t.ms_rb + (E + 1);
+  t.stats = t.ms_u + (E + 1);
   return t;
 }
 
 // One warp builds the tables from expert_offsets (warp scans).  PAIRS: the units are pairs of row
-// blocks of the experts with >= kPairMinBlocks blocks; otherwise the row blocks of the others.
+// blocks of the experts with more than kSingleMaxRows rows; otherwise the single row block of each
+// of the others.
 template <bool PAIRS>
 __device__ __forceinline__ void build_tables(const Tables& tb, const FfnArgs& args, int lane) {
   const int E = args.E;
-  int carry_r = 0, carry_u = 0;
+  int carry_r = 0, carry_u = 0, n_single = 0, n_pairs = 0;
   for (int e0 = 0; e0 < E; e0 += 32) {
     const int e = e0 + lane;
     int lo = 0, hi = 0;
     if (e < E) {
-      lo = min(__ldg(args.expert_offsets + e), args.max_rows);
-      hi = min(__ldg(args.expert_offsets + e + 1), args.max_rows);
+      // L2 loads: the pair kernel may start before the kernel ahead of it has finished
+      lo = min(__ldcg(args.expert_offsets + e), args.max_rows);
+      hi = min(__ldcg(args.expert_offsets + e + 1), args.max_rows);
     }
     const int mt = (max(hi - lo, 0) + BM - 1) / BM;
-    const bool paired = mt >= kPairMinBlocks;
+    const bool paired = hi - lo > kSingleMaxRows;
     const int u = PAIRS ? (paired ? (mt + 1) / 2 : 0) : (paired ? 0 : mt);
+    n_single += __popc(__ballot_sync(0xFFFFFFFFu, !paired && mt == 1));
+    n_pairs += paired ? (mt + 1) / 2 : 0;
     int ir = mt, iu = u;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -371,11 +379,37 @@ __device__ __forceinline__ void build_tables(const Tables& tb, const FfnArgs& ar
     carry_r += __shfl_sync(0xFFFFFFFFu, ir, 31);
     carry_u += __shfl_sync(0xFFFFFFFFu, iu, 31);
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) n_pairs += __shfl_xor_sync(0xFFFFFFFFu, n_pairs, o);
   if (lane == 0) {
     tb.ms_rb[E] = carry_r;
     tb.ms_u[E] = carry_u;
-    tb.off[E] = min(__ldg(args.expert_offsets + E), args.max_rows);
+    tb.off[E] = min(__ldcg(args.expert_offsets + E), args.max_rows);
+    tb.stats[0] = n_single;
+    tb.stats[1] = n_pairs;
   }
+}
+
+// CTAs of the single-block kernel that work while the pair kernel runs beside it on the other
+// SMs: the grid's share of the two kinds of work, each at a per-SM rate.  A single-block expert
+// streams its 3 H F bf16 weights (85 GB/s per SM) and a pair of row blocks does 6 * 256 * H * F
+// flops (9 TFLOP/s per SM on the 2-CTA tiles), so the ratio does not depend on H and F.  The scale
+// factor 1.5 was the best of 1.0 / 1.5 / 2.0 / 2.5 / 3.0 on B200 for a routing with 100 single-block
+// experts beside 29 larger ones (FFN 3.61-3.64 ms against 3.69-3.77 at 1.0; the two kinds slow each
+// other down when they run together).  Rounded to whole clusters of two, at least one cluster
+// when there is such work.
+#ifndef MOE_SINGLE_SHARE_SCALE
+#define MOE_SINGLE_SHARE_SCALE 1.5f
+#endif
+__device__ __forceinline__ int single_kernel_ctas(const Tables& tb, int grid) {
+  const int n_single = tb.stats[0], n_pairs = tb.stats[1];
+  if (n_single == 0) return 0;
+  if (n_pairs == 0) return grid;
+  const float t_single = static_cast<float>(n_single) * 6.0f / 85e9f;
+  const float t_pairs = static_cast<float>(n_pairs) * 1536.0f / 9e12f;
+  const float share = MOE_SINGLE_SHARE_SCALE * t_single / (t_single + t_pairs);
+  int g = 2 * static_cast<int>(0.5f * share * static_cast<float>(grid) + 0.5f);
+  return max(2, min(grid, g));
 }
 
 struct FTile {
@@ -592,7 +626,7 @@ __device__ __forceinline__ void release_schedule(int* sched) {
 }
 
 // ================================================================================================
-// Pair kernel: experts with >= kPairMinBlocks row blocks; 2-CTA clusters, cta_group::2.
+// Pair kernel: experts with more than kSingleMaxRows rows; 2-CTA clusters, cta_group::2.
 // ================================================================================================
 __global__ void __launch_bounds__(kThreads, 1)
     ffn_pair_kernel(const __grid_constant__ CUtensorMap tm_x,
@@ -628,10 +662,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   } else if (warp == 2) {
-    griddep_wait();
     build_tables<true>(tb, args, lane);
   }
-  griddep_wait();
+  // No wait for the single-block kernel launched ahead: its experts are disjoint from these, and
+  // this grid can only start once every CTA of that kernel has passed its own wait for the
+  // dispatch, so the packed rows and offsets are complete (they are read through L2).  The wait at
+  // the end makes this grid's completion imply that kernel's too.
   griddep_launch_dependents();
   tc_fence_before();
   __syncthreads();
@@ -826,6 +862,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                  "r"(kTmemCols)
                  : "memory");
   }
+  griddep_wait();  // the single-block kernel ahead has completed too
 }
 
 // ================================================================================================
@@ -841,7 +878,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tm_d256, const FfnArgs args) {
   constexpr int kStages = kStagesSingle;
   constexpr int kBTileBytes = 2 * kBHalfBytes;  // all 256 weight rows
-  constexpr int kStageBytes = kATileBytes + kBTileBytes;
+  constexpr int kStageBytes = kASingleBytes + kBTileBytes;
+  // The MMA reads 128 A rows: rows 64..127 come from the B tile behind the A box and feed only
+  // accumulator rows that are never stored (the expert has at most 64 rows).
   extern __shared__ uint8_t smem_raw[];
   const int E = args.E;
   const Ring s = carve(smem_raw, E, kStages, kStageBytes);
@@ -868,6 +907,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     build_tables<false>(tb, args, lane);
   }
   griddep_wait();
+  // the pair kernel launched behind this one may start as soon as every CTA gets here
   griddep_launch_dependents();
   tc_fence_before();
   __syncthreads();
@@ -877,8 +917,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int total_tiles = U * (n1 + n2);
   const uint32_t tiles_base = smem_addr(s.tiles);
   volatile int* abort_flag = s.abort_flag;
+  // This grid is launched as 2-CTA clusters, one CTA per SM; only the first single_kernel_ctas()
+  // CTAs work, the others leave at once so that the pair kernel gets their SMs (whole pairs).
+  const bool working = static_cast<int>(blockIdx.x) < single_kernel_ctas(tb, gridDim.x);
 
-  if (warp == 0) {
+  if (!working) {
+    // nothing to do: fall through to the common exit
+  } else if (warp == 0) {
     // ---- TMA producer ----------------------------------------------------------------------------
     if (lane == 0) {
       int stage = 0;
@@ -901,20 +946,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const FTile t = fdecode(tb, E, n1, n2, tile);
         const int m_blk = t.unit;
         const int row_a = tb.off[t.e] + m_blk * BM;
-        const int rows = min(BM, tb.off[t.e + 1] - row_a);
-        const int bi = small_box_index(rows);
+        const int rows = min(kSingleMaxRows, tb.off[t.e + 1] - row_a);
+        const int bi = small_box_index(rows);  // 16, 32 or 64 rows
         const uint32_t stage_tx = a_box_bytes(rows) + kBTileBytes;
         int nkb;
         const CUtensorMap* ma;
         int row_b;
         if (t.phase == 1) {
           nkb = kb1;
-          ma = bi < 3 ? &tm_xs.m[bi] : &tm_x;
+          ma = &tm_xs.m[bi];
           row_b = t.e * args.F + t.n_blk * 128;
         } else {
           if (!gemm2_acquire(args, tb, t.e, m_blk, n1, n2, ab)) break;
           nkb = kb2;
-          ma = bi < 3 ? &tm_hs.m[bi] : &tm_h;
+          ma = &tm_hs.m[bi];
           row_b = t.e * args.H + t.n_blk * 256;
         }
         bool ok = true;
@@ -924,7 +969,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           const uint32_t a_dst = tiles_base + stage * kStageBytes;
-          const uint32_t b_dst = a_dst + kATileBytes;
+          const uint32_t b_dst = a_dst + kASingleBytes;
           const uint32_t fb = smem_addr(&s.full[stage]);
           mbar_arrive_expect_tx(fb, stage_tx);
           tma_load_2d(a_dst, ma, fb, kb * BK, row_a);
@@ -976,7 +1021,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t a_addr = tiles_base + stage * kStageBytes;
-          const uint32_t b_addr = a_addr + kATileBytes;
+          const uint32_t b_addr = a_addr + kASingleBytes;
 #pragma unroll
           for (int kk = 0; kk < BK / UMMA_K; ++kk)
             tc_mma1(d_tmem, sw128_desc(a_addr + kk * UMMA_K * 2),
@@ -1096,11 +1141,14 @@ bool make_tmap(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t cols, u
 
 }  // namespace
 
-// Persistent grid of the pair kernel: as many 2-CTA clusters as can be resident at once (one CTA
-// per SM), looked up once per device and shared-memory size.
-static cudaError_t pair_grid(const cudaLaunchConfig_t& cfg_in, int* grid) {
+// Persistent grid of 2-CTA clusters of `kernel`: as many clusters as can be resident at once (one
+// CTA per SM), looked up once per device, kernel and shared-memory size.
+using FfnKernel = void (*)(CUtensorMap, SmallBoxMaps, CUtensorMap, CUtensorMap, CUtensorMap,
+                           SmallBoxMaps, CUtensorMap, FfnArgs);
+static cudaError_t cluster_grid(FfnKernel kernel, const cudaLaunchConfig_t& cfg_in, int* grid) {
   struct Entry {
     int dev;
+    FfnKernel kernel;
     size_t smem;
     int grid;
   };
@@ -1110,18 +1158,19 @@ static cudaError_t pair_grid(const cudaLaunchConfig_t& cfg_in, int* grid) {
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   for (int i = 0; i < n_cache; ++i)
-    if (cache[i].dev == dev && cache[i].smem == cfg_in.dynamicSmemBytes) {
+    if (cache[i].dev == dev && cache[i].kernel == kernel &&
+        cache[i].smem == cfg_in.dynamicSmemBytes) {
       *grid = cache[i].grid;
       return cudaSuccess;
     }
   cudaLaunchConfig_t cfg = cfg_in;
   cfg.gridDim = dim3(2 * (num_sms() / 2));
   int clusters = 0;
-  err = cudaOccupancyMaxActiveClusters(&clusters, ffn_pair_kernel, &cfg);
+  err = cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg);
   if (err != cudaSuccess) return err;
   if (clusters < 1) return cudaErrorInvalidConfiguration;
   *grid = 2 * (clusters < num_sms() / 2 ? clusters : num_sms() / 2);
-  if (n_cache < 16) cache[n_cache++] = Entry{dev, cfg_in.dynamicSmemBytes, *grid};
+  if (n_cache < 16) cache[n_cache++] = Entry{dev, kernel, cfg_in.dynamicSmemBytes, *grid};
   return cudaSuccess;
 }
 
@@ -1185,48 +1234,51 @@ cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp
       !make_tmap(&tm_d256, w_down, static_cast<uint64_t>(E) * H, F, 256))
     return cudaErrorInvalidValue;
 
-  // 1. experts with >= 2 row blocks: 2-CTA clusters
-  {
-    const FfnArgs fa{expert_offsets, E, max_rows, H, F, h, static_cast<__nv_bfloat16*>(expert_out),
-                     status, done, used, sched};
-    const size_t smem = ring_smem_bytes(E, kStagesPair, kATileBytes + kBHalfBytes);
-    err = cudaFuncSetAttribute(ffn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem));
-    if (err != cudaSuccess) return err;
-    cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int grid = 0;
-    err = pair_grid(cfg, &grid);
-    if (err != cudaSuccess) return err;
-    cfg.gridDim = dim3(grid);
-    cfg.numAttrs = MOE_USE_PDL ? 2 : 1;
-    err = cudaLaunchKernelEx(&cfg, ffn_pair_kernel, tm_x, tm_xs, tm_g, tm_u, tm_h, tm_hs, tm_d128,
-                             fa);
-    if (err != cudaSuccess) return err;
-  }
-  // 2. experts with one row block: one CTA per tile
-  {
-    const FfnArgs fa{expert_offsets, E, max_rows, H, F, h, static_cast<__nv_bfloat16*>(expert_out),
-                     status, done, used, sched + 2};
-    const size_t smem = ring_smem_bytes(E, kStagesSingle, kATileBytes + 2 * kBHalfBytes);
-    err = cudaFuncSetAttribute(ffn_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem));
-    if (err != cudaSuccess) return err;
-    err = launch_pdl(ffn_single_kernel, dim3(num_sms()), dim3(kThreads), smem, s, tm_x, tm_xs, tm_g,
-                     tm_u, tm_h, tm_hs, tm_d256, fa);
-    if (err != cudaSuccess) return err;
-  }
+  // Both kernels are persistent grids of 2-CTA clusters, one CTA per SM.  The single-block kernel
+  // goes first: its CTAs beyond its share of the work leave at once, and the pair kernel, launched
+  // programmatically behind it, starts on those SMs without waiting for it (it waits at its end).
+  const FfnArgs fa_single{expert_offsets, E, max_rows, H, F, h,
+                          static_cast<__nv_bfloat16*>(expert_out), status, done, used, sched + 2};
+  const FfnArgs fa_pair{expert_offsets, E, max_rows, H, F, h,
+                        static_cast<__nv_bfloat16*>(expert_out), status, done, used, sched};
+  const size_t smem_single = ring_smem_bytes(E, kStagesSingle, kASingleBytes + 2 * kBHalfBytes);
+  const size_t smem_pair = ring_smem_bytes(E, kStagesPair, kATileBytes + kBHalfBytes);
+  err = cudaFuncSetAttribute(ffn_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem_single));
+  if (err != cudaSuccess) return err;
+  err = cudaFuncSetAttribute(ffn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem_pair));
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  int grid_single = 0, grid_pair = 0;
+  cfg.numAttrs = 1;
+  cfg.dynamicSmemBytes = smem_single;
+  err = cluster_grid(ffn_single_kernel, cfg, &grid_single);
+  if (err != cudaSuccess) return err;
+  cfg.dynamicSmemBytes = smem_pair;
+  err = cluster_grid(ffn_pair_kernel, cfg, &grid_pair);
+  if (err != cudaSuccess) return err;
+  cfg.numAttrs = MOE_USE_PDL ? 2 : 1;
+  cfg.gridDim = dim3(grid_single);
+  cfg.dynamicSmemBytes = smem_single;
+  err = cudaLaunchKernelEx(&cfg, ffn_single_kernel, tm_x, tm_xs, tm_g, tm_u, tm_h, tm_hs, tm_d256,
+                           fa_single);
+  if (err != cudaSuccess) return err;
+  cfg.gridDim = dim3(grid_pair);
+  cfg.dynamicSmemBytes = smem_pair;
+  err = cudaLaunchKernelEx(&cfg, ffn_pair_kernel, tm_x, tm_xs, tm_g, tm_u, tm_h, tm_hs, tm_d128,
+                           fa_pair);
+  if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 
