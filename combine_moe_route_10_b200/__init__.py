@@ -10,11 +10,13 @@ from ._lib import (EXPORTS, LIB_PATH, MOE_ERR_CUDA, MOE_ERR_INVALID_ARG, MOE_ERR
                    MOE_PAYLOAD_BF16, MOE_PAYLOAD_FP8_E4M3_B128, MoeError, load, moe_abi_version,
                    moe_capacity, moe_combine, moe_dispatch, moe_dispatch_noalloc,
                    moe_dispatch_workspace_size,
-                   moe_expert_ffn, moe_ffn_workspace_size, moe_route, moe_sync_status,
+                   moe_expert_ffn, moe_expert_ffn_list, moe_ffn_weight_list_bytes,
+                   moe_ffn_weight_list_init, moe_ffn_workspace_size, moe_route, moe_sync_status,
                    status_string)
 from .layer import MoeShuffle
 
 __all__ = ["MoeShuffle", "MoeError", "load", "moe_route", "moe_dispatch", "moe_expert_ffn",
+           "moe_expert_ffn_list", "moe_ffn_weight_list_bytes", "moe_ffn_weight_list_init",
            "moe_combine", "moe_sync_status", "moe_dispatch_noalloc", "moe_capacity", "moe_dispatch_workspace_size",
            "moe_ffn_workspace_size", "moe_abi_version", "status_string", "EXPORTS", "LIB_PATH",
            "MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_INVALID_TOPK", "MOE_ERR_UNSUPPORTED",

@@ -24,7 +24,8 @@ MOE_PAYLOAD_FP8_E4M3_B128 = 1
 EXPORTS = ["moe_abi_version", "moe_status_string", "moe_capacity", "moe_route",
            "moe_dispatch_workspace_size", "moe_dispatch", "moe_dispatch_noalloc",
            "moe_ffn_workspace_size",
-           "moe_expert_ffn", "moe_combine", "moe_sync_status"]
+           "moe_expert_ffn", "moe_ffn_weight_list_bytes", "moe_ffn_weight_list_init",
+           "moe_expert_ffn_list", "moe_combine", "moe_sync_status"]
 
 _lib = None
 
@@ -55,6 +56,9 @@ def load() -> ctypes.CDLL:
         "moe_dispatch_noalloc": (I, [P, I, I, P, I, I, I, I, I, P, P, P, P, P, P, P, P, P]),
         "moe_ffn_workspace_size": (Z, [I, I, I, I, I]),
         "moe_expert_ffn": (I, [P, P, I, P, I, I, I, I, P, P, P, P, P, Z, P]),
+        "moe_ffn_weight_list_bytes": (Z, [I]),
+        "moe_ffn_weight_list_init": (I, [P, P, P, I, I, I, P, P]),
+        "moe_expert_ffn_list": (I, [P, P, I, P, I, I, I, I, P, P, P, Z, P]),
         "moe_combine": (I, [P, I, P, P, I, I, I, P, P, P]),
         "moe_sync_status": (I, [P, P]),
     }
@@ -143,6 +147,33 @@ def moe_expert_ffn(send, send_scales, payload, expert_offsets, max_rows, E, H, F
                                max_rows, E, H, F, _ptr(w_gate), _ptr(w_up), _ptr(w_down),
                                _ptr(expert_out), _ptr(ws), ws_bytes, _stream(stream))
     return _check(st, "moe_expert_ffn", raise_on_error)
+
+
+def moe_ffn_weight_list_bytes(E) -> int:
+    return load().moe_ffn_weight_list_bytes(E)
+
+
+def moe_ffn_weight_list_init(w_gate, w_up, w_down, E, H, F, wlist, stream=None,
+                             raise_on_error=True):
+    """Per-expert weight descriptors into the device buffer ``wlist``: w_gate / w_up / w_down are
+    sequences of E per-expert tensors ([F,H], [F,H], [H,F] bf16, each its own allocation)."""
+    arr = ctypes.c_void_p * E
+    g = arr(*[_ptr(t) for t in w_gate])
+    u = arr(*[_ptr(t) for t in w_up])
+    d = arr(*[_ptr(t) for t in w_down])
+    st = load().moe_ffn_weight_list_init(ctypes.cast(g, ctypes.c_void_p),
+                                         ctypes.cast(u, ctypes.c_void_p),
+                                         ctypes.cast(d, ctypes.c_void_p), E, H, F, _ptr(wlist),
+                                         _stream(stream))
+    return _check(st, "moe_ffn_weight_list_init", raise_on_error)
+
+
+def moe_expert_ffn_list(send, send_scales, payload, expert_offsets, max_rows, E, H, F, wlist,
+                        expert_out, ws, ws_bytes, stream=None, raise_on_error=True):
+    st = load().moe_expert_ffn_list(_ptr(send), _ptr(send_scales), payload, _ptr(expert_offsets),
+                                    max_rows, E, H, F, _ptr(wlist), _ptr(expert_out), _ptr(ws),
+                                    ws_bytes, _stream(stream))
+    return _check(st, "moe_expert_ffn_list", raise_on_error)
 
 
 def moe_combine(expert_out, max_rows, slot_row, topk_w, T, k, H, y, status=None, stream=None,

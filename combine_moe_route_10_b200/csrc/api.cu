@@ -140,7 +140,51 @@ moe_status_t moe_expert_ffn(const void* send, const float* send_scales, moe_payl
   if (!aligned(ws, 256) || ws_bytes < moe::ffn_workspace_bytes(max_rows, H, F, fp8 ? 1 : 0, E))
     return MOE_ERR_WORKSPACE;
   return from_cuda(moe::launch_expert_ffn(send, send_scales, fp8 ? 1 : 0, expert_offsets, max_rows,
-                                          E, H, F, w_gate, w_up, w_down, expert_out, ws,
+                                          E, H, F, w_gate, w_up, w_down, nullptr, expert_out, ws,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_ffn_weight_list_bytes(int E) {
+  if (E < 1 || E > kMaxE) return 0;
+  return moe::ffn_weight_list_bytes(E);
+}
+
+moe_status_t moe_ffn_weight_list_init(const void* const* w_gate, const void* const* w_up,
+                                      const void* const* w_down, int E, int H, int F, void* list,
+                                      moe_stream_t stream) {
+  if (E < 1 || E > kMaxE || H < 1 || F < 1) return MOE_ERR_INVALID_ARG;
+  if (H % 64 != 0 || F % 64 != 0) return MOE_ERR_UNSUPPORTED;
+  if (w_gate == nullptr || w_up == nullptr || w_down == nullptr || list == nullptr ||
+      !aligned(list, 64))
+    return MOE_ERR_INVALID_ARG;
+  for (int e = 0; e < E; ++e)
+    if (w_gate[e] == nullptr || w_up[e] == nullptr || w_down[e] == nullptr ||
+        !aligned(w_gate[e], 16) || !aligned(w_up[e], 16) || !aligned(w_down[e], 16))
+      return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::ffn_weight_list_init(w_gate, w_up, w_down, E, H, F, list,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_expert_ffn_list(const void* send, const float* send_scales, moe_payload_t payload,
+                                 const int32_t* expert_offsets, int max_rows, int E, int H, int F,
+                                 const void* list, void* expert_out, void* ws, size_t ws_bytes,
+                                 moe_stream_t stream) {
+  if (max_rows < 0 || E < 1 || E > kMaxE || H < 1 || F < 1) return MOE_ERR_INVALID_ARG;
+  if (payload != MOE_PAYLOAD_BF16 && payload != MOE_PAYLOAD_FP8_E4M3_B128)
+    return MOE_ERR_INVALID_ARG;
+  const bool fp8 = payload == MOE_PAYLOAD_FP8_E4M3_B128;
+  if (H % 64 != 0 || F % 64 != 0 || (fp8 && H % 128 != 0)) return MOE_ERR_UNSUPPORTED;
+  if (expert_offsets == nullptr || list == nullptr || ws == nullptr || !aligned(list, 64))
+    return MOE_ERR_INVALID_ARG;
+  if (max_rows > 0 && (send == nullptr || expert_out == nullptr || (fp8 && send_scales == nullptr)))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(send, 16) || !aligned(expert_out, 16) || !aligned(expert_offsets, 4) ||
+      !aligned(send_scales, 4))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(ws, 256) || ws_bytes < moe::ffn_workspace_bytes(max_rows, H, F, fp8 ? 1 : 0, E))
+    return MOE_ERR_WORKSPACE;
+  return from_cuda(moe::launch_expert_ffn(send, send_scales, fp8 ? 1 : 0, expert_offsets, max_rows,
+                                          E, H, F, nullptr, nullptr, nullptr, list, expert_out, ws,
                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 

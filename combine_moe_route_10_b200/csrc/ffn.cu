@@ -37,6 +37,10 @@
 #include <cudaTypedefs.h>
 #include <cuda_fp8.h>
 
+#include <string.h>
+
+#include <vector>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -316,7 +320,29 @@ struct FfnArgs {
   int* done;                      // [row blocks] GEMM-1 completion counters, zero on entry
   int* used;                      // [row blocks] GEMM-2 tiles that passed the wait, zero on entry
   int* sched;                     // [2] this kernel's next tile to claim, CTAs that finished
+  // Per-expert weight descriptors (moe_ffn_weight_list_init): 4 per expert (gate, up, down with
+  // 128-row and 256-row boxes), rows local to the expert; nullptr: the grid-constant maps of the
+  // contiguous [E, ...] weights, rows global.
+  const CUtensorMap* wlist;
 };
+
+// The descriptor of the weight tile a tile loads, and its first row.  `which`: 0 gate, 1 up,
+// 2 down (128-row box), 3 down (256-row box); `local_row` is the row inside expert e's matrix.
+__device__ __forceinline__ const CUtensorMap* weight_map(const FfnArgs& args, const CUtensorMap* tm,
+                                                         int e, int which, int local_row,
+                                                         int rows_per_expert, int& row) {
+  if (args.wlist == nullptr) {
+    row = e * rows_per_expert + local_row;
+    return tm;
+  }
+  const CUtensorMap* m = args.wlist + 4 * e + which;
+  // the descriptors were written to global memory by a copy before this launch
+  asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(
+                   reinterpret_cast<uint64_t>(m))
+               : "memory");
+  row = local_row;
+  return m;
+}
 
 struct Tables {
   int* off;     // [E+1] row offsets (clamped to max_rows)
@@ -602,12 +628,13 @@ __device__ __forceinline__ bool warp_take_tile(const Ring& s, int& qi, uint32_t&
   return okq;
 }
 
+// Prefetch of the descriptors in kernel parameter space (the weight maps only when they are used).
 __device__ __forceinline__ void prefetch_maps(const CUtensorMap* a, const CUtensorMap* b,
                                               const CUtensorMap* c, const CUtensorMap* d,
                                               const CUtensorMap* e, const SmallBoxMaps& xs,
-                                              const SmallBoxMaps& hs) {
-  const CUtensorMap* all[5] = {a, b, c, d, e};
-  for (int i = 0; i < 5; ++i)
+                                              const SmallBoxMaps& hs, bool weights) {
+  const CUtensorMap* all[5] = {a, d, b, c, e};  // x, h, then the three weight maps
+  for (int i = 0; i < (weights ? 5 : 2); ++i)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(all[i])) : "memory");
   for (int i = 0; i < 3; ++i) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xs.m[i])) : "memory");
@@ -652,7 +679,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       init_ring(s, kStages, 8, kPairQueueConsumers);  // acc_empty: four epilogue warps per CTA
-      prefetch_maps(&tm_x, &tm_g, &tm_u, &tm_h, &tm_d128, tm_xs, tm_hs);
+      prefetch_maps(&tm_x, &tm_g, &tm_u, &tm_h, &tm_d128, tm_xs, tm_hs, args.wlist == nullptr);
     }
   } else if (warp == 1) {
     // the same warp of both CTAs allocates, as cta_group::2 requires
@@ -723,14 +750,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (t.phase == 1) {
           nkb = kb1;
           ma = bi < 3 ? &tm_xs.m[bi] : &tm_x;
-          mb = rank == 0 ? &tm_g : &tm_u;  // gate rows -> accumulator columns 0..127, up -> 128..
-          row_b = t.e * args.F + t.n_blk * 128;
+          // gate rows -> accumulator columns 0..127, up rows -> 128..255
+          mb = weight_map(args, rank == 0 ? &tm_g : &tm_u, t.e, static_cast<int>(rank),
+                          t.n_blk * 128, args.F, row_b);
         } else {
           if (rows > 0 && !gemm2_acquire(args, tb, t.e, m_blk, n1, n2, ab)) break;
           nkb = kb2;
           ma = bi < 3 ? &tm_hs.m[bi] : &tm_h;
-          mb = &tm_d128;
-          row_b = t.e * args.H + t.n_blk * 256 + static_cast<int>(rank) * 128;
+          mb = weight_map(args, &tm_d128, t.e, 2, t.n_blk * 256 + static_cast<int>(rank) * 128,
+                          args.H, row_b);
         }
         bool ok = true;
         for (int kb = 0; kb < nkb; ++kb) {
@@ -894,7 +922,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       init_ring(s, kStages, 4, kSingleQueueConsumers);
-      prefetch_maps(&tm_x, &tm_g, &tm_u, &tm_h, &tm_d256, tm_xs, tm_hs);
+      prefetch_maps(&tm_x, &tm_g, &tm_u, &tm_h, &tm_d256, tm_xs, tm_hs, args.wlist == nullptr);
     }
   } else if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -950,17 +978,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int bi = small_box_index(rows);  // 16, 32 or 64 rows
         const uint32_t stage_tx = a_box_bytes(rows) + kBTileBytes;
         int nkb;
-        const CUtensorMap* ma;
+        const CUtensorMap *ma, *mb0, *mb1 = nullptr;
         int row_b;
         if (t.phase == 1) {
           nkb = kb1;
           ma = &tm_xs.m[bi];
-          row_b = t.e * args.F + t.n_blk * 128;
+          mb0 = weight_map(args, &tm_g, t.e, 0, t.n_blk * 128, args.F, row_b);
+          mb1 = weight_map(args, &tm_u, t.e, 1, t.n_blk * 128, args.F, row_b);
         } else {
           if (!gemm2_acquire(args, tb, t.e, m_blk, n1, n2, ab)) break;
           nkb = kb2;
           ma = &tm_hs.m[bi];
-          row_b = t.e * args.H + t.n_blk * 256;
+          mb0 = weight_map(args, &tm_d256, t.e, 3, t.n_blk * 256, args.H, row_b);
         }
         bool ok = true;
         for (int kb = 0; kb < nkb; ++kb) {
@@ -975,10 +1004,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(a_dst, ma, fb, kb * BK, row_a);
           if (t.phase == 1) {
             // gate rows -> B rows 0..127 (accumulator columns 0..127), up rows -> 128..255
-            tma_load_2d(b_dst, &tm_g, fb, kb * BK, row_b);
-            tma_load_2d(b_dst + kBHalfBytes, &tm_u, fb, kb * BK, row_b);
+            tma_load_2d(b_dst, mb0, fb, kb * BK, row_b);
+            tma_load_2d(b_dst + kBHalfBytes, mb1, fb, kb * BK, row_b);
           } else {
-            tma_load_2d(b_dst, &tm_d256, fb, kb * BK, row_b);
+            tma_load_2d(b_dst, mb0, fb, kb * BK, row_b);
           }
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -1189,10 +1218,26 @@ size_t ffn_workspace_bytes(int max_rows, int H, int F, int fp8, int E) {
   return 256 + h_bytes + x_bytes + round256((2 * ffn_counter_count(max_rows, E) + 4) * sizeof(int));
 }
 
+size_t ffn_weight_list_bytes(int E) { return static_cast<size_t>(E) * 4 * sizeof(CUtensorMap); }
+
+cudaError_t ffn_weight_list_init(const void* const* w_gate, const void* const* w_up,
+                                 const void* const* w_down, int E, int H, int F, void* list,
+                                 cudaStream_t s) {
+  std::vector<CUtensorMap> maps(static_cast<size_t>(E) * 4);
+  for (int e = 0; e < E; ++e) {
+    CUtensorMap* m = maps.data() + 4 * static_cast<size_t>(e);
+    if (!make_tmap(m + 0, w_gate[e], F, H, 128) || !make_tmap(m + 1, w_up[e], F, H, 128) ||
+        !make_tmap(m + 2, w_down[e], H, F, 128) || !make_tmap(m + 3, w_down[e], H, F, 256))
+      return cudaErrorInvalidValue;
+  }
+  // from pageable memory: the call returns once the host array has been taken
+  return cudaMemcpyAsync(list, maps.data(), ffn_weight_list_bytes(E), cudaMemcpyHostToDevice, s);
+}
+
 cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp8,
                               const int32_t* expert_offsets, int max_rows, int E, int H, int F,
                               const void* w_gate, const void* w_up, const void* w_down,
-                              void* expert_out, void* ws, cudaStream_t s) {
+                              const void* wlist, void* expert_out, void* ws, cudaStream_t s) {
   if (max_rows == 0) return cudaSuccess;
   char* base = static_cast<char*>(ws);
   int* status = reinterpret_cast<int*>(base);
@@ -1226,21 +1271,30 @@ cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp
     if (!make_tmap(&tm_xs.m[i], a_src, max_rows, H, small_box_rows(i)) ||
         !make_tmap(&tm_hs.m[i], h, max_rows, F, small_box_rows(i)))
       return cudaErrorInvalidValue;
-  if (!make_tmap(&tm_x, a_src, max_rows, H, BM) ||
-      !make_tmap(&tm_g, w_gate, static_cast<uint64_t>(E) * F, H, 128) ||
-      !make_tmap(&tm_u, w_up, static_cast<uint64_t>(E) * F, H, 128) ||
-      !make_tmap(&tm_h, h, max_rows, F, BM) ||
-      !make_tmap(&tm_d128, w_down, static_cast<uint64_t>(E) * H, F, 128) ||
-      !make_tmap(&tm_d256, w_down, static_cast<uint64_t>(E) * H, F, 256))
+  if (!make_tmap(&tm_x, a_src, max_rows, H, BM) || !make_tmap(&tm_h, h, max_rows, F, BM))
     return cudaErrorInvalidValue;
+  if (wlist != nullptr) {
+    // the kernels take each expert's descriptors from the list; these are never read
+    memset(&tm_g, 0, sizeof(CUtensorMap));
+    memset(&tm_u, 0, sizeof(CUtensorMap));
+    memset(&tm_d128, 0, sizeof(CUtensorMap));
+    memset(&tm_d256, 0, sizeof(CUtensorMap));
+  } else if (!make_tmap(&tm_g, w_gate, static_cast<uint64_t>(E) * F, H, 128) ||
+             !make_tmap(&tm_u, w_up, static_cast<uint64_t>(E) * F, H, 128) ||
+             !make_tmap(&tm_d128, w_down, static_cast<uint64_t>(E) * H, F, 128) ||
+             !make_tmap(&tm_d256, w_down, static_cast<uint64_t>(E) * H, F, 256)) {
+    return cudaErrorInvalidValue;
+  }
+  const CUtensorMap* wl = static_cast<const CUtensorMap*>(wlist);
 
   // Both kernels are persistent grids of 2-CTA clusters, one CTA per SM.  The single-block kernel
   // goes first: its CTAs beyond its share of the work leave at once, and the pair kernel, launched
   // programmatically behind it, starts on those SMs without waiting for it (it waits at its end).
   const FfnArgs fa_single{expert_offsets, E, max_rows, H, F, h,
-                          static_cast<__nv_bfloat16*>(expert_out), status, done, used, sched + 2};
+                          static_cast<__nv_bfloat16*>(expert_out), status, done, used, sched + 2,
+                          wl};
   const FfnArgs fa_pair{expert_offsets, E, max_rows, H, F, h,
-                        static_cast<__nv_bfloat16*>(expert_out), status, done, used, sched};
+                        static_cast<__nv_bfloat16*>(expert_out), status, done, used, sched, wl};
   const size_t smem_single = ring_smem_bytes(E, kStagesSingle, kASingleBytes + 2 * kBHalfBytes);
   const size_t smem_pair = ring_smem_bytes(E, kStagesPair, kATileBytes + kBHalfBytes);
   err = cudaFuncSetAttribute(ffn_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -71,9 +71,17 @@ cudaError_t launch_combine(const void* expert_out, int max_rows, const int32_t* 
 // dequantised rows [max_rows, H] bf16, then the GEMM-1 completion counters.
 size_t ffn_workspace_bytes(int max_rows, int H, int F, int fp8, int E);
 
+// wlist == nullptr: the weights are contiguous [E, F, H] / [E, H, F] arrays; otherwise the
+// per-expert descriptors written by ffn_weight_list_init (and w_gate / w_up / w_down are unused).
 cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp8,
                               const int32_t* expert_offsets, int max_rows, int E, int H, int F,
                               const void* w_gate, const void* w_up, const void* w_down,
-                              void* expert_out, void* ws, cudaStream_t s);
+                              const void* wlist, void* expert_out, void* ws, cudaStream_t s);
+
+// Per-expert weight descriptors: four 128-byte TMA descriptors per expert.
+size_t ffn_weight_list_bytes(int E);
+cudaError_t ffn_weight_list_init(const void* const* w_gate, const void* const* w_up,
+                                 const void* const* w_down, int E, int H, int F, void* list,
+                                 cudaStream_t s);
 
 }  // namespace moe

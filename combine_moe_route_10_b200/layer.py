@@ -116,6 +116,37 @@ class MoeShuffle:
                             self.max_rows, self.E, self.H, self.F, w_gate, w_up, w_down,
                             self.expert_out, self.ws_ffn, self.ws_ffn_bytes, stream)
 
+    def expert_weight_list(self, w_gate, w_up, w_down) -> torch.Tensor:
+        """Device descriptors of per-expert weights at separate addresses (sequences of E tensors
+        [F,H], [F,H], [H,F] bf16); the weights must stay where they are while the list is used."""
+        for e in range(self.E):
+            expect(w_gate[e], (self.F, self.H), torch.bfloat16, f"w_gate[{e}]", self.device)
+            expect(w_up[e], (self.F, self.H), torch.bfloat16, f"w_up[{e}]", self.device)
+            expect(w_down[e], (self.H, self.F), torch.bfloat16, f"w_down[{e}]", self.device)
+        n = _lib.moe_ffn_weight_list_bytes(self.E)
+        wlist = torch.empty(n, dtype=torch.uint8, device=self.device)
+        _lib.moe_ffn_weight_list_init(list(w_gate), list(w_up), list(w_down), self.E, self.H,
+                                      self.F, wlist)
+        torch.cuda.synchronize(self.device)
+        return wlist
+
+    def expert_ffn_list(self, wlist, send=None, send_scales=None, expert_offsets=None, stream=None):
+        """expert_ffn with the weights of ``expert_weight_list``."""
+        expect(wlist, (_lib.moe_ffn_weight_list_bytes(self.E),), torch.uint8, "wlist", self.device)
+        if send is not None:
+            expect(send, (self.max_rows, self.H), self.send.dtype, "send", self.device)
+        if send_scales is not None:
+            expect(send_scales, (self.max_rows, self.H // 128), torch.float32, "send_scales",
+                   self.device)
+        if expert_offsets is not None:
+            expect(expert_offsets, (self.E + 1,), torch.int32, "expert_offsets", self.device)
+        _lib.moe_expert_ffn_list(self.send if send is None else send,
+                                 self.send_scales if send_scales is None else send_scales,
+                                 self.payload,
+                                 self.expert_offsets if expert_offsets is None else expert_offsets,
+                                 self.max_rows, self.E, self.H, self.F, wlist, self.expert_out,
+                                 self.ws_ffn, self.ws_ffn_bytes, stream)
+
     def combine(self, expert_out=None, slot_row=None, topk_w=None, stream=None):
         if expert_out is not None:
             expect(expert_out, (self.max_rows, self.H), torch.bfloat16, "expert_out", self.device)

@@ -199,6 +199,36 @@ moe_status_t moe_expert_ffn(const void* send, const float* send_scales, moe_payl
                             void* expert_out, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * Per-expert weight lists: experts whose weights live at separate addresses (each its own
+ * allocation, e.g. local experts next to experts prefetched from elsewhere), consumed by the grouped
+ * FFN without first copying them into one [E, ...] block ("DWDP: 在NVL72上的高性能分布式权重数据
+ * 并行", sections 消除D2D时延开销 and 关键优化实施: the grouped GEMM takes a TensorList and picks
+ * each expert's buffer inside the kernel, instead of merging split weights device to device).
+ *
+ * moe_ffn_weight_list_bytes: bytes of the device buffer moe_ffn_weight_list_init fills (four
+ * 128-byte TMA descriptors per expert); 0 for E outside [1, 1024].
+ *
+ * moe_ffn_weight_list_init: set-up call, once per set of weight addresses.
+ *   w_gate, w_up   HOST arrays of E device pointers, each bf16 [F, H] (16-byte aligned)
+ *   w_down         HOST array of E device pointers, each bf16 [H, F]
+ *   list           device buffer >= moe_ffn_weight_list_bytes(E), 64-byte aligned (caller-owned)
+ * Enqueues a host-to-device copy on `stream` from pageable memory (the call returns once the host
+ * data has been taken; it is not meant for stream capture).  The weights must stay at these
+ * addresses while the list is used.  Limits: H % 64 == 0, F % 64 == 0, E <= 1024.
+ *
+ * moe_expert_ffn_list: moe_expert_ffn with the weights given by a list instead of three [E, ...]
+ * arrays; same arguments otherwise, and the same results bit for bit (same tiles, same k order).
+ */
+size_t moe_ffn_weight_list_bytes(int E);
+moe_status_t moe_ffn_weight_list_init(const void* const* w_gate, const void* const* w_up,
+                                      const void* const* w_down, int E, int H, int F, void* list,
+                                      moe_stream_t stream);
+moe_status_t moe_expert_ffn_list(const void* send, const float* send_scales, moe_payload_t payload,
+                                 const int32_t* expert_offsets, int max_rows, int E, int H, int F,
+                                 const void* list, void* expert_out, void* ws, size_t ws_bytes,
+                                 moe_stream_t stream);
+
+/*
  * Combine: y[t] = bf16( sum_{j=0..k-1, slot_row[t,j] >= 0} topk_w[t,j] * expert_out[slot_row[t,j]] )
  * accumulated in fp32 in slot order j = 0, 1, ... with each product and sum rounded to fp32
  * separately (the NCCL EP page, section 2.1: the combine loops over the top-k slots and adds each

@@ -155,3 +155,30 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "libmoe.so"))
     with pytest.raises(ImportError):
         _lib.load()
+
+
+def test_weight_list_calls_reject_bad_arguments(lib):
+    """The per-expert weight-list entry points validate on the host before touching the GPU."""
+    import ctypes
+    assert pkg.moe_ffn_weight_list_bytes(8) == 8 * 4 * 128        # four descriptors per expert
+    assert pkg.moe_ffn_weight_list_bytes(0) == 0
+    assert pkg.moe_ffn_weight_list_bytes(1025) == 0
+    ptrs = (ctypes.c_void_p * 2)(FAKE, FAKE)
+    p = ctypes.cast(ptrs, ctypes.c_void_p)
+    init = lambda **kw: lib.moe_ffn_weight_list_init(
+        kw.get("g", p), p, p, kw.get("E", 2), kw.get("H", 256), kw.get("F", 512),
+        kw.get("list", FAKE), None)
+    assert init(g=None) == pkg.MOE_ERR_INVALID_ARG
+    assert init(H=200) == pkg.MOE_ERR_UNSUPPORTED
+    assert init(list=FAKE + 32) == pkg.MOE_ERR_INVALID_ARG          # not 64-byte aligned
+    assert init(E=0) == pkg.MOE_ERR_INVALID_ARG
+    bad = ctypes.cast((ctypes.c_void_p * 2)(FAKE, FAKE + 8), ctypes.c_void_p)
+    assert init(g=bad) == pkg.MOE_ERR_INVALID_ARG                    # a misaligned expert
+    ffn = lambda **kw: lib.moe_expert_ffn_list(
+        FAKE, None, kw.get("payload", 0), FAKE, 64, 8, kw.get("H", 256), 512,
+        kw.get("list", FAKE), FAKE, FAKE, kw.get("ws_bytes", 1 << 30), None)
+    assert ffn(list=None) == pkg.MOE_ERR_INVALID_ARG
+    assert ffn(list=FAKE + 16) == pkg.MOE_ERR_INVALID_ARG
+    assert ffn(H=200) == pkg.MOE_ERR_UNSUPPORTED
+    assert ffn(payload=1) == pkg.MOE_ERR_INVALID_ARG                 # FP8 without scales
+    assert ffn(ws_bytes=100) == pkg.MOE_ERR_WORKSPACE
