@@ -45,7 +45,7 @@ import numpy as np
 from .numerics import bf16_bits, bf16_from_bits, bf16_round, e4m3_decode, e4m3_encode_satfinite
 
 __all__ = ["capacity", "route", "dispatch_plan", "dispatch_payload", "expert_ffn", "combine",
-           "pipeline", "QBLOCK"]
+           "pipeline", "QBLOCK", "quantize_rows_fp8", "dequantize_rows_fp8", "expert_ffn_w8"]
 
 QBLOCK = 128   # elements per FP8 scale block
 E4M3_MAX_F32 = np.float32(448.0)
@@ -231,6 +231,58 @@ def expert_ffn(send_rows_f64: np.ndarray, expert_offsets, w_gate_bits, w_up_bits
         g = x @ wg.T
         u = x @ wu.T
         del wg, wu
+        h = bf16_round(g / (1.0 + np.exp(-g)) * u)
+        wd = bf16_from_bits(w_down_bits[e]).astype(np.float64)
+        y = h @ wd.T
+        h_out[r] = bf16_bits(h)
+        y_out[r] = bf16_bits(y)
+    return h_out, y_out
+
+
+def quantize_rows_fp8(values):
+    """Rows -> (e4m3 codes, one fp32 scale per row): scale = amax / 448 of the row's fp32 values
+    (1 when amax = 0), code = e4m3 round-to-nearest-even, saturating, of the fp32 quotient
+    value / scale.  The per-block quantiser of the FP8 payload, with the whole row as the block
+    (used for FP8 expert weights, one scale per output row, and for the FFN's own FP8 input rows).
+
+    ``values``: float array [rows, K] whose entries are fp32 values (e.g. bf16 values)."""
+    x = np.asarray(values, dtype=np.float32)
+    amax = np.max(np.abs(x), axis=1) if x.shape[1] else np.zeros(x.shape[0], dtype=np.float32)
+    scale = np.where(amax == 0, np.float32(1.0), amax / np.float32(E4M3_MAX_F32)).astype(np.float32)
+    q = (x / scale[:, None]).astype(np.float32)            # fp32 IEEE division
+    return e4m3_encode_satfinite(q), scale
+
+
+def dequantize_rows_fp8(codes, scales) -> np.ndarray:
+    """Exact values (float64) of e4m3 codes times their row's fp32 scale."""
+    return e4m3_decode(codes) * np.asarray(scales, dtype=np.float64)[..., None]
+
+
+def expert_ffn_w8(send_rows_f64: np.ndarray, expert_offsets, wg_codes, wg_scales, wu_codes,
+                  wu_scales, w_down_bits, rows=None):
+    """Grouped SwiGLU FFN with FP8 gate / up weights (W8A8 first projection).
+
+    Per packed row x (its FFN input values, as for ``expert_ffn``): the row is quantised on its own,
+    (qx, sx) = quantize_rows_fp8(x); the gate and up weights are e4m3 codes with one fp32 scale per
+    output row.  For expert e: g = sx * sg[f] * sum_h qx[h] qg[f, h] (exact values, fp64), the same
+    for u; h = bf16(g * sigmoid(g) * u); y = bf16(h W_down[e]^T) with bf16 down weights (fp64
+    accumulate).  Returns (h, y) as bf16 bit patterns like ``expert_ffn``."""
+    off = np.asarray(expert_offsets, dtype=np.int64)
+    E = off.size - 1
+    S = int(off[E])
+    F, H = wg_codes.shape[1], wg_codes.shape[2]
+    want = np.arange(S) if rows is None else np.asarray(rows, dtype=np.int64)
+    h_out = np.full((S, F), 0x7FC0, dtype=np.uint16)
+    y_out = np.full((S, H), 0x7FC0, dtype=np.uint16)
+    for e in range(E):
+        lo, hi = off[e], off[e + 1]
+        r = want[(want >= lo) & (want < hi)]
+        if r.size == 0:
+            continue
+        qx, sx = quantize_rows_fp8(np.asarray(send_rows_f64[r], dtype=np.float64))
+        xq = dequantize_rows_fp8(qx, sx)
+        g = xq @ dequantize_rows_fp8(wg_codes[e], wg_scales[e]).T
+        u = xq @ dequantize_rows_fp8(wu_codes[e], wu_scales[e]).T
         h = bf16_round(g / (1.0 + np.exp(-g)) * u)
         wd = bf16_from_bits(w_down_bits[e]).astype(np.float64)
         y = h @ wd.T
