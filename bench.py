@@ -262,6 +262,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--flush", default="write-read", choices=["write", "write-read"])
+    ap.add_argument("--no-w8", action="store_true",
+                    help="skip the extra timing of the step with FP8 gate / up weights")
     ap.add_argument("--e2e-eager", action="store_true",
                     help="end-to-end loop calls forward eagerly instead of replaying CUDA graphs")
     args = ap.parse_args()
@@ -312,6 +314,7 @@ def main():
         "e2e": head["e2e"],
         "gpu_launches": head["gpu_launches"],
         "clocks": clocks,
+        "fp8_weights": head.get("fp8_weights"),
         "workloads": {n: {k: v for k, v in r.items() if k != "e2e"} for n, r in extra.items()},
         "workloads_note": "the other large workloads, each timed the same way in the same run "
                           "(own warm-up, L2 flush, metric and breakdown steps); gpu_launches counts "
@@ -425,7 +428,8 @@ def measure(w, args, dev, world: int, rank: int, e2e: bool) -> dict:
         roof = {"bound": "tensor", "achieved": ach, "peak": p, "unit": "TFLOP/s", "frac": ach / p,
                 "frac_burst": ach / pk["bf16_tflops"], "frac_nominal": ach / NOMINAL["bf16_tflops"]}
     roof.update({
-        "kernel": ("fused_ffn_kernel (one persistent launch: GEMM-1 gate|up + SwiGLU, GEMM-2 down)"
+        "kernel": ("ffn_pair_kernel (2-CTA tiles, experts of > 64 rows) + ffn_single_kernel "
+                   "(experts of <= 64 rows): GEMM-1 gate|up + SwiGLU and GEMM-2 down in each"
                    + (" + dequant_fp8_kernel" if w.payload == "fp8" else "") + " = moe_expert_ffn"),
         "traffic": FFN_TRAFFIC.get(w.name), "peak_source": pk_src,
         "algorithmic_bytes": alg["ffn_bytes"], "algorithmic_flops": alg["ffn_flops"],
@@ -446,14 +450,85 @@ def measure(w, args, dev, world: int, rank: int, e2e: bool) -> dict:
                 "GB/s": gbs(alg["ffn_bytes"], t_ffn)},
         "combine": shuffle_stage(alg["combine"], t_comb),
     }
-    launches_per_step = 5 + (1 if w.payload == "fp8" else 0)   # route, count, rank_permute, FFN, combine
+    # route, count + rank_permute (dispatch), the two FFN kernels (+ the FP8 dequantisation), combine
+    launches_per_step = 6 + (1 if w.payload == "fp8" else 0)
     out = {"value": agg["value"], "ms_per_step": agg["ms_per_step"], "config": config_of(w, args),
            "roofline": roof, "stages": stages, "kept_rows": S, "active_experts": active,
            "gpu_launches": 2 * launches_per_step * args.steps,  # metric + breakdown steps
            "e2e": e2e_out}
+    if not args.no_w8:
+        out["fp8_weights"] = measure_w8(w, m, d, args, stream, flush_l2, world, dev, S, active, pk)
     del m, d, flush, flush_rd
     torch.cuda.empty_cache()
     return out
+
+
+def measure_w8(w, m, d, args, stream, flush_l2, world, dev, S, active, pk) -> dict:
+    """The same step with FP8 gate / up weights (W8A8 first projection, bf16 down projection): the
+    weights are quantised once beforehand, outside the timed region; each step quantises its FFN
+    input rows inside the FFN call.  K metric steps interleaved with K steps that time the FFN."""
+    import torch.distributed as dist
+    gq, gs, uq, us = m.quantize_expert_weights_fp8(d["w_gate"], d["w_up"])
+
+    def step():
+        m.route(d["logits"])
+        m.dispatch(d["x"])
+        m.expert_ffn_w8(gq, gs, uq, us, d["w_down"])
+        m.combine()
+
+    for _ in range(args.warmup):
+        flush_l2()
+        step()
+    torch.cuda.synchronize()
+    if m.status() != 0:
+        raise SystemExit(f"{w.name}: device status after the FP8-weight warm-up")
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        e = ev[i]
+        flush_l2()
+        e[0].record(stream)
+        step()
+        e[1].record(stream)
+        flush_l2()
+        m.route(d["logits"])
+        m.dispatch(d["x"])
+        e[2].record(stream)
+        m.expert_ffn_w8(gq, gs, uq, us, d["w_down"])
+        e[3].record(stream)
+        m.combine()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    if m.status() != 0:
+        raise SystemExit(f"{w.name}: device status after the FP8-weight steps")
+    agg = aggregate(sum(e[0].elapsed_time(e[1]) for e in ev), w.T, args.steps, dev)
+    t_ffn = sum(e[2].elapsed_time(e[3]) for e in ev) / args.steps
+    fp8 = w.payload == "fp8"
+    wbytes = active * (2 * w.H * w.F + w.H * w.F * 2 + 2 * w.F * 4)   # e4m3 gate/up + scales, bf16 down
+    rows = S * w.H * (1 if fp8 else 2) + (S * (w.H // 128) * 4 if fp8 else 0) + S * w.H * 2
+    ffn_bytes = wbytes + rows
+    flops8, flops16 = 4 * S * w.H * w.F, 2 * S * w.H * w.F
+    hbm = pk["hbm_gbs"]
+    p16 = pk["bf16_tflops_sustained"]
+    p8 = 2.0 * p16          # dense e4m3 = 2 x dense bf16 (nominal ratio 4.5 / 2.25 PFLOP/s)
+    t_bytes = ffn_bytes / (hbm * 1e9)
+    t_flops = flops8 / (p8 * 1e12) + flops16 / (p16 * 1e12)
+    bound = max(t_bytes, t_flops)
+    return {"value": agg["value"], "ms_per_step": agg["ms_per_step"], "ffn_ms": t_ffn,
+            "ffn_GB/s": ffn_bytes / (t_ffn * 1e-3) / 1e9,
+            "ffn_TFLOP/s": (flops8 + flops16) / (t_ffn * 1e-3) / 1e12,
+            "roofline": {"bound": "hbm" if t_bytes >= t_flops else "tensor",
+                         "frac_of_max_time_bound": bound / (t_ffn * 1e-3),
+                         "algorithmic_bytes": ffn_bytes, "flops_e4m3": flops8,
+                         "flops_bf16": flops16, "peak_hbm_gbs": hbm,
+                         "peak_e4m3_tflops": p8, "peak_bf16_tflops": p16,
+                         "peak_note": "e4m3 peak = 2 x the measured sustained bf16 figure"},
+            "gpu_launches": 2 * (7 + (1 if fp8 else 0)) * args.steps,
+            "note": "gate / up weights e4m3 with one fp32 scale per row (quantised before timing), "
+                    "FFN input rows quantised per row inside the step, down projection bf16"}
 
 
 def e2e_run(w, m, d, args, dev, world: int, stream) -> dict:

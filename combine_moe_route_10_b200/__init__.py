@@ -11,12 +11,14 @@ from ._lib import (EXPORTS, LIB_PATH, MOE_ERR_CUDA, MOE_ERR_INVALID_ARG, MOE_ERR
                    moe_capacity, moe_combine, moe_dispatch, moe_dispatch_noalloc,
                    moe_dispatch_workspace_size,
                    moe_expert_ffn, moe_expert_ffn_list, moe_ffn_weight_list_bytes,
-                   moe_ffn_weight_list_init, moe_ffn_workspace_size, moe_route, moe_sync_status,
+                   moe_ffn_weight_list_init, moe_ffn_workspace_size, moe_expert_ffn_w8,
+                   moe_ffn_w8_workspace_size, moe_quantize_rows_fp8, moe_route, moe_sync_status,
                    status_string)
 from .layer import MoeShuffle
 
 __all__ = ["MoeShuffle", "MoeError", "load", "moe_route", "moe_dispatch", "moe_expert_ffn",
            "moe_expert_ffn_list", "moe_ffn_weight_list_bytes", "moe_ffn_weight_list_init",
+           "moe_expert_ffn_w8", "moe_ffn_w8_workspace_size", "moe_quantize_rows_fp8",
            "moe_combine", "moe_sync_status", "moe_dispatch_noalloc", "moe_capacity", "moe_dispatch_workspace_size",
            "moe_ffn_workspace_size", "moe_abi_version", "status_string", "EXPORTS", "LIB_PATH",
            "MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_INVALID_TOPK", "MOE_ERR_UNSUPPORTED",

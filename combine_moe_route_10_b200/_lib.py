@@ -25,7 +25,8 @@ EXPORTS = ["moe_abi_version", "moe_status_string", "moe_capacity", "moe_route",
            "moe_dispatch_workspace_size", "moe_dispatch", "moe_dispatch_noalloc",
            "moe_ffn_workspace_size",
            "moe_expert_ffn", "moe_ffn_weight_list_bytes", "moe_ffn_weight_list_init",
-           "moe_expert_ffn_list", "moe_combine", "moe_sync_status"]
+           "moe_expert_ffn_list", "moe_quantize_rows_fp8", "moe_ffn_w8_workspace_size",
+           "moe_expert_ffn_w8", "moe_combine", "moe_sync_status"]
 
 _lib = None
 
@@ -59,6 +60,9 @@ def load() -> ctypes.CDLL:
         "moe_ffn_weight_list_bytes": (Z, [I]),
         "moe_ffn_weight_list_init": (I, [P, P, P, I, I, I, P, P]),
         "moe_expert_ffn_list": (I, [P, P, I, P, I, I, I, I, P, P, P, Z, P]),
+        "moe_quantize_rows_fp8": (I, [P, I, I, P, P, P]),
+        "moe_ffn_w8_workspace_size": (Z, [I, I, I, I, I]),
+        "moe_expert_ffn_w8": (I, [P, P, I, P, I, I, I, I, P, P, P, P, P, P, P, Z, P]),
         "moe_combine": (I, [P, I, P, P, I, I, I, P, P, P]),
         "moe_sync_status": (I, [P, P]),
     }
@@ -174,6 +178,25 @@ def moe_expert_ffn_list(send, send_scales, payload, expert_offsets, max_rows, E,
                                     max_rows, E, H, F, _ptr(wlist), _ptr(expert_out), _ptr(ws),
                                     ws_bytes, _stream(stream))
     return _check(st, "moe_expert_ffn_list", raise_on_error)
+
+
+def moe_quantize_rows_fp8(x, rows, K, codes, scales, stream=None, raise_on_error=True):
+    st = load().moe_quantize_rows_fp8(_ptr(x), rows, K, _ptr(codes), _ptr(scales), _stream(stream))
+    return _check(st, "moe_quantize_rows_fp8", raise_on_error)
+
+
+def moe_ffn_w8_workspace_size(max_rows, E, H, F, payload) -> int:
+    return load().moe_ffn_w8_workspace_size(max_rows, E, H, F, payload)
+
+
+def moe_expert_ffn_w8(send, send_scales, payload, expert_offsets, max_rows, E, H, F, w_gate_q,
+                      w_gate_scale, w_up_q, w_up_scale, w_down, expert_out, ws, ws_bytes,
+                      stream=None, raise_on_error=True):
+    st = load().moe_expert_ffn_w8(_ptr(send), _ptr(send_scales), payload, _ptr(expert_offsets),
+                                  max_rows, E, H, F, _ptr(w_gate_q), _ptr(w_gate_scale),
+                                  _ptr(w_up_q), _ptr(w_up_scale), _ptr(w_down), _ptr(expert_out),
+                                  _ptr(ws), ws_bytes, _stream(stream))
+    return _check(st, "moe_expert_ffn_w8", raise_on_error)
 
 
 def moe_combine(expert_out, max_rows, slot_row, topk_w, T, k, H, y, status=None, stream=None,

@@ -140,8 +140,8 @@ moe_status_t moe_expert_ffn(const void* send, const float* send_scales, moe_payl
   if (!aligned(ws, 256) || ws_bytes < moe::ffn_workspace_bytes(max_rows, H, F, fp8 ? 1 : 0, E))
     return MOE_ERR_WORKSPACE;
   return from_cuda(moe::launch_expert_ffn(send, send_scales, fp8 ? 1 : 0, expert_offsets, max_rows,
-                                          E, H, F, w_gate, w_up, w_down, nullptr, expert_out, ws,
-                                          reinterpret_cast<cudaStream_t>(stream)));
+                                          E, H, F, w_gate, w_up, w_down, nullptr, nullptr, nullptr,
+                                          expert_out, ws, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 size_t moe_ffn_weight_list_bytes(int E) {
@@ -184,7 +184,52 @@ moe_status_t moe_expert_ffn_list(const void* send, const float* send_scales, moe
   if (!aligned(ws, 256) || ws_bytes < moe::ffn_workspace_bytes(max_rows, H, F, fp8 ? 1 : 0, E))
     return MOE_ERR_WORKSPACE;
   return from_cuda(moe::launch_expert_ffn(send, send_scales, fp8 ? 1 : 0, expert_offsets, max_rows,
-                                          E, H, F, nullptr, nullptr, nullptr, list, expert_out, ws,
+                                          E, H, F, nullptr, nullptr, nullptr, list, nullptr,
+                                          nullptr, expert_out, ws,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_quantize_rows_fp8(const void* x, int rows, int K, void* codes, float* scales,
+                                   moe_stream_t stream) {
+  if (rows < 0 || K < 8) return MOE_ERR_INVALID_ARG;
+  if (K % 16 != 0) return MOE_ERR_UNSUPPORTED;
+  if (rows > 0 && (x == nullptr || codes == nullptr || scales == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scales, 4)) return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_quantize_rows_fp8(x, rows, K, codes, scales,
+                                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_ffn_w8_workspace_size(int max_rows, int E, int H, int F, moe_payload_t payload) {
+  if (max_rows < 0 || E < 1 || H < 1 || F < 1) return 0;
+  return moe::ffn_workspace_bytes(max_rows, H, F, payload == MOE_PAYLOAD_FP8_E4M3_B128, E, 1);
+}
+
+moe_status_t moe_expert_ffn_w8(const void* send, const float* send_scales, moe_payload_t payload,
+                               const int32_t* expert_offsets, int max_rows, int E, int H, int F,
+                               const void* w_gate_q, const float* w_gate_scale,
+                               const void* w_up_q, const float* w_up_scale, const void* w_down,
+                               void* expert_out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (max_rows < 0 || E < 1 || E > kMaxE || H < 1 || F < 1) return MOE_ERR_INVALID_ARG;
+  if (payload != MOE_PAYLOAD_BF16 && payload != MOE_PAYLOAD_FP8_E4M3_B128)
+    return MOE_ERR_INVALID_ARG;
+  const bool fp8 = payload == MOE_PAYLOAD_FP8_E4M3_B128;
+  if (H % 64 != 0 || F % 64 != 0 || (fp8 && H % 128 != 0)) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(E) * F > INT32_MAX || static_cast<long long>(E) * H > INT32_MAX)
+    return MOE_ERR_UNSUPPORTED;
+  if (expert_offsets == nullptr || w_gate_q == nullptr || w_gate_scale == nullptr ||
+      w_up_q == nullptr || w_up_scale == nullptr || w_down == nullptr || ws == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (max_rows > 0 && (send == nullptr || expert_out == nullptr || (fp8 && send_scales == nullptr)))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(send, 16) || !aligned(w_gate_q, 16) || !aligned(w_up_q, 16) ||
+      !aligned(w_down, 16) || !aligned(expert_out, 16) || !aligned(expert_offsets, 4) ||
+      !aligned(send_scales, 4) || !aligned(w_gate_scale, 8) || !aligned(w_up_scale, 8))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(ws, 256) || ws_bytes < moe::ffn_workspace_bytes(max_rows, H, F, fp8 ? 1 : 0, E, 1))
+    return MOE_ERR_WORKSPACE;
+  return from_cuda(moe::launch_expert_ffn(send, send_scales, fp8 ? 1 : 0, expert_offsets, max_rows,
+                                          E, H, F, w_gate_q, w_up_q, w_down, nullptr, w_gate_scale,
+                                          w_up_scale, expert_out, ws,
                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -124,6 +124,25 @@ __device__ __forceinline__ void tc_mma1(uint32_t d_tmem, uint64_t a_desc, uint64
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// kind::f8f6f4 (e4m3 x e4m3 -> fp32), the first projection with FP8 weights
+__device__ __forceinline__ void tc_mma1_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tc_mma2_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // cta_group::2 (pair kernel)
 // Arrive once on the mbarrier at this shared-memory offset in BOTH CTAs of the pair when the MMAs
 // issued so far have completed.
@@ -244,6 +263,14 @@ __host__ __device__ constexpr uint32_t make_idesc(int M, int N) {
          | (static_cast<uint32_t>(M >> 4) << 24);     // M / 16
 }
 
+// Instruction descriptor of tcgen05.mma kind::f8f6f4: fp32 accumulator, e4m3 A and B (format code
+// 0 for both), both K-major.
+__host__ __device__ constexpr uint32_t make_idesc_e4m3(int M, int N) {
+  return (1u << 4)                                    // D format: f32
+         | (static_cast<uint32_t>(N >> 3) << 17)      // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);     // M / 16
+}
+
 __device__ __forceinline__ int owner_of(const int* start, int E, int idx) {
   int lo = 0, hi = E - 1;
   while (lo < hi) {  // largest expert whose first unit is <= idx (it owns the tile)
@@ -324,7 +351,18 @@ struct FfnArgs {
   // 128-row and 256-row boxes), rows local to the expert; nullptr: the grid-constant maps of the
   // contiguous [E, ...] weights, rows global.
   const CUtensorMap* wlist;
+  // FP8 first projection (all three non-null) or bf16 (all null): the A and gate / up maps then
+  // hold e4m3 codes, x_scale [max_rows] the input rows' scales, g_scale / u_scale [E*F] the
+  // weight rows' scales.
+  const float* x_scale;
+  const float* g_scale;
+  const float* u_scale;
 };
+
+// Elements of the K dimension one 128-byte swizzled smem row holds: 64 bf16 or 128 e4m3.
+__device__ __forceinline__ int k_per_stage(const FfnArgs& a, int phase) {
+  return (phase == 1 && a.x_scale != nullptr) ? 128 : BK;
+}
 
 // The descriptor of the weight tile a tile loads, and its first row.  `which`: 0 gate, 1 up,
 // 2 down (128-row box), 3 down (256-row box); `local_row` is the row inside expert e's matrix.
@@ -487,6 +525,8 @@ __device__ __forceinline__ void epilogue_tile(const FfnArgs& args, const Tables&
   const bool row_ok = row < tb.off[e + 1];
   if (phase == 1) {
     __nv_bfloat16* out_row = args.h + static_cast<size_t>(row) * args.F;
+    const bool w8 = args.x_scale != nullptr;
+    const float sx = (w8 && row_ok) ? args.x_scale[row] : 1.0f;
 #pragma unroll 1
     for (int c = 0; c < 128; c += 32) {
       uint32_t g[32], u[32];
@@ -495,12 +535,24 @@ __device__ __forceinline__ void epilogue_tile(const FfnArgs& args, const Tables&
       tmem_wait_ld();
       const int col = n_blk * 128 + c;
       if (row_ok && col < args.F) {
+        // FP8 first projection: g = sx * sw * sum(qx qw), the row's scale times each weight row's
+        // scale (columns past F read as 0; they are not stored).  F % 64 == 0, so a 32-column chunk
+        // is either wholly inside F or wholly outside.
+        const float2* sg2 = w8 ? reinterpret_cast<const float2*>(args.g_scale + static_cast<size_t>(e) * args.F + col) : nullptr;
+        const float2* su2 = w8 ? reinterpret_cast<const float2*>(args.u_scale + static_cast<size_t>(e) * args.F + col) : nullptr;
         uint32_t packed[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float h0 = silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i]));
-          const float h1 = silu_mul(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1]));
-          packed[i] = pack_bf16x2(h0, h1);
+          float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+          float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+          if (w8) {
+            const float2 a = __ldg(sg2 + i), b = __ldg(su2 + i);
+            g0 *= sx * a.x;
+            g1 *= sx * a.y;
+            u0 *= sx * b.x;
+            u1 *= sx * b.y;
+          }
+          packed[i] = pack_bf16x2(silu_mul(g0, u0), silu_mul(g1, u1));
         }
         uint4* dst = reinterpret_cast<uint4*>(out_row + col);
 #pragma unroll
@@ -673,7 +725,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t rank = cluster_rank();  // CTA 0 claims the tiles and issues the MMAs
   const int n1 = (args.F + 127) / 128;   // GEMM-1 column blocks (128 h columns each)
   const int n2 = (args.H + 255) / 256;   // GEMM-2 column blocks (256 output columns each)
-  const int kb1 = (args.H + BK - 1) / BK, kb2 = (args.F + BK - 1) / BK;
+  const int ks1 = k_per_stage(args, 1);  // K elements per GEMM-1 stage: 64 bf16 or 128 e4m3
+  const int kb1 = (args.H + ks1 - 1) / ks1, kb2 = (args.F + BK - 1) / BK;
+  const bool w8 = args.x_scale != nullptr;
   const Abort ab{s.abort_flag, peer_addr(smem_addr(s.abort_flag), rank ^ 1u), true, args.status};
 
   if (warp == 0) {
@@ -769,14 +823,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t a_dst = tiles_base + stage * kStageBytes;
           const uint32_t b_dst = a_dst + kATileBytes;
           const uint32_t fb = smem_addr(&s.full[stage]);
+          const int kx = kb * (t.phase == 1 ? ks1 : BK);
           if (rank == 0) {
             mbar_arrive_expect_tx(fb, stage_tx);
-            if (rows > 0) tma_load_2d(a_dst, ma, fb, kb * BK, row_a);
-            tma_load_2d(b_dst, mb, fb, kb * BK, row_b);
+            if (rows > 0) tma_load_2d(a_dst, ma, fb, kx, row_a);
+            tma_load_2d(b_dst, mb, fb, kx, row_b);
           } else {
             const uint32_t fb0 = peer_addr(fb, 0);
-            if (rows > 0) tma_load_2d_to_leader(a_dst, ma, fb0, kb * BK, row_a);
-            tma_load_2d_to_leader(b_dst, mb, fb0, kb * BK, row_b);
+            if (rows > 0) tma_load_2d_to_leader(a_dst, ma, fb0, kx, row_a);
+            tma_load_2d_to_leader(b_dst, mb, fb0, kx, row_b);
           }
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -803,7 +858,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ---- MMA issuer (CTA 0): M = 256 over the pair, N = 256 ------------------------------------
     if (rank == 0 && lane == 0) {
-      const uint32_t idesc = make_idesc(2 * BM, 256);
+      const uint32_t idesc16 = make_idesc(2 * BM, 256), idesc8 = make_idesc_e4m3(2 * BM, 256);
       int stage = 0;
       uint32_t phase = 0;
       bool issued_any = false;
@@ -813,7 +868,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         int tile;
         if (!take_tile(s, qi, qph, false, ab, tile)) break;
         if (tile < 0) break;
-        const int nkb = tile < U * n1 ? kb1 : kb2;
+        const bool g1 = tile < U * n1;
+        const int nkb = g1 ? kb1 : kb2;
+        const bool f8 = g1 && w8;  // e4m3 operands: K = 32 per MMA, the same 32 bytes of a row
         const int acc = it & 1;
         const uint32_t acc_parity = (it >> 1) & 1;
         if (!wait_bar(smem_addr(&s.acc_empty[acc]), acc_parity ^ 1u, ab)) break;
@@ -829,9 +886,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t a_addr = tiles_base + stage * kStageBytes;
           const uint32_t b_addr = a_addr + kATileBytes;
 #pragma unroll
-          for (int kk = 0; kk < BK / UMMA_K; ++kk)
-            tc_mma2(d_tmem, sw128_desc(a_addr + kk * UMMA_K * 2),
-                    sw128_desc(b_addr + kk * UMMA_K * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+            const uint64_t ad = sw128_desc(a_addr + kk * 32), bd = sw128_desc(b_addr + kk * 32);
+            if (f8)
+              tc_mma2_f8(d_tmem, ad, bd, idesc8, (kb | kk) != 0 ? 1u : 0u);
+            else
+              tc_mma2(d_tmem, ad, bd, idesc16, (kb | kk) != 0 ? 1u : 0u);
+          }
           issued_any = true;
           tc_commit2_both(smem_addr(&s.empty[stage]));
           if (++stage == kStages) {
@@ -916,7 +977,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n1 = (args.F + 127) / 128;
   const int n2 = (args.H + 255) / 256;
-  const int kb1 = (args.H + BK - 1) / BK, kb2 = (args.F + BK - 1) / BK;
+  const int ks1 = k_per_stage(args, 1);  // K elements per GEMM-1 stage: 64 bf16 or 128 e4m3
+  const int kb1 = (args.H + ks1 - 1) / ks1, kb2 = (args.F + BK - 1) / BK;
+  const bool w8 = args.x_scale != nullptr;
   const Abort ab{s.abort_flag, 0u, false, args.status};
 
   if (warp == 0) {
@@ -1000,14 +1063,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t a_dst = tiles_base + stage * kStageBytes;
           const uint32_t b_dst = a_dst + kASingleBytes;
           const uint32_t fb = smem_addr(&s.full[stage]);
+          const int kx = kb * (t.phase == 1 ? ks1 : BK);
           mbar_arrive_expect_tx(fb, stage_tx);
-          tma_load_2d(a_dst, ma, fb, kb * BK, row_a);
+          tma_load_2d(a_dst, ma, fb, kx, row_a);
           if (t.phase == 1) {
             // gate rows -> B rows 0..127 (accumulator columns 0..127), up rows -> 128..255
-            tma_load_2d(b_dst, mb0, fb, kb * BK, row_b);
-            tma_load_2d(b_dst + kBHalfBytes, mb1, fb, kb * BK, row_b);
+            tma_load_2d(b_dst, mb0, fb, kx, row_b);
+            tma_load_2d(b_dst + kBHalfBytes, mb1, fb, kx, row_b);
           } else {
-            tma_load_2d(b_dst, mb0, fb, kb * BK, row_b);
+            tma_load_2d(b_dst, mb0, fb, kx, row_b);
           }
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -1026,7 +1090,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ---- MMA issuer (M = 128, N = 256) ---------------------------------------------------------
     if (lane == 0) {
-      const uint32_t idesc = make_idesc(BM, 256);
+      const uint32_t idesc16 = make_idesc(BM, 256), idesc8 = make_idesc_e4m3(BM, 256);
       int stage = 0;
       uint32_t phase = 0;
       bool issued_any = false;
@@ -1036,7 +1100,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         int tile;
         if (!take_tile(s, qi, qph, false, ab, tile)) break;
         if (tile < 0) break;
-        const int nkb = tile < U * n1 ? kb1 : kb2;
+        const bool g1 = tile < U * n1;
+        const int nkb = g1 ? kb1 : kb2;
+        const bool f8 = g1 && w8;  // e4m3 operands: K = 32 per MMA, the same 32 bytes of a row
         const int acc = it & 1;
         const uint32_t acc_parity = (it >> 1) & 1;
         if (!wait_bar(smem_addr(&s.acc_empty[acc]), acc_parity ^ 1u, ab)) break;
@@ -1052,9 +1118,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t a_addr = tiles_base + stage * kStageBytes;
           const uint32_t b_addr = a_addr + kASingleBytes;
 #pragma unroll
-          for (int kk = 0; kk < BK / UMMA_K; ++kk)
-            tc_mma1(d_tmem, sw128_desc(a_addr + kk * UMMA_K * 2),
-                    sw128_desc(b_addr + kk * UMMA_K * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+            const uint64_t ad = sw128_desc(a_addr + kk * 32), bd = sw128_desc(b_addr + kk * 32);
+            if (f8)
+              tc_mma1_f8(d_tmem, ad, bd, idesc8, (kb | kk) != 0 ? 1u : 0u);
+            else
+              tc_mma1(d_tmem, ad, bd, idesc16, (kb | kk) != 0 ? 1u : 0u);
+          }
           issued_any = true;
           tc_commit1(smem_addr(&s.empty[stage]));
           if (++stage == kStages) {
@@ -1138,6 +1208,49 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// FP8 rows with one scale per row (FP8 weights, and the FFN's own input rows for the FP8 first
+// projection): one warp per row.  scale = amax / 448 (1 when amax == 0); code = e4m3
+// round-to-nearest-even, saturating, of the fp32 IEEE quotient value / scale.  Rows [0, n) with
+// n = min(*n_rows_dev, n_rows) when n_rows_dev is given, else n_rows.
+__global__ void __launch_bounds__(256)
+    quant_rows_fp8_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ n_rows_dev,
+                          int n_rows, int K, uint8_t* __restrict__ codes,
+                          float* __restrict__ scales) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int rows = n_rows_dev != nullptr ? min(__ldg(n_rows_dev), n_rows) : n_rows;
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  const int nv = K / 8;  // 16-byte vectors of 8 bf16 per row
+  for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < rows; r += gridDim.x * wpb) {
+    const uint4* row = src + static_cast<size_t>(r) * nv;
+    float amax = 0.0f;
+    for (int v = lane; v < nv; v += 32) {
+      const uint4 w = ld_nc_v4(row + v);
+      const uint32_t q[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(q[i])), fabsf(bf16_hi(q[i]))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+    const float sc = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f);
+    uint2* out = reinterpret_cast<uint2*>(codes + static_cast<size_t>(r) * K);
+    for (int v = lane; v < nv; v += 32) {
+      const uint4 w = ld_nc_v4(row + v);
+      const uint32_t q[4] = {w.x, w.y, w.z, w.w};
+      uint32_t packed[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 pr = make_float2(__fdiv_rn(bf16_lo(q[i]), sc), __fdiv_rn(bf16_hi(q[i]), sc));
+        packed[i] = static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(pr, __NV_SATFINITE, __NV_E4M3));
+      }
+      out[v] = make_uint2(packed[0] | (packed[1] << 16), packed[2] | (packed[3] << 16));
+    }
+    if (lane == 0) scales[r] = sc;
+  }
+}
+
 // ---- host side -----------------------------------------------------------------------------------
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -1168,7 +1281,41 @@ bool make_tmap(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t cols, u
   return r == CUDA_SUCCESS;
 }
 
+// 2-D tensor of bytes (e4m3 codes) [rows, cols] read in boxes of box_rows x 128 with the 128-byte
+// swizzle: the same shared-memory rows as a box_rows x 64 bf16 box.
+bool make_tmap_u8(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {128u, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+cudaError_t launch_quant_rows(const void* src, const int32_t* n_rows_dev, int n_rows, int K,
+                              void* codes, float* scales, cudaStream_t s) {
+  if (n_rows == 0) return cudaSuccess;
+  long long blocks = (static_cast<long long>(n_rows) + 7) / 8;
+  const long long cap = static_cast<long long>(num_sms()) * 8;
+  if (blocks > cap) blocks = cap;
+  return launch_pdl(quant_rows_fp8_kernel, dim3(static_cast<int>(blocks)), dim3(256), 0, s,
+                    static_cast<const uint4*>(src), n_rows_dev, n_rows, K,
+                    static_cast<uint8_t*>(codes), scales);
+}
+
 }  // namespace
+
+cudaError_t launch_quantize_rows_fp8(const void* x, int rows, int K, void* codes, float* scales,
+                                     cudaStream_t s) {
+  const cudaError_t err = launch_quant_rows(x, nullptr, rows, K, codes, scales, s);
+  if (err != cudaSuccess) return err;
+  return cudaGetLastError();
+}
 
 // Persistent grid of 2-CTA clusters of `kernel`: as many clusters as can be resident at once (one
 // CTA per SM), looked up once per device, kernel and shared-memory size.
@@ -1212,10 +1359,18 @@ static size_t ffn_counter_count(int max_rows, int E) {
   return static_cast<size_t>(max_rows) / BM + static_cast<size_t>(E) + 1;
 }
 
-size_t ffn_workspace_bytes(int max_rows, int H, int F, int fp8, int E) {
+// W8 (FP8 first projection): after the dequantised rows, the input rows' e4m3 codes [max_rows, H]
+// and their scales fp32 [max_rows].
+static size_t ffn_w8_bytes(int max_rows, int H) {
+  return round256(static_cast<size_t>(max_rows) * H) + round256(static_cast<size_t>(max_rows) * 4);
+}
+
+size_t ffn_workspace_bytes(int max_rows, int H, int F, int fp8, int E, int w8) {
   const size_t h_bytes = round256(static_cast<size_t>(max_rows) * F * 2);
   const size_t x_bytes = fp8 ? round256(static_cast<size_t>(max_rows) * H * 2) : 0;
-  return 256 + h_bytes + x_bytes + round256((2 * ffn_counter_count(max_rows, E) + 4) * sizeof(int));
+  const size_t q_bytes = w8 ? ffn_w8_bytes(max_rows, H) : 0;
+  return 256 + h_bytes + x_bytes + q_bytes +
+         round256((2 * ffn_counter_count(max_rows, E) + 4) * sizeof(int));
 }
 
 size_t ffn_weight_list_bytes(int E) { return static_cast<size_t>(E) * 4 * sizeof(CUtensorMap); }
@@ -1237,8 +1392,11 @@ cudaError_t ffn_weight_list_init(const void* const* w_gate, const void* const* w
 cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp8,
                               const int32_t* expert_offsets, int max_rows, int E, int H, int F,
                               const void* w_gate, const void* w_up, const void* w_down,
-                              const void* wlist, void* expert_out, void* ws, cudaStream_t s) {
+                              const void* wlist, const float* w_gate_scale,
+                              const float* w_up_scale, void* expert_out, void* ws,
+                              cudaStream_t s) {
   if (max_rows == 0) return cudaSuccess;
+  const bool w8 = w_gate_scale != nullptr;
   char* base = static_cast<char*>(ws);
   int* status = reinterpret_cast<int*>(base);
   __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(base + 256);
@@ -1247,6 +1405,13 @@ cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp
   if (fp8) {
     xdq = reinterpret_cast<uint4*>(base + off);
     off += round256(static_cast<size_t>(max_rows) * H * 2);
+  }
+  uint8_t* xq = nullptr;
+  float* xs = nullptr;
+  if (w8) {
+    xq = reinterpret_cast<uint8_t*>(base + off);
+    xs = reinterpret_cast<float*>(base + off + round256(static_cast<size_t>(max_rows) * H));
+    off += ffn_w8_bytes(max_rows, H);
   }
   int* done = reinterpret_cast<int*>(base + off);
   int* used = done + ffn_counter_count(max_rows, E);
@@ -1265,15 +1430,29 @@ cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp
     if (err != cudaSuccess) return err;
     a_src = xdq;
   }
+  if (w8) {
+    // the FFN input rows, each quantised on its own: e4m3 codes and one scale per row
+    err = launch_quant_rows(a_src, expert_offsets + E, max_rows, H, xq, xs, s);
+    if (err != cudaSuccess) return err;
+  }
   CUtensorMap tm_x, tm_g, tm_u, tm_h, tm_d128, tm_d256;
   SmallBoxMaps tm_xs, tm_hs;
   for (int i = 0; i < 3; ++i)
-    if (!make_tmap(&tm_xs.m[i], a_src, max_rows, H, small_box_rows(i)) ||
+    if (!(w8 ? make_tmap_u8(&tm_xs.m[i], xq, max_rows, H, small_box_rows(i))
+             : make_tmap(&tm_xs.m[i], a_src, max_rows, H, small_box_rows(i))) ||
         !make_tmap(&tm_hs.m[i], h, max_rows, F, small_box_rows(i)))
       return cudaErrorInvalidValue;
-  if (!make_tmap(&tm_x, a_src, max_rows, H, BM) || !make_tmap(&tm_h, h, max_rows, F, BM))
+  if (!(w8 ? make_tmap_u8(&tm_x, xq, max_rows, H, BM) : make_tmap(&tm_x, a_src, max_rows, H, BM)) ||
+      !make_tmap(&tm_h, h, max_rows, F, BM))
     return cudaErrorInvalidValue;
-  if (wlist != nullptr) {
+  if (w8) {
+    // e4m3 gate / up codes [E * F, H]; the down projection stays bf16
+    if (!make_tmap_u8(&tm_g, w_gate, static_cast<uint64_t>(E) * F, H, 128) ||
+        !make_tmap_u8(&tm_u, w_up, static_cast<uint64_t>(E) * F, H, 128) ||
+        !make_tmap(&tm_d128, w_down, static_cast<uint64_t>(E) * H, F, 128) ||
+        !make_tmap(&tm_d256, w_down, static_cast<uint64_t>(E) * H, F, 256))
+      return cudaErrorInvalidValue;
+  } else if (wlist != nullptr) {
     // the kernels take each expert's descriptors from the list; these are never read
     memset(&tm_g, 0, sizeof(CUtensorMap));
     memset(&tm_u, 0, sizeof(CUtensorMap));
@@ -1292,9 +1471,10 @@ cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp
   // programmatically behind it, starts on those SMs without waiting for it (it waits at its end).
   const FfnArgs fa_single{expert_offsets, E, max_rows, H, F, h,
                           static_cast<__nv_bfloat16*>(expert_out), status, done, used, sched + 2,
-                          wl};
+                          wl, xs, w_gate_scale, w_up_scale};
   const FfnArgs fa_pair{expert_offsets, E, max_rows, H, F, h,
-                        static_cast<__nv_bfloat16*>(expert_out), status, done, used, sched, wl};
+                        static_cast<__nv_bfloat16*>(expert_out), status, done, used, sched, wl,
+                        xs, w_gate_scale, w_up_scale};
   const size_t smem_single = ring_smem_bytes(E, kStagesSingle, kASingleBytes + 2 * kBHalfBytes);
   const size_t smem_pair = ring_smem_bytes(E, kStagesPair, kATileBytes + kBHalfBytes);
   err = cudaFuncSetAttribute(ffn_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -69,14 +69,22 @@ cudaError_t launch_combine(const void* expert_out, int max_rows, const int32_t* 
 
 // FFN workspace layout: [0,4) status, [256, ..) h [max_rows, F] bf16, then for the FP8 payload the
 // dequantised rows [max_rows, H] bf16, then the GEMM-1 completion counters.
-size_t ffn_workspace_bytes(int max_rows, int H, int F, int fp8, int E);
+// w8: room for the FFN input rows' e4m3 codes [max_rows, H] and scales [max_rows] as well.
+size_t ffn_workspace_bytes(int max_rows, int H, int F, int fp8, int E, int w8 = 0);
 
 // wlist == nullptr: the weights are contiguous [E, F, H] / [E, H, F] arrays; otherwise the
 // per-expert descriptors written by ffn_weight_list_init (and w_gate / w_up / w_down are unused).
+// w_gate_scale / w_up_scale non-null: w_gate / w_up are e4m3 codes [E, F, H] with one fp32 scale
+// per row [E, F] (FP8 first projection); wlist must then be nullptr.
 cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp8,
                               const int32_t* expert_offsets, int max_rows, int E, int H, int F,
                               const void* w_gate, const void* w_up, const void* w_down,
-                              const void* wlist, void* expert_out, void* ws, cudaStream_t s);
+                              const void* wlist, const float* w_gate_scale,
+                              const float* w_up_scale, void* expert_out, void* ws, cudaStream_t s);
+
+// Rows of bf16 [rows, K] -> e4m3 codes [rows, K] + one fp32 scale per row (amax / 448).
+cudaError_t launch_quantize_rows_fp8(const void* x, int rows, int K, void* codes, float* scales,
+                                     cudaStream_t s);
 
 // Per-expert weight descriptors: four 128-byte TMA descriptors per expert.
 size_t ffn_weight_list_bytes(int E);

@@ -73,6 +73,7 @@ class MoeShuffle:
         self.ws_dispatch = torch.zeros(self.ws_dispatch_bytes, dtype=torch.uint8, device=dev)
         self.ws_ffn_bytes = _lib.moe_ffn_workspace_size(S, E, H, F, self.payload)
         self.ws_ffn = torch.zeros(self.ws_ffn_bytes, dtype=torch.uint8, device=dev)
+        self.ws_ffn_w8 = None  # allocated by the first expert_ffn_w8 call
 
     # -- views into the FFN workspace ----------------------------------------------------------
     @property
@@ -147,6 +148,52 @@ class MoeShuffle:
                                  self.max_rows, self.E, self.H, self.F, wlist, self.expert_out,
                                  self.ws_ffn, self.ws_ffn_bytes, stream)
 
+    def quantize_expert_weights_fp8(self, w_gate, w_up):
+        """FP8 gate / up weights for ``expert_ffn_w8``: (gate codes, gate scales, up codes, up
+        scales), e4m3 [E,F,H] with one fp32 scale per row [E,F].  Set-up, outside the step."""
+        expect(w_gate, (self.E, self.F, self.H), torch.bfloat16, "w_gate", self.device)
+        expect(w_up, (self.E, self.F, self.H), torch.bfloat16, "w_up", self.device)
+        out = []
+        for w in (w_gate, w_up):
+            q = torch.empty((self.E, self.F, self.H), dtype=torch.uint8, device=self.device)
+            sc = torch.empty((self.E, self.F), dtype=torch.float32, device=self.device)
+            _lib.moe_quantize_rows_fp8(w, self.E * self.F, self.H, q, sc)
+            out += [q, sc]
+        return tuple(out)
+
+    def expert_ffn_w8(self, w_gate_q, w_gate_scale, w_up_q, w_up_scale, w_down, send=None,
+                      send_scales=None, expert_offsets=None, stream=None):
+        """expert_ffn with FP8 gate / up weights (``quantize_expert_weights_fp8``) and bf16 down
+        weights; the FFN input rows are quantised to FP8 per row inside the call."""
+        expect(w_gate_q, (self.E, self.F, self.H), torch.uint8, "w_gate_q", self.device)
+        expect(w_up_q, (self.E, self.F, self.H), torch.uint8, "w_up_q", self.device)
+        expect(w_gate_scale, (self.E, self.F), torch.float32, "w_gate_scale", self.device)
+        expect(w_up_scale, (self.E, self.F), torch.float32, "w_up_scale", self.device)
+        expect(w_down, (self.E, self.H, self.F), torch.bfloat16, "w_down", self.device)
+        if send is not None:
+            expect(send, (self.max_rows, self.H), self.send.dtype, "send", self.device)
+        if send_scales is not None:
+            expect(send_scales, (self.max_rows, self.H // 128), torch.float32, "send_scales",
+                   self.device)
+        if expert_offsets is not None:
+            expect(expert_offsets, (self.E + 1,), torch.int32, "expert_offsets", self.device)
+        if self.ws_ffn_w8 is None:
+            n = _lib.moe_ffn_w8_workspace_size(self.max_rows, self.E, self.H, self.F, self.payload)
+            self.ws_ffn_w8 = torch.zeros(n, dtype=torch.uint8, device=self.device)
+        _lib.moe_expert_ffn_w8(self.send if send is None else send,
+                               self.send_scales if send_scales is None else send_scales,
+                               self.payload,
+                               self.expert_offsets if expert_offsets is None else expert_offsets,
+                               self.max_rows, self.E, self.H, self.F, w_gate_q, w_gate_scale,
+                               w_up_q, w_up_scale, w_down, self.expert_out, self.ws_ffn_w8,
+                               self.ws_ffn_w8.numel(), stream)
+
+    @property
+    def h_w8(self) -> torch.Tensor:
+        """The bf16 SwiGLU intermediate of the last ``expert_ffn_w8`` call [max_rows, F]."""
+        n = self.max_rows * self.F * 2
+        return self.ws_ffn_w8[256:256 + n].view(torch.bfloat16).view(self.max_rows, self.F)
+
     def combine(self, expert_out=None, slot_row=None, topk_w=None, stream=None):
         if expert_out is not None:
             expect(expert_out, (self.max_rows, self.H), torch.bfloat16, "expert_out", self.device)
@@ -190,4 +237,5 @@ class MoeShuffle:
         """Synchronise and return (then clear) the device status of the dispatch and FFN stages."""
         a = _lib.moe_sync_status(self.ws_dispatch, stream)
         b = _lib.moe_sync_status(self.ws_ffn, stream)
-        return a if a != _lib.MOE_OK else b
+        c = _lib.moe_sync_status(self.ws_ffn_w8, stream) if self.ws_ffn_w8 is not None else 0
+        return a if a != _lib.MOE_OK else (b if b != _lib.MOE_OK else c)

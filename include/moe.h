@@ -229,6 +229,40 @@ moe_status_t moe_expert_ffn_list(const void* send, const float* send_scales, moe
                                  moe_stream_t stream);
 
 /*
+ * FP8 expert weights for the first projection (W8A8), with the down projection kept in bf16.  The
+ * DWDP page's expert weights are low-precision values with scales ("DWDP: 在NVL72上的高性能分布式
+ * 权重数据并行", 关键优化实施: NvFp4WeightView's w3_w1 weights and their scale tensors); here the
+ * gate and up weights are e4m3 with one fp32 scale per output row, and each FFN input row is
+ * quantised on its own the same way, so g = sx * sw * sum(qx * qw) exactly factorises and the
+ * tensor cores run tcgen05.mma kind::f8f6f4 on the codes.
+ *
+ * moe_quantize_rows_fp8: rows of bf16 x [rows, K] -> e4m3 codes [rows, K] and fp32 scales [rows]:
+ *   scale = amax / 448 of the row (1 when amax == 0), code = e4m3 round-to-nearest-even, saturating,
+ *   of the fp32 IEEE quotient x / scale (the rule of the FP8 payload, with the whole row as the
+ *   block).  Set-up call for the weights (w_gate and w_up as [E*F, H]).  Limits: K % 16 == 0;
+ *   x and codes 16-byte aligned.
+ *
+ * moe_ffn_w8_workspace_size / moe_expert_ffn_w8: moe_expert_ffn with
+ *   w_gate_q, w_up_q      e4m3 codes [E, F, H] (16-byte aligned)
+ *   w_gate_scale,
+ *   w_up_scale            fp32 [E, F] (8-byte aligned): the rows' scales
+ *   w_down                bf16 [E, H, F] as for moe_expert_ffn
+ * and a workspace of moe_ffn_w8_workspace_size (it also holds the input rows' codes and scales).
+ * For expert e and each packed row x (for the FP8 payload, its dequantised bf16 values):
+ *   (qx, sx) = per-row FP8 of x;  g[f] = sx * sg[e,f] * sum_h qx[h] qg[e,f,h], u likewise (fp32
+ *   accumulate);  h = bf16(silu(g) * u);  expert_out = bf16(h . W_down[e]^T).
+ * Limits as for moe_expert_ffn.
+ */
+moe_status_t moe_quantize_rows_fp8(const void* x, int rows, int K, void* codes, float* scales,
+                                   moe_stream_t stream);
+size_t moe_ffn_w8_workspace_size(int max_rows, int E, int H, int F, moe_payload_t payload);
+moe_status_t moe_expert_ffn_w8(const void* send, const float* send_scales, moe_payload_t payload,
+                               const int32_t* expert_offsets, int max_rows, int E, int H, int F,
+                               const void* w_gate_q, const float* w_gate_scale,
+                               const void* w_up_q, const float* w_up_scale, const void* w_down,
+                               void* expert_out, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * Combine: y[t] = bf16( sum_{j=0..k-1, slot_row[t,j] >= 0} topk_w[t,j] * expert_out[slot_row[t,j]] )
  * accumulated in fp32 in slot order j = 0, 1, ... with each product and sum rounded to fp32
  * separately (the NCCL EP page, section 2.1: the combine loops over the top-k slots and adds each
