@@ -15,8 +15,11 @@ from ._lib import (EXPORTS, LIB_PATH, MOE_ERR_CUDA, MOE_ERR_INVALID_ARG, MOE_ERR
                    moe_ffn_w8_workspace_size, moe_quantize_rows_fp8, moe_route, moe_sync_status,
                    status_string)
 from .layer import MoeShuffle
+from .ep import MoeEP, TorchComm
+from ._lib import MOE_ERR_INVALID_COUNTS, moe_ep_regroup
 
-__all__ = ["MoeShuffle", "MoeError", "load", "moe_route", "moe_dispatch", "moe_expert_ffn",
+__all__ = ["MoeShuffle", "MoeEP", "TorchComm", "moe_ep_regroup", "MOE_ERR_INVALID_COUNTS",
+           "MoeError", "load", "moe_route", "moe_dispatch", "moe_expert_ffn",
            "moe_expert_ffn_list", "moe_ffn_weight_list_bytes", "moe_ffn_weight_list_init",
            "moe_expert_ffn_w8", "moe_ffn_w8_workspace_size", "moe_quantize_rows_fp8",
            "moe_combine", "moe_sync_status", "moe_dispatch_noalloc", "moe_capacity", "moe_dispatch_workspace_size",

@@ -18,6 +18,7 @@ MOE_ERR_UNSUPPORTED = 3
 MOE_ERR_CUDA = 4
 MOE_ERR_WORKSPACE = 5
 MOE_ERR_TIMEOUT = 6
+MOE_ERR_INVALID_COUNTS = 7
 MOE_PAYLOAD_BF16 = 0
 MOE_PAYLOAD_FP8_E4M3_B128 = 1
 
@@ -26,7 +27,7 @@ EXPORTS = ["moe_abi_version", "moe_status_string", "moe_capacity", "moe_route",
            "moe_ffn_workspace_size",
            "moe_expert_ffn", "moe_ffn_weight_list_bytes", "moe_ffn_weight_list_init",
            "moe_expert_ffn_list", "moe_quantize_rows_fp8", "moe_ffn_w8_workspace_size",
-           "moe_expert_ffn_w8", "moe_combine", "moe_sync_status"]
+           "moe_expert_ffn_w8", "moe_ep_regroup", "moe_combine", "moe_sync_status"]
 
 _lib = None
 
@@ -63,6 +64,7 @@ def load() -> ctypes.CDLL:
         "moe_quantize_rows_fp8": (I, [P, I, I, P, P, P]),
         "moe_ffn_w8_workspace_size": (Z, [I, I, I, I, I]),
         "moe_expert_ffn_w8": (I, [P, P, I, P, I, I, I, I, P, P, P, P, P, P, P, Z, P]),
+        "moe_ep_regroup": (I, [P, I, I, I, I, I, I, I, I, P, P, Z, P, P, Z, P, P, P]),
         "moe_combine": (I, [P, I, P, P, I, I, I, P, P, P]),
         "moe_sync_status": (I, [P, P]),
     }
@@ -197,6 +199,16 @@ def moe_expert_ffn_w8(send, send_scales, payload, expert_offsets, max_rows, E, H
                                   _ptr(w_up_q), _ptr(w_up_scale), _ptr(w_down), _ptr(expert_out),
                                   _ptr(ws), ws_bytes, _stream(stream))
     return _check(st, "moe_expert_ffn_w8", raise_on_error)
+
+
+def moe_ep_regroup(counts, A, B, src_order, src_stride, src_rows, dst_order, dst_stride, dst_rows,
+                   src, dst, row_bytes, src_aux=None, dst_aux=None, aux_row_bytes=0,
+                   dst_offsets=None, status=None, stream=None, raise_on_error=True):
+    st = load().moe_ep_regroup(_ptr(counts), A, B, src_order, src_stride, src_rows, dst_order,
+                               dst_stride, dst_rows, _ptr(src), _ptr(dst), row_bytes,
+                               _ptr(src_aux), _ptr(dst_aux), aux_row_bytes, _ptr(dst_offsets),
+                               _ptr(status), _stream(stream))
+    return _check(st, "moe_ep_regroup", raise_on_error)
 
 
 def moe_combine(expert_out, max_rows, slot_row, topk_w, T, k, H, y, status=None, stream=None,

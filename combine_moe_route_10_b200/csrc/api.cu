@@ -53,6 +53,7 @@ const char* moe_status_string(moe_status_t st) {
     case MOE_ERR_CUDA: return "MOE_ERR_CUDA: CUDA launch or runtime error";
     case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace too small or misaligned";
     case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT: a bounded device wait ran out";
+    case MOE_ERR_INVALID_COUNTS: return "MOE_ERR_INVALID_COUNTS: row counts do not fit the buffers";
   }
   return "unknown moe_status_t";
 }
@@ -233,6 +234,31 @@ moe_status_t moe_expert_ffn_w8(const void* send, const float* send_scales, moe_p
                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 
+moe_status_t moe_ep_regroup(const int32_t* counts, int A, int B, int src_order, int src_stride,
+                            int src_rows, int dst_order, int dst_stride, int dst_rows,
+                            const void* src, void* dst, size_t row_bytes, const void* src_aux,
+                            void* dst_aux, size_t aux_row_bytes, int32_t* dst_offsets,
+                            int32_t* status, moe_stream_t stream) {
+  if (A < 1 || B < 1 || static_cast<long long>(A) * B > moe::kMaxRegroupSegments)
+    return MOE_ERR_INVALID_ARG;
+  if ((src_order != 0 && src_order != 1) || (dst_order != 0 && dst_order != 1))
+    return MOE_ERR_INVALID_ARG;
+  if (src_stride < 0 || dst_stride < 0 || src_rows < 0 || dst_rows < 0) return MOE_ERR_INVALID_ARG;
+  if (counts == nullptr || !aligned(counts, 4) || !aligned(status, 4) || !aligned(dst_offsets, 4))
+    return MOE_ERR_INVALID_ARG;
+  if (row_bytes == 0 || row_bytes % 4 != 0 || src == nullptr || dst == nullptr ||
+      !aligned(src, 4) || !aligned(dst, 4) || src == dst)
+    return MOE_ERR_INVALID_ARG;
+  if (aux_row_bytes != 0 && (aux_row_bytes % 4 != 0 || src_aux == nullptr || dst_aux == nullptr ||
+                             !aligned(src_aux, 4) || !aligned(dst_aux, 4) || src_aux == dst_aux))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_ep_regroup(
+      counts, A, B, src_order, src_stride, src_rows, dst_order, dst_stride, dst_rows, src, dst,
+      row_bytes, aux_row_bytes ? src_aux : nullptr, aux_row_bytes ? dst_aux : nullptr,
+      aux_row_bytes, dst_offsets, reinterpret_cast<int*>(status),
+      reinterpret_cast<cudaStream_t>(stream)));
+}
+
 moe_status_t moe_combine(const void* expert_out, int max_rows, const int32_t* slot_row,
                          const float* topk_w, int T, int k, int H, void* y, int32_t* status,
                          moe_stream_t stream) {
@@ -259,6 +285,7 @@ moe_status_t moe_sync_status(void* ws, moe_stream_t stream) {
   if (word != 0 && cudaMemset(ws, 0, sizeof(int)) != cudaSuccess) return from_cuda(cudaErrorUnknown);
   if (word & moe::kStatusInvalidTopk) return MOE_ERR_INVALID_TOPK;
   if (word & moe::kStatusTimeout) return MOE_ERR_TIMEOUT;
+  if (word & moe::kStatusBadCounts) return MOE_ERR_INVALID_COUNTS;
   return MOE_OK;
 }
 

@@ -92,4 +92,11 @@ cudaError_t ffn_weight_list_init(const void* const* w_gate, const void* const* w
                                  const void* const* w_down, int E, int H, int F, void* list,
                                  cudaStream_t s);
 
+// Segmented row copy between the layouts on the two sides of an expert-parallel all-to-all.
+cudaError_t launch_ep_regroup(const int32_t* counts, int A, int B, int src_order, int src_stride,
+                              int src_rows, int dst_order, int dst_stride, int dst_rows,
+                              const void* src, void* dst, size_t row_bytes, const void* src_aux,
+                              void* dst_aux, size_t aux_row_bytes, int32_t* dst_offsets,
+                              int* status, cudaStream_t s);
+
 }  // namespace moe

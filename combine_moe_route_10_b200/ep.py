@@ -1,0 +1,270 @@
+"""Expert parallelism over a process group: one process per GPU, rank r owns experts
+[r*E_loc, (r+1)*E_loc) with E_loc = E / R, and the rows cross the ranks in two all-to-alls.
+
+One step on every rank, on its own T tokens (the NCCL EP page, sections 1 and 2: a dispatch
+exchange to the experts' owners and a combine exchange back; the ThunderEP page, section 2.1:
+one contiguous block per destination):
+
+  1. route + dispatch with R ranks: the send buffer is destination-major, expert-major inside a
+     destination's block; ``rank_offsets`` are the send displacements and ``expert_counts`` viewed
+     as [R, E_loc] are the per-(destination, expert) row counts;
+  2. all-to-all of those counts: rank r learns ``recv_counts[s][e]``, the rows source s sends to
+     its local expert e;
+  3. all-to-all of the rows (and, for the FP8 payload, their block scales);
+  4. regroup the received source-major rows expert-major (``moe_ep_regroup``), which also writes
+     the local expert offsets, and run the grouped FFN over the E_loc local experts;
+  5. regroup the FFN output back to source-major order and return it with the reverse all-to-all;
+  6. combine: the returned rows sit exactly where the dispatch put the sent ones, so the weighted
+     combine uses the dispatch's ``slot_row`` unchanged.
+
+Two exchange modes (the NCCL EP page, section 2.2):
+  * ``"ht"`` (high throughput): packed variable-size blocks.  The host reads the send and receive
+    sizes once per step (one small device-to-host copy after the count exchange), so a step cannot
+    be captured in a CUDA graph.
+  * ``"ll"`` (low latency): every (source, destination) block is padded to M = T * min(k, E_loc)
+    rows, the most one source can send to one destination, so every all-to-all has equal, fixed
+    splits: no host synchronisation, and a whole step can be captured in a CUDA graph.  The padding
+    is one more regroup on each side.
+
+Every row of a token meets the same kernels as on a single device: the received rows of expert e
+are ordered by (source rank, source token), which is the single-device dispatch order over the
+rank-major concatenation of all ranks' tokens, so the FFN and the combine see identical operands,
+and the output equals the single-device output bit for bit.
+
+Capacity limits are not applied under expert parallelism (a per-expert limit over all ranks' tokens
+needs the counts of every lower rank before the dispatch).  The local steps run through ``ops``
+(the CUDA library by default); the exchanges go through ``comm`` (``torch.distributed`` by
+default: NCCL between GPUs).
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+from . import _lib
+from .layer import expect
+
+A_MAJOR, B_MAJOR = 0, 1
+
+
+class CudaOps:
+    """The local steps of an expert-parallel rank on this GPU: the C-ABI calls of libmoe.so."""
+
+    def __init__(self, device):
+        _lib.load()
+        self.device = device
+
+    def workspace(self, nbytes):
+        return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=self.device)
+
+    def route(self, logits, T, E, k, renormalize, topk_idx, topk_w):
+        _lib.moe_route(logits, T, E, k, renormalize, topk_idx, topk_w, None)
+
+    def dispatch(self, x, T, H, topk_idx, k, E, R, payload, send, send_scales, expert_counts,
+                 expert_offsets, rank_offsets, slot_row, row_token, ws):
+        _lib.moe_dispatch(x, T, H, topk_idx, k, E, R, 0, payload, send, send_scales,
+                          expert_counts, expert_offsets, rank_offsets, slot_row, row_token, ws,
+                          ws.numel())
+
+    def regroup(self, counts, A, B, src_order, src_stride, src, dst_order, dst_stride, dst,
+                src_aux=None, dst_aux=None, dst_offsets=None, status=None):
+        _lib.moe_ep_regroup(counts, A, B, src_order, src_stride, src.shape[0], dst_order,
+                            dst_stride, dst.shape[0], src, dst, src[0].numel() * src.element_size(),
+                            src_aux, dst_aux,
+                            0 if src_aux is None else src_aux[0].numel() * src_aux.element_size(),
+                            dst_offsets, status)
+
+    def expert_ffn(self, rows, scales, payload, offsets, max_rows, E, H, F, w_gate, w_up, w_down,
+                   out, ws):
+        _lib.moe_expert_ffn(rows, scales, payload, offsets, max_rows, E, H, F, w_gate, w_up,
+                            w_down, out, ws, ws.numel())
+
+    def combine(self, expert_out, max_rows, slot_row, topk_w, T, k, H, y):
+        _lib.moe_combine(expert_out, max_rows, slot_row, topk_w, T, k, H, y, None)
+
+    def sync_status(self, ws) -> int:
+        return _lib.moe_sync_status(ws)
+
+
+class TorchComm:
+    """The exchange over a ``torch.distributed`` process group (NCCL over NVLink between GPUs;
+    gloo on CPU): ``all_to_all(out, inp, out_splits, in_splits)`` splits along dim 0, equal splits
+    when the lists are None."""
+
+    def __init__(self, group=None):
+        self.group = group
+        self.rank = dist.get_rank(group)
+        self.size = dist.get_world_size(group)
+
+    def all_to_all(self, out, inp, out_splits=None, in_splits=None):
+        dist.all_to_all_single(out, inp, out_splits, in_splits, group=self.group)
+
+
+def _rows_as_bytes(t: torch.Tensor) -> torch.Tensor:
+    """A [n, ...] buffer as uint8 [n, row_bytes], so that every backend exchanges it as bytes."""
+    return t.view(torch.uint8).view(t.shape[0], -1)
+
+
+class MoeEP:
+    """One expert-parallel MoE layer on this rank: T local tokens of width H, E experts over the
+    R ranks of ``comm`` (E % R == 0), top-k, SwiGLU FFN width F.
+
+    ``mode`` is "ht" or "ll" (see the module docstring); ``payload`` is "bf16" or "fp8" (e4m3 codes
+    plus one fp32 scale per 128 elements cross the exchange; the FFN output returns in bf16).
+    ``recv_rows`` is the initial receive capacity in rows for "ht" (grown when a step needs more;
+    default T*k); "ll" always holds R*M rows.  Weights are this rank's experts only:
+    ``w_gate``, ``w_up`` [E_loc, F, H] and ``w_down`` [E_loc, H, F], bf16.
+    ``comm`` carries the all-to-alls (default: ``TorchComm`` over the default process group).
+    """
+
+    def __init__(self, T: int, H: int, E: int, k: int, F: int, comm=None, payload: str = "bf16",
+                 mode: str = "ht", renormalize: bool = True, recv_rows: int | None = None,
+                 device="cuda", ops=None):
+        if mode not in ("ht", "ll"):
+            raise ValueError("mode must be 'ht' or 'll'")
+        if payload not in ("bf16", "fp8"):
+            raise ValueError("payload must be 'bf16' or 'fp8'")
+        self.comm = TorchComm() if comm is None else comm
+        self.R = self.comm.size
+        self.rank = self.comm.rank
+        if E % self.R != 0:
+            raise ValueError(f"E={E} is not a multiple of the {self.R} ranks")
+        self.T, self.H, self.E, self.k, self.F = T, H, E, k, F
+        self.E_loc = E // self.R
+        self.mode = mode
+        self.renormalize = bool(renormalize)
+        self.fp8 = payload == "fp8"
+        self.payload = _lib.MOE_PAYLOAD_FP8_E4M3_B128 if self.fp8 else _lib.MOE_PAYLOAD_BF16
+        dev = torch.device(device)
+        if dev.type == "cuda" and dev.index is None:
+            dev = torch.device("cuda", torch.cuda.current_device())
+        self.device = dev
+        self.ops = CudaOps(dev) if ops is None else ops
+        i32 = dict(dtype=torch.int32, device=dev)
+        S = T * k
+        self.M = T * min(k, self.E_loc)  # most rows one source sends one destination
+        self.row_dtype = torch.uint8 if self.fp8 else torch.bfloat16
+        self.nb = H // 128 if self.fp8 else 0  # scale blocks per row
+        # local side: route, dispatch, combine on this rank's tokens
+        self.topk_idx = torch.empty((T, k), **i32)
+        self.topk_w = torch.empty((T, k), dtype=torch.float32, device=dev)
+        self.send = torch.empty((S, H), dtype=self.row_dtype, device=dev)
+        self.send_scales = torch.empty((S, self.nb), dtype=torch.float32, device=dev) \
+            if self.fp8 else None
+        self.expert_counts = torch.empty(E, **i32)
+        self.expert_offsets = torch.empty(E + 1, **i32)
+        self.rank_offsets = torch.empty(self.R + 1, **i32)
+        self.slot_row = torch.empty((T, k), **i32)
+        self.row_token = torch.empty(max(S, 1), **i32)
+        self.ret = torch.empty((S, H), dtype=torch.bfloat16, device=dev)  # returned FFN rows
+        self.y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        self.ws_dispatch = self.ops.workspace(_lib.moe_dispatch_workspace_size(T, E, k))
+        # the status word of the regroups (counts from other ranks are checked on the device)
+        self.ws_regroup = self.ops.workspace(256)
+        # expert side
+        self.recv_counts = torch.empty(self.R * self.E_loc, **i32)
+        self.local_offsets = torch.empty(self.E_loc + 1, **i32)
+        if mode == "ll":
+            P = self.R * self.M
+            self.send_pad = torch.empty((P, H), dtype=self.row_dtype, device=dev)
+            self.send_pad_scales = torch.empty((P, self.nb), dtype=torch.float32, device=dev) \
+                if self.fp8 else None
+            self.ret_pad = torch.empty((P, H), dtype=torch.bfloat16, device=dev)
+            self._alloc_expert_side(P)
+        else:
+            self._alloc_expert_side(max(int(recv_rows) if recv_rows else S, 1))
+            self._sizes = torch.empty(self.R + 1 + self.R * self.E_loc, dtype=torch.int32,
+                                      pin_memory=dev.type == "cuda")
+
+    def _alloc_expert_side(self, rows: int):
+        dev, H = self.device, self.H
+        self.cap = rows
+        self.recv = torch.empty((rows, H), dtype=self.row_dtype, device=dev)
+        self.recv_scales = torch.empty((rows, self.nb), dtype=torch.float32, device=dev) \
+            if self.fp8 else None
+        self.grouped = torch.empty((rows, H), dtype=self.row_dtype, device=dev)
+        self.grouped_scales = torch.empty((rows, self.nb), dtype=torch.float32, device=dev) \
+            if self.fp8 else None
+        self.expert_out = torch.empty((rows, H), dtype=torch.bfloat16, device=dev)
+        self.back = torch.empty((rows, H), dtype=torch.bfloat16, device=dev)
+        self.ws_ffn = self.ops.workspace(
+            _lib.moe_ffn_workspace_size(rows, self.E_loc, H, self.F, self.payload))
+
+    # -- the exchange -------------------------------------------------------------------------
+    def _all_to_all(self, out, inp, out_splits=None, in_splits=None):
+        self.comm.all_to_all(out, inp, out_splits, in_splits)
+
+    def _exchange_rows(self, out, inp, out_splits, in_splits):
+        self._all_to_all(_rows_as_bytes(out), _rows_as_bytes(inp), out_splits, in_splits)
+
+    def _ht_sizes(self):
+        """Send and receive row counts per peer: one device-to-host copy after the count exchange."""
+        R = self.R
+        self._sizes[:R + 1].copy_(self.rank_offsets, non_blocking=True)
+        self._sizes[R + 1:].copy_(self.recv_counts, non_blocking=True)
+        if self.device.type == "cuda":
+            torch.cuda.current_stream(self.device).synchronize()
+        ro = self._sizes[:R + 1].tolist()
+        rc = self._sizes[R + 1:].view(R, self.E_loc).sum(1).tolist()
+        send_splits = [ro[d + 1] - ro[d] for d in range(R)]
+        return send_splits, [int(v) for v in rc]
+
+    # -- one step -----------------------------------------------------------------------------
+    def forward(self, logits, x, w_gate, w_up, w_down) -> torch.Tensor:
+        T, H, E, k, R, E_loc = self.T, self.H, self.E, self.k, self.R, self.E_loc
+        dev = self.device
+        expect(logits, (T, E), torch.float32, "logits", dev)
+        expect(x, (T, H), torch.bfloat16, "x", dev)
+        expect(w_gate, (E_loc, self.F, H), torch.bfloat16, "w_gate", dev)
+        expect(w_up, (E_loc, self.F, H), torch.bfloat16, "w_up", dev)
+        expect(w_down, (E_loc, H, self.F), torch.bfloat16, "w_down", dev)
+        ops = self.ops
+        ops.route(logits, T, E, k, self.renormalize, self.topk_idx, self.topk_w)
+        ops.dispatch(x, T, H, self.topk_idx, k, E, R, self.payload, self.send, self.send_scales,
+                     self.expert_counts, self.expert_offsets, self.rank_offsets, self.slot_row,
+                     self.row_token, self.ws_dispatch)
+        # counts: expert_counts is [R destinations, E_loc] already
+        self._all_to_all(self.recv_counts, self.expert_counts)
+        st = self.ws_regroup
+        if self.mode == "ht":
+            send_splits, recv_splits = self._ht_sizes()
+            n_recv = sum(recv_splits)
+            if n_recv > self.cap:
+                self._alloc_expert_side(max(n_recv, self.cap + self.cap // 4))
+            n_send = sum(send_splits)
+            self._exchange_rows(self.recv[:n_recv], self.send[:n_send], recv_splits, send_splits)
+            if self.fp8:
+                self._all_to_all(self.recv_scales[:n_recv], self.send_scales[:n_send],
+                                 recv_splits, send_splits)
+            src_stride = 0
+        else:
+            ops.regroup(self.expert_counts, R, E_loc, A_MAJOR, 0, self.send, A_MAJOR, self.M,
+                        self.send_pad, self.send_scales, self.send_pad_scales, None, st)
+            self._exchange_rows(self.recv, self.send_pad, None, None)
+            if self.fp8:
+                self._all_to_all(self.recv_scales, self.send_pad_scales)
+            src_stride = self.M
+        # expert-major for the grouped FFN; local_offsets are the FFN's expert offsets
+        ops.regroup(self.recv_counts, R, E_loc, A_MAJOR, src_stride, self.recv, B_MAJOR, 0,
+                    self.grouped, self.recv_scales, self.grouped_scales, self.local_offsets, st)
+        ops.expert_ffn(self.grouped, self.grouped_scales, self.payload, self.local_offsets,
+                       self.cap, E_loc, H, self.F, w_gate, w_up, w_down, self.expert_out,
+                       self.ws_ffn)
+        ops.regroup(self.recv_counts, R, E_loc, B_MAJOR, 0, self.expert_out, A_MAJOR, src_stride,
+                    self.back, None, None, None, st)
+        if self.mode == "ht":
+            self._exchange_rows(self.ret[:n_send], self.back[:n_recv], send_splits, recv_splits)
+        else:
+            self._exchange_rows(self.ret_pad, self.back, None, None)
+            ops.regroup(self.expert_counts, R, E_loc, A_MAJOR, self.M, self.ret_pad, A_MAJOR, 0,
+                        self.ret, None, None, None, st)
+        ops.combine(self.ret, self.ret.shape[0], self.slot_row, self.topk_w, T, k, H, self.y)
+        return self.y
+
+    def status(self) -> int:
+        """Synchronise; the first non-OK device status of this rank's dispatch, regroups and FFN."""
+        for ws in (self.ws_dispatch, self.ws_regroup, self.ws_ffn):
+            st = self.ops.sync_status(ws)
+            if st != _lib.MOE_OK:
+                return st
+        return _lib.MOE_OK

@@ -52,7 +52,8 @@ typedef enum {
   MOE_ERR_UNSUPPORTED = 3,  /* valid but not implemented here (e.g. H % 64 != 0)                  */
   MOE_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed                               */
   MOE_ERR_WORKSPACE = 5,    /* workspace too small or not 256-byte aligned                        */
-  MOE_ERR_TIMEOUT = 6       /* a bounded device-side wait ran out; the kernel stopped early       */
+  MOE_ERR_TIMEOUT = 6,      /* a bounded device-side wait ran out; the kernel stopped early       */
+  MOE_ERR_INVALID_COUNTS = 7 /* row counts (found on the device) do not fit the buffers they describe */
 } moe_status_t;
 
 typedef enum {
@@ -278,9 +279,51 @@ moe_status_t moe_combine(const void* expert_out, int max_rows, const int32_t* sl
                          moe_stream_t stream);
 
 /*
+ * moe_ep_regroup: the row moves on both sides of an expert-parallel all-to-all, as one segmented
+ * copy.
+ *
+ * With expert parallelism over R ranks, rank r owns experts [r*E_loc, (r+1)*E_loc), E_loc = E/R.
+ * A rank's moe_dispatch with that R leaves its send buffer destination-major (rank_offsets are the
+ * send displacements) and, inside each destination's block, expert-major; expert_counts viewed as
+ * [R, E_loc] counts the rows of every (destination, expert) segment.  After the exchange, the
+ * receiver holds R source blocks, source s's block holding recv_counts[s][e] rows of each local
+ * expert e in turn (the NCCL EP page, section 2.2: packed per-destination buffers in the
+ * high-throughput mode, one [E x M x H] block per peer in the low-latency mode; the ThunderEP page,
+ * section 2.1: one contiguous block per destination).  The grouped FFN wants those rows
+ * expert-major, and the return trip wants them back in source-major order.
+ *
+ * counts [A, B] int32 (device, row-major) names A*B segments; segment (a, b) holds counts[a][b]
+ * rows of row_bytes bytes.  Each side lays the segments out in one of two orders:
+ *   order 0 (a-major): segment (a, b) follows (a, b-1); block a starts at row a*stride, or, with
+ *                      stride 0, right after block a-1 (packed);
+ *   order 1 (b-major): segment (a, b) follows (a-1, b); block b starts at row b*stride, or packed.
+ * Row q of segment (a, b) moves from its src position to its dst position; rows of neither side
+ * outside the segments are left untouched.  An optional second payload (src_aux / dst_aux,
+ * aux_row_bytes per row, e.g. the FP8 block scales) moves with the same row map.
+ *   receive side:  A = R sources, B = E_loc, src order 0 (stride 0, or the padded block rows),
+ *                  dst order 1 packed, dst_offsets [E_loc + 1] gets the expert offsets for the FFN;
+ *   return trip:   the same counts with src and dst swapped;
+ *   low-latency padding of the send buffer: A = R destinations, B = E_loc, src order 0 packed,
+ *                  dst order 0 with stride M (and back).
+ * src_rows / dst_rows are the row capacities of the two buffers; a position outside them, a
+ * negative count, or a block longer than its stride is not copied, and records
+ * MOE_ERR_INVALID_COUNTS in *status (a word read by moe_sync_status, may be NULL): the counts come
+ * from other ranks, so the device checks them.  dst_offsets (may be NULL) gets the packed b-major
+ * start of every b and the total at [B].
+ * Limits: A*B <= 4096; row_bytes and aux_row_bytes multiples of 4 (16-byte vectors when rows and
+ * pointers allow); src != dst.  Asynchronous on `stream`.
+ */
+moe_status_t moe_ep_regroup(const int32_t* counts, int A, int B, int src_order, int src_stride,
+                            int src_rows, int dst_order, int dst_stride, int dst_rows,
+                            const void* src, void* dst, size_t row_bytes, const void* src_aux,
+                            void* dst_aux, size_t aux_row_bytes, int32_t* dst_offsets,
+                            int32_t* status, moe_stream_t stream);
+
+/*
  * Synchronise `stream`, read the device status word at the start of a dispatch or FFN workspace
  * (or any status word given to moe_combine / moe_dispatch_noalloc), clear it, and report it:
- * MOE_OK, MOE_ERR_INVALID_TOPK or MOE_ERR_TIMEOUT (MOE_ERR_CUDA if the stream itself failed).
+ * MOE_OK, MOE_ERR_INVALID_TOPK, MOE_ERR_TIMEOUT or MOE_ERR_INVALID_COUNTS (MOE_ERR_CUDA if the
+ * stream itself failed).
  * This is how device-side findings reach the host as the error codes of the NCCL EP page's table
  * ("NCCL EP架构解析", section 5.1: INVALID_TOPK for a routing index out of range, CUDA_ERROR for a
  * failed kernel).  It is the only call of the library that waits for the GPU.

@@ -162,3 +162,15 @@ def l2_flush_bytes() -> int:
     """Size of the scratch write that evicts the B200's 126 MB L2 between timed iterations."""
     return 256 * 1024 * 1024
 
+
+
+def make_ep_inputs(w: Workload, ranks: int, seed: int = 0, device: str = "cpu"):
+    """Inputs of an expert-parallel step over ``ranks`` ranks: every rank has its own T tokens
+    (``make_inputs`` with seed ``1000 * seed + 1 + rank``, weights left out) and the expert weights
+    are those of ``make_inputs(w, seed)``.  Returns ``{"logits": [per rank], "x": [per rank],
+    "w_gate", "w_up", "w_down"}``; rank r keeps experts [r*E/ranks, (r+1)*E/ranks) of the weights."""
+    full = make_inputs(w, seed=seed, device=device, weights=True)
+    per = [make_inputs(w, seed=1000 * seed + 1 + r, device=device, weights=False)
+           for r in range(ranks)]
+    return {"logits": [p["logits"] for p in per], "x": [p["x"] for p in per],
+            "w_gate": full["w_gate"], "w_up": full["w_up"], "w_down": full["w_down"]}

@@ -45,7 +45,8 @@ import numpy as np
 from .numerics import bf16_bits, bf16_from_bits, bf16_round, e4m3_decode, e4m3_encode_satfinite
 
 __all__ = ["capacity", "route", "dispatch_plan", "dispatch_payload", "expert_ffn", "combine",
-           "pipeline", "QBLOCK", "quantize_rows_fp8", "dequantize_rows_fp8", "expert_ffn_w8"]
+           "pipeline", "QBLOCK", "quantize_rows_fp8", "dequantize_rows_fp8", "expert_ffn_w8",
+           "ep_segment_rows", "ep_regroup", "ep_pipeline"]
 
 QBLOCK = 128   # elements per FP8 scale block
 E4M3_MAX_F32 = np.float32(448.0)
@@ -333,4 +334,100 @@ def pipeline(logits, x_bf16_bits, w_gate_bits, w_up_bits, w_down_bits, k: int, R
                h=h, expert_out=y_e)
     if ffn_rows is None:
         out["y"] = combine(y_e, plan["slot_row"], w, T, H)
+    return out
+
+
+# ---- expert parallelism across ranks ------------------------------------------------------------
+
+def ep_segment_rows(counts, order: int, stride: int):
+    """Row position of every row of a segmented layout: {(a, b, q): row}.
+
+    ``counts`` [A, B]: segment (a, b) holds counts[a][b] rows.  Order 0 (a-major): for a = 0..A-1,
+    for b = 0..B-1, the segment's rows in turn; block a (all of its b) starts at row a*stride, or
+    right after block a-1 when stride is 0.  Order 1 (b-major): the same with the roles of a and b
+    swapped (for b, for a).  This is the layout of a sender's per-destination blocks (the ThunderEP
+    page, section 2.1: one contiguous block per destination, expert-major inside) and of a
+    receiver's per-source blocks (the NCCL EP page, section 2.2: packed blocks in the high-throughput
+    mode, fixed-size per-peer blocks in the low-latency mode)."""
+    c = np.asarray(counts, dtype=np.int64)
+    A, B = c.shape
+    pos = {}
+    outer, inner = (A, B) if order == 0 else (B, A)
+    row = 0
+    for o in range(outer):
+        if stride > 0:
+            row = o * stride
+        for i in range(inner):
+            a, b = (o, i) if order == 0 else (i, o)
+            for q in range(int(c[a, b])):
+                pos[(a, b, q)] = row
+                row += 1
+    return pos
+
+
+def ep_regroup(counts, src, src_order: int, src_stride: int, dst, dst_order: int,
+               dst_stride: int):
+    """Move every row of every segment from its position in the source layout to its position in
+    the destination layout (``ep_segment_rows``); other rows of ``dst`` are left as they are.
+    Returns ``dst`` and the packed b-major start of every b (the total at [B])."""
+    c = np.asarray(counts, dtype=np.int64)
+    ps = ep_segment_rows(c, src_order, src_stride)
+    pd = ep_segment_rows(c, dst_order, dst_stride)
+    for key, r in ps.items():
+        dst[pd[key]] = src[r]
+    col = c.sum(axis=0)
+    offsets = np.zeros(c.shape[1] + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(col)
+    return dst, offsets
+
+
+def ep_pipeline(logits_ranks, x_ranks, w_gate_bits, w_up_bits, w_down_bits, k: int,
+                fp8: bool = False, renormalize: bool = True):
+    """The path with expert parallelism over R = len(logits_ranks) ranks, each with its own tokens.
+
+    Rank r owns experts [r*E/R, (r+1)*E/R).  Every rank routes its own tokens and packs its send
+    buffer for R destinations (``dispatch_plan`` with R); destination d receives, from every source
+    s in rank order, the rows of block d of s, expert-major over d's experts (the NCCL EP page,
+    sections 1 and 2: a dispatch exchange to the experts' owners); it regroups them expert-major and
+    runs the grouped FFN over its own experts; each output row goes back to the slot of its sender
+    that it came from (the combine exchange), and every rank combines its own tokens.
+    Returns the list of per-rank outputs y (bf16 bit patterns [T_r, H])."""
+    R = len(logits_ranks)
+    E = np.asarray(logits_ranks[0]).shape[1]
+    E_loc = E // R
+    per = []
+    for r in range(R):
+        idx, w, _ = route(logits_ranks[r], k, renormalize)
+        plan = dispatch_plan(idx, E, R, 0)
+        send, scales = dispatch_payload(x_ranks[r], plan, fp8)
+        per.append((idx, w, plan, send, scales))
+    H = per[0][3].shape[1]
+    back = [np.zeros((p[2]["S"], H), dtype=np.uint16) for p in per]
+    for d in range(R):
+        # counts[s][e]: rows source s sends to local expert e of rank d
+        counts = np.array([p[2]["expert_counts"][d * E_loc:(d + 1) * E_loc] for p in per])
+        blocks = [p[3][p[2]["rank_offsets"][d]:p[2]["rank_offsets"][d + 1]] for p in per]
+        recv = np.concatenate(blocks, axis=0)
+        grouped, off = ep_regroup(counts, recv, 0, 0, np.zeros_like(recv), 1, 0)
+        if fp8:
+            sblocks = [p[4][p[2]["rank_offsets"][d]:p[2]["rank_offsets"][d + 1]] for p in per]
+            rs = np.concatenate(sblocks, axis=0)
+            gs, _ = ep_regroup(counts, rs, 0, 0, np.zeros_like(rs), 1, 0)
+        else:
+            gs = None
+        xin = ffn_inputs(grouped, gs, fp8)
+        _, y_e = expert_ffn(xin, off, w_gate_bits[d * E_loc:(d + 1) * E_loc],
+                            w_up_bits[d * E_loc:(d + 1) * E_loc],
+                            w_down_bits[d * E_loc:(d + 1) * E_loc])
+        ret, _ = ep_regroup(counts, y_e, 1, 0, np.zeros_like(y_e), 0, 0)
+        # source s's rows sit at [sum of earlier sources' block sizes, ...) of ret
+        base = 0
+        for s, p in enumerate(per):
+            n = int(counts[s].sum())
+            lo = p[2]["rank_offsets"][d]
+            back[s][lo:lo + n] = ret[base:base + n]
+            base += n
+    out = []
+    for r, (idx, w, plan, _, _) in enumerate(per):
+        out.append(combine(back[r], plan["slot_row"], w, idx.shape[0], H))
     return out

@@ -182,3 +182,49 @@ def test_weight_list_calls_reject_bad_arguments(lib):
     assert ffn(H=200) == pkg.MOE_ERR_UNSUPPORTED
     assert ffn(payload=1) == pkg.MOE_ERR_INVALID_ARG                 # FP8 without scales
     assert ffn(ws_bytes=100) == pkg.MOE_ERR_WORKSPACE
+
+
+def _declared_prototypes():
+    """{name: (return type, [parameter types])} of every function declared in include/moe.h."""
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = {}
+    for m in re.finditer(r"([A-Za-z_][A-Za-z0-9_ \*]*?)\b(moe_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", src):
+        ret, name, params = m.group(1).strip(), m.group(2), m.group(3).strip()
+        if params in ("", "void"):
+            types = []
+        else:
+            types = []
+            for p in params.split(","):
+                p = " ".join(p.split())
+                # drop the parameter name: the last identifier
+                t = re.sub(r"\b[A-Za-z_][A-Za-z0-9_]*\s*$", "", p).strip()
+                types.append(t)
+        out[name] = (ret, types)
+    return out
+
+
+def _ctype_for(c_type: str):
+    import ctypes
+    if "*" in c_type or c_type == "moe_stream_t":
+        return ctypes.c_void_p
+    return {"int": ctypes.c_int, "size_t": ctypes.c_size_t, "double": ctypes.c_double,
+            "moe_payload_t": ctypes.c_int, "moe_status_t": ctypes.c_int}[c_type]
+
+
+def test_binding_signatures_match_the_header(lib):
+    """Every ctypes prototype of the binding has the header's parameter count and kinds: a
+    pointer passed where the table says int would be truncated to 32 bits."""
+    import ctypes
+    protos = _declared_prototypes()
+    assert set(protos) == set(declared_functions())
+    for name, (ret, types) in protos.items():
+        fn = getattr(lib, name)
+        assert fn.argtypes is not None, name
+        assert len(fn.argtypes) == len(types), (name, len(fn.argtypes), types)
+        for i, (got, t) in enumerate(zip(fn.argtypes, types)):
+            assert got == _ctype_for(t), (name, i, t, got)
+        if ret == "const char*":
+            assert fn.restype == ctypes.c_char_p, name
+        else:
+            assert fn.restype == _ctype_for(ret), (name, ret, fn.restype)

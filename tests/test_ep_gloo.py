@@ -1,0 +1,111 @@
+"""Expert parallelism over real process groups on CPU: gloo ranks run ``MoeEP`` (count exchange,
+split sizes, padded low-latency blocks, regrouping, the return trip) with oracle-backed local steps,
+and every rank's output must equal, bit for bit, its slice of the single-device oracle over all
+ranks' tokens."""
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import moe_inputs as mi
+from oracle import moe
+from oracle.numerics import bf16_bits
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+T_RANK = 40  # tokens per rank (the fp64 FFN stays quick)
+
+
+def _inputs(R, payload):
+    w = mi.get("tiny")
+    d = mi.make_ep_inputs(w, R, seed=5)
+    lg = [t[:T_RANK].contiguous() for t in d["logits"]]
+    xs = [t[:T_RANK].contiguous() for t in d["x"]]
+    # rank 0's tokens never pick the last rank's experts: a zero-row block in every exchange
+    E_loc = w.E // R
+    lg[0][:, w.E - E_loc:] -= 50.0
+    return w, lg, xs, d
+
+
+def _rank_main(rank, world, port, out):
+    from combine_moe_route_10_b200.ep import MoeEP, TorchComm
+    from _ep_oracle_ops import OracleOps
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        res = {}
+        for payload in ("bf16", "fp8"):
+            w, lg, xs, d = _inputs(world, payload)
+            E_loc = w.E // world
+            sl = slice(rank * E_loc, (rank + 1) * E_loc)
+            for mode, recv_rows in (("ht", 8), ("ll", None)):      # ht starts small and grows
+                ops = OracleOps()
+                ep = MoeEP(T_RANK, w.H, w.E, w.k, w.F, comm=TorchComm(), payload=payload,
+                           mode=mode, recv_rows=recv_rows, device="cpu", ops=ops)
+                for _ in range(2):                                  # a second step reuses buffers
+                    y = ep.forward(lg[rank], xs[rank], d["w_gate"][sl].contiguous(),
+                                   d["w_up"][sl].contiguous(), d["w_down"][sl].contiguous())
+                res[(payload, mode)] = (y.view(torch.int16).numpy().view(np.uint16).copy(),
+                                        ops.calls.count("regroup") // 2)
+        out[rank] = res
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_gloo_ranks_match_the_single_device_oracle(world):
+    port = _free_port()
+    with mp.get_context("spawn").Manager() as m:
+        out = m.dict()
+        mp.start_processes(_rank_main, args=(world, port, out), nprocs=world, join=True,
+                           start_method="spawn")
+        res = dict(out)
+    assert set(res) == set(range(world))
+    for payload in ("bf16", "fp8"):
+        w, lg, xs, d = _inputs(world, payload)
+        wb = [bf16_bits(d[key].float().numpy()) for key in ("w_gate", "w_up", "w_down")]
+        ref = moe.pipeline(np.concatenate([a.numpy() for a in lg]),
+                           np.concatenate([bf16_bits(a.float().numpy()) for a in xs]), *wb, w.k,
+                           world, fp8=payload == "fp8")["y"]
+        for mode, regroups in (("ht", 2), ("ll", 4)):
+            for r in range(world):
+                y, n_regroup = res[r][(payload, mode)]
+                assert n_regroup == regroups, (payload, mode)
+                assert np.array_equal(y, ref[r * T_RANK:(r + 1) * T_RANK]), (payload, mode, r)
+
+
+def test_thread_loopback_matches_the_oracle_too():
+    """The in-process R-rank emulation used by the single-GPU tests gives the same results."""
+    from combine_moe_route_10_b200.ep import MoeEP
+    from _ep_loopback import run_ranks
+    from _ep_oracle_ops import OracleOps
+    R = 4
+    w, lg, xs, d = _inputs(R, "bf16")
+    E_loc = w.E // R
+
+    def rank(r, comm):
+        sl = slice(r * E_loc, (r + 1) * E_loc)
+        out = {}
+        for mode in ("ht", "ll"):
+            ep = MoeEP(T_RANK, w.H, w.E, w.k, w.F, comm=comm, mode=mode, device="cpu",
+                       ops=OracleOps())
+            y = ep.forward(lg[r], xs[r], d["w_gate"][sl].contiguous(), d["w_up"][sl].contiguous(),
+                           d["w_down"][sl].contiguous())
+            out[mode] = y.view(torch.int16).numpy().view(np.uint16).copy()
+        return out
+
+    res = run_ranks(R, rank)
+    wb = [bf16_bits(d[key].float().numpy()) for key in ("w_gate", "w_up", "w_down")]
+    ref = moe.pipeline(np.concatenate([a.numpy() for a in lg]),
+                       np.concatenate([bf16_bits(a.float().numpy()) for a in xs]), *wb, w.k, R)["y"]
+    for r in range(R):
+        for mode in ("ht", "ll"):
+            assert np.array_equal(res[r][mode], ref[r * T_RANK:(r + 1) * T_RANK]), (mode, r)
