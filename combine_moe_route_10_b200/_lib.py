@@ -19,6 +19,8 @@ MOE_ERR_CUDA = 4
 MOE_ERR_WORKSPACE = 5
 MOE_ERR_TIMEOUT = 6
 MOE_ERR_INVALID_COUNTS = 7
+MOE_EP_PULL = 0
+MOE_EP_PUSH = 1
 MOE_PAYLOAD_BF16 = 0
 MOE_PAYLOAD_FP8_E4M3_B128 = 1
 
@@ -27,7 +29,7 @@ EXPORTS = ["moe_abi_version", "moe_status_string", "moe_capacity", "moe_route",
            "moe_ffn_workspace_size",
            "moe_expert_ffn", "moe_ffn_weight_list_bytes", "moe_ffn_weight_list_init",
            "moe_expert_ffn_list", "moe_quantize_rows_fp8", "moe_ffn_w8_workspace_size",
-           "moe_expert_ffn_w8", "moe_ep_regroup", "moe_combine", "moe_sync_status"]
+           "moe_expert_ffn_w8", "moe_ep_regroup", "moe_ep_exchange", "moe_combine", "moe_sync_status"]
 
 _lib = None
 
@@ -65,6 +67,7 @@ def load() -> ctypes.CDLL:
         "moe_ffn_w8_workspace_size": (Z, [I, I, I, I, I]),
         "moe_expert_ffn_w8": (I, [P, P, I, P, I, I, I, I, P, P, P, P, P, P, P, Z, P]),
         "moe_ep_regroup": (I, [P, I, I, I, I, I, I, I, I, P, P, Z, P, P, Z, P, P, P]),
+        "moe_ep_exchange": (I, [P, I, I, I, I, P, P, I, P, P, I, Z, Z, P, P, P]),
         "moe_combine": (I, [P, I, P, P, I, I, I, P, P, P]),
         "moe_sync_status": (I, [P, P]),
     }
@@ -209,6 +212,16 @@ def moe_ep_regroup(counts, A, B, src_order, src_stride, src_rows, dst_order, dst
                                _ptr(src_aux), _ptr(dst_aux), aux_row_bytes, _ptr(dst_offsets),
                                _ptr(status), _stream(stream))
     return _check(st, "moe_ep_regroup", raise_on_error)
+
+
+def moe_ep_exchange(all_counts, R, E, rank, direction, peer_rows, peer_aux, peer_rows_cap,
+                    local_rows, local_aux, local_rows_cap, row_bytes, aux_row_bytes=0,
+                    local_offsets=None, status=None, stream=None, raise_on_error=True):
+    st = load().moe_ep_exchange(_ptr(all_counts), R, E, rank, direction, _ptr(peer_rows),
+                                _ptr(peer_aux), peer_rows_cap, _ptr(local_rows), _ptr(local_aux),
+                                local_rows_cap, row_bytes, aux_row_bytes, _ptr(local_offsets),
+                                _ptr(status), _stream(stream))
+    return _check(st, "moe_ep_exchange", raise_on_error)
 
 
 def moe_combine(expert_out, max_rows, slot_row, topk_w, T, k, H, y, status=None, stream=None,

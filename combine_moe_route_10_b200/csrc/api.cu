@@ -259,6 +259,33 @@ moe_status_t moe_ep_regroup(const int32_t* counts, int A, int B, int src_order, 
       reinterpret_cast<cudaStream_t>(stream)));
 }
 
+moe_status_t moe_ep_exchange(const int32_t* all_counts, int R, int E, int rank, int direction,
+                             const uint64_t* peer_rows, const uint64_t* peer_aux,
+                             int peer_rows_cap, void* local_rows, void* local_aux,
+                             int local_rows_cap, size_t row_bytes, size_t aux_row_bytes,
+                             int32_t* local_offsets, int32_t* status, moe_stream_t stream) {
+  if (R < 1 || R > moe::kMaxEpRanks || E < R || E % R != 0 || E > moe::kMaxRegroupSegments)
+    return MOE_ERR_INVALID_ARG;
+  if (rank < 0 || rank >= R || (direction != MOE_EP_PULL && direction != MOE_EP_PUSH))
+    return MOE_ERR_INVALID_ARG;
+  if (peer_rows_cap < 0 || local_rows_cap < 0) return MOE_ERR_INVALID_ARG;
+  if (all_counts == nullptr || peer_rows == nullptr || local_rows == nullptr ||
+      !aligned(all_counts, 4) || !aligned(peer_rows, 8) || !aligned(local_rows, 4) ||
+      !aligned(status, 4) || !aligned(local_offsets, 4))
+    return MOE_ERR_INVALID_ARG;
+  if (row_bytes == 0 || row_bytes % 4 != 0) return MOE_ERR_INVALID_ARG;
+  if (aux_row_bytes != 0 && (aux_row_bytes % 4 != 0 || peer_aux == nullptr ||
+                             local_aux == nullptr || !aligned(peer_aux, 8) ||
+                             !aligned(local_aux, 4)))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_ep_exchange(
+      all_counts, R, E, rank, direction == MOE_EP_PUSH ? 1 : 0,
+      reinterpret_cast<const unsigned long long*>(peer_rows),
+      reinterpret_cast<const unsigned long long*>(peer_aux), peer_rows_cap, local_rows,
+      aux_row_bytes ? local_aux : nullptr, local_rows_cap, row_bytes, aux_row_bytes, local_offsets,
+      reinterpret_cast<int*>(status), reinterpret_cast<cudaStream_t>(stream)));
+}
+
 moe_status_t moe_combine(const void* expert_out, int max_rows, const int32_t* slot_row,
                          const float* topk_w, int T, int k, int H, void* y, int32_t* status,
                          moe_stream_t stream) {

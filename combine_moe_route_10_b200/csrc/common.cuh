@@ -12,8 +12,10 @@ constexpr int kStatusInvalidTopk = 1;  // an expert id outside [0, E) was seen
 constexpr int kStatusTimeout = 2;      // a bounded pipeline wait ran out
 constexpr int kStatusBadCounts = 4;    // exchanged row counts do not fit the buffers they describe
 
-// Largest count matrix (segments) the expert-parallel regrouping takes.
+// Largest count matrix (segments) the expert-parallel regrouping and exchange take, and the most
+// ranks of an exchange.
 constexpr int kMaxRegroupSegments = 4096;
+constexpr int kMaxEpRanks = 1024;
 
 // Bound on any single device-side wait (ns of %globaltimer).  A healthy wait in these kernels is
 // microseconds; one second means something upstream is broken, and the kernel gives up cleanly.

@@ -20,19 +20,19 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / kWarp;
 constexpr int kItems = kMaxRegroupSegments / kThreads;  // scan items per thread
 
-// Exclusive scan of n <= kMaxRegroupSegments counts, read in the order item(i), into out[item(i)]
-// (out[n] = total); items past n read as 0.  All threads of the CTA take part.  The sums are taken
-// in 64 bits: a negative count, a count above `limit`, or a total above `limit` sets `bad` (the
-// stored starts are then meaningless and must not be used).
-template <typename Item>
-__device__ void block_scan(const int32_t* __restrict__ counts, int n, Item item, long long limit,
-                           int* out, long long* warp_tot, bool& bad) {
+// Exclusive scan of n <= kMaxRegroupSegments counts: item i reads counts[read(i)] and its exclusive
+// prefix goes to out[slot(i)] (out[n] = total); items past n read as 0.  All threads of the CTA take
+// part.  The sums are taken in 64 bits: a negative count, a count above `limit`, or a total above
+// `limit` sets `bad` (the stored starts are then meaningless and must not be used).
+template <typename Read, typename Slot>
+__device__ void block_scan(const int32_t* __restrict__ counts, int n, Read read, Slot slot,
+                           long long limit, int* out, long long* warp_tot, bool& bad) {
   long long v[kItems];
   long long run = 0;
 #pragma unroll
   for (int i = 0; i < kItems; ++i) {
     const int j = threadIdx.x * kItems + i;
-    long long c = j < n ? __ldg(counts + item(j)) : 0;
+    long long c = j < n ? __ldg(counts + read(j)) : 0;
     if (c < 0 || c > limit) { bad = true; c = 0; }
     v[i] = run;
     run += c;
@@ -52,7 +52,7 @@ __device__ void block_scan(const int32_t* __restrict__ counts, int n, Item item,
 #pragma unroll
   for (int i = 0; i < kItems; ++i) {
     const int j = threadIdx.x * kItems + i;
-    if (j < n) out[item(j)] = static_cast<int>(base + v[i]);
+    if (j < n) out[slot(j)] = static_cast<int>(base + v[i]);
   }
   if (threadIdx.x == kThreads - 1) {
     if (base + run > limit) bad = true;
@@ -98,6 +98,11 @@ __device__ __forceinline__ void copy_row(const unsigned char* __restrict__ src,
   for (; i < n; i += kWarp) __stcs(d + i, __ldcs(s + i));
 }
 
+__host__ __device__ __forceinline__ bool vec16_ok(const void* a, const void* b, size_t bytes) {
+  return bytes % 16 == 0 && reinterpret_cast<uintptr_t>(a) % 16 == 0 &&
+         reinterpret_cast<uintptr_t>(b) % 16 == 0;
+}
+
 struct Payload {
   const unsigned char* src;
   unsigned char* dst;
@@ -121,9 +126,11 @@ __global__ void __launch_bounds__(kThreads)
   bool bad = false;
   // no segment and no total can exceed the smaller buffer
   const long long limit = src_side.rows < dst_side.rows ? src_side.rows : dst_side.rows;
-  block_scan(counts, n, [](int j) { return j; }, limit, am, warp_tot, bad);
+  const auto same = [](int j) { return j; };
+  block_scan(counts, n, same, same, limit, am, warp_tot, bad);
   // b-major order visits (a, b) as j = b*A + a
-  block_scan(counts, n, [A, B](int j) { return (j % A) * B + j / A; }, limit, bm, warp_tot, bad);
+  const auto transposed = [A, B](int j) { return (j % A) * B + j / A; };
+  block_scan(counts, n, transposed, transposed, limit, bm, warp_tot, bad);
   if (bad) s_bad = 1;
   __syncthreads();
   if (s_bad) {
@@ -178,12 +185,119 @@ __global__ void __launch_bounds__(kThreads)
   if (oob && lane == 0) record_status(status, kStatusBadCounts);
 }
 
-bool vec16_ok(const void* a, const void* b, size_t bytes) {
-  return bytes % 16 == 0 && reinterpret_cast<uintptr_t>(a) % 16 == 0 &&
-         reinterpret_cast<uintptr_t>(b) % 16 == 0;
+// ---- the exchange over peer memory -------------------------------------------------------------
+//
+// Rank `rank` of R owns experts [rank*E_loc, (rank+1)*E_loc).  all_counts [R, E] holds every rank's
+// expert_counts (the dispatch's kept rows per expert), so source s's rows for this rank's expert e
+// sit in s's packed expert-major buffer from row  sum_{e' < rank*E_loc + e} all_counts[s][e']  on.
+// Pull: every such row is read from the source's buffer (a peer pointer) and written expert-major
+// into this rank's buffer (b-major over (s, e), packed), with the local expert offsets.  Push: the
+// reverse, from this rank's expert-major buffer into every source's buffer at the same positions.
+
+__global__ void __launch_bounds__(kThreads)
+    ep_exchange_kernel(const int32_t* __restrict__ all_counts, int R, int E, int rank, int E_loc,
+                       int push, const unsigned long long* __restrict__ peer_rows,
+                       const unsigned long long* __restrict__ peer_aux, int peer_cap,
+                       unsigned char* __restrict__ local_rows, unsigned char* __restrict__ local_aux,
+                       int local_cap, size_t row_bytes, size_t aux_bytes,
+                       int32_t* __restrict__ local_offsets, int* status) {
+  __shared__ int am[kMaxRegroupSegments + 1];  // packed (s, e) starts, s-major
+  __shared__ int bm[kMaxRegroupSegments + 1];  // packed (s, e) starts, e-major; bm[e] starts expert e
+  __shared__ long long block0[kMaxEpRanks];      // first row of this rank's block in source s
+  __shared__ long long warp_tot[kWarps];
+  __shared__ int s_bad;
+  griddep_wait();
+  griddep_launch_dependents();
+  const int n = R * E_loc;
+  const int e0 = rank * E_loc;
+  if (threadIdx.x == 0) s_bad = 0;
+  bool bad = false;
+  // the rows received from all sources fill this rank's buffer; each source's block is checked
+  // against the peer capacity below
+  const long long limit = local_cap;
+  const auto read_s_major = [E, E_loc, e0](int j) { return (j / E_loc) * E + e0 + j % E_loc; };
+  const auto same = [](int j) { return j; };
+  block_scan(all_counts, n, read_s_major, same, limit, am, warp_tot, bad);
+  // e-major order visits (s, e) as j = e*R + s
+  const auto read_e_major = [R, E, e0](int j) { return (j % R) * E + e0 + j / R; };
+  const auto slot_e_major = [R, E_loc](int j) { return (j % R) * E_loc + j / R; };
+  block_scan(all_counts, n, read_e_major, slot_e_major, limit, bm, warp_tot, bad);
+  // block starts: one warp per source sums the counts of the experts before this rank's
+  const int lane = threadIdx.x % kWarp, warp = threadIdx.x / kWarp;
+  for (int src = warp; src < R; src += kWarps) {
+    long long sum = 0;
+    for (int e = lane; e < e0; e += kWarp) {
+      const long long c = __ldg(all_counts + static_cast<long long>(src) * E + e);
+      if (c < 0) bad = true;
+      sum += c;
+    }
+#pragma unroll
+    for (int d = kWarp / 2; d > 0; d >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, d);
+    if (lane == 0) block0[src] = sum;
+  }
+  if (bad) s_bad = 1;
+  __syncthreads();
+  // this rank's block of every source must lie inside the source's buffer
+  for (int src = threadIdx.x; src < R; src += kThreads) {
+    const long long len = am[(src + 1) * E_loc] - am[src * E_loc];
+    if (block0[src] + len > peer_cap) s_bad = 1;
+  }
+  __syncthreads();
+  const int total = am[n];
+  if (s_bad) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) record_status(status, kStatusBadCounts);
+    return;
+  }
+  if (local_offsets != nullptr && blockIdx.x == 0) {
+    for (int e = threadIdx.x; e <= E_loc; e += kThreads) local_offsets[e] = e < E_loc ? bm[e] : total;
+  }
+  for (int r = blockIdx.x * kWarps + warp; r < total; r += gridDim.x * kWarps) {
+    int lo = 0, hi = n - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (am[mid] <= r) lo = mid; else hi = mid - 1;
+    }
+    const int src = lo / E_loc, q = r - am[lo];
+    const long long pp = block0[src] + (am[lo] - am[src * E_loc]) + q;  // row in the peer's buffer
+    const long long pl = static_cast<long long>(bm[lo]) + q;             // row in this rank's
+    unsigned char* peer = reinterpret_cast<unsigned char*>(peer_rows[src]);
+    const unsigned char* from = push ? local_rows + pl * row_bytes : peer + pp * row_bytes;
+    unsigned char* to = push ? peer + pp * row_bytes : local_rows + pl * row_bytes;
+    if (vec16_ok(from, to, row_bytes)) copy_row<uint4>(from, to, row_bytes, lane);
+    else copy_row<uint32_t>(from, to, row_bytes, lane);
+    if (aux_bytes != 0) {
+      unsigned char* pa = reinterpret_cast<unsigned char*>(peer_aux[src]);
+      const unsigned char* af = push ? local_aux + pl * aux_bytes : pa + pp * aux_bytes;
+      unsigned char* at = push ? pa + pp * aux_bytes : local_aux + pl * aux_bytes;
+      if (vec16_ok(af, at, aux_bytes)) copy_row<uint4>(af, at, aux_bytes, lane);
+      else copy_row<uint32_t>(af, at, aux_bytes, lane);
+    }
+  }
+  // stores into other GPUs' memory: make them visible system-wide before this grid completes
+  if (push) __threadfence_system();
 }
 
+
+
 }  // namespace
+
+cudaError_t launch_ep_exchange(const int32_t* all_counts, int R, int E, int rank, int push,
+                               const unsigned long long* peer_rows,
+                               const unsigned long long* peer_aux, int peer_cap, void* local_rows,
+                               void* local_aux, int local_cap, size_t row_bytes, size_t aux_bytes,
+                               int32_t* local_offsets, int* status, cudaStream_t s) {
+  const int E_loc = E / R;
+  long long blocks = (static_cast<long long>(local_cap) + kWarps - 1) / kWarps;
+  if (blocks > 2LL * num_sms()) blocks = 2LL * num_sms();
+  if (blocks < 1) blocks = 1;
+  const cudaError_t err = launch_pdl(
+      ep_exchange_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0, s, all_counts, R,
+      E, rank, E_loc, push, peer_rows, aux_bytes ? peer_aux : nullptr, peer_cap,
+      static_cast<unsigned char*>(local_rows), static_cast<unsigned char*>(local_aux), local_cap,
+      row_bytes, aux_bytes, local_offsets, status);
+  if (err != cudaSuccess) return err;
+  return cudaGetLastError();
+}
 
 cudaError_t launch_ep_regroup(const int32_t* counts, int A, int B, int src_order, int src_stride,
                               int src_rows, int dst_order, int dst_stride, int dst_rows,

@@ -92,6 +92,13 @@ cudaError_t ffn_weight_list_init(const void* const* w_gate, const void* const* w
                                  const void* const* w_down, int E, int H, int F, void* list,
                                  cudaStream_t s);
 
+// Rows between this rank's expert-major buffer and every source's packed buffer (peer pointers).
+cudaError_t launch_ep_exchange(const int32_t* all_counts, int R, int E, int rank, int push,
+                               const unsigned long long* peer_rows,
+                               const unsigned long long* peer_aux, int peer_cap, void* local_rows,
+                               void* local_aux, int local_cap, size_t row_bytes, size_t aux_bytes,
+                               int32_t* local_offsets, int* status, cudaStream_t s);
+
 // Segmented row copy between the layouts on the two sides of an expert-parallel all-to-all.
 cudaError_t launch_ep_regroup(const int32_t* counts, int A, int B, int src_order, int src_stride,
                               int src_rows, int dst_order, int dst_stride, int dst_rows,

@@ -26,6 +26,18 @@ Two exchange modes (the NCCL EP page, section 2.2):
     splits: no host synchronisation, and a whole step can be captured in a CUDA graph.  The padding
     is one more regroup on each side.
 
+A third mode moves the rows over peer memory instead of through all-to-alls (the NCCL EP page,
+section 1: kernels that load and store other GPUs' memory over NVLink; section 2.1: the dispatch
+delivers each token to its expert owner's buffer and the combine reads the outputs back):
+  * ``"p2p"``: the send and return buffers of every rank are mapped into every other rank
+    (``comm.alloc_shared``: torch symmetric memory between GPUs).  After the dispatch, one
+    all-gather of the [E] counts gives every rank the whole [R, E] count matrix (and orders it after
+    every rank's dispatch); ``moe_ep_exchange`` then pulls each rank's rows from the sources' send
+    buffers straight into its expert-major FFN input (exchange and regroup in one kernel), and after
+    the FFN pushes the outputs straight into the sources' return buffers; a stream-ordered barrier
+    later, every rank combines.  No row passes through a staging buffer, no host synchronisation,
+    and the step can be captured in a CUDA graph.
+
 Every row of a token meets the same kernels as on a single device: the received rows of expert e
 are ordered by (source rank, source token), which is the single-device dispatch order over the
 rank-major concatenation of all ranks' tokens, so the FFN and the combine see identical operands,
@@ -82,22 +94,62 @@ class CudaOps:
     def combine(self, expert_out, max_rows, slot_row, topk_w, T, k, H, y):
         _lib.moe_combine(expert_out, max_rows, slot_row, topk_w, T, k, H, y, None)
 
+    def peer_table(self, tensors):
+        return torch.tensor([t.data_ptr() for t in tensors], dtype=torch.int64).to(self.device)
+
+    def exchange(self, all_counts, R, E, rank, direction, peer_rows, peer_aux, peer_cap, local,
+                 local_aux, local_offsets=None, status=None):
+        _lib.moe_ep_exchange(all_counts, R, E, rank, direction, peer_rows, peer_aux, peer_cap,
+                             local, local_aux, local.shape[0],
+                             local[0].numel() * local.element_size(),
+                             0 if local_aux is None else local_aux[0].numel() * local_aux.element_size(),
+                             local_offsets, status)
+
     def sync_status(self, ws) -> int:
         return _lib.moe_sync_status(ws)
 
 
 class TorchComm:
     """The exchange over a ``torch.distributed`` process group (NCCL over NVLink between GPUs;
-    gloo on CPU): ``all_to_all(out, inp, out_splits, in_splits)`` splits along dim 0, equal splits
-    when the lists are None."""
+    gloo on CPU).
 
-    def __init__(self, group=None):
+    ``all_to_all(out, inp, out_splits, in_splits)`` splits along dim 0 (equal splits when the lists
+    are None); ``all_gather(out, inp)`` concatenates every rank's ``inp`` in rank order;
+    ``barrier()`` is a one-element all-reduce, ordered on the current stream like any collective;
+    ``alloc_shared(shape, dtype, device)`` returns this rank's buffer and every rank's buffer as
+    mapped on this GPU (torch symmetric memory; with one rank and ``symmetric`` False, a plain
+    allocation)."""
+
+    def __init__(self, group=None, symmetric: bool = False):
         self.group = group
         self.rank = dist.get_rank(group)
         self.size = dist.get_world_size(group)
+        self.symmetric = symmetric
+        self._handles = []
+        self._one = None
 
     def all_to_all(self, out, inp, out_splits=None, in_splits=None):
         dist.all_to_all_single(out, inp, out_splits, in_splits, group=self.group)
+
+    def all_gather(self, out, inp):
+        dist.all_gather_into_tensor(out, inp, group=self.group)
+
+    def barrier(self, device):
+        if self._one is None:
+            self._one = torch.zeros(1, dtype=torch.int32, device=device)
+        dist.all_reduce(self._one, group=self.group)
+
+    def alloc_shared(self, shape, dtype, device):
+        if self.size == 1 and not self.symmetric:
+            t = torch.empty(shape, dtype=dtype, device=device)
+            return t, [t]
+        if torch.device(device).type != "cuda":
+            raise NotImplementedError("peer buffers need CUDA devices")
+        import torch.distributed._symmetric_memory as symm_mem
+        t = symm_mem.empty(*shape, dtype=dtype, device=device)
+        h = symm_mem.rendezvous(t, self.group if self.group is not None else dist.group.WORLD)
+        self._handles.append(h)  # keeps the peer mappings alive
+        return t, [h.get_buffer(r, tuple(shape), dtype) for r in range(self.size)]
 
 
 def _rows_as_bytes(t: torch.Tensor) -> torch.Tensor:
@@ -120,8 +172,8 @@ class MoeEP:
     def __init__(self, T: int, H: int, E: int, k: int, F: int, comm=None, payload: str = "bf16",
                  mode: str = "ht", renormalize: bool = True, recv_rows: int | None = None,
                  device="cuda", ops=None):
-        if mode not in ("ht", "ll"):
-            raise ValueError("mode must be 'ht' or 'll'")
+        if mode not in ("ht", "ll", "p2p"):
+            raise ValueError("mode must be 'ht', 'll' or 'p2p'")
         if payload not in ("bf16", "fp8"):
             raise ValueError("payload must be 'bf16' or 'fp8'")
         self.comm = TorchComm() if comm is None else comm
@@ -148,15 +200,28 @@ class MoeEP:
         # local side: route, dispatch, combine on this rank's tokens
         self.topk_idx = torch.empty((T, k), **i32)
         self.topk_w = torch.empty((T, k), dtype=torch.float32, device=dev)
-        self.send = torch.empty((S, H), dtype=self.row_dtype, device=dev)
-        self.send_scales = torch.empty((S, self.nb), dtype=torch.float32, device=dev) \
-            if self.fp8 else None
+        if mode == "p2p":
+            # every rank's send and return buffers, as mapped on this GPU
+            self.send, peers = self.comm.alloc_shared((max(S, 1), H), self.row_dtype, dev)
+            self.peer_send = self._pointers(peers)
+            self.send_scales, self.peer_send_scales = None, None
+            if self.fp8:
+                self.send_scales, peers = self.comm.alloc_shared((max(S, 1), self.nb),
+                                                                 torch.float32, dev)
+                self.peer_send_scales = self._pointers(peers)
+            self.ret, peers = self.comm.alloc_shared((max(S, 1), H), torch.bfloat16, dev)
+            self.peer_ret = self._pointers(peers)
+            self.all_counts = torch.empty(self.R * E, **i32)
+        else:
+            self.send = torch.empty((S, H), dtype=self.row_dtype, device=dev)
+            self.send_scales = torch.empty((S, self.nb), dtype=torch.float32, device=dev) \
+                if self.fp8 else None
+            self.ret = torch.empty((S, H), dtype=torch.bfloat16, device=dev)  # returned rows
         self.expert_counts = torch.empty(E, **i32)
         self.expert_offsets = torch.empty(E + 1, **i32)
         self.rank_offsets = torch.empty(self.R + 1, **i32)
         self.slot_row = torch.empty((T, k), **i32)
         self.row_token = torch.empty(max(S, 1), **i32)
-        self.ret = torch.empty((S, H), dtype=torch.bfloat16, device=dev)  # returned FFN rows
         self.y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
         self.ws_dispatch = self.ops.workspace(_lib.moe_dispatch_workspace_size(T, E, k))
         # the status word of the regroups (counts from other ranks are checked on the device)
@@ -164,7 +229,9 @@ class MoeEP:
         # expert side
         self.recv_counts = torch.empty(self.R * self.E_loc, **i32)
         self.local_offsets = torch.empty(self.E_loc + 1, **i32)
-        if mode == "ll":
+        if mode == "p2p":
+            self._alloc_expert_side(self.R * self.M)
+        elif mode == "ll":
             P = self.R * self.M
             self.send_pad = torch.empty((P, H), dtype=self.row_dtype, device=dev)
             self.send_pad_scales = torch.empty((P, self.nb), dtype=torch.float32, device=dev) \
@@ -189,6 +256,11 @@ class MoeEP:
         self.back = torch.empty((rows, H), dtype=torch.bfloat16, device=dev)
         self.ws_ffn = self.ops.workspace(
             _lib.moe_ffn_workspace_size(rows, self.E_loc, H, self.F, self.payload))
+
+    def _pointers(self, tensors):
+        """The buffers as the exchange step takes them (``ops.peer_table``: for the CUDA library,
+        a device array of their addresses, int64 [R])."""
+        return self.ops.peer_table(tensors)
 
     # -- the exchange -------------------------------------------------------------------------
     def _all_to_all(self, out, inp, out_splits=None, in_splits=None):
@@ -223,9 +295,11 @@ class MoeEP:
         ops.dispatch(x, T, H, self.topk_idx, k, E, R, self.payload, self.send, self.send_scales,
                      self.expert_counts, self.expert_offsets, self.rank_offsets, self.slot_row,
                      self.row_token, self.ws_dispatch)
+        st = self.ws_regroup
+        if self.mode == "p2p":
+            return self._forward_p2p(w_gate, w_up, w_down, st)
         # counts: expert_counts is [R destinations, E_loc] already
         self._all_to_all(self.recv_counts, self.expert_counts)
-        st = self.ws_regroup
         if self.mode == "ht":
             send_splits, recv_splits = self._ht_sizes()
             n_recv = sum(recv_splits)
@@ -259,6 +333,24 @@ class MoeEP:
             ops.regroup(self.expert_counts, R, E_loc, A_MAJOR, self.M, self.ret_pad, A_MAJOR, 0,
                         self.ret, None, None, None, st)
         ops.combine(self.ret, self.ret.shape[0], self.slot_row, self.topk_w, T, k, H, self.y)
+        return self.y
+
+    def _forward_p2p(self, w_gate, w_up, w_down, st):
+        T, H, E, k, R = self.T, self.H, self.E, self.k, self.R
+        ops, S = self.ops, self.send.shape[0]
+        # the whole [R, E] count matrix; as a collective it also follows every rank's dispatch
+        self.comm.all_gather(self.all_counts, self.expert_counts)
+        ops.exchange(self.all_counts, R, E, self.rank, _lib.MOE_EP_PULL, self.peer_send,
+                     self.peer_send_scales, S, self.grouped, self.grouped_scales,
+                     self.local_offsets, st)
+        ops.expert_ffn(self.grouped, self.grouped_scales, self.payload, self.local_offsets,
+                       self.cap, self.E_loc, H, self.F, w_gate, w_up, w_down, self.expert_out,
+                       self.ws_ffn)
+        ops.exchange(self.all_counts, R, E, self.rank, _lib.MOE_EP_PUSH, self.peer_ret, None, S,
+                     self.expert_out, None, None, st)
+        # every rank's pushes into this rank's return buffer are complete after the barrier
+        self.comm.barrier(self.device)
+        ops.combine(self.ret, S, self.slot_row, self.topk_w, T, k, H, self.y)
         return self.y
 
     def status(self) -> int:

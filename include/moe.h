@@ -320,6 +320,44 @@ moe_status_t moe_ep_regroup(const int32_t* counts, int A, int B, int src_order, 
                             int32_t* status, moe_stream_t stream);
 
 /*
+ * moe_ep_exchange: the expert-parallel exchange over peer memory, fused with the regrouping: one
+ * kernel moves every row between this rank's expert-major buffer and the other ranks' packed
+ * buffers, reading (pull) or writing (push) the other GPUs' memory directly over NVLink (the NCCL
+ * EP page, section 1: kernels that load and store peer memory over NVLink in place of staged
+ * copies; section 2.1: the dispatch writes each token into the expert owner's receive buffer and
+ * the combine reads the outputs back).
+ *
+ * Rank `rank` of R owns experts [rank*E_loc, (rank+1)*E_loc), E_loc = E / R.  all_counts [R, E]
+ * int32 (device, this rank's copy, e.g. from an all-gather) holds every rank's expert_counts from
+ * its moe_dispatch; source s's packed expert-major buffer then holds the rows for this rank's
+ * expert e from row  sum_{e' < rank*E_loc + e} all_counts[s][e']  on.  peer_rows [R] (device, 64-bit
+ * addresses) holds the base of every rank's packed buffer as this GPU sees it (its own buffer for
+ * s = rank, peer mappings for the others); peer_aux [R] likewise for the second payload (the FP8
+ * block scales; NULL when aux_row_bytes is 0).
+ *   MOE_EP_PULL: rows move from the sources' buffers into local_rows, expert-major over this rank's
+ *                experts and, within an expert, source-major (packed); local_offsets [E_loc + 1]
+ *                (may be NULL) gets the expert offsets for moe_expert_ffn;
+ *   MOE_EP_PUSH: the reverse (local_rows expert-major into every source's buffer at the same
+ *                positions), e.g. the FFN outputs into each source's combine input.  The kernel
+ *                ends with a system-scope fence, so its stores are visible to the other GPUs once
+ *                it has completed.
+ * The caller orders the exchange against the other ranks: the sources' buffers must be complete
+ * before a pull (e.g. a stream-ordered collective after every rank's dispatch) and the pushes of
+ * every rank must be complete before a source reads its buffer.  peer_rows_cap / local_rows_cap are
+ * the row capacities of every peer buffer and of local_rows; a negative count, or a block or total
+ * that does not fit them, copies nothing and records MOE_ERR_INVALID_COUNTS in *status (may be
+ * NULL).  Rows move with 16-byte vectors when sizes and addresses allow, else 4-byte words.
+ * Limits: R <= 1024, E <= 4096, E % R == 0, row_bytes and aux_row_bytes multiples of 4.
+ */
+#define MOE_EP_PULL 0
+#define MOE_EP_PUSH 1
+moe_status_t moe_ep_exchange(const int32_t* all_counts, int R, int E, int rank, int direction,
+                             const uint64_t* peer_rows, const uint64_t* peer_aux,
+                             int peer_rows_cap, void* local_rows, void* local_aux,
+                             int local_rows_cap, size_t row_bytes, size_t aux_row_bytes,
+                             int32_t* local_offsets, int32_t* status, moe_stream_t stream);
+
+/*
  * Synchronise `stream`, read the device status word at the start of a dispatch or FFN workspace
  * (or any status word given to moe_combine / moe_dispatch_noalloc), clear it, and report it:
  * MOE_OK, MOE_ERR_INVALID_TOPK, MOE_ERR_TIMEOUT or MOE_ERR_INVALID_COUNTS (MOE_ERR_CUDA if the

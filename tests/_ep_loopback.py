@@ -1,13 +1,16 @@
 """R expert-parallel ranks in one process, one thread per rank (test infrastructure).
 
-``LoopbackComm`` implements the all-to-all of ``MoeEP`` (split along dim 0, block s of the output
-from source s) by copying between the ranks' tensors: every rank deposits its input, waits for all
-ranks on a host barrier, copies its blocks from every source, and waits again before its input can
-be overwritten.  On one GPU, all threads issue their work to the same (default) stream, so the
+``LoopbackComm`` implements the collectives of ``MoeEP`` by copying between the ranks' tensors:
+for the all-to-all (split along dim 0, block s of the output from source s) and the all-gather,
+every rank deposits its input, waits for all ranks on a host barrier, copies from every source, and
+waits again before its input can be overwritten; ``alloc_shared`` hands every rank the other ranks'
+buffers themselves (one address space: the peer-memory exchange reads and writes them directly).  On one GPU, all threads issue their work to the same (default) stream, so the
 copies run after every rank's producing kernels and before any later overwrite: no kernel ever
 waits on another.
 """
 import threading
+
+import torch
 
 
 class LoopbackHub:
@@ -36,6 +39,29 @@ class LoopbackComm:
             out[pos:pos + n].copy_(src[lo:lo + n])
             pos += n
         hub.barrier.wait()
+
+
+    def all_gather(self, out, inp):
+        hub, R = self.hub, self.hub.R
+        hub.slots[self.rank] = inp
+        hub.barrier.wait()
+        n = inp.shape[0]
+        for s in range(R):
+            out[s * n:(s + 1) * n].copy_(hub.slots[s])
+        hub.barrier.wait()
+
+    def barrier(self, device=None):
+        self.hub.barrier.wait()
+
+    def alloc_shared(self, shape, dtype, device):
+        """Every rank allocates its own buffer; all ranks see all of them (one address space)."""
+        hub = self.hub
+        t = torch.empty(shape, dtype=dtype, device=device)
+        hub.slots[self.rank] = t
+        hub.barrier.wait()
+        peers = list(hub.slots)
+        hub.barrier.wait()
+        return t, peers
 
 
 def run_ranks(R: int, fn):

@@ -62,6 +62,37 @@ class OracleOps:
         if dst_offsets is not None:
             dst_offsets.copy_(torch.from_numpy(off.astype(np.int32)))
 
+    def peer_table(self, tensors):
+        return list(tensors)
+
+    def exchange(self, all_counts, R, E, rank, direction, peer_rows, peer_aux, peer_cap, local,
+                 local_aux, local_offsets=None, status=None):
+        """Peer-memory exchange on CPU: ``peer_rows`` / ``peer_aux`` are the ranks' tensors."""
+        self.calls.append("exchange")
+        E_loc = E // R
+        C = all_counts.numpy().reshape(R, E).astype(np.int64)
+        mine = C[:, rank * E_loc:(rank + 1) * E_loc]
+        starts = [int(C[s, :rank * E_loc].sum()) for s in range(R)]
+        lens = [int(mine[s].sum()) for s in range(R)]
+        n = sum(lens)
+        for peers, loc in ((peer_rows, local), (peer_aux, local_aux)):
+            if peers is None or loc is None:
+                continue
+            lb = _bytes(loc)
+            if direction == 0:      # pull: sources' blocks, source-major, then expert-major
+                blocks = np.concatenate([_bytes(peers[s])[starts[s]:starts[s] + lens[s]]
+                                         for s in range(R)], axis=0)
+                grouped, off = moe.ep_regroup(mine, blocks, 0, 0, np.zeros_like(blocks), 1, 0)
+                lb[:n] = grouped
+                if local_offsets is not None and loc is local:
+                    local_offsets.copy_(torch.from_numpy(off.astype(np.int32)))
+            else:                   # push: expert-major back to source-major, into the sources
+                back, _ = moe.ep_regroup(mine, lb[:n], 1, 0, np.zeros_like(lb[:n]), 0, 0)
+                pos = 0
+                for s in range(R):
+                    _bytes(peers[s])[starts[s]:starts[s] + lens[s]] = back[pos:pos + lens[s]]
+                    pos += lens[s]
+
     def expert_ffn(self, rows, scales, payload, offsets, max_rows, E, H, F, w_gate, w_up, w_down,
                    out, ws):
         self.calls.append("expert_ffn")

@@ -83,7 +83,8 @@ def test_gloo_ranks_match_the_single_device_oracle(world):
 
 
 def test_thread_loopback_matches_the_oracle_too():
-    """The in-process R-rank emulation used by the single-GPU tests gives the same results."""
+    """The in-process R-rank emulation used by the single-GPU tests gives the same results, and
+    runs the peer-memory mode (one address space) as well."""
     from combine_moe_route_10_b200.ep import MoeEP
     from _ep_loopback import run_ranks
     from _ep_oracle_ops import OracleOps
@@ -94,18 +95,23 @@ def test_thread_loopback_matches_the_oracle_too():
     def rank(r, comm):
         sl = slice(r * E_loc, (r + 1) * E_loc)
         out = {}
-        for mode in ("ht", "ll"):
-            ep = MoeEP(T_RANK, w.H, w.E, w.k, w.F, comm=comm, mode=mode, device="cpu",
-                       ops=OracleOps())
-            y = ep.forward(lg[r], xs[r], d["w_gate"][sl].contiguous(), d["w_up"][sl].contiguous(),
-                           d["w_down"][sl].contiguous())
+        for mode in ("ht", "ll", "p2p"):
+            ep = MoeEP(T_RANK, w.H, w.E, w.k, w.F, comm=comm, payload=payload, mode=mode,
+                       device="cpu", ops=OracleOps())
+            for _ in range(2):
+                y = ep.forward(lg[r], xs[r], d["w_gate"][sl].contiguous(),
+                               d["w_up"][sl].contiguous(), d["w_down"][sl].contiguous())
             out[mode] = y.view(torch.int16).numpy().view(np.uint16).copy()
         return out
 
-    res = run_ranks(R, rank)
-    wb = [bf16_bits(d[key].float().numpy()) for key in ("w_gate", "w_up", "w_down")]
-    ref = moe.pipeline(np.concatenate([a.numpy() for a in lg]),
-                       np.concatenate([bf16_bits(a.float().numpy()) for a in xs]), *wb, w.k, R)["y"]
-    for r in range(R):
-        for mode in ("ht", "ll"):
-            assert np.array_equal(res[r][mode], ref[r * T_RANK:(r + 1) * T_RANK]), (mode, r)
+    for payload in ("bf16", "fp8"):
+        w, lg, xs, d = _inputs(R, payload)
+        res = run_ranks(R, rank)
+        wb = [bf16_bits(d[key].float().numpy()) for key in ("w_gate", "w_up", "w_down")]
+        ref = moe.pipeline(np.concatenate([a.numpy() for a in lg]),
+                           np.concatenate([bf16_bits(a.float().numpy()) for a in xs]), *wb, w.k,
+                           R, fp8=payload == "fp8")["y"]
+        for r in range(R):
+            for mode in ("ht", "ll", "p2p"):
+                assert np.array_equal(res[r][mode], ref[r * T_RANK:(r + 1) * T_RANK]), \
+                    (payload, mode, r)

@@ -8,8 +8,12 @@
   ranks' buffers, no kernel waits on another) must give every rank exactly its slice of the
   single-device path over all ranks' tokens, in both exchange modes and both payloads; one small
   case is also held to the oracle's parity bar.
+* ``moe_ep_exchange`` (the exchange over peer memory fused with the regrouping) against the
+  oracle-backed restatement, pulling from and pushing into separate buffers of every rank; counts
+  that do not fit copy nothing and report MOE_ERR_INVALID_COUNTS.
 * ``MoeEP`` over a real NCCL process group of one rank, eager and captured in a CUDA graph (the
-  low-latency mode needs no host synchronisation).
+  low-latency and peer-memory modes need no host synchronisation), and through torch symmetric
+  memory.
 """
 import socket
 
@@ -96,6 +100,69 @@ def test_regroup_rejects_counts_that_do_not_fit(cuda):
     assert _lib.moe_sync_status(status) == 0
 
 
+@pytest.mark.parametrize("width,aux", [(256, 0), (7, 3), (512, 56)])
+def test_exchange_pull_and_push_match_oracle(cuda, width, aux):
+    from combine_moe_route_10_b200 import _lib
+    from _ep_oracle_ops import OracleOps
+    g = np.random.default_rng(width + aux)
+    R, E, rank = 3, 6, 1
+    C = g.integers(0, 30, size=(R, E)).astype(np.int32)
+    C[2, 2:4] = 0                                   # source 2 sends this rank nothing
+    cap = int(C.sum(axis=1).max()) + 4
+    dt = torch.bfloat16 if width % 2 == 0 else torch.float32
+    peers = [torch.randn(cap, width, device=cuda).to(dt) for _ in range(R)]
+    peers_aux = [torch.randn(cap, aux, device=cuda) for _ in range(R)] if aux else None
+    n_loc = int(C[:, 2:4].sum())
+    local = torch.full((n_loc + 5, width), 3.0, device=cuda, dtype=dt)
+    local_aux = torch.full((n_loc + 5, aux), -2.0, device=cuda) if aux else None
+    offs = torch.full((3,), -7, dtype=torch.int32, device=cuda)
+    status = torch.zeros(64, dtype=torch.int32, device=cuda)
+    ac = torch.from_numpy(C.reshape(-1)).to(cuda)
+    table = lambda ts: torch.tensor([t.data_ptr() for t in ts], dtype=torch.int64, device=cuda)
+    rb = width * local.element_size()
+    # expected: the same step on CPU copies with the oracle's layouts
+    o = OracleOps()
+    cpu_peers = [t.cpu() for t in peers]
+    cpu_aux = [t.cpu() for t in peers_aux] if aux else None
+    exp_local, exp_aux = local.cpu(), (local_aux.cpu() if aux else None)
+    exp_offs = torch.zeros(3, dtype=torch.int32)
+    o.exchange(ac.cpu(), R, E, rank, 0, cpu_peers, cpu_aux, cap, exp_local, exp_aux, exp_offs)
+    _lib.moe_ep_exchange(ac, R, E, rank, _lib.MOE_EP_PULL, table(peers),
+                         table(peers_aux) if aux else None, cap, local, local_aux,
+                         local.shape[0], rb, aux * 4, offs, status)
+    assert _lib.moe_sync_status(status) == 0
+    assert torch.equal(local.cpu(), exp_local)
+    assert torch.equal(offs.cpu(), exp_offs)
+    if aux:
+        assert torch.equal(local_aux.cpu(), exp_aux)
+    # push the (new) local rows back into every source's buffer
+    local2 = torch.randn(n_loc + 5, width, device=cuda).to(dt)
+    o.exchange(ac.cpu(), R, E, rank, 1, cpu_peers, None, cap, local2.cpu(), None)
+    _lib.moe_ep_exchange(ac, R, E, rank, _lib.MOE_EP_PUSH, table(peers), None, cap, local2, None,
+                         local2.shape[0], rb, 0, None, status)
+    assert _lib.moe_sync_status(status) == 0
+    for s_ in range(R):
+        assert torch.equal(peers[s_].cpu(), cpu_peers[s_]), s_
+
+
+def test_exchange_rejects_counts_that_do_not_fit(cuda):
+    from combine_moe_route_10_b200 import _lib
+    R, E, rank, cap = 2, 4, 1, 10
+    peers = [torch.zeros(cap, 64, device=cuda, dtype=torch.bfloat16) for _ in range(R)]
+    table = torch.tensor([t.data_ptr() for t in peers], dtype=torch.int64, device=cuda)
+    status = torch.zeros(64, dtype=torch.int32, device=cuda)
+    for C in (np.array([[1, -1, 2, 2], [0, 0, 1, 1]]),   # a negative count before this rank's block
+              np.array([[5, 4, 1, 1], [0, 0, 1, 1]]),    # source 0: block ends at row 11 > 10
+              np.array([[0, 0, 9, 0], [0, 0, 0, 9]])):   # 18 rows into a 10-row local buffer
+        local = torch.zeros(cap, 64, device=cuda, dtype=torch.bfloat16)
+        peers[0].fill_(1.0)
+        _lib.moe_ep_exchange(torch.from_numpy(C.astype(np.int32).reshape(-1)).to(cuda), R, E, rank,
+                             _lib.MOE_EP_PULL, table, None, cap, local, None, cap, 128, 0, None,
+                             status)
+        assert _lib.moe_sync_status(status) == _lib.MOE_ERR_INVALID_COUNTS, C
+        assert int(local.abs().sum().item()) == 0
+
+
 def _single_device(w, d, R_total, payload):
     from combine_moe_route_10_b200 import MoeShuffle
     T = sum(t.shape[0] for t in d["x"])
@@ -124,7 +191,7 @@ def _ep_threads(w, d, R, payload, mode, steps=2):
 
 
 @pytest.mark.parametrize("name", ["tiny", "train-small", "finegrained-small", "decode-small"])
-@pytest.mark.parametrize("mode", ["ht", "ll"])
+@pytest.mark.parametrize("mode", ["ht", "ll", "p2p"])
 def test_four_emulated_ranks_equal_the_single_device_path(cuda, name, mode):
     R = 4
     w = mi.get(name)
@@ -174,40 +241,69 @@ def test_nccl_one_rank_eager_and_graph(cuda):
     y_ref = _single_device(w, d, 1, "bf16")
     dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0,
                             world_size=1, device_id=cuda)
-    g = None
+    graphs = []
     try:
-        for mode in ("ht", "ll"):
+        for mode in ("ht", "ll", "p2p"):
             ep = MoeEP(w.T, w.H, w.E, w.k, w.F, mode=mode)
             y = ep.forward(d["logits"][0], d["x"][0], d["w_gate"], d["w_up"], d["w_down"])
             torch.cuda.synchronize()
             assert ep.status() == 0
             assert torch.equal(y, y_ref), mode
-        # the low-latency step has fixed splits and no host synchronisation: capture it
-        ep = MoeEP(w.T, w.H, w.E, w.k, w.F, mode="ll")
-        logits = d["logits"][0].clone()
-        x = d["x"][0].clone()
-        ep.forward(logits, x, d["w_gate"], d["w_up"], d["w_down"])
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        s = torch.cuda.Stream()
-        s.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(s):
-            with torch.cuda.graph(g, capture_error_mode="thread_local"):
-                ep.forward(logits, x, d["w_gate"], d["w_up"], d["w_down"])
-        torch.cuda.current_stream().wait_stream(s)
-        ep.y.zero_()
-        g.replay()
-        torch.cuda.synchronize()
-        assert torch.equal(ep.y, y_ref)
-        # new inputs written into the captured tensors
         d2 = mi.make_ep_inputs(w, 1, seed=8, device="cuda")
-        logits.copy_(d2["logits"][0])
-        x.copy_(d2["x"][0])
-        g.replay()
-        torch.cuda.synchronize()
         d2["w_gate"], d2["w_up"], d2["w_down"] = d["w_gate"], d["w_up"], d["w_down"]
-        assert torch.equal(ep.y, _single_device(w, d2, 1, "bf16"))
+        y_ref2 = _single_device(w, d2, 1, "bf16")
+        # the low-latency and peer-memory steps have no host synchronisation: capture them
+        graphs = []
+        for mode in ("ll", "p2p"):
+            ep = MoeEP(w.T, w.H, w.E, w.k, w.F, mode=mode)
+            logits = d["logits"][0].clone()
+            x = d["x"][0].clone()
+            ep.forward(logits, x, d["w_gate"], d["w_up"], d["w_down"])
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            graphs.append(g)
+            s = torch.cuda.Stream()
+            s.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(s):
+                with torch.cuda.graph(g, capture_error_mode="thread_local"):
+                    ep.forward(logits, x, d["w_gate"], d["w_up"], d["w_down"])
+            torch.cuda.current_stream().wait_stream(s)
+            ep.y.zero_()
+            g.replay()
+            torch.cuda.synchronize()
+            assert torch.equal(ep.y, y_ref), mode
+            # new inputs written into the captured tensors
+            logits.copy_(d2["logits"][0])
+            x.copy_(d2["x"][0])
+            g.replay()
+            torch.cuda.synchronize()
+            assert torch.equal(ep.y, y_ref2), mode
     finally:
-        del g
+        graphs = None
+        g = None
+        torch.cuda.synchronize()
+        dist.destroy_process_group()
+
+
+def test_nccl_one_rank_peer_mode_through_symmetric_memory(cuda):
+    """The peer buffers of the p2p mode through torch symmetric memory (the mapping used between
+    GPUs), at one rank."""
+    import torch.distributed as dist
+    from combine_moe_route_10_b200.ep import MoeEP, TorchComm
+    w = mi.get("finegrained-small")
+    d = mi.make_ep_inputs(w, 1, seed=9, device="cuda")
+    y_ref = _single_device(w, d, 1, "fp8")
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0,
+                            world_size=1, device_id=cuda)
+    try:
+        ep = MoeEP(w.T, w.H, w.E, w.k, w.F, comm=TorchComm(symmetric=True), payload="fp8",
+                   mode="p2p")
+        for _ in range(2):
+            y = ep.forward(d["logits"][0], d["x"][0], d["w_gate"], d["w_up"], d["w_down"])
+        torch.cuda.synchronize()
+        assert ep.status() == 0
+        assert torch.equal(y, y_ref)
+        del ep
+    finally:
         torch.cuda.synchronize()
         dist.destroy_process_group()
