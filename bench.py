@@ -14,6 +14,12 @@ in the same run and reported under ``workloads``.
 Multi-GPU (torchrun): every rank runs an independent replica of the workload (its own batch of T
 tokens, emulated expert-parallel ranks inside each GPU), no data-path collective; the step time is
 the max over ranks and ``value`` counts the tokens of all ranks ("weak" scaling).
+
+The line's ``expert_parallel`` object times the expert-parallel step (``MoeEP``, peer-memory mode)
+on the train shapes over the run's ranks: every rank owns E/N experts and its own T tokens, rows
+cross the ranks through the fused exchange kernel (at N = 1, a one-rank NCCL group: the exchange
+is a local move and the number shows the cost of the expert-parallel machinery).  With N > 1 it
+runs only with ``--ep``.
 """
 from __future__ import annotations
 
@@ -266,6 +272,10 @@ def main():
                     help="skip the extra timing of the step with FP8 gate / up weights")
     ap.add_argument("--e2e-eager", action="store_true",
                     help="end-to-end loop calls forward eagerly instead of replaying CUDA graphs")
+    ap.add_argument("--ep", action="store_true",
+                    help="time the expert-parallel step across the ranks when N > 1 (always at N = 1)")
+    ap.add_argument("--no-ep", action="store_true", help="skip the expert-parallel timing")
+    ap.add_argument("--ep-workload", default="train", choices=sorted(mi.WORKLOADS))
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -295,6 +305,9 @@ def main():
     sampler.start()
     head = measure(w, args, dev, world, rank, e2e=True)
     extra = {n: measure(mi.get(n), args, dev, world, rank, e2e=False) for n in also}
+    ep = None
+    if not args.no_ep and (world == 1 or args.ep):
+        ep = measure_ep(mi.get(args.ep_workload), args, dev, world, rank)
     clocks = sampler.stop()
 
     line = {
@@ -319,6 +332,7 @@ def main():
         "workloads_note": "the other large workloads, each timed the same way in the same run "
                           "(own warm-up, L2 flush, metric and breakdown steps); gpu_launches counts "
                           "the headline workload's timed region only",
+        "expert_parallel": ep,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         d_cpu = {k: v.cpu() for k, v in mi.make_inputs(w, seed=rank, device=str(dev)).items()}
@@ -461,6 +475,106 @@ def measure(w, args, dev, world: int, rank: int, e2e: bool) -> dict:
     del m, d, flush, flush_rd
     torch.cuda.empty_cache()
     return out
+
+
+def measure_ep(w, args, dev, world: int, rank: int) -> dict:
+    """The expert-parallel step (peer-memory mode) on workload ``w``'s shapes over this run's ranks:
+    rank r owns experts [r*E/N, (r+1)*E/N) and its own T tokens.  K metric steps (events at step
+    boundaries, max over ranks) interleaved with K steps that time the pull and push exchange
+    kernels; L2 flushed before every step."""
+    import datetime
+    import socket
+
+    import torch.distributed as dist
+    from combine_moe_route_10_b200 import _lib
+    from combine_moe_route_10_b200.ep import MoeEP, TorchComm
+
+    own_group = not dist.is_initialized()
+    if own_group:
+        with socket.socket() as so:
+            so.bind(("127.0.0.1", 0))
+            port = so.getsockname()[1]
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0,
+                                world_size=1, timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    try:
+        R = dist.get_world_size()
+        E_loc = w.E // R
+        d = mi.make_ep_inputs(w, R, seed=0, device=str(dev))
+        sl = slice(rank * E_loc, (rank + 1) * E_loc)
+        logits, x = d["logits"][rank], d["x"][rank]
+        wg, wu, wd = (d[k][sl].contiguous() for k in ("w_gate", "w_up", "w_down"))
+        del d
+        ep = MoeEP(w.T, w.H, w.E, w.k, w.F, comm=TorchComm(symmetric=R > 1), payload=w.payload,
+                   mode="p2p", device=dev)
+        flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+        stream = torch.cuda.current_stream(dev)
+        for _ in range(args.warmup):
+            flush.fill_(1)
+            ep.forward(logits, x, wg, wu, wd)
+        torch.cuda.synchronize()
+        if ep.status() != 0:
+            raise SystemExit(f"expert-parallel {w.name}: device status after warm-up")
+        n_recv = int(ep.local_offsets[E_loc].item())
+        S = ep.send.shape[0]
+        row_b = w.H * ep.send.element_size() + ep.nb * 4
+        st = ep.ws_regroup
+        step_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)]
+                   for _ in range(args.steps)]
+        x_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)]
+                for _ in range(args.steps)]
+        dist.barrier()
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            flush.fill_(1)
+            step_ev[i][0].record(stream)
+            ep.forward(logits, x, wg, wu, wd)
+            step_ev[i][1].record(stream)
+            # the two exchange kernels of the step just taken, timed on their own
+            flush.fill_(1)
+            e = x_ev[i]
+            e[0].record(stream)
+            _lib.moe_ep_exchange(ep.all_counts, R, w.E, rank, _lib.MOE_EP_PULL, ep.peer_send,
+                                 ep.peer_send_scales, S, ep.grouped, ep.grouped_scales, ep.cap,
+                                 w.H * ep.send.element_size(), ep.nb * 4, ep.local_offsets, st)
+            e[1].record(stream)
+            flush.fill_(1)
+            e[2].record(stream)
+            _lib.moe_ep_exchange(ep.all_counts, R, w.E, rank, _lib.MOE_EP_PUSH, ep.peer_ret, None,
+                                 S, ep.expert_out, None, ep.cap, w.H * 2, 0, None, st)
+            e[3].record(stream)
+            ep.comm.barrier(dev)  # the pushes into the other ranks end before their next step
+        torch.cuda.synchronize()
+        dist.barrier()
+        if ep.status() != 0:
+            raise SystemExit(f"expert-parallel {w.name}: device status after timing")
+        agg = aggregate(sum(a.elapsed_time(b) for a, b in step_ev), w.T, args.steps, dev)
+        t_pull = sum(e[0].elapsed_time(e[1]) for e in x_ev) / args.steps
+        t_push = sum(e[2].elapsed_time(e[3]) for e in x_ev) / args.steps
+        pk, _ = peaks()
+        hbm = pk["hbm_gbs"]
+
+        def kern(b, t):
+            g = b / (t * 1e-3) / 1e9
+            return {"ms": t, "GB/s": g, "frac": g / hbm, "bytes": b}
+
+        out = {"mode": "p2p", "workload": w.name, "ranks": R, "experts_per_rank": E_loc,
+               "value": agg["value"], "unit": "tokens/s", "ms_per_step": agg["ms_per_step"],
+               "received_rows": n_recv,
+               "exchange": {
+                   # each received row is read once and written once; at one rank both are HBM
+                   "pull": kern(2 * n_recv * row_b, t_pull),
+                   "push": kern(2 * n_recv * w.H * 2, t_push)},
+               "note": ("tokens/s counts every rank's T tokens over the slowest rank's step; "
+                        "exchange frac is of the measured HBM copy rate (at one rank every peer "
+                        "buffer is local; across GPUs the remote share is NVLink-bound)")}
+        del ep, flush, wg, wu, wd
+        torch.cuda.empty_cache()
+        return out
+    finally:
+        if own_group:
+            torch.cuda.synchronize()
+            dist.destroy_process_group()
 
 
 def measure_w8(w, m, d, args, stream, flush_l2, world, dev, S, active, pk) -> dict:

@@ -86,7 +86,7 @@ __device__ __forceinline__ void copy_row(const unsigned char* __restrict__ src,
   const V* s = reinterpret_cast<const V*>(src);
   V* d = reinterpret_cast<V*>(dst);
   const int n = static_cast<int>(bytes / sizeof(V));
-  constexpr int kU = 4;
+  constexpr int kU = 4;  // vectors in flight per lane (2 KB per warp for 16-byte vectors)
   int i = lane;
   for (; i + (kU - 1) * kWarp < n; i += kU * kWarp) {
     V t[kU];
@@ -110,7 +110,11 @@ struct Payload {
   int vec16;     // rows and base addresses allow 16-byte vectors (else 4-byte words)
 };
 
-__global__ void __launch_bounds__(kThreads)
+// Up to kCtasPerSm CTAs per SM (64 registers a thread): the copies are latency-bound per warp, so
+// the grid keeps as many warps in flight as the registers allow.
+constexpr int kCtasPerSm = 4;
+
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
     ep_regroup_kernel(const int32_t* __restrict__ counts, int A, int B, Side src_side,
                       Side dst_side, Payload p0, Payload p1, int32_t* __restrict__ dst_offsets,
                       int* status) {
@@ -194,7 +198,7 @@ __global__ void __launch_bounds__(kThreads)
 // into this rank's buffer (b-major over (s, e), packed), with the local expert offsets.  Push: the
 // reverse, from this rank's expert-major buffer into every source's buffer at the same positions.
 
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
     ep_exchange_kernel(const int32_t* __restrict__ all_counts, int R, int E, int rank, int E_loc,
                        int push, const unsigned long long* __restrict__ peer_rows,
                        const unsigned long long* __restrict__ peer_aux, int peer_cap,
@@ -288,7 +292,7 @@ cudaError_t launch_ep_exchange(const int32_t* all_counts, int R, int E, int rank
                                int32_t* local_offsets, int* status, cudaStream_t s) {
   const int E_loc = E / R;
   long long blocks = (static_cast<long long>(local_cap) + kWarps - 1) / kWarps;
-  if (blocks > 2LL * num_sms()) blocks = 2LL * num_sms();
+  if (blocks > kCtasPerSm * static_cast<long long>(num_sms())) blocks = kCtasPerSm * static_cast<long long>(num_sms());
   if (blocks < 1) blocks = 1;
   const cudaError_t err = launch_pdl(
       ep_exchange_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0, s, all_counts, R,
@@ -313,7 +317,7 @@ cudaError_t launch_ep_regroup(const int32_t* counts, int A, int B, int src_order
   // rows moved are at most the smaller capacity; one warp per row, a few waves at most
   const long long rows = src_rows < dst_rows ? src_rows : dst_rows;
   long long blocks = (rows + kWarps - 1) / kWarps;
-  if (blocks > 2LL * num_sms()) blocks = 2LL * num_sms();
+  if (blocks > kCtasPerSm * static_cast<long long>(num_sms())) blocks = kCtasPerSm * static_cast<long long>(num_sms());
   if (blocks < 1) blocks = 1;
   const cudaError_t err =
       launch_pdl(ep_regroup_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0, s,
