@@ -46,7 +46,7 @@ from .numerics import bf16_bits, bf16_from_bits, bf16_round, e4m3_decode, e4m3_e
 
 __all__ = ["capacity", "route", "dispatch_plan", "dispatch_payload", "expert_ffn", "combine",
            "pipeline", "QBLOCK", "quantize_rows_fp8", "dequantize_rows_fp8", "expert_ffn_w8",
-           "ep_segment_rows", "ep_regroup", "ep_pipeline"]
+           "ep_segment_rows", "ep_regroup", "ep_pipeline", "backward"]
 
 QBLOCK = 128   # elements per FP8 scale block
 E4M3_MAX_F32 = np.float32(448.0)
@@ -430,4 +430,142 @@ def ep_pipeline(logits_ranks, x_ranks, w_gate_bits, w_up_bits, w_down_bits, k: i
     out = []
     for r, (idx, w, plan, _, _) in enumerate(per):
         out.append(combine(back[r], plan["slot_row"], w, idx.shape[0], H))
+    return out
+
+
+# ---- backward ------------------------------------------------------------------------------------
+
+def backward(fwd, dy_bits, logits, w_gate_bits, w_up_bits, w_down_bits, renormalize: bool = True,
+             fp8: bool = False, exact: bool = False):
+    """Gradients of the path for an output gradient dy [T,H] (bf16 bit patterns), given the forward
+    intermediates ``fwd`` of ``pipeline`` (routing, plan, payload, expert outputs).
+
+    The training step of the NCCL EP page (section 3.2) reuses the forward's routing: the gradient is
+    dispatched through the same plan, the experts run backward, and the gradients are combined back.
+    In that order:
+
+    1. Combine backward, for every kept slot (t, j) -> row:
+       d_eo[row] = bf16(fp32(w[t,j] * dy[t]))  (y = sum_j w[t,j] eo[row]; the bf16 rounding of y is
+       taken as the identity), and the routing-weight gradient d_w[t,j] = sum_h dy[t,h] eo[row,h]
+       (exact, stored fp32); a dropped slot has d_w = 0.
+    2. Expert backward on the packed rows of expert e, x the FFN input values (as in the forward):
+       g = x Wg^T, u = x Wu^T, s = sigmoid(g), h = bf16(g s u) (recomputed as the forward made it),
+       dh = d_eo Wd, dg = bf16(dh u s (1 + g (1 - s))), du = bf16(dh g s),
+       dx_rows = bf16(dg Wg + du Wu), dWd = d_eo^T h, dWg = dg^T x, dWu = du^T x (fp64 sums; the
+       weight gradients stored fp32).
+    3. Combine of the input gradients: dx[t] = bf16(sum over kept j of dx_rows[slot_row[t,j]]),
+       fp32 in slot order (the forward combine with unit weights).
+    4. Router: with ``renormalize`` the weights are the softmax of the selected logits, so for a
+       selected expert i of token t  d_logits[t,i] = w_i (d_w_i - sum_j w_j d_w_j), 0 elsewhere;
+       otherwise they are the full-E softmax p, and d_logits[t,i] = p_i (d_i - sum_e p_e d_e) with
+       d_i = d_w of the slot that selected i (0 for unselected experts).  fp64, stored fp32.
+
+    ``exact`` skips every bf16 rounding above and uses the expert outputs without their rounding
+    (all fp64), for checks against finite differences.
+    Returns a dict of dx (bf16 bits [T,H], or float64 when exact), d_logits fp32 [T,E], d_w fp32
+    [T,k], d_w_gate / d_w_up fp32 [E,F,H], d_w_down fp32 [E,H,F], and the intermediates d_eo,
+    dg, du, dx_rows (bf16 bits, or float64 when exact) in packed row order."""
+    rnd = (lambda a: np.asarray(a, dtype=np.float64)) if exact else bf16_round
+    slot_row = np.asarray(fwd["slot_row"], dtype=np.int64)
+    w = np.asarray(fwd["topk_w"], dtype=np.float32)
+    idx = np.asarray(fwd["topk_idx"], dtype=np.int64)
+    off = np.asarray(fwd["expert_offsets"], dtype=np.int64)
+    T, k = slot_row.shape
+    E = off.size - 1
+    S = int(off[E])
+    dy = bf16_from_bits(np.asarray(dy_bits, dtype=np.uint16)).astype(np.float64)
+    H = dy.shape[1]
+    F = w_gate_bits.shape[1]
+    xin = ffn_inputs(fwd["send"], fwd["send_scales"], fp8)
+    if exact:
+        # the expert outputs without their bf16 roundings
+        eo = np.zeros((S, H))
+        for e in range(E):
+            lo, hi = off[e], off[e + 1]
+            if hi == lo:
+                continue
+            x = np.asarray(xin[lo:hi], dtype=np.float64)
+            g = x @ bf16_from_bits(w_gate_bits[e]).astype(np.float64).T
+            u = x @ bf16_from_bits(w_up_bits[e]).astype(np.float64).T
+            eo[lo:hi] = (g / (1.0 + np.exp(-g)) * u) @ bf16_from_bits(w_down_bits[e]).astype(
+                np.float64).T
+    else:
+        eo = bf16_from_bits(np.asarray(fwd["expert_out"], dtype=np.uint16)).astype(np.float64)
+    # 1. combine backward
+    d_eo = np.zeros((S, H), dtype=np.float64)
+    d_w = np.zeros((T, k), dtype=np.float64)
+    for t in range(T):
+        for j in range(k):
+            row = slot_row[t, j]
+            if row < 0:
+                continue
+            prod = dy[t] * float(w[t, j])
+            d_eo[row] = prod if exact else prod.astype(np.float32)
+            d_w[t, j] = float(np.dot(dy[t], eo[row]))
+    d_eo = rnd(d_eo)
+    # 2. expert backward
+    dg_all = np.zeros((S, F))
+    du_all = np.zeros((S, F))
+    dxr = np.zeros((S, H))
+    dWg = np.zeros((E, F, H))
+    dWu = np.zeros((E, F, H))
+    dWd = np.zeros((E, H, F))
+    for e in range(E):
+        lo, hi = off[e], off[e + 1]
+        if hi == lo:
+            continue
+        x = np.asarray(xin[lo:hi], dtype=np.float64)
+        wg = bf16_from_bits(w_gate_bits[e]).astype(np.float64)
+        wu = bf16_from_bits(w_up_bits[e]).astype(np.float64)
+        wd = bf16_from_bits(w_down_bits[e]).astype(np.float64)
+        g = x @ wg.T
+        u = x @ wu.T
+        sg = 1.0 / (1.0 + np.exp(-g))
+        h = rnd(g * sg * u)
+        de = d_eo[lo:hi]
+        dh = de @ wd
+        dg = rnd(dh * u * sg * (1.0 + g * (1.0 - sg)))
+        du = rnd(dh * g * sg)
+        dxr[lo:hi] = rnd(dg @ wg + du @ wu)
+        dWd[e] = de.T @ h
+        dWg[e] = dg.T @ x
+        dWu[e] = du.T @ x
+        dg_all[lo:hi] = dg
+        du_all[lo:hi] = du
+    # 3. combine of the input gradients (unit weights, fp32 in slot order)
+    if exact:
+        dx = np.zeros((T, H))
+        for t in range(T):
+            for j in range(k):
+                if slot_row[t, j] >= 0:
+                    dx[t] += dxr[slot_row[t, j]]
+    else:
+        dx = combine(bf16_bits(dxr), slot_row, np.ones((T, k), dtype=np.float32), T, H)
+    # 4. router
+    L = np.asarray(logits, dtype=np.float64)
+    d_logits = np.zeros_like(L)
+    for t in range(T):
+        if renormalize:
+            wt = w[t].astype(np.float64)
+            c = float(np.dot(wt, d_w[t]))
+            for j in range(k):
+                d_logits[t, idx[t, j]] = wt[j] * (d_w[t, j] - c)
+        else:
+            p = np.exp(L[t] - L[t].max())
+            p /= p.sum()
+            d = np.zeros(L.shape[1])
+            for j in range(k):
+                d[idx[t, j]] = d_w[t, j]
+            d_logits[t] = p * (d - float(np.dot(p, d)))
+    out = {"dx": dx, "d_logits": d_logits.astype(np.float32),
+           "d_w": d_w.astype(np.float32),
+           "d_w_gate": dWg if exact else dWg.astype(np.float32),
+           "d_w_up": dWu if exact else dWu.astype(np.float32),
+           "d_w_down": dWd if exact else dWd.astype(np.float32)}
+    if exact:
+        out.update(d_eo=d_eo, dg=dg_all, du=du_all, dx_rows=dxr, d_logits=d_logits,
+                   d_w=d_w)
+    else:
+        out.update(d_eo=bf16_bits(d_eo), dg=bf16_bits(dg_all), du=bf16_bits(du_all),
+                   dx_rows=bf16_bits(dxr))
     return out
