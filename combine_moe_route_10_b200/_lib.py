@@ -29,7 +29,7 @@ EXPORTS = ["moe_abi_version", "moe_status_string", "moe_capacity", "moe_route",
            "moe_ffn_workspace_size",
            "moe_expert_ffn", "moe_ffn_weight_list_bytes", "moe_ffn_weight_list_init",
            "moe_expert_ffn_list", "moe_quantize_rows_fp8", "moe_ffn_w8_workspace_size",
-           "moe_expert_ffn_w8", "moe_ep_regroup", "moe_ep_exchange", "moe_combine", "moe_sync_status"]
+           "moe_expert_ffn_w8", "moe_backward_workspace_size", "moe_backward", "moe_ep_regroup", "moe_ep_exchange", "moe_combine", "moe_sync_status"]
 
 _lib = None
 
@@ -66,6 +66,9 @@ def load() -> ctypes.CDLL:
         "moe_quantize_rows_fp8": (I, [P, I, I, P, P, P]),
         "moe_ffn_w8_workspace_size": (Z, [I, I, I, I, I]),
         "moe_expert_ffn_w8": (I, [P, P, I, P, I, I, I, I, P, P, P, P, P, P, P, Z, P]),
+        "moe_backward_workspace_size": (Z, [I, I, I, I, I]),
+        "moe_backward": (I, [P, I, I, I, I, I, P, I, P, P, P, P, I, P, P, P, P, P, P, P, P, P, P,
+                             P, P, Z, P]),
         "moe_ep_regroup": (I, [P, I, I, I, I, I, I, I, I, P, P, Z, P, P, Z, P, P, P]),
         "moe_ep_exchange": (I, [P, I, I, I, I, P, P, I, P, P, I, Z, Z, P, P, P]),
         "moe_combine": (I, [P, I, P, P, I, I, I, P, P, P]),
@@ -202,6 +205,23 @@ def moe_expert_ffn_w8(send, send_scales, payload, expert_offsets, max_rows, E, H
                                   _ptr(w_up_q), _ptr(w_up_scale), _ptr(w_down), _ptr(expert_out),
                                   _ptr(ws), ws_bytes, _stream(stream))
     return _check(st, "moe_expert_ffn_w8", raise_on_error)
+
+
+def moe_backward_workspace_size(max_rows, T, k, H, F) -> int:
+    return load().moe_backward_workspace_size(max_rows, T, k, H, F)
+
+
+def moe_backward(dy, T, H, k, E, F, logits, renormalize, topk_idx, topk_w, slot_row,
+                 expert_offsets, max_rows, ffn_input, expert_out, w_gate, w_up, w_down, dx,
+                 d_logits, d_topk_w, d_w_gate, d_w_up, d_w_down, ws, ws_bytes, stream=None,
+                 raise_on_error=True):
+    st = load().moe_backward(_ptr(dy), T, H, k, E, F, _ptr(logits), int(renormalize),
+                             _ptr(topk_idx), _ptr(topk_w), _ptr(slot_row), _ptr(expert_offsets),
+                             max_rows, _ptr(ffn_input), _ptr(expert_out), _ptr(w_gate),
+                             _ptr(w_up), _ptr(w_down), _ptr(dx), _ptr(d_logits), _ptr(d_topk_w),
+                             _ptr(d_w_gate), _ptr(d_w_up), _ptr(d_w_down), _ptr(ws), ws_bytes,
+                             _stream(stream))
+    return _check(st, "moe_backward", raise_on_error)
 
 
 def moe_ep_regroup(counts, A, B, src_order, src_stride, src_rows, dst_order, dst_stride, dst_rows,

@@ -286,6 +286,42 @@ moe_status_t moe_ep_exchange(const int32_t* all_counts, int R, int E, int rank, 
       reinterpret_cast<int*>(status), reinterpret_cast<cudaStream_t>(stream)));
 }
 
+size_t moe_backward_workspace_size(int max_rows, int T, int k, int H, int F) {
+  if (max_rows < 0 || T < 0 || k < 1 || H < 1 || F < 1) return 0;
+  return moe::backward_workspace_bytes(max_rows, T, k, H, F);
+}
+
+moe_status_t moe_backward(const void* dy, int T, int H, int k, int E, int F, const float* logits,
+                          int renormalize, const int32_t* topk_idx, const float* topk_w,
+                          const int32_t* slot_row, const int32_t* expert_offsets, int max_rows,
+                          const void* ffn_input, const void* expert_out, const void* w_gate,
+                          const void* w_up, const void* w_down, void* dx, float* d_logits,
+                          float* d_topk_w, float* d_w_gate, float* d_w_up, float* d_w_down,
+                          void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (T < 0 || k < 1 || k > 32 || E < 1 || E > 1024 || k > E || max_rows < 0 || H < 8 || F < 1)
+    return MOE_ERR_INVALID_ARG;
+  if (static_cast<long long>(T) * k > max_rows) return MOE_ERR_INVALID_ARG;
+  if (H % 64 != 0 || F % 64 != 0) return MOE_ERR_UNSUPPORTED;
+  const void* need[] = {topk_idx, topk_w, slot_row, expert_offsets, w_gate, w_up, w_down,
+                        d_logits, d_topk_w, d_w_gate, d_w_up, d_w_down, ws};
+  for (const void* q : need)
+    if (q == nullptr) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (dy == nullptr || dx == nullptr || ffn_input == nullptr || expert_out == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (!renormalize && logits == nullptr) return MOE_ERR_INVALID_ARG;
+  const void* a16[] = {dy, dx, ffn_input, expert_out, w_gate, w_up, w_down, d_w_gate, d_w_up,
+                       d_w_down};
+  for (const void* q : a16)
+    if (!aligned(q, 16)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(ws, 256)) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < moe::backward_workspace_bytes(max_rows, T, k, H, F)) return MOE_ERR_WORKSPACE;
+  return from_cuda(moe::launch_backward(dy, T, H, k, E, F, logits, renormalize, topk_idx, topk_w,
+                                        slot_row, expert_offsets, max_rows, ffn_input, expert_out,
+                                        w_gate, w_up, w_down, dx, d_logits, d_topk_w, d_w_gate,
+                                        d_w_up, d_w_down, ws,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
 moe_status_t moe_combine(const void* expert_out, int max_rows, const int32_t* slot_row,
                          const float* topk_w, int T, int k, int H, void* y, int32_t* status,
                          moe_stream_t stream) {

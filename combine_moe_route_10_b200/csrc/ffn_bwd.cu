@@ -1,0 +1,735 @@
+// Backward of the MoE layer: the gradient goes back through the forward's plan (the training step
+// of the NCCL EP page, section 3.2: the backward reuses the forward's routing handle, dispatches the
+// output gradient to the experts, runs the experts backward and combines the gradients).
+//
+//   1. combine_bwd_kernel (warp per token): d_eo[row] = bf16(w[t,j] * dy[t]) for every kept slot,
+//      the routing-weight gradient d_w[t,j] = <dy[t], eo[row]>, and from it the router's logit
+//      gradient (softmax backward over the selected k, or over all E without renormalisation).
+//   2. bwd_gemm_kernel<kRecompute> (tcgen05, M = 128 rows, 64 h columns): recomputes g = x Wg^T and
+//      u = x Wu^T and computes dh = d_eo Wd in the same K loop over H (three TMEM accumulators; Wd
+//      is read MN-major), then the SwiGLU backward in the epilogue: h, dg, du (bf16).
+//   3. bwd_gemm_kernel<kInputGrad> (M = 128, N = 256): dx_rows = dg Wg + du Wu, one K loop over
+//      2F, the weights read MN-major.
+//   4. bwd_gemm_kernel<kWeightGrad> (M = 128, N = 256, K = the expert's rows): dWd = d_eo^T h,
+//      dWg = dg^T x, dWu = du^T x in fp32, both operands MN-major; the rows past the expert's end in
+//      the last K block are zeroed in shared memory before the MMA reads them.
+//   5. the forward combine with unit weights: dx[t] = bf16(sum of dx_rows of its kept slots).
+//
+// The GEMM kernels are persistent (one CTA per SM, a static tile order), warp-specialised like the
+// forward's single-CTA kernel: warp 0 = TMA producer, warp 1 = TMEM allocation and the MMA thread,
+// warps 2..5 = epilogue, two accumulators so that an epilogue overlaps the next tile's MMAs.  Every
+// wait is bounded (kStatusTimeout); no TMA multicast.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace moe {
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kUK = 16;
+constexpr int kBwdThreads = 192;
+constexpr int kTmemColsBwd = 512;
+constexpr int kAccStride = 256;  // TMEM columns between the two accumulators
+constexpr int kNF1 = 64;         // h columns per recompute tile
+constexpr int kNOut = 256;       // output columns per input-gradient / weight-gradient tile
+
+enum Mode { kRecompute = 1, kInputGrad = 2, kWeightGrad = 3 };
+
+template <int MODE>
+struct Cfg {
+  // recompute: x + d_eo (16 KB each) + Wg, Wu, Wd^T (8 KB each); others: A 16 KB + B 32 KB
+  static constexpr int kStageBytes = MODE == kRecompute ? 2 * 16384 + 3 * 8192 : 16384 + 32768;
+  static constexpr int kStages = MODE == kRecompute ? 3 : 4;
+};
+
+// ---- PTX wrappers -----------------------------------------------------------------------------
+__device__ __forceinline__ void tma2d(uint32_t dst, const CUtensorMap* tm, uint32_t bar, int x,
+                                      int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void commit(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                    uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory descriptor of a bf16 tile with the 128-byte swizzle (layout type 2, version 1).
+// K-major: rows of 128 bytes hold 64 k values, 8-row groups 1024 bytes apart (stride byte offset;
+// the leading byte offset is unused).  MN-major: rows of 128 bytes hold 64 m (or n) values of one
+// k, 8-k groups 1024 bytes apart (stride byte offset), and the next 64 m values lie `lbo` bytes
+// further (the next TMA box: leading byte offset).
+__device__ __forceinline__ uint64_t desc_k(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>(1) << 16) |
+         (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
+         (static_cast<uint64_t>(2) << 61);
+}
+__device__ __forceinline__ uint64_t desc_mn(uint32_t saddr, uint32_t lbo) {
+  return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) |
+         (static_cast<uint64_t>(lbo >> 4) << 16) | (static_cast<uint64_t>(1024 >> 4) << 32) |
+         (static_cast<uint64_t>(1) << 46) | (static_cast<uint64_t>(2) << 61);
+}
+// kind::f16 instruction descriptor: fp32 D, bf16 A and B, a_mn / b_mn = MN-major operands.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(a_mn) << 15) |
+         (static_cast<uint32_t>(b_mn) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ bool bwait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                      int* status) {
+  return wait_phase(bar, parity, abort_flag, status);
+}
+// Wait for a barrier phase regardless of the abort flag (a CTA draining its own copies / MMAs).
+__device__ __forceinline__ void bdrain(uint32_t bar, uint32_t parity) {
+  const unsigned long long t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity) && global_timer_ns() - t0 <= kWaitLimitNs) {
+  }
+}
+
+struct BwdArgs {
+  const int32_t* expert_offsets;  // [E + 1], packed rows of every expert
+  int E, H, F, max_rows;
+  void* out0;  // recompute: h; input grad: dx_rows; weight grad: dWd
+  void* out1;  // recompute: dg;                       weight grad: dWg
+  void* out2;  // recompute: du;                       weight grad: dWu
+  int* status;
+};
+
+// Tiles of every expert (prefix in shared memory) and the decoding of a tile index.
+struct Tile {
+  int e, p, mb, nb;  // expert, sub-problem (weight grad), row / output block, column block
+};
+template <int MODE>
+__device__ __forceinline__ int tiles_of(const BwdArgs& a, int rows, int p) {
+  if (MODE == kRecompute) return ((rows + kBM - 1) / kBM) * (a.F / kNF1);
+  if (MODE == kInputGrad) return ((rows + kBM - 1) / kBM) * ((a.H + kNOut - 1) / kNOut);
+  // weight gradients: p = 0 dWd [H, F]; p = 1, 2 dWg, dWu [F, H]
+  const int M = p == 0 ? a.H : a.F, N = p == 0 ? a.F : a.H;
+  return ((M + kBM - 1) / kBM) * ((N + kNOut - 1) / kNOut);
+}
+
+template <int MODE>
+__device__ __forceinline__ Tile decode(const BwdArgs& a, const int* start, int tile) {
+  // start[i] = first tile of item i, items = experts (x 3 sub-problems for the weight grads)
+  const int n_items = MODE == kWeightGrad ? 3 * a.E : a.E;
+  int lo = 0, hi = n_items - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (start[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
+  Tile t;
+  t.p = MODE == kWeightGrad ? lo / a.E : 0;
+  t.e = MODE == kWeightGrad ? lo % a.E : lo;
+  const int local = tile - start[lo];
+  int ncol;
+  if (MODE == kRecompute) ncol = a.F / kNF1;
+  else if (MODE == kInputGrad) ncol = (a.H + kNOut - 1) / kNOut;
+  else ncol = ((t.p == 0 ? a.F : a.H) + kNOut - 1) / kNOut;
+  t.mb = local / ncol;
+  t.nb = local % ncol;
+  return t;
+}
+
+template <int MODE>
+__device__ __forceinline__ int k_blocks(const BwdArgs& a, int rows) {
+  if (MODE == kRecompute) return a.H / kBK;
+  if (MODE == kInputGrad) return 2 * (a.F / kBK);
+  return (rows + kBK - 1) / kBK;
+}
+
+// Operand maps of a mode (unused ones are zero).
+struct BwdMaps {
+  CUtensorMap m[6];
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_gemm_kernel(const __grid_constant__ BwdMaps maps, const BwdArgs args) {
+  constexpr int kStages = Cfg<MODE>::kStages;
+  constexpr int kStageBytes = Cfg<MODE>::kStageBytes;
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte aligned stages, then barriers, then the tile prefix table
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + kStages * kStageBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kStages;
+  uint64_t* acc_full = bars + 2 * kStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* fix_bar = acc_empty + 2;
+  uint64_t* drain_bar = fix_bar + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* start = reinterpret_cast<int*>(tmem_slot + 4);  // [items + 1]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = args.E;
+  const int n_items = MODE == kWeightGrad ? 3 * E : E;
+
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(smem_addr(&full[i]), 1);
+      mbar_init(smem_addr(&empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_addr(&acc_full[i]), 1);
+      mbar_init(smem_addr(&acc_empty[i]), 4);
+    }
+    mbar_init(smem_addr(fix_bar), 1);
+    mbar_init(smem_addr(drain_bar), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  } else if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(tmem_slot)),
+                 "r"(kTmemColsBwd)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  griddep_wait();
+  griddep_launch_dependents();
+  if (warp == 2 && lane == 0) {
+    int run = 0;
+    for (int i = 0; i < n_items; ++i) {
+      start[i] = run;
+      const int e = i % E;
+      const int rows = __ldg(args.expert_offsets + e + 1) - __ldg(args.expert_offsets + e);
+      run += tiles_of<MODE>(args, rows, i / E);
+    }
+    start[n_items] = run;
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = start[n_items];
+  const uint32_t stage0 = smem_addr(base);
+
+  if (warp == 0) {
+    // ---- TMA producer (lane 0 issues; the whole warp zeroes a ragged K tail) ----------------------
+    int stage = 0;
+    uint32_t phase = 0, fix_phase = 0;
+    uint32_t issued_mask = 0, issued_parity = 0;
+    bool stop = false;
+    for (int tile = blockIdx.x; tile < total && !stop; tile += gridDim.x) {
+      const Tile t = decode<MODE>(args, start, tile);
+      const int off = __ldg(args.expert_offsets + t.e);
+      const int rows = __ldg(args.expert_offsets + t.e + 1) - off;
+      const int nkb = k_blocks<MODE>(args, rows);
+      for (int kb = 0; kb < nkb; ++kb) {
+        int ok = 1;
+        if (lane == 0) ok = bwait(smem_addr(&empty[stage]), phase ^ 1u, abort_flag, args.status);
+        if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) {
+          stop = true;
+          break;
+        }
+        const uint32_t a = stage0 + stage * kStageBytes;
+        const uint32_t fb = smem_addr(&full[stage]);
+        if (MODE == kRecompute) {
+          if (lane == 0) {
+            const int kx = kb * kBK, row0 = off + t.mb * kBM, f0 = t.nb * kNF1;
+            mbar_arrive_expect_tx(fb, kStageBytes);
+            tma2d(a, &maps.m[0], fb, kx, row0);                        // x rows (K-major)
+            tma2d(a + 16384, &maps.m[1], fb, kx, row0);                // d_eo rows (K-major)
+            tma2d(a + 32768, &maps.m[2], fb, kx, t.e * args.F + f0);   // Wg rows (K-major)
+            tma2d(a + 40960, &maps.m[3], fb, kx, t.e * args.F + f0);   // Wu rows (K-major)
+            tma2d(a + 49152, &maps.m[4], fb, f0, t.e * args.H + kx);   // Wd: 64 h x 64 f (MN-major)
+          }
+        } else if (MODE == kInputGrad) {
+          if (lane == 0) {
+            const int nf = args.F / kBK;
+            const bool up = kb >= nf;
+            const int kx = (up ? kb - nf : kb) * kBK, row0 = off + t.mb * kBM, n0 = t.nb * kNOut;
+            mbar_arrive_expect_tx(fb, kStageBytes);
+            tma2d(a, &maps.m[up ? 1 : 0], fb, kx, row0);  // dg or du rows (K-major)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)  // Wg or Wu: 64 f x 64 h per box (MN-major)
+              tma2d(a + 16384 + i * 8192, &maps.m[up ? 3 : 2], fb, n0 + 64 * i,
+                    t.e * args.F + kx);
+          }
+        } else {
+          // A: 2 boxes of 64 m x 64 rows, B: 4 boxes of 64 n x 64 rows, all MN-major
+          const CUtensorMap* ma = &maps.m[t.p == 0 ? 0 : (t.p == 1 ? 1 : 2)];  // d_eo, dg, du
+          const CUtensorMap* mb = &maps.m[t.p == 0 ? 3 : 4];                   // h, x
+          const int y = off + kb * kBK, m0 = t.mb * kBM, n0 = t.nb * kNOut;
+          const int valid = min(kBK, rows - kb * kBK);
+          const uint32_t bar = valid == kBK ? fb : smem_addr(fix_bar);
+          if (lane == 0) {
+            mbar_arrive_expect_tx(bar, kStageBytes);
+            tma2d(a, ma, bar, m0, y);
+            tma2d(a + 8192, ma, bar, m0 + 64, y);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) tma2d(a + 16384 + i * 8192, mb, bar, n0 + 64 * i, y);
+          }
+          if (valid < kBK) {
+            // rows past the expert's end: zero them in all six boxes, then release the stage
+            // every lane waits, so that its stores below follow the copy's writes
+            const int got = bwait(smem_addr(fix_bar), fix_phase, abort_flag, args.status) ? 1 : 0;
+            fix_phase ^= 1u;
+            if (__all_sync(0xFFFFFFFFu, got) == 0) {
+              stop = true;
+              break;
+            }
+            uint4* s = reinterpret_cast<uint4*>(base + stage * kStageBytes);
+            const int per_box = (kBK - valid) * 8;  // 16-byte chunks in the rows to clear
+            for (int i = lane; i < 6 * per_box; i += 32) {
+              const int box = i / per_box, c = i % per_box;
+              s[box * 512 + valid * 8 + c] = make_uint4(0u, 0u, 0u, 0u);
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(fb);
+          }
+        }
+        issued_mask |= 1u << stage;
+        issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (*abort_flag && lane == 0) {
+      for (int st = 0; st < kStages; ++st)
+        if (issued_mask & (1u << st)) bdrain(smem_addr(&full[st]), (issued_parity >> st) & 1u);
+    }
+  } else if (warp == 1) {
+    // ---- MMA thread ---------------------------------------------------------------------------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool issued_any = false;
+      int it = 0;
+      for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+        const Tile t = decode<MODE>(args, start, tile);
+        const int rows = __ldg(args.expert_offsets + t.e + 1) - __ldg(args.expert_offsets + t.e);
+        const int nkb = k_blocks<MODE>(args, rows);
+        const int acc = it & 1;
+        if (!bwait(smem_addr(&acc_empty[acc]), ((it >> 1) & 1) ^ 1u, abort_flag, args.status))
+          break;
+        fence_after();
+        const uint32_t d = tmem_base + acc * kAccStride;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!bwait(smem_addr(&full[stage]), phase, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          const uint32_t a = stage0 + stage * kStageBytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / kUK; ++kk) {
+            const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+            if (MODE == kRecompute) {
+              constexpr uint32_t iK = idesc_bf16(kBM, kNF1, 0, 0), iMN = idesc_bf16(kBM, kNF1, 0, 1);
+              const uint64_t ax = desc_k(a + kk * 32), ae = desc_k(a + 16384 + kk * 32);
+              mma(d, ax, desc_k(a + 32768 + kk * 32), iK, accum);            // g
+              mma(d + 64, ax, desc_k(a + 40960 + kk * 32), iK, accum);       // u
+              mma(d + 128, ae, desc_mn(a + 49152 + kk * 2048, 8192), iMN, accum);  // dh
+            } else if (MODE == kInputGrad) {
+              constexpr uint32_t iMN = idesc_bf16(kBM, kNOut, 0, 1);
+              mma(d, desc_k(a + kk * 32), desc_mn(a + 16384 + kk * 2048, 8192), iMN, accum);
+            } else {
+              constexpr uint32_t iMM = idesc_bf16(kBM, kNOut, 1, 1);
+              mma(d, desc_mn(a + kk * 2048, 8192), desc_mn(a + 16384 + kk * 2048, 8192), iMM,
+                  accum);
+            }
+          }
+          issued_any = true;
+          commit(smem_addr(&empty[stage]));
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        // a tile without K blocks (an expert with no rows) has nothing to wait for: the epilogue
+        // writes zeros; the commit still orders it after the previous tile's MMAs
+        commit(smem_addr(&acc_full[acc]));
+      }
+      if (issued_any) {
+        commit(smem_addr(drain_bar));
+        bdrain(smem_addr(drain_bar), 0);
+      }
+    }
+  } else {
+    // ---- epilogue: warp (w & 3) owns TMEM lanes (= tile rows) [32 (w & 3), +32) ----------------------
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+      const Tile t = decode<MODE>(args, start, tile);
+      const int off = __ldg(args.expert_offsets + t.e);
+      const int rows = __ldg(args.expert_offsets + t.e + 1) - off;
+      const int acc = it & 1;
+      int ok = 1;
+      if (lane == 0) ok = bwait(smem_addr(&acc_full[acc]), (it >> 1) & 1, abort_flag, args.status);
+      if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) break;
+      fence_after();
+      const uint32_t tb = tmem_base + acc * kAccStride + (static_cast<uint32_t>(quarter * 32) << 16);
+      if (MODE == kRecompute) {
+        const bool valid = t.mb * kBM + r < rows;
+        const size_t row = static_cast<size_t>(off + t.mb * kBM + r);
+        __nv_bfloat16* h_out = static_cast<__nv_bfloat16*>(args.out0);
+        __nv_bfloat16* dg_out = static_cast<__nv_bfloat16*>(args.out1);
+        __nv_bfloat16* du_out = static_cast<__nv_bfloat16*>(args.out2);
+#pragma unroll 1
+        for (int c = 0; c < kNF1; c += 32) {
+          uint32_t g[32], u[32], dh[32];
+          ld32(tb + c, g);
+          ld32(tb + 64 + c, u);
+          ld32(tb + 128 + c, dh);
+          ld_wait();
+          uint32_t ph[16], pg[16], pu[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float hv[2], dgv[2], duv[2];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const float gv = __uint_as_float(g[2 * i + q]), uv = __uint_as_float(u[2 * i + q]);
+              const float dv = __uint_as_float(dh[2 * i + q]);
+              const float sg = 1.0f / (1.0f + expf(-gv));
+              const float silu = gv * sg;
+              hv[q] = silu * uv;
+              dgv[q] = dv * uv * sg * (1.0f + gv * (1.0f - sg));
+              duv[q] = dv * silu;
+            }
+            ph[i] = pack_bf16x2(hv[0], hv[1]);
+            pg[i] = pack_bf16x2(dgv[0], dgv[1]);
+            pu[i] = pack_bf16x2(duv[0], duv[1]);
+          }
+          if (valid) {
+            const size_t col = static_cast<size_t>(t.nb * kNF1 + c);
+            uint4* hp = reinterpret_cast<uint4*>(h_out + row * args.F + col);
+            uint4* gp = reinterpret_cast<uint4*>(dg_out + row * args.F + col);
+            uint4* up = reinterpret_cast<uint4*>(du_out + row * args.F + col);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              hp[v] = make_uint4(ph[4 * v], ph[4 * v + 1], ph[4 * v + 2], ph[4 * v + 3]);
+              gp[v] = make_uint4(pg[4 * v], pg[4 * v + 1], pg[4 * v + 2], pg[4 * v + 3]);
+              up[v] = make_uint4(pu[4 * v], pu[4 * v + 1], pu[4 * v + 2], pu[4 * v + 3]);
+            }
+          }
+        }
+      } else if (MODE == kInputGrad) {
+        const bool valid = t.mb * kBM + r < rows;
+        const size_t row = static_cast<size_t>(off + t.mb * kBM + r);
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out0);
+#pragma unroll 1
+        for (int c = 0; c < kNOut; c += 32) {
+          const int col = t.nb * kNOut + c;
+          if (col >= args.H) break;  // uniform over the warp
+          uint32_t v[32];
+          ld32(tb + c, v);
+          ld_wait();
+          if (valid) {
+            uint4* p = reinterpret_cast<uint4*>(out + row * args.H + col);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              p[q] = make_uint4(
+                  pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
+                  pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+                  pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+                  pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+          }
+        }
+      } else {
+        const int M = t.p == 0 ? args.H : args.F, N = t.p == 0 ? args.F : args.H;
+        const int m = t.mb * kBM + r;
+        float* out = static_cast<float*>(t.p == 0 ? args.out0 : (t.p == 1 ? args.out1 : args.out2));
+        const size_t row = static_cast<size_t>(t.e) * M + m;
+        const bool any_k = rows > 0;  // uniform over the warp
+#pragma unroll 1
+        for (int c = 0; c < kNOut; c += 32) {
+          const int col = t.nb * kNOut + c;
+          if (col >= N) break;
+          uint32_t v[32];
+          if (any_k) {
+            ld32(tb + c, v);
+            ld_wait();
+          } else {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) v[q] = 0u;
+          }
+          if (m < M) {
+            uint4* p = reinterpret_cast<uint4*>(out + row * N + col);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) p[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          }
+        }
+      }
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_addr(&acc_empty[acc]));
+    }
+  }
+
+  fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(kTmemColsBwd)
+                 : "memory");
+  }
+}
+
+// ---- combine backward and the router's gradient (warp per token) ---------------------------------
+// d_eo[row] = bf16(fp32(w * dy)) for every kept slot; d_w[t,j] = <dy[t], eo[row]> (0 for a dropped
+// slot); d_logits[t, :] from d_w (softmax backward); ones[t,j] = 1 (the unit weights of the final
+// combine of the input gradients).
+__global__ void __launch_bounds__(256)
+    combine_bwd_kernel(const uint4* __restrict__ dy, const uint4* __restrict__ eo, int max_rows,
+                       const int32_t* __restrict__ slot_row, const float* __restrict__ topk_w,
+                       const int32_t* __restrict__ topk_idx, const float* __restrict__ logits,
+                       int renormalize, int T, int k, int E, int H, uint4* __restrict__ d_eo,
+                       float* __restrict__ d_w, float* __restrict__ d_logits,
+                       float* __restrict__ ones) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int nv = H / 8;
+  for (int t = blockIdx.x * 8 + (threadIdx.x >> 5); t < T; t += gridDim.x * 8) {
+    float dot[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) dot[j] = 0.0f;
+    for (int v = lane; v < nv; v += 32) {
+      const uint4 g = ld_nc_v4(dy + static_cast<size_t>(t) * nv + v);
+      const uint32_t gw[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (j >= k) break;
+        const int row = __ldg(slot_row + t * k + j);
+        if (row < 0 || row >= max_rows) continue;
+        const float w = __ldg(topk_w + t * k + j);
+        const uint4 o = ld_nc_v4(eo + static_cast<size_t>(row) * nv + v);
+        const uint32_t ow[4] = {o.x, o.y, o.z, o.w};
+        uint32_t pk[4];
+        float acc = dot[j];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float g0 = bf16_lo(gw[q]), g1 = bf16_hi(gw[q]);
+          acc = fmaf(g0, bf16_lo(ow[q]), acc);
+          acc = fmaf(g1, bf16_hi(ow[q]), acc);
+          pk[q] = pack_bf16x2(__fmul_rn(w, g0), __fmul_rn(w, g1));
+        }
+        dot[j] = acc;
+        d_eo[static_cast<size_t>(row) * nv + v] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+    }
+    // d_w in every lane (butterfly sums), then the softmax backward
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      if (j >= k) break;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) dot[j] += __shfl_xor_sync(0xFFFFFFFFu, dot[j], o);
+      const int row = __ldg(slot_row + t * k + j);
+      if (row < 0 || row >= max_rows) dot[j] = 0.0f;
+    }
+    if (lane == 0) {
+      for (int j = 0; j < k; ++j) {
+        d_w[t * k + j] = dot[j];
+        ones[t * k + j] = 1.0f;
+      }
+    }
+    float* dl = d_logits + static_cast<size_t>(t) * E;
+    if (renormalize) {
+      float c = 0.0f;
+      for (int j = 0; j < k; ++j) c = fmaf(__ldg(topk_w + t * k + j), dot[j], c);
+      for (int e = lane; e < E; e += 32) dl[e] = 0.0f;
+      __syncwarp();
+      if (lane == 0)
+        for (int j = 0; j < k; ++j)
+          dl[__ldg(topk_idx + t * k + j)] = __ldg(topk_w + t * k + j) * (dot[j] - c);
+    } else {
+      // p = softmax over all E logits; d_e = d_w of the slot that selected e, else 0
+      const float* lg = logits + static_cast<size_t>(t) * E;
+      float mx = -INFINITY;
+      for (int e = lane; e < E; e += 32) mx = fmaxf(mx, __ldg(lg + e));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+      float sum = 0.0f, pd = 0.0f;
+      for (int e = lane; e < E; e += 32) {
+        const float p = expf(__ldg(lg + e) - mx);
+        sum += p;
+        for (int j = 0; j < k; ++j)
+          if (__ldg(topk_idx + t * k + j) == e) pd += p * dot[j];
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+        pd += __shfl_xor_sync(0xFFFFFFFFu, pd, o);
+      }
+      const float c = pd / sum;
+      for (int e = lane; e < E; e += 32) {
+        const float p = expf(__ldg(lg + e) - mx) / sum;
+        float d = 0.0f;
+        for (int j = 0; j < k; ++j)
+          if (__ldg(topk_idx + t * k + j) == e) d = dot[j];
+        dl[e] = p * (d - c);
+      }
+    }
+  }
+}
+
+// ---- host ---------------------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// bf16 [rows, cols] (cols contiguous), boxes of 64 columns x box_rows rows, 128-byte swizzle,
+// out-of-range elements read as zero.
+bool tmap_bf16(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64u, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE>
+size_t bwd_smem() {
+  return 1024 + static_cast<size_t>(Cfg<MODE>::kStages) * Cfg<MODE>::kStageBytes + 256 +
+         4 * (3 * 1024 + 1);
+}
+
+template <int MODE>
+cudaError_t launch_bwd_gemm(const BwdMaps& maps, const BwdArgs& a, cudaStream_t s) {
+  const size_t smem = bwd_smem<MODE>();
+  static int configured[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(bwd_gemm_kernel<MODE>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    configured[dev] = 1;
+  }
+  return launch_pdl(bwd_gemm_kernel<MODE>, dim3(num_sms()), dim3(kBwdThreads), smem, s, maps, a);
+}
+
+}  // namespace
+
+size_t backward_workspace_bytes(int max_rows, int T, int k, int H, int F) {
+  const size_t r = static_cast<size_t>(max_rows > 0 ? max_rows : 1);
+  const size_t tk = static_cast<size_t>(T > 0 ? T : 1) * static_cast<size_t>(k > 0 ? k : 1);
+  auto up = [](size_t b) { return (b + 255) / 256 * 256; };
+  // status | d_eo [r,H] | h, dg, du [r,F] | dx_rows [r,H] | ones [T,k]
+  return 256 + up(r * H * 2) + 3 * up(r * F * 2) + up(r * H * 2) + up(tk * 4);
+}
+
+cudaError_t launch_backward(const void* dy, int T, int H, int k, int E, int F, const float* logits,
+                            int renormalize, const int32_t* topk_idx, const float* topk_w,
+                            const int32_t* slot_row, const int32_t* expert_offsets, int max_rows,
+                            const void* ffn_input, const void* expert_out, const void* w_gate,
+                            const void* w_up, const void* w_down, void* dx, float* d_logits,
+                            float* d_topk_w, float* d_w_gate, float* d_w_up, float* d_w_down,
+                            void* ws, cudaStream_t s) {
+  auto up = [](size_t b) { return (b + 255) / 256 * 256; };
+  const size_t r = static_cast<size_t>(max_rows > 0 ? max_rows : 1);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  int* status = reinterpret_cast<int*>(w);
+  uint8_t* p = w + 256;
+  void* d_eo = p;     p += up(r * H * 2);
+  void* h = p;        p += up(r * F * 2);
+  void* dg = p;       p += up(r * F * 2);
+  void* du = p;       p += up(r * F * 2);
+  void* dx_rows = p;  p += up(r * H * 2);
+  float* ones = reinterpret_cast<float*>(p);
+  if (T == 0) return cudaSuccess;
+
+  {
+    int blocks = (T + 7) / 8;
+    if (blocks > 8 * num_sms()) blocks = 8 * num_sms();
+    const cudaError_t e = launch_pdl(
+        combine_bwd_kernel, dim3(blocks), dim3(256), 0, s, static_cast<const uint4*>(dy),
+        static_cast<const uint4*>(expert_out), max_rows, slot_row, topk_w, topk_idx, logits,
+        renormalize, T, k, E, H, static_cast<uint4*>(d_eo), d_topk_w, d_logits, ones);
+    if (e != cudaSuccess) return e;
+  }
+  BwdArgs a{expert_offsets, E, H, F, max_rows, nullptr, nullptr, nullptr, status};
+  BwdMaps m1{}, m2{}, m3{};
+  const uint64_t mr = static_cast<uint64_t>(max_rows);
+  if (!tmap_bf16(&m1.m[0], ffn_input, mr, H, 128) || !tmap_bf16(&m1.m[1], d_eo, mr, H, 128) ||
+      !tmap_bf16(&m1.m[2], w_gate, static_cast<uint64_t>(E) * F, H, 64) ||
+      !tmap_bf16(&m1.m[3], w_up, static_cast<uint64_t>(E) * F, H, 64) ||
+      !tmap_bf16(&m1.m[4], w_down, static_cast<uint64_t>(E) * H, F, 64))
+    return cudaErrorInvalidValue;
+  if (!tmap_bf16(&m2.m[0], dg, mr, F, 128) || !tmap_bf16(&m2.m[1], du, mr, F, 128) ||
+      !tmap_bf16(&m2.m[2], w_gate, static_cast<uint64_t>(E) * F, H, 64) ||
+      !tmap_bf16(&m2.m[3], w_up, static_cast<uint64_t>(E) * F, H, 64))
+    return cudaErrorInvalidValue;
+  if (!tmap_bf16(&m3.m[0], d_eo, mr, H, 64) || !tmap_bf16(&m3.m[1], dg, mr, F, 64) ||
+      !tmap_bf16(&m3.m[2], du, mr, F, 64) || !tmap_bf16(&m3.m[3], h, mr, F, 64) ||
+      !tmap_bf16(&m3.m[4], ffn_input, mr, H, 64))
+    return cudaErrorInvalidValue;
+  a.out0 = h;
+  a.out1 = dg;
+  a.out2 = du;
+  cudaError_t e = launch_bwd_gemm<kRecompute>(m1, a, s);
+  if (e != cudaSuccess) return e;
+  a.out0 = dx_rows;
+  a.out1 = a.out2 = nullptr;
+  e = launch_bwd_gemm<kInputGrad>(m2, a, s);
+  if (e != cudaSuccess) return e;
+  a.out0 = d_w_down;
+  a.out1 = d_w_gate;
+  a.out2 = d_w_up;
+  e = launch_bwd_gemm<kWeightGrad>(m3, a, s);
+  if (e != cudaSuccess) return e;
+  e = launch_combine(dx_rows, max_rows, slot_row, ones, T, k, H, dx, nullptr, s);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace moe

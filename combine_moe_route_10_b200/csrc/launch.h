@@ -92,6 +92,16 @@ cudaError_t ffn_weight_list_init(const void* const* w_gate, const void* const* w
                                  const void* const* w_down, int E, int H, int F, void* list,
                                  cudaStream_t s);
 
+// Backward of the layer (workspace: status | d_eo | h, dg, du | dx_rows | unit weights).
+size_t backward_workspace_bytes(int max_rows, int T, int k, int H, int F);
+cudaError_t launch_backward(const void* dy, int T, int H, int k, int E, int F, const float* logits,
+                            int renormalize, const int32_t* topk_idx, const float* topk_w,
+                            const int32_t* slot_row, const int32_t* expert_offsets, int max_rows,
+                            const void* ffn_input, const void* expert_out, const void* w_gate,
+                            const void* w_up, const void* w_down, void* dx, float* d_logits,
+                            float* d_topk_w, float* d_w_gate, float* d_w_up, float* d_w_down,
+                            void* ws, cudaStream_t s);
+
 // Rows between this rank's expert-major buffer and every source's packed buffer (peer pointers).
 cudaError_t launch_ep_exchange(const int32_t* all_counts, int R, int E, int rank, int push,
                                const unsigned long long* peer_rows,

@@ -207,6 +207,62 @@ class MoeShuffle:
                          self.topk_w if topk_w is None else topk_w, self.T, self.k, self.H,
                          self.y, None, stream)
 
+    # -- backward ------------------------------------------------------------------------------
+    def backward(self, dy, logits, w_gate, w_up, w_down, stream=None) -> dict:
+        """Gradients for the output gradient ``dy`` [T,H] bf16, after ``forward`` on the same
+        tensors (its routing, plan, FFN input rows and expert outputs are reused).  Returns a dict
+        of dx bf16 [T,H], d_logits fp32 [T,E], d_topk_w fp32 [T,k], d_w_gate / d_w_up fp32
+        [E,F,H], d_w_down fp32 [E,H,F] (buffers owned by this object, overwritten by the next
+        call)."""
+        bf16, f32 = torch.bfloat16, torch.float32
+        expect(dy, (self.T, self.H), bf16, "dy", self.device)
+        expect(logits, (self.T, self.E), f32, "logits", self.device)
+        expect(w_gate, (self.E, self.F, self.H), bf16, "w_gate", self.device)
+        expect(w_up, (self.E, self.F, self.H), bf16, "w_up", self.device)
+        expect(w_down, (self.E, self.H, self.F), bf16, "w_down", self.device)
+        if getattr(self, "grads", None) is None:
+            dev = self.device
+            self.grads = {
+                "dx": torch.empty((self.T, self.H), dtype=bf16, device=dev),
+                "d_logits": torch.empty((self.T, self.E), dtype=f32, device=dev),
+                "d_topk_w": torch.empty((self.T, self.k), dtype=f32, device=dev),
+                "d_w_gate": torch.empty((self.E, self.F, self.H), dtype=f32, device=dev),
+                "d_w_up": torch.empty((self.E, self.F, self.H), dtype=f32, device=dev),
+                "d_w_down": torch.empty((self.E, self.H, self.F), dtype=f32, device=dev),
+            }
+            n = _lib.moe_backward_workspace_size(self.max_rows, self.T, self.k, self.H, self.F)
+            self.ws_bwd = torch.zeros(n, dtype=torch.uint8, device=dev)
+        g = self.grads
+        ffn_input = self.send if not self.fp8 else self.dequantized_rows
+        _lib.moe_backward(dy, self.T, self.H, self.k, self.E, self.F, logits, self.renormalize,
+                          self.topk_idx, self.topk_w, self.slot_row, self.expert_offsets,
+                          self.max_rows, ffn_input, self.expert_out, w_gate, w_up, w_down,
+                          g["dx"], g["d_logits"], g["d_topk_w"], g["d_w_gate"], g["d_w_up"],
+                          g["d_w_down"], self.ws_bwd, self.ws_bwd.numel(), stream)
+        return g
+
+    def backward_intermediate(self, name: str) -> torch.Tensor:
+        """A view into the backward workspace: "d_eo", "dx_rows" [max_rows, H] or "h", "dg",
+        "du" [max_rows, F] (bf16), as the last ``backward`` left them."""
+        up = lambda b: (b + 255) // 256 * 256  # noqa: E731
+        r, H, F = max(self.max_rows, 1), self.H, self.F
+        sizes = [("d_eo", r * H * 2, H), ("h", r * F * 2, F), ("dg", r * F * 2, F),
+                 ("du", r * F * 2, F), ("dx_rows", r * H * 2, H)]
+        off = 256
+        for key, nbytes, cols in sizes:
+            if key == name:
+                return self.ws_bwd[off:off + nbytes].view(torch.bfloat16).view(r, cols)
+            off += up(nbytes)
+        raise KeyError(name)
+
+    @property
+    def dequantized_rows(self) -> torch.Tensor:
+        """The FP8 payload's bf16 FFN input rows [max_rows, H] (in the FFN workspace, after h)."""
+        up = lambda b: (b + 255) // 256 * 256  # noqa: E731
+        off = 256 + up(self.max_rows * self.F * 2)
+        n = self.max_rows * self.H * 2
+        return self.ws_ffn[off:off + n].view(torch.bfloat16).view(self.max_rows, self.H)
+
     def forward(self, logits, x, w_gate, w_up, w_down, stream=None) -> torch.Tensor:
         self.route(logits, stream)
         self.dispatch(x, stream=stream)

@@ -279,6 +279,38 @@ moe_status_t moe_combine(const void* expert_out, int max_rows, const int32_t* sl
                          moe_stream_t stream);
 
 /*
+ * moe_backward: gradients of the layer for an output gradient dy, reusing the forward's routing and
+ * plan (the NCCL EP page, section 3.2: the training step's backward dispatches the output gradient
+ * through the forward's handle to the experts, runs them backward, and combines the gradients).
+ *   1. combine backward, per kept slot (t, j) -> row: d_eo[row] = bf16(fp32(topk_w[t,j] * dy[t]))
+ *      and d_topk_w[t,j] = <dy[t], expert_out[row]> (0 for a dropped slot);
+ *   2. expert backward (tcgen05 GEMMs): g = x Wg^T, u = x Wu^T recomputed, dh = d_eo Wd,
+ *      dg = bf16(dh u s (1 + g (1 - s))), du = bf16(dh g s) with s = sigmoid(g),
+ *      dx_rows = bf16(dg Wg + du Wu), d_w_down = d_eo^T h, d_w_gate = dg^T x, d_w_up = du^T x
+ *      (fp32 accumulation; h = bf16(g s u) as in the forward);
+ *   3. dx[t] = bf16(sum over kept slots of dx_rows[slot_row[t,j]]), fp32 in slot order;
+ *   4. d_logits [T,E]: with renormalize, for a selected expert i: w_i (d_w_i - sum_j w_j d_w_j), 0
+ *      elsewhere; without, the full-E softmax backward p_e (d_e - sum p d) (logits needed).
+ * Inputs from the forward: topk_idx, topk_w, slot_row, expert_offsets (moe_route / moe_dispatch),
+ * ffn_input = the FFN's input rows bf16 [max_rows, H] (the send buffer for the bf16 payload; the
+ * dequantised rows of the FFN workspace for the FP8 payload), expert_out bf16 [max_rows, H]; the
+ * weights as for moe_expert_ffn.  Outputs (device, caller-owned): dx bf16 [T,H], d_logits fp32
+ * [T,E], d_topk_w fp32 [T,k], d_w_gate / d_w_up fp32 [E,F,H], d_w_down fp32 [E,H,F] (every element
+ * written, zeros for experts without rows).  ws: moe_backward_workspace_size bytes, 256-byte
+ * aligned; it holds [status | d_eo bf16 [max_rows,H] | h, dg, du bf16 [max_rows,F] | dx_rows bf16
+ * [max_rows,H] | unit weights fp32 [T,k]], each part 256-byte aligned.
+ * Limits: H % 64 == 0, F % 64 == 0 (MOE_ERR_UNSUPPORTED), k <= 32, E <= 1024, T*k <= max_rows.
+ */
+size_t moe_backward_workspace_size(int max_rows, int T, int k, int H, int F);
+moe_status_t moe_backward(const void* dy, int T, int H, int k, int E, int F, const float* logits,
+                          int renormalize, const int32_t* topk_idx, const float* topk_w,
+                          const int32_t* slot_row, const int32_t* expert_offsets, int max_rows,
+                          const void* ffn_input, const void* expert_out, const void* w_gate,
+                          const void* w_up, const void* w_down, void* dx, float* d_logits,
+                          float* d_topk_w, float* d_w_gate, float* d_w_up, float* d_w_down,
+                          void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * moe_ep_regroup: the row moves on both sides of an expert-parallel all-to-all, as one segmented
  * copy.
  *

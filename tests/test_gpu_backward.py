@@ -1,0 +1,108 @@
+"""The backward pass on the GPU through the C ABI (``moe_backward``) against the oracle's backward.
+
+The oracle is given the GPU forward's own routing, plan, FFN input rows and expert outputs, so the
+comparison covers the backward kernels alone: d_eo bit-exact (one fp32 product, one bf16 rounding),
+the unit-weight combine of dx_rows bit-exact, the recomputed h, dg, du, dx_rows and dx within the
+bf16 parity bar, the fp32 weight gradients, routing-weight and logit gradients within 1e-2 of the
+largest element.  Workloads: every small one (ragged F and H tails, the FP8 payload, capacity drops,
+E = 256 with k = 8), both weight modes, and an expert with no rows.
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs as mi
+from _helpers import (assert_close_bf16, bf16_values as bf16_vals, bits16, combine_magnitude,
+                      combine_row_atol, ffn_row_atol, np_)
+from oracle.numerics import bf16_bits as bits_of
+from oracle import moe
+
+pytestmark = pytest.mark.gpu
+
+
+def _rel_max(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    return float(np.max(np.abs(got - ref)) / max(np.max(np.abs(ref)), 1e-30))
+
+
+def _run(name, renormalize=True, seed=11, zero_expert=None):
+    from combine_moe_route_10_b200 import MoeShuffle
+    w = mi.get(name)
+    d = mi.make_inputs(w, seed=seed, device="cuda")
+    if zero_expert is not None:
+        d["logits"][:, zero_expert] = -1e4  # nobody routes here: an expert without rows
+    cap = moe.capacity(w.capacity_factor, w.T, w.k, w.E)
+    m = MoeShuffle(w.T, w.H, w.E, w.k, w.R, w.F, payload=w.payload, capacity=cap,
+                   renormalize=renormalize)
+    m.forward(d["logits"], d["x"], d["w_gate"], d["w_up"], d["w_down"])
+    g = torch.Generator(device="cuda").manual_seed(seed + 1)
+    dy = torch.randn((w.T, w.H), generator=g, device="cuda").to(torch.bfloat16)
+    grads = m.backward(dy, d["logits"], d["w_gate"], d["w_up"], d["w_down"])
+    torch.cuda.synchronize()
+    assert m.status() == 0
+    fp8 = w.payload == "fp8"
+    S = int(m.expert_offsets[w.E].item())
+    fwd = {"slot_row": np_(m.slot_row), "topk_w": np_(m.topk_w), "topk_idx": np_(m.topk_idx),
+           "expert_offsets": np_(m.expert_offsets), "expert_out": bits16(m.expert_out)[:S]}
+    if fp8:
+        fwd["send"] = np_(m.send.view(torch.uint8))[:S]
+        fwd["send_scales"] = np_(m.send_scales)[:S]
+    else:
+        fwd["send"] = bits16(m.send)[:S]
+        fwd["send_scales"] = None
+    ref = moe.backward(fwd, bits16(dy), np_(d["logits"]), bits16(d["w_gate"]), bits16(d["w_up"]),
+                       bits16(d["w_down"]), renormalize=renormalize, fp8=fp8)
+    return w, m, d, grads, ref, S
+
+
+def _check(w, m, m_w, grads, ref, S, what):
+    # 1. combine backward: one fp32 product and one bf16 rounding per element
+    assert np.array_equal(bits16(m.backward_intermediate("d_eo"))[:S], ref["d_eo"]), what
+    # 2. expert backward (fp32 accumulation on the tensor cores against fp64)
+    # the recomputed h against the forward's h (itself held to the oracle by the FFN tests)
+    assert_close_bf16(bits16(m.backward_intermediate("h"))[:S], bits16(m.h)[:S], f"{what} h")
+    for key in ("dg", "du"):
+        assert_close_bf16(bits16(m.backward_intermediate(key))[:S], ref[key], f"{what} {key}")
+    # dx_rows = dg Wg + du Wu: a one-ulp flip of a bf16 dg or du (fp32 against fp64 before the
+    # rounding) moves it by ulp * |W|, the same allowance as the forward's expert_out for h flips
+    dg_du = np.maximum(np.abs(bf16_vals(ref["dg"])), np.abs(bf16_vals(ref["du"])))
+    w_gu = torch.maximum(m_w["w_gate"].abs(), m_w["w_up"].abs())
+    dxr_atol = ffn_row_atol(bits_of(dg_du), np_(m.expert_offsets), w_gu)
+    assert_close_bf16(bits16(m.backward_intermediate("dx_rows"))[:S], ref["dx_rows"],
+                      f"{what} dx_rows", row_atol=dxr_atol)
+    # 3. dx: the unit-weight combine of the GPU's own dx_rows is bit-exact
+    dx_rows = bits16(m.backward_intermediate("dx_rows"))
+    comb = moe.combine(dx_rows, np_(m.slot_row), np.ones((w.T, w.k), np.float32), w.T, w.H)
+    assert np.array_equal(bits16(grads["dx"]), comb), what
+    # dx sums k rows that may cancel: its elements are held to the size of their summands, as
+    # the forward's combine output is
+    ones = np.ones((w.T, w.k), np.float32)
+    assert_close_bf16(bits16(grads["dx"]), ref["dx"], f"{what} dx",
+                      combine_magnitude(ref["dx_rows"], np_(m.slot_row), ones),
+                      combine_row_atol(ref["dx_rows"], np_(m.slot_row), ones, dxr_atol))
+    # 4. fp32 gradients
+    for key in ("d_w_gate", "d_w_up", "d_w_down"):
+        assert _rel_max(np_(grads[key]), ref[key]) <= 1e-2, (what, key)
+    assert _rel_max(np_(grads["d_topk_w"]), ref["d_w"]) <= 1e-2, what
+    assert _rel_max(np_(grads["d_logits"]), ref["d_logits"]) <= 1e-2, what
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode-small", "train-small", "skewed-small",
+                                  "finegrained-small"])
+def test_backward_matches_oracle(cuda, name):
+    w, m, d, grads, ref, S = _run(name)
+    _check(w, m, d, grads, ref, S, name)
+
+
+def test_backward_full_softmax_weights(cuda):
+    w, m, d, grads, ref, S = _run("train-small", renormalize=False)
+    _check(w, m, d, grads, ref, S, "train-small full softmax")
+
+
+def test_backward_expert_without_rows_gets_zero_weight_gradients(cuda):
+    w, m, d, grads, ref, S = _run("tiny", zero_expert=3)
+    assert int(m.expert_counts[3].item()) == 0
+    for key in ("d_w_gate", "d_w_up", "d_w_down"):
+        assert float(grads[key][3].abs().max().item()) == 0.0, key
+    _check(w, m, d, grads, ref, S, "tiny, expert 3 idle")
