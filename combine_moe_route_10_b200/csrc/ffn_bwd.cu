@@ -6,8 +6,9 @@
 //      the routing-weight gradient d_w[t,j] = <dy[t], eo[row]>, and from it the router's logit
 //      gradient (softmax backward over the selected k, or over all E without renormalisation).
 //   2. bwd_gemm_kernel<kRecompute> (tcgen05, M = 128 rows, 64 h columns): recomputes g = x Wg^T and
-//      u = x Wu^T and computes dh = d_eo Wd in the same K loop over H (three TMEM accumulators; Wd
-//      is read MN-major), then the SwiGLU backward in the epilogue: h, dg, du (bf16).
+//      u = x Wu^T (one N = 128 MMA over the stacked gate and up rows) and computes dh = d_eo Wd
+//      (Wd read MN-major) in the same K loop over H, then the SwiGLU backward in the epilogue:
+//      h, dg, du (bf16).
 //   3. bwd_gemm_kernel<kInputGrad> (M = 128, N = 256): dx_rows = dg Wg + du Wu, one K loop over
 //      2F, the weights read MN-major.
 //   4. bwd_gemm_kernel<kWeightGrad> (M = 128, N = 256, K = the expert's rows): dWd = d_eo^T h,
@@ -158,12 +159,19 @@ __device__ __forceinline__ Tile decode(const BwdArgs& a, const int* start, int t
   t.p = MODE == kWeightGrad ? lo / a.E : 0;
   t.e = MODE == kWeightGrad ? lo % a.E : lo;
   const int local = tile - start[lo];
-  int ncol;
-  if (MODE == kRecompute) ncol = a.F / kNF1;
-  else if (MODE == kInputGrad) ncol = (a.H + kNOut - 1) / kNOut;
-  else ncol = ((t.p == 0 ? a.F : a.H) + kNOut - 1) / kNOut;
-  t.mb = local / ncol;
-  t.nb = local % ncol;
+  if (MODE == kWeightGrad) {
+    // both operands (the expert's rows) stay in L2 across the output blocks
+    const int ncol = ((t.p == 0 ? a.F : a.H) + kNOut - 1) / kNOut;
+    t.mb = local / ncol;
+    t.nb = local % ncol;
+  } else {
+    // row blocks fastest: the tiles running at the same time share one weight slice, which then
+    // crosses HBM once per expert instead of once per row block
+    const int rows = __ldg(a.expert_offsets + t.e + 1) - __ldg(a.expert_offsets + t.e);
+    const int nrow = (rows + kBM - 1) / kBM;
+    t.mb = local % nrow;
+    t.nb = local / nrow;
+  }
   return t;
 }
 
@@ -174,10 +182,28 @@ __device__ __forceinline__ int k_blocks(const BwdArgs& a, int rows) {
   return (rows + kBK - 1) / kBK;
 }
 
-// Operand maps of a mode (unused ones are zero).
+// Operand maps of a mode (unused ones are zero); the weight-gradient mode also gets the three
+// output maps (fp32 [E][M][N], 32 x 32 boxes with the 128-byte swizzle) for its TMA stores.
 struct BwdMaps {
   CUtensorMap m[6];
+  CUtensorMap out[3];
 };
+constexpr int kStageOutBytes = 32 * 32 * 4;  // one epilogue warp's 32 x 32 fp32 block
+
+__device__ __forceinline__ void tma_store3d(const CUtensorMap* tm, uint32_t src, int x, int y,
+                                            int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(tm)),
+      "r"(src), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// The shared-memory source of every store issued so far has been read.
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 template <int MODE>
 __global__ void __launch_bounds__(kBwdThreads, 1)
@@ -188,7 +214,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   // 1024-byte aligned stages, then barriers, then the tile prefix table
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + kStages * kStageBytes);
+  constexpr int kOutBytes = MODE == kWeightGrad ? 4 * kStageOutBytes : 0;
+  uint8_t* out_stage = base + kStages * kStageBytes;  // 1024-aligned: [4 warps][32 x 32 fp32]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(out_stage + kOutBytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + kStages;
   uint64_t* acc_full = bars + 2 * kStages;
@@ -357,11 +385,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           for (int kk = 0; kk < kBK / kUK; ++kk) {
             const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
             if (MODE == kRecompute) {
-              constexpr uint32_t iK = idesc_bf16(kBM, kNF1, 0, 0), iMN = idesc_bf16(kBM, kNF1, 0, 1);
-              const uint64_t ax = desc_k(a + kk * 32), ae = desc_k(a + 16384 + kk * 32);
-              mma(d, ax, desc_k(a + 32768 + kk * 32), iK, accum);            // g
-              mma(d + 64, ax, desc_k(a + 40960 + kk * 32), iK, accum);       // u
-              mma(d + 128, ae, desc_mn(a + 49152 + kk * 2048, 8192), iMN, accum);  // dh
+              // the Wg and Wu boxes are adjacent: one N = 128 operand of 128 K-major rows gives
+              // g in accumulator columns 0..63 and u in 64..127
+              constexpr uint32_t iGU = idesc_bf16(kBM, 2 * kNF1, 0, 0);
+              constexpr uint32_t iMN = idesc_bf16(kBM, kNF1, 0, 1);
+              mma(d, desc_k(a + kk * 32), desc_k(a + 32768 + kk * 32), iGU, accum);       // g | u
+              mma(d + 128, desc_k(a + 16384 + kk * 32), desc_mn(a + 49152 + kk * 2048, 8192), iMN,
+                  accum);                                                                  // dh
             } else if (MODE == kInputGrad) {
               constexpr uint32_t iMN = idesc_bf16(kBM, kNOut, 0, 1);
               mma(d, desc_k(a + kk * 32), desc_mn(a + 16384 + kk * 2048, 8192), iMN, accum);
@@ -470,11 +500,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
         }
       } else {
-        const int M = t.p == 0 ? args.H : args.F, N = t.p == 0 ? args.F : args.H;
-        const int m = t.mb * kBM + r;
-        float* out = static_cast<float*>(t.p == 0 ? args.out0 : (t.p == 1 ? args.out1 : args.out2));
-        const size_t row = static_cast<size_t>(t.e) * M + m;
+        // each 32 x 32 block: TMEM -> registers (lane = row) -> this warp's staging block in the
+        // 128-byte swizzled layout -> one TMA store (rows past M and columns past N are clipped)
+        const int N = t.p == 0 ? args.F : args.H;
+        const CUtensorMap* om = &maps.out[t.p];
         const bool any_k = rows > 0;  // uniform over the warp
+        uint8_t* stg = out_stage + quarter * kStageOutBytes;
+        const uint32_t stg_addr = smem_addr(stg);
 #pragma unroll 1
         for (int c = 0; c < kNOut; c += 32) {
           const int col = t.nb * kNOut + c;
@@ -487,10 +519,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
             for (int q = 0; q < 32; ++q) v[q] = 0u;
           }
-          if (m < M) {
-            uint4* p = reinterpret_cast<uint4*>(out + row * N + col);
+          // the previous block's store has read the staging block
+          if (lane == 0) bulk_wait_read();
+          __syncwarp();
+          uint4* row_p = reinterpret_cast<uint4*>(stg + lane * 128);
 #pragma unroll
-            for (int q = 0; q < 8; ++q) p[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          for (int q = 0; q < 8; ++q)
+            row_p[q ^ (lane & 7)] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) {
+            tma_store3d(om, stg_addr, col, t.mb * kBM + quarter * 32, t.e);
+            bulk_commit();
           }
         }
       }
@@ -500,6 +540,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   }
 
+  if (MODE == kWeightGrad && warp >= 2 && lane == 0) bulk_wait_all();
   fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -526,22 +567,24 @@ __global__ void __launch_bounds__(256)
   const int lane = threadIdx.x & 31;
   const int nv = H / 8;
   for (int t = blockIdx.x * 8 + (threadIdx.x >> 5); t < T; t += gridDim.x * 8) {
-    float dot[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) dot[j] = 0.0f;
-    for (int v = lane; v < nv; v += 32) {
-      const uint4 g = ld_nc_v4(dy + static_cast<size_t>(t) * nv + v);
-      const uint32_t gw[4] = {g.x, g.y, g.z, g.w};
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        if (j >= k) break;
-        const int row = __ldg(slot_row + t * k + j);
-        if (row < 0 || row >= max_rows) continue;
-        const float w = __ldg(topk_w + t * k + j);
-        const uint4 o = ld_nc_v4(eo + static_cast<size_t>(row) * nv + v);
-        const uint32_t ow[4] = {o.x, o.y, o.z, o.w};
+    // slot j's routing data and, after its pass over H, its d_w live in lane j
+    const int my_row = lane < k ? __ldg(slot_row + t * k + lane) : -1;
+    const float my_w = lane < k ? __ldg(topk_w + t * k + lane) : 0.0f;
+    const int my_e = lane < k ? __ldg(topk_idx + t * k + lane) : -1;
+    float my_dw = 0.0f;
+    const uint4* dy_row = dy + static_cast<size_t>(t) * nv;
+    for (int j = 0; j < k; ++j) {
+      const int row = __shfl_sync(0xFFFFFFFFu, my_row, j);
+      if (row < 0 || row >= max_rows) continue;  // uniform over the warp
+      const float w = __shfl_sync(0xFFFFFFFFu, my_w, j);
+      const uint4* eo_row = eo + static_cast<size_t>(row) * nv;
+      uint4* de_row = d_eo + static_cast<size_t>(row) * nv;
+      float acc = 0.0f;
+      for (int v = lane; v < nv; v += 32) {
+        const uint4 g = ld_nc_v4(dy_row + v);  // the token's row: from L1 / L2 after the first slot
+        const uint4 o = ld_nc_v4(eo_row + v);
+        const uint32_t gw[4] = {g.x, g.y, g.z, g.w}, ow[4] = {o.x, o.y, o.z, o.w};
         uint32_t pk[4];
-        float acc = dot[j];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const float g0 = bf16_lo(gw[q]), g1 = bf16_hi(gw[q]);
@@ -549,34 +592,25 @@ __global__ void __launch_bounds__(256)
           acc = fmaf(g1, bf16_hi(ow[q]), acc);
           pk[q] = pack_bf16x2(__fmul_rn(w, g0), __fmul_rn(w, g1));
         }
-        dot[j] = acc;
-        d_eo[static_cast<size_t>(row) * nv + v] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        st_cs_v4(de_row + v, make_uint4(pk[0], pk[1], pk[2], pk[3]));
       }
-    }
-    // d_w in every lane (butterfly sums), then the softmax backward
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      if (j >= k) break;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) dot[j] += __shfl_xor_sync(0xFFFFFFFFu, dot[j], o);
-      const int row = __ldg(slot_row + t * k + j);
-      if (row < 0 || row >= max_rows) dot[j] = 0.0f;
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+      if (lane == j) my_dw = acc;
     }
-    if (lane == 0) {
-      for (int j = 0; j < k; ++j) {
-        d_w[t * k + j] = dot[j];
-        ones[t * k + j] = 1.0f;
-      }
+    if (lane < k) {
+      d_w[t * k + lane] = my_dw;
+      ones[t * k + lane] = 1.0f;
     }
     float* dl = d_logits + static_cast<size_t>(t) * E;
     if (renormalize) {
-      float c = 0.0f;
-      for (int j = 0; j < k; ++j) c = fmaf(__ldg(topk_w + t * k + j), dot[j], c);
+      // d_logits[e_j] = w_j (d_w_j - sum_i w_i d_w_i); the other experts get 0
+      float c = my_w * my_dw;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xFFFFFFFFu, c, o);
       for (int e = lane; e < E; e += 32) dl[e] = 0.0f;
       __syncwarp();
-      if (lane == 0)
-        for (int j = 0; j < k; ++j)
-          dl[__ldg(topk_idx + t * k + j)] = __ldg(topk_w + t * k + j) * (dot[j] - c);
+      if (lane < k) dl[my_e] = my_w * (my_dw - c);
     } else {
       // p = softmax over all E logits; d_e = d_w of the slot that selected e, else 0
       const float* lg = logits + static_cast<size_t>(t) * E;
@@ -584,25 +618,19 @@ __global__ void __launch_bounds__(256)
       for (int e = lane; e < E; e += 32) mx = fmaxf(mx, __ldg(lg + e));
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-      float sum = 0.0f, pd = 0.0f;
-      for (int e = lane; e < E; e += 32) {
-        const float p = expf(__ldg(lg + e) - mx);
-        sum += p;
-        for (int j = 0; j < k; ++j)
-          if (__ldg(topk_idx + t * k + j) == e) pd += p * dot[j];
-      }
+      float sum = 0.0f;
+      for (int e = lane; e < E; e += 32) sum += expf(__ldg(lg + e) - mx);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
-        pd += __shfl_xor_sync(0xFFFFFFFFu, pd, o);
-      }
-      const float c = pd / sum;
-      for (int e = lane; e < E; e += 32) {
-        const float p = expf(__ldg(lg + e) - mx) / sum;
-        float d = 0.0f;
-        for (int j = 0; j < k; ++j)
-          if (__ldg(topk_idx + t * k + j) == e) d = dot[j];
-        dl[e] = p * (d - c);
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+      // sum_e p_e d_e over the selected experts only (d is 0 elsewhere)
+      float pd = lane < k ? expf(__ldg(lg + my_e) - mx) / sum * my_dw : 0.0f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) pd += __shfl_xor_sync(0xFFFFFFFFu, pd, o);
+      for (int e = lane; e < E; e += 32) dl[e] = -(expf(__ldg(lg + e) - mx) / sum) * pd;
+      __syncwarp();
+      if (lane < k) {
+        const float p = expf(__ldg(lg + my_e) - mx) / sum;
+        dl[my_e] = p * (my_dw - pd);
       }
     }
   }
@@ -638,8 +666,22 @@ bool tmap_bf16(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t cols, u
 
 template <int MODE>
 size_t bwd_smem() {
-  return 1024 + static_cast<size_t>(Cfg<MODE>::kStages) * Cfg<MODE>::kStageBytes + 256 +
-         4 * (3 * 1024 + 1);
+  return 1024 + static_cast<size_t>(Cfg<MODE>::kStages) * Cfg<MODE>::kStageBytes +
+         (MODE == kWeightGrad ? 4 * kStageOutBytes : 0) + 256 + 4 * (3 * 1024 + 1);
+}
+
+// fp32 [E][M][N] (N contiguous) written in 32 x 32 boxes from a 128-byte-swizzled staging block;
+// elements outside [E][M][N] are not written.
+bool tmap_f32_out(CUtensorMap* tm, void* ptr, uint64_t E, uint64_t M, uint64_t N) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {N, M, E};
+  cuuint64_t strides[2] = {N * 4, M * N * 4};
+  cuuint32_t box[3] = {32u, 32u, 1u};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int MODE>
@@ -711,7 +753,9 @@ cudaError_t launch_backward(const void* dy, int T, int H, int k, int E, int F, c
     return cudaErrorInvalidValue;
   if (!tmap_bf16(&m3.m[0], d_eo, mr, H, 64) || !tmap_bf16(&m3.m[1], dg, mr, F, 64) ||
       !tmap_bf16(&m3.m[2], du, mr, F, 64) || !tmap_bf16(&m3.m[3], h, mr, F, 64) ||
-      !tmap_bf16(&m3.m[4], ffn_input, mr, H, 64))
+      !tmap_bf16(&m3.m[4], ffn_input, mr, H, 64) ||
+      !tmap_f32_out(&m3.out[0], d_w_down, E, H, F) || !tmap_f32_out(&m3.out[1], d_w_gate, E, F, H) ||
+      !tmap_f32_out(&m3.out[2], d_w_up, E, F, H))
     return cudaErrorInvalidValue;
   a.out0 = h;
   a.out1 = dg;
