@@ -272,6 +272,7 @@ def main():
                     help="skip the extra timing of the step with FP8 gate / up weights")
     ap.add_argument("--e2e-eager", action="store_true",
                     help="end-to-end loop calls forward eagerly instead of replaying CUDA graphs")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward timing")
     ap.add_argument("--ep", action="store_true",
                     help="time the expert-parallel step across the ranks when N > 1 (always at N = 1)")
     ap.add_argument("--no-ep", action="store_true", help="skip the expert-parallel timing")
@@ -328,6 +329,7 @@ def main():
         "gpu_launches": head["gpu_launches"],
         "clocks": clocks,
         "fp8_weights": head.get("fp8_weights"),
+        "backward": head.get("backward"),
         "workloads": {n: {k: v for k, v in r.items() if k != "e2e"} for n, r in extra.items()},
         "workloads_note": "the other large workloads, each timed the same way in the same run "
                           "(own warm-up, L2 flush, metric and breakdown steps); gpu_launches counts "
@@ -472,9 +474,63 @@ def measure(w, args, dev, world: int, rank: int, e2e: bool) -> dict:
            "e2e": e2e_out}
     if not args.no_w8:
         out["fp8_weights"] = measure_w8(w, m, d, args, stream, flush_l2, world, dev, S, active, pk)
+    if not args.no_backward:
+        out["backward"] = measure_backward(w, m, d, args, stream, flush_l2, world, dev, S, pk)
     del m, d, flush, flush_rd
     torch.cuda.empty_cache()
     return out
+
+
+def measure_backward(w, m, d, args, stream, flush_l2, world, dev, S, pk) -> dict:
+    """The backward of the step (``moe_backward`` after the forward just timed, reusing its routing,
+    plan and expert outputs): K steps behind an L2 flush, CUDA events around each call, max over
+    ranks.  Tensor work 16 S H F flops (the recompute of g and u, dh, dx_rows and the three weight
+    gradients); bytes: the weights read once, the fp32 weight gradients of all E experts written
+    once, dy and the expert outputs read and dx written once (the gradient rows the kernels hand
+    to each other are this implementation's own traffic)."""
+    import torch.distributed as dist
+    g = torch.Generator(device=dev).manual_seed(7)
+    dy = torch.randn((w.T, w.H), generator=g, device=dev).to(torch.bfloat16)
+
+    def step():
+        m.backward(dy, d["logits"], d["w_gate"], d["w_up"], d["w_down"])
+
+    for _ in range(args.warmup):
+        flush_l2()
+        step()
+    torch.cuda.synchronize()
+    if m.status() != 0:
+        raise SystemExit(f"{w.name}: device status after the backward warm-up")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for a, b in ev:
+        flush_l2()
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), dev) / args.steps
+    if m.status() != 0:
+        raise SystemExit(f"{w.name}: device status after the backward timing")
+    flops = 16.0 * S * w.H * w.F
+    bytes_ = (3.0 * w.E * w.H * w.F * (2 + 4)            # weights read, fp32 gradients written
+              + w.T * w.H * 2 * 2 + S * w.H * 2 * 2)     # dy, dx; expert outputs, FFN input rows
+    t_tc = flops / (pk["bf16_tflops_sustained"] * 1e12)
+    t_hbm = bytes_ / (pk["hbm_gbs"] * 1e9)
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"ms": ms, "tokens_per_s": w.T / (ms * 1e-3), "TFLOP/s": tf,
+            "frac_tensor": tf / pk["bf16_tflops_sustained"],
+            "GB/s_algorithmic": bytes_ / (ms * 1e-3) / 1e9,
+            "bound": "tensor" if t_tc >= t_hbm else "hbm",
+            "frac_of_max_time_bound": max(t_tc, t_hbm) / (ms * 1e-3),
+            "algorithmic_flops": flops, "algorithmic_bytes": bytes_,
+            "kernels": "combine_bwd_kernel, bwd_gemm_kernel<recompute g|u + dh + SwiGLU backward>, "
+                       "bwd_gemm_kernel<dx_rows>, bwd_gemm_kernel<dW, TMA-store epilogue>, "
+                       "combine_kernel (unit weights) = moe_backward",
+            "gpu_launches_per_step": 5}
 
 
 def measure_ep(w, args, dev, world: int, rank: int) -> dict:

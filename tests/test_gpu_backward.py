@@ -106,3 +106,86 @@ def test_backward_expert_without_rows_gets_zero_weight_gradients(cuda):
     for key in ("d_w_gate", "d_w_up", "d_w_down"):
         assert float(grads[key][3].abs().max().item()) == 0.0, key
     _check(w, m, d, grads, ref, S, "tiny, expert 3 idle")
+
+
+def _sub_problem(m, w, e, S):
+    """The forward restricted to expert e's rows: its tokens' slots that landed in e (the others
+    dropped), expert offsets [0, n], as the oracle's backward takes them."""
+    off = np_(m.expert_offsets)
+    lo, hi = int(off[e]), int(off[e + 1])
+    sr = np_(m.slot_row).astype(np.int64)
+    keep = (sr >= lo) & (sr < hi)
+    toks = np.unique(np.nonzero(keep)[0])
+    sub_sr = np.where(keep[toks], sr[toks] - lo, -1).astype(np.int32)
+    return lo, hi, toks, sub_sr
+
+
+@pytest.mark.parametrize("name", ["train", "skewed", "finegrained"])
+def test_backward_full_size(cuda, name):
+    """Full size, as the benchmark runs it: d_eo bit-exact on every row, d_topk_w and d_logits on
+    every token, dx bit-exact against the unit-weight combine of the GPU's dx_rows on every token,
+    and for two whole experts (the smallest and the largest of at most 1024 rows) the oracle's
+    backward on their rows: dg, du, dx_rows and the three weight-gradient matrices."""
+    from combine_moe_route_10_b200 import MoeShuffle
+    w = mi.get(name)
+    d = mi.make_inputs(w, seed=0, device="cuda")
+    cap = moe.capacity(w.capacity_factor, w.T, w.k, w.E)
+    m = MoeShuffle(w.T, w.H, w.E, w.k, w.R, w.F, payload=w.payload, capacity=cap)
+    m.forward(d["logits"], d["x"], d["w_gate"], d["w_up"], d["w_down"])
+    g = torch.Generator(device="cuda").manual_seed(5)
+    dy = torch.randn((w.T, w.H), generator=g, device="cuda").to(torch.bfloat16)
+    grads = m.backward(dy, d["logits"], d["w_gate"], d["w_up"], d["w_down"])
+    torch.cuda.synchronize()
+    assert m.status() == 0
+    fp8 = w.payload == "fp8"
+    S = int(m.expert_offsets[w.E].item())
+    sr = np_(m.slot_row).astype(np.int64)
+    tw = np_(m.topk_w)
+    dyf = np_(dy.float())
+    eo = np_(m.expert_out[:S].float()).astype(np.float64)
+    # every row: d_eo = bf16(fp32(w) * fp32(dy)); every slot: d_w = <dy, eo>
+    d_eo = bits16(m.backward_intermediate("d_eo"))[:S]
+    d_w_ref = np.zeros(sr.shape)
+    for j in range(w.k):
+        ok = sr[:, j] >= 0
+        rows = sr[ok, j]
+        prod = (tw[ok, j][:, None].astype(np.float32) * dyf[ok]).astype(np.float32)
+        assert np.array_equal(d_eo[rows], bits_of(prod.astype(np.float64))), (name, j)
+        d_w_ref[ok, j] = np.einsum("th,th->t", dyf[ok].astype(np.float64), eo[rows])
+    assert _rel_max(np_(grads["d_topk_w"]), d_w_ref) <= 1e-2, name
+    # d_logits from d_w (renormalised top-k softmax)
+    idx = np_(m.topk_idx).astype(np.int64)
+    dl_ref = np.zeros((w.T, w.E))
+    c = np.sum(tw * d_w_ref, axis=1)
+    np.put_along_axis(dl_ref, idx, tw * (d_w_ref - c[:, None]), axis=1)
+    assert _rel_max(np_(grads["d_logits"]), dl_ref) <= 1e-2, name
+    # dx: the unit-weight combine of the GPU's dx_rows, every token
+    dx_rows = bits16(m.backward_intermediate("dx_rows"))
+    comb = moe.combine(dx_rows, np_(m.slot_row), np.ones((w.T, w.k), np.float32), w.T, w.H)
+    assert np.array_equal(bits16(grads["dx"]), comb), name
+    # two whole experts through the oracle
+    counts = np.diff(np_(m.expert_offsets))
+    nz = np.nonzero(counts)[0]
+    small = int(nz[np.argmin(counts[nz])])
+    big_c = [e for e in nz if counts[e] <= 1024]
+    big = int(max(big_c, key=lambda e: counts[e]))
+    wb = [bits16(d[k_]) for k_ in ("w_gate", "w_up", "w_down")]
+    send_rows = (np_(m.send.view(torch.uint8)) if fp8 else bits16(m.send))
+    for e in sorted({small, big}):
+        lo, hi, toks, sub_sr = _sub_problem(m, w, e, S)
+        fwd = {"slot_row": sub_sr, "topk_w": tw[toks], "topk_idx": idx[toks].astype(np.int32),
+               "expert_offsets": np.array([0, hi - lo]), "expert_out": bits16(m.expert_out)[lo:hi],
+               "send": send_rows[lo:hi],
+               "send_scales": np_(m.send_scales)[lo:hi] if fp8 else None}
+        ref = moe.backward(fwd, bits16(dy)[toks], np_(d["logits"])[toks], wb[0][e:e + 1],
+                           wb[1][e:e + 1], wb[2][e:e + 1], fp8=fp8)
+        what = f"{name} expert {e} ({hi - lo} rows)"
+        assert np.array_equal(d_eo[lo:hi], ref["d_eo"]), what
+        for key in ("dg", "du"):
+            assert_close_bf16(bits16(m.backward_intermediate(key))[lo:hi], ref[key], f"{what} {key}")
+        dg_du = np.maximum(np.abs(bf16_vals(ref["dg"])), np.abs(bf16_vals(ref["du"])))
+        w_gu = torch.maximum(d["w_gate"][e:e + 1].abs(), d["w_up"][e:e + 1].abs())
+        dxr_atol = ffn_row_atol(bits_of(dg_du), np.array([0, hi - lo]), w_gu)
+        assert_close_bf16(dx_rows[lo:hi], ref["dx_rows"], f"{what} dx_rows", row_atol=dxr_atol)
+        for key in ("d_w_gate", "d_w_up", "d_w_down"):
+            assert _rel_max(np_(grads[key][e]), ref[key][0]) <= 1e-2, (what, key)
