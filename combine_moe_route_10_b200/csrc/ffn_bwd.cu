@@ -5,10 +5,10 @@
 //   1. combine_bwd_kernel (warp per token): d_eo[row] = bf16(w[t,j] * dy[t]) for every kept slot,
 //      the routing-weight gradient d_w[t,j] = <dy[t], eo[row]>, and from it the router's logit
 //      gradient (softmax backward over the selected k, or over all E without renormalisation).
-//   2. bwd_gemm_kernel<kRecompute> (tcgen05, M = 128 rows, 64 h columns): recomputes g = x Wg^T and
-//      u = x Wu^T (one N = 128 MMA over the stacked gate and up rows) and computes dh = d_eo Wd
-//      (Wd read MN-major) in the same K loop over H, then the SwiGLU backward in the epilogue:
-//      h, dg, du (bf16).
+//   2. bwd_gemm_kernel<kRecompute> (tcgen05, M = 128 rows, 128 h columns, k = 32 per stage with the
+//      64-byte swizzle): recomputes g = x Wg^T and u = x Wu^T (one N = 256 MMA over the stacked
+//      gate and up rows) and computes dh = d_eo Wd (N = 128, Wd read MN-major) in the same K loop
+//      over H, then the SwiGLU backward in the epilogue: h, dg, du (bf16).
 //   3. bwd_gemm_kernel<kInputGrad> (M = 128, N = 256): dx_rows = dg Wg + du Wu, one K loop over
 //      2F, the weights read MN-major.
 //   4. bwd_gemm_kernel<kWeightGrad> (M = 128, N = 256, K = the expert's rows): dWd = d_eo^T h,
@@ -35,16 +35,21 @@ constexpr int kUK = 16;
 constexpr int kBwdThreads = 192;
 constexpr int kTmemColsBwd = 512;
 constexpr int kAccStride = 256;  // TMEM columns between the two accumulators
-constexpr int kNF1 = 64;         // h columns per recompute tile
+constexpr int kNF1 = 128;        // h columns per recompute tile
+constexpr int kBK1 = 32;         // recompute: k per stage (64-byte rows, 64-byte swizzle)
 constexpr int kNOut = 256;       // output columns per input-gradient / weight-gradient tile
 
 enum Mode { kRecompute = 1, kInputGrad = 2, kWeightGrad = 3 };
 
 template <int MODE>
 struct Cfg {
-  // recompute: x + d_eo (16 KB each) + Wg, Wu, Wd^T (8 KB each); others: A 16 KB + B 32 KB
-  static constexpr int kStageBytes = MODE == kRecompute ? 2 * 16384 + 3 * 8192 : 16384 + 32768;
-  static constexpr int kStages = MODE == kRecompute ? 3 : 4;
+  // recompute: x, d_eo, Wg, Wu (128 rows x 32 k, 8 KB each) + Wd^T (32 k x 128 f, 8 KB): 40 KB;
+  // others: A 16 KB + B 32 KB
+  static constexpr int kStageBytes = MODE == kRecompute ? 5 * 8192 : 16384 + 32768;
+  static constexpr int kStages = MODE == kRecompute ? 5 : 4;
+  // the recompute's accumulators (g | u 256 columns, dh 128) fill one TMEM set; the others
+  // alternate between two so that an epilogue overlaps the next tile's MMAs
+  static constexpr int kAccBufs = MODE == kRecompute ? 1 : 2;
 };
 
 // ---- PTX wrappers -----------------------------------------------------------------------------
@@ -101,6 +106,13 @@ __device__ __forceinline__ uint64_t desc_k(uint32_t saddr) {
          (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
          (static_cast<uint64_t>(2) << 61);
 }
+// K-major tile with the 64-byte swizzle (layout type 4): rows of 64 bytes hold 32 k values, 8-row
+// groups 512 bytes apart.
+__device__ __forceinline__ uint64_t desc_k64(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>(1) << 16) |
+         (static_cast<uint64_t>(512 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
+         (static_cast<uint64_t>(4) << 61);
+}
 __device__ __forceinline__ uint64_t desc_mn(uint32_t saddr, uint32_t lbo) {
   return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) |
          (static_cast<uint64_t>(lbo >> 4) << 16) | (static_cast<uint64_t>(1024 >> 4) << 32) |
@@ -139,7 +151,7 @@ struct Tile {
 };
 template <int MODE>
 __device__ __forceinline__ int tiles_of(const BwdArgs& a, int rows, int p) {
-  if (MODE == kRecompute) return ((rows + kBM - 1) / kBM) * (a.F / kNF1);
+  if (MODE == kRecompute) return ((rows + kBM - 1) / kBM) * ((a.F + kNF1 - 1) / kNF1);
   if (MODE == kInputGrad) return ((rows + kBM - 1) / kBM) * ((a.H + kNOut - 1) / kNOut);
   // weight gradients: p = 0 dWd [H, F]; p = 1, 2 dWg, dWu [F, H]
   const int M = p == 0 ? a.H : a.F, N = p == 0 ? a.F : a.H;
@@ -177,7 +189,7 @@ __device__ __forceinline__ Tile decode(const BwdArgs& a, const int* start, int t
 
 template <int MODE>
 __device__ __forceinline__ int k_blocks(const BwdArgs& a, int rows) {
-  if (MODE == kRecompute) return a.H / kBK;
+  if (MODE == kRecompute) return a.H / kBK1;
   if (MODE == kInputGrad) return 2 * (a.F / kBK);
   return (rows + kBK - 1) / kBK;
 }
@@ -291,13 +303,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t fb = smem_addr(&full[stage]);
         if (MODE == kRecompute) {
           if (lane == 0) {
-            const int kx = kb * kBK, row0 = off + t.mb * kBM, f0 = t.nb * kNF1;
+            // 128 x 32 K-major boxes (64-byte swizzle); Wd as two 32 h x 64 f MN-major boxes.
+            // Gate / up rows past the expert's F (another expert's, or zero fill) only reach
+            // accumulator columns the epilogue does not store.
+            const int kx = kb * kBK1, row0 = off + t.mb * kBM, f0 = t.nb * kNF1;
             mbar_arrive_expect_tx(fb, kStageBytes);
-            tma2d(a, &maps.m[0], fb, kx, row0);                        // x rows (K-major)
-            tma2d(a + 16384, &maps.m[1], fb, kx, row0);                // d_eo rows (K-major)
-            tma2d(a + 32768, &maps.m[2], fb, kx, t.e * args.F + f0);   // Wg rows (K-major)
-            tma2d(a + 40960, &maps.m[3], fb, kx, t.e * args.F + f0);   // Wu rows (K-major)
-            tma2d(a + 49152, &maps.m[4], fb, f0, t.e * args.H + kx);   // Wd: 64 h x 64 f (MN-major)
+            tma2d(a, &maps.m[0], fb, kx, row0);                        // x rows
+            tma2d(a + 8192, &maps.m[1], fb, kx, row0);                 // d_eo rows
+            tma2d(a + 16384, &maps.m[2], fb, kx, t.e * args.F + f0);   // Wg rows
+            tma2d(a + 24576, &maps.m[3], fb, kx, t.e * args.F + f0);   // Wu rows
+            tma2d(a + 32768, &maps.m[4], fb, f0, t.e * args.H + kx);       // Wd f0 .. f0 + 63
+            tma2d(a + 36864, &maps.m[4], fb, f0 + 64, t.e * args.H + kx);  // Wd f0 + 64 ..
           }
         } else if (MODE == kInputGrad) {
           if (lane == 0) {
@@ -368,9 +384,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const Tile t = decode<MODE>(args, start, tile);
         const int rows = __ldg(args.expert_offsets + t.e + 1) - __ldg(args.expert_offsets + t.e);
         const int nkb = k_blocks<MODE>(args, rows);
-        const int acc = it & 1;
-        if (!bwait(smem_addr(&acc_empty[acc]), ((it >> 1) & 1) ^ 1u, abort_flag, args.status))
-          break;
+        constexpr int kBufs = Cfg<MODE>::kAccBufs;
+        const int acc = kBufs == 2 ? (it & 1) : 0;
+        const uint32_t acc_par = kBufs == 2 ? ((it >> 1) & 1) : (it & 1);
+        if (!bwait(smem_addr(&acc_empty[acc]), acc_par ^ 1u, abort_flag, args.status)) break;
         fence_after();
         const uint32_t d = tmem_base + acc * kAccStride;
         bool ok = true;
@@ -382,16 +399,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           fence_after();
           const uint32_t a = stage0 + stage * kStageBytes;
 #pragma unroll
-          for (int kk = 0; kk < kBK / kUK; ++kk) {
+          for (int kk = 0; kk < (MODE == kRecompute ? kBK1 : kBK) / kUK; ++kk) {
             const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
             if (MODE == kRecompute) {
-              // the Wg and Wu boxes are adjacent: one N = 128 operand of 128 K-major rows gives
-              // g in accumulator columns 0..63 and u in 64..127
+              // the Wg and Wu boxes are adjacent: one N = 256 operand of 256 K-major rows gives g
+              // in accumulator columns 0..127 and u in 128..255; dh in 256..383
               constexpr uint32_t iGU = idesc_bf16(kBM, 2 * kNF1, 0, 0);
               constexpr uint32_t iMN = idesc_bf16(kBM, kNF1, 0, 1);
-              mma(d, desc_k(a + kk * 32), desc_k(a + 32768 + kk * 32), iGU, accum);       // g | u
-              mma(d + 128, desc_k(a + 16384 + kk * 32), desc_mn(a + 49152 + kk * 2048, 8192), iMN,
-                  accum);                                                                  // dh
+              mma(d, desc_k64(a + kk * 32), desc_k64(a + 16384 + kk * 32), iGU, accum);  // g | u
+              mma(d + 256, desc_k64(a + 8192 + kk * 32), desc_mn(a + 32768 + kk * 2048, 4096),
+                  iMN, accum);                                                            // dh
             } else if (MODE == kInputGrad) {
               constexpr uint32_t iMN = idesc_bf16(kBM, kNOut, 0, 1);
               mma(d, desc_k(a + kk * 32), desc_mn(a + 16384 + kk * 2048, 8192), iMN, accum);
@@ -427,9 +444,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const Tile t = decode<MODE>(args, start, tile);
       const int off = __ldg(args.expert_offsets + t.e);
       const int rows = __ldg(args.expert_offsets + t.e + 1) - off;
-      const int acc = it & 1;
+      constexpr int kBufs = Cfg<MODE>::kAccBufs;
+      const int acc = kBufs == 2 ? (it & 1) : 0;
+      const uint32_t acc_par = kBufs == 2 ? ((it >> 1) & 1) : (it & 1);
       int ok = 1;
-      if (lane == 0) ok = bwait(smem_addr(&acc_full[acc]), (it >> 1) & 1, abort_flag, args.status);
+      if (lane == 0) ok = bwait(smem_addr(&acc_full[acc]), acc_par, abort_flag, args.status);
       if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) break;
       fence_after();
       const uint32_t tb = tmem_base + acc * kAccStride + (static_cast<uint32_t>(quarter * 32) << 16);
@@ -441,10 +460,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         __nv_bfloat16* du_out = static_cast<__nv_bfloat16*>(args.out2);
 #pragma unroll 1
         for (int c = 0; c < kNF1; c += 32) {
+          if (t.nb * kNF1 + c >= args.F) break;  // uniform over the warp
           uint32_t g[32], u[32], dh[32];
           ld32(tb + c, g);
-          ld32(tb + 64 + c, u);
-          ld32(tb + 128 + c, dh);
+          ld32(tb + kNF1 + c, u);
+          ld32(tb + 2 * kNF1 + c, dh);
           ld_wait();
           uint32_t ph[16], pg[16], pu[16];
 #pragma unroll
@@ -650,18 +670,21 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
   return fn;
 }
 
-// bf16 [rows, cols] (cols contiguous), boxes of 64 columns x box_rows rows, 128-byte swizzle,
-// out-of-range elements read as zero.
-bool tmap_bf16(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+// bf16 [rows, cols] (cols contiguous), boxes of box_cols (64: 128-byte swizzle; 32: 64-byte
+// swizzle) x box_rows, out-of-range elements read as zero.
+bool tmap_bf16(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows,
+               uint32_t box_cols = 64) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
   if (enc == nullptr) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {64u, box_rows};
+  cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle sw =
+      box_cols == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int MODE>
@@ -742,10 +765,11 @@ cudaError_t launch_backward(const void* dy, int T, int H, int k, int E, int F, c
   BwdArgs a{expert_offsets, E, H, F, max_rows, nullptr, nullptr, nullptr, status};
   BwdMaps m1{}, m2{}, m3{};
   const uint64_t mr = static_cast<uint64_t>(max_rows);
-  if (!tmap_bf16(&m1.m[0], ffn_input, mr, H, 128) || !tmap_bf16(&m1.m[1], d_eo, mr, H, 128) ||
-      !tmap_bf16(&m1.m[2], w_gate, static_cast<uint64_t>(E) * F, H, 64) ||
-      !tmap_bf16(&m1.m[3], w_up, static_cast<uint64_t>(E) * F, H, 64) ||
-      !tmap_bf16(&m1.m[4], w_down, static_cast<uint64_t>(E) * H, F, 64))
+  if (!tmap_bf16(&m1.m[0], ffn_input, mr, H, 128, 32) ||
+      !tmap_bf16(&m1.m[1], d_eo, mr, H, 128, 32) ||
+      !tmap_bf16(&m1.m[2], w_gate, static_cast<uint64_t>(E) * F, H, 128, 32) ||
+      !tmap_bf16(&m1.m[3], w_up, static_cast<uint64_t>(E) * F, H, 128, 32) ||
+      !tmap_bf16(&m1.m[4], w_down, static_cast<uint64_t>(E) * H, F, 32))
     return cudaErrorInvalidValue;
   if (!tmap_bf16(&m2.m[0], dg, mr, F, 128) || !tmap_bf16(&m2.m[1], du, mr, F, 128) ||
       !tmap_bf16(&m2.m[2], w_gate, static_cast<uint64_t>(E) * F, H, 64) ||

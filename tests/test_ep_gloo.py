@@ -115,3 +115,43 @@ def test_thread_loopback_matches_the_oracle_too():
             for mode in ("ht", "ll", "p2p"):
                 assert np.array_equal(res[r][mode], ref[r * T_RANK:(r + 1) * T_RANK]), \
                     (payload, mode, r)
+
+
+def _dying_rank_main(rank, world, port, out):
+    import datetime
+    from combine_moe_route_10_b200.ep import MoeEP, TorchComm
+    from _ep_oracle_ops import OracleOps
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world, timeout=datetime.timedelta(seconds=5))
+    w, lg, xs, d = _inputs(world, "bf16")
+    E_loc = w.E // world
+    sl = slice(rank * E_loc, (rank + 1) * E_loc)
+    ep = MoeEP(T_RANK, w.H, w.E, w.k, w.F, comm=TorchComm(), mode="ht", device="cpu",
+               ops=OracleOps())
+    if rank == world - 1:
+        out[rank] = "left"
+        return  # leaves between steps: never joins the exchange (its group is torn down at exit)
+    try:
+        ep.forward(lg[rank], xs[rank], d["w_gate"][sl].contiguous(), d["w_up"][sl].contiguous(),
+                   d["w_down"][sl].contiguous())
+        out[rank] = "no error"
+    except Exception as e:  # the collective ends with an error instead of waiting for good
+        out[rank] = f"error: {type(e).__name__}"
+
+
+def test_a_rank_that_leaves_ends_the_others_collectives_with_an_error():
+    """A rank that leaves before the exchange: the other ranks' next collective ends with an error
+    within the process group's timeout (a host-side failure; no device is involved)."""
+    world, port = 4, _free_port()
+    with mp.get_context("spawn").Manager() as m:
+        out = m.dict()
+        ctx = mp.start_processes(_dying_rank_main, args=(world, port, out), nprocs=world,
+                                 join=False, start_method="spawn")
+        import time
+        t0 = time.time()
+        while not ctx.join(timeout=1):
+            assert time.time() - t0 < 120, "ranks did not finish"
+        res = dict(out)
+    assert res[world - 1] == "left"
+    for r in range(world - 1):
+        assert res[r].startswith("error"), (r, res[r])
