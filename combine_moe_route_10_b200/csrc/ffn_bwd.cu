@@ -29,7 +29,8 @@
 namespace moe {
 namespace {
 
-constexpr int kBM = 128;
+constexpr int kBM = 128;         // rows of a tile held by one CTA of the pair (one TMEM lane each)
+constexpr int kPairM = 256;      // rows (or output rows) of a pair tile
 constexpr int kBK = 64;
 constexpr int kUK = 16;
 constexpr int kBwdThreads = 192;
@@ -41,18 +42,60 @@ constexpr int kNOut = 256;       // output columns per input-gradient / weight-g
 
 enum Mode { kRecompute = 1, kInputGrad = 2, kWeightGrad = 3 };
 
+// Per CTA of a pair: its own 128 rows of A and half of B.
 template <int MODE>
 struct Cfg {
-  // recompute: x, d_eo, Wg, Wu (128 rows x 32 k, 8 KB each) + Wd^T (32 k x 128 f, 8 KB): 40 KB;
-  // others: A 16 KB + B 32 KB
-  static constexpr int kStageBytes = MODE == kRecompute ? 5 * 8192 : 16384 + 32768;
-  static constexpr int kStages = MODE == kRecompute ? 5 : 4;
+  // recompute: x, d_eo (128 rows x 32 k, 8 KB each), the gate (CTA 0) or up (CTA 1) block of
+  // 128 rows x 32 k (8 KB), 64 f columns of Wd^T x 32 k (4 KB): 28 KB.  Others: A 16 KB + half of
+  // B 16 KB.
+  static constexpr int kStageBytes = MODE == kRecompute ? 3 * 8192 + 4096 : 16384 + 16384;
+  static constexpr int kStages = MODE == kRecompute ? 7 : 6;
   // the recompute's accumulators (g | u 256 columns, dh 128) fill one TMEM set; the others
   // alternate between two so that an epilogue overlaps the next tile's MMAs
   static constexpr int kAccBufs = MODE == kRecompute ? 1 : 2;
 };
 
 // ---- PTX wrappers -----------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cta_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Shared::cluster address of the same shared-memory offset in CTA `rank` of the pair.
+__device__ __forceinline__ uint32_t mapa(uint32_t local, uint32_t rank) {
+  uint32_t out;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(local), "r"(rank));
+  return out;
+}
+__device__ __forceinline__ void pair_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+// Count `bytes` of transactions done on the other CTA's mbarrier (a signal without an arrival).
+constexpr uint32_t kTailToken = 16;
+__device__ __forceinline__ void complete_tx_remote(uint32_t cluster_addr, uint32_t bytes) {
+  asm volatile("mbarrier.complete_tx.relaxed.cluster.shared::cluster.b64 [%0], %1;" ::"r"(
+                   cluster_addr),
+               "r"(bytes)
+               : "memory");
+}
+// Arrive on the other CTA's mbarrier, releasing this thread's prior writes at cluster scope.
+__device__ __forceinline__ void arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+__device__ __forceinline__ bool try_wait_cl(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// CTA 0's copy into its own shared memory, completing on its own barrier.
 __device__ __forceinline__ void tma2d(uint32_t dst, const CUtensorMap* tm, uint32_t bar, int x,
                                       int y) {
   asm volatile(
@@ -61,23 +104,41 @@ __device__ __forceinline__ void tma2d(uint32_t dst, const CUtensorMap* tm, uint3
       "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(bar)
       : "memory");
 }
+// CTA 1's copy into its own shared memory, completing its bytes on CTA 0's barrier `bar_cta0`
+// (a shared::cluster address); a plain, not multicast, load.
+__device__ __forceinline__ void tma2d_to_leader(uint32_t dst, const CUtensorMap* tm,
+                                                uint32_t bar_cta0, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(bar_cta0)
+      : "memory");
+}
 __device__ __forceinline__ void fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
 __device__ __forceinline__ void fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-__device__ __forceinline__ void commit(uint32_t bar) {
+// Arrive once on the mbarrier at this offset in BOTH CTAs when the MMAs issued so far complete.
+__device__ __forceinline__ void commit_both(uint32_t bar) {
   asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar),
+      "h"(static_cast<uint16_t>(3))
       : "memory");
+}
+__device__ __forceinline__ void commit_local(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
 }
 __device__ __forceinline__ void mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
                                     uint32_t acc) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
       "l"(a), "l"(b), "r"(idesc), "r"(acc)
       : "memory");
 }
@@ -96,18 +157,17 @@ __device__ __forceinline__ void ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 __device__ __forceinline__ void ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// Shared-memory descriptor of a bf16 tile with the 128-byte swizzle (layout type 2, version 1).
-// K-major: rows of 128 bytes hold 64 k values, 8-row groups 1024 bytes apart (stride byte offset;
-// the leading byte offset is unused).  MN-major: rows of 128 bytes hold 64 m (or n) values of one
-// k, 8-k groups 1024 bytes apart (stride byte offset), and the next 64 m values lie `lbo` bytes
-// further (the next TMA box: leading byte offset).
+// Shared-memory descriptors (version 1).  K-major, 128-byte swizzle (layout type 2): rows of 128
+// bytes hold 64 k values, 8-row groups 1024 bytes apart (stride byte offset; the leading byte offset
+// is unused).  K-major, 64-byte swizzle (layout type 4): rows of 64 bytes hold 32 k values, 8-row
+// groups 512 bytes apart.  MN-major, 128-byte swizzle: rows of 128 bytes hold 64 m (or n) values
+// of one k, 8-k groups 1024 bytes apart (stride byte offset), and the next 64 m values lie `lbo`
+// bytes further (the next TMA box: leading byte offset).
 __device__ __forceinline__ uint64_t desc_k(uint32_t saddr) {
   return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>(1) << 16) |
          (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
          (static_cast<uint64_t>(2) << 61);
 }
-// K-major tile with the 64-byte swizzle (layout type 4): rows of 64 bytes hold 32 k values, 8-row
-// groups 512 bytes apart.
 __device__ __forceinline__ uint64_t desc_k64(uint32_t saddr) {
   return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>(1) << 16) |
          (static_cast<uint64_t>(512 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
@@ -125,14 +185,26 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-__device__ __forceinline__ bool bwait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+// Bounded wait on a barrier phase (arrivals may come from either CTA of the pair).  False if this
+// CTA aborts or the limit runs out (which records kStatusTimeout and raises the abort).
+__device__ __forceinline__ bool cwait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                       int* status) {
-  return wait_phase(bar, parity, abort_flag, status);
-}
-// Wait for a barrier phase regardless of the abort flag (a CTA draining its own copies / MMAs).
-__device__ __forceinline__ void bdrain(uint32_t bar, uint32_t parity) {
+  if (try_wait_cl(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
-  while (!mbar_try_wait(bar, parity) && global_timer_ns() - t0 <= kWaitLimitNs) {
+  while (true) {
+    if (try_wait_cl(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      record_status(status, kStatusTimeout);
+      return false;
+    }
+  }
+}
+// The same wait regardless of the abort flag (a CTA draining its own copies / MMAs).
+__device__ __forceinline__ void cdrain(uint32_t bar, uint32_t parity) {
+  const unsigned long long t0 = global_timer_ns();
+  while (!try_wait_cl(bar, parity) && global_timer_ns() - t0 <= kWaitLimitNs) {
   }
 }
 
@@ -145,17 +217,17 @@ struct BwdArgs {
   int* status;
 };
 
-// Tiles of every expert (prefix in shared memory) and the decoding of a tile index.
+// Pair tiles of every item (prefix in shared memory) and the decoding of a tile index.
 struct Tile {
-  int e, p, mb, nb;  // expert, sub-problem (weight grad), row / output block, column block
+  int e, p, mb, nb;  // expert, sub-problem (weight grad), 256-row block, column block
 };
 template <int MODE>
 __device__ __forceinline__ int tiles_of(const BwdArgs& a, int rows, int p) {
-  if (MODE == kRecompute) return ((rows + kBM - 1) / kBM) * ((a.F + kNF1 - 1) / kNF1);
-  if (MODE == kInputGrad) return ((rows + kBM - 1) / kBM) * ((a.H + kNOut - 1) / kNOut);
+  if (MODE == kRecompute) return ((rows + kPairM - 1) / kPairM) * ((a.F + kNF1 - 1) / kNF1);
+  if (MODE == kInputGrad) return ((rows + kPairM - 1) / kPairM) * ((a.H + kNOut - 1) / kNOut);
   // weight gradients: p = 0 dWd [H, F]; p = 1, 2 dWg, dWu [F, H]
   const int M = p == 0 ? a.H : a.F, N = p == 0 ? a.F : a.H;
-  return ((M + kBM - 1) / kBM) * ((N + kNOut - 1) / kNOut);
+  return ((M + kPairM - 1) / kPairM) * ((N + kNOut - 1) / kNOut);
 }
 
 template <int MODE>
@@ -180,7 +252,7 @@ __device__ __forceinline__ Tile decode(const BwdArgs& a, const int* start, int t
     // row blocks fastest: the tiles running at the same time share one weight slice, which then
     // crosses HBM once per expert instead of once per row block
     const int rows = __ldg(a.expert_offsets + t.e + 1) - __ldg(a.expert_offsets + t.e);
-    const int nrow = (rows + kBM - 1) / kBM;
+    const int nrow = (rows + kPairM - 1) / kPairM;
     t.mb = local % nrow;
     t.nb = local / nrow;
   }
@@ -217,13 +289,17 @@ __device__ __forceinline__ void bulk_wait_read() {
 }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// One 2-CTA cluster per pair of SMs; both CTAs walk the same tile sequence.  CTA 0 (the leader)
+// owns the full and accumulator-empty barriers that count both CTAs, and its MMA thread issues
+// every MMA of the pair; each CTA's epilogue reads its own TMEM (its 128 rows).
 template <int MODE>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_gemm_kernel(const __grid_constant__ BwdMaps maps, const BwdArgs args) {
   constexpr int kStages = Cfg<MODE>::kStages;
   constexpr int kStageBytes = Cfg<MODE>::kStageBytes;
+  constexpr int kBufs = Cfg<MODE>::kAccBufs;
   extern __shared__ uint8_t smem_raw[];
-  // 1024-byte aligned stages, then barriers, then the tile prefix table
+  // 1024-byte aligned stages, then the store staging, barriers and the tile prefix table
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   constexpr int kOutBytes = MODE == kWeightGrad ? 4 * kStageOutBytes : 0;
@@ -239,28 +315,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* start = reinterpret_cast<int*>(tmem_slot + 4);  // [items + 1]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cta_rank();
   const int E = args.E;
   const int n_items = MODE == kWeightGrad ? 3 * E : E;
+  const int cid = static_cast<int>(blockIdx.x) >> 1, ncl = static_cast<int>(gridDim.x) >> 1;
 
   if (warp == 0 && lane == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(smem_addr(&full[i]), 1);
-      mbar_init(smem_addr(&empty[i]), 1);
+      mbar_init(smem_addr(&full[i]), 1);   // CTA 0's copy: its arrival + both CTAs' bytes
+      mbar_init(smem_addr(&empty[i]), 1);  // each CTA's own: the multicast commit
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_addr(&acc_full[i]), 1);
-      mbar_init(smem_addr(&acc_empty[i]), 4);
+      mbar_init(smem_addr(&acc_full[i]), 1);   // each CTA's own: the multicast commit
+      mbar_init(smem_addr(&acc_empty[i]), 8);  // CTA 0's copy: four epilogue warps of each CTA
     }
     mbar_init(smem_addr(fix_bar), 1);
     mbar_init(smem_addr(drain_bar), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   } else if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+    // the same warp of both CTAs allocates, as cta_group::2 requires
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_addr(tmem_slot)),
                  "r"(kTmemColsBwd)
                  : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
   griddep_wait();
   griddep_launch_dependents();
@@ -276,6 +355,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
   fence_before();
   __syncthreads();
+  pair_sync();  // both CTAs' barriers are initialised before any remote arrive or copy
   fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total = start[n_items];
@@ -287,78 +367,103 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint32_t phase = 0, fix_phase = 0;
     uint32_t issued_mask = 0, issued_parity = 0;
     bool stop = false;
-    for (int tile = blockIdx.x; tile < total && !stop; tile += gridDim.x) {
+    for (int tile = cid; tile < total && !stop; tile += ncl) {
       const Tile t = decode<MODE>(args, start, tile);
       const int off = __ldg(args.expert_offsets + t.e);
       const int rows = __ldg(args.expert_offsets + t.e + 1) - off;
       const int nkb = k_blocks<MODE>(args, rows);
+      const int half = static_cast<int>(rank) * kBM;  // this CTA's rows / columns of the tile
       for (int kb = 0; kb < nkb; ++kb) {
         int ok = 1;
-        if (lane == 0) ok = bwait(smem_addr(&empty[stage]), phase ^ 1u, abort_flag, args.status);
+        if (lane == 0) ok = cwait(smem_addr(&empty[stage]), phase ^ 1u, abort_flag, args.status);
         if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) {
           stop = true;
           break;
         }
         const uint32_t a = stage0 + stage * kStageBytes;
-        const uint32_t fb = smem_addr(&full[stage]);
-        if (MODE == kRecompute) {
+        const uint32_t fb = smem_addr(&full[stage]);  // CTA 0's copy counts both CTAs
+        const uint32_t fb0 = mapa(fb, 0);
+        // CTA 0 arrives once and announces the pair's bytes; CTA 1's copies complete on CTA 0's
+        // barrier
+        auto load = [&](const CUtensorMap* tm, uint32_t dst, int x, int y) {
+          if (rank == 0) tma2d(dst, tm, fb, x, y);
+          else tma2d_to_leader(dst, tm, fb0, x, y);
+        };
+        bool tail = false;
+        int valid = kBK;
+        if (MODE == kWeightGrad) {
+          valid = min(kBK, rows - kb * kBK);
+          tail = valid < kBK;
+        }
+        if (!tail) {
           if (lane == 0) {
-            // 128 x 32 K-major boxes (64-byte swizzle); Wd as two 32 h x 64 f MN-major boxes.
-            // Gate / up rows past the expert's F (another expert's, or zero fill) only reach
-            // accumulator columns the epilogue does not store.
-            const int kx = kb * kBK1, row0 = off + t.mb * kBM, f0 = t.nb * kNF1;
-            mbar_arrive_expect_tx(fb, kStageBytes);
-            tma2d(a, &maps.m[0], fb, kx, row0);                        // x rows
-            tma2d(a + 8192, &maps.m[1], fb, kx, row0);                 // d_eo rows
-            tma2d(a + 16384, &maps.m[2], fb, kx, t.e * args.F + f0);   // Wg rows
-            tma2d(a + 24576, &maps.m[3], fb, kx, t.e * args.F + f0);   // Wu rows
-            tma2d(a + 32768, &maps.m[4], fb, f0, t.e * args.H + kx);       // Wd f0 .. f0 + 63
-            tma2d(a + 36864, &maps.m[4], fb, f0 + 64, t.e * args.H + kx);  // Wd f0 + 64 ..
-          }
-        } else if (MODE == kInputGrad) {
-          if (lane == 0) {
-            const int nf = args.F / kBK;
-            const bool up = kb >= nf;
-            const int kx = (up ? kb - nf : kb) * kBK, row0 = off + t.mb * kBM, n0 = t.nb * kNOut;
-            mbar_arrive_expect_tx(fb, kStageBytes);
-            tma2d(a, &maps.m[up ? 1 : 0], fb, kx, row0);  // dg or du rows (K-major)
-#pragma unroll
-            for (int i = 0; i < 4; ++i)  // Wg or Wu: 64 f x 64 h per box (MN-major)
-              tma2d(a + 16384 + i * 8192, &maps.m[up ? 3 : 2], fb, n0 + 64 * i,
-                    t.e * args.F + kx);
+            if (rank == 0) mbar_arrive_expect_tx(fb, 2 * kStageBytes);
+            if (MODE == kRecompute) {
+              // x and d_eo: this CTA's 128 rows x 32 k; B: the gate (CTA 0) or up (CTA 1) block of
+              // 128 rows x 32 k, then 64 of the tile's 128 f columns of Wd^T.  Rows past the
+              // expert's F only reach accumulator columns the epilogue does not store.
+              const int kx = kb * kBK1, row0 = off + t.mb * kPairM + half, f0 = t.nb * kNF1;
+              load(&maps.m[0], a, kx, row0);
+              load(&maps.m[1], a + 8192, kx, row0);
+              load(&maps.m[rank == 0 ? 2 : 3], a + 16384, kx, t.e * args.F + f0);
+              load(&maps.m[4], a + 24576, f0 + static_cast<int>(rank) * 64, t.e * args.H + kx);
+            } else if (MODE == kInputGrad) {
+              const int nf = args.F / kBK;
+              const bool up = kb >= nf;
+              const int kx = (up ? kb - nf : kb) * kBK, row0 = off + t.mb * kPairM + half;
+              const int n0 = t.nb * kNOut + half;
+              load(&maps.m[up ? 1 : 0], a, kx, row0);  // dg or du rows (K-major)
+              // Wg or Wu: this CTA's 128 of the tile's 256 h columns, 64 f each (MN-major)
+              load(&maps.m[up ? 3 : 2], a + 16384, n0, t.e * args.F + kx);
+              load(&maps.m[up ? 3 : 2], a + 24576, n0 + 64, t.e * args.F + kx);
+            } else {
+              const CUtensorMap* ma = &maps.m[t.p == 0 ? 0 : (t.p == 1 ? 1 : 2)];  // d_eo, dg, du
+              const CUtensorMap* mb = &maps.m[t.p == 0 ? 3 : 4];                   // h, x
+              const int y = off + kb * kBK, m0 = t.mb * kPairM + half, n0 = t.nb * kNOut + half;
+              load(ma, a, m0, y);
+              load(ma, a + 8192, m0 + 64, y);
+              load(mb, a + 16384, n0, y);
+              load(mb, a + 24576, n0 + 64, y);
+            }
           }
         } else {
-          // A: 2 boxes of 64 m x 64 rows, B: 4 boxes of 64 n x 64 rows, all MN-major
-          const CUtensorMap* ma = &maps.m[t.p == 0 ? 0 : (t.p == 1 ? 1 : 2)];  // d_eo, dg, du
-          const CUtensorMap* mb = &maps.m[t.p == 0 ? 3 : 4];                   // h, x
-          const int y = off + kb * kBK, m0 = t.mb * kBM, n0 = t.nb * kNOut;
-          const int valid = min(kBK, rows - kb * kBK);
-          const uint32_t bar = valid == kBK ? fb : smem_addr(fix_bar);
+          // the expert's last rows: this CTA's copies complete on its own barrier, the rows past
+          // the end are zeroed in all four boxes; then CTA 0 arrives on its full barrier expecting
+          // a 16-byte token from CTA 1, which CTA 1 completes (after a cluster-scope fence) once
+          // its own rows are zeroed
+          const uint32_t xb = smem_addr(fix_bar);
           if (lane == 0) {
-            mbar_arrive_expect_tx(bar, kStageBytes);
-            tma2d(a, ma, bar, m0, y);
-            tma2d(a + 8192, ma, bar, m0 + 64, y);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) tma2d(a + 16384 + i * 8192, mb, bar, n0 + 64 * i, y);
+            const CUtensorMap* ma = &maps.m[t.p == 0 ? 0 : (t.p == 1 ? 1 : 2)];
+            const CUtensorMap* mb = &maps.m[t.p == 0 ? 3 : 4];
+            const int y = off + kb * kBK, m0 = t.mb * kPairM + half, n0 = t.nb * kNOut + half;
+            mbar_arrive_expect_tx(xb, kStageBytes);
+            tma2d(a, ma, xb, m0, y);
+            tma2d(a + 8192, ma, xb, m0 + 64, y);
+            tma2d(a + 16384, mb, xb, n0, y);
+            tma2d(a + 24576, mb, xb, n0 + 64, y);
           }
-          if (valid < kBK) {
-            // rows past the expert's end: zero them in all six boxes, then release the stage
-            // every lane waits, so that its stores below follow the copy's writes
-            const int got = bwait(smem_addr(fix_bar), fix_phase, abort_flag, args.status) ? 1 : 0;
-            fix_phase ^= 1u;
-            if (__all_sync(0xFFFFFFFFu, got) == 0) {
-              stop = true;
-              break;
+          // every lane waits, so that its stores below follow the copy's writes
+          const int got = cwait(xb, fix_phase, abort_flag, args.status) ? 1 : 0;
+          fix_phase ^= 1u;
+          if (__all_sync(0xFFFFFFFFu, got) == 0) {
+            stop = true;
+            break;
+          }
+          uint4* sm = reinterpret_cast<uint4*>(base + stage * kStageBytes);
+          const int per_box = (kBK - valid) * 8;  // 16-byte chunks in the rows to clear
+          for (int i = lane; i < 4 * per_box; i += 32) {
+            const int box = i / per_box, c = i % per_box;
+            sm[box * 512 + valid * 8 + c] = make_uint4(0u, 0u, 0u, 0u);
+          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) {
+            if (rank == 0) {
+              mbar_arrive_expect_tx(fb, kTailToken);
+            } else {
+              asm volatile("fence.acq_rel.cluster;" ::: "memory");
+              complete_tx_remote(fb0, kTailToken);
             }
-            uint4* s = reinterpret_cast<uint4*>(base + stage * kStageBytes);
-            const int per_box = (kBK - valid) * 8;  // 16-byte chunks in the rows to clear
-            for (int i = lane; i < 6 * per_box; i += 32) {
-              const int box = i / per_box, c = i % per_box;
-              s[box * 512 + valid * 8 + c] = make_uint4(0u, 0u, 0u, 0u);
-            }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            __syncwarp();
-            if (lane == 0) mbar_arrive(fb);
           }
         }
         issued_mask |= 1u << stage;
@@ -369,30 +474,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
     }
-    if (*abort_flag && lane == 0) {
+    if (*abort_flag && lane == 0 && rank == 0) {
+      // CTA 0's barriers count both CTAs' bytes: wait for the latest phase of each stage
       for (int st = 0; st < kStages; ++st)
-        if (issued_mask & (1u << st)) bdrain(smem_addr(&full[st]), (issued_parity >> st) & 1u);
+        if (issued_mask & (1u << st)) cdrain(smem_addr(&full[st]), (issued_parity >> st) & 1u);
     }
   } else if (warp == 1) {
-    // ---- MMA thread ---------------------------------------------------------------------------------
-    if (lane == 0) {
+    // ---- MMA thread (CTA 0 only): M = 256 over the pair ---------------------------------------------
+    if (rank == 0 && lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       bool issued_any = false;
       int it = 0;
-      for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+      for (int tile = cid; tile < total; tile += ncl, ++it) {
         const Tile t = decode<MODE>(args, start, tile);
         const int rows = __ldg(args.expert_offsets + t.e + 1) - __ldg(args.expert_offsets + t.e);
         const int nkb = k_blocks<MODE>(args, rows);
-        constexpr int kBufs = Cfg<MODE>::kAccBufs;
         const int acc = kBufs == 2 ? (it & 1) : 0;
         const uint32_t acc_par = kBufs == 2 ? ((it >> 1) & 1) : (it & 1);
-        if (!bwait(smem_addr(&acc_empty[acc]), acc_par ^ 1u, abort_flag, args.status)) break;
+        if (!cwait(smem_addr(&acc_empty[acc]), acc_par ^ 1u, abort_flag, args.status)) break;
         fence_after();
         const uint32_t d = tmem_base + acc * kAccStride;
         bool ok = true;
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!bwait(smem_addr(&full[stage]), phase, abort_flag, args.status)) {
+          if (!cwait(smem_addr(&full[stage]), phase, abort_flag, args.status)) {
             ok = false;
             break;
           }
@@ -402,59 +507,60 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           for (int kk = 0; kk < (MODE == kRecompute ? kBK1 : kBK) / kUK; ++kk) {
             const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
             if (MODE == kRecompute) {
-              // the Wg and Wu boxes are adjacent: one N = 256 operand of 256 K-major rows gives g
-              // in accumulator columns 0..127 and u in 128..255; dh in 256..383
-              constexpr uint32_t iGU = idesc_bf16(kBM, 2 * kNF1, 0, 0);
-              constexpr uint32_t iMN = idesc_bf16(kBM, kNF1, 0, 1);
-              mma(d, desc_k64(a + kk * 32), desc_k64(a + 16384 + kk * 32), iGU, accum);  // g | u
-              mma(d + 256, desc_k64(a + 8192 + kk * 32), desc_mn(a + 32768 + kk * 2048, 4096),
-                  iMN, accum);                                                            // dh
+              // g | u: N = 256 (CTA 0's gate rows -> columns 0..127, CTA 1's up rows -> 128..255);
+              // dh: N = 128 (64 f columns of Wd^T in each CTA) in columns 256..383
+              constexpr uint32_t iGU = idesc_bf16(kPairM, 2 * kNF1, 0, 0);
+              constexpr uint32_t iMN = idesc_bf16(kPairM, kNF1, 0, 1);
+              mma(d, desc_k64(a + kk * 32), desc_k64(a + 16384 + kk * 32), iGU, accum);
+              mma(d + 256, desc_k64(a + 8192 + kk * 32), desc_mn(a + 24576 + kk * 2048, 4096),
+                  iMN, accum);
             } else if (MODE == kInputGrad) {
-              constexpr uint32_t iMN = idesc_bf16(kBM, kNOut, 0, 1);
+              constexpr uint32_t iMN = idesc_bf16(kPairM, kNOut, 0, 1);
               mma(d, desc_k(a + kk * 32), desc_mn(a + 16384 + kk * 2048, 8192), iMN, accum);
             } else {
-              constexpr uint32_t iMM = idesc_bf16(kBM, kNOut, 1, 1);
+              constexpr uint32_t iMM = idesc_bf16(kPairM, kNOut, 1, 1);
               mma(d, desc_mn(a + kk * 2048, 8192), desc_mn(a + 16384 + kk * 2048, 8192), iMM,
                   accum);
             }
           }
           issued_any = true;
-          commit(smem_addr(&empty[stage]));
+          commit_both(smem_addr(&empty[stage]));
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        // a tile without K blocks (an expert with no rows) has nothing to wait for: the epilogue
-        // writes zeros; the commit still orders it after the previous tile's MMAs
-        commit(smem_addr(&acc_full[acc]));
+        // a tile without K blocks (an expert with no rows) has nothing to wait for: the epilogues
+        // write zeros; the commit still orders it after the previous tile's MMAs
+        commit_both(smem_addr(&acc_full[acc]));
       }
       if (issued_any) {
-        commit(smem_addr(drain_bar));
-        bdrain(smem_addr(drain_bar), 0);
+        commit_local(smem_addr(drain_bar));
+        cdrain(smem_addr(drain_bar), 0);
       }
     }
   } else {
-    // ---- epilogue: warp (w & 3) owns TMEM lanes (= tile rows) [32 (w & 3), +32) ----------------------
+    // ---- epilogue: warp (w & 3) owns TMEM lanes (= this CTA's rows) [32 (w & 3), +32) -------------
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
+    const int r = static_cast<int>(rank) * kBM + quarter * 32 + lane;  // row of the pair tile
+    const uint32_t acc_empty0 = mapa(smem_addr(&acc_empty[0]), 0);
+    const uint32_t acc_empty1 = mapa(smem_addr(&acc_empty[1]), 0);
     int it = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+    for (int tile = cid; tile < total; tile += ncl, ++it) {
       const Tile t = decode<MODE>(args, start, tile);
       const int off = __ldg(args.expert_offsets + t.e);
       const int rows = __ldg(args.expert_offsets + t.e + 1) - off;
-      constexpr int kBufs = Cfg<MODE>::kAccBufs;
       const int acc = kBufs == 2 ? (it & 1) : 0;
       const uint32_t acc_par = kBufs == 2 ? ((it >> 1) & 1) : (it & 1);
       int ok = 1;
-      if (lane == 0) ok = bwait(smem_addr(&acc_full[acc]), acc_par, abort_flag, args.status);
+      if (lane == 0) ok = cwait(smem_addr(&acc_full[acc]), acc_par, abort_flag, args.status);
       if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) break;
       fence_after();
       const uint32_t tb = tmem_base + acc * kAccStride + (static_cast<uint32_t>(quarter * 32) << 16);
       if (MODE == kRecompute) {
-        const bool valid = t.mb * kBM + r < rows;
-        const size_t row = static_cast<size_t>(off + t.mb * kBM + r);
+        const bool valid = t.mb * kPairM + r < rows;
+        const size_t row = static_cast<size_t>(off + t.mb * kPairM + r);
         __nv_bfloat16* h_out = static_cast<__nv_bfloat16*>(args.out0);
         __nv_bfloat16* dg_out = static_cast<__nv_bfloat16*>(args.out1);
         __nv_bfloat16* du_out = static_cast<__nv_bfloat16*>(args.out2);
@@ -498,8 +604,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
         }
       } else if (MODE == kInputGrad) {
-        const bool valid = t.mb * kBM + r < rows;
-        const size_t row = static_cast<size_t>(off + t.mb * kBM + r);
+        const bool valid = t.mb * kPairM + r < rows;
+        const size_t row = static_cast<size_t>(off + t.mb * kPairM + r);
         __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out0);
 #pragma unroll 1
         for (int c = 0; c < kNOut; c += 32) {
@@ -527,18 +633,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const bool any_k = rows > 0;  // uniform over the warp
         uint8_t* stg = out_stage + quarter * kStageOutBytes;
         const uint32_t stg_addr = smem_addr(stg);
+        if (!any_k) {
+          // an expert without rows: one zero block, stored to every 32-column block of this
+          // warp's rows without waiting in between (the source does not change)
+          if (lane == 0) bulk_wait_read();
+          __syncwarp();
+          uint4* row_p = reinterpret_cast<uint4*>(stg + lane * 128);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) row_p[q] = make_uint4(0u, 0u, 0u, 0u);
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) {
+            for (int c = 0; c < kNOut && t.nb * kNOut + c < N; c += 32)
+              tma_store3d(om, stg_addr, t.nb * kNOut + c,
+                          t.mb * kPairM + static_cast<int>(rank) * kBM + quarter * 32, t.e);
+            bulk_commit();
+          }
+        }
 #pragma unroll 1
-        for (int c = 0; c < kNOut; c += 32) {
+        for (int c = 0; any_k && c < kNOut; c += 32) {
           const int col = t.nb * kNOut + c;
           if (col >= N) break;
           uint32_t v[32];
-          if (any_k) {
-            ld32(tb + c, v);
-            ld_wait();
-          } else {
-#pragma unroll
-            for (int q = 0; q < 32; ++q) v[q] = 0u;
-          }
+          ld32(tb + c, v);
+          ld_wait();
           // the previous block's store has read the staging block
           if (lane == 0) bulk_wait_read();
           __syncwarp();
@@ -549,23 +667,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           __syncwarp();
           if (lane == 0) {
-            tma_store3d(om, stg_addr, col, t.mb * kBM + quarter * 32, t.e);
+            tma_store3d(om, stg_addr, col,
+                        t.mb * kPairM + static_cast<int>(rank) * kBM + quarter * 32, t.e);
             bulk_commit();
           }
         }
       }
       fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_addr(&acc_empty[acc]));
+      if (lane == 0) {
+        const uint32_t ae = acc == 0 ? acc_empty0 : acc_empty1;
+        if (rank == 0) mbar_arrive(smem_addr(&acc_empty[acc]));
+        else arrive_remote(ae);
+      }
     }
   }
 
   if (MODE == kWeightGrad && warp >= 2 && lane == 0) bulk_wait_all();
   fence_before();
   __syncthreads();
+  pair_sync();  // no MMA of the pair is in flight when either CTA frees its TMEM
   if (warp == 1) {
     fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                  "r"(kTmemColsBwd)
                  : "memory");
   }
@@ -710,17 +834,38 @@ bool tmap_f32_out(CUtensorMap* tm, void* ptr, uint64_t E, uint64_t M, uint64_t N
 template <int MODE>
 cudaError_t launch_bwd_gemm(const BwdMaps& maps, const BwdArgs& a, cudaStream_t s) {
   const size_t smem = bwd_smem<MODE>();
-  static int configured[64] = {0};
+  static int grid_of[64] = {0};
   int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(bwd_gemm_kernel<MODE>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               static_cast<int>(smem));
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kBwdThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  if (grid_of[dev] == 0) {
+    cudaError_t e = cudaFuncSetAttribute(bwd_gemm_kernel<MODE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    configured[dev] = 1;
+    // as many pairs as can be resident at once (one CTA per SM)
+    cfg.gridDim = dim3(2 * (num_sms() / 2));
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, bwd_gemm_kernel<MODE>, &cfg);
+    if (e != cudaSuccess) return e;
+    if (clusters < 1) return cudaErrorLaunchOutOfResources;
+    grid_of[dev] = 2 * min(clusters, num_sms() / 2);
   }
-  return launch_pdl(bwd_gemm_kernel<MODE>, dim3(num_sms()), dim3(kBwdThreads), smem, s, maps, a);
+  cfg.gridDim = dim3(grid_of[dev]);
+  cfg.numAttrs = MOE_USE_PDL ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, bwd_gemm_kernel<MODE>, maps, a);
 }
 
 }  // namespace
