@@ -29,7 +29,7 @@ EXPORTS = ["moe_abi_version", "moe_status_string", "moe_capacity", "moe_route",
            "moe_ffn_workspace_size",
            "moe_expert_ffn", "moe_ffn_weight_list_bytes", "moe_ffn_weight_list_init",
            "moe_expert_ffn_list", "moe_quantize_rows_fp8", "moe_ffn_w8_workspace_size",
-           "moe_expert_ffn_w8", "moe_backward_workspace_size", "moe_backward", "moe_ep_regroup", "moe_ep_exchange", "moe_combine", "moe_sync_status"]
+           "moe_expert_ffn_w8", "moe_backward_workspace_size", "moe_backward", "moe_combine_backward", "moe_expert_backward_workspace_size", "moe_expert_backward", "moe_ep_regroup", "moe_ep_exchange", "moe_combine", "moe_sync_status"]
 
 _lib = None
 
@@ -69,6 +69,9 @@ def load() -> ctypes.CDLL:
         "moe_backward_workspace_size": (Z, [I, I, I, I, I]),
         "moe_backward": (I, [P, I, I, I, I, I, P, I, P, P, P, P, I, P, P, P, P, P, P, P, P, P, P,
                              P, P, Z, P]),
+        "moe_combine_backward": (I, [P, I, I, I, I, P, I, P, P, P, I, P, P, P, P, P]),
+        "moe_expert_backward_workspace_size": (Z, [I, I]),
+        "moe_expert_backward": (I, [P, P, P, I, I, I, I, P, P, P, P, P, P, P, P, Z, P]),
         "moe_ep_regroup": (I, [P, I, I, I, I, I, I, I, I, P, P, Z, P, P, Z, P, P, P]),
         "moe_ep_exchange": (I, [P, I, I, I, I, P, P, I, P, P, I, Z, Z, P, P, P]),
         "moe_combine": (I, [P, I, P, P, I, I, I, P, P, P]),
@@ -222,6 +225,30 @@ def moe_backward(dy, T, H, k, E, F, logits, renormalize, topk_idx, topk_w, slot_
                              _ptr(d_w_gate), _ptr(d_w_up), _ptr(d_w_down), _ptr(ws), ws_bytes,
                              _stream(stream))
     return _check(st, "moe_backward", raise_on_error)
+
+
+def moe_combine_backward(dy, T, H, k, E, logits, renormalize, topk_idx, topk_w, slot_row,
+                         max_rows, expert_out, d_eo, d_topk_w, d_logits, stream=None,
+                         raise_on_error=True):
+    st = load().moe_combine_backward(_ptr(dy), T, H, k, E, _ptr(logits), int(renormalize),
+                                     _ptr(topk_idx), _ptr(topk_w), _ptr(slot_row), max_rows,
+                                     _ptr(expert_out), _ptr(d_eo), _ptr(d_topk_w), _ptr(d_logits),
+                                     _stream(stream))
+    return _check(st, "moe_combine_backward", raise_on_error)
+
+
+def moe_expert_backward_workspace_size(max_rows, F) -> int:
+    return load().moe_expert_backward_workspace_size(max_rows, F)
+
+
+def moe_expert_backward(ffn_input, d_eo, expert_offsets, max_rows, E, H, F, w_gate, w_up, w_down,
+                        dx_rows, d_w_gate, d_w_up, d_w_down, ws, ws_bytes, stream=None,
+                        raise_on_error=True):
+    st = load().moe_expert_backward(_ptr(ffn_input), _ptr(d_eo), _ptr(expert_offsets), max_rows, E,
+                                    H, F, _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(dx_rows),
+                                    _ptr(d_w_gate), _ptr(d_w_up), _ptr(d_w_down), _ptr(ws),
+                                    ws_bytes, _stream(stream))
+    return _check(st, "moe_expert_backward", raise_on_error)
 
 
 def moe_ep_regroup(counts, A, B, src_order, src_stride, src_rows, dst_order, dst_stride, dst_rows,

@@ -322,6 +322,59 @@ moe_status_t moe_backward(const void* dy, int T, int H, int k, int E, int F, con
                                         reinterpret_cast<cudaStream_t>(stream)));
 }
 
+moe_status_t moe_combine_backward(const void* dy, int T, int H, int k, int E, const float* logits,
+                                  int renormalize, const int32_t* topk_idx, const float* topk_w,
+                                  const int32_t* slot_row, int max_rows, const void* expert_out,
+                                  void* d_eo, float* d_topk_w, float* d_logits,
+                                  moe_stream_t stream) {
+  if (T < 0 || k < 1 || k > 32 || E < 1 || E > 1024 || k > E || max_rows < 0 || H < 8)
+    return MOE_ERR_INVALID_ARG;
+  if (H % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (T > 0 && (dy == nullptr || topk_idx == nullptr || topk_w == nullptr || slot_row == nullptr ||
+                expert_out == nullptr || d_eo == nullptr || d_topk_w == nullptr ||
+                d_logits == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (!renormalize && T > 0 && logits == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned(dy, 16) || !aligned(expert_out, 16) || !aligned(d_eo, 16)) return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_combine_backward(
+      dy, T, H, k, E, logits, renormalize, topk_idx, topk_w, slot_row, max_rows, expert_out, d_eo,
+      d_topk_w, d_logits, nullptr, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_expert_backward_workspace_size(int max_rows, int F) {
+  if (max_rows < 0 || F < 1) return 0;
+  return moe::expert_backward_workspace_bytes(max_rows, F);
+}
+
+moe_status_t moe_expert_backward(const void* ffn_input, const void* d_eo,
+                                 const int32_t* expert_offsets, int max_rows, int E, int H, int F,
+                                 const void* w_gate, const void* w_up, const void* w_down,
+                                 void* dx_rows, float* d_w_gate, float* d_w_up, float* d_w_down,
+                                 void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (E < 1 || E > 1024 || max_rows < 0 || H < 64 || F < 64) return MOE_ERR_INVALID_ARG;
+  if (H % 64 != 0 || F % 64 != 0) return MOE_ERR_UNSUPPORTED;
+  const void* need[] = {expert_offsets, w_gate, w_up, w_down, d_w_gate, d_w_up, d_w_down, ws};
+  for (const void* q : need)
+    if (q == nullptr) return MOE_ERR_INVALID_ARG;
+  if (max_rows > 0 && (ffn_input == nullptr || d_eo == nullptr || dx_rows == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  const void* a16[] = {ffn_input, d_eo, dx_rows, w_gate, w_up, w_down, d_w_gate, d_w_up, d_w_down};
+  for (const void* q : a16)
+    if (!aligned(q, 16)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(ws, 256)) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < moe::expert_backward_workspace_bytes(max_rows, F)) return MOE_ERR_WORKSPACE;
+  auto up = [](size_t b) { return (b + 255) / 256 * 256; };
+  const size_t r = static_cast<size_t>(max_rows > 0 ? max_rows : 1);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  void* h = w + 256;
+  void* dg = w + 256 + up(r * F * 2);
+  void* du = w + 256 + 2 * up(r * F * 2);
+  return from_cuda(moe::launch_expert_backward(
+      ffn_input, d_eo, expert_offsets, max_rows, E, H, F, w_gate, w_up, w_down, dx_rows, d_w_gate,
+      d_w_up, d_w_down, reinterpret_cast<int*>(w), h, dg, du,
+      reinterpret_cast<cudaStream_t>(stream)));
+}
+
 moe_status_t moe_combine(const void* expert_out, int max_rows, const int32_t* slot_row,
                          const float* topk_w, int T, int k, int H, void* y, int32_t* status,
                          moe_stream_t stream) {

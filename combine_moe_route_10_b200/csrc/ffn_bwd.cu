@@ -697,7 +697,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
 // ---- combine backward and the router's gradient (warp per token) ---------------------------------
 // d_eo[row] = bf16(fp32(w * dy)) for every kept slot; d_w[t,j] = <dy[t], eo[row]> (0 for a dropped
-// slot); d_logits[t, :] from d_w (softmax backward); ones[t,j] = 1 (the unit weights of the final
+// slot); d_logits[t, :] from d_w (softmax backward); ones[t,j] = 1 when given (the unit weights of the final
 // combine of the input gradients).
 __global__ void __launch_bounds__(256)
     combine_bwd_kernel(const uint4* __restrict__ dy, const uint4* __restrict__ eo, int max_rows,
@@ -744,7 +744,7 @@ __global__ void __launch_bounds__(256)
     }
     if (lane < k) {
       d_w[t * k + lane] = my_dw;
-      ones[t * k + lane] = 1.0f;
+      if (ones != nullptr) ones[t * k + lane] = 1.0f;
     }
     float* dl = d_logits + static_cast<size_t>(t) * E;
     if (renormalize) {
@@ -878,35 +878,31 @@ size_t backward_workspace_bytes(int max_rows, int T, int k, int H, int F) {
   return 256 + up(r * H * 2) + 3 * up(r * F * 2) + up(r * H * 2) + up(tk * 4);
 }
 
-cudaError_t launch_backward(const void* dy, int T, int H, int k, int E, int F, const float* logits,
-                            int renormalize, const int32_t* topk_idx, const float* topk_w,
-                            const int32_t* slot_row, const int32_t* expert_offsets, int max_rows,
-                            const void* ffn_input, const void* expert_out, const void* w_gate,
-                            const void* w_up, const void* w_down, void* dx, float* d_logits,
-                            float* d_topk_w, float* d_w_gate, float* d_w_up, float* d_w_down,
-                            void* ws, cudaStream_t s) {
-  auto up = [](size_t b) { return (b + 255) / 256 * 256; };
-  const size_t r = static_cast<size_t>(max_rows > 0 ? max_rows : 1);
-  uint8_t* w = static_cast<uint8_t*>(ws);
-  int* status = reinterpret_cast<int*>(w);
-  uint8_t* p = w + 256;
-  void* d_eo = p;     p += up(r * H * 2);
-  void* h = p;        p += up(r * F * 2);
-  void* dg = p;       p += up(r * F * 2);
-  void* du = p;       p += up(r * F * 2);
-  void* dx_rows = p;  p += up(r * H * 2);
-  float* ones = reinterpret_cast<float*>(p);
+cudaError_t launch_combine_backward(const void* dy, int T, int H, int k, int E,
+                                   const float* logits, int renormalize, const int32_t* topk_idx,
+                                   const float* topk_w, const int32_t* slot_row, int max_rows,
+                                   const void* expert_out, void* d_eo, float* d_topk_w,
+                                   float* d_logits, float* ones, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
+  int blocks = (T + 7) / 8;
+  if (blocks > 8 * num_sms()) blocks = 8 * num_sms();
+  return launch_pdl(combine_bwd_kernel, dim3(blocks), dim3(256), 0, s,
+                    static_cast<const uint4*>(dy), static_cast<const uint4*>(expert_out),
+                    max_rows, slot_row, topk_w, topk_idx, logits, renormalize, T, k, E, H,
+                    static_cast<uint4*>(d_eo), d_topk_w, d_logits, ones);
+}
 
-  {
-    int blocks = (T + 7) / 8;
-    if (blocks > 8 * num_sms()) blocks = 8 * num_sms();
-    const cudaError_t e = launch_pdl(
-        combine_bwd_kernel, dim3(blocks), dim3(256), 0, s, static_cast<const uint4*>(dy),
-        static_cast<const uint4*>(expert_out), max_rows, slot_row, topk_w, topk_idx, logits,
-        renormalize, T, k, E, H, static_cast<uint4*>(d_eo), d_topk_w, d_logits, ones);
-    if (e != cudaSuccess) return e;
-  }
+size_t expert_backward_workspace_bytes(int max_rows, int F) {
+  const size_t r = static_cast<size_t>(max_rows > 0 ? max_rows : 1);
+  return 256 + 3 * ((r * F * 2 + 255) / 256 * 256);  // status | h, dg, du [r, F]
+}
+
+cudaError_t launch_expert_backward(const void* ffn_input, const void* d_eo,
+                                   const int32_t* expert_offsets, int max_rows, int E, int H, int F,
+                                   const void* w_gate, const void* w_up, const void* w_down,
+                                   void* dx_rows, float* d_w_gate, float* d_w_up, float* d_w_down,
+                                   int* status, void* h, void* dg, void* du, cudaStream_t s) {
+  if (max_rows == 0) return cudaSuccess;
   BwdArgs a{expert_offsets, E, H, F, max_rows, nullptr, nullptr, nullptr, status};
   BwdMaps m1{}, m2{}, m3{};
   const uint64_t mr = static_cast<uint64_t>(max_rows);
@@ -939,6 +935,35 @@ cudaError_t launch_backward(const void* dy, int T, int H, int k, int E, int F, c
   a.out1 = d_w_gate;
   a.out2 = d_w_up;
   e = launch_bwd_gemm<kWeightGrad>(m3, a, s);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_backward(const void* dy, int T, int H, int k, int E, int F, const float* logits,
+                            int renormalize, const int32_t* topk_idx, const float* topk_w,
+                            const int32_t* slot_row, const int32_t* expert_offsets, int max_rows,
+                            const void* ffn_input, const void* expert_out, const void* w_gate,
+                            const void* w_up, const void* w_down, void* dx, float* d_logits,
+                            float* d_topk_w, float* d_w_gate, float* d_w_up, float* d_w_down,
+                            void* ws, cudaStream_t s) {
+  auto up = [](size_t b) { return (b + 255) / 256 * 256; };
+  const size_t r = static_cast<size_t>(max_rows > 0 ? max_rows : 1);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  int* status = reinterpret_cast<int*>(w);
+  uint8_t* p = w + 256;
+  void* d_eo = p;     p += up(r * H * 2);
+  void* h = p;        p += up(r * F * 2);
+  void* dg = p;       p += up(r * F * 2);
+  void* du = p;       p += up(r * F * 2);
+  void* dx_rows = p;  p += up(r * H * 2);
+  float* ones = reinterpret_cast<float*>(p);
+  if (T == 0) return cudaSuccess;
+  cudaError_t e = launch_combine_backward(dy, T, H, k, E, logits, renormalize, topk_idx, topk_w,
+                                          slot_row, max_rows, expert_out, d_eo, d_topk_w,
+                                          d_logits, ones, s);
+  if (e != cudaSuccess) return e;
+  e = launch_expert_backward(ffn_input, d_eo, expert_offsets, max_rows, E, H, F, w_gate, w_up,
+                             w_down, dx_rows, d_w_gate, d_w_up, d_w_down, status, h, dg, du, s);
   if (e != cudaSuccess) return e;
   e = launch_combine(dx_rows, max_rows, slot_row, ones, T, k, H, dx, nullptr, s);
   if (e != cudaSuccess) return e;

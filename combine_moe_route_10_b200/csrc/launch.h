@@ -92,6 +92,20 @@ cudaError_t ffn_weight_list_init(const void* const* w_gate, const void* const* w
                                  const void* const* w_down, int E, int H, int F, void* list,
                                  cudaStream_t s);
 
+// The backward's two halves: the combine backward (d_eo, routing-weight and logit gradients, the
+// unit weights of the final combine when `ones` is given) and the experts' GEMMs (workspace:
+// status | h, dg, du).
+cudaError_t launch_combine_backward(const void* dy, int T, int H, int k, int E,
+                                   const float* logits, int renormalize, const int32_t* topk_idx,
+                                   const float* topk_w, const int32_t* slot_row, int max_rows,
+                                   const void* expert_out, void* d_eo, float* d_topk_w,
+                                   float* d_logits, float* ones, cudaStream_t s);
+size_t expert_backward_workspace_bytes(int max_rows, int F);
+cudaError_t launch_expert_backward(const void* ffn_input, const void* d_eo,
+                                   const int32_t* expert_offsets, int max_rows, int E, int H, int F,
+                                   const void* w_gate, const void* w_up, const void* w_down,
+                                   void* dx_rows, float* d_w_gate, float* d_w_up, float* d_w_down,
+                                   int* status, void* h, void* dg, void* du, cudaStream_t s);
 // Backward of the layer (workspace: status | d_eo | h, dg, du | dx_rows | unit weights).
 size_t backward_workspace_bytes(int max_rows, int T, int k, int H, int F);
 cudaError_t launch_backward(const void* dy, int T, int H, int k, int E, int F, const float* logits,

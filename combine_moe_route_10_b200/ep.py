@@ -105,6 +105,24 @@ class CudaOps:
                              0 if local_aux is None else local_aux[0].numel() * local_aux.element_size(),
                              local_offsets, status)
 
+    def combine_backward(self, dy, T, H, k, E, logits, renormalize, topk_idx, topk_w, slot_row,
+                         expert_out, d_eo, d_topk_w, d_logits):
+        _lib.moe_combine_backward(dy, T, H, k, E, logits, renormalize, topk_idx, topk_w, slot_row,
+                                  expert_out.shape[0], expert_out, d_eo, d_topk_w, d_logits)
+
+    def expert_backward(self, ffn_input, d_eo, offsets, max_rows, E, H, F, w_gate, w_up, w_down,
+                        dx_rows, d_w_gate, d_w_up, d_w_down, ws):
+        _lib.moe_expert_backward(ffn_input, d_eo, offsets, max_rows, E, H, F, w_gate, w_up, w_down,
+                                 dx_rows, d_w_gate, d_w_up, d_w_down, ws, ws.numel())
+
+    def ffn_input_rows(self, rows, scales, payload, ffn_ws, max_rows, H, F):
+        """The FFN input rows as bf16 [max_rows, H]: the rows themselves, or, for the FP8 payload,
+        the dequantised rows the last expert FFN call left in its workspace (after h)."""
+        if payload != _lib.MOE_PAYLOAD_FP8_E4M3_B128:
+            return rows
+        off = 256 + (max_rows * F * 2 + 255) // 256 * 256
+        return ffn_ws[off:off + max_rows * H * 2].view(torch.bfloat16).view(max_rows, H)
+
     def sync_status(self, ws) -> int:
         return _lib.moe_sync_status(ws)
 
@@ -306,6 +324,7 @@ class MoeEP:
             if n_recv > self.cap:
                 self._alloc_expert_side(max(n_recv, self.cap + self.cap // 4))
             n_send = sum(send_splits)
+            self._ht_splits = (send_splits, recv_splits)  # the backward retraces them
             self._exchange_rows(self.recv[:n_recv], self.send[:n_send], recv_splits, send_splits)
             if self.fp8:
                 self._all_to_all(self.recv_scales[:n_recv], self.send_scales[:n_send],
@@ -353,9 +372,106 @@ class MoeEP:
         ops.combine(self.ret, S, self.slot_row, self.topk_w, T, k, H, self.y)
         return self.y
 
+    # -- backward ------------------------------------------------------------------------------
+    def _alloc_backward(self):
+        dev, H, S = self.device, self.H, self.send.shape[0]
+        bf16, f32 = torch.bfloat16, torch.float32
+        E_loc, F = self.E_loc, self.F
+        if self.mode == "p2p":
+            # the experts' ranks pull d_eo from the sources and push dx_rows back into them
+            self.b_d_eo, peers = self.comm.alloc_shared((S, H), bf16, dev)
+            self.b_peer_d_eo = self._pointers(peers)
+            self.b_dret, peers = self.comm.alloc_shared((S, H), bf16, dev)
+            self.b_peer_dret = self._pointers(peers)
+        else:
+            self.b_d_eo = torch.empty((S, H), dtype=bf16, device=dev)
+            self.b_dret = torch.empty((S, H), dtype=bf16, device=dev)
+            P = self.cap if self.mode == "ht" else self.R * self.M
+            self.b_recv = torch.empty((P, H), dtype=bf16, device=dev)      # d_eo, source order
+            self.b_back = torch.empty((P, H), dtype=bf16, device=dev)      # dx_rows, source order
+            if self.mode == "ll":
+                self.b_send_pad = torch.empty((self.R * self.M, H), dtype=bf16, device=dev)
+                self.b_ret_pad = torch.empty((self.R * self.M, H), dtype=bf16, device=dev)
+        self.b_cap = self.cap
+        self.b_d_eo_grouped = torch.empty((self.cap, H), dtype=bf16, device=dev)
+        self.b_dx_rows = torch.empty((self.cap, H), dtype=bf16, device=dev)
+        self.ws_ebwd = self.ops.workspace(
+            _lib.moe_expert_backward_workspace_size(self.cap, F))
+        self.ones = torch.ones((self.T, self.k), dtype=f32, device=dev)
+        self.grads = {
+            "dx": torch.empty((self.T, H), dtype=bf16, device=dev),
+            "d_logits": torch.empty((self.T, self.E), dtype=f32, device=dev),
+            "d_topk_w": torch.empty((self.T, self.k), dtype=f32, device=dev),
+            "d_w_gate": torch.empty((E_loc, F, H), dtype=f32, device=dev),
+            "d_w_up": torch.empty((E_loc, F, H), dtype=f32, device=dev),
+            "d_w_down": torch.empty((E_loc, H, F), dtype=f32, device=dev),
+        }
+
+    def backward(self, dy, logits, w_gate, w_up, w_down) -> dict:
+        """Gradients for the output gradient ``dy`` [T,H] bf16 of this rank's tokens, after
+        ``forward`` (its routing, plan, exchanged rows and counts are reused): the combine backward
+        on this rank (the d_eo rows, the routing-weight and logit gradients), d_eo to the experts'
+        owners the way the rows went, the experts' backward there (the weight gradients of this
+        rank's experts), dx_rows back the way the outputs came, and the unit-weight combine.
+        Returns dx bf16 [T,H], d_logits fp32 [T,E], d_topk_w fp32 [T,k] for this rank's tokens
+        and d_w_gate / d_w_up fp32 [E_loc,F,H], d_w_down fp32 [E_loc,H,F] for its experts."""
+        T, H, E, k, R, E_loc = self.T, self.H, self.E, self.k, self.R, self.E_loc
+        dev = self.device
+        expect(dy, (T, H), torch.bfloat16, "dy", dev)
+        expect(logits, (T, E), torch.float32, "logits", dev)
+        expect(w_gate, (E_loc, self.F, H), torch.bfloat16, "w_gate", dev)
+        expect(w_up, (E_loc, self.F, H), torch.bfloat16, "w_up", dev)
+        expect(w_down, (E_loc, H, self.F), torch.bfloat16, "w_down", dev)
+        if getattr(self, "grads", None) is None or self.b_cap != self.cap:
+            self._alloc_backward()
+        ops, g, st = self.ops, self.grads, self.ws_regroup
+        S = self.send.shape[0]
+        ops.combine_backward(dy, T, H, k, E, logits, self.renormalize, self.topk_idx, self.topk_w,
+                             self.slot_row, self.ret, self.b_d_eo, g["d_topk_w"], g["d_logits"])
+        if self.mode == "p2p":
+            self.comm.barrier(dev)  # every rank's d_eo rows are written
+            ops.exchange(self.all_counts, R, E, self.rank, _lib.MOE_EP_PULL, self.b_peer_d_eo,
+                         None, S, self.b_d_eo_grouped, None, None, st)
+        elif self.mode == "ht":
+            send_splits, recv_splits = self._ht_splits
+            n_send, n_recv = sum(send_splits), sum(recv_splits)
+            self._exchange_rows(self.b_recv[:n_recv], self.b_d_eo[:n_send], recv_splits,
+                                send_splits)
+            ops.regroup(self.recv_counts, R, E_loc, A_MAJOR, 0, self.b_recv, B_MAJOR, 0,
+                        self.b_d_eo_grouped, None, None, None, st)
+        else:
+            ops.regroup(self.expert_counts, R, E_loc, A_MAJOR, 0, self.b_d_eo, A_MAJOR, self.M,
+                        self.b_send_pad, None, None, None, st)
+            self._exchange_rows(self.b_recv, self.b_send_pad, None, None)
+            ops.regroup(self.recv_counts, R, E_loc, A_MAJOR, self.M, self.b_recv, B_MAJOR, 0,
+                        self.b_d_eo_grouped, None, None, None, st)
+        x_rows = ops.ffn_input_rows(self.grouped, self.grouped_scales, self.payload, self.ws_ffn,
+                                    self.cap, H, self.F)
+        ops.expert_backward(x_rows, self.b_d_eo_grouped, self.local_offsets, self.cap, E_loc, H,
+                            self.F, w_gate, w_up, w_down, self.b_dx_rows, g["d_w_gate"],
+                            g["d_w_up"], g["d_w_down"], self.ws_ebwd)
+        if self.mode == "p2p":
+            ops.exchange(self.all_counts, R, E, self.rank, _lib.MOE_EP_PUSH, self.b_peer_dret,
+                         None, S, self.b_dx_rows, None, None, st)
+            self.comm.barrier(dev)  # every rank's pushes into this rank's buffer are complete
+        elif self.mode == "ht":
+            ops.regroup(self.recv_counts, R, E_loc, B_MAJOR, 0, self.b_dx_rows, A_MAJOR, 0,
+                        self.b_back, None, None, None, st)
+            self._exchange_rows(self.b_dret[:n_send], self.b_back[:n_recv], send_splits,
+                                recv_splits)
+        else:
+            ops.regroup(self.recv_counts, R, E_loc, B_MAJOR, 0, self.b_dx_rows, A_MAJOR, self.M,
+                        self.b_back, None, None, None, st)
+            self._exchange_rows(self.b_ret_pad, self.b_back, None, None)
+            ops.regroup(self.expert_counts, R, E_loc, A_MAJOR, self.M, self.b_ret_pad, A_MAJOR, 0,
+                        self.b_dret, None, None, None, st)
+        ops.combine(self.b_dret, S, self.slot_row, self.ones, T, k, H, g["dx"])
+        return g
+
     def status(self) -> int:
         """Synchronise; the first non-OK device status of this rank's dispatch, regroups and FFN."""
-        for ws in (self.ws_dispatch, self.ws_regroup, self.ws_ffn):
+        for ws in (self.ws_dispatch, self.ws_regroup, self.ws_ffn) + (
+                (self.ws_ebwd,) if getattr(self, "ws_ebwd", None) is not None else ()):
             st = self.ops.sync_status(ws)
             if st != _lib.MOE_OK:
                 return st

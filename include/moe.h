@@ -311,6 +311,32 @@ moe_status_t moe_backward(const void* dy, int T, int H, int k, int E, int F, con
                           void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * The two halves of moe_backward, for callers that move rows between them (expert parallelism):
+ *   moe_combine_backward: step 1 of moe_backward on this rank's tokens: d_eo [max_rows, H] bf16 in
+ *     the dispatch's row layout (rows of kept slots written), d_topk_w fp32 [T,k], d_logits fp32
+ *     [T,E].  expert_out holds the expert outputs of this rank's slots in the same row layout.
+ *   moe_expert_backward: step 2 on expert-major rows: ffn_input and d_eo bf16 [max_rows, H] laid
+ *     out by expert_offsets [E+1] (the experts' rows in the order their forward used), dx_rows
+ *     bf16 [max_rows, H] out, and the fp32 weight gradients of these E experts.  ws:
+ *     moe_expert_backward_workspace_size(max_rows, F) bytes, 256-byte aligned, holding
+ *     [status | h, dg, du bf16 [max_rows, F]]; device findings (a bounded wait that ran out) are
+ *     read with moe_sync_status(ws).
+ * moe_backward is exactly moe_combine_backward, moe_expert_backward and a moe_combine of dx_rows
+ * with unit weights.  Limits as for moe_backward.
+ */
+moe_status_t moe_combine_backward(const void* dy, int T, int H, int k, int E, const float* logits,
+                                  int renormalize, const int32_t* topk_idx, const float* topk_w,
+                                  const int32_t* slot_row, int max_rows, const void* expert_out,
+                                  void* d_eo, float* d_topk_w, float* d_logits,
+                                  moe_stream_t stream);
+size_t moe_expert_backward_workspace_size(int max_rows, int F);
+moe_status_t moe_expert_backward(const void* ffn_input, const void* d_eo,
+                                 const int32_t* expert_offsets, int max_rows, int E, int H, int F,
+                                 const void* w_gate, const void* w_up, const void* w_down,
+                                 void* dx_rows, float* d_w_gate, float* d_w_up, float* d_w_down,
+                                 void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * moe_ep_regroup: the row moves on both sides of an expert-parallel all-to-all, as one segmented
  * copy.
  *

@@ -46,7 +46,8 @@ from .numerics import bf16_bits, bf16_from_bits, bf16_round, e4m3_decode, e4m3_e
 
 __all__ = ["capacity", "route", "dispatch_plan", "dispatch_payload", "expert_ffn", "combine",
            "pipeline", "QBLOCK", "quantize_rows_fp8", "dequantize_rows_fp8", "expert_ffn_w8",
-           "ep_segment_rows", "ep_regroup", "ep_pipeline", "backward"]
+           "ep_segment_rows", "ep_regroup", "ep_pipeline", "backward", "combine_backward",
+           "router_backward", "expert_backward"]
 
 QBLOCK = 128   # elements per FP8 scale block
 E4M3_MAX_F32 = np.float32(448.0)
@@ -435,75 +436,72 @@ def ep_pipeline(logits_ranks, x_ranks, w_gate_bits, w_up_bits, w_down_bits, k: i
 
 # ---- backward ------------------------------------------------------------------------------------
 
-def backward(fwd, dy_bits, logits, w_gate_bits, w_up_bits, w_down_bits, renormalize: bool = True,
-             fp8: bool = False, exact: bool = False):
-    """Gradients of the path for an output gradient dy [T,H] (bf16 bit patterns), given the forward
-    intermediates ``fwd`` of ``pipeline`` (routing, plan, payload, expert outputs).
-
-    The training step of the NCCL EP page (section 3.2) reuses the forward's routing: the gradient is
-    dispatched through the same plan, the experts run backward, and the gradients are combined back.
-    In that order:
-
-    1. Combine backward, for every kept slot (t, j) -> row:
-       d_eo[row] = bf16(fp32(w[t,j] * dy[t]))  (y = sum_j w[t,j] eo[row]; the bf16 rounding of y is
-       taken as the identity), and the routing-weight gradient d_w[t,j] = sum_h dy[t,h] eo[row,h]
-       (exact, stored fp32); a dropped slot has d_w = 0.
-    2. Expert backward on the packed rows of expert e, x the FFN input values (as in the forward):
-       g = x Wg^T, u = x Wu^T, s = sigmoid(g), h = bf16(g s u) (recomputed as the forward made it),
-       dh = d_eo Wd, dg = bf16(dh u s (1 + g (1 - s))), du = bf16(dh g s),
-       dx_rows = bf16(dg Wg + du Wu), dWd = d_eo^T h, dWg = dg^T x, dWu = du^T x (fp64 sums; the
-       weight gradients stored fp32).
-    3. Combine of the input gradients: dx[t] = bf16(sum over kept j of dx_rows[slot_row[t,j]]),
-       fp32 in slot order (the forward combine with unit weights).
-    4. Router: with ``renormalize`` the weights are the softmax of the selected logits, so for a
-       selected expert i of token t  d_logits[t,i] = w_i (d_w_i - sum_j w_j d_w_j), 0 elsewhere;
-       otherwise they are the full-E softmax p, and d_logits[t,i] = p_i (d_i - sum_e p_e d_e) with
-       d_i = d_w of the slot that selected i (0 for unselected experts).  fp64, stored fp32.
-
-    ``exact`` skips every bf16 rounding above and uses the expert outputs without their rounding
-    (all fp64), for checks against finite differences.
-    Returns a dict of dx (bf16 bits [T,H], or float64 when exact), d_logits fp32 [T,E], d_w fp32
-    [T,k], d_w_gate / d_w_up fp32 [E,F,H], d_w_down fp32 [E,H,F], and the intermediates d_eo,
-    dg, du, dx_rows (bf16 bits, or float64 when exact) in packed row order."""
-    rnd = (lambda a: np.asarray(a, dtype=np.float64)) if exact else bf16_round
-    slot_row = np.asarray(fwd["slot_row"], dtype=np.int64)
-    w = np.asarray(fwd["topk_w"], dtype=np.float32)
-    idx = np.asarray(fwd["topk_idx"], dtype=np.int64)
-    off = np.asarray(fwd["expert_offsets"], dtype=np.int64)
-    T, k = slot_row.shape
-    E = off.size - 1
-    S = int(off[E])
+def combine_backward(dy_bits, slot_row, topk_w, expert_out_f64, S: int, exact: bool = False):
+    """Step 1 of the backward (the gradient of the combine), for every kept slot (t, j) -> row:
+    d_eo[row] = bf16(fp32(w[t,j] * dy[t])) (the bf16 rounding of y taken as the identity) and
+    d_w[t,j] = sum_h dy[t,h] eo[row,h] (exact); a dropped slot has d_w = 0.  ``expert_out_f64`` holds
+    the expert outputs' values [S,H].  ``exact`` keeps d_eo in fp64.  Returns (d_eo float64 [S,H],
+    d_w float64 [T,k])."""
+    sr = np.asarray(slot_row, dtype=np.int64)
+    w = np.asarray(topk_w, dtype=np.float32)
     dy = bf16_from_bits(np.asarray(dy_bits, dtype=np.uint16)).astype(np.float64)
+    T, k = sr.shape
     H = dy.shape[1]
-    F = w_gate_bits.shape[1]
-    xin = ffn_inputs(fwd["send"], fwd["send_scales"], fp8)
-    if exact:
-        # the expert outputs without their bf16 roundings
-        eo = np.zeros((S, H))
-        for e in range(E):
-            lo, hi = off[e], off[e + 1]
-            if hi == lo:
-                continue
-            x = np.asarray(xin[lo:hi], dtype=np.float64)
-            g = x @ bf16_from_bits(w_gate_bits[e]).astype(np.float64).T
-            u = x @ bf16_from_bits(w_up_bits[e]).astype(np.float64).T
-            eo[lo:hi] = (g / (1.0 + np.exp(-g)) * u) @ bf16_from_bits(w_down_bits[e]).astype(
-                np.float64).T
-    else:
-        eo = bf16_from_bits(np.asarray(fwd["expert_out"], dtype=np.uint16)).astype(np.float64)
-    # 1. combine backward
     d_eo = np.zeros((S, H), dtype=np.float64)
     d_w = np.zeros((T, k), dtype=np.float64)
     for t in range(T):
         for j in range(k):
-            row = slot_row[t, j]
+            row = sr[t, j]
             if row < 0:
                 continue
             prod = dy[t] * float(w[t, j])
             d_eo[row] = prod if exact else prod.astype(np.float32)
-            d_w[t, j] = float(np.dot(dy[t], eo[row]))
-    d_eo = rnd(d_eo)
-    # 2. expert backward
+            d_w[t, j] = float(np.dot(dy[t], expert_out_f64[row]))
+    return (d_eo if exact else bf16_round(d_eo)), d_w
+
+
+def router_backward(logits, topk_idx, topk_w, d_w, renormalize: bool = True):
+    """Step 4: the router's logit gradient from the routing-weight gradient.  With ``renormalize``
+    the weights are the softmax of the selected logits, so for a selected expert i of token t
+    d_logits[t,i] = w_i (d_w_i - sum_j w_j d_w_j), 0 elsewhere; otherwise they are the full-E
+    softmax p, and d_logits[t,i] = p_i (d_i - sum_e p_e d_e) with d_i = d_w of the slot that
+    selected i (0 for unselected experts).  fp64 [T,E]."""
+    L = np.asarray(logits, dtype=np.float64)
+    idx = np.asarray(topk_idx, dtype=np.int64)
+    w = np.asarray(topk_w, dtype=np.float32)
+    T, k = idx.shape
+    d_logits = np.zeros_like(L)
+    for t in range(T):
+        if renormalize:
+            wt = w[t].astype(np.float64)
+            c = float(np.dot(wt, d_w[t]))
+            for j in range(k):
+                d_logits[t, idx[t, j]] = wt[j] * (d_w[t, j] - c)
+        else:
+            p = np.exp(L[t] - L[t].max())
+            p /= p.sum()
+            d = np.zeros(L.shape[1])
+            for j in range(k):
+                d[idx[t, j]] = d_w[t, j]
+            d_logits[t] = p * (d - float(np.dot(p, d)))
+    return d_logits
+
+
+def expert_backward(xin, d_eo, expert_offsets, w_gate_bits, w_up_bits, w_down_bits,
+                    exact: bool = False):
+    """Step 2: the experts' backward on their packed rows, x = the FFN input values (as in the
+    forward) and d_eo = the output gradient of the rows (float64 [S,H]).  For expert e:
+    g = x Wg^T, u = x Wu^T, s = sigmoid(g), h = bf16(g s u) (recomputed as the forward made it),
+    dh = d_eo Wd, dg = bf16(dh u s (1 + g (1 - s))), du = bf16(dh g s),
+    dx_rows = bf16(dg Wg + du Wu), dWd = d_eo^T h, dWg = dg^T x, dWu = du^T x (fp64 sums).
+    ``exact`` skips the bf16 roundings.  Returns a dict of float64 arrays dg, du [S,F], dx_rows
+    [S,H], d_w_gate, d_w_up [E,F,H], d_w_down [E,H,F]."""
+    rnd = (lambda a: np.asarray(a, dtype=np.float64)) if exact else bf16_round
+    off = np.asarray(expert_offsets, dtype=np.int64)
+    E = off.size - 1
+    S = int(off[E])
+    H = w_gate_bits.shape[2]
+    F = w_gate_bits.shape[1]
     dg_all = np.zeros((S, F))
     du_all = np.zeros((S, F))
     dxr = np.zeros((S, H))
@@ -532,7 +530,51 @@ def backward(fwd, dy_bits, logits, w_gate_bits, w_up_bits, w_down_bits, renormal
         dWu[e] = du.T @ x
         dg_all[lo:hi] = dg
         du_all[lo:hi] = du
-    # 3. combine of the input gradients (unit weights, fp32 in slot order)
+    return {"dg": dg_all, "du": du_all, "dx_rows": dxr, "d_w_gate": dWg, "d_w_up": dWu,
+            "d_w_down": dWd}
+
+
+def backward(fwd, dy_bits, logits, w_gate_bits, w_up_bits, w_down_bits, renormalize: bool = True,
+             fp8: bool = False, exact: bool = False):
+    """Gradients of the path for an output gradient dy [T,H] (bf16 bit patterns), given the forward
+    intermediates ``fwd`` of ``pipeline`` (routing, plan, payload, expert outputs).
+
+    The training step of the NCCL EP page (section 3.2) reuses the forward's routing: the gradient is
+    dispatched through the same plan, the experts run backward, and the gradients are combined back.
+    In that order: ``combine_backward`` (step 1), ``expert_backward`` (step 2), the combine of the
+    input gradients dx[t] = bf16(sum over kept j of dx_rows[slot_row[t,j]]), fp32 in slot order (the
+    forward combine with unit weights; step 3), and ``router_backward`` (step 4).
+
+    ``exact`` skips every bf16 rounding and uses the expert outputs without their rounding (all
+    fp64), for checks against finite differences.
+    Returns a dict of dx (bf16 bits [T,H], or float64 when exact), d_logits fp32 [T,E], d_w fp32
+    [T,k], d_w_gate / d_w_up fp32 [E,F,H], d_w_down fp32 [E,H,F], and the intermediates d_eo,
+    dg, du, dx_rows (bf16 bits, or float64 when exact) in packed row order."""
+    slot_row = np.asarray(fwd["slot_row"], dtype=np.int64)
+    w = np.asarray(fwd["topk_w"], dtype=np.float32)
+    off = np.asarray(fwd["expert_offsets"], dtype=np.int64)
+    T, k = slot_row.shape
+    E = off.size - 1
+    S = int(off[E])
+    H = np.asarray(dy_bits).shape[1]
+    xin = ffn_inputs(fwd["send"], fwd["send_scales"], fp8)
+    if exact:
+        # the expert outputs without their bf16 roundings
+        eo = np.zeros((S, H))
+        for e in range(E):
+            lo, hi = off[e], off[e + 1]
+            if hi == lo:
+                continue
+            x = np.asarray(xin[lo:hi], dtype=np.float64)
+            g = x @ bf16_from_bits(w_gate_bits[e]).astype(np.float64).T
+            u = x @ bf16_from_bits(w_up_bits[e]).astype(np.float64).T
+            eo[lo:hi] = (g / (1.0 + np.exp(-g)) * u) @ bf16_from_bits(w_down_bits[e]).astype(
+                np.float64).T
+    else:
+        eo = bf16_from_bits(np.asarray(fwd["expert_out"], dtype=np.uint16)).astype(np.float64)
+    d_eo, d_w = combine_backward(dy_bits, slot_row, w, eo, S, exact)
+    ex = expert_backward(xin, d_eo, off, w_gate_bits, w_up_bits, w_down_bits, exact)
+    dxr = ex["dx_rows"]
     if exact:
         dx = np.zeros((T, H))
         for t in range(T):
@@ -541,31 +583,15 @@ def backward(fwd, dy_bits, logits, w_gate_bits, w_up_bits, w_down_bits, renormal
                     dx[t] += dxr[slot_row[t, j]]
     else:
         dx = combine(bf16_bits(dxr), slot_row, np.ones((T, k), dtype=np.float32), T, H)
-    # 4. router
-    L = np.asarray(logits, dtype=np.float64)
-    d_logits = np.zeros_like(L)
-    for t in range(T):
-        if renormalize:
-            wt = w[t].astype(np.float64)
-            c = float(np.dot(wt, d_w[t]))
-            for j in range(k):
-                d_logits[t, idx[t, j]] = wt[j] * (d_w[t, j] - c)
-        else:
-            p = np.exp(L[t] - L[t].max())
-            p /= p.sum()
-            d = np.zeros(L.shape[1])
-            for j in range(k):
-                d[idx[t, j]] = d_w[t, j]
-            d_logits[t] = p * (d - float(np.dot(p, d)))
+    d_logits = router_backward(logits, fwd["topk_idx"], w, d_w, renormalize)
     out = {"dx": dx, "d_logits": d_logits.astype(np.float32),
            "d_w": d_w.astype(np.float32),
-           "d_w_gate": dWg if exact else dWg.astype(np.float32),
-           "d_w_up": dWu if exact else dWu.astype(np.float32),
-           "d_w_down": dWd if exact else dWd.astype(np.float32)}
+           "d_w_gate": ex["d_w_gate"] if exact else ex["d_w_gate"].astype(np.float32),
+           "d_w_up": ex["d_w_up"] if exact else ex["d_w_up"].astype(np.float32),
+           "d_w_down": ex["d_w_down"] if exact else ex["d_w_down"].astype(np.float32)}
     if exact:
-        out.update(d_eo=d_eo, dg=dg_all, du=du_all, dx_rows=dxr, d_logits=d_logits,
-                   d_w=d_w)
+        out.update(d_eo=d_eo, dg=ex["dg"], du=ex["du"], dx_rows=dxr, d_logits=d_logits, d_w=d_w)
     else:
-        out.update(d_eo=bf16_bits(d_eo), dg=bf16_bits(dg_all), du=bf16_bits(du_all),
+        out.update(d_eo=bf16_bits(d_eo), dg=bf16_bits(ex["dg"]), du=bf16_bits(ex["du"]),
                    dx_rows=bf16_bits(dxr))
     return out

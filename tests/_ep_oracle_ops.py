@@ -108,5 +108,42 @@ class OracleOps:
         self.calls.append("combine")
         _u16(y)[:] = moe.combine(_u16(expert_out), slot_row.numpy(), topk_w.numpy(), T, H)
 
+    def combine_backward(self, dy, T, H, k, E, logits, renormalize, topk_idx, topk_w, slot_row,
+                         expert_out, d_eo, d_topk_w, d_logits):
+        self.calls.append("combine_backward")
+        S = expert_out.shape[0]
+        eo = moe.bf16_from_bits(_u16(expert_out)).astype(np.float64)
+        de, dw = moe.combine_backward(_u16(dy), slot_row.numpy(), topk_w.numpy(), eo, S)
+        sr = slot_row.numpy()
+        rows = sr[sr >= 0]
+        _u16(d_eo)[rows] = moe.bf16_bits(de[rows])
+        d_topk_w.copy_(torch.from_numpy(dw.astype(np.float32)))
+        dl = moe.router_backward(logits.numpy(), topk_idx.numpy(), topk_w.numpy(), dw, renormalize)
+        d_logits.copy_(torch.from_numpy(dl.astype(np.float32)))
+
+    def expert_backward(self, ffn_input, d_eo, offsets, max_rows, E, H, F, w_gate, w_up, w_down,
+                        dx_rows, d_w_gate, d_w_up, d_w_down, ws):
+        self.calls.append("expert_backward")
+        off = offsets.numpy().astype(np.int64)
+        S = int(off[E])
+        xin = moe.bf16_from_bits(_u16(ffn_input)[:S]).astype(np.float64)
+        de = moe.bf16_from_bits(_u16(d_eo)[:S]).astype(np.float64)
+        r = moe.expert_backward(xin, de, off, _u16(w_gate), _u16(w_up), _u16(w_down))
+        _u16(dx_rows)[:S] = moe.bf16_bits(r["dx_rows"])
+        d_w_gate.copy_(torch.from_numpy(r["d_w_gate"].astype(np.float32)))
+        d_w_up.copy_(torch.from_numpy(r["d_w_up"].astype(np.float32)))
+        d_w_down.copy_(torch.from_numpy(r["d_w_down"].astype(np.float32)))
+
+    def ffn_input_rows(self, rows, scales, payload, ffn_ws, max_rows, H, F):
+        if payload != 1:
+            return rows
+        # the FP8 payload's FFN input: the dequantised rows as bf16 (rows past the received ones
+        # hold whatever the buffer held; they are never read)
+        with np.errstate(over="ignore", invalid="ignore"):
+            vals = moe.ffn_inputs(rows.numpy(), scales.numpy(), True)
+        out = torch.empty((max_rows, H), dtype=torch.bfloat16)
+        _u16(out)[:] = moe.bf16_bits(vals)
+        return out
+
     def sync_status(self, ws) -> int:
         return 0

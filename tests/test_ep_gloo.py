@@ -155,3 +155,50 @@ def test_a_rank_that_leaves_ends_the_others_collectives_with_an_error():
     assert res[world - 1] == "left"
     for r in range(world - 1):
         assert res[r].startswith("error"), (r, res[r])
+
+
+def test_thread_ranks_backward_matches_the_single_device_oracle():
+    """MoeEP.backward over 4 thread ranks (oracle-backed steps), all three exchange modes and both
+    payloads: every rank's dx, d_logits and d_topk_w and its experts' weight gradients equal the
+    single-device oracle's backward over all ranks' tokens, bit for bit."""
+    from combine_moe_route_10_b200.ep import MoeEP
+    from _ep_loopback import run_ranks
+    from _ep_oracle_ops import OracleOps
+    R = 4
+    for payload in ("bf16", "fp8"):
+        w, lg, xs, d = _inputs(R, payload)
+        E_loc = w.E // R
+        g = torch.Generator().manual_seed(3)
+        dys = [torch.randn((T_RANK, w.H), generator=g).to(torch.bfloat16) for _ in range(R)]
+
+        def rank(r, comm):
+            sl = slice(r * E_loc, (r + 1) * E_loc)
+            wts = [d[key][sl].contiguous() for key in ("w_gate", "w_up", "w_down")]
+            out = {}
+            for mode in ("ht", "ll", "p2p"):
+                ep = MoeEP(T_RANK, w.H, w.E, w.k, w.F, comm=comm, payload=payload, mode=mode,
+                           device="cpu", ops=OracleOps())
+                ep.forward(lg[r], xs[r], *wts)
+                gr = ep.backward(dys[r], lg[r], *wts)
+                out[mode] = {key: v.clone() for key, v in gr.items()}
+            return out
+
+        res = run_ranks(R, rank)
+        wb = [bf16_bits(d[key].float().numpy()) for key in ("w_gate", "w_up", "w_down")]
+        fwd = moe.pipeline(np.concatenate([a.numpy() for a in lg]),
+                           np.concatenate([bf16_bits(a.float().numpy()) for a in xs]), *wb, w.k, R,
+                           fp8=payload == "fp8")
+        ref = moe.backward(fwd, np.concatenate([bf16_bits(a.float().numpy()) for a in dys]),
+                           np.concatenate([a.numpy() for a in lg]), *wb, fp8=payload == "fp8")
+        for r in range(R):
+            ts = slice(r * T_RANK, (r + 1) * T_RANK)
+            es = slice(r * E_loc, (r + 1) * E_loc)
+            for mode in ("ht", "ll", "p2p"):
+                got = res[r][mode]
+                what = (payload, mode, r)
+                assert np.array_equal(got["dx"].view(torch.int16).numpy().view(np.uint16),
+                                      ref["dx"][ts]), what
+                assert np.array_equal(got["d_logits"].numpy(), ref["d_logits"][ts]), what
+                assert np.array_equal(got["d_topk_w"].numpy(), ref["d_w"][ts]), what
+                for key in ("d_w_gate", "d_w_up", "d_w_down"):
+                    assert np.array_equal(got[key].numpy(), ref[key][es]), (what, key)

@@ -307,3 +307,47 @@ def test_nccl_one_rank_peer_mode_through_symmetric_memory(cuda):
     finally:
         torch.cuda.synchronize()
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("name", ["tiny", "train-small", "finegrained-small"])
+@pytest.mark.parametrize("mode", ["ht", "ll", "p2p"])
+def test_four_emulated_ranks_backward_equals_the_single_device_backward(cuda, name, mode):
+    """MoeEP.backward over 4 thread ranks on one GPU: dx, d_logits and d_topk_w of every rank and
+    the weight gradients of its experts equal MoeShuffle.backward over all ranks' tokens, bit for
+    bit (every row meets the same kernels in the same order)."""
+    from combine_moe_route_10_b200 import MoeShuffle
+    from combine_moe_route_10_b200.ep import MoeEP
+    R = 4
+    w = mi.get(name)
+    d = mi.make_ep_inputs(w, R, seed=12, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(13)
+    dys = [torch.randn((w.T, w.H), generator=g, device="cuda").to(torch.bfloat16)
+           for _ in range(R)]
+    T = R * w.T
+    single = MoeShuffle(T, w.H, w.E, w.k, R, w.F, payload=w.payload)
+    logits = torch.cat(d["logits"]).contiguous()
+    single.forward(logits, torch.cat(d["x"]).contiguous(), d["w_gate"], d["w_up"], d["w_down"])
+    ref = single.backward(torch.cat(dys).contiguous(), logits, d["w_gate"], d["w_up"],
+                          d["w_down"])
+    torch.cuda.synchronize()
+    assert single.status() == 0
+    E_loc = w.E // R
+
+    def rank(r, comm):
+        sl = slice(r * E_loc, (r + 1) * E_loc)
+        wts = [d[key][sl].contiguous() for key in ("w_gate", "w_up", "w_down")]
+        ep = MoeEP(w.T, w.H, w.E, w.k, w.F, comm=comm, payload=w.payload, mode=mode)
+        ep.forward(d["logits"][r], d["x"][r], *wts)
+        gr = ep.backward(dys[r], d["logits"][r], *wts)
+        torch.cuda.synchronize()
+        assert ep.status() == 0
+        return {key: v.clone() for key, v in gr.items()}
+
+    res = run_ranks(R, rank)
+    for r in range(R):
+        ts = slice(r * w.T, (r + 1) * w.T)
+        es = slice(r * E_loc, (r + 1) * E_loc)
+        for key in ("dx", "d_logits", "d_topk_w"):
+            assert torch.equal(res[r][key], ref[key][ts]), (name, mode, r, key)
+        for key in ("d_w_gate", "d_w_up", "d_w_down"):
+            assert torch.equal(res[r][key], ref[key][es]), (name, mode, r, key)

@@ -105,9 +105,9 @@ def test_rounded_backward_is_close_to_exact():
         assert np.max(np.abs(x - y)) <= 0.03 * np.max(np.abs(y)), name
 
 
-def test_planted_swiglu_derivative_mistake_is_caught():
-    """silu'(g) = s (1 + g (1 - s)): the oracle's backward with the bracket dropped (planted in a
-    copy of its source) no longer matches the finite differences."""
+def test_planted_swiglu_derivative_mistake_is_caught(monkeypatch):
+    """silu'(g) = s (1 + g (1 - s)): the oracle's expert backward with the bracket dropped (planted
+    in a copy of its source) no longer matches the finite differences."""
     import inspect
     logits, xb, wg, wu, wd, dyb, k = _case(3)
     fwd = moe.pipeline(logits, xb, wg, wu, wd, k, 2)
@@ -116,9 +116,10 @@ def test_planted_swiglu_derivative_mistake_is_caught():
                    fwd["topk_idx"], fwd["slot_row"], True)
     good = moe.backward(fwd, dyb, logits, wg, wu, wd, exact=True)
     assert np.allclose(good["d_w_gate"], fd["d_w_gate"], atol=1e-6)
-    text = inspect.getsource(moe.backward)
+    text = inspect.getsource(moe.expert_backward)
     assert "(1.0 + g * (1.0 - sg))" in text
     ns = dict(vars(moe))
     exec(compile(text.replace("(1.0 + g * (1.0 - sg))", "1.0"), "planted", "exec"), ns)
-    bad = ns["backward"](fwd, dyb, logits, wg, wu, wd, exact=True)
+    monkeypatch.setattr(moe, "expert_backward", ns["expert_backward"])
+    bad = moe.backward(fwd, dyb, logits, wg, wu, wd, exact=True)
     assert not np.allclose(bad["d_w_gate"], fd["d_w_gate"], atol=1e-4)
