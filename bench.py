@@ -605,6 +605,26 @@ def measure_ep(w, args, dev, world: int, rank: int) -> dict:
         if ep.status() != 0:
             raise SystemExit(f"expert-parallel {w.name}: device status after timing")
         agg = aggregate(sum(a.elapsed_time(b) for a, b in step_ev), w.T, args.steps, dev)
+        # the backward of the last forward: d_eo to the experts' owners, the experts' backward,
+        # dx_rows back (the same exchange as the forward's), K calls behind an L2 flush
+        g = torch.Generator(device=dev).manual_seed(9)
+        dy = torch.randn((w.T, w.H), generator=g, device=dev).to(torch.bfloat16)
+        for _ in range(args.warmup):
+            flush.fill_(1)
+            ep.backward(dy, logits, wg, wu, wd)
+        bwd_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)]
+                  for _ in range(args.steps)]
+        dist.barrier()
+        torch.cuda.synchronize()
+        for a, b in bwd_ev:
+            flush.fill_(1)
+            a.record(stream)
+            ep.backward(dy, logits, wg, wu, wd)
+            b.record(stream)
+        torch.cuda.synchronize()
+        if ep.status() != 0:
+            raise SystemExit(f"expert-parallel {w.name}: device status after the backward")
+        bwd_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in bwd_ev), dev) / args.steps
         t_pull = sum(e[0].elapsed_time(e[1]) for e in x_ev) / args.steps
         t_push = sum(e[2].elapsed_time(e[3]) for e in x_ev) / args.steps
         pk, _ = peaks()
@@ -616,6 +636,8 @@ def measure_ep(w, args, dev, world: int, rank: int) -> dict:
 
         out = {"mode": "p2p", "workload": w.name, "ranks": R, "experts_per_rank": E_loc,
                "value": agg["value"], "unit": "tokens/s", "ms_per_step": agg["ms_per_step"],
+               "backward_ms": bwd_ms,
+               "train_step_tokens_per_s": R * w.T / ((agg["ms_per_step"] + bwd_ms) * 1e-3),
                "received_rows": n_recv,
                "exchange": {
                    # each received row is read once and written once; at one rank both are HBM

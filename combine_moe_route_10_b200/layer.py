@@ -289,9 +289,27 @@ class MoeShuffle:
                 out.copy_(self.y)
         return g
 
+    def capture_step(self, logits, x, w_gate, w_up, w_down, dy) -> torch.cuda.CUDAGraph:
+        """Record a training step, ``forward`` then ``backward`` for the output gradient ``dy``, on
+        these exact tensors as one CUDA graph (neither half synchronises with the host).  Each
+        ``replay()`` reruns both with whatever ``logits`` / ``x`` / ``dy`` (and the weights) hold;
+        the gradients land in ``self.grads``.  One eager step runs first, outside the capture."""
+        self.forward(logits, x, w_gate, w_up, w_down)
+        self.backward(dy, logits, w_gate, w_up, w_down)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            self.forward(logits, x, w_gate, w_up, w_down)
+            self.backward(dy, logits, w_gate, w_up, w_down)
+        return g
+
     def status(self, stream=None) -> int:
-        """Synchronise and return (then clear) the device status of the dispatch and FFN stages."""
-        a = _lib.moe_sync_status(self.ws_dispatch, stream)
-        b = _lib.moe_sync_status(self.ws_ffn, stream)
-        c = _lib.moe_sync_status(self.ws_ffn_w8, stream) if self.ws_ffn_w8 is not None else 0
-        return a if a != _lib.MOE_OK else (b if b != _lib.MOE_OK else c)
+        """Synchronise and return (then clear) the device status of the dispatch, FFN and backward
+        stages."""
+        found = [_lib.moe_sync_status(self.ws_dispatch, stream),
+                 _lib.moe_sync_status(self.ws_ffn, stream)]
+        if self.ws_ffn_w8 is not None:
+            found.append(_lib.moe_sync_status(self.ws_ffn_w8, stream))
+        if getattr(self, "ws_bwd", None) is not None:
+            found.append(_lib.moe_sync_status(self.ws_bwd, stream))
+        return next((st for st in found if st != _lib.MOE_OK), _lib.MOE_OK)

@@ -189,3 +189,32 @@ def test_backward_full_size(cuda, name):
         assert_close_bf16(dx_rows[lo:hi], ref["dx_rows"], f"{what} dx_rows", row_atol=dxr_atol)
         for key in ("d_w_gate", "d_w_up", "d_w_down"):
             assert _rel_max(np_(grads[key][e]), ref[key][0]) <= 1e-2, (what, key)
+
+
+def test_training_step_graph_replays_the_eager_step(cuda):
+    """forward + backward captured as one CUDA graph: a replay on new inputs written into the
+    captured tensors gives exactly the eager step's outputs and gradients."""
+    from combine_moe_route_10_b200 import MoeShuffle
+    w = mi.get("train-small")
+    d = mi.make_inputs(w, seed=21, device="cuda")
+    d2 = mi.make_inputs(w, seed=22, device="cuda", weights=False)
+    g = torch.Generator(device="cuda").manual_seed(23)
+    dy = torch.randn((w.T, w.H), generator=g, device="cuda").to(torch.bfloat16)
+    dy2 = torch.randn((w.T, w.H), generator=g, device="cuda").to(torch.bfloat16)
+    # eager reference on the second inputs
+    ref = MoeShuffle(w.T, w.H, w.E, w.k, w.R, w.F)
+    y_ref = ref.forward(d2["logits"], d2["x"], d["w_gate"], d["w_up"], d["w_down"]).clone()
+    g_ref = {k_: v.clone() for k_, v in
+             ref.backward(dy2, d2["logits"], d["w_gate"], d["w_up"], d["w_down"]).items()}
+    m = MoeShuffle(w.T, w.H, w.E, w.k, w.R, w.F)
+    logits, x, dyb = d["logits"].clone(), d["x"].clone(), dy.clone()
+    graph = m.capture_step(logits, x, d["w_gate"], d["w_up"], d["w_down"], dyb)
+    logits.copy_(d2["logits"])
+    x.copy_(d2["x"])
+    dyb.copy_(dy2)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert m.status() == 0
+    assert torch.equal(m.y, y_ref)
+    for key, v in g_ref.items():
+        assert torch.equal(m.grads[key], v), key
