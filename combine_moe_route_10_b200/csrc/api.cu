@@ -302,13 +302,15 @@ moe_status_t moe_backward(const void* dy, int T, int H, int k, int E, int F, con
     return MOE_ERR_INVALID_ARG;
   if (static_cast<long long>(T) * k > max_rows) return MOE_ERR_INVALID_ARG;
   if (H % 64 != 0 || F % 64 != 0) return MOE_ERR_UNSUPPORTED;
-  const void* need[] = {topk_idx, topk_w, slot_row, expert_offsets, w_gate, w_up, w_down,
-                        d_logits, d_topk_w, d_w_gate, d_w_up, d_w_down, ws};
+  const void* need[] = {expert_offsets, w_gate, w_up, w_down, d_w_gate, d_w_up, d_w_down, ws};
   for (const void* q : need)
     if (q == nullptr) return MOE_ERR_INVALID_ARG;
-  if (T > 0 && (dy == nullptr || dx == nullptr || ffn_input == nullptr || expert_out == nullptr))
+  // the per-token arrays are empty (possibly NULL) for an empty batch
+  if (T > 0 && (dy == nullptr || dx == nullptr || ffn_input == nullptr || expert_out == nullptr ||
+                topk_idx == nullptr || topk_w == nullptr || slot_row == nullptr ||
+                d_logits == nullptr || d_topk_w == nullptr))
     return MOE_ERR_INVALID_ARG;
-  if (!renormalize && logits == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!renormalize && T > 0 && logits == nullptr) return MOE_ERR_INVALID_ARG;
   const void* a16[] = {dy, dx, ffn_input, expert_out, w_gate, w_up, w_down, d_w_gate, d_w_up,
                        d_w_down};
   for (const void* q : a16)

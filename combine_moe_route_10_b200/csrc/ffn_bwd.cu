@@ -902,7 +902,14 @@ cudaError_t launch_expert_backward(const void* ffn_input, const void* d_eo,
                                    const void* w_gate, const void* w_up, const void* w_down,
                                    void* dx_rows, float* d_w_gate, float* d_w_up, float* d_w_down,
                                    int* status, void* h, void* dg, void* du, cudaStream_t s) {
-  if (max_rows == 0) return cudaSuccess;
+  if (max_rows == 0) {
+    // no rows at all: every expert's gradients are zero
+    const size_t n = static_cast<size_t>(E) * H * F * sizeof(float);
+    cudaError_t e = cudaMemsetAsync(d_w_gate, 0, n, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(d_w_up, 0, n, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(d_w_down, 0, n, s);
+    return e;
+  }
   BwdArgs a{expert_offsets, E, H, F, max_rows, nullptr, nullptr, nullptr, status};
   BwdMaps m1{}, m2{}, m3{};
   const uint64_t mr = static_cast<uint64_t>(max_rows);
@@ -957,7 +964,11 @@ cudaError_t launch_backward(const void* dy, int T, int H, int k, int E, int F, c
   void* du = p;       p += up(r * F * 2);
   void* dx_rows = p;  p += up(r * H * 2);
   float* ones = reinterpret_cast<float*>(p);
-  if (T == 0) return cudaSuccess;
+  if (T == 0) {
+    return launch_expert_backward(ffn_input, d_eo, expert_offsets, 0, E, H, F, w_gate, w_up,
+                                  w_down, dx_rows, d_w_gate, d_w_up, d_w_down, status, h, dg, du,
+                                  s);
+  }
   cudaError_t e = launch_combine_backward(dy, T, H, k, E, logits, renormalize, topk_idx, topk_w,
                                           slot_row, max_rows, expert_out, d_eo, d_topk_w,
                                           d_logits, ones, s);

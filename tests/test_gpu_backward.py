@@ -218,3 +218,42 @@ def test_training_step_graph_replays_the_eager_step(cuda):
     assert torch.equal(m.y, y_ref)
     for key, v in g_ref.items():
         assert torch.equal(m.grads[key], v), key
+
+
+@pytest.mark.parametrize("T,H,E,k,R,F,payload,cf", [
+    (0, 128, 4, 2, 2, 128, "bf16", 0.0),      # empty batch
+    (1, 128, 1, 1, 1, 128, "bf16", 0.0),      # one token, one expert
+    (3, 64, 2, 2, 1, 64, "bf16", 0.0),        # 6 rows in all, one k-block
+    (5, 256, 4, 1, 2, 192, "fp8", 0.0),       # FP8 payload, tiny T, F not a multiple of 128
+    (64, 320, 16, 4, 4, 64, "bf16", 1.0),     # H not a multiple of 256, drops at capacity 16
+    (200, 192, 8, 8, 8, 128, "bf16", 0.0),    # k = E
+    (64, 128, 1024, 32, 32, 64, "bf16", 0.0),  # E and k at their limits: ~2 rows per expert
+    (300, 128, 8, 2, 2, 64, "bf16", 0.01),    # capacity 1: almost every slot dropped
+])
+def test_backward_edge_shapes(cuda, T, H, E, k, R, F, payload, cf):
+    from combine_moe_route_10_b200 import MoeShuffle
+    w = mi.Workload("edge", T, H, E, k, R, F, payload=payload, capacity_factor=cf)
+    d = mi.make_inputs(w, seed=31, device="cuda")
+    cap = moe.capacity(cf, T, k, E)
+    m = MoeShuffle(T, H, E, k, R, F, payload=payload, capacity=cap)
+    m.forward(d["logits"], d["x"], d["w_gate"], d["w_up"], d["w_down"])
+    g = torch.Generator(device="cuda").manual_seed(32)
+    dy = torch.randn((T, H), generator=g, device="cuda").to(torch.bfloat16)
+    grads = m.backward(dy, d["logits"], d["w_gate"], d["w_up"], d["w_down"])
+    torch.cuda.synchronize()
+    assert m.status() == 0
+    if T == 0:
+        for key in ("d_w_gate", "d_w_up", "d_w_down"):
+            assert float(grads[key].abs().max().item()) == 0.0, key
+        return
+    fp8 = payload == "fp8"
+    S = int(m.expert_offsets[E].item())
+    fwd = {"slot_row": np_(m.slot_row), "topk_w": np_(m.topk_w), "topk_idx": np_(m.topk_idx),
+           "expert_offsets": np_(m.expert_offsets), "expert_out": bits16(m.expert_out)[:S],
+           "send": np_(m.send.view(torch.uint8))[:S] if fp8 else bits16(m.send)[:S],
+           "send_scales": np_(m.send_scales)[:S] if fp8 else None}
+    ref = moe.backward(fwd, bits16(dy), np_(d["logits"]), bits16(d["w_gate"]), bits16(d["w_up"]),
+                       bits16(d["w_down"]), fp8=fp8)
+    if cf:
+        assert (np_(m.slot_row) < 0).any()
+    _check(w, m, d, grads, ref, S, f"edge T{T} E{E} k{k}")
