@@ -80,6 +80,9 @@ _SMALL = [
 # tensor-bound like train's (about 1000 rows per expert) while all buffers fit in about 1 GB.
 _PROFILE = [
     Workload("train-e2", 2048, 4096, 2, 1, 2, 14336),
+    # the skewed shapes (H=7168, F=2048, about 256 rows per expert) with 16 experts: the expert
+    # FFN streams its weights like skewed's while the buffers stay at about 2 GB
+    Workload("skewed-e16", 2048, 7168, 16, 2, 16, 2048),
 ]
 WORKLOADS: Dict[str, Workload] = {w.name: w for w in _FULL + _SMALL + _PROFILE}
 
