@@ -385,6 +385,10 @@ def measure(w, args, dev, world: int, rank: int, e2e: bool) -> dict:
         raise SystemExit(f"{w.name}: device status {st} after warm-up")
     S = int(m.expert_offsets[w.E].item())
     active = int((m.expert_counts > 0).sum().item())
+    # rows the FFN's MMAs compute: a 2-CTA tile covers 256 of an expert's rows (experts of more
+    # than 64 rows), a 1-CTA tile 128 (the others); the padding is work the tensor cores do
+    counts = m.expert_counts.cpu().tolist()
+    padded_rows = sum((-(-c // 256) * 256) if c > 64 else (128 if c > 0 else 0) for c in counts)
 
     # Timed region: K metric steps interleaved with K breakdown steps, so both see the same clocks.
     # Metric steps (value, ms_per_step) have events only at step boundaries, so consecutive kernels
@@ -450,7 +454,11 @@ def measure(w, args, dev, world: int, rank: int, e2e: bool) -> dict:
         "traffic": FFN_TRAFFIC.get(w.name), "peak_source": pk_src,
         "algorithmic_bytes": alg["ffn_bytes"], "algorithmic_flops": alg["ffn_flops"],
         "impl_overhead_bytes": alg["ffn_impl_overhead"],
-        "frac_of_max_time_bound": max(ffn_t_hbm, ffn_t_tc) / (t_ffn * 1e-3)})
+        "frac_of_max_time_bound": max(ffn_t_hbm, ffn_t_tc) / (t_ffn * 1e-3),
+        # the bound with the MMAs' padded rows: what the tile shapes leave the kernel to reach
+        "padded_rows": padded_rows,
+        "frac_of_padded_bound": max(ffn_t_hbm, alg["ffn_flops"] * padded_rows / max(S, 1)
+                                    / (pk["bf16_tflops_sustained"] * 1e12)) / (t_ffn * 1e-3)})
 
     def gbs(b, t):
         return b / (t * 1e-3) / 1e9
