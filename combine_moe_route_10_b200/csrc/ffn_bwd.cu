@@ -5,21 +5,25 @@
 //   1. combine_bwd_kernel (warp per token): d_eo[row] = bf16(w[t,j] * dy[t]) for every kept slot,
 //      the routing-weight gradient d_w[t,j] = <dy[t], eo[row]>, and from it the router's logit
 //      gradient (softmax backward over the selected k, or over all E without renormalisation).
-//   2. bwd_gemm_kernel<kRecompute> (tcgen05, M = 128 rows, 128 h columns, k = 32 per stage with the
-//      64-byte swizzle): recomputes g = x Wg^T and u = x Wu^T (one N = 256 MMA over the stacked
-//      gate and up rows) and computes dh = d_eo Wd (N = 128, Wd read MN-major) in the same K loop
-//      over H, then the SwiGLU backward in the epilogue: h, dg, du (bf16).
-//   3. bwd_gemm_kernel<kInputGrad> (M = 128, N = 256): dx_rows = dg Wg + du Wu, one K loop over
+//   2. bwd_gemm_kernel<kRecompute> (tcgen05, M = 256 rows over a CTA pair, 128 h columns, k = 32
+//      per stage with the 64-byte swizzle): recomputes g = x Wg^T and u = x Wu^T (one N = 256 MMA:
+//      CTA 0 stages the gate rows, CTA 1 the up rows) and computes dh = d_eo Wd (N = 128, Wd read
+//      MN-major) in the same K loop over H, then the SwiGLU backward in the epilogue: h, dg, du
+//      (bf16).
+//   3. bwd_gemm_kernel<kInputGrad> (M = 256, N = 256): dx_rows = dg Wg + du Wu, one K loop over
 //      2F, the weights read MN-major.
-//   4. bwd_gemm_kernel<kWeightGrad> (M = 128, N = 256, K = the expert's rows): dWd = d_eo^T h,
+//   4. bwd_gemm_kernel<kWeightGrad> (M = 256, N = 256, K = the expert's rows): dWd = d_eo^T h,
 //      dWg = dg^T x, dWu = du^T x in fp32, both operands MN-major; the rows past the expert's end in
-//      the last K block are zeroed in shared memory before the MMA reads them.
+//      the last K block are zeroed in shared memory before the MMA reads them; TMA stores.
 //   5. the forward combine with unit weights: dx[t] = bf16(sum of dx_rows of its kept slots).
+//   (moe_combine_backward is step 1 alone, moe_expert_backward steps 2-4.)
 //
-// The GEMM kernels are persistent (one CTA per SM, a static tile order), warp-specialised like the
-// forward's single-CTA kernel: warp 0 = TMA producer, warp 1 = TMEM allocation and the MMA thread,
-// warps 2..5 = epilogue, two accumulators so that an epilogue overlaps the next tile's MMAs.  Every
-// wait is bounded (kStatusTimeout); no TMA multicast.
+// The GEMM kernels are persistent 2-CTA clusters (tcgen05.mma.cta_group::2, one CTA per SM, a
+// static tile order shared by both CTAs), warp-specialised like the forward's pair kernel: warp 0
+// = TMA producer (CTA 1's copies complete on CTA 0's barriers), warp 1 = TMEM allocation and, in
+// CTA 0, the MMA thread of the pair, warps 2..5 = epilogue of the CTA's 128 rows; two accumulators
+// (one for the recompute) so that an epilogue overlaps the next tile's MMAs.  Every wait is bounded
+// (kStatusTimeout); no TMA multicast.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
