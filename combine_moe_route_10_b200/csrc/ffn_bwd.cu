@@ -234,25 +234,39 @@ __device__ __forceinline__ int tiles_of(const BwdArgs& a, int rows, int p) {
   return ((M + kPairM - 1) / kPairM) * ((N + kNOut - 1) / kNOut);
 }
 
+// Weight gradients: every (sub-problem, expert) item has the same tile count, so a tile's item is a
+// division (no table).
+__device__ __forceinline__ int wgrad_tiles_per_item(const BwdArgs& a) {
+  return ((a.H + kPairM - 1) / kPairM) * ((a.F + kNOut - 1) / kNOut);
+}
+
 template <int MODE>
 __device__ __forceinline__ Tile decode(const BwdArgs& a, const int* start, int tile) {
-  // start[i] = first tile of item i, items = experts (x 3 sub-problems for the weight grads)
-  const int n_items = MODE == kWeightGrad ? 3 * a.E : a.E;
+  if (MODE == kWeightGrad) {
+    // items p*E + e in order; dWd [H, F] and dWg, dWu [F, H] have the same 256 x 256 tile count
+    const int per = wgrad_tiles_per_item(a);
+    const int item = tile / per, local = tile - item * per;
+    Tile t;
+    t.p = item / a.E;
+    t.e = item % a.E;
+    // both operands (the expert's rows) stay in L2 across the output blocks
+    const int ncol = ((t.p == 0 ? a.F : a.H) + kNOut - 1) / kNOut;
+    t.mb = local / ncol;
+    t.nb = local % ncol;
+    return t;
+  }
+  // start[i] = first tile of expert i
+  const int n_items = a.E;
   int lo = 0, hi = n_items - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
     if (start[mid] <= tile) lo = mid; else hi = mid - 1;
   }
   Tile t;
-  t.p = MODE == kWeightGrad ? lo / a.E : 0;
-  t.e = MODE == kWeightGrad ? lo % a.E : lo;
+  t.p = 0;
+  t.e = lo;
   const int local = tile - start[lo];
-  if (MODE == kWeightGrad) {
-    // both operands (the expert's rows) stay in L2 across the output blocks
-    const int ncol = ((t.p == 0 ? a.F : a.H) + kNOut - 1) / kNOut;
-    t.mb = local / ncol;
-    t.nb = local % ncol;
-  } else {
+  {
     // row blocks fastest: the tiles running at the same time share one weight slice, which then
     // crosses HBM once per expert instead of once per row block
     const int rows = __ldg(a.expert_offsets + t.e + 1) - __ldg(a.expert_offsets + t.e);
@@ -287,9 +301,12 @@ __device__ __forceinline__ void tma_store3d(const CUtensorMap* tm, uint32_t src,
       : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// The shared-memory source of every store issued so far has been read.
+// The shared-memory source of every store issued so far has been read (_1: all but the latest).
 __device__ __forceinline__ void bulk_wait_read() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read_1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
@@ -306,8 +323,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   // 1024-byte aligned stages, then the store staging, barriers and the tile prefix table
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  constexpr int kOutBytes = MODE == kWeightGrad ? 4 * kStageOutBytes : 0;
-  uint8_t* out_stage = base + kStages * kStageBytes;  // 1024-aligned: [4 warps][32 x 32 fp32]
+  constexpr int kOutBytes = MODE == kWeightGrad ? 8 * kStageOutBytes : 0;
+  uint8_t* out_stage = base + kStages * kStageBytes;  // 1024-aligned: [4 warps][2][32 x 32 fp32]
   uint64_t* bars = reinterpret_cast<uint64_t*>(out_stage + kOutBytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + kStages;
@@ -347,7 +364,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
   griddep_wait();
   griddep_launch_dependents();
-  if (warp == 2 && lane == 0) {
+  if (MODE == kWeightGrad) {
+    if (threadIdx.x == 0) start[0] = 3 * E * wgrad_tiles_per_item(args);  // the tile count
+  } else if (warp == 2 && lane == 0) {
     int run = 0;
     for (int i = 0; i < n_items; ++i) {
       start[i] = run;
@@ -362,7 +381,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   pair_sync();  // both CTAs' barriers are initialised before any remote arrive or copy
   fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = start[n_items];
+  const int total = MODE == kWeightGrad ? start[0] : start[n_items];
   const uint32_t stage0 = smem_addr(base);
 
   if (warp == 0) {
@@ -550,6 +569,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int r = static_cast<int>(rank) * kBM + quarter * 32 + lane;  // row of the pair tile
     const uint32_t acc_empty0 = mapa(smem_addr(&acc_empty[0]), 0);
     const uint32_t acc_empty1 = mapa(smem_addr(&acc_empty[1]), 0);
+    // weight gradients: the stores of consecutive blocks, across tiles too, alternate between
+    // this warp's two staging blocks
+    int chunk = 0;
     int it = 0;
     for (int tile = cid; tile < total; tile += ncl, ++it) {
       const Tile t = decode<MODE>(args, start, tile);
@@ -635,24 +657,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int N = t.p == 0 ? args.F : args.H;
         const CUtensorMap* om = &maps.out[t.p];
         const bool any_k = rows > 0;  // uniform over the warp
-        uint8_t* stg = out_stage + quarter * kStageOutBytes;
+        uint8_t* stg = out_stage + 2 * quarter * kStageOutBytes;  // this warp's two blocks
         const uint32_t stg_addr = smem_addr(stg);
         if (!any_k) {
           // an expert without rows: one zero block, stored to every 32-column block of this
           // warp's rows without waiting in between (the source does not change)
+          const int zb = chunk & 1;
           if (lane == 0) bulk_wait_read();
           __syncwarp();
-          uint4* row_p = reinterpret_cast<uint4*>(stg + lane * 128);
+          uint4* row_p = reinterpret_cast<uint4*>(stg + zb * kStageOutBytes + lane * 128);
 #pragma unroll
           for (int q = 0; q < 8; ++q) row_p[q] = make_uint4(0u, 0u, 0u, 0u);
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           __syncwarp();
           if (lane == 0) {
             for (int c = 0; c < kNOut && t.nb * kNOut + c < N; c += 32)
-              tma_store3d(om, stg_addr, t.nb * kNOut + c,
+              tma_store3d(om, stg_addr + zb * kStageOutBytes, t.nb * kNOut + c,
                           t.mb * kPairM + static_cast<int>(rank) * kBM + quarter * 32, t.e);
             bulk_commit();
           }
+          ++chunk;
         }
 #pragma unroll 1
         for (int c = 0; any_k && c < kNOut; c += 32) {
@@ -661,20 +685,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           uint32_t v[32];
           ld32(tb + c, v);
           ld_wait();
-          // the previous block's store has read the staging block
-          if (lane == 0) bulk_wait_read();
+          // alternate staging blocks: the store issued two blocks ago (same block) has read it,
+          // the previous block's store may still be reading the other one
+          const int b = chunk & 1;
+          if (lane == 0) bulk_wait_read_1();
           __syncwarp();
-          uint4* row_p = reinterpret_cast<uint4*>(stg + lane * 128);
+          uint4* row_p = reinterpret_cast<uint4*>(stg + b * kStageOutBytes + lane * 128);
 #pragma unroll
           for (int q = 0; q < 8; ++q)
             row_p[q ^ (lane & 7)] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           __syncwarp();
           if (lane == 0) {
-            tma_store3d(om, stg_addr, col,
+            tma_store3d(om, stg_addr + b * kStageOutBytes, col,
                         t.mb * kPairM + static_cast<int>(rank) * kBM + quarter * 32, t.e);
             bulk_commit();
           }
+          ++chunk;
         }
       }
       fence_before();
@@ -817,8 +844,10 @@ bool tmap_bf16(CUtensorMap* tm, const void* ptr, uint64_t rows, uint64_t cols, u
 
 template <int MODE>
 size_t bwd_smem() {
+  // stages, store staging, barriers, and the tile table (E + 1 entries; none for the weights)
   return 1024 + static_cast<size_t>(Cfg<MODE>::kStages) * Cfg<MODE>::kStageBytes +
-         (MODE == kWeightGrad ? 4 * kStageOutBytes : 0) + 256 + 4 * (3 * 1024 + 1);
+         (MODE == kWeightGrad ? 8 * kStageOutBytes : 0) + 256 +
+         (MODE == kWeightGrad ? 16 : 4 * (1024 + 1));
 }
 
 // fp32 [E][M][N] (N contiguous) written in 32 x 32 boxes from a 128-byte-swizzled staging block;
