@@ -162,6 +162,21 @@ def algorithmic(w, S: int, active_experts: int):
                 ffn_impl_overhead=overhead, ffn_flops=ffn_flops, combine=combine)
 
 
+def ffn_mma_rows(n: int) -> int:
+    """Rows the FFN's MMAs compute for an expert of n rows: a 128-row tile up to 64 rows (one
+    CTA), the rows rounded up to 16 per chunk of at most 256 up to 512 rows (weights as M, rows as
+    N), pairs of 128-row blocks beyond."""
+    if n <= 0:
+        return 0
+    if n <= 64:
+        return 128
+    if n <= 512:
+        c = -(-n // 256)
+        per = -(-(-(-n // c)) // 16) * 16
+        return sum(-(-min(per, n - u * per) // 16) * 16 for u in range(c))
+    return -(-n // 256) * 256
+
+
 def cpu_baseline_run(w, d_cpu, budget_s: float = 12.0, n_tokens: int | None = None):
     """Oracle pipeline on a bounded token sample (the first n tokens).  Returns (tokens/s, info)."""
     import numpy as np
@@ -388,7 +403,7 @@ def measure(w, args, dev, world: int, rank: int, e2e: bool) -> dict:
     # rows the FFN's MMAs compute: a 2-CTA tile covers 256 of an expert's rows (experts of more
     # than 64 rows), a 1-CTA tile 128 (the others); the padding is work the tensor cores do
     counts = m.expert_counts.cpu().tolist()
-    padded_rows = sum((-(-c // 256) * 256) if c > 64 else (128 if c > 0 else 0) for c in counts)
+    padded_rows = sum(ffn_mma_rows(int(c)) for c in counts)
 
     # Timed region: K metric steps interleaved with K breakdown steps, so both see the same clocks.
     # Metric steps (value, ms_per_step) have events only at step boundaries, so consecutive kernels
