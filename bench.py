@@ -164,16 +164,11 @@ def algorithmic(w, S: int, active_experts: int):
 
 def ffn_mma_rows(n: int) -> int:
     """Rows the FFN's MMAs compute for an expert of n rows: a 128-row tile up to 64 rows (one
-    CTA), the rows rounded up to 16 per chunk of at most 256 up to 512 rows (weights as M, rows as
-    N), pairs of 128-row blocks beyond."""
+    CTA), pairs of 128-row blocks (256 rows per 2-CTA tile) beyond."""
     if n <= 0:
         return 0
     if n <= 64:
         return 128
-    if n <= 512:
-        c = -(-n // 256)
-        per = -(-(-(-n // c)) // 16) * 16
-        return sum(-(-min(per, n - u * per) // 16) * 16 for u in range(c))
     return -(-n // 256) * 256
 
 

@@ -19,14 +19,6 @@
 //   columns.  GEMM-1 puts the gate rows in CTA 0's half of B and the up rows in CTA 1's.  CTA 1's
 //   TMA loads complete their bytes on CTA 0's barriers, CTA 0's single MMA thread issues for both
 //   and its commits arrive on both CTAs' barriers (multicast commit, not multicast loads).
-//   Experts of 65..512 rows run in the same kernel with the operands swapped, so that an expert of
-//   160 rows does not compute 256: the weights are the M = 256 operand (CTA v: GEMM-1 gate rows of
-//   64 columns of h in TMEM lanes 0..63 and the matching up rows in lanes 64..127; GEMM-2 128 rows
-//   of W_down) and the expert's rows are N, in one or two chunks of at most 256 rows rounded up to
-//   16 (CTA v stages half of them).  Each CTA loads three boxes per k-step (gate, up, rows; two in
-//   GEMM-2), and the epilogue reads each TMEM lane as one column of h or of the output across the
-//   chunk's rows; the gate and up warps of a lane range swap half of each 32-row chunk through
-//   shared memory to form SwiGLU.
 // * ffn_single_kernel: experts with at most 64 rows (a tile is bound by streaming the expert's
 //   weights, not by the MMA).  One CTA per tile: tcgen05.mma.cta_group::1 (M = 128, N = 256),
 //   40 KB stages (an A box of 16, 32 or 64 rows + the whole weight tile), five in flight.
@@ -65,10 +57,6 @@ constexpr int kATileBytes = BM * BK * 2;   // 16 KB: 128 rows of A
 constexpr int kBHalfBytes = 128 * BK * 2;  // 16 KB: 128 weight rows
 // Experts with at most this many rows run in the single-block kernel, the others in the pair kernel.
 constexpr int kSingleMaxRows = 64;
-// Pair-kernel experts with at most this many rows run with the operands swapped (weights as the
-// MMA's M = 256, the expert's rows as N, a multiple of 16), in one or two chunks of at most 256
-// rows.  Experts with more rows run as pairs of 128-row blocks.
-constexpr int kSwapMaxRows = 512;
 // Pair kernel: six 32-KB stages (A rows + half of B).  Single kernel: five 40-KB stages (an A box of
 // at most 64 rows + all 256 rows of B).
 constexpr int kStagesPair = 6;
@@ -179,16 +167,6 @@ __device__ __forceinline__ void tc_mma2(uint32_t d_tmem, uint64_t a_desc, uint64
       "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
-}
-
-// A pair kernel load: CTA 0 completes on its own barrier `bar`, CTA 1 on CTA 0's (`bar` is then
-// the shared::cluster address of CTA 0's barrier).
-__device__ __forceinline__ void pair_load(uint32_t rank, uint32_t dst, const CUtensorMap* tm,
-                                          uint32_t bar, int x, int y) {
-  if (rank == 0)
-    tma_load_2d(dst, tm, bar, x, y);
-  else
-    tma_load_2d_to_leader(dst, tm, bar, x, y);
 }
 
 // ---- cluster helpers ---------------------------------------------------------------------------
@@ -331,28 +309,21 @@ __device__ __forceinline__ bool wait_counter(const int* p, int target, const Abo
   }
 }
 
-// Tensor maps of the row operands (input rows, h) with row boxes of 16, 32, ..., 112: a block
-// with few rows loads only its rows rounded up to 16 (the stale rows above them in shared memory
-// feed only accumulator rows or columns the epilogue does not store); 128 rows use the full map.
-constexpr int kSmallBoxes = 7;
+// Tensor maps of the A operand (input rows, h) with row boxes of 16, 32 and 64: a row block with
+// few rows loads only the rows it has (the stale rows above them in shared memory feed only
+// accumulator rows the epilogue does not store).
 struct SmallBoxMaps {
-  CUtensorMap m[kSmallBoxes];
+  CUtensorMap m[3];
 };
-__host__ __device__ constexpr int small_box_rows(int i) { return 16 * (i + 1); }
-// Index of the box for `rows` rows: 0..6 a small box, 7 the full 128-row map.
+__host__ __device__ constexpr int small_box_rows(int i) { return 16 << i; }
 __device__ __forceinline__ int small_box_index(int rows) {
-  return rows <= 0 ? 0 : min((rows + 15) / 16, 8) - 1;
+  return rows <= 16 ? 0 : (rows <= 32 ? 1 : (rows <= 64 ? 2 : 3));
 }
-// Gate and up weight maps with 64-row boxes: a swapped GEMM-1 tile stages 64 gate rows (TMEM
-// lanes 0..63) and the 64 up rows of the same columns (lanes 64..127) per CTA.
-struct SwapMaps {
-  CUtensorMap g64, u64;
-};
 // Bytes of the A box that covers `rows` rows (0 when there are none).
 __device__ __forceinline__ uint32_t a_box_bytes(int rows) {
   if (rows <= 0) return 0u;
   const int bi = small_box_index(rows);
-  return bi < kSmallBoxes ? static_cast<uint32_t>(small_box_rows(bi) * BK * 2) : kATileBytes;
+  return bi < 3 ? static_cast<uint32_t>(small_box_rows(bi) * BK * 2) : kATileBytes;
 }
 
 // ---- tile schedule -------------------------------------------------------------------------------
@@ -376,8 +347,9 @@ struct FfnArgs {
   int* done;                      // [row blocks] GEMM-1 completion counters, zero on entry
   int* used;                      // [row blocks] GEMM-2 tiles that passed the wait, zero on entry
   int* sched;                     // [2] this kernel's next tile to claim, CTAs that finished
-  // Per-expert weight descriptors (moe_ffn_weight_list_init): kListMaps per expert, rows local to
-  // the expert; nullptr: the grid-constant maps of the contiguous [E, ...] weights, rows global.
+  // Per-expert weight descriptors (moe_ffn_weight_list_init): 4 per expert (gate, up, down with
+  // 128-row and 256-row boxes), rows local to the expert; nullptr: the grid-constant maps of the
+  // contiguous [E, ...] weights, rows global.
   const CUtensorMap* wlist;
   // FP8 first projection (all three non-null) or bf16 (all null): the A and gate / up maps then
   // hold e4m3 codes, x_scale [max_rows] the input rows' scales, g_scale / u_scale [E*F] the
@@ -392,13 +364,8 @@ __device__ __forceinline__ int k_per_stage(const FfnArgs& a, int phase) {
   return (phase == 1 && a.x_scale != nullptr) ? 128 : BK;
 }
 
-// Descriptors per expert in a weight list: gate, up (128-row boxes), down (128- and 256-row
-// boxes), gate, up (64-row boxes).
-constexpr int kListMaps = 6;
-
 // The descriptor of the weight tile a tile loads, and its first row.  `which`: 0 gate, 1 up,
-// 2 down (128-row box), 3 down (256-row box), 4 gate, 5 up (64-row boxes); `local_row` is the row
-// inside expert e's matrix.
+// 2 down (128-row box), 3 down (256-row box); `local_row` is the row inside expert e's matrix.
 __device__ __forceinline__ const CUtensorMap* weight_map(const FfnArgs& args, const CUtensorMap* tm,
                                                          int e, int which, int local_row,
                                                          int rows_per_expert, int& row) {
@@ -406,34 +373,13 @@ __device__ __forceinline__ const CUtensorMap* weight_map(const FfnArgs& args, co
     row = e * rows_per_expert + local_row;
     return tm;
   }
-  const CUtensorMap* m = args.wlist + kListMaps * e + which;
+  const CUtensorMap* m = args.wlist + 4 * e + which;
   // the descriptors were written to global memory by a copy before this launch
   asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(
                    reinterpret_cast<uint64_t>(m))
                : "memory");
   row = local_row;
   return m;
-}
-
-// Whether an expert of n rows runs with swapped operands in the pair kernel.
-__device__ __forceinline__ bool swapped(int n) { return n > kSingleMaxRows && n <= kSwapMaxRows; }
-// Chunk `unit` of a swapped expert of n rows: ceil(n / 256) chunks of equal size rounded up to 16
-// rows (the last one holds the remainder); `n_mma` is the MMA's N, the chunk's rows rounded up to
-// 16, so each CTA of the pair stages n_mma / 2 (a multiple of 8) of them.
-struct SwapChunk {
-  int row0;   // first row of the chunk inside the expert
-  int rows;   // real rows
-  int n_mma;  // MMA N
-};
-__host__ __device__ constexpr int swap_chunks(int n) { return (n + 255) / 256; }
-__device__ __forceinline__ SwapChunk swap_chunk(int n, int unit) {
-  const int c = swap_chunks(n);
-  const int per = ((n + c - 1) / c + 15) / 16 * 16;
-  SwapChunk k;
-  k.row0 = unit * per;
-  k.rows = min(per, n - k.row0);
-  k.n_mma = (k.rows + 15) / 16 * 16;
-  return k;
 }
 
 struct Tables {
@@ -474,12 +420,9 @@ __device__ __forceinline__ void build_tables(const Tables& tb, const FfnArgs& ar
     }
     const int mt = (max(hi - lo, 0) + BM - 1) / BM;
     const bool paired = hi - lo > kSingleMaxRows;
-    // pair-kernel units: chunks of a swapped expert, else pairs of row blocks (a chunk never
-    // outnumbers the row blocks, so unit u of expert e may use GEMM-1 counter ms_rb[e] + u)
-    const int pu = swapped(hi - lo) ? swap_chunks(hi - lo) : (mt + 1) / 2;
-    const int u = PAIRS ? (paired ? pu : 0) : (paired ? 0 : mt);
+    const int u = PAIRS ? (paired ? (mt + 1) / 2 : 0) : (paired ? 0 : mt);
     n_single += __popc(__ballot_sync(0xFFFFFFFFu, !paired && mt == 1));
-    n_pairs += paired ? pu : 0;
+    n_pairs += paired ? (mt + 1) / 2 : 0;
     int ir = mt, iu = u;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -559,19 +502,17 @@ __device__ __forceinline__ FTile fdecode(const Tables& tb, int E, int n1, int n2
   return t;
 }
 
-// GEMM-2 producer side of counter slot `slot`: wait until `writers` epilogue warps have published
-// their rows of h, then the last of the `readers` GEMM-2 producers of the slot to get here returns
-// both counters to zero, so the workspace is ready for the next call without a memset.  A row
-// block (slot ms_rb[e] + m_blk) has 4 * n1 writers (four warps of one CTA per GEMM-1 tile) and n2
-// readers; a swapped chunk (slot ms_rb[e] + chunk) has 8 * n1 writers (both CTAs of every GEMM-1
-// tile write some of its columns) and 2 * n2 readers (both CTAs load half of its rows).
-__device__ __forceinline__ bool gemm2_acquire(const FfnArgs& args, int slot, int writers,
-                                              int readers, const Abort& ab) {
-  if (!wait_counter(args.done + slot, writers, ab)) return false;
+// GEMM-2 producer side of row block m_blk of expert e: wait for its rows of h, then the last of the
+// n2 GEMM-2 tiles of the block to get here returns both counters to zero, so the workspace is
+// ready for the next call without a memset.
+__device__ __forceinline__ bool gemm2_acquire(const FfnArgs& args, const Tables& tb, int e,
+                                              int m_blk, int n1, int n2, const Abort& ab) {
+  const int rb = tb.ms_rb[e] + m_blk;
+  if (!wait_counter(args.done + rb, 4 * n1, ab)) return false;
   asm volatile("fence.proxy.async.global;" ::: "memory");
-  if (atomicAdd(args.used + slot, 1) == readers - 1) {
-    atomicExch(args.done + slot, 0);
-    atomicExch(args.used + slot, 0);
+  if (atomicAdd(args.used + rb, 1) == n2 - 1) {
+    atomicExch(args.done + rb, 0);
+    atomicExch(args.used + rb, 0);
   }
   return true;
 }
@@ -648,144 +589,10 @@ __device__ __forceinline__ void epilogue_tile(const FfnArgs& args, const Tables&
   }
 }
 
-// Bounded wait until the shared-memory counter *p, written by another warp of this CTA, reaches
-// `target`.  False if the CTA aborts or the limit runs out (which raises the abort).
-__device__ __forceinline__ bool wait_smem_count(const volatile int* p, int target,
-                                                const Abort& ab) {
-  if (*p >= target) return true;
-  const unsigned long long t0 = global_timer_ns();
-  while (true) {
-    if (*p >= target) return true;
-    if (*ab.local) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
-      ab.raise_timeout();
-      return false;
-    }
-  }
-}
-
-// Epilogue of a swapped tile for this warp's 32 accumulator lanes: TMEM lanes are weight rows of
-// this CTA's half of M, TMEM columns are the chunk's rows.
-// * GEMM-1: lanes 0..63 hold gate rows f = n_blk * 128 + 64 rank + (lane index), lanes 64..127
-//   the up rows of the same f, so quadrant q (gate) and quadrant q + 2 (up) form warp pair
-//   p = q & 1 with f = n_blk * 128 + 64 rank + 32 p + lane.  Per 32-column chunk the gate warp
-//   passes g of columns 16..31 to the up warp and receives u of columns 0..15 (shared memory,
-//   full / empty sequence counters, bounded waits), so the gate warp computes h for columns
-//   0..15 and the up warp for columns 16..31.  `xseq` counts this warp's exchanges (both warps of
-//   a pair take the same tiles and chunks, so their counts agree).
-// * GEMM-2: lane l of quadrant q holds output column n_blk * 256 + 128 rank + 32 q + l.
-// Stores: lanes l and l ^ 1 hold adjacent columns; the even lane writes both of them for the even
-// rows, the odd lane for the odd rows, so every store is a 4-byte pair.
-// Returns false if the CTA aborts during an exchange.
-__device__ __forceinline__ bool epilogue_swap(const FfnArgs& args, const Tables& tb, float* xchg,
-                                              volatile int* xflag, int phase, int e, int unit,
-                                              int n_blk, uint32_t t_acc, int quarter, int lane,
-                                              uint32_t rank, int& xseq, const Abort& ab) {
-  const int n_e = tb.off[e + 1] - tb.off[e];
-  const SwapChunk ch = swap_chunk(n_e, unit);
-  const int row0 = tb.off[e] + ch.row0;  // row of accumulator column 0
-  const bool odd = (lane & 1) != 0;
-  if (phase == 1) {
-    const bool gate = quarter < 2;
-    const int p = quarter & 1;
-    const int f = n_blk * 128 + static_cast<int>(rank) * 64 + p * 32 + lane;
-    const bool w8 = args.x_scale != nullptr;
-    float sg = 1.0f, su = 1.0f;
-    if (w8 && f < args.F) {
-      sg = __ldg(args.g_scale + static_cast<size_t>(e) * args.F + f);
-      su = __ldg(args.u_scale + static_cast<size_t>(e) * args.F + f);
-    }
-    const int fc = f - (odd ? 1 : 0);  // even: F % 64 == 0, so fc and fc + 1 are both in or out
-    const int sdir = gate ? 0 : 1;     // 0: gate -> up, 1: up -> gate
-    float* sbuf = xchg + (p * 2 + sdir) * 512;
-    const float* rbuf = xchg + (p * 2 + (sdir ^ 1)) * 512;
-    volatile int* sfl = xflag + p * 4 + sdir * 2;        // [full, empty] of what this warp sends
-    volatile int* rfl = xflag + p * 4 + (sdir ^ 1) * 2;  // ... of what it receives
-#pragma unroll 1
-    for (int c0 = 0; c0 < ch.rows; c0 += 32) {
-      uint32_t a[32];
-      tmem_ld32(t_acc + c0, a);
-      tmem_wait_ld();
-      ++xseq;
-      // send: the partner has taken the previous exchange out of this buffer
-      if (!wait_smem_count(sfl + 1, xseq - 1, ab)) return false;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) sbuf[i * 32 + lane] = __uint_as_float(gate ? a[16 + i] : a[i]);
-      __syncwarp();
-      if (lane == 0) {
-        __threadfence_block();
-        sfl[0] = xseq;
-      }
-      // receive
-      if (!wait_smem_count(rfl, xseq, ab)) return false;
-      __threadfence_block();
-      float other[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) other[i] = rbuf[i * 32 + lane];
-      __syncwarp();
-      if (lane == 0) {
-        __threadfence_block();
-        rfl[1] = xseq;
-      }
-      const int cb = c0 + (gate ? 0 : 16);  // first column of this warp's (g, u) pairs
-      float hv[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float g = gate ? __uint_as_float(a[i]) : other[i];
-        float u = gate ? other[i] : __uint_as_float(a[16 + i]);
-        if (w8) {
-          // the FP8 first projection's scales: the row's (this column's) times the weight row's
-          const float sx = cb + i < ch.rows ? __ldg(args.x_scale + row0 + cb + i) : 1.0f;
-          g *= sx * sg;
-          u *= sx * su;
-        }
-        hv[i] = silu_mul(g, u);
-      }
-#pragma unroll
-      for (int i = 0; i < 16; i += 2) {
-        const float theirs = __shfl_xor_sync(0xFFFFFFFFu, odd ? hv[i] : hv[i + 1], 1);
-        const int c = cb + i + (odd ? 1 : 0);
-        if (c < ch.rows && fc < args.F)
-          *reinterpret_cast<uint32_t*>(args.h + static_cast<size_t>(row0 + c) * args.F + fc) =
-              odd ? pack_bf16x2(theirs, hv[i + 1]) : pack_bf16x2(hv[i], theirs);
-      }
-    }
-    // publish: this warp's columns of h for the chunk are written
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-    __threadfence();
-    __syncwarp();
-    if (lane == 0) red_release_add(args.done + tb.ms_rb[e] + unit, 1);
-  } else {
-    const int hc = n_blk * 256 + static_cast<int>(rank) * 128 + quarter * 32 + lane - (odd ? 1 : 0);
-    const bool col_ok = hc < args.H;  // even: H % 64 == 0
-#pragma unroll 1
-    for (int c0 = 0; c0 < ch.rows; c0 += 32) {
-      uint32_t a[32];
-      tmem_ld32(t_acc + c0, a);
-      tmem_wait_ld();
-#pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        const float v0 = __uint_as_float(a[i]), v1 = __uint_as_float(a[i + 1]);
-        const float theirs = __shfl_xor_sync(0xFFFFFFFFu, odd ? v0 : v1, 1);
-        const int c = c0 + i + (odd ? 1 : 0);
-        if (col_ok && c < ch.rows)
-          *reinterpret_cast<uint32_t*>(args.out + static_cast<size_t>(row0 + c) * args.H + hc) =
-              odd ? pack_bf16x2(theirs, v1) : pack_bf16x2(v0, theirs);
-      }
-    }
-  }
-  return true;
-}
-
 // Shared-memory layout common to both kernels: the stage ring, the mbarriers, the tile queue and
 // the tables.
 struct Ring {
   uint8_t* tiles;
-  // pair kernel: the swapped GEMM-1 epilogue's exchange between the gate and up warps of each of
-  // two warp pairs, [pair][direction][16 columns][32 lanes] fp32, and its sequence flags
-  // [pair][direction][full, empty]
-  float* xchg;
-  volatile int* xflag;
   uint64_t *full, *empty, *acc_full, *acc_empty, *drain, *q_full, *q_empty;
   int* tile_q;  // [kTileQ] claimed tile ids (-1: no more tiles)
   uint32_t* tmem_base;
@@ -793,23 +600,12 @@ struct Ring {
   Tables tb;
 };
 
-constexpr int kXchgFloats = 2 * 2 * 16 * 32;
-constexpr int kXchgBytes = kXchgFloats * 4 + 8 * 4;
-
-__device__ __forceinline__ Ring carve(uint8_t* raw, int E, int stages, int stage_bytes,
-                                      bool xchg) {
+__device__ __forceinline__ Ring carve(uint8_t* raw, int E, int stages, int stage_bytes) {
   Ring s;
   const uint32_t a = smem_addr(raw);
   uint8_t* p = raw + ((1024u - (a & 1023u)) & 1023u);
   s.tiles = p;
   p += static_cast<size_t>(stages) * stage_bytes;
-  s.xchg = nullptr;
-  s.xflag = nullptr;
-  if (xchg) {
-    s.xchg = reinterpret_cast<float*>(p);
-    s.xflag = reinterpret_cast<volatile int*>(s.xchg + kXchgFloats);
-    p += kXchgBytes;
-  }
   s.full = reinterpret_cast<uint64_t*>(p);
   s.empty = s.full + stages;
   s.acc_full = s.empty + stages;
@@ -824,8 +620,8 @@ __device__ __forceinline__ Ring carve(uint8_t* raw, int E, int stages, int stage
   return s;
 }
 
-size_t ring_smem_bytes(int E, int stages, int stage_bytes, bool xchg) {
-  return 1024 + static_cast<size_t>(stages) * stage_bytes + (xchg ? kXchgBytes : 0) +
+size_t ring_smem_bytes(int E, int stages, int stage_bytes) {
+  return 1024 + static_cast<size_t>(stages) * stage_bytes +
          8 * (2 * static_cast<size_t>(stages) + 5 + 2 * kTileQ) + 16 +
          sizeof(int) * (static_cast<size_t>(table_ints(E)) + 2 + kTileQ);
 }
@@ -846,8 +642,6 @@ __device__ __forceinline__ void init_ring(const Ring& s, int stages, int acc_emp
     mbar_init(smem_addr(&s.q_empty[i]), q_consumers);
   }
   *s.abort_flag = 0;
-  if (s.xflag != nullptr)
-    for (int i = 0; i < 8; ++i) s.xflag[i] = 0;
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -894,7 +688,7 @@ __device__ __forceinline__ void prefetch_maps(const CUtensorMap* a, const CUtens
   const CUtensorMap* all[5] = {a, d, b, c, e};  // x, h, then the three weight maps
   for (int i = 0; i < (weights ? 5 : 2); ++i)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(all[i])) : "memory");
-  for (int i = 0; i < kSmallBoxes; ++i) {
+  for (int i = 0; i < 3; ++i) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xs.m[i])) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&hs.m[i])) : "memory");
   }
@@ -920,13 +714,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tm_u,
                     const __grid_constant__ CUtensorMap tm_h,
                     const __grid_constant__ SmallBoxMaps tm_hs,
-                    const __grid_constant__ CUtensorMap tm_d128,
-                    const __grid_constant__ SwapMaps tm_gu, const FfnArgs args) {
+                    const __grid_constant__ CUtensorMap tm_d128, const FfnArgs args) {
   constexpr int kStages = kStagesPair;
   constexpr int kStageBytes = kATileBytes + kBHalfBytes;
   extern __shared__ uint8_t smem_raw[];
   const int E = args.E;
-  const Ring s = carve(smem_raw, E, kStages, kStageBytes, true);
+  const Ring s = carve(smem_raw, E, kStages, kStageBytes);
   const Tables& tb = s.tb;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();  // CTA 0 claims the tiles and issues the MMAs
@@ -941,10 +734,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       init_ring(s, kStages, 8, kPairQueueConsumers);  // acc_empty: four epilogue warps per CTA
       prefetch_maps(&tm_x, &tm_g, &tm_u, &tm_h, &tm_d128, tm_xs, tm_hs, args.wlist == nullptr);
-      if (args.wlist == nullptr) {
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_gu.g64)) : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_gu.u64)) : "memory");
-      }
     }
   } else if (warp == 1) {
     // the same warp of both CTAs allocates, as cta_group::2 requires
@@ -999,62 +788,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (tile < 0) break;
         const FTile t = fdecode(tb, E, n1, n2, tile);
-        const int n_e = tb.off[t.e + 1] - tb.off[t.e];
-        if (swapped(n_e)) {
-          // A: 128 weight rows of this CTA's half of M; B: this CTA's half of the chunk's rows
-          const SwapChunk ch = swap_chunk(n_e, t.unit);
-          const int half = ch.n_mma / 2;
-          const int b_rows = (half + 15) / 16 * 16;  // staged as one box of 16 .. 128 rows
-          const int row_b = tb.off[t.e] + ch.row0 + static_cast<int>(rank) * half;
-          const uint32_t stage_tx = 2u * (kATileBytes + static_cast<uint32_t>(b_rows) * 128u);
-          int nkb, w_row;
-          const CUtensorMap *mbig, *mw0, *mw1 = nullptr;
-          const SmallBoxMaps* msmall;
-          if (t.phase == 1) {
-            nkb = kb1;
-            const int f0 = t.n_blk * 128 + static_cast<int>(rank) * 64;
-            mw0 = weight_map(args, &tm_gu.g64, t.e, 4, f0, args.F, w_row);
-            mw1 = weight_map(args, &tm_gu.u64, t.e, 5, f0, args.F, w_row);
-            mbig = &tm_x;
-            msmall = &tm_xs;
-          } else {
-            if (!gemm2_acquire(args, tb.ms_rb[t.e] + t.unit, 8 * n1, 2 * n2, ab)) break;
-            nkb = kb2;
-            mw0 = weight_map(args, &tm_d128, t.e, 2,
-                             t.n_blk * 256 + static_cast<int>(rank) * 128, args.H, w_row);
-            mbig = &tm_h;
-            msmall = &tm_hs;
-          }
-          const CUtensorMap* b_box = b_rows == BM ? mbig : &msmall->m[b_rows / 16 - 1];
-          bool ok = true;
-          for (int kb = 0; kb < nkb; ++kb) {
-            if (!wait_bar(smem_addr(&s.empty[stage]), phase ^ 1u, ab)) {
-              ok = false;
-              break;
-            }
-            const uint32_t a_dst = tiles_base + stage * kStageBytes;
-            const uint32_t b_dst = a_dst + kATileBytes;
-            const uint32_t fb = smem_addr(&s.full[stage]);
-            const uint32_t bar = rank == 0 ? fb : peer_addr(fb, 0);
-            const int kx = kb * (t.phase == 1 ? ks1 : BK);
-            if (rank == 0) mbar_arrive_expect_tx(fb, stage_tx);
-            if (t.phase == 1) {
-              pair_load(rank, a_dst, mw0, bar, kx, w_row);                    // gate rows
-              pair_load(rank, a_dst + kATileBytes / 2, mw1, bar, kx, w_row);  // up rows
-            } else {
-              pair_load(rank, a_dst, mw0, bar, kx, w_row);
-            }
-            pair_load(rank, b_dst, b_box, bar, kx, row_b);
-            issued_mask |= 1u << stage;
-            issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
-            if (++stage == kStages) {
-              stage = 0;
-              phase ^= 1u;
-            }
-          }
-          if (!ok) break;
-          continue;
-        }
         const int m_blk = 2 * t.unit + static_cast<int>(rank);  // this CTA's row block
         const int row_a = tb.off[t.e] + m_blk * BM;
         const int rows = m_blk < tb.mt[t.e] ? min(BM, tb.off[t.e + 1] - row_a) : 0;
@@ -1070,14 +803,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         int row_b;
         if (t.phase == 1) {
           nkb = kb1;
-          ma = bi < kSmallBoxes ? &tm_xs.m[bi] : &tm_x;
+          ma = bi < 3 ? &tm_xs.m[bi] : &tm_x;
           // gate rows -> accumulator columns 0..127, up rows -> 128..255
           mb = weight_map(args, rank == 0 ? &tm_g : &tm_u, t.e, static_cast<int>(rank),
                           t.n_blk * 128, args.F, row_b);
         } else {
-          if (rows > 0 && !gemm2_acquire(args, tb.ms_rb[t.e] + m_blk, 4 * n1, n2, ab)) break;
+          if (rows > 0 && !gemm2_acquire(args, tb, t.e, m_blk, n1, n2, ab)) break;
           nkb = kb2;
-          ma = bi < kSmallBoxes ? &tm_hs.m[bi] : &tm_h;
+          ma = bi < 3 ? &tm_hs.m[bi] : &tm_h;
           mb = weight_map(args, &tm_d128, t.e, 2, t.n_blk * 256 + static_cast<int>(rank) * 128,
                           args.H, row_b);
         }
@@ -1125,6 +858,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ---- MMA issuer (CTA 0): M = 256 over the pair, N = 256 ------------------------------------
     if (rank == 0 && lane == 0) {
+      const uint32_t idesc16 = make_idesc(2 * BM, 256), idesc8 = make_idesc_e4m3(2 * BM, 256);
       int stage = 0;
       uint32_t phase = 0;
       bool issued_any = false;
@@ -1137,10 +871,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool g1 = tile < U * n1;
         const int nkb = g1 ? kb1 : kb2;
         const bool f8 = g1 && w8;  // e4m3 operands: K = 32 per MMA, the same 32 bytes of a row
-        const FTile t = fdecode(tb, E, n1, n2, tile);
-        const int n_e = tb.off[t.e + 1] - tb.off[t.e];
-        const int n_mma = swapped(n_e) ? swap_chunk(n_e, t.unit).n_mma : 256;
-        const uint32_t idesc = f8 ? make_idesc_e4m3(2 * BM, n_mma) : make_idesc(2 * BM, n_mma);
         const int acc = it & 1;
         const uint32_t acc_parity = (it >> 1) & 1;
         if (!wait_bar(smem_addr(&s.acc_empty[acc]), acc_parity ^ 1u, ab)) break;
@@ -1159,9 +889,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < BK / UMMA_K; ++kk) {
             const uint64_t ad = sw128_desc(a_addr + kk * 32), bd = sw128_desc(b_addr + kk * 32);
             if (f8)
-              tc_mma2_f8(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+              tc_mma2_f8(d_tmem, ad, bd, idesc8, (kb | kk) != 0 ? 1u : 0u);
             else
-              tc_mma2(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+              tc_mma2(d_tmem, ad, bd, idesc16, (kb | kk) != 0 ? 1u : 0u);
           }
           issued_any = true;
           tc_commit2_both(smem_addr(&s.empty[stage]));
@@ -1185,7 +915,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t acc_empty0 = smem_addr(&s.acc_empty[0]);
     int qi = 0;
     uint32_t qph = 0;
-    int xseq = 0;
     for (int it = 0;; ++it) {
       int tile;
       if (!warp_take_tile(s, qi, qph, rank != 0, ab, lane, tile) || tile < 0) break;
@@ -1197,13 +926,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!__shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + acc * kAccCols + (static_cast<uint32_t>(quarter * 32) << 16);
-      if (swapped(tb.off[t.e + 1] - tb.off[t.e])) {
-        if (!epilogue_swap(args, tb, s.xchg, s.xflag, t.phase, t.e, t.unit, t.n_blk, t_row,
-                           quarter, lane, rank, xseq, ab))
-          break;
-      } else
-        epilogue_tile(args, tb, t.phase, t.e, 2 * t.unit + static_cast<int>(rank), t.n_blk, t_row,
-                      r_local, lane);
+      epilogue_tile(args, tb, t.phase, t.e, 2 * t.unit + static_cast<int>(rank), t.n_blk, t_row,
+                    r_local, lane);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -1248,7 +972,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // accumulator rows that are never stored (the expert has at most 64 rows).
   extern __shared__ uint8_t smem_raw[];
   const int E = args.E;
-  const Ring s = carve(smem_raw, E, kStages, kStageBytes, false);
+  const Ring s = carve(smem_raw, E, kStages, kStageBytes);
   const Tables& tb = s.tb;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n1 = (args.F + 127) / 128;
@@ -1314,7 +1038,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int m_blk = t.unit;
         const int row_a = tb.off[t.e] + m_blk * BM;
         const int rows = min(kSingleMaxRows, tb.off[t.e + 1] - row_a);
-        const int bi = small_box_index(rows);  // 16 .. 64 rows
+        const int bi = small_box_index(rows);  // 16, 32 or 64 rows
         const uint32_t stage_tx = a_box_bytes(rows) + kBTileBytes;
         int nkb;
         const CUtensorMap *ma, *mb0, *mb1 = nullptr;
@@ -1325,7 +1049,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mb0 = weight_map(args, &tm_g, t.e, 0, t.n_blk * 128, args.F, row_b);
           mb1 = weight_map(args, &tm_u, t.e, 1, t.n_blk * 128, args.F, row_b);
         } else {
-          if (!gemm2_acquire(args, tb.ms_rb[t.e] + m_blk, 4 * n1, n2, ab)) break;
+          if (!gemm2_acquire(args, tb, t.e, m_blk, n1, n2, ab)) break;
           nkb = kb2;
           ma = &tm_hs.m[bi];
           mb0 = weight_map(args, &tm_d256, t.e, 3, t.n_blk * 256, args.H, row_b);
@@ -1595,10 +1319,12 @@ cudaError_t launch_quantize_rows_fp8(const void* x, int rows, int K, void* codes
 
 // Persistent grid of 2-CTA clusters of `kernel`: as many clusters as can be resident at once (one
 // CTA per SM), looked up once per device, kernel and shared-memory size.
-static cudaError_t cluster_grid(const void* kernel, const cudaLaunchConfig_t& cfg_in, int* grid) {
+using FfnKernel = void (*)(CUtensorMap, SmallBoxMaps, CUtensorMap, CUtensorMap, CUtensorMap,
+                           SmallBoxMaps, CUtensorMap, FfnArgs);
+static cudaError_t cluster_grid(FfnKernel kernel, const cudaLaunchConfig_t& cfg_in, int* grid) {
   struct Entry {
     int dev;
-    const void* kernel;
+    FfnKernel kernel;
     size_t smem;
     int grid;
   };
@@ -1647,19 +1373,16 @@ size_t ffn_workspace_bytes(int max_rows, int H, int F, int fp8, int E, int w8) {
          round256((2 * ffn_counter_count(max_rows, E) + 4) * sizeof(int));
 }
 
-size_t ffn_weight_list_bytes(int E) {
-  return static_cast<size_t>(E) * kListMaps * sizeof(CUtensorMap);
-}
+size_t ffn_weight_list_bytes(int E) { return static_cast<size_t>(E) * 4 * sizeof(CUtensorMap); }
 
 cudaError_t ffn_weight_list_init(const void* const* w_gate, const void* const* w_up,
                                  const void* const* w_down, int E, int H, int F, void* list,
                                  cudaStream_t s) {
-  std::vector<CUtensorMap> maps(static_cast<size_t>(E) * kListMaps);
+  std::vector<CUtensorMap> maps(static_cast<size_t>(E) * 4);
   for (int e = 0; e < E; ++e) {
-    CUtensorMap* m = maps.data() + kListMaps * static_cast<size_t>(e);
+    CUtensorMap* m = maps.data() + 4 * static_cast<size_t>(e);
     if (!make_tmap(m + 0, w_gate[e], F, H, 128) || !make_tmap(m + 1, w_up[e], F, H, 128) ||
-        !make_tmap(m + 2, w_down[e], H, F, 128) || !make_tmap(m + 3, w_down[e], H, F, 256) ||
-        !make_tmap(m + 4, w_gate[e], F, H, 64) || !make_tmap(m + 5, w_up[e], F, H, 64))
+        !make_tmap(m + 2, w_down[e], H, F, 128) || !make_tmap(m + 3, w_down[e], H, F, 256))
       return cudaErrorInvalidValue;
   }
   // from pageable memory: the call returns once the host array has been taken
@@ -1714,8 +1437,7 @@ cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp
   }
   CUtensorMap tm_x, tm_g, tm_u, tm_h, tm_d128, tm_d256;
   SmallBoxMaps tm_xs, tm_hs;
-  SwapMaps tm_gu;
-  for (int i = 0; i < kSmallBoxes; ++i)
+  for (int i = 0; i < 3; ++i)
     if (!(w8 ? make_tmap_u8(&tm_xs.m[i], xq, max_rows, H, small_box_rows(i))
              : make_tmap(&tm_xs.m[i], a_src, max_rows, H, small_box_rows(i))) ||
         !make_tmap(&tm_hs.m[i], h, max_rows, F, small_box_rows(i)))
@@ -1727,8 +1449,6 @@ cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp
     // e4m3 gate / up codes [E * F, H]; the down projection stays bf16
     if (!make_tmap_u8(&tm_g, w_gate, static_cast<uint64_t>(E) * F, H, 128) ||
         !make_tmap_u8(&tm_u, w_up, static_cast<uint64_t>(E) * F, H, 128) ||
-        !make_tmap_u8(&tm_gu.g64, w_gate, static_cast<uint64_t>(E) * F, H, 64) ||
-        !make_tmap_u8(&tm_gu.u64, w_up, static_cast<uint64_t>(E) * F, H, 64) ||
         !make_tmap(&tm_d128, w_down, static_cast<uint64_t>(E) * H, F, 128) ||
         !make_tmap(&tm_d256, w_down, static_cast<uint64_t>(E) * H, F, 256))
       return cudaErrorInvalidValue;
@@ -1738,11 +1458,8 @@ cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp
     memset(&tm_u, 0, sizeof(CUtensorMap));
     memset(&tm_d128, 0, sizeof(CUtensorMap));
     memset(&tm_d256, 0, sizeof(CUtensorMap));
-    memset(&tm_gu, 0, sizeof(SwapMaps));
   } else if (!make_tmap(&tm_g, w_gate, static_cast<uint64_t>(E) * F, H, 128) ||
              !make_tmap(&tm_u, w_up, static_cast<uint64_t>(E) * F, H, 128) ||
-             !make_tmap(&tm_gu.g64, w_gate, static_cast<uint64_t>(E) * F, H, 64) ||
-             !make_tmap(&tm_gu.u64, w_up, static_cast<uint64_t>(E) * F, H, 64) ||
              !make_tmap(&tm_d128, w_down, static_cast<uint64_t>(E) * H, F, 128) ||
              !make_tmap(&tm_d256, w_down, static_cast<uint64_t>(E) * H, F, 256)) {
     return cudaErrorInvalidValue;
@@ -1758,9 +1475,8 @@ cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp
   const FfnArgs fa_pair{expert_offsets, E, max_rows, H, F, h,
                         static_cast<__nv_bfloat16*>(expert_out), status, done, used, sched, wl,
                         xs, w_gate_scale, w_up_scale};
-  const size_t smem_single =
-      ring_smem_bytes(E, kStagesSingle, kASingleBytes + 2 * kBHalfBytes, false);
-  const size_t smem_pair = ring_smem_bytes(E, kStagesPair, kATileBytes + kBHalfBytes, true);
+  const size_t smem_single = ring_smem_bytes(E, kStagesSingle, kASingleBytes + 2 * kBHalfBytes);
+  const size_t smem_pair = ring_smem_bytes(E, kStagesPair, kATileBytes + kBHalfBytes);
   err = cudaFuncSetAttribute(ffn_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem_single));
   if (err != cudaSuccess) return err;
@@ -1781,10 +1497,10 @@ cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp
   int grid_single = 0, grid_pair = 0;
   cfg.numAttrs = 1;
   cfg.dynamicSmemBytes = smem_single;
-  err = cluster_grid(reinterpret_cast<const void*>(ffn_single_kernel), cfg, &grid_single);
+  err = cluster_grid(ffn_single_kernel, cfg, &grid_single);
   if (err != cudaSuccess) return err;
   cfg.dynamicSmemBytes = smem_pair;
-  err = cluster_grid(reinterpret_cast<const void*>(ffn_pair_kernel), cfg, &grid_pair);
+  err = cluster_grid(ffn_pair_kernel, cfg, &grid_pair);
   if (err != cudaSuccess) return err;
   cfg.numAttrs = MOE_USE_PDL ? 2 : 1;
   cfg.gridDim = dim3(grid_single);
@@ -1795,7 +1511,7 @@ cudaError_t launch_expert_ffn(const void* send, const float* send_scales, int fp
   cfg.gridDim = dim3(grid_pair);
   cfg.dynamicSmemBytes = smem_pair;
   err = cudaLaunchKernelEx(&cfg, ffn_pair_kernel, tm_x, tm_xs, tm_g, tm_u, tm_h, tm_hs, tm_d128,
-                           tm_gu, fa_pair);
+                           fa_pair);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }

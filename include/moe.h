@@ -206,7 +206,7 @@ moe_status_t moe_expert_ffn(const void* send, const float* send_scales, moe_payl
  * 并行", sections 消除D2D时延开销 and 关键优化实施: the grouped GEMM takes a TensorList and picks
  * each expert's buffer inside the kernel, instead of merging split weights device to device).
  *
- * moe_ffn_weight_list_bytes: bytes of the device buffer moe_ffn_weight_list_init fills (six
+ * moe_ffn_weight_list_bytes: bytes of the device buffer moe_ffn_weight_list_init fills (four
  * 128-byte TMA descriptors per expert); 0 for E outside [1, 1024].
  *
  * moe_ffn_weight_list_init: set-up call, once per set of weight addresses.

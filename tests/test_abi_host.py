@@ -160,7 +160,7 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
 def test_weight_list_calls_reject_bad_arguments(lib):
     """The per-expert weight-list entry points validate on the host before touching the GPU."""
     import ctypes
-    assert pkg.moe_ffn_weight_list_bytes(8) == 8 * 6 * 128        # six descriptors per expert
+    assert pkg.moe_ffn_weight_list_bytes(8) == 8 * 4 * 128        # four descriptors per expert
     assert pkg.moe_ffn_weight_list_bytes(0) == 0
     assert pkg.moe_ffn_weight_list_bytes(1025) == 0
     ptrs = (ctypes.c_void_p * 2)(FAKE, FAKE)

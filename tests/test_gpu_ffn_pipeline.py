@@ -199,18 +199,18 @@ def test_ffn_workspace_reused_across_calls_with_different_routing(cuda):
 
 
 @pytest.mark.parametrize("rows,H,F", [
-    ([150, 200, 256, 129, 180, 222, 140, 255], 256, 320),  # one chunk each (N = rows rounded to 16)
-    ([150, 200, 256, 40, 300, 129, 0, 180], 256, 320),     # plus single-CTA, two-chunk and empty
-    ([130, 0, 0, 0, 0, 0, 0, 0], 256, 320),                # a single expert
-    # the swapped-operand limits: 64 (single CTA) / 65 (N = 80), 256 / 257 (two chunks), 512 (two
-    # full chunks) / 513 (pairs of row blocks); ragged H (the second 256-column block half out)
+    ([150, 200, 256, 129, 180, 222, 140, 255], 256, 320),  # every expert: two 128-row blocks
+    ([150, 200, 256, 40, 300, 129, 0, 180], 256, 320),     # plus 1-, 3- and 0-block experts
+    ([130, 0, 0, 0, 0, 0, 0, 0], 256, 320),                # a single two-block expert
+    # the kernel limits: 64 rows (single CTA) / 65 (a pair whose second block is empty); 256 / 257
+    # and 512 / 513 (one, two and three pairs); ragged H (the second 256-column block half out)
     ([64, 65, 80, 96, 256, 257, 511, 512, 513, 17], 320, 192),
     ([65, 512, 513, 1000], 64, 128),                       # one k-step of GEMM-1, F below 128 cols
 ])
 def test_ffn_two_block_experts(cuda, rows, H, F):
-    """Experts of 65..512 rows run with the operands swapped (weights as M, the expert's rows as N
-    in chunks of at most 256), next to single-CTA experts (at most 64 rows), pairs of 128-row blocks
-    (more than 512) and empty ones."""
+    """Experts of 65..256 rows (two 128-row blocks, the second one ragged or empty) next to experts
+    of one, three, four and more blocks and empty ones: each pair of blocks is one 2-CTA tile, and
+    the blocks of an expert read the same weight column blocks."""
     from combine_moe_route_10_b200 import MoeShuffle
     E = len(rows)
     off = np.concatenate([[0], np.cumsum(rows)]).astype(np.int32)
