@@ -383,7 +383,7 @@ __device__ __forceinline__ const CUtensorMap* weight_map(const FfnArgs& args, co
 }
 
 struct Tables {
-  int* off;     // [E+1] row offsets (clamped to max_rows)
+  int* off;     // [E+1] row offsets (clamped to [0, max_rows])
   int* mt;      // [E]   row blocks per expert
   int* units;   // [E]   units of this kernel's class per expert (0 for the other class)
   int* ms_rb;   // [E+1] first global row block of each expert (over all experts)
@@ -415,8 +415,8 @@ __device__ __forceinline__ void build_tables(const Tables& tb, const FfnArgs& ar
     int lo = 0, hi = 0;
     if (e < E) {
       // L2 loads: the pair kernel may start before the kernel ahead of it has finished
-      lo = min(__ldcg(args.expert_offsets + e), args.max_rows);
-      hi = min(__ldcg(args.expert_offsets + e + 1), args.max_rows);
+      lo = min(max(__ldcg(args.expert_offsets + e), 0), args.max_rows);
+      hi = min(max(__ldcg(args.expert_offsets + e + 1), 0), args.max_rows);
     }
     const int mt = (max(hi - lo, 0) + BM - 1) / BM;
     const bool paired = hi - lo > kSingleMaxRows;
@@ -448,7 +448,7 @@ __device__ __forceinline__ void build_tables(const Tables& tb, const FfnArgs& ar
   if (lane == 0) {
     tb.ms_rb[E] = carry_r;
     tb.ms_u[E] = carry_u;
-    tb.off[E] = min(__ldcg(args.expert_offsets + E), args.max_rows);
+    tb.off[E] = min(max(__ldcg(args.expert_offsets + E), 0), args.max_rows);
     tb.stats[0] = n_single;
     tb.stats[1] = n_pairs;
   }

@@ -221,6 +221,15 @@ struct BwdArgs {
   int* status;
 };
 
+// Rows [off, off + rows) of expert e, its offsets clamped to [0, max_rows] as in the forward, so
+// that offsets past the row buffers (a caller's mistake) make no tile read or write outside them.
+__device__ __forceinline__ int expert_span(const BwdArgs& a, int e, int& rows) {
+  const int lo = min(max(__ldg(a.expert_offsets + e), 0), a.max_rows);
+  const int hi = min(max(__ldg(a.expert_offsets + e + 1), 0), a.max_rows);
+  rows = max(hi - lo, 0);
+  return lo;
+}
+
 // Pair tiles of every item (prefix in shared memory) and the decoding of a tile index.
 struct Tile {
   int e, p, mb, nb;  // expert, sub-problem (weight grad), 256-row block, column block
@@ -269,7 +278,8 @@ __device__ __forceinline__ Tile decode(const BwdArgs& a, const int* start, int t
   {
     // row blocks fastest: the tiles running at the same time share one weight slice, which then
     // crosses HBM once per expert instead of once per row block
-    const int rows = __ldg(a.expert_offsets + t.e + 1) - __ldg(a.expert_offsets + t.e);
+    int rows;
+    expert_span(a, t.e, rows);
     const int nrow = (rows + kPairM - 1) / kPairM;
     t.mb = local % nrow;
     t.nb = local / nrow;
@@ -370,8 +380,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     int run = 0;
     for (int i = 0; i < n_items; ++i) {
       start[i] = run;
-      const int e = i % E;
-      const int rows = __ldg(args.expert_offsets + e + 1) - __ldg(args.expert_offsets + e);
+      int rows;
+      expert_span(args, i % E, rows);
       run += tiles_of<MODE>(args, rows, i / E);
     }
     start[n_items] = run;
@@ -392,8 +402,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool stop = false;
     for (int tile = cid; tile < total && !stop; tile += ncl) {
       const Tile t = decode<MODE>(args, start, tile);
-      const int off = __ldg(args.expert_offsets + t.e);
-      const int rows = __ldg(args.expert_offsets + t.e + 1) - off;
+      int rows;
+      const int off = expert_span(args, t.e, rows);
       const int nkb = k_blocks<MODE>(args, rows);
       const int half = static_cast<int>(rank) * kBM;  // this CTA's rows / columns of the tile
       for (int kb = 0; kb < nkb; ++kb) {
@@ -511,7 +521,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int it = 0;
       for (int tile = cid; tile < total; tile += ncl, ++it) {
         const Tile t = decode<MODE>(args, start, tile);
-        const int rows = __ldg(args.expert_offsets + t.e + 1) - __ldg(args.expert_offsets + t.e);
+        int rows;
+        expert_span(args, t.e, rows);
         const int nkb = k_blocks<MODE>(args, rows);
         const int acc = kBufs == 2 ? (it & 1) : 0;
         const uint32_t acc_par = kBufs == 2 ? ((it >> 1) & 1) : (it & 1);
@@ -575,8 +586,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     int it = 0;
     for (int tile = cid; tile < total; tile += ncl, ++it) {
       const Tile t = decode<MODE>(args, start, tile);
-      const int off = __ldg(args.expert_offsets + t.e);
-      const int rows = __ldg(args.expert_offsets + t.e + 1) - off;
+      int rows;
+      const int off = expert_span(args, t.e, rows);
       const int acc = kBufs == 2 ? (it & 1) : 0;
       const uint32_t acc_par = kBufs == 2 ? ((it >> 1) & 1) : (it & 1);
       int ok = 1;

@@ -52,3 +52,48 @@ def test_ffn_wait_timeout_is_reported_and_recoverable(cuda):
     assert_ffn_and_combine(bits16(m.h)[:o["S"]], bits16(m.expert_out)[:o["S"]], bits16(m.y), o["h"],
                            o["expert_out"], o["y"], o["expert_offsets"], d["w_down"],
                            o["slot_row"], o["topk_w"], "after recovery")
+
+
+@pytest.mark.parametrize("bad", [[0, 90, 150, 400], [-50, 90, 150, 200]])
+def test_expert_offsets_outside_the_buffers_are_clamped(cuda, bad):
+    """Expert offsets past max_rows or below zero (a caller's mistake, not a fault): the FFN and the
+    expert backward clamp them to [0, max_rows], so every result equals the one for the clamped
+    offsets, and the rows past max_rows in oversized output buffers keep their contents."""
+    from combine_moe_route_10_b200 import _lib
+    E, H, F, S, SPARE = 3, 128, 128, 200, 64
+    g = torch.Generator(device="cuda").manual_seed(5)
+    x = mi.randn_bf16((S, H), g)
+    d_eo = mi.randn_bf16((S, H), g)
+    wg, wu = mi.randn_bf16((E, F, H), g, 0.05), mi.randn_bf16((E, F, H), g, 0.05)
+    wd = mi.randn_bf16((E, H, F), g, 0.05)
+    good = torch.tensor([0, 90, 150, 200], dtype=torch.int32, device="cuda")
+    sentinel = torch.full((SPARE, H), 7.0, dtype=torch.bfloat16, device="cuda")
+
+    def forward(off):
+        eo = torch.zeros((S + SPARE, H), dtype=torch.bfloat16, device="cuda")
+        eo[S:] = sentinel
+        nb = _lib.moe_ffn_workspace_size(S, E, H, F, _lib.MOE_PAYLOAD_BF16)
+        ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+        _lib.moe_expert_ffn(x, None, _lib.MOE_PAYLOAD_BF16, off, S, E, H, F, wg, wu, wd, eo, ws, nb)
+        assert _lib.moe_sync_status(ws) == _lib.MOE_OK
+        return eo
+
+    def backward(off):
+        dx_rows = torch.zeros((S + SPARE, H), dtype=torch.bfloat16, device="cuda")
+        dx_rows[S:] = sentinel
+        grads = [torch.zeros((E, F, H), dtype=torch.float32, device="cuda") for _ in range(2)]
+        dwd = torch.zeros((E, H, F), dtype=torch.float32, device="cuda")
+        nb = _lib.moe_expert_backward_workspace_size(S, F)
+        ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+        _lib.moe_expert_backward(x, d_eo, off, S, E, H, F, wg, wu, wd, dx_rows, grads[0], grads[1],
+                                 dwd, ws, nb)
+        assert _lib.moe_sync_status(ws) == _lib.MOE_OK
+        return dx_rows, grads[0], grads[1], dwd
+
+    off_bad = torch.tensor(bad, dtype=torch.int32, device="cuda")
+    eo_bad, eo_good = forward(off_bad), forward(good)
+    assert torch.equal(eo_bad, eo_good)
+    assert torch.equal(eo_bad[S:], sentinel)
+    for a, b in zip(backward(off_bad), backward(good)):
+        assert torch.equal(a, b)
+    assert torch.equal(backward(off_bad)[0][S:], sentinel)
