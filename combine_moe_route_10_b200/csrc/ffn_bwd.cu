@@ -756,7 +756,9 @@ __global__ void __launch_bounds__(256)
     // slot j's routing data and, after its pass over H, its d_w live in lane j
     const int my_row = lane < k ? __ldg(slot_row + t * k + lane) : -1;
     const float my_w = lane < k ? __ldg(topk_w + t * k + lane) : 0.0f;
-    const int my_e = lane < k ? __ldg(topk_idx + t * k + lane) : -1;
+    int my_e = lane < k ? __ldg(topk_idx + t * k + lane) : -1;
+    // an expert id outside [0, E) (rejected by the forward's dispatch) gives no d_logits entry
+    if (static_cast<unsigned>(my_e) >= static_cast<unsigned>(E)) my_e = -1;
     float my_dw = 0.0f;
     const uint4* dy_row = dy + static_cast<size_t>(t) * nv;
     for (int j = 0; j < k; ++j) {
@@ -796,7 +798,7 @@ __global__ void __launch_bounds__(256)
       for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xFFFFFFFFu, c, o);
       for (int e = lane; e < E; e += 32) dl[e] = 0.0f;
       __syncwarp();
-      if (lane < k) dl[my_e] = my_w * (my_dw - c);
+      if (my_e >= 0) dl[my_e] = my_w * (my_dw - c);
     } else {
       // p = softmax over all E logits; d_e = d_w of the slot that selected e, else 0
       const float* lg = logits + static_cast<size_t>(t) * E;
@@ -809,12 +811,12 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
       // sum_e p_e d_e over the selected experts only (d is 0 elsewhere)
-      float pd = lane < k ? expf(__ldg(lg + my_e) - mx) / sum * my_dw : 0.0f;
+      float pd = my_e >= 0 ? expf(__ldg(lg + my_e) - mx) / sum * my_dw : 0.0f;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) pd += __shfl_xor_sync(0xFFFFFFFFu, pd, o);
       for (int e = lane; e < E; e += 32) dl[e] = -(expf(__ldg(lg + e) - mx) / sum) * pd;
       __syncwarp();
-      if (lane < k) {
+      if (my_e >= 0) {
         const float p = expf(__ldg(lg + my_e) - mx) / sum;
         dl[my_e] = p * (my_dw - pd);
       }

@@ -291,7 +291,10 @@ moe_status_t moe_combine(const void* expert_out, int max_rows, const int32_t* sl
  *   3. dx[t] = bf16(sum over kept slots of dx_rows[slot_row[t,j]]), fp32 in slot order;
  *   4. d_logits [T,E]: with renormalize, for a selected expert i: w_i (d_w_i - sum_j w_j d_w_j), 0
  *      elsewhere; without, the full-E softmax backward p_e (d_e - sum p d) (logits needed).
- * Inputs from the forward: topk_idx, topk_w, slot_row, expert_offsets (moe_route / moe_dispatch),
+ * Inputs from the forward: topk_idx, topk_w, slot_row, expert_offsets (moe_route / moe_dispatch;
+ * a slot whose expert id lies outside [0, E), which moe_dispatch reports as MOE_ERR_INVALID_TOPK,
+ * adds nothing to d_logits, a slot_row outside [0, max_rows) marks a dropped slot, and
+ * expert_offsets are clamped to [0, max_rows]),
  * ffn_input = the FFN's input rows bf16 [max_rows, H] (the send buffer for the bf16 payload; the
  * dequantised rows of the FFN workspace for the FP8 payload), expert_out bf16 [max_rows, H]; the
  * weights as for moe_expert_ffn.  Outputs (device, caller-owned): dx bf16 [T,H], d_logits fp32

@@ -257,3 +257,45 @@ def test_backward_edge_shapes(cuda, T, H, E, k, R, F, payload, cf):
     if cf:
         assert (np_(m.slot_row) < 0).any()
     _check(w, m, d, grads, ref, S, f"edge T{T} E{E} k{k}")
+
+
+@pytest.mark.parametrize("renormalize", [True, False])
+def test_combine_backward_skips_expert_ids_outside_range(cuda, renormalize):
+    """An expert id outside [0, E) in one slot (which the forward's dispatch rejects): the combine
+    backward's d_eo and d_topk_w do not depend on ids and stay the same; in d_logits the slot adds
+    no entry, and every entry of the other slots and tokens is unchanged."""
+    from combine_moe_route_10_b200 import MoeShuffle, _lib
+    w = mi.get("tiny")
+    d = mi.make_inputs(w, seed=4, device="cuda")
+    m = MoeShuffle(w.T, w.H, w.E, w.k, w.R, w.F, renormalize=renormalize)
+    m.forward(d["logits"], d["x"], d["w_gate"], d["w_up"], d["w_down"])
+    g = torch.Generator(device="cuda").manual_seed(9)
+    dy = torch.randn((w.T, w.H), generator=g, device="cuda").to(torch.bfloat16)
+    idx_bad = m.topk_idx.clone()
+    t, j = 3, 1
+    e_dropped = int(idx_bad[t, j].item())
+    idx_bad[t, j] = w.E + 5
+
+    def run(idx):
+        d_eo = torch.zeros((m.max_rows, w.H), dtype=torch.bfloat16, device="cuda")
+        d_w = torch.zeros((w.T, w.k), dtype=torch.float32, device="cuda")
+        d_lg = torch.full((w.T, w.E), 123.0, dtype=torch.float32, device="cuda")
+        _lib.moe_combine_backward(dy, w.T, w.H, w.k, w.E, d["logits"], renormalize, idx,
+                                  m.topk_w, m.slot_row, m.max_rows, m.expert_out, d_eo, d_w, d_lg)
+        torch.cuda.synchronize()
+        return d_eo, d_w, d_lg
+
+    eo_ok, dw_ok, lg_ok = run(m.topk_idx)
+    eo_bad, dw_bad, lg_bad = run(idx_bad)
+    assert torch.equal(eo_bad, eo_ok) and torch.equal(dw_bad, dw_ok)
+    others = [r for r in range(w.T) if r != t]
+    assert torch.equal(lg_bad[others], lg_ok[others])
+    if renormalize:
+        # the other slots keep their entries (c sums over every slot's w d_w, ids aside); the
+        # dropped slot's expert, chosen by no other slot of the token, now reads 0
+        assert bool((m.topk_idx[t] == e_dropped).sum() == 1)
+        expect = lg_ok[t].clone()
+        expect[e_dropped] = 0.0
+        assert torch.equal(lg_bad[t], expect)
+    else:
+        assert torch.isfinite(lg_bad[t]).all()
