@@ -129,6 +129,22 @@ def test_workspace_sizes(lib):
     assert pkg.moe_ffn_workspace_size(100, 8, 256, 512, pkg.MOE_PAYLOAD_BF16) >= 256 + 100 * 512 * 2
 
 
+@pytest.mark.parametrize("max_rows,E,H,F", [(100, 8, 256, 512), (32768, 256, 7168, 2048),
+                                            (1, 1, 128, 64)])
+def test_ffn_workspace_layout_matches_the_python_views(lib, max_rows, E, H, F):
+    """The binding reads two parts of the FFN workspace directly: h at byte 256 and, for the FP8
+    payload, the dequantised bf16 input rows right after h (``MoeShuffle.dequantized_rows``, the
+    expert-parallel backward's FFN input rows), and the failure test writes the GEMM-1 counters
+    after those.  The library's size is exactly that layout: status | h | (FP8: rows) | counters,
+    each part rounded up to 256 bytes."""
+    up = lambda b: (b + 255) // 256 * 256  # noqa: E731
+    h = up(max_rows * F * 2)
+    counters = up((2 * (max_rows // 128 + E + 1) + 4) * 4)
+    assert pkg.moe_ffn_workspace_size(max_rows, E, H, F, pkg.MOE_PAYLOAD_BF16) == 256 + h + counters
+    assert pkg.moe_ffn_workspace_size(max_rows, E, H, F, pkg.MOE_PAYLOAD_FP8_E4M3_B128) == (
+        256 + h + up(max_rows * H * 2) + counters)
+
+
 def test_ffn_and_combine_reject_bad_arguments(lib):
     ffn = lambda **kw: lib.moe_expert_ffn(
         kw.get("send", FAKE), kw.get("scales", None), kw.get("payload", 0), FAKE,
