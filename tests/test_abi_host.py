@@ -145,6 +145,32 @@ def test_ffn_workspace_layout_matches_the_python_views(lib, max_rows, E, H, F):
         256 + h + up(max_rows * H * 2) + counters)
 
 
+@pytest.mark.parametrize("max_rows,T,k,H,F", [(8192, 4096, 2, 4096, 14336), (5, 3, 2, 64, 64),
+                                              (0, 0, 1, 128, 128)])
+def test_backward_workspace_layout_matches_the_python_views(lib, max_rows, T, k, H, F):
+    """``MoeShuffle.backward_intermediate`` reads d_eo, h, dg, du and dx_rows at fixed offsets of
+    the backward workspace: status | d_eo [r,H] | h, dg, du [r,F] | dx_rows [r,H] | unit weights
+    [T,k] fp32, each part rounded up to 256 bytes (r = max(max_rows, 1)); the expert backward's own
+    workspace is status | h, dg, du."""
+    up = lambda b: (b + 255) // 256 * 256  # noqa: E731
+    r, tk = max(max_rows, 1), max(T, 1) * k
+    assert pkg.moe_backward_workspace_size(max_rows, T, k, H, F) == (
+        256 + 2 * up(r * H * 2) + 3 * up(r * F * 2) + up(tk * 4))
+    assert pkg.moe_expert_backward_workspace_size(max_rows, F) == 256 + 3 * up(r * F * 2)
+
+
+def test_package_exports_every_binding_function():
+    """Every moe_* function of the binding (one per C entry point, moe_status_string aside, which
+    the binding wraps as status_string) is part of the package's public names."""
+    import inspect
+    from combine_moe_route_10_b200 import _lib
+    names = {n for n, f in inspect.getmembers(_lib, inspect.isfunction) if n.startswith("moe_")}
+    assert names and names <= set(pkg.__all__)
+    assert all(hasattr(pkg, n) for n in pkg.__all__)
+    consts = {n for n in dir(_lib) if n.startswith("MOE_")}
+    assert consts <= set(pkg.__all__)
+
+
 def test_ffn_and_combine_reject_bad_arguments(lib):
     ffn = lambda **kw: lib.moe_expert_ffn(
         kw.get("send", FAKE), kw.get("scales", None), kw.get("payload", 0), FAKE,
